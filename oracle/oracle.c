@@ -1,0 +1,527 @@
+/*
+ * oracle.c -- plain, slow CPU oracle for compressed-KV sparse decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or constant
+ * generator with the CUDA library; every step is written out here from the
+ * pages' statement of the method.
+ *
+ * Sources (pages, by title and section):
+ *  [P1] "DeepSeek V4.1 Flash KV Cache压缩实战：FP4+CSA2+CED将显存降至1/4"
+ *       (gtnt.cn): 3.1 FP4 group quantisation, 3.2 CSA2 compression,
+ *       4.1 KV-size estimate, 4.3 parameter table.
+ *  [P2] "DeepSeek V1 到 V4.1-Flash，单 token 的 global KV 如何从 389,000 B
+ *       压缩到 890 B的？" (acejoy.com): part 1 "KV Cache 到底有多大";
+ *       part 3 breakthrough 2 (MLA 512+64), breakthrough 4 (SWA-128,
+ *       indexer top-512, CSA 2:1); part 4 "CSA2：三种模式", "P4 main KV",
+ *       "890 字节是怎么算出来的".
+ *
+ * Readings where the pages leave a step open (each is documented with the
+ * function that takes it):
+ *  R1 gate: one D-vector g gives one logit per token; the pair's weights are
+ *     the softmax of the two logits.  The logit difference is accumulated in
+ *     a fixed order (lane-of-32 partial sums over 8-channel chunks, then a
+ *     xor tree), because the quantised codes downstream depend on the exact
+ *     fp32 entry.
+ *  R2 exp: written here from the Cody-Waite argument reduction and a
+ *     degree-13 Taylor polynomial (Horner form), so that the gate weight is
+ *     the same bits on every implementation of this specification.
+ *  R3 grouping: latent and RoPE segments are grouped separately; a segment's
+ *     last group may be short.
+ *  R4 scale: s = absmax / 6 in fp32, stored as fp32 or rounded (RNE,
+ *     saturating) to an unsigned E4M3 byte; elements are divided by the
+ *     decoded scale and rounded to nearest-even onto the E2M1 grid.
+ *  R5 attention: one joint softmax over the selected entries and the window
+ *     tokens; values are the first Dv (latent) channels of each key.
+ *
+ * Compile with -ffp-contract=off: every fused multiply-add below is an
+ * explicit fma() call and nothing else may be contracted.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_INVALID 1
+#define ORC_ERR_CAPACITY 2
+
+#define ORC_SCALE_F32 0
+#define ORC_SCALE_UE4M3 1
+
+#define ORC_MODE_FULL 0
+#define ORC_MODE_REINDEX 1
+#define ORC_MODE_REUSE 2
+
+/* status bits reported by the pack / attention oracles */
+#define ORC_ST_NONFINITE 1u
+#define ORC_ST_BAD_INDEX 2u
+
+typedef struct {
+    int latent_dim;  /* Dv: latent channels, also the value width        */
+    int rope_dim;    /* RoPE channels appended to the key                 */
+    int group;       /* FP4 group size G                                  */
+    int scale_fmt;   /* ORC_SCALE_F32 or ORC_SCALE_UE4M3                  */
+    int idx_dim;     /* indexer key width Di                              */
+    int topk;        /* K                                                 */
+    int window;      /* W                                                 */
+    int n_heads;     /* H                                                 */
+    double sm_scale; /* softmax scale applied to q.k                      */
+} orc_cfg;
+
+/* ------------------------------------------------------------------ */
+/* KV-size formula: [P2] part 1 "KV Cache 到底有多大" and [P1] 4.1.
+ * bytes per token = 2 (K and V) x layers x heads x head_dim x bytes.    */
+uint64_t orc_kv_bytes_per_token(int64_t layers, int64_t heads, int64_t dim,
+                                int64_t bytes_per_elem) {
+    return (uint64_t)(2 * layers * heads * dim * bytes_per_elem);
+}
+
+/* ------------------------------------------------------------------ */
+/* R2: exp(x) in fp64.  Cody-Waite: x = n*ln2 + r with ln2 split into a
+ * 32-significant-bit head (so n*LN2_HI is exact for |n| < 2^11) and the
+ * rounded remainder; e^r from the Taylor series to degree 13 (truncation
+ * below 4e-18 for |r| <= ln2/2); the result is scaled by an exactly built
+ * power of two.  Inputs above 709 give +inf; inputs below -708 give 0 (a
+ * subnormal exp never changes 1 + exp in the gate).                      */
+static const double ORC_LN2_HI = 0x1.62e42feep-1;
+static const double ORC_LN2_LO = 0x1.a39ef35793c76p-33;
+static const double ORC_INV_LN2 = 0x1.71547652b82fep+0;
+static const double ORC_INV_FACT[14] = {
+    0x1.0p+0,              0x1.0p+0,              0x1.0p-1,
+    0x1.5555555555555p-3,  0x1.5555555555555p-5,  0x1.1111111111111p-7,
+    0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
+    0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+    0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+
+double orc_exp(double x) {
+    if (x != x) return x;
+    if (x > 709.0) return INFINITY;
+    if (x < -708.0) return 0.0;
+    double n = nearbyint(x * ORC_INV_LN2); /* round-half-even, default mode */
+    double r = fma(-n, ORC_LN2_HI, x);
+    r = fma(-n, ORC_LN2_LO, r);
+    double p = ORC_INV_FACT[13];
+    for (int k = 12; k >= 0; --k) p = fma(p, r, ORC_INV_FACT[k]);
+    int64_t bits = ((int64_t)n + 1023) << 52;
+    double two_n;
+    memcpy(&two_n, &bits, sizeof two_n);
+    return p * two_n;
+}
+
+/* ------------------------------------------------------------------ */
+/* E2M1 ([P1] 3.1; [P2] "P4 main KV"): 1 sign, 2 exponent, 1 mantissa bit.
+ * Magnitude codes 0..7 are {0, 0.5, 1, 1.5, 2, 3, 4, 6}; bit 3 is the sign. */
+static const float ORC_E2M1_MAG[8] = {0.0f, 0.5f, 1.0f, 1.5f,
+                                      2.0f, 3.0f, 4.0f, 6.0f};
+
+float orc_e2m1_value(int code) {
+    float m = ORC_E2M1_MAG[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* Round to the nearest grid magnitude; a tie goes to the even code (code
+ * bit 0 clear); magnitudes past 6 saturate to 6.  A result of magnitude 0
+ * is stored as +0 (code 0).  Non-finite input is the caller's business.   */
+int orc_e2m1_encode(float v) {
+    double m = fabs((double)v);
+    int best = 0;
+    double best_d = m; /* distance to magnitude 0 */
+    for (int c = 1; c < 8; ++c) {
+        double d = fabs(m - (double)ORC_E2M1_MAG[c]);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    if (m > 6.0) best = 7;
+    if (best == 0) return 0;
+    return (v < 0.0f) ? (best | 8) : best;
+}
+
+/* E4M3 (OCP "fn": bias 7, no infinities, 0x7F/0xFF are NaN, max 448). */
+float orc_e4m3_value(int b) {
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    float v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexpf((float)m, -9);
+    else
+        v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return s ? -v : v;
+}
+
+/* Unsigned E4M3 encode for v >= 0: nearest of the 127 finite non-negative
+ * values by exhaustive search, ties to the even code, saturating at 448.  */
+int orc_e4m3_encode(float v) {
+    if (!(v > 0.0f)) return 0;
+    if (v >= 448.0f) return 0x7E;
+    double x = (double)v;
+    int best = 0;
+    double best_d = x;
+    for (int b = 1; b <= 0x7E; ++b) {
+        double d = fabs(x - (double)orc_e4m3_value(b));
+        if (d < best_d || (d == best_d && (b & 1) == 0 && (best & 1) == 1)) {
+            best = b;
+            best_d = d;
+        }
+    }
+    return best;
+}
+
+/* ------------------------------------------------------------------ */
+/* R3 grouping and the record layout.                                 */
+int orc_n_groups(int latent, int rope, int group) {
+    return (latent + group - 1) / group + (rope + group - 1) / group;
+}
+
+/* Record = [codes: one byte per channel pair, even channel in the low
+ * nibble][scales in group order][zero padding to a 16-byte multiple].
+ * The padded size is the stride of the record array.                   */
+int orc_record_bytes(const orc_cfg* c, int padded) {
+    int d = c->latent_dim + c->rope_dim;
+    int sb = (c->scale_fmt == ORC_SCALE_F32) ? 4 : 1;
+    int n = d / 2 + orc_n_groups(c->latent_dim, c->rope_dim, c->group) * sb;
+    return padded ? (n + 15) / 16 * 16 : n;
+}
+
+/* group boundaries: fills start[] / len[] with the channel range of each
+ * group; returns the number of groups                                   */
+static int orc_groups(const orc_cfg* c, int* start, int* len) {
+    int g = 0;
+    for (int s = 0; s < c->latent_dim; s += c->group, ++g) {
+        start[g] = s;
+        len[g] = (c->latent_dim - s < c->group) ? c->latent_dim - s : c->group;
+    }
+    for (int s = 0; s < c->rope_dim; s += c->group, ++g) {
+        start[g] = c->latent_dim + s;
+        len[g] = (c->rope_dim - s < c->group) ? c->rope_dim - s : c->group;
+    }
+    return g;
+}
+
+/* ------------------------------------------------------------------ */
+/* R1: the 2:1 compression of a token pair ([P2] breakthrough 4 "CSA 把每 2
+ * 个 token 的 KV 压成 1 条"; [P1] 3.2 "main key compressor").
+ * logit_t = g . k_t; (w0, w1) = softmax(logit_0, logit_1);
+ * entry = w0 k_0 + w1 k_1.
+ * Fixed evaluation order: delta = logit_0 - logit_1 = sum_d g_d (k0_d - k1_d)
+ * accumulated by 32 partial sums; channel chunk c = [8c, 8c+8) goes to
+ * partial c mod 32, chunks in increasing order and channels in increasing
+ * order inside a chunk, each term added with one fma.  The partials are
+ * then combined by a xor tree over offsets 16, 8, 4, 2, 1.              */
+double orc_gate_delta(const float* k0, const float* k1, const float* g, int D) {
+    double acc[32];
+    for (int l = 0; l < 32; ++l) acc[l] = 0.0;
+    for (int c = 0; c * 8 < D; ++c) {
+        int l = c % 32;
+        for (int t = 0; t < 8 && 8 * c + t < D; ++t) {
+            int d = 8 * c + t;
+            double diff = (double)k0[d] - (double)k1[d];
+            acc[l] = fma((double)g[d], diff, acc[l]);
+        }
+    }
+    for (int off = 16; off >= 1; off >>= 1) {
+        double nxt[32];
+        for (int l = 0; l < 32; ++l) nxt[l] = acc[l] + acc[l ^ off];
+        memcpy(acc, nxt, sizeof acc);
+    }
+    return acc[0];
+}
+
+void orc_compress_pair(const float* k0, const float* k1, const float* g, int D,
+                       float* e) {
+    double delta = orc_gate_delta(k0, k1, g, D);
+    double w0 = 1.0 / (1.0 + orc_exp(-delta));
+    double w1 = 1.0 - w0;
+    for (int d = 0; d < D; ++d)
+        e[d] = (float)fma(w0, (double)k0[d], w1 * (double)k1[d]);
+}
+
+/* ------------------------------------------------------------------ */
+/* R4: FP4 group quantisation of one entry into one record ([P1] 3.1;
+ * [P2] "P4 main KV").  Returns the number of non-finite inputs, which are
+ * treated as 0 for both the group maximum and their code.               */
+int orc_quantize_entry(const orc_cfg* c, const float* e, uint8_t* rec) {
+    int D = c->latent_dim + c->rope_dim;
+    int start[1024], len[1024];
+    int ng = orc_groups(c, start, len);
+    int nonfinite = 0;
+    memset(rec, 0, (size_t)orc_record_bytes(c, 1));
+    for (int gi = 0; gi < ng; ++gi) {
+        float a = 0.0f;
+        for (int d = start[gi]; d < start[gi] + len[gi]; ++d) {
+            float x = e[d];
+            if (!isfinite(x)) continue;
+            if (fabsf(x) > a) a = fabsf(x);
+        }
+        float s = a / 6.0f;
+        if (c->scale_fmt == ORC_SCALE_UE4M3) {
+            int sb = orc_e4m3_encode(s);
+            rec[D / 2 + gi] = (uint8_t)sb;
+            s = orc_e4m3_value(sb);
+        } else {
+            memcpy(rec + D / 2 + 4 * gi, &s, 4);
+        }
+        for (int d = start[gi]; d < start[gi] + len[gi]; ++d) {
+            float x = e[d];
+            int code = 0;
+            if (!isfinite(x))
+                ++nonfinite;
+            else if (s > 0.0f)
+                code = orc_e2m1_encode(x / s);
+            rec[d / 2] |= (uint8_t)((d & 1) ? (code << 4) : code);
+        }
+    }
+    return nonfinite;
+}
+
+/* Dequantisation before attention ([P2] "P4 main KV": FP4 is storage
+ * only): x = E2M1(code) * scale, in fp32.                               */
+void orc_dequantize_entry(const orc_cfg* c, const uint8_t* rec, float* x) {
+    int D = c->latent_dim + c->rope_dim;
+    int start[1024], len[1024];
+    int ng = orc_groups(c, start, len);
+    for (int gi = 0; gi < ng; ++gi) {
+        float s;
+        if (c->scale_fmt == ORC_SCALE_UE4M3)
+            s = orc_e4m3_value(rec[D / 2 + gi]);
+        else
+            memcpy(&s, rec + D / 2 + 4 * gi, 4);
+        for (int d = start[gi]; d < start[gi] + len[gi]; ++d) {
+            int code = (d & 1) ? (rec[d / 2] >> 4) : (rec[d / 2] & 15);
+            x[d] = orc_e2m1_value(code) * s;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Pack: append n_new/2 compressed entries per sequence, with their
+ * indexer keys, at position n_entries[b]; then advance n_entries[b].
+ * tokens [B][n_new][D] fp32 (bf16 inputs widened exactly by the caller),
+ * idxk_new [B][n_new/2][Di], records [B][cap][record_bytes(padded)],
+ * idx_cache [B][cap][Di].                                               */
+int orc_pack(const orc_cfg* c, int B, int n_new, const float* tokens,
+             const float* g, const int8_t* idxk_new, int cap, uint8_t* records,
+             int8_t* idx_cache, int32_t* n_entries, uint32_t* status) {
+    int D = c->latent_dim + c->rope_dim;
+    int rb = orc_record_bytes(c, 1);
+    int half = n_new / 2;
+    if (n_new < 0 || (n_new & 1)) return ORC_ERR_INVALID;
+    for (int b = 0; b < B; ++b)
+        if (n_entries[b] < 0 || n_entries[b] + half > cap) return ORC_ERR_CAPACITY;
+    float* e = (float*)malloc(sizeof(float) * (size_t)D);
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < half; ++i) {
+            const float* k0 = tokens + ((size_t)b * n_new + 2 * i) * D;
+            const float* k1 = k0 + D;
+            int64_t pos = n_entries[b] + i;
+            orc_compress_pair(k0, k1, g, D, e);
+            if (orc_quantize_entry(c, e, records + ((size_t)b * cap + pos) * rb))
+                *status |= ORC_ST_NONFINITE;
+            memcpy(idx_cache + ((size_t)b * cap + pos) * c->idx_dim,
+                   idxk_new + ((size_t)b * half + i) * c->idx_dim,
+                   (size_t)c->idx_dim);
+        }
+        n_entries[b] += half;
+    }
+    free(e);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Lightweight indexer ([P2] breakthrough 4 "用一个轻量索引器给所有历史
+ * token 打分"): score_j = sum_d q_d k_{j,d}, int8 x int8 -> int32.       */
+void orc_index_scores(const int8_t* q, const int8_t* keys, int n, int di,
+                      int32_t* scores) {
+    for (int j = 0; j < n; ++j) {
+        int32_t s = 0;
+        for (int d = 0; d < di; ++d) s += (int32_t)q[d] * (int32_t)keys[(size_t)j * di + d];
+        scores[j] = s;
+    }
+}
+
+typedef struct {
+    int32_t score;
+    int32_t idx;
+} orc_scored;
+
+static int orc_by_score_desc_idx_asc(const void* pa, const void* pb) {
+    const orc_scored* a = (const orc_scored*)pa;
+    const orc_scored* b = (const orc_scored*)pb;
+    if (a->score != b->score) return (a->score > b->score) ? -1 : 1;
+    return (a->idx < b->idx) ? -1 : (a->idx > b->idx);
+}
+
+static int orc_int_asc(const void* pa, const void* pb) {
+    int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    return (a > b) - (a < b);
+}
+
+/* Top-K ([P2] breakthrough 4 "只挑分数最高的 512 个"): order all n
+ * entries by (score descending, index ascending), keep the first
+ * min(k, n), write them sorted by index ascending and pad with -1.
+ * Returns the number kept.                                              */
+int orc_topk(const int32_t* scores, int n, int k, int32_t* out) {
+    orc_scored* v = (orc_scored*)malloc(sizeof(orc_scored) * (size_t)(n > 0 ? n : 1));
+    for (int j = 0; j < n; ++j) {
+        v[j].score = scores[j];
+        v[j].idx = j;
+    }
+    qsort(v, (size_t)n, sizeof(orc_scored), orc_by_score_desc_idx_asc);
+    int kept = n < k ? n : k;
+    for (int i = 0; i < kept; ++i) out[i] = v[i].idx;
+    qsort(out, (size_t)kept, sizeof(int32_t), orc_int_asc);
+    for (int i = kept; i < k; ++i) out[i] = -1;
+    free(v);
+    return kept;
+}
+
+/* index + top-K for a batch; scores (optional) [B][cap] receives the
+ * visible scores (entries past n_entries[b] are left untouched).        */
+int orc_index_topk(const orc_cfg* c, int B, const int8_t* idx_q,
+                   const int8_t* idx_cache, int cap, const int32_t* n_entries,
+                   int32_t* topk, int32_t* scores_out) {
+    int32_t* s = (int32_t*)malloc(sizeof(int32_t) * (size_t)(cap > 0 ? cap : 1));
+    for (int b = 0; b < B; ++b) {
+        int n = n_entries[b];
+        if (n < 0 || n > cap) {
+            free(s);
+            return ORC_ERR_CAPACITY;
+        }
+        orc_index_scores(idx_q + (size_t)b * c->idx_dim,
+                         idx_cache + (size_t)b * cap * c->idx_dim, n, c->idx_dim, s);
+        if (scores_out) memcpy(scores_out + (size_t)b * cap, s, sizeof(int32_t) * (size_t)n);
+        orc_topk(s, n, c->topk, topk + (size_t)b * c->topk);
+    }
+    free(s);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* R5: decode attention for one query token, all heads, in fp64 ([P2]
+ * breakthrough 2: heads share one 512+64 latent entry, values are the
+ * latent; breakthrough 4: window + top-512 global branch).
+ * q [H][D], keys [nk][D]; out [H][Dv]; lse [H] (natural log).
+ * nk == 0 gives out = 0 and lse = -inf.                                 */
+void orc_attention(const float* q, int H, int D, int Dv, const float* keys,
+                   int nk, double sm_scale, double* out, double* lse) {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1));
+    for (int h = 0; h < H; ++h) {
+        double* o = out + (size_t)h * Dv;
+        for (int d = 0; d < Dv; ++d) o[d] = 0.0;
+        if (nk == 0) {
+            lse[h] = -INFINITY;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int j = 0; j < nk; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc += (double)q[(size_t)h * D + d] * (double)keys[(size_t)j * D + d];
+            s[j] = sm_scale * acc;
+            if (s[j] > m) m = s[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j < nk; ++j) {
+            s[j] = exp(s[j] - m);
+            l += s[j];
+        }
+        for (int j = 0; j < nk; ++j) {
+            double p = s[j] / l;
+            for (int d = 0; d < Dv; ++d) o[d] += p * (double)keys[(size_t)j * D + d];
+        }
+        lse[h] = m + log(l);
+    }
+    free(s);
+}
+
+/* Sparse decode attention for a batch: keys = dequantised records of the
+ * selected entries (index -1 is padding and skipped) followed by the
+ * window's window_len raw tokens.  Indices outside [0, n_entries[b]) are
+ * skipped and reported through *status.
+ * q [B][H][D]; records [B][cap][rb]; topk [B][K]; window [B][W][D];
+ * out [B][H][Dv]; lse [B][H].                                           */
+int orc_sparse_decode(const orc_cfg* c, int B, const float* q,
+                      const uint8_t* records, int cap, const int32_t* n_entries,
+                      const int32_t* topk, const float* window, int window_len,
+                      double* out, double* lse, uint32_t* status) {
+    int D = c->latent_dim + c->rope_dim, Dv = c->latent_dim, H = c->n_heads;
+    int rb = orc_record_bytes(c, 1);
+    if (window_len < 0 || window_len > c->window) return ORC_ERR_INVALID;
+    float* keys = (float*)malloc(sizeof(float) * (size_t)(c->topk + c->window + 1) * D);
+    for (int b = 0; b < B; ++b) {
+        int nk = 0;
+        for (int i = 0; i < c->topk; ++i) {
+            int32_t j = topk[(size_t)b * c->topk + i];
+            if (j == -1) continue;
+            if (j < 0 || j >= n_entries[b]) {
+                *status |= ORC_ST_BAD_INDEX;
+                continue;
+            }
+            orc_dequantize_entry(c, records + ((size_t)b * cap + j) * rb, keys + (size_t)nk * D);
+            ++nk;
+        }
+        for (int t = 0; t < window_len; ++t, ++nk)
+            memcpy(keys + (size_t)nk * D, window + ((size_t)b * c->window + t) * D,
+                   sizeof(float) * (size_t)D);
+        orc_attention(q + (size_t)b * H * D, H, D, Dv, keys, nk, c->sm_scale,
+                      out + (size_t)b * H * Dv, lse + (size_t)b * H);
+    }
+    free(keys);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* CSA2 layer group ([P2] part 4 "CSA2：三种模式，40 层只存 4 份"):
+ *  Full    -- scores the stored cache with its own indexer q, own top-K;
+ *  Reindex -- borrows the Full layer's stored main KV and indexer K and
+ *             rescores with its own indexer q;
+ *  Reuse   -- borrows the latest Full/Reindex layer's top-K indices.
+ * Every layer has its own q and its own window.  All layers of the call
+ * read the one stored cache (the Full layer's).  Arrays are layer-major:
+ * q [L][B][H][D], idx_q [L][B][Di], windows [L][B][W][D],
+ * out [L][B][H][Dv], lse [L][B][H], topk [L][B][K].                     */
+int orc_group_step(const orc_cfg* c, int n_layers, const int* modes, int B,
+                   const float* q, const int8_t* idx_q, const float* windows,
+                   int window_len, const uint8_t* records,
+                   const int8_t* idx_cache, int cap, const int32_t* n_entries,
+                   double* out, double* lse, int32_t* topk, uint32_t* status) {
+    int D = c->latent_dim + c->rope_dim, Dv = c->latent_dim, H = c->n_heads;
+    int K = c->topk;
+    if (n_layers < 1 || modes[0] == ORC_MODE_REUSE) return ORC_ERR_INVALID;
+    int head = -1;
+    for (int l = 0; l < n_layers; ++l) {
+        int32_t* tk = topk + (size_t)l * B * K;
+        if (modes[l] == ORC_MODE_FULL || modes[l] == ORC_MODE_REINDEX) {
+            int rc = orc_index_topk(c, B, idx_q + (size_t)l * B * c->idx_dim,
+                                    idx_cache, cap, n_entries, tk, NULL);
+            if (rc) return rc;
+            head = l;
+        } else if (modes[l] == ORC_MODE_REUSE) {
+            memcpy(tk, topk + (size_t)head * B * K, sizeof(int32_t) * (size_t)B * K);
+        } else {
+            return ORC_ERR_INVALID;
+        }
+        int rc = orc_sparse_decode(c, B, q + (size_t)l * B * H * D, records, cap,
+                                   n_entries, tk,
+                                   windows + (size_t)l * B * c->window * D,
+                                   window_len, out + (size_t)l * B * H * Dv,
+                                   lse + (size_t)l * B * H, status);
+        if (rc) return rc;
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Bytes resident for one sequence ([P2] "890 字节是怎么算出来的": count
+ * the FP4 main entry with its scales plus the indexer key): stored
+ * records (padded to the record stride, or not) + int8 indexer rows +
+ * every layer's own window of raw keys.                                 */
+uint64_t orc_bytes_resident(const orc_cfg* c, int64_t entries, int n_layers,
+                            int window_elem_bytes, int padded) {
+    int64_t D = c->latent_dim + c->rope_dim;
+    return (uint64_t)(entries * orc_record_bytes(c, padded) + entries * c->idx_dim +
+                      (int64_t)n_layers * c->window * D * window_elem_bytes);
+}
