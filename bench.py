@@ -1,0 +1,498 @@
+"""Benchmark: sparse FP4-KV decode query-tokens/s and achieved HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one decode token for every sequence of the batch through the whole
+hot path: pack of the token pair that completes at this step (2:1 gated
+compression, FP4 group quantisation, indexer-key append), then the CSA2
+layer group (indexer scan + exact top-K on every Full/Reindex layer, sparse
+attention over top-K + window on every layer).  The K timed steps are
+captured into one CUDA graph and replayed once between barriers; the time is
+taken with CUDA events on the launching stream, max over ranks.  Inputs are
+seeded synthetic tensors shaped like the pages' workloads (no weights, no
+datasets).  With N > 1 (torchrun) each rank decodes its own batch of
+sequences (independent problems, no collective on the data path: weak
+scaling).
+
+--impl reference times the CPU oracle on the same workload and metric
+(bounded per-step sample: one sequence) on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse FP4-KV decode query-tokens/s; achieved HBM GB/s vs 8 TB/s"
+UNIT = "query-tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", default="batch32x128k")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- bytes
+def record_unpadded(w):
+    n_groups = -(-w.latent // w.group) + -(-w.rope // w.group)
+    return w.dim // 2 + n_groups * (1 if w.scale_fmt == 1 else 4)
+
+
+def act_bytes(w):
+    return 2 if w.act == "bf16" else 4
+
+
+def scan_bytes(w, n):
+    """Algorithmic bytes of one indexer scan over n entries, one sequence."""
+    return n * w.idx_dim + w.idx_dim
+
+
+def attn_bytes(w):
+    """Algorithmic bytes of one attention problem (one sequence, one layer)."""
+    a = act_bytes(w)
+    return (w.topk * record_unpadded(w) + w.window * w.dim * a + w.heads * w.dim * a
+            + w.heads * w.latent * 4 + w.topk * 4)
+
+
+def pack_bytes(w, entries):
+    """Algorithmic bytes of packing `entries` entries (2 raw tokens each)."""
+    return entries * (2 * w.dim * act_bytes(w) + record_unpadded(w) + 2 * w.idx_dim)
+
+
+def step_bytes(w, n):
+    heads = sum(1 for m in w.modes if m != 2)
+    return w.batch * (pack_bytes(w, 1) + heads * scan_bytes(w, n) + w.layers * attn_bytes(w))
+
+
+# ----------------------------------------------------------------------------- peaks / clocks
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, enabled=True):
+        self.proc = None
+        self.out = os.path.join("/tmp", f"kvc_clocks_{os.getpid()}.csv")
+        self.gpu = gpu_index
+        if enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=open(self.out, "w"), stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.out):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        sm = sorted(r[0] for r in rows)
+        loaded = [r for r in rows if r[0] >= 0.5 * max(sm)]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v == "Active"})
+        med = float(np.median([r[0] for r in loaded]))
+        return {"sm_mhz": med, "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def traffic_for(kernel):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the kernel source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.split("=", 1)
+            kv[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "fp4_compressed_kv_b200", "csrc", kv.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if h != kv.get("source_sha256_16"):
+        return None
+    return kv
+
+
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_decode_sample(w, seconds, seed_shift=0):
+    """Time the CPU oracle on single-sequence decode steps of workload w.
+    Returns (steps, elapsed_s, description).  Setup (packing the prefix with the
+    oracle) is not timed; each timed step packs one pair, then runs the layer
+    group (scan + top-K per Full/Reindex layer, attention per layer)."""
+    import torch
+
+    import oracle
+    from fp4_compressed_kv_b200 import synth
+    ws = w.scaled(batch=1, seed=w.seed + seed_shift)
+    T = ws.context
+    inp = synth.make_inputs(ws, "cpu", with_tokens=False)
+    cfg = oracle.make_cfg(ws.latent, ws.rope, ws.group, ws.scale_fmt, ws.idx_dim, ws.topk,
+                          ws.window, ws.heads, ws.sm_scale)
+    N = ws.entries
+    cap = N + 4096
+    rb = oracle.record_bytes(cfg)
+    rec = np.zeros((1, cap, rb), np.uint8)
+    ic = np.zeros((1, cap, ws.idx_dim), np.int8)
+    ic[0, :N] = inp["idx_k"][0].numpy()
+    # records: the oracle packs its own entries; only the ones a step can select
+    # matter, but the sample packs a full contiguous prefix block so any index
+    # is valid (entries beyond the packed block are packed lazily below).
+    n = np.array([N], np.int32)
+    g = torch.Generator().manual_seed(ws.seed + 99)
+    gate = inp["gate"].numpy()
+    q = inp["q"].float().numpy()
+    iq = inp["idx_q"].numpy()
+    win = inp["windows"].float().numpy()
+    packed = np.zeros(cap, bool)
+
+    def ensure(idx_rows):
+        need = [int(j) for j in idx_rows if j >= 0 and not packed[j]]
+        if not need:
+            return
+        toks = (torch.randn(len(need), 2, ws.dim, generator=g) ).to(ws.torch_dtype).float().numpy()
+        for t, j in zip(toks, need):
+            e = oracle.compress_pair(t[0], t[1], gate)
+            rec[0, j] = oracle.quantize_entry(cfg, e)[0]
+            packed[j] = True
+
+    steps = 0
+    t_start = time.perf_counter()
+    timed = 0.0
+    while timed < seconds or steps == 0:
+        # one decode step: pack the completed pair, then the layer group
+        t0 = time.perf_counter()
+        newt = torch.randn(1, 2, ws.dim, generator=g).to(ws.torch_dtype).float().numpy()
+        newk = torch.randint(-127, 128, (1, 1, ws.idx_dim), generator=g, dtype=torch.int8).numpy()
+        if n[0] >= cap:
+            n[0] = N
+        oracle.pack(cfg, newt, gate, newk, rec, ic, n)
+        packed[n[0] - 1] = True
+        t1 = time.perf_counter()
+        # the records a step may select must exist: pack them (untimed)
+        tk_all = [oracle.index_topk(cfg, iq[l], ic, n) for l in range(ws.layers)
+                  if ws.modes[l] != 2]
+        for tk in tk_all:
+            ensure(tk[0])
+        t2 = time.perf_counter()
+        oracle.group_step(cfg, list(ws.modes), q, iq, win, ws.window, rec, ic, n)
+        t3 = time.perf_counter()
+        timed += (t1 - t0) + (t3 - t2)
+        steps += 1
+        if time.perf_counter() - t_start > 10 * seconds:
+            break
+    desc = (f"{steps} single-sequence decode steps of {w.name} (N={N} entries, "
+            f"{ws.layers} layer(s), 1 core, oracle C code)")
+    return steps, timed, desc
+
+
+# ----------------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from fp4_compressed_kv_b200 import build, kvc, synth
+    from fp4_compressed_kv_b200 import dist as kd
+
+    rank, world, local = kd.world()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    build.build()
+
+    w0 = synth.WORKLOADS[args.config]
+    w = kd.rank_workload(w0, rank)  # each rank decodes its own sequences
+    cfg = kvc.config_for(w)
+    B, L, H = w.batch, w.layers, w.heads
+    N0 = w.entries
+    cap = N0 + args.warmup + args.steps + 64
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+
+    # ---- build the cache: pack the whole context on the device (untimed)
+    inp = synth.make_inputs(w, dev)
+    cache = kvc.Cache(cfg, B, cap, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kvc.pack(cfg, inp["tokens"], inp["gate"], inp["idx_k"], cache, status=status)
+    torch.cuda.synchronize()
+    del inp["tokens"]
+    torch.cuda.empty_cache()
+    gate = inp["gate"]
+    q, idx_q, windows = inp["q"], inp["idx_q"], inp["windows"]
+    ws = kvc.workspace(cfg, B, cap, device=dev)
+    out = torch.empty(L, B, H, w.latent, device=dev)
+    lse = torch.empty(L, B, H, device=dev)
+    topk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
+    nsteps = args.warmup + args.steps
+    newp = synth.make_new_tokens(w, 2 * nsteps, dev)
+    pair_tok = [newp["tokens"][:, 2 * s:2 * s + 2].contiguous() for s in range(nsteps)]
+    pair_idx = [newp["idx_k"][:, s:s + 1].contiguous() for s in range(nsteps)]
+    modes = list(w.modes)
+
+    def step(s):
+        kvc.pack(cfg, pair_tok[s], gate, pair_idx[s], cache, status=status)
+        kvc.layer_group_step(cfg, modes, q, idx_q, windows, w.window, cache, out, topk, ws,
+                             lse=lse, status=status)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    # ---- capture the K timed steps into one graph (events per kernel inside)
+    kvc.trace_begin(16 * args.steps + 16)
+    launches0 = kvc.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(args.warmup, nsteps):
+            step(s)
+    launches = kvc.launch_count() - launches0
+    kvc.trace_end()
+    n_before = cache.n_entries.clone()
+
+    clocks = Clocks(local, enabled=not args.no_clocks)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kd.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kd.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    assert status.item() == 0, f"device status {status.item()}"
+    n_after = cache.n_entries.clone()
+    assert torch.all(n_after - n_before == args.steps)
+
+    ms_max = kd.max_over_ranks(ms, device=dev)
+    value = kd.job_throughput(args.steps, B, world, ms_max)
+
+    # per-kernel device times from the traced launches inside the timed graph
+    kernels = {}
+    for name in ("pack", "pack_commit", "index_scan", "topk_collect", "topk_finalize",
+                 "attn_mma", "attn_simt", "attn_merge"):
+        cnt, tot = kvc.trace_kernel(name)
+        if cnt:
+            kernels[name] = {"launches": cnt, "ms_total": round(tot, 4),
+                             "us_avg": round(1e3 * tot / cnt, 2)}
+    n_mean = N0 + args.warmup + (args.steps + 1) / 2.0  # entries visible during the timed steps
+    heads_layers = sum(1 for m in modes if m != 2)
+    per_launch = {
+        "index_scan": B * scan_bytes(w, n_mean),
+        "attn_mma": B * attn_bytes(w),
+        "attn_simt": B * attn_bytes(w),
+        "pack": B * pack_bytes(w, 1),
+    }
+    dominant = max(kernels, key=lambda k: kernels[k]["ms_total"])
+    peak, peak_kind = peaks()
+    dom = kernels[dominant]
+    achieved = per_launch.get(dominant, 0) / (dom["us_avg"] * 1e-6) / 1e9
+    traffic = traffic_for(dominant)
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_kind} hbm_gbs",
+                "bytes_per_launch": int(per_launch.get(dominant, 0)),
+                "traffic": (int(float(traffic["dram_bytes_per_launch"])) if traffic else None)}
+    sb = step_bytes(w, n_mean)
+    step_gbs = sb / (ms_max / args.steps * 1e-3) / 1e9
+
+    # ---- pack throughput on fresh tokens (the batched workload's pack case)
+    pack_info = None
+    if w.pack_new:
+        pk = synth.make_new_tokens(w, w.pack_new, dev, seed_offset=11)
+        pcache = kvc.Cache(cfg, B, w.pack_new // 2, device=dev)
+        for _ in range(3):
+            pcache.n_entries.zero_()
+            kvc.pack(cfg, pk["tokens"], gate, pk["idx_k"], pcache, status=status)
+        torch.cuda.synchronize()
+        reps = max(5, args.steps)
+        kvc.trace_begin(4 * reps + 8)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            pcache.n_entries.zero_()
+            kvc.pack(cfg, pk["tokens"], gate, pk["idx_k"], pcache, status=status)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        kvc.trace_end()
+        pms = e0.elapsed_time(e1) / reps
+        cnt, tot = kvc.trace_kernel("pack")
+        kus = 1e3 * tot / cnt
+        pbytes = pack_bytes(w, B * w.pack_new // 2)
+        pack_info = {"new_tokens_per_seq": w.pack_new, "tokens_per_s": round(B * w.pack_new / (pms / 1e3)),
+                     "ms_per_call": round(pms, 4), "kernel_us": round(kus, 2),
+                     "kernel_gbs": round(pbytes / (kus * 1e-6) / 1e9, 1),
+                     "kernel_frac": round(pbytes / (kus * 1e-6) / 1e9 / peak, 4),
+                     "bytes_per_call": int(pbytes)}
+        del pk, pcache
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hiq = idx_q.cpu().pin_memory()
+        htok = newp["tokens"][:, :2].cpu().pin_memory()
+        hidx = newp["idx_k"][:, :1].cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq, diq = torch.empty_like(q), torch.empty_like(idx_q)
+        dtok, didx = torch.empty_like(pair_tok[0]), torch.empty_like(pair_idx[0])
+        reps = args.steps
+        cache.n_entries.copy_(n_before)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            diq.copy_(hiq, non_blocking=True)
+            dtok.copy_(htok, non_blocking=True)
+            didx.copy_(hidx, non_blocking=True)
+            kvc.pack(cfg, dtok, gate, didx, cache, status=status)
+            kvc.layer_group_step(cfg, modes, dq, diq, windows, w.window, cache, out, topk, ws,
+                                 lse=lse, status=status)
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        cache.n_entries.copy_(n_before)
+        kd.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te_ms = kd.max_over_ranks(e0.elapsed_time(e1), device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hiq, htok, hidx))
+        d2h = sum(t.numel() * t.element_size() for t in (hout, hlse))
+        e2e = {"value": round(kd.job_throughput(reps, B, world, te_ms), 1), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(te_ms / reps, 4)}
+
+    # ---- CPU oracle baseline (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        steps_c, secs, desc = oracle_decode_sample(w0, args.cpu_seconds)
+        cpu = {"value": round(steps_c / secs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": desc, "seconds": round(secs, 2)}
+
+    del graph
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.act == "bf16" else "f32",
+        "data": "synthetic (seeded; no weights or datasets)",
+        "config": {"workload": w.name, "batch_per_gpu": B, "context_tokens": w.context,
+                   "entries": N0, "layers": [["Full", "Reindex", "Reuse"][m] for m in modes],
+                   "heads": H, "latent": w.latent, "rope": w.rope, "group": w.group,
+                   "scale": "ue4m3" if w.scale_fmt == 1 else "f32", "topk": w.topk,
+                   "window": w.window, "idx_dim": w.idx_dim, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (indexer scan reads %.0f MB per step)"
+                         % (B * scan_bytes(w, N0) * heads_layers / 1e6),
+                   "timing": "K steps in one CUDA graph, CUDA events, max over ranks"},
+        "hbm_gbs_step": round(step_gbs, 1),
+        "step_frac_of_peak": round(step_gbs / peak, 4),
+        "step_bytes": int(sb),
+        "roofline": roofline,
+        "kernels": kernels,
+        "pack": pack_info,
+        "bytes_resident_per_token": {
+            "unpadded": round(kvc.bytes_resident(cfg, N0, L, False) / w.context, 2),
+            "padded": round(kvc.bytes_resident(cfg, N0, L, True) / w.context, 2)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        kd.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    from fp4_compressed_kv_b200 import synth
+    from fp4_compressed_kv_b200 import dist as kd
+    rank, world, _ = kd.world()
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.config]
+    # warm-up samples, then K timed samples of one single-sequence step each
+    oracle_decode_sample(w, 0.0)
+    total_steps, total_s = 0, 0.0
+    for k in range(args.steps):
+        s, secs, desc = oracle_decode_sample(w, 0.0, seed_shift=k + 1)
+        total_steps += s
+        total_s += secs
+    v = total_steps / total_s
+    res = {"metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_s / total_steps, 2),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded; no weights or datasets)", "impl": "reference",
+           "config": {"workload": w.name, "batch_per_gpu": w.batch, "context_tokens": w.context,
+                      "entries": w.entries, "sample": "one sequence per step"},
+           "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

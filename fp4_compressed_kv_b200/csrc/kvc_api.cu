@@ -1,0 +1,429 @@
+// kvc_api.cu -- the C ABI of libkvc.so: argument validation, workspace
+// layout, CSA2 layer-group orchestration, tracing and the format codecs.
+// Every entry point validates on the host and then only enqueues kernels on
+// the caller's stream; nothing here allocates device memory or synchronises.
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+#include <atomic>
+
+#include "kvc_internal.cuh"
+
+namespace kvc {
+
+bool derive_shape(const kvc_config* c, Shape* s) {
+    if (!c) return false;
+    if (c->latent_dim <= 0 || c->latent_dim % 8 || c->rope_dim < 0 || c->rope_dim % 8) return false;
+    const int D = c->latent_dim + c->rope_dim;
+    if (D > 1024) return false;
+    const int G = c->group;
+    if (G < 8 || G > 256 || (G & (G - 1)) || c->latent_dim % G) return false;
+    if (c->scale_fmt != KVC_SCALE_F32 && c->scale_fmt != KVC_SCALE_UE4M3) return false;
+    const int di = c->idx_dim;
+    if (di != 16 && di != 32 && di != 64 && di != 128 && di != 256) return false;
+    if (c->topk < 1 || c->topk > 2048) return false;
+    if (c->window < 0 || c->window > 65536) return false;
+    if (c->n_heads < 1 || c->n_heads > 256) return false;
+    if (!(c->sm_scale > 0.f) || !(c->sm_scale < 1e30f)) return false;
+    if (c->act_dtype != KVC_F32 && c->act_dtype != KVC_BF16) return false;
+    s->D = D;
+    s->Dv = c->latent_dim;
+    s->G = G;
+    s->lpg = G / 8;
+    s->n_groups = (c->latent_dim + G - 1) / G + (c->rope_dim + G - 1) / G;
+    s->code_bytes = D / 2;
+    s->scale_bytes = c->scale_fmt == KVC_SCALE_UE4M3 ? 1 : 4;
+    s->rec_unpadded = s->code_bytes + s->n_groups * s->scale_bytes;
+    s->rb = (s->rec_unpadded + 15) / 16 * 16;
+    s->act_bytes = c->act_dtype == KVC_BF16 ? 2 : 4;
+    return true;
+}
+
+// ------------------------------------------------------------------ tracing
+namespace {
+struct TraceState {
+    std::mutex mu;
+    bool on = false;
+    int max = 0;
+    std::vector<cudaEvent_t> ev;  // 2 per launch
+    std::vector<std::string> name;
+    int used = 0;
+    int open = -1;
+};
+TraceState& trace() {
+    static TraceState t;
+    return t;
+}
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void trace_before(const char* name, cudaStream_t s) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    TraceState& t = trace();
+    std::lock_guard<std::mutex> lk(t.mu);
+    t.open = -1;
+    if (!t.on || t.used >= t.max) return;
+    t.open = t.used++;
+    t.name[t.open] = name;
+    cudaEventRecord(t.ev[2 * t.open], s);
+}
+
+void trace_after(cudaStream_t s) {
+    TraceState& t = trace();
+    std::lock_guard<std::mutex> lk(t.mu);
+    if (t.open >= 0) cudaEventRecord(t.ev[2 * t.open + 1], s);
+    t.open = -1;
+}
+
+// ------------------------------------------------------------------ codecs
+namespace {
+__global__ void codec_kernel(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ out,
+                             int e4m3) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = x[i];
+        uint32_t r;
+        if (e4m3) {
+            r = e4m3_from_f32(v);
+        } else {
+            float w[8] = {fminf(fmaxf(v, -6.f), 6.f), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            r = e2m1x8_from_f32(w) & 15u;
+        }
+        out[i] = (uint8_t)r;
+    }
+}
+}  // namespace
+
+cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    trace_before("fp4_codec", s);
+    codec_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, n, out, e4m3);
+    trace_after(s);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ workspace
+namespace {
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+    size_t scores, hist, cands, part_o, part_ml, total;
+};
+WsLayout ws_layout(const kvc_config& c, const Shape& sh, int batch, int cap) {
+    WsLayout w;
+    size_t off = 0;
+    w.scores = off;
+    off = up(off + (size_t)batch * cap * 4);
+    w.hist = off;  // hist [B][kBins] followed by cand_count [B]
+    off = up(off + (size_t)batch * (kBins + 1) * 4);
+    w.cands = off;
+    off = up(off + (size_t)batch * kMaxCand * 8);
+    w.part_o = off;
+    off = up(off + (size_t)batch * c.n_heads * kMaxSplit * sh.Dv * 4);
+    w.part_ml = off;
+    off = up(off + (size_t)batch * c.n_heads * kMaxSplit * 2 * 4);
+    w.total = off;
+    return w;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool device_ok() {
+    static int checked[64] = {};  // 0 unknown, 1 ok, 2 bad
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (checked[dev] == 0) {
+        int major = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        checked[dev] = major == 10 ? 1 : 2;
+    }
+    return checked[dev] == 1;
+}
+
+kvc_status check_cache(const kvc_cache* cache, const Shape& sh) {
+    if (!cache || !cache->records || !cache->idx_k || !cache->n_entries) return KVC_ERR_INVALID;
+    if (cache->batch < 0 || cache->capacity < 0) return KVC_ERR_INVALID;
+    if (cache->batch > 65535) return KVC_ERR_CAPACITY;  // batch is a grid dimension
+    if (!aligned(cache->records, 16) || !aligned(cache->idx_k, 16) || !aligned(cache->n_entries, 4))
+        return KVC_ERR_INVALID;
+    if ((int64_t)cache->capacity * sh.rb > ((int64_t)1 << 40)) return KVC_ERR_CAPACITY;
+    return KVC_OK;
+}
+
+kvc_status check_ws(void* ws, size_t ws_bytes, const kvc_config& c, const Shape& sh, int batch,
+                    int cap, WsLayout* w) {
+    *w = ws_layout(c, sh, batch, cap);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < w->total) return KVC_ERR_WORKSPACE;
+    return KVC_OK;
+}
+
+kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* cache,
+                    int32_t* topk, int32_t* scores, unsigned char* ws, const WsLayout& w,
+                    uint32_t* st, cudaStream_t s) {
+    TopkArgs a;
+    a.idx_q = idx_q;
+    a.idx_k = cache->idx_k;
+    a.n_entries = cache->n_entries;
+    a.batch = cache->batch;
+    a.capacity = cache->capacity;
+    a.topk = c.topk;
+    a.di = c.idx_dim;
+    a.topk_idx = topk;
+    a.scores = scores ? scores : reinterpret_cast<int32_t*>(ws + w.scores);
+    a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
+    a.cand_count = a.hist + (size_t)cache->batch * kBins;
+    a.cands = reinterpret_cast<unsigned long long*>(ws + w.cands);
+    a.status = st;
+    return launch_index_topk(a, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+kvc_status run_attn(const kvc_config& c, const Shape& sh, const void* q, const kvc_cache* cache,
+                    const int32_t* topk, const void* window, int window_len, float* out,
+                    float* lse, unsigned char* ws, const WsLayout& w, uint32_t* st,
+                    cudaStream_t s) {
+    AttnArgs a;
+    a.q = q;
+    a.records = static_cast<const uint8_t*>(cache->records);
+    a.n_entries = cache->n_entries;
+    a.topk_idx = topk;
+    a.window = window;
+    a.window_len = window_len;
+    a.window_stride = c.window;
+    a.batch = cache->batch;
+    a.capacity = cache->capacity;
+    a.out = out;
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float*>(ws + w.part_o);
+    a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+    a.status = st;
+    return launch_attention(c, sh, a, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+}  // namespace
+
+}  // namespace kvc
+
+using namespace kvc;
+
+extern "C" {
+
+size_t kvc_record_bytes(const kvc_config* cfg) {
+    Shape sh;
+    return derive_shape(cfg, &sh) ? (size_t)sh.rb : 0;
+}
+
+size_t kvc_bytes_resident(const kvc_config* cfg, int64_t entries, int n_layers, int padded) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh) || entries < 0 || n_layers < 0) return 0;
+    const int64_t rec = padded ? sh.rb : sh.rec_unpadded;
+    return (size_t)(entries * rec + entries * cfg->idx_dim +
+                    (int64_t)n_layers * cfg->window * sh.D * sh.act_bytes);
+}
+
+size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh) || batch < 0 || capacity < 0) return 0;
+    return ws_layout(*cfg, sh, batch, capacity).total;
+}
+
+kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new, const float* gate,
+                    const int8_t* idx_k_new, const kvc_cache* cache, uint32_t* dev_status,
+                    void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    kvc_status st = check_cache(cache, sh);
+    if (st != KVC_OK) return st;
+    if (n_new < 0 || (n_new & 1)) return KVC_ERR_INVALID;
+    if (n_new == 0 || cache->batch == 0) return KVC_OK;
+    if (n_new / 2 > cache->capacity) return KVC_ERR_CAPACITY;
+    if (!tokens || !gate || !idx_k_new) return KVC_ERR_INVALID;
+    if (!aligned(tokens, 16) || !aligned(gate, 16) || !aligned(idx_k_new, 16)) return KVC_ERR_INVALID;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    PackArgs a;
+    a.tokens = tokens;
+    a.n_new = n_new;
+    a.batch = cache->batch;
+    a.capacity = cache->capacity;
+    a.gate = gate;
+    a.idx_k_new = idx_k_new;
+    a.records = static_cast<uint8_t*>(cache->records);
+    a.idx_k = cache->idx_k;
+    a.n_entries = cache->n_entries;
+    a.status = dev_status;
+    return launch_pack(*cfg, sh, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVC_OK
+                                                                                     : KVC_ERR_CUDA;
+}
+
+kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q, const kvc_cache* cache,
+                          int32_t* topk_idx, int32_t* scores, void* ws, size_t ws_bytes,
+                          uint32_t* dev_status, void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    kvc_status st = check_cache(cache, sh);
+    if (st != KVC_OK) return st;
+    if (cache->batch == 0) return KVC_OK;
+    if (!idx_q || !topk_idx || !aligned(idx_q, 16) || !aligned(topk_idx, 4)) return KVC_ERR_INVALID;
+    if (scores && !aligned(scores, 4)) return KVC_ERR_INVALID;
+    WsLayout w;
+    if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    return run_topk(*cfg, idx_q, cache, topk_idx, scores, static_cast<unsigned char*>(ws), w,
+                    dev_status, static_cast<cudaStream_t>(stream));
+}
+
+kvc_status kvc_sparse_decode_attn(const kvc_config* cfg, const void* q, const kvc_cache* cache,
+                                  const int32_t* topk_idx, const void* window, int window_len,
+                                  float* out, float* lse, void* ws, size_t ws_bytes,
+                                  uint32_t* dev_status, void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    kvc_status st = check_cache(cache, sh);
+    if (st != KVC_OK) return st;
+    if (cache->batch == 0) return KVC_OK;
+    if (window_len < 0 || window_len > cfg->window) return KVC_ERR_INVALID;
+    if (!q || !topk_idx || !out || (window_len > 0 && !window)) return KVC_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(topk_idx, 4) ||
+        (window && !aligned(window, 16)) || (lse && !aligned(lse, 4)))
+        return KVC_ERR_INVALID;
+    WsLayout w;
+    if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    return run_attn(*cfg, sh, q, cache, topk_idx, window, window_len, out, lse,
+                    static_cast<unsigned char*>(ws), w, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers, const int32_t* modes,
+                                const void* q, const int8_t* idx_q, const void* windows,
+                                int window_len, const kvc_cache* cache, float* out, float* lse,
+                                int32_t* topk, void* ws, size_t ws_bytes, uint32_t* dev_status,
+                                void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    kvc_status st = check_cache(cache, sh);
+    if (st != KVC_OK) return st;
+    if (n_layers < 1 || !modes) return KVC_ERR_INVALID;
+    for (int l = 0; l < n_layers; ++l)
+        if (modes[l] != KVC_FULL && modes[l] != KVC_REINDEX && modes[l] != KVC_REUSE)
+            return KVC_ERR_INVALID;
+    if (modes[0] == KVC_REUSE) return KVC_ERR_INVALID;
+    if (cache->batch == 0) return KVC_OK;
+    if (window_len < 0 || window_len > cfg->window) return KVC_ERR_INVALID;
+    if (!q || !idx_q || !out || !topk || (window_len > 0 && !windows)) return KVC_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(idx_q, 16) || !aligned(out, 16) || !aligned(topk, 4) ||
+        (windows && !aligned(windows, 16)) || (lse && !aligned(lse, 4)))
+        return KVC_ERR_INVALID;
+    const size_t B = (size_t)cache->batch, H = (size_t)cfg->n_heads;
+    const size_t q_stride = B * H * sh.D * sh.act_bytes;
+    const size_t w_stride = B * (size_t)cfg->window * sh.D * sh.act_bytes;
+    if (q_stride % 16 || (w_stride % 16) || (B * cfg->idx_dim) % 16) return KVC_ERR_INVALID;
+    WsLayout w;
+    if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    const size_t K = (size_t)cfg->topk;
+    int head = -1;
+    for (int l = 0; l < n_layers; ++l) {
+        int32_t* tk = topk + (size_t)l * B * K;
+        if (modes[l] == KVC_FULL || modes[l] == KVC_REINDEX) {
+            // Full scores its stored cache; Reindex rescores the same stored
+            // (Full layer's) cache with its own indexer query.
+            st = run_topk(*cfg, idx_q + (size_t)l * B * cfg->idx_dim, cache, tk, nullptr, wsb, w,
+                          dev_status, s);
+            if (st != KVC_OK) return st;
+            head = l;
+        } else {
+            if (cudaMemcpyAsync(tk, topk + (size_t)head * B * K, B * K * 4, cudaMemcpyDeviceToDevice,
+                                s) != cudaSuccess)
+                return KVC_ERR_CUDA;
+        }
+        st = run_attn(*cfg, sh, static_cast<const unsigned char*>(q) + l * q_stride, cache, tk,
+                      windows ? static_cast<const unsigned char*>(windows) + l * w_stride : nullptr,
+                      window_len, out + (size_t)l * B * H * sh.Dv, lse ? lse + (size_t)l * B * H : nullptr,
+                      wsb, w, dev_status, s);
+        if (st != KVC_OK) return st;
+    }
+    return KVC_OK;
+}
+
+kvc_status kvc_e2m1_encode(const float* x, int64_t n, uint8_t* codes, void* stream) {
+    if (n < 0 || (n > 0 && (!x || !codes))) return KVC_ERR_INVALID;
+    if (n > 0 && !device_ok()) return KVC_ERR_DEVICE;
+    return launch_fp4_codec(x, n, codes, 0, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KVC_OK
+               : KVC_ERR_CUDA;
+}
+
+kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stream) {
+    if (n < 0 || (n > 0 && (!x || !bytes))) return KVC_ERR_INVALID;
+    if (n > 0 && !device_ok()) return KVC_ERR_DEVICE;
+    return launch_fp4_codec(x, n, bytes, 1, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KVC_OK
+               : KVC_ERR_CUDA;
+}
+
+kvc_status kvc_trace_begin(int max_launches) {
+    if (max_launches < 1 || max_launches > (1 << 20)) return KVC_ERR_INVALID;
+    TraceState& t = trace();
+    std::lock_guard<std::mutex> lk(t.mu);
+    for (cudaEvent_t e : t.ev) cudaEventDestroy(e);
+    t.ev.assign(2 * (size_t)max_launches, nullptr);
+    for (auto& e : t.ev)
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            t.on = false;
+            return KVC_ERR_CUDA;
+        }
+    t.name.assign(max_launches, std::string());
+    t.max = max_launches;
+    t.used = 0;
+    t.on = true;
+    return KVC_OK;
+}
+
+kvc_status kvc_trace_end(void) {
+    TraceState& t = trace();
+    std::lock_guard<std::mutex> lk(t.mu);
+    t.on = false;
+    return KVC_OK;
+}
+
+kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms) {
+    if (!name || !launches || !total_ms) return KVC_ERR_INVALID;
+    TraceState& t = trace();
+    std::lock_guard<std::mutex> lk(t.mu);
+    int cnt = 0;
+    double sum = 0.0;
+    for (int i = 0; i < t.used; ++i) {
+        if (t.name[i] != name) continue;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, t.ev[2 * i], t.ev[2 * i + 1]) != cudaSuccess) return KVC_ERR_CUDA;
+        ++cnt;
+        sum += ms;
+    }
+    *launches = cnt;
+    *total_ms = sum;
+    return KVC_OK;
+}
+
+uint64_t kvc_launch_count(void) { return g_launches.load(); }
+
+const char* kvc_status_string(kvc_status s) {
+    switch (s) {
+        case KVC_OK: return "ok";
+        case KVC_ERR_INVALID: return "invalid argument or configuration";
+        case KVC_ERR_CAPACITY: return "size exceeds capacity";
+        case KVC_ERR_CUDA: return "CUDA launch or runtime error";
+        case KVC_ERR_UNSUPPORTED: return "unsupported shape";
+        case KVC_ERR_TIMEOUT: return "bounded wait timed out";
+        case KVC_ERR_DEVICE: return "no sm_100 device current";
+        case KVC_ERR_WORKSPACE: return "workspace null, misaligned or too small";
+    }
+    return "unknown status";
+}
+
+const char* kvc_version(void) { return "kvc 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+// kvc_internal.cuh -- declarations shared by the kernels and the C ABI of
+// libkvc.so.  Not installed; the public interface is include/kvc.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvc.h"
+
+namespace kvc {
+
+// Indexer histogram: 2048 bins over the biased int8 x int8 score range.
+constexpr int kBins = 2048;
+// Candidates per sequence kept for the in-shared-memory top-K finish.
+constexpr int kMaxCand = 4096;
+// Upper bound on the number of key splits of one attention problem.
+constexpr int kMaxSplit = 16;
+// Keys per attention chunk.
+constexpr int kChunk = 64;
+// Bound on polls of an mbarrier or flag before a kernel gives up.
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+// Shape facts derived once from a kvc_config.
+struct Shape {
+    int D;          // latent + rope
+    int Dv;         // latent
+    int G;          // group size
+    int lpg;        // lanes (8-channel chunks) per group: G / 8
+    int n_groups;   // latent groups + rope groups
+    int code_bytes; // D / 2
+    int scale_bytes;// 1 (UE4M3) or 4 (fp32)
+    int rec_unpadded;
+    int rb;         // record stride (padded to 16)
+    int act_bytes;  // 2 (bf16) or 4 (fp32)
+};
+
+bool derive_shape(const kvc_config* c, Shape* s);
+
+// Score bias and histogram shift for indexer width di: every int8 x int8 dot
+// of width di lies in [-di*127*128, di*128*128]; adding di*127*128 makes it
+// non-negative and below 2^(log2(di)+15), so >> (log2(di)+4) gives a bin in
+// [0, 2048).
+inline int score_shift(int di) {
+    int l = 0;
+    while ((1 << l) < di) ++l;
+    return l + 4;
+}
+inline int score_bias(int di) { return di * 127 * 128; }
+
+// ------------------------------------------------------------------ tracing
+void trace_before(const char* name, cudaStream_t s);
+void trace_after(cudaStream_t s);
+
+// ------------------------------------------------------------------ launchers
+struct PackArgs {
+    const void* tokens;
+    int n_new, batch, capacity;
+    const float* gate;
+    const int8_t* idx_k_new;
+    uint8_t* records;
+    int8_t* idx_k;
+    int32_t* n_entries;
+    uint32_t* status;
+};
+cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
+                        cudaStream_t s);
+
+struct TopkArgs {
+    const int8_t* idx_q;   // [B][Di]
+    const int8_t* idx_k;   // [B][cap][Di]
+    const int32_t* n_entries;
+    int batch, capacity, topk, di;
+    int32_t* topk_idx;     // [B][K]
+    int32_t* scores;       // [B][cap] (user buffer or workspace)
+    int32_t* hist;         // [B][kBins] (zeroed by the launcher)
+    int32_t* cand_count;   // [B]        (zeroed by the launcher)
+    unsigned long long* cands;  // [B][kMaxCand]
+    uint32_t* status;
+};
+cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
+
+struct AttnArgs {
+    const void* q;          // [B][H][D]
+    const uint8_t* records; // [B][cap][rb]
+    const int32_t* n_entries;
+    const int32_t* topk_idx;// [B][K]
+    const void* window;     // [B][W][D]
+    int window_len, window_stride, batch, capacity;
+    float* out;             // [B][H][Dv]
+    float* lse;             // [B][H] or null
+    float* part_o;          // [B][H][kMaxSplit][Dv]
+    float* part_ml;         // [B][H][kMaxSplit][2]
+    uint32_t* status;
+};
+cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArgs& a,
+                             cudaStream_t s);
+
+cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3,
+                             cudaStream_t s);
+
+// ------------------------------------------------------------------ device helpers
+#ifdef __CUDACC__
+__device__ __forceinline__ void set_status(uint32_t* st, uint32_t bit) {
+    if (st) atomicOr(st, bit);
+}
+
+// Round-to-nearest-even, saturating conversion of a non-negative fp32 to an
+// E4M3 byte (hardware cvt; the value sits in the low byte).
+__device__ __forceinline__ uint32_t e4m3_from_f32(float s) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(s));
+    return r & 0xFFu;
+}
+
+// Exact decode of an E4M3 byte (sign ignored: scales are unsigned).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    if (e == 0) return (float)m * 0x1.0p-9f;
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Eight fp32 values already in [-6, 6] -> eight E2M1 codes in one word,
+// value 2t in the low nibble of byte t; codes of magnitude 0 lose their sign.
+__device__ __forceinline__ uint32_t e2m1x8_from_f32(const float v[8]) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+          "f"(v[7]));
+    const uint32_t mag = w & 0x77777777u;
+    const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;
+    return w & (0x77777777u | nonzero);
+}
+#endif
+
+}  // namespace kvc

@@ -1,0 +1,212 @@
+/*
+ * kvc.h -- C ABI of the compressed-KV sparse decode library (libkvc.so).
+ *
+ * The library implements, on one B200 GPU (sm_100a), the decode hot path of
+ * attention over a KV cache whose entries are compressed 2:1 across tokens
+ * and stored as FP4 E2M1 with per-group scales, as described on two pages:
+ *
+ *  [A] "DeepSeek V1 到 V4.1-Flash，单 token 的 global KV 如何从 389,000 B 压缩到
+ *      890 B的？" (acejoy.com) -- part 3 breakthrough 2 (MLA entry: 512 latent
+ *      + 64 RoPE channels shared by all heads), breakthrough 4 (128-token
+ *      sliding window; a lightweight indexer scores all history and keeps the
+ *      top 512; CSA compresses every 2 tokens into 1 entry), part 4 "CSA2：三种
+ *      模式" (Full / Reindex / Reuse layers), "P4 main KV" (E2M1 with shared
+ *      scales, dequantised before attention), "890 字节是怎么算出来的".
+ *  [B] "DeepSeek V4.1 Flash KV Cache压缩实战：FP4+CSA2+CED将显存降至1/4"
+ *      (gtnt.cn) -- 3.1 (FP4 group quantisation), 3.2 (2:1 key compressor),
+ *      4.3 (group size 32/64/128, ratio 2x).
+ *
+ * Conventions shared by every call
+ *  - Every pointer argument except `cfg`, `cache` and host arrays named as
+ *    such is a DEVICE pointer on the current CUDA device.  The caller owns all
+ *    memory; the library never allocates device memory, never frees, and never
+ *    synchronises.  Work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and the call returns before it runs.
+ *  - Host-detectable errors (bad configuration, null or misaligned pointers,
+ *    sizes out of range, workspace too small) return a kvc_status before
+ *    anything is enqueued.  A failed launch returns KVC_ERR_CUDA.
+ *  - Anomalies only the device can see are OR-ed into `*dev_status` (a device
+ *    uint32; may be NULL) as KVC_DEV_* bits; read it after the stream
+ *    synchronises.  Kernels never trap, and every wait inside a kernel is
+ *    bounded: when a bound is hit the kernel sets KVC_DEV_TIMEOUT and returns.
+ *  - Records and token/query/window rows must start on 16-byte boundaries.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVC_OK = 0,
+    KVC_ERR_INVALID = 1,     /* bad argument or configuration                */
+    KVC_ERR_CAPACITY = 2,    /* a size exceeds what the buffers or kernel hold */
+    KVC_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed          */
+    KVC_ERR_UNSUPPORTED = 4, /* valid but not implemented for this shape      */
+    KVC_ERR_TIMEOUT = 5,
+    KVC_ERR_DEVICE = 6,      /* no sm_100 device current                      */
+    KVC_ERR_WORKSPACE = 7    /* workspace pointer null, misaligned or too small */
+} kvc_status;
+
+typedef enum { KVC_SCALE_F32 = 0, KVC_SCALE_UE4M3 = 1 } kvc_scale_fmt;
+typedef enum { KVC_FULL = 0, KVC_REINDEX = 1, KVC_REUSE = 2 } kvc_mode;
+typedef enum { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
+
+/* device status bits */
+#define KVC_DEV_NONFINITE 0x1u  /* pack met a NaN/Inf channel (coded as 0)     */
+#define KVC_DEV_BAD_INDEX 0x2u  /* a top-K index outside [-1, n_entries)       */
+#define KVC_DEV_CAPACITY 0x4u   /* pack would pass the cache capacity          */
+#define KVC_DEV_TIMEOUT 0x8u    /* a bounded in-kernel wait gave up            */
+#define KVC_DEV_BAD_LENGTH 0x10u /* n_entries outside [0, capacity]            */
+
+/* Shape and format of one compressed cache and its decode attention.
+ *  latent_dim  Dv, latent channels; also the value width ([A] breakthrough 2: 512)
+ *  rope_dim    RoPE channels appended to every key ([A]: 64); D = latent + rope
+ *  group       FP4 group size G ([B] 4.3: 32/64/128); latent and RoPE are grouped
+ *              separately and the last RoPE group may be short
+ *  scale_fmt   per-group scale: fp32, or unsigned E4M3 (one byte)
+ *  idx_dim     int8 indexer key width Di ([A] "890 字节": 128)
+ *  topk        K entries kept by the indexer ([A] breakthrough 4: 512)
+ *  window      W, sliding-window length ([A] breakthrough 4: 128)
+ *  n_heads     H query heads sharing each entry
+ *  sm_scale    softmax scale applied to q.k
+ *  act_dtype   dtype of raw tokens, queries and window keys (fp32 or bf16)   */
+typedef struct {
+    int32_t latent_dim, rope_dim, group, scale_fmt;
+    int32_t idx_dim, topk, window, n_heads;
+    float sm_scale;
+    int32_t act_dtype;
+} kvc_config;
+
+/* One stored cache (the Full layer's).  Caller-owned device buffers:
+ *  records    [batch][capacity][kvc_record_bytes(cfg)] bytes, 16-byte aligned.
+ *             Record = [D/2 bytes of E2M1 codes, channel 2c in the low nibble of
+ *             byte c][one scale per group, in group order: 1 byte UE4M3 or 4
+ *             bytes fp32][zero padding to a multiple of 16 bytes]
+ *  idx_k      [batch][capacity][idx_dim] int8 indexer keys
+ *  n_entries  [batch] int32, entries stored per sequence (visible to the
+ *             indexer: entries 0 .. n_entries-1)                            */
+typedef struct {
+    void* records;
+    int8_t* idx_k;
+    int32_t* n_entries;
+    int32_t batch, capacity;
+} kvc_cache;
+
+/* Bytes of one record (with padding) = the record stride. 0 if cfg invalid. */
+size_t kvc_record_bytes(const kvc_config* cfg);
+
+/* Bytes resident per sequence for `entries` stored entries and `n_layers`
+ * layers each holding its own window of W raw keys (record bytes with or
+ * without padding + indexer rows + windows) -- the per-token accounting of
+ * [A] "890 字节是怎么算出来的" applied to this cache. 0 if cfg invalid.      */
+size_t kvc_bytes_resident(const kvc_config* cfg, int64_t entries, int n_layers,
+                          int padded);
+
+/* Device workspace needed by kvc_index_topk, kvc_sparse_decode_attn and
+ * kvc_layer_group_step for `batch` sequences of up to `capacity` entries. */
+size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity);
+
+/* Append n_new raw tokens per sequence (A1-A3 of the hot path).
+ * tokens    [batch][n_new][D] act_dtype; n_new even: token pairs (2i, 2i+1) are
+ *           compressed into one entry ([A] breakthrough 4 "CSA 把每 2 个 token
+ *           的 KV 压成 1 条"; [B] 3.2).  The pair's weights are the softmax of
+ *           the two gate logits g.k; the weighted sum is quantised per group
+ *           to E2M1 with scale absmax/6 ([B] 3.1; [A] "P4 main KV").
+ * gate      [D] fp32 gate vector g.
+ * idx_k_new [batch][n_new/2][idx_dim] int8 indexer keys of the new entries.
+ * Entries are written at positions n_entries[b] .. n_entries[b]+n_new/2-1 and
+ * n_entries[b] then advances by n_new/2.  If that would pass the capacity the
+ * sequence is left unchanged and KVC_DEV_CAPACITY is set.  NaN/Inf channels are
+ * coded 0, left out of the group maximum, and set KVC_DEV_NONFINITE.         */
+kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,
+                    const float* gate, const int8_t* idx_k_new,
+                    const kvc_cache* cache, uint32_t* dev_status, void* stream);
+
+/* Indexer scoring and exact top-K (A4-A5; [A] breakthrough 4 "用一个轻量索引器
+ * 给所有历史 token 打分，只挑分数最高的 512 个"; part 4 "CSA2").
+ * idx_q     [batch][idx_dim] int8 indexer queries.
+ * score_j = sum_d idx_q[d] * idx_k[j][d] in int32 over the visible entries.
+ * topk_idx  [batch][topk] int32 out: the topk highest scores, ties to the lower
+ *           index, written in ascending index order; -1 pads when fewer than
+ *           topk entries are visible.
+ * scores    [batch][capacity] int32 out, or NULL; when given it receives every
+ *           visible score (positions past n_entries are not written).
+ * ws        device workspace of at least kvc_workspace_bytes(cfg, batch,
+ *           capacity) bytes, 256-byte aligned; its contents need no
+ *           initialisation and are scratch after the call.               */
+kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
+                          const kvc_cache* cache, int32_t* topk_idx,
+                          int32_t* scores, void* ws, size_t ws_bytes,
+                          uint32_t* dev_status, void* stream);
+
+/* Sparse decode attention (A6-A10; [A] breakthrough 2 and 4, "P4 main KV").
+ * q         [batch][n_heads][D] act_dtype queries (already in latent space).
+ * topk_idx  [batch][topk] int32 selected entries; -1 entries are skipped, any
+ *           other index outside [0, n_entries[b]) is skipped and sets
+ *           KVC_DEV_BAD_INDEX.
+ * window    [batch][window][D] act_dtype raw keys of the sliding window; the
+ *           first window_len (0 <= window_len <= cfg->window) rows are used.
+ * One softmax runs jointly over the dequantised selected entries and the
+ * window keys; values are the first latent_dim channels of each key.
+ * out       [batch][n_heads][latent_dim] fp32; lse [batch][n_heads] fp32
+ *           natural-log sum of exp of the scaled logits, or NULL.  With no key
+ *           at all the output row is 0 and lse is -inf.                   */
+kvc_status kvc_sparse_decode_attn(const kvc_config* cfg, const void* q,
+                                  const kvc_cache* cache, const int32_t* topk_idx,
+                                  const void* window, int window_len, float* out,
+                                  float* lse, void* ws, size_t ws_bytes,
+                                  uint32_t* dev_status, void* stream);
+
+/* One decode step through a CSA2 layer group (A11; [A] part 4 "CSA2：三种模式，
+ * 40 层只存 4 份"): layers run in order on `stream`.
+ *  Full    -- indexer top-K with its own idx_q over `cache`, then attention;
+ *  Reindex -- same over the Full layer's stored cache and keys, own idx_q;
+ *  Reuse   -- attention with the top-K of the latest Full/Reindex layer.
+ * Every layer uses its own q and window.  modes is a HOST array of n_layers
+ * kvc_mode values; modes[0] must be Full or Reindex.  Device arrays are
+ * layer-major: q [L][batch][H][D], idx_q [L][batch][Di], windows
+ * [L][batch][W][D], out [L][batch][H][Dv], lse [L][batch][H] (or NULL),
+ * topk [L][batch][K] (receives every layer's indices; Reuse layers get a copy
+ * of their head's).                                                       */
+kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers,
+                                const int32_t* modes, const void* q,
+                                const int8_t* idx_q, const void* windows,
+                                int window_len, const kvc_cache* cache,
+                                float* out, float* lse, int32_t* topk, void* ws,
+                                size_t ws_bytes, uint32_t* dev_status,
+                                void* stream);
+
+/* E2M1 / E4M3 codecs as the pack kernel applies them (format utilities).
+ * kvc_e2m1_encode: x [n] fp32 -> codes [n] uint8 (0..15), round to nearest
+ * even on the grid {0, 0.5, 1, 1.5, 2, 3, 4, 6}, saturating, -0 stored as 0.
+ * kvc_e4m3_encode: x [n] fp32 >= 0 -> bytes [n], round to nearest even,
+ * saturating at 448.                                                       */
+kvc_status kvc_e2m1_encode(const float* x, int64_t n, uint8_t* codes, void* stream);
+kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stream);
+
+/* Tracing.  Between kvc_trace_begin and kvc_trace_end every kernel the
+ * library enqueues is bracketed by a pair of CUDA events (at most
+ * max_launches launches are recorded).  kvc_trace_kernel, called after the
+ * traced work has completed, returns the number of recorded launches of the
+ * kernel named `name` and their summed device time in milliseconds.  Names:
+ * "pack", "pack_commit", "index_scan", "topk_collect", "topk_finalize",
+ * "attn_mma", "attn_simt", "attn_merge", "fp4_codec".                      */
+kvc_status kvc_trace_begin(int max_launches);
+kvc_status kvc_trace_end(void);
+kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);
+
+/* Number of kernels the library has enqueued since it was loaded. */
+uint64_t kvc_launch_count(void);
+
+const char* kvc_status_string(kvc_status s);
+const char* kvc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVC_H */

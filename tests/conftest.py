@@ -18,3 +18,15 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def kvc():
+    """The C-ABI binding on a CUDA device; the library must exist (no fallback)."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from fp4_compressed_kv_b200 import build, kvc as binding
+    build.build()
+    binding.lib()
+    return binding

@@ -1,0 +1,97 @@
+"""CPU checks of the C ABI: libkvc.so builds, loads and exports every function
+include/kvc.h declares; host-side size arithmetic matches the oracle; host
+validation rejects bad arguments before any device work, and with no sm_100
+device current the calls fail loudly instead of falling back."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+from fp4_compressed_kv_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp4_compressed_kv_b200 import build, kvc
+    build.build()
+    return kvc
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvc.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvc_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 15
+    so = lib.lib()
+    for n in names:
+        assert hasattr(so, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r" T (kvc_\w+)", out))
+    assert set(names) <= exported
+    assert lib.version().startswith("kvc")
+
+
+def test_sizes_match_oracle(lib, orc):
+    for name, w in synth.WORKLOADS.items():
+        cfg = lib.config_for(w)
+        ocfg = orc.make_cfg(w.latent, w.rope, w.group, w.scale_fmt, w.idx_dim, w.topk, w.window,
+                            w.heads, w.sm_scale)
+        assert lib.record_bytes(cfg) == orc.record_bytes(ocfg, True), name
+        for padded in (False, True):
+            assert lib.bytes_resident(cfg, w.entries, w.layers, padded) == \
+                orc.bytes_resident(ocfg, w.entries, w.layers, 2 if w.act == "bf16" else 4, padded)
+        assert lib.workspace_bytes(cfg, w.batch, w.entries) > 0
+    w = synth.WORKLOADS["stack1m"]
+    assert lib.bytes_resident(lib.config_for(w), 500_000, 20, False) == 219_949_120
+
+
+def test_invalid_configs_rejected(lib):
+    base = synth.WORKLOADS["mla32k"]
+    for field, value in [("group", 48), ("group", 1024), ("latent_dim", 500), ("idx_dim", 100),
+                         ("topk", 0), ("topk", 5000), ("scale_fmt", 3), ("act_dtype", 7),
+                         ("sm_scale", 0.0), ("n_heads", 0)]:
+        cfg = lib.config_for(base)
+        setattr(cfg, field, value)
+        assert lib.record_bytes(cfg) == 0, field
+        assert lib.workspace_bytes(cfg, 1, 10) == 0, field
+
+
+def test_host_validation_before_device(lib):
+    so = lib.lib()
+    cfg = lib.config_for(synth.WORKLOADS["tiny"])
+    cache = lib.CacheStruct(16, 16, 16, 1, 8)  # fake aligned addresses: never dereferenced
+    # odd n_new is invalid whatever the device
+    assert so.kvc_pack(C.byref(cfg), C.c_void_p(16), 3, C.c_void_p(16), C.c_void_p(16),
+                       C.byref(cache), None, None) == 1
+    # misaligned tokens
+    assert so.kvc_pack(C.byref(cfg), C.c_void_p(17), 2, C.c_void_p(16), C.c_void_p(16),
+                       C.byref(cache), None, None) == 1
+    # too-small workspace
+    assert so.kvc_index_topk(C.byref(cfg), C.c_void_p(16), C.byref(cache), C.c_void_p(16), None,
+                             C.c_void_p(256), 16, None, None) == 7
+    # Reuse as the first layer
+    modes = (C.c_int32 * 2)(2, 0)
+    assert so.kvc_layer_group_step(C.byref(cfg), 2, modes, C.c_void_p(16), C.c_void_p(16),
+                                   C.c_void_p(16), 32, C.byref(cache), C.c_void_p(16), None,
+                                   C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 1
+
+
+def test_no_device_fails_loudly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    so = lib.lib()
+    cfg = lib.config_for(synth.WORKLOADS["tiny"])
+    cache = lib.CacheStruct(16, 16, 16, 1, 8)
+    rc = so.kvc_pack(C.byref(cfg), C.c_void_p(16), 2, C.c_void_p(16), C.c_void_p(16),
+                     C.byref(cache), None, None)
+    assert rc == 6  # KVC_ERR_DEVICE: nothing was enqueued

@@ -1,0 +1,107 @@
+"""GPU pack (2:1 compression + FP4 group quantisation + indexer append) vs the
+oracle: bit-exact records (codes, scales, zero padding) and indexer rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_compressed_kv_b200 import synth
+from helpers import f32, oracle_cfg, oracle_pack
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_pack(kvc, w, tokens, gate, idx_k, capacity=None, chunks=None):
+    cfg = kvc.config_for(w)
+    B, T = tokens.shape[:2]
+    cache = kvc.Cache(cfg, B, capacity or T // 2)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    step = chunks or T
+    for t0 in range(0, T, step):
+        kvc.pack(cfg, tokens[:, t0:t0 + step].contiguous(), gate,
+                 idx_k[:, t0 // 2:(t0 + step) // 2].contiguous(), cache, status=st)
+    torch.cuda.synchronize()
+    return cache, int(st.item())
+
+
+@pytest.mark.parametrize("name", ["tiny", "mla32k"])
+def test_pack_bit_exact_full(kvc, name):
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w)  # CPU generator
+    rec, ic, n, ost = oracle_pack(w, inp["tokens"], inp["gate"], inp["idx_k"])
+    cache, st = _gpu_pack(kvc, w, inp["tokens"].cuda(), inp["gate"].cuda(), inp["idx_k"].cuda())
+    assert st == ost == 0
+    assert cache.n_entries.cpu().tolist() == n.tolist()
+    g = cache.records.cpu().numpy()
+    diff = np.argwhere(g != rec)
+    assert diff.size == 0, f"{len(diff)} bytes differ, first {diff[:5].tolist()}"
+    assert np.array_equal(cache.idx_k.cpu().numpy(), ic)
+
+
+def test_pack_group64_batch_ragged_appends(kvc):
+    """Group 64 (the batched workload's format), 3 sequences, appends in odd-sized pieces."""
+    w = synth.WORKLOADS["batch32x128k"].scaled(batch=3, context=3000)
+    inp = synth.make_inputs(w)
+    rec, ic, n, _ = oracle_pack(w, inp["tokens"], inp["gate"], inp["idx_k"], capacity=1600)
+    cache, st = _gpu_pack(kvc, w, inp["tokens"].cuda(), inp["gate"].cuda(), inp["idx_k"].cuda(),
+                          capacity=1600, chunks=998)
+    assert st == 0
+    assert cache.n_entries.cpu().tolist() == [1500] * 3
+    assert np.array_equal(cache.records.cpu().numpy(), rec)
+    assert np.array_equal(cache.idx_k.cpu().numpy(), ic)
+
+
+def test_pack_capacity_and_nonfinite_flags(kvc):
+    w = synth.WORKLOADS["mla32k"].scaled(context=64)
+    inp = synth.make_inputs(w)
+    tok = inp["tokens"].clone()
+    tok[0, 5, 17] = float("nan")
+    tok[0, 9, 600 - 64] = float("inf")
+    rec, ic, n, ost = oracle_pack(w, tok, inp["gate"], inp["idx_k"])
+    cache, st = _gpu_pack(kvc, w, tok.cuda(), inp["gate"].cuda(), inp["idx_k"].cuda())
+    assert ost == oracle.ST_NONFINITE and st == kvc.DEV_NONFINITE
+    assert np.array_equal(cache.records.cpu().numpy(), rec)
+    # one more pair does not fit: sequence unchanged, capacity bit set
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    before = cache.records.clone()
+    kvc.pack(kvc.config_for(w), tok[:, :2].cuda().contiguous(), inp["gate"].cuda(),
+             inp["idx_k"][:, :1].cuda().contiguous(), cache, status=st2)
+    torch.cuda.synchronize()
+    assert st2.item() == kvc.DEV_CAPACITY
+    assert cache.n_entries.item() == 32 and torch.equal(cache.records, before)
+
+
+def test_pack_host_validation(kvc):
+    w = synth.WORKLOADS["tiny"]
+    cfg = kvc.config_for(w)
+    cache = kvc.Cache(cfg, 1, 16)
+    tok = torch.zeros(1, 3, 80, device="cuda")
+    with pytest.raises(kvc.KvcError):
+        kvc.pack(cfg, tok, torch.zeros(80, device="cuda"), torch.zeros(1, 1, 32, dtype=torch.int8,
+                                                                        device="cuda"), cache)
+    bad = kvc.config_for(w)
+    bad.group = 48
+    with pytest.raises(kvc.KvcError):
+        kvc.pack(bad, tok[:, :2].contiguous(), torch.zeros(80, device="cuda"),
+                 torch.zeros(1, 1, 32, dtype=torch.int8, device="cuda"), cache)
+
+
+def test_codecs_match_oracle(kvc):
+    """Hardware E2M1 / E4M3 conversions against the oracle's nearest-even search."""
+    rng = np.random.default_rng(0)
+    grid = np.array([oracle.e2m1_value(c) for c in range(8)])
+    mids = (grid[1:] + grid[:-1]) / 2
+    xs = np.concatenate([grid, -grid, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, 9),
+                         rng.uniform(-7, 7, 20000), [7.0, -100.0, 1e30, -0.0]]).astype(np.float32)
+    codes = torch.empty(xs.size, dtype=torch.uint8, device="cuda")
+    kvc.e2m1_encode(torch.from_numpy(xs).cuda(), codes)
+    want = np.array([oracle.e2m1_encode(float(x)) for x in xs])
+    got = codes.cpu().numpy()
+    assert np.array_equal(got, want), xs[got != want][:10]
+    vals = np.array([oracle.e4m3_value(b) for b in range(0x7F)])
+    ys = np.concatenate([vals, (vals[1:] + vals[:-1]) / 2, np.exp(rng.uniform(-14, 6.2, 20000)),
+                         [500.0, 1e9, 0.0]]).astype(np.float32)
+    out = torch.empty(ys.size, dtype=torch.uint8, device="cuda")
+    kvc.e4m3_encode(torch.from_numpy(ys).cuda(), out)
+    want = np.array([oracle.e4m3_encode(float(y)) for y in ys])
+    assert np.array_equal(out.cpu().numpy(), want)

@@ -1,0 +1,110 @@
+"""GPU indexer scores and top-K vs the oracle: bit-exact int32 scores and
+index sets (ties to the lower index), ragged lengths, K >= N, forced ties
+(including the heavy-tie path that overflows the candidate list)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_compressed_kv_b200 import synth
+from helpers import oracle_cfg, topk_set_equal
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(kvc, w, idx_k, idx_q, n_entries, capacity):
+    cfg = kvc.config_for(w)
+    B = idx_k.shape[0]
+    cache = kvc.Cache(cfg, B, capacity)
+    cache.idx_k[:, : idx_k.shape[1]] = idx_k.cuda()
+    cache.n_entries.copy_(torch.as_tensor(n_entries, dtype=torch.int32))
+    tk = torch.empty(B, w.topk, dtype=torch.int32, device="cuda")
+    sc = torch.zeros(B, capacity, dtype=torch.int32, device="cuda")
+    ws = kvc.workspace(cfg, B, capacity)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvc.index_topk(cfg, idx_q.cuda().contiguous(), cache, tk, ws, scores=sc, status=st)
+    torch.cuda.synchronize()
+    return tk.cpu().numpy(), sc.cpu().numpy(), int(st.item())
+
+
+def _oracle(w, idx_k, idx_q, n_entries, capacity):
+    cfg = oracle_cfg(w)
+    ic = np.zeros((idx_k.shape[0], capacity, w.idx_dim), np.int8)
+    ic[:, : idx_k.shape[1]] = idx_k.numpy()
+    return oracle.index_topk(cfg, idx_q.numpy(), ic, np.asarray(n_entries, np.int32),
+                             want_scores=True)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mla32k"])
+def test_topk_bit_exact(kvc, name):
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w, with_tokens=False)
+    n = [w.entries] * w.batch
+    tk, sc, st = _run(kvc, w, inp["idx_k"], inp["idx_q"][0], n, w.entries)
+    otk, osc = _oracle(w, inp["idx_k"], inp["idx_q"][0], n, w.entries)
+    assert st == 0
+    assert np.array_equal(sc, osc)
+    topk_set_equal(tk, otk)
+
+
+def test_topk_ragged_batch(kvc):
+    w = synth.WORKLOADS["csa2group"].scaled(batch=6, context=2 * 9000)
+    inp = synth.make_inputs(w, with_tokens=False)
+    n = [9000, 5000, 513, 512, 100, 0]
+    cap = 9008
+    tk, sc, st = _run(kvc, w, inp["idx_k"], inp["idx_q"][0], n, cap)
+    otk, osc = _oracle(w, inp["idx_k"], inp["idx_q"][0], n, cap)
+    assert st == 0
+    for b in range(6):
+        assert np.array_equal(sc[b, : n[b]], osc[b, : n[b]])
+    topk_set_equal(tk, otk)
+    assert np.all(tk[4, 100:] == -1) and np.all(tk[5] == -1)
+
+
+@pytest.mark.parametrize("pattern", ["constant", "few_values", "duplicated_rows", "top_tie"])
+def test_topk_forced_ties(kvc, pattern):
+    w = synth.WORKLOADS["mla32k"].scaled(context=2 * 20000)
+    g = torch.Generator().manual_seed(11)
+    N = w.entries
+    idx_q = torch.randint(-127, 128, (1, 128), generator=g, dtype=torch.int8)
+    if pattern == "constant":        # every score equal: heavy-tie path
+        idx_k = torch.full((1, N, 128), 3, dtype=torch.int8)
+    elif pattern == "few_values":    # 4 distinct rows, thousands of ties each
+        rows = torch.randint(-127, 128, (4, 128), generator=g, dtype=torch.int8)
+        idx_k = rows[torch.randint(0, 4, (N,), generator=g)].unsqueeze(0)
+    elif pattern == "duplicated_rows":
+        rows = torch.randint(-127, 128, (N // 8, 128), generator=g, dtype=torch.int8)
+        idx_k = rows.repeat_interleave(8, 0).unsqueeze(0)
+    else:                            # the threshold falls inside a block of equal scores
+        idx_k = torch.randint(-20, 21, (1, N, 128), generator=g, dtype=torch.int8)
+        idx_k[0, 1000:1800] = idx_k[0, 7]
+    tk, sc, st = _run(kvc, w, idx_k, idx_q, [N], N)
+    otk, osc = _oracle(w, idx_k, idx_q, [N], N)
+    assert st == 0 and np.array_equal(sc, osc)
+    topk_set_equal(tk, otk)
+
+
+def test_topk_extreme_scores(kvc):
+    """Rows at the ends of the int8 x int8 range land in the first and last bins."""
+    w = synth.WORKLOADS["tiny"].scaled(context=2 * 300)
+    N = w.entries
+    idx_q = torch.full((1, 32), -128, dtype=torch.int8)
+    idx_k = torch.randint(-127, 128, (1, N, 32), generator=torch.Generator().manual_seed(3),
+                          dtype=torch.int8)
+    idx_k[0, 10] = -128   # max score 32*16384
+    idx_k[0, 20] = 127    # min score
+    tk, sc, st = _run(kvc, w, idx_k, idx_q, [N], N)
+    otk, osc = _oracle(w, idx_k, idx_q, [N], N)
+    assert sc[0, 10] == 32 * 128 * 128 and np.array_equal(sc, osc)
+    topk_set_equal(tk, otk)
+
+
+def test_topk_workspace_validation(kvc):
+    w = synth.WORKLOADS["tiny"]
+    cfg = kvc.config_for(w)
+    cache = kvc.Cache(cfg, 1, 64)
+    tk = torch.empty(1, w.topk, dtype=torch.int32, device="cuda")
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.index_topk(cfg, torch.zeros(1, 32, dtype=torch.int8, device="cuda"), cache, tk, small)
+    assert e.value.status == 7
