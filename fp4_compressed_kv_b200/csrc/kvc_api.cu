@@ -58,6 +58,16 @@ TraceState& trace() {
 std::atomic<uint64_t> g_launches{0};
 }  // namespace
 
+// Inside stream capture a plain event record only marks a dependency; an
+// external record becomes a graph node that records the event on replay.
+static void record(cudaEvent_t e, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(e, s);
+}
+
 void trace_before(const char* name, cudaStream_t s) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     TraceState& t = trace();
@@ -66,13 +76,13 @@ void trace_before(const char* name, cudaStream_t s) {
     if (!t.on || t.used >= t.max) return;
     t.open = t.used++;
     t.name[t.open] = name;
-    cudaEventRecord(t.ev[2 * t.open], s);
+    record(t.ev[2 * t.open], s);
 }
 
 void trace_after(cudaStream_t s) {
     TraceState& t = trace();
     std::lock_guard<std::mutex> lk(t.mu);
-    if (t.open >= 0) cudaEventRecord(t.ev[2 * t.open + 1], s);
+    if (t.open >= 0) record(t.ev[2 * t.open + 1], s);
     t.open = -1;
 }
 

@@ -1,0 +1,96 @@
+"""Run one hot-path call a few times on synthetic inputs, for profilers.
+
+    python -m fp4_compressed_kv_b200.profile_case --kernel scan|attn|pack|step \
+        [--config NAME] [--batch B] [--entries N] [--iters 3]
+
+scan  kvc_index_topk over B sequences of N int8 indexer rows (the indexer
+      scan, collect and finalize kernels), inputs from the workload's shapes.
+attn  kvc_sparse_decode_attn: B sequences, each with a cache of N packed
+      entries, a top-K drawn uniformly from them and a full window.
+pack  kvc_pack of the workload's pack case (pack_new raw tokens per sequence,
+      or 4096 when the workload has none).
+step  one decode step of the workload (pack of one pair + layer group).
+Sizes default to the workload's; pass --batch/--entries to shrink a case so a
+profiler capture stays small (keep the streamed bytes above the 126 MB L2).
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from fp4_compressed_kv_b200 import build, kvc, synth
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("--kernel", required=True, choices=["scan", "attn", "pack", "step"])
+    p.add_argument("--config", default="batch32x128k")
+    p.add_argument("--batch", type=int, default=0)
+    p.add_argument("--entries", type=int, default=0)
+    p.add_argument("--iters", type=int, default=3)
+    a = p.parse_args()
+    build.build()
+    w = synth.WORKLOADS[a.config]
+    if a.batch:
+        w = w.scaled(batch=a.batch)
+    if a.entries:
+        w = w.scaled(context=2 * a.entries)
+    cfg = kvc.config_for(w)
+    dev = torch.device("cuda")
+    g = synth.generator(dev, w.seed)
+    B, N = w.batch, w.entries
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    if a.kernel in ("scan", "step", "attn"):
+        cache = kvc.Cache(cfg, B, N + a.iters + 8, device=dev)
+        ws = kvc.workspace(cfg, B, cache.capacity, device=dev)
+    if a.kernel in ("scan", "step"):
+        cache.idx_k[:, :N] = torch.randint(-127, 128, (B, N, w.idx_dim), generator=g, device=dev,
+                                           dtype=torch.int8)
+        cache.n_entries.fill_(N)
+    if a.kernel == "scan":
+        q = torch.randint(-127, 128, (B, w.idx_dim), generator=g, device=dev, dtype=torch.int8)
+        tk = torch.empty(B, w.topk, dtype=torch.int32, device=dev)
+        for _ in range(a.iters):
+            kvc.index_topk(cfg, q, cache, tk, ws, status=st)
+    elif a.kernel == "attn":
+        # pack N entries per sequence from fresh raw tokens, in slices
+        gate = (torch.randn(w.dim, generator=g, device=dev) / w.dim ** 0.5).float()
+        step_tok = 8192
+        for t0 in range(0, 2 * N, step_tok):
+            n = min(step_tok, 2 * N - t0)
+            nt = synth.make_new_tokens(w, n, dev, seed_offset=t0)
+            kvc.pack(cfg, nt["tokens"], gate, nt["idx_k"], cache, status=st)
+        tk = torch.sort(torch.stack([torch.randperm(N, generator=g, device=dev)[: w.topk]
+                                     for _ in range(B)]), dim=1).values.int().contiguous()
+        q = torch.randn(B, w.heads, w.dim, generator=g, device=dev).to(w.torch_dtype)
+        win = torch.randn(B, w.window, w.dim, generator=g, device=dev).to(w.torch_dtype)
+        out = torch.empty(B, w.heads, w.latent, device=dev)
+        for _ in range(a.iters):
+            kvc.sparse_decode_attn(cfg, q, cache, tk, win, w.window, out, ws, status=st)
+    elif a.kernel == "pack":
+        n_new = w.pack_new or 4096
+        nt = synth.make_new_tokens(w, n_new, dev)
+        gate = (torch.randn(w.dim, generator=g, device=dev) / w.dim ** 0.5).float()
+        pc = kvc.Cache(cfg, B, n_new // 2, device=dev)
+        for _ in range(a.iters):
+            pc.n_entries.zero_()
+            kvc.pack(cfg, nt["tokens"], gate, nt["idx_k"], pc, status=st)
+    else:  # step
+        inp = synth.make_inputs(w, dev, with_tokens=False)
+        L = w.layers
+        nt = synth.make_new_tokens(w, 2, dev)
+        out = torch.empty(L, B, w.heads, w.latent, device=dev)
+        tk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
+        cache.records.random_(0, 120, generator=g)  # arbitrary codes, scale bytes below NaN
+        for _ in range(a.iters):
+            kvc.pack(cfg, nt["tokens"], inp["gate"], nt["idx_k"], cache, status=st)
+            kvc.layer_group_step(cfg, list(w.modes), inp["q"], inp["idx_q"], inp["windows"],
+                                 w.window, cache, out, tk, ws, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, st.item()
+    print(f"profile_case {a.kernel} {w.name} B={B} N={N} iters={a.iters} ok")
+
+
+if __name__ == "__main__":
+    main()
