@@ -60,6 +60,7 @@ def _lib():
             "kvc_workspace_bytes": (Z, [P, I, I]),
             "kvc_pack": (S, [P, P, I, P, P, P, P, P]),
             "kvc_index_topk": (S, [P, P, P, P, P, P, Z, P, P]),
+            "kvc_index_topk_noalloc": (S, [P, P, P, P, P, P, P]),
             "kvc_sparse_decode_attn": (S, [P, P, P, P, P, I, P, P, P, Z, P, P]),
             "kvc_layer_group_step": (S, [P, I, P, P, P, P, I, P, P, P, P, P, Z, P, P]),
             "kvc_e2m1_encode": (S, [P, C.c_int64, P, P]),
@@ -170,6 +171,15 @@ def index_topk(cfg, idx_q, cache: Cache, topk_out, ws, scores=None, status=None,
     _check("kvc_index_topk", _lib().kvc_index_topk(C.byref(cfg), _ptr(idx_q), C.byref(cs),
                                                    _ptr(topk_out), _ptr(scores), p, n,
                                                    _ptr(status), _stream(stream)))
+
+
+def index_topk_noalloc(cfg, idx_q, cache: Cache, topk_out, scores=None, status=None,
+                       stream=None):
+    """kvc_index_topk with the library's fixed scratch (no workspace argument)."""
+    cs = cache.struct()
+    _check("kvc_index_topk_noalloc", _lib().kvc_index_topk_noalloc(
+        C.byref(cfg), _ptr(idx_q), C.byref(cs), _ptr(topk_out), _ptr(scores), _ptr(status),
+        _stream(stream)))
 
 
 def sparse_decode_attn(cfg, q, cache: Cache, topk, window, window_len, out, ws, lse=None,

@@ -144,6 +144,28 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
                           int32_t* scores, void* ws, size_t ws_bytes,
                           uint32_t* dev_status, void* stream);
 
+/* kvc_index_topk without a workspace argument, for callers that cannot
+ * allocate device memory: a plugin whose host framework owns every device
+ * allocation and passes it only its inputs and outputs, or a latency-critical
+ * path where cudaMalloc's implicit device synchronisation is not allowed.  The
+ * pages have no counterpart of this call; it computes exactly what
+ * kvc_index_topk computes (same kernels, same results).
+ * Its scratch (scores, histograms, counters, candidate lists) is a fixed
+ * array inside the library, about 6.5 MiB, held on every GPU that loads the
+ * library until the process exits.  Limits: batch <= 64 and
+ * batch * capacity <= 1,048,576 entries; larger problems return
+ * KVC_ERR_CAPACITY before anything is enqueued.  The call allocates nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the one array and it keeps the last call's
+ * contents: the parts that must start at zero are cleared on `stream` by each
+ * call, but calls whose work overlaps on the GPU (different streams, or
+ * different host threads on one device) race on it.                      */
+kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t* idx_q,
+                                  const kvc_cache* cache, int32_t* topk_idx,
+                                  int32_t* scores, uint32_t* dev_status,
+                                  void* stream);
+
 /* Sparse decode attention (A6-A10; [A] breakthrough 2 and 4, "P4 main KV").
  * q         [batch][n_heads][D] act_dtype queries (already in latent space).
  * topk_idx  [batch][topk] int32 selected entries; -1 entries are skipped, any
