@@ -1,7 +1,9 @@
 """CPU oracle for compressed-KV sparse decode (test infrastructure only).
 
-The arithmetic lives in ``oracle.c`` (plain C, fp64 where the pages fix no
-precision, compiled with ``-ffp-contract=off``).  This module compiles it
+The arithmetic lives in ``oracle.c`` (plain C, compiled with
+``-ffp-contract=off``): fp64 where the pages fix no precision and no quantised
+value depends on it (attention), fp32 for the compression gate whose result
+decides the FP4 codes (the kernel's precision).  This module compiles it
 into ``liboracle.so`` next to the source and wraps every entry point for
 numpy arrays.  Only the tests, the smoke check and the benchmark's CPU
 baseline leg may import it; the product library never does.
@@ -63,14 +65,14 @@ def lib():
         P = C.c_void_p
         sig = {
             "orc_kv_bytes_per_token": (C.c_uint64, [C.c_int64] * 4),
-            "orc_exp": (C.c_double, [C.c_double]),
+            "orc_expf": (C.c_float, [C.c_float]),
             "orc_e2m1_value": (C.c_float, [C.c_int]),
             "orc_e2m1_encode": (C.c_int, [C.c_float]),
             "orc_e4m3_value": (C.c_float, [C.c_int]),
             "orc_e4m3_encode": (C.c_int, [C.c_float]),
             "orc_n_groups": (C.c_int, [C.c_int] * 3),
             "orc_record_bytes": (C.c_int, [P, C.c_int]),
-            "orc_gate_delta": (C.c_double, [P, P, P, C.c_int]),
+            "orc_gate_delta": (C.c_float, [P, P, P, C.c_int]),
             "orc_compress_pair": (None, [P, P, P, C.c_int, P]),
             "orc_quantize_entry": (C.c_int, [P, P, P]),
             "orc_dequantize_entry": (None, [P, P, P]),
@@ -106,8 +108,9 @@ def kv_bytes_per_token(layers, heads, dim, bytes_per_elem) -> int:
     return int(lib().orc_kv_bytes_per_token(layers, heads, dim, bytes_per_elem))
 
 
-def exp(x: float) -> float:
-    return lib().orc_exp(float(x))
+def expf(x: float) -> float:
+    """The fp32 exp of the gate (its result as a Python float)."""
+    return lib().orc_expf(float(x))
 
 
 def e2m1_value(code: int) -> float:

@@ -20,13 +20,13 @@
  * Readings where the pages leave a step open (each is documented with the
  * function that takes it):
  *  R1 gate: one D-vector g gives one logit per token; the pair's weights are
- *     the softmax of the two logits.  The logit difference is accumulated in
- *     a fixed order (lane-of-32 partial sums over 8-channel chunks, then a
- *     xor tree), because the quantised codes downstream depend on the exact
- *     fp32 entry.
- *  R2 exp: written here from the Cody-Waite argument reduction and a
- *     degree-13 Taylor polynomial (Horner form), so that the gate weight is
- *     the same bits on every implementation of this specification.
+ *     the softmax of the two logits.  The pages fix no precision for this
+ *     step; the quantised codes downstream depend on the exact fp32 entry, so
+ *     it is evaluated in fp32 in a fixed order (8 partial sums over 8-channel
+ *     chunks, then a xor tree), the precision and order the GPU kernel uses.
+ *  R2 exp: written here in fp32 from the Cody-Waite argument reduction and a
+ *     degree-7 Taylor polynomial (Horner form), so that the gate weight is the
+ *     same bits on every implementation of this specification.
  *  R3 grouping: latent and RoPE segments are grouped separately; a segment's
  *     last group may be short.
  *  R4 scale: s = absmax / 6 in fp32, stored as fp32 or rounded (RNE,
@@ -79,33 +79,31 @@ uint64_t orc_kv_bytes_per_token(int64_t layers, int64_t heads, int64_t dim,
 }
 
 /* ------------------------------------------------------------------ */
-/* R2: exp(x) in fp64.  Cody-Waite: x = n*ln2 + r with ln2 split into a
- * 32-significant-bit head (so n*LN2_HI is exact for |n| < 2^11) and the
- * rounded remainder; e^r from the Taylor series to degree 13 (truncation
- * below 4e-18 for |r| <= ln2/2); the result is scaled by an exactly built
- * power of two.  Inputs above 709 give +inf; inputs below -708 give 0 (a
- * subnormal exp never changes 1 + exp in the gate).                      */
-static const double ORC_LN2_HI = 0x1.62e42feep-1;
-static const double ORC_LN2_LO = 0x1.a39ef35793c76p-33;
-static const double ORC_INV_LN2 = 0x1.71547652b82fep+0;
-static const double ORC_INV_FACT[14] = {
-    0x1.0p+0,              0x1.0p+0,              0x1.0p-1,
-    0x1.5555555555555p-3,  0x1.5555555555555p-5,  0x1.1111111111111p-7,
-    0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
-    0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
-    0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+/* R2: exp(x) in fp32.  Cody-Waite: x = n*ln2 + r with ln2 split into a
+ * 16-significant-bit head (so n*LN2_HI is exact for |n| < 2^8) and the
+ * rounded remainder; e^r from the Taylor series to degree 7 (truncation
+ * below 6e-9 for |r| <= ln2/2, under half an fp32 ulp of e^r); the result is
+ * scaled by an exactly built power of two.  Inputs above 88 give +inf;
+ * inputs below -87 give 0 (there exp(x) < 2^-125 and 1 + exp(x) == 1 in the
+ * gate).                                                                */
+static const float ORC_LN2_HI_F = 0x1.62e4p-1f;
+static const float ORC_LN2_LO_F = 0x1.7f7d1cp-20f;
+static const float ORC_INV_LN2_F = 0x1.715476p+0f;
+static const float ORC_INV_FACT_F[8] = {
+    0x1.0p+0f, 0x1.0p+0f, 0x1.0p-1f, 0x1.555556p-3f,
+    0x1.555556p-5f, 0x1.111112p-7f, 0x1.6c16c2p-10f, 0x1.a01a02p-13f};
 
-double orc_exp(double x) {
+float orc_expf(float x) {
     if (x != x) return x;
-    if (x > 709.0) return INFINITY;
-    if (x < -708.0) return 0.0;
-    double n = nearbyint(x * ORC_INV_LN2); /* round-half-even, default mode */
-    double r = fma(-n, ORC_LN2_HI, x);
-    r = fma(-n, ORC_LN2_LO, r);
-    double p = ORC_INV_FACT[13];
-    for (int k = 12; k >= 0; --k) p = fma(p, r, ORC_INV_FACT[k]);
-    int64_t bits = ((int64_t)n + 1023) << 52;
-    double two_n;
+    if (x > 88.0f) return INFINITY;
+    if (x < -87.0f) return 0.0f;
+    float n = nearbyintf(x * ORC_INV_LN2_F); /* round-half-even, default mode */
+    float r = fmaf(-n, ORC_LN2_HI_F, x);
+    r = fmaf(-n, ORC_LN2_LO_F, r);
+    float p = ORC_INV_FACT_F[7];
+    for (int k = 6; k >= 0; --k) p = fmaf(p, r, ORC_INV_FACT_F[k]);
+    int32_t bits = ((int32_t)n + 127) << 23;
+    float two_n;
     memcpy(&two_n, &bits, sizeof two_n);
     return p * two_n;
 }
@@ -205,26 +203,27 @@ static int orc_groups(const orc_cfg* c, int* start, int* len) {
 /* R1: the 2:1 compression of a token pair ([P2] breakthrough 4 "CSA 把每 2
  * 个 token 的 KV 压成 1 条"; [P1] 3.2 "main key compressor").
  * logit_t = g . k_t; (w0, w1) = softmax(logit_0, logit_1);
- * entry = w0 k_0 + w1 k_1.
+ * entry = w0 k_0 + w1 k_1, everything in fp32.
  * Fixed evaluation order: delta = logit_0 - logit_1 = sum_d g_d (k0_d - k1_d)
- * accumulated by 32 partial sums; channel chunk c = [8c, 8c+8) goes to
- * partial c mod 32, chunks in increasing order and channels in increasing
- * order inside a chunk, each term added with one fma.  The partials are
- * then combined by a xor tree over offsets 16, 8, 4, 2, 1.              */
-double orc_gate_delta(const float* k0, const float* k1, const float* g, int D) {
-    double acc[32];
-    for (int l = 0; l < 32; ++l) acc[l] = 0.0;
+ * accumulated by 8 partial sums; channel chunk c = [8c, 8c+8) goes to
+ * partial c mod 8, chunks in increasing order and channels in increasing
+ * order inside a chunk, each term added with one fmaf after an fp32
+ * subtraction.  The partials are combined by a xor tree over offsets 4, 2, 1.
+ * w0 = 1 / (1 + exp(-delta)), w1 = 1 - w0, entry_d = fmaf(w0, k0_d, w1 * k1_d). */
+float orc_gate_delta(const float* k0, const float* k1, const float* g, int D) {
+    float acc[8];
+    for (int l = 0; l < 8; ++l) acc[l] = 0.0f;
     for (int c = 0; c * 8 < D; ++c) {
-        int l = c % 32;
+        int l = c % 8;
         for (int t = 0; t < 8 && 8 * c + t < D; ++t) {
             int d = 8 * c + t;
-            double diff = (double)k0[d] - (double)k1[d];
-            acc[l] = fma((double)g[d], diff, acc[l]);
+            float diff = k0[d] - k1[d];
+            acc[l] = fmaf(g[d], diff, acc[l]);
         }
     }
-    for (int off = 16; off >= 1; off >>= 1) {
-        double nxt[32];
-        for (int l = 0; l < 32; ++l) nxt[l] = acc[l] + acc[l ^ off];
+    for (int off = 4; off >= 1; off >>= 1) {
+        float nxt[8];
+        for (int l = 0; l < 8; ++l) nxt[l] = acc[l] + acc[l ^ off];
         memcpy(acc, nxt, sizeof acc);
     }
     return acc[0];
@@ -232,11 +231,10 @@ double orc_gate_delta(const float* k0, const float* k1, const float* g, int D) {
 
 void orc_compress_pair(const float* k0, const float* k1, const float* g, int D,
                        float* e) {
-    double delta = orc_gate_delta(k0, k1, g, D);
-    double w0 = 1.0 / (1.0 + orc_exp(-delta));
-    double w1 = 1.0 - w0;
-    for (int d = 0; d < D; ++d)
-        e[d] = (float)fma(w0, (double)k0[d], w1 * (double)k1[d]);
+    float delta = orc_gate_delta(k0, k1, g, D);
+    float w0 = 1.0f / (1.0f + orc_expf(-delta));
+    float w1 = 1.0f - w0;
+    for (int d = 0; d < D; ++d) e[d] = fmaf(w0, k0[d], w1 * k1[d]);
 }
 
 /* ------------------------------------------------------------------ */

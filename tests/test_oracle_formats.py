@@ -5,7 +5,7 @@
 - E2M1: the grid derived from the bit layout the pages state, the printed
   magnitude list, the tie table, saturation, and a brute-force sweep.
 - E4M3 scales: decode of all 256 bytes and RNE encode vs torch's float8_e4m3fn.
-- exp: against the C library's exp within 2 ulp.
+- exp (fp32, gate only): against the C library's exp within 3 fp32 ulp.
 """
 import math
 import os
@@ -149,12 +149,18 @@ def test_e4m3_encode_matches_torch_rne(orc):
 
 
 # ------------------------------------------------------------------ exp
-def test_exp_within_two_ulp(orc):
+def _f32_ulp(x):
+    x = np.float32(abs(x))
+    return float(np.spacing(x))
+
+
+def test_expf_within_three_ulp(orc):
     rnd = random.Random(7)
-    xs = [rnd.uniform(-708, 709) for _ in range(20000)] + [rnd.uniform(-2, 2) for _ in range(20000)]
-    xs += [0.0, 1.0, -1.0, 0.5 * math.log(2), -0.5 * math.log(2), 708.9, -707.9]
+    xs = [rnd.uniform(-87, 88) for _ in range(20000)] + [rnd.uniform(-2, 2) for _ in range(20000)]
+    xs += [0.0, 1.0, -1.0, 0.5 * math.log(2), -0.5 * math.log(2), 87.9, -86.9]
     for x in xs:
-        got, want = orc.exp(x), math.exp(x)
-        assert abs(got - want) <= 2 * math.ulp(want), x
-    assert orc.exp(0.0) == 1.0
-    assert orc.exp(710.0) == math.inf and orc.exp(-709.0) == 0.0
+        x = float(np.float32(x))
+        got, want = orc.expf(x), math.exp(x)
+        assert abs(got - want) <= 3 * _f32_ulp(want), x
+    assert orc.expf(0.0) == 1.0
+    assert orc.expf(89.0) == math.inf and orc.expf(-88.0) == 0.0
