@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse FP4-KV decode query-tokens/s; achieved HBM GB/s vs 8 TB/s"
 UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNELS = ("pack", "pack_commit", "index_scan", "topk_collect", "topk_finalize", "attn_mma",
+KERNELS = ("pack", "pack_commit", "index_scan", "topk_select", "attn_tc05", "attn_mma",
            "attn_simt", "attn_merge")
 
 
@@ -348,6 +348,7 @@ def run_ours(args):
     heads_layers = sum(1 for m in modes if m != 2)
     per_launch = {
         "index_scan": B * scan_bytes(w, n_mean),
+        "attn_tc05": B * attn_bytes(w),
         "attn_mma": B * attn_bytes(w),
         "attn_simt": B * attn_bytes(w),
         "pack": B * pack_bytes(w, 1),

@@ -166,28 +166,52 @@ attn_simt_kernel(AttnArgs a, Shape sh, int H, int K, float scale_log2, int chunk
 }
 
 // ----------------------------------------------------------------------------
-// merge of split partials: grid (H, B), 128 threads
+// merge of split partials: grid (H, B), 128 threads; all split loads of a
+// thread are issued together
 __global__ void __launch_bounds__(128)
 attn_merge_kernel(AttnArgs a, int H, int Dv, int nsplit) {
-    const int h = blockIdx.x, b = blockIdx.y;
+    __shared__ float s_w[kMaxSplit];
+    __shared__ float s_inv, s_lse;
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const size_t row0 = ((size_t)b * H + h) * kMaxSplit;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, a.part_ml[(row0 + s) * 2]);
-    float wts[kMaxSplit];
-    float L = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-        const float ms = a.part_ml[(row0 + s) * 2];
-        wts[s] = (M == -INFINITY) ? 0.f : exp2f(ms - M);
-        L += wts[s] * a.part_ml[(row0 + s) * 2 + 1];
+    if (tid < 32) {
+        const float m = tid < nsplit ? __ldcg(a.part_ml + (row0 + tid) * 2) : -INFINITY;
+        const float l = tid < nsplit ? __ldcg(a.part_ml + (row0 + tid) * 2 + 1) : 0.f;
+        float M = m;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = (M == -INFINITY || tid >= nsplit) ? 0.f : exp2f(m - M);
+        float L = w * l;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (tid < kMaxSplit) s_w[tid] = w;
+        if (tid == 0) {
+            s_inv = L > 0.f ? 1.f / L : 0.f;
+            s_lse = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+        }
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int d = threadIdx.x; d < Dv; d += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < nsplit; ++s) acc = fmaf(wts[s], a.part_o[(row0 + s) * Dv + d], acc);
-        a.out[((size_t)b * H + h) * Dv + d] = acc * inv;
+    __syncthreads();
+    const float inv = s_inv;
+    for (int d = tid * 4; d < Dv; d += 128 * 4) {
+        float4 v[kMaxSplit];
+#pragma unroll
+        for (int s = 0; s < kMaxSplit; ++s)
+            if (s < nsplit)
+                v[s] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (row0 + s) * Dv + d));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int s = 0; s < kMaxSplit; ++s)
+            if (s < nsplit) {
+                const float w = s_w[s];
+                acc.x = fmaf(w, v[s].x, acc.x);
+                acc.y = fmaf(w, v[s].y, acc.y);
+                acc.z = fmaf(w, v[s].z, acc.z);
+                acc.w = fmaf(w, v[s].w, acc.w);
+            }
+        *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h) * Dv + d) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
-    if (threadIdx.x == 0 && a.lse)
-        a.lse[(size_t)b * H + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    if (tid == 0 && a.lse) a.lse[(size_t)b * H + h] = s_lse;
 }
 
 // ----------------------------------------------------------------------------
@@ -474,6 +498,9 @@ bool tc_supported(const kvc_config& c, const Shape& sh) {
 
 }  // namespace
 
+bool tc05_supported(const kvc_config& c, const Shape& sh);
+int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& a, cudaStream_t s);
+
 cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                              cudaStream_t s) {
     if (a.batch == 0) return cudaSuccess;
@@ -487,7 +514,10 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaError_t err;
     int nsplit;
-    if (tc_supported(c, sh)) {
+    if (tc05_supported(c, sh)) {
+        nsplit = launch_attention_tc05(c, sh, a, s);
+        if (nsplit < 0) return cudaErrorLaunchFailure;
+    } else if (tc_supported(c, sh)) {
         const int nchunks = (total + tc::CK - 1) / tc::CK;
         int want = sms / a.batch;
         if (want < 1) want = 1;

@@ -1,0 +1,434 @@
+// attn_tc05.cu -- sparse decode attention on the 5th-generation tensor cores
+// (tcgen05 MMA, accumulators in tensor memory) for the MLA shape: 64 query
+// heads sharing 576-channel entries (512 latent + 64 RoPE), values = latent.
+//
+// Method: "DeepSeek V1 到 V4.1-Flash，单 token 的 global KV 如何从 389,000 B
+// 压缩到 890 B的？" (acejoy.com) part 3 breakthrough 2 (heads share one latent
+// entry, absorbed up-projections), breakthrough 4 (top-512 entries + 128-token
+// window), part 4 "P4 main KV" (FP4 is dequantised before attention).  One
+// softmax runs jointly over the selected entries and the window keys.
+//
+// One CTA (256 threads) owns one chunk of 96 keys of one sequence:
+//  1. cp.async gathers the 96 selected records (16-byte rows) and window rows;
+//     Q (64 x 576 bf16) lands in a 128B-swizzled K-major tile.
+//  2. Records are dequantised in registers (E2M1 x scale, exact in bf16 for
+//     UE4M3 scales) into the K tile, 128B-swizzled K-major: 9 atoms of 64
+//     channels x 96 keys.
+//  3. One thread issues S = Q K^T: 36 tcgen05.mma (M=128, N=96, K=16) into
+//     TMEM; rows 64..127 of the A operand read the next atom (don't-care rows).
+//  4. Warps 0-1 read their head's S row from TMEM (one thread per head), take
+//     max / exp2 / sum in fp32 and write P (bf16) 128B-swizzled K-major.
+//  5. One thread issues O^T = V^T P^T: the K tile's latent atoms read as an
+//     MN-major operand (no second copy), 4 x 6 tcgen05.mma (M=128 channels,
+//     N=64 heads, K=16 keys) into TMEM.
+//  6. All warps read O^T from TMEM and store the chunk's partial (m, l, O);
+//     attn_merge combines the chunks of a sequence by log-sum-exp.
+// Every wait on an mbarrier is bounded by a 2-second clock; on expiry the CTA
+// sets KVC_DEV_TIMEOUT, frees its tensor memory and returns.
+#include "kvc_internal.cuh"
+
+namespace kvc {
+namespace tc05 {
+
+constexpr int H = 64, D = 576, DV = 512, CK = 96, NT = 256;
+constexpr int NATOM = D / 64;                   // 9 channel atoms of 64
+constexpr int KGRP = CK / 8;                    // 12 groups of 8 keys
+constexpr uint32_t Q_BYTES = NATOM * 8 * 1024;  // 64 rows: 8 row groups per atom
+constexpr uint32_t K_ATOM = KGRP * 1024;        // one channel atom of the K tile
+constexpr uint32_t K_BYTES = NATOM * K_ATOM;
+constexpr uint32_t RAW_STRIDE = 320;            // record bytes reserved per key
+constexpr uint32_t RAW_BYTES = CK * RAW_STRIDE;
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+constexpr uint32_t OFF_RAW = OFF_K + K_BYTES;   // P (16 KB) reuses this after dequant
+constexpr uint32_t OFF_P = OFF_RAW;
+constexpr uint32_t OFF_MISC = OFF_RAW + RAW_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 3072 + 1024;  // + misc + table + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL = 0, O_COL = 128;
+
+// instruction descriptors (kind::f16): D f32, A and B bf16, M = 128
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(CK >> 3) << 17) |
+                              ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) /* A MN-major */ |
+                              ((uint32_t)(H >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// shared-memory matrix descriptor, 128-byte swizzle, sm100 version field
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(addr), "r"(count));
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// bounded wait for phase `parity` of an mbarrier; false after ~2 s
+__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if ((i & 255) == 255 && global_ns() - t0 > 2000000000ull) return false;
+    }
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mbar)
+        : "memory");
+}
+// 32 lanes x 32 consecutive columns of 32 bits: thread i gets lane (base+i)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+    const uint32_t m = c & 7u;  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6
+    const float mag =
+        m < 4u ? 0.5f * (float)m : (float)(1u << (m >> 1)) * (1.0f + 0.5f * (m & 1u)) * 0.5f;
+    return (c & 8u) ? -mag : mag;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// byte offset of 16-byte chunk `c16` of row `r` inside a 128B-swizzled block
+// whose rows are 128 bytes and whose 8-row groups are 1024 bytes apart
+__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c16) {
+    return (r >> 3) * 1024u + (r & 7u) * 128u + ((c16 ^ (r & 7u)) << 4);
+}
+
+__global__ void __launch_bounds__(NT, 1)
+attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int ue4m3) {
+    extern __shared__ unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzled tiles
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (base - raw_base);
+    const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sP = base + OFF_P;
+    unsigned char* raw = smem + OFF_RAW;
+    int* kind = reinterpret_cast<int*>(smem + OFF_MISC);                 // [CK]
+    float* mrow = reinterpret_cast<float*>(smem + OFF_MISC + 512);       // [H]
+    float* lrow = mrow + H;                                              // [H]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_MISC + 1536);  // S done, O done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 1600);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 2048);  // [256] bf16x2
+
+    const int b = blockIdx.y, split = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = a.n_entries[b];
+    const bool len_ok = n >= 0 && n <= a.capacity;
+    const int total = K + a.window_len;
+    const int rb = sh.rb;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    if (tid == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (tid < CK) {
+        const int j = split * CK + tid;
+        int k = -1;
+        if (j < total && len_ok) {
+            if (j < K) {
+                const int idx = a.topk_idx[(size_t)b * K + j];
+                if (idx >= 0 && idx < n)
+                    k = idx;
+                else if (idx != -1)
+                    set_status(a.status, KVC_DEV_BAD_INDEX);
+            } else {
+                k = -2 - (j - K);  // window row
+            }
+        }
+        kind[tid] = k;
+    }
+    {  // code-pair table: byte -> (E2M1(low nibble), E2M1(high nibble)) as bf16x2
+        lut[tid] = pack_bf16(e2m1_value(tid & 15u), e2m1_value(tid >> 4));
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- 1. gathers: Q (swizzled), records (raw rows), window rows (swizzled)
+    {
+        const unsigned char* qg = static_cast<const unsigned char*>(a.q) + (size_t)b * H * D * 2;
+        for (int p = tid; p < H * (D / 8); p += NT) {
+            const int h = p / (D / 8), c = p - h * (D / 8);
+            cp_async16(sQ + (c >> 3) * 8192u + swz(h, c & 7), qg + (size_t)h * D * 2 + c * 16);
+        }
+        const int pieces = rb >> 4;
+        for (int p = tid; p < CK * pieces; p += NT) {
+            const int s = p / pieces, pc = p - s * pieces;
+            const int k = kind[s];
+            if (k >= 0)
+                cp_async16(smem_u32(raw + s * RAW_STRIDE + pc * 16),
+                           a.records + ((size_t)b * a.capacity + k) * rb + pc * 16);
+        }
+        for (int p = tid; p < CK * (D / 8); p += NT) {
+            const int s = p / (D / 8), c = p - s * (D / 8);
+            const int k = kind[s];
+            const uint32_t dst = sK + (c >> 3) * K_ATOM + swz(s, c & 7);
+            if (k <= -2) {
+                const int t = -2 - k;
+                cp_async16(dst, static_cast<const unsigned char*>(a.window) +
+                                    ((size_t)b * a.window_stride + t) * D * 2 + c * 16);
+            } else if (k == -1) {
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(0u), "r"(0u),
+                             "r"(0u), "r"(0u));
+            }
+        }
+        cp_async_wait_all();
+    }
+    __syncthreads();
+
+    // ---- 2. dequantise records into the swizzled K tile.  UE4M3 scales: a
+    // byte of two codes -> bf16x2 table entry, times the bf16x2 scale (the
+    // products have at most 6 significant bits, so the bf16 multiply is exact).
+    if (ue4m3) {
+        for (int p = tid; p < CK * (D / 8); p += NT) {
+            const int s = p / (D / 8), c = p - s * (D / 8);
+            if (kind[s] < 0) continue;
+            const unsigned char* rec = raw + s * RAW_STRIDE;
+            const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + c * 4);
+            const float sc = e4m3_to_f32(rec[sh.code_bytes + c / sh.lpg]);
+            const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc, sc);
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t e = lut[(codes >> (8 * k)) & 0xFFu];
+                const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e), s2);
+                w[k] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                             sK + (c >> 3) * K_ATOM + swz(s, c & 7)),
+                         "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+        }
+    } else {
+        for (int p = tid; p < CK * (D / 8); p += NT) {
+            const int s = p / (D / 8), c = p - s * (D / 8);
+            if (kind[s] < 0) continue;
+            const unsigned char* rec = raw + s * RAW_STRIDE;
+            const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + c * 4);
+            const float sc = reinterpret_cast<const float*>(rec + sh.code_bytes)[c / sh.lpg];
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                w[k] = pack_bf16(e2m1_value((codes >> (8 * k)) & 15u) * sc,
+                                 e2m1_value((codes >> (8 * k + 4)) & 15u) * sc);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                             sK + (c >> 3) * K_ATOM + swz(s, c & 7)),
+                         "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+        }
+    }
+    fence_async_smem();
+    __syncthreads();
+
+    // ---- 3. S = Q K^T (one thread issues)
+    if (tid == 0) {
+        tc_fence_after();
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t at = ks >> 2, koff = (ks & 3) * 32;
+            mma_bf16(tmem + S_COL, sdesc(sQ + at * 8192u + koff, 16, 1024),
+                     sdesc(sK + at * K_ATOM + koff, 16, 1024), kIdescQK, ks > 0);
+        }
+        mma_commit(smem_u32(&bars[0]));
+    }
+    bool ok = __syncthreads_and(mbar_wait(smem_u32(&bars[0]), 0)) != 0;
+    tc_fence_after();
+
+    // ---- 4. softmax: warps 0-1, one thread per head row of S
+    if (ok && warp < 2) {
+        const int h = warp * 32 + lane;
+        float sv[CK];
+#pragma unroll
+        for (int c0 = 0; c0 < CK; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + S_COL + c0, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[c0 + i] = __uint_as_float(r[i]);
+        }
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < CK; ++j) {
+            const float x = kind[j] == -1 ? -INFINITY : sv[j] * scale_log2;
+            sv[j] = x;
+            m = fmaxf(m, x);
+        }
+        float l = 0.f;
+#pragma unroll
+        for (int cj = 0; cj < CK / 8; ++cj) {
+            float p[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                p[u] = m == -INFINITY ? 0.f : exp2f(sv[cj * 8 + u] - m);
+                l += p[u];
+            }
+            const uint32_t dst = sP + (cj >> 3) * 8192u + swz(h, cj & 7);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst),
+                         "r"(pack_bf16(p[0], p[1])), "r"(pack_bf16(p[2], p[3])),
+                         "r"(pack_bf16(p[4], p[5])), "r"(pack_bf16(p[6], p[7])));
+        }
+        mrow[h] = m;
+        lrow[h] = l;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- 5. O^T = V^T P^T (one thread issues); V^T = latent atoms of the K tile
+    if (ok && tid == 0) {
+        tc_fence_after();
+        for (int mt = 0; mt < DV / 128; ++mt)
+            for (int kk = 0; kk < CK / 16; ++kk)
+                mma_bf16(tmem + O_COL + 64 * mt,
+                         sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
+                         sdesc(sP + (kk >> 2) * 8192u + (kk & 3) * 32u, 16, 1024), kIdescPV,
+                         kk > 0);
+        mma_commit(smem_u32(&bars[1]));
+    }
+    bool ok2 = false;
+    if (ok) ok2 = mbar_wait(smem_u32(&bars[1]), 0);
+    const bool ok_s = ok;
+    ok = __syncthreads_and(ok2) != 0;
+    tc_fence_after();
+
+    // ---- 6. epilogue: thread = one latent channel, 64 heads from TMEM
+    if (ok) {
+        const int g = warp & 3;                 // TMEM lanes 32g .. 32g+31
+        for (int t = 0; t < 2; ++t) {
+            const int mt = (warp >> 2) * 2 + t;
+            const int d = mt * 128 + g * 32 + lane;
+            for (int h0 = 0; h0 < H; h0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
+                if (nsplit == 1) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float l = lrow[h0 + i];
+                        a.out[((size_t)b * H + h0 + i) * DV + d] =
+                            l > 0.f ? __uint_as_float(r[i]) / l : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        a.part_o[(((size_t)b * H + h0 + i) * kMaxSplit + split) * DV + d] =
+                            __uint_as_float(r[i]);
+                }
+            }
+        }
+        if (tid < H) {
+            const float m = mrow[tid], l = lrow[tid];
+            if (nsplit == 1) {
+                if (a.lse) a.lse[(size_t)b * H + tid] = l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f
+                                                                : -INFINITY;
+            } else {
+                const size_t row = ((size_t)b * H + tid) * kMaxSplit + split;
+                a.part_ml[row * 2] = m;
+                a.part_ml[row * 2 + 1] = l;
+            }
+        }
+    } else {
+        // a bounded wait gave up: flag it, give the MMAs that were issued one
+        // more bounded wait, then free the tensor memory
+        if (tid == 0) {
+            set_status(a.status, KVC_DEV_TIMEOUT);
+            mbar_wait(smem_u32(&bars[0]), 0);
+            if (ok_s) mbar_wait(smem_u32(&bars[1]), 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                     "r"(TMEM_COLS));
+    }
+}
+
+}  // namespace tc05
+
+bool tc05_supported(const kvc_config& c, const Shape& sh) {
+    return c.act_dtype == KVC_BF16 && c.n_heads == tc05::H && sh.D == tc05::D &&
+           sh.Dv == tc05::DV && sh.rb <= (int)tc05::RAW_STRIDE;
+}
+
+// Launches the chunks of every sequence; returns the number of splits (chunks)
+// so the caller merges them, or a negative value on a launch error.
+int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& a,
+                          cudaStream_t s) {
+    const int total = c.topk + a.window_len;
+    const int nsplit = (total + tc05::CK - 1) / tc05::CK;
+    if (nsplit > kMaxSplit) return -1;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(tc05::attn_tc05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc05::SMEM_BYTES) != cudaSuccess)
+            return -1;
+        attr_set[dev] = true;
+    }
+    trace_before("attn_tc05", s);
+    tc05::attn_tc05_kernel<<<dim3(nsplit, a.batch), tc05::NT, tc05::SMEM_BYTES, s>>>(
+        a, sh, c.topk, c.sm_scale * 1.4426950408889634f, nsplit,
+        c.scale_fmt == KVC_SCALE_UE4M3);
+    trace_after(s);
+    return cudaGetLastError() == cudaSuccess ? nsplit : -1;
+}
+
+}  // namespace kvc

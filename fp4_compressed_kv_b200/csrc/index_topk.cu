@@ -11,22 +11,23 @@
 // Design (B200): the scan is a pure HBM stream of 128-byte int8 rows.
 //  1. index_scan: a grid of CTAs tiles every sequence's visible entries;
 //     Di/16 lanes share a row, each loading 16 bytes (coalesced 512-byte warp
-//     loads, 4 rows in flight per lane), dp4a + xor-shuffle reduce to the
+//     loads, 8 rows in flight per lane), dp4a + xor-shuffle reduce to the
 //     score.  Each score is stored (4 bytes beside the 128 read) and counted
-//     in a 2048-bin shared-memory histogram of its biased value; the CTA then
-//     adds its non-zero bins to the sequence's global histogram.
-//  2. topk_collect: every CTA rebuilds the threshold bin t from the global
-//     histogram (the highest bin whose suffix count reaches K) and appends
-//     the (score, index) keys of entries in bins >= t to a candidate list
-//     (warp-aggregated atomics).  Typically K + a few dozen candidates.
-//  3. topk_finalize: one CTA per sequence.  Entries above bin t are all in;
-//     the r = K - count(bins > t) best of bin t are chosen by exact ranking
-//     of 64-bit keys (score, ~index); the K winners are then placed in index
-//     order by rank counting.  If more than kMaxCand candidates reached the
-//     list (heavy ties), a slower exact path finds the threshold score and
-//     the index cut-off with a second histogram and compacts the scores in
-//     index order.
-// No kernel waits on another CTA: the three launches are stream-ordered.
+//     in a 2048-bin shared-memory histogram of its biased value; the CTA adds
+//     its non-zero bins to the sequence's histogram.  The last scan CTA of a
+//     sequence (a fenced counter; nobody waits) derives the threshold bin t
+//     (the highest bin whose suffix count reaches K) and the count above it.
+//  2. topk_select: a CTA per tile of 2,048 scores compacts the (score, index)
+//     keys of its entries in bins >= t, in index order, into the tile's own
+//     slot (block prefix sum; typically a few dozen per tile).  The last CTA
+//     of a sequence to finish completes the selection without sorting the
+//     output: the r = K - above best keys of bin t (a bitonic sort of the few
+//     tie candidates) give the cut-off key k*, every candidate with key >= k*
+//     is selected, and a prefix sum over the tiles places the winners -- the
+//     tiles are in index order, so the output is too.  If more than kMaxTies
+//     entries share bin t, an exact slower path finds the threshold score and
+//     the index cut-off with a second histogram and compacts the scores.
+// No CTA waits on another: the two launches are stream-ordered.
 #include "kvc_internal.cuh"
 
 namespace kvc {
@@ -45,44 +46,51 @@ __device__ __forceinline__ int key_index(unsigned long long k) {
     return (int)(~(uint32_t)(k & 0xffffffffull));
 }
 
+// Block-wide exclusive prefix sum of one int per thread; returns the block total.
+__device__ int block_excl_scan(int v, int* excl, int* sh_warp) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += u;
+    }
+    __syncthreads();
+    if (lane == 31) sh_warp[w] = x;
+    __syncthreads();
+    int pre = 0, total = 0;
+    for (int i = 0; i < nw; ++i) {
+        if (i < w) pre += sh_warp[i];
+        total += sh_warp[i];
+    }
+    *excl = pre + x - v;
+    return total;
+}
+
 // Block-wide: threshold bin t = the highest bin whose suffix count >= K, and
-// the count of entries in bins above t.  Requires total >= K.  blockDim.x
-// must be a multiple of 32 and divide kBins.
-__device__ void find_threshold(const int32_t* __restrict__ hist, int K, int* t_out,
-                               int* above_out, int* sh_warp) {
+// the count of entries in bins above t, from a histogram already staged in
+// shared memory.  Requires total >= K.  blockDim.x must divide kBins.
+__device__ void find_threshold(const int* s_hist, int K, int* t_out, int* above_out,
+                               int* sh_warp) {
     const int nt = blockDim.x, tid = threadIdx.x;
     const int per = kBins / nt;
-    if (tid == 0) {
-        *t_out = 0;
-        *above_out = 0;
-    }
     // thread tid covers bins [kBins - (tid+1)*per, kBins - tid*per): thread 0 the top
     const int hi = kBins - tid * per, lo = hi - per;
     int local = 0;
-    for (int b = lo; b < hi; ++b) local += hist[b];
-    // inclusive prefix over threads (top bins first)
-    int v = local;
-    const int lane = tid & 31, w = tid >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-    }
-    if (lane == 31) sh_warp[w] = v;
-    __syncthreads();
-    int warp_prefix = 0;
-    for (int i = 0; i < w; ++i) warp_prefix += sh_warp[i];
-    const int incl = v + warp_prefix;
-    const int excl = incl - local;  // count strictly above bin hi-1
+    for (int b = lo; b < hi; ++b) local += s_hist[b];
+    int excl;
+    // prefix over threads in order: thread 0 holds the top bins
+    block_excl_scan(local, &excl, sh_warp);
+    const int incl = excl + local;
     if (excl < K && incl >= K) {
         int run = excl;
         for (int b = hi - 1; b >= lo; --b) {
-            if (run + hist[b] >= K) {
+            if (run + s_hist[b] >= K) {
                 *t_out = b;
                 *above_out = run;
                 break;
             }
-            run += hist[b];
+            run += s_hist[b];
         }
     }
     __syncthreads();
@@ -91,10 +99,12 @@ __device__ void find_threshold(const int32_t* __restrict__ hist, int K, int* t_o
 template <int DI>
 __global__ void __launch_bounds__(kThreads)
 index_scan_kernel(TopkArgs a, int tile, int bias, int shift) {
-    __shared__ int hist[kBins];
+    __shared__ __align__(16) int hist[kBins];
+    __shared__ int sh_warp[kThreads / 32];
+    __shared__ int s_last, s_t, s_above;
     constexpr int TPR = DI / 16;   // lanes per row
     constexpr int RPW = 32 / TPR;  // rows per warp step
-    constexpr int UNROLL = 4;
+    constexpr int UNROLL = 8;
     const int b = blockIdx.y;
     const int n = a.n_entries[b];
     if (n < 0 || n > a.capacity) {
@@ -139,145 +149,196 @@ index_scan_kernel(TopkArgs a, int tile, int bias, int shift) {
         }
     }
     __syncthreads();
-    int32_t* gh = a.hist + (size_t)b * kBins;
+    int32_t* gh = a.counters + (size_t)b * kBins;
     for (int i = threadIdx.x; i < kBins; i += kThreads)
         if (hist[i]) atomicAdd(&gh[i], hist[i]);
+    if (n <= a.topk) return;  // everything is selected; no threshold needed
+
+    // the last scan CTA of this sequence derives the threshold
+    __threadfence();
+    __syncthreads();
+    const int nctas = (n + tile - 1) / tile;
+    if (threadIdx.x == 0)
+        s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) == nctas - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int i = threadIdx.x * 4; i < kBins; i += kThreads * 4)
+        *reinterpret_cast<int4*>(hist + i) = __ldcg(reinterpret_cast<const int4*>(gh + i));
+    if (threadIdx.x == 0) s_t = s_above = 0;
+    __syncthreads();
+    find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
+    if (threadIdx.x == 0) {
+        a.thr[2 * b] = s_t;
+        a.thr[2 * b + 1] = s_above;
+    }
 }
+
+// In-place block bitonic sort of p (a power of two) keys; descending when
+// `desc`.  Every thread of the block must call it.
+template <typename Key>
+__device__ void block_bitonic(Key* k, int p, bool desc) {
+    for (int size = 2; size <= p; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < p; i += blockDim.x) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const bool up = ((i & size) == 0) != desc;  // ascending run
+                    const Key x = k[i], y = k[j];
+                    if ((x > y) == up) {
+                        k[i] = y;
+                        k[j] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+constexpr size_t kSelSmem = (size_t)kMaxTies * 8 + (size_t)kMaxSelTiles * 4 * 2;
 
 __global__ void __launch_bounds__(kThreads)
-topk_collect_kernel(TopkArgs a, int tile, int bias, int shift) {
-    __shared__ int sh_warp[kThreads / 32];
-    __shared__ int s_t, s_above;
-    const int b = blockIdx.y;
-    const int n = a.n_entries[b];
-    if (n < 0 || n > a.capacity || n <= a.topk) return;
-    const int start = blockIdx.x * tile;
-    if (start >= n) return;
-    const int end = min(start + tile, n);
-    find_threshold(a.hist + (size_t)b * kBins, a.topk, &s_t, &s_above, sh_warp);
-    const int t = s_t;
-    const int32_t* sc = a.scores + (size_t)b * a.capacity;
-    unsigned long long* cand = a.cands + (size_t)b * kMaxCand;
-    const int lane = threadIdx.x & 31;
-    for (int base = start; base < end; base += kThreads) {
-        const int j = base + threadIdx.x;
-        int s = 0;
-        bool take = false;
-        if (j < end) {
-            s = __ldcg(sc + j);
-            take = score_bin(s, bias, shift) >= t;
-        }
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        if (m) {
-            int first = 0;
-            if (lane == 0) first = atomicAdd(&a.cand_count[b], __popc(m));
-            first = __shfl_sync(0xffffffffu, first, 0);
-            if (take) {
-                const int pos = first + __popc(m & ((1u << lane) - 1u));
-                if (pos < kMaxCand) cand[pos] = make_key(s, j, bias);
-            }
-        }
-    }
-}
-
-// Block-wide exclusive prefix sum of one int per thread; returns the block total.
-__device__ int block_excl_scan(int v, int* excl, int* sh_warp) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += u;
-    }
-    __syncthreads();
-    if (lane == 31) sh_warp[w] = x;
-    __syncthreads();
-    int pre = 0, total = 0;
-    for (int i = 0; i < nw; ++i) {
-        if (i < w) pre += sh_warp[i];
-        total += sh_warp[i];
-    }
-    *excl = pre + x - v;
-    return total;
-}
-
-constexpr int kFinThreads = 1024;
-
-__global__ void __launch_bounds__(kFinThreads)
-topk_finalize_kernel(TopkArgs a, int bias, int shift) {
+topk_select_kernel(TopkArgs a, int bias, int shift) {
     extern __shared__ __align__(16) unsigned char smem[];
-    unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem);  // kMaxCand
-    int* tie = reinterpret_cast<int*>(keys + kMaxCand);                      // kMaxCand
-    int* sel = tie + kMaxCand;                                               // <= K
-    __shared__ int sh_warp[kFinThreads / 32];
-    __shared__ int s_t, s_above, s_ntie, s_nsel, s_low, s_gt;
-
-    const int b = blockIdx.x, K = a.topk;
-    int32_t* out = a.topk_idx + (size_t)b * K;
+    unsigned long long* ties = reinterpret_cast<unsigned long long*>(smem);  // kMaxTies
+    int* cnt = reinterpret_cast<int*>(ties + kMaxTies);                       // per tile
+    int* off = cnt + kMaxSelTiles;                                            // per tile
+    __shared__ int sh_warp[kThreads / 32];
+    __shared__ int s_last, s_nt, s_low, s_gt;
+    __shared__ unsigned long long s_kstar;
+    const int b = blockIdx.y, K = a.topk, tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
     const int n = a.n_entries[b];
+    int32_t* out = a.topk_idx + (size_t)b * K;
     if (n < 0 || n > a.capacity) {
-        for (int i = threadIdx.x; i < K; i += blockDim.x) out[i] = -1;
+        if (blockIdx.x == 0)
+            for (int i = tid; i < K; i += kThreads) out[i] = -1;
         return;
     }
     if (n <= K) {
-        for (int i = threadIdx.x; i < K; i += blockDim.x) out[i] = i < n ? i : -1;
+        if (blockIdx.x == 0)
+            for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
-    const int32_t* hist = a.hist + (size_t)b * kBins;
-    find_threshold(hist, K, &s_t, &s_above, sh_warp);
-    const int t = s_t, r = K - s_above;  // take r entries of bin t
-    const int M = __ldcg(a.cand_count + b);
+    const int ntiles = (n + kSelTile - 1) / kSelTile;
+    const int tile = blockIdx.x;
+    if (tile >= ntiles) return;
+    const int t = __ldcg(a.thr + 2 * b), above = __ldcg(a.thr + 2 * b + 1);
+    const int32_t* sc = a.scores + (size_t)b * a.capacity;
+    const int ctiles = sel_tiles(a.capacity);
+    unsigned long long* cand = a.cands + ((size_t)b * ctiles + tile) * kSelTile;
 
-    if (M <= kMaxCand) {
-        if (threadIdx.x == 0) s_ntie = s_nsel = 0;
+    // ---- compact this tile's candidates (bins >= t) in index order
+    {
+        int v[8];
+        const int j0 = tile * kSelTile + tid * 8;
+        if (j0 + 8 <= n && ((reinterpret_cast<uintptr_t>(sc + j0) & 15) == 0)) {
+            const int4 x0 = __ldcg(reinterpret_cast<const int4*>(sc + j0));
+            const int4 x1 = __ldcg(reinterpret_cast<const int4*>(sc + j0) + 1);
+            v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+            v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = (j0 + u < n) ? __ldcg(sc + j0 + u) : 0;
+        }
+        unsigned take = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (j0 + u < n && score_bin(v[u], bias, shift) >= t) take |= 1u << u;
+        int pos;
+        const int total = block_excl_scan(__popc(take), &pos, sh_warp);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (take & (1u << u)) cand[pos++] = make_key(v[u], j0 + u, bias);
+        if (tid == 0) a.tile_count[(size_t)b * ctiles + tile] = total;
+    }
+    // ---- the last CTA of this sequence to finish completes the selection
+    __threadfence();
+    __syncthreads();
+    if (tid == 0)
+        s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + a.batch + b, 1) == ntiles - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    const unsigned long long* cb = a.cands + (size_t)b * ctiles * kSelTile;
+    for (int i = tid; i < ntiles; i += kThreads) cnt[i] = __ldcg(a.tile_count + (size_t)b * ctiles + i);
+    if (tid == 0) s_nt = 0;
+    __syncthreads();
+    // the tie candidates: keys of bin t (a warp per tile)
+    const int r = K - above;
+    for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
+        const unsigned long long* ct = cb + (size_t)ti * kSelTile;
+        for (int i = lane; i < cnt[ti]; i += 32) {
+            const unsigned long long k = __ldcg(ct + i);
+            if ((int)((k >> 32) >> shift) == t) {
+                const int p = atomicAdd(&s_nt, 1);
+                if (p < kMaxTies) ties[p] = k;
+            }
+        }
+    }
+    __syncthreads();
+    const int nt = s_nt;
+    if (nt <= kMaxTies) {
+        int p2 = 1;
+        while (p2 < nt) p2 <<= 1;
+        for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;  // sorts last
         __syncthreads();
-        const unsigned long long* cand = a.cands + (size_t)b * kMaxCand;
-        for (int i = threadIdx.x; i < M; i += blockDim.x) {
-            const unsigned long long k = __ldcg(cand + i);
-            keys[i] = k;
-            const int bin = (int)((k >> 32) >> shift);
-            if (bin == t) {
-                tie[atomicAdd(&s_ntie, 1)] = i;
-            } else {
-                const int p = atomicAdd(&s_nsel, 1);
-                if (p < K) sel[p] = key_index(k);
+        block_bitonic(ties, p2, true);
+        if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;  // r-th best of bin t
+        __syncthreads();
+        const unsigned long long kstar = s_kstar;
+        // winners per tile, prefix over tiles, then write in index order
+        for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
+            const unsigned long long* ct = cb + (size_t)ti * kSelTile;
+            int c = 0;
+            for (int i = lane; i < cnt[ti]; i += 32) c += __ldcg(ct + i) >= kstar;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+            if (lane == 0) off[ti] = c;
+        }
+        __syncthreads();
+        int run = 0;
+        for (int base = 0; base < ntiles; base += kThreads) {
+            const int i = base + tid;
+            const int c = i < ntiles ? off[i] : 0;
+            int ex;
+            const int tot = block_excl_scan(c, &ex, sh_warp);
+            if (i < ntiles) off[i] = run + ex;
+            run += tot;
+            __syncthreads();
+        }
+        for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
+            const unsigned long long* ct = cb + (size_t)ti * kSelTile;
+            int o = off[ti];
+            for (int i0 = 0; i0 < cnt[ti]; i0 += 32) {
+                const int i = i0 + lane;
+                const unsigned long long k = i < cnt[ti] ? __ldcg(ct + i) : 0ull;
+                const bool sel = i < cnt[ti] && k >= kstar;
+                const unsigned m = __ballot_sync(0xffffffffu, sel);
+                const int p = o + __popc(m & ((1u << lane) - 1u));
+                if (sel && p < K) out[p] = key_index(k);
+                o += __popc(m);
             }
         }
         __syncthreads();
-        const int nt = s_ntie;
-        for (int i = threadIdx.x; i < nt; i += blockDim.x) {
-            const unsigned long long k = keys[tie[i]];
-            int rank = 0;
-            for (int j = 0; j < nt; ++j) rank += keys[tie[j]] > k;
-            if (rank < r) {
-                const int p = atomicAdd(&s_nsel, 1);
-                if (p < K) sel[p] = key_index(k);
-            }
-        }
-        __syncthreads();
-        // s_nsel == K here; place winners in ascending index order
-        for (int i = threadIdx.x; i < K; i += blockDim.x) {
-            const int v = sel[i];
-            int pos = 0;
-            for (int j = 0; j < K; ++j) pos += sel[j] < v;
-            out[pos] = v;
-        }
+        for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
         return;
     }
 
     // Heavy ties: exact threshold score inside bin t from a second histogram
     // over the low `shift` bits (<= 4096 bins), then an index-order pass.
-    int* h2 = reinterpret_cast<int*>(smem);  // 1 << shift ints (<= 16 KB)
+    int* h2 = reinterpret_cast<int*>(smem);
     const int nb2 = 1 << shift;
-    for (int i = threadIdx.x; i < nb2; i += blockDim.x) h2[i] = 0;
+    for (int i = tid; i < nb2; i += kThreads) h2[i] = 0;
     __syncthreads();
-    const int32_t* sc = a.scores + (size_t)b * a.capacity;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    for (int j = tid; j < n; j += kThreads) {
         const int v = __ldcg(sc + j) + bias;
         if ((v >> shift) == t) atomicAdd(&h2[v & (nb2 - 1)], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         int run = 0, low = 0;
         for (int i = nb2 - 1; i >= 0; --i) {
             if (run + h2[i] >= r) {
@@ -286,15 +347,15 @@ topk_finalize_kernel(TopkArgs a, int bias, int shift) {
             }
             run += h2[i];
         }
-        s_low = low;       // threshold score = (t << shift | low) - bias
-        s_gt = run;        // entries of bin t above the threshold score
+        s_low = low;  // threshold score = (t << shift | low) - bias
+        s_gt = run;   // entries of bin t above the threshold score
     }
     __syncthreads();
     const int thr = ((t << shift) | s_low) - bias;
     const int need_eq = r - s_gt;  // entries equal to thr to take, lowest index first
     int taken = 0, eq_seen = 0;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int j = base + threadIdx.x;
+    for (int base = 0; base < n; base += kThreads) {
+        const int j = base + tid;
         const int s = j < n ? __ldcg(sc + j) : INT32_MIN;
         const int is_eq = (j < n && s == thr) ? 1 : 0;
         int eq_before;
@@ -306,7 +367,7 @@ topk_finalize_kernel(TopkArgs a, int bias, int shift) {
         taken += take_total;
         eq_seen += eq_total;
     }
-    for (int i = taken + threadIdx.x; i < K; i += blockDim.x) out[i] = -1;
+    for (int i = taken + tid; i < K; i += kThreads) out[i] = -1;
 }
 
 template <int DI>
@@ -316,17 +377,14 @@ cudaError_t launch_scan(const TopkArgs& a, int tile, int bias, int shift, cudaSt
     return cudaGetLastError();
 }
 
-size_t finalize_smem() {
-    return (size_t)kMaxCand * 8 + (size_t)kMaxCand * 4 + 2048 * 4;
-}
-
 }  // namespace
 
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     if (a.batch == 0) return cudaSuccess;
     const int bias = score_bias(a.di), shift = score_shift(a.di);
-    // zero the histograms and candidate counters (adjacent in the workspace)
-    cudaError_t err = cudaMemsetAsync(a.hist, 0, (size_t)a.batch * (kBins + 1) * sizeof(int32_t), s);
+    // zero the histograms and the finished-CTA counters (adjacent in the workspace)
+    cudaError_t err =
+        cudaMemsetAsync(a.counters, 0, topk_counter_words(a.batch) * sizeof(int32_t), s);
     if (err != cudaSuccess) return err;
     // scan tile: aim for about 4 CTAs per SM over the whole batch
     const long long rows = (long long)a.batch * a.capacity;
@@ -344,25 +402,18 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     }
     trace_after(s);
     if (err != cudaSuccess) return err;
-    {
-        const int ctile = 16384;
-        dim3 grid((a.capacity + ctile - 1) / ctile, a.batch);
-        trace_before("topk_collect", s);
-        topk_collect_kernel<<<grid, kThreads, 0, s>>>(a, ctile, bias, shift);
-        trace_after(s);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    }
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        err = cudaFuncSetAttribute(topk_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)finalize_smem());
+        err = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kSelSmem);
         if (err != cudaSuccess) return err;
         attr_set[dev] = true;
     }
-    trace_before("topk_finalize", s);
-    topk_finalize_kernel<<<a.batch, kFinThreads, finalize_smem(), s>>>(a, bias, shift);
+    dim3 grid(sel_tiles(a.capacity), a.batch);
+    trace_before("topk_select", s);
+    topk_select_kernel<<<grid, kThreads, kSelSmem, s>>>(a, bias, shift);
     trace_after(s);
     return cudaGetLastError();
 }

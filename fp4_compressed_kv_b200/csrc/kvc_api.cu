@@ -121,17 +121,22 @@ constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t scores, hist, cands, part_o, part_ml, total;
+    size_t scores, counters, thr, tile_count, cands, part_o, part_ml, total;
 };
 WsLayout ws_layout(const kvc_config& c, const Shape& sh, int batch, int cap) {
     WsLayout w;
     size_t off = 0;
+    const size_t tiles = (size_t)batch * sel_tiles(cap);
     w.scores = off;
     off = up(off + (size_t)batch * cap * 4);
-    w.hist = off;  // hist [B][kBins] followed by cand_count [B]
-    off = up(off + (size_t)batch * (kBins + 1) * 4);
+    w.counters = off;  // histograms [B][kBins], finished scan CTAs [B], finished select CTAs [B]
+    off = up(off + topk_counter_words(batch) * 4);
+    w.thr = off;
+    off = up(off + (size_t)batch * 2 * 4);
+    w.tile_count = off;
+    off = up(off + tiles * 4);
     w.cands = off;
-    off = up(off + (size_t)batch * kMaxCand * 8);
+    off = up(off + tiles * kSelTile * 8);
     w.part_o = off;
     off = up(off + (size_t)batch * c.n_heads * kMaxSplit * sh.Dv * 4);
     w.part_ml = off;
@@ -174,6 +179,7 @@ kvc_status check_ws(void* ws, size_t ws_bytes, const kvc_config& c, const Shape&
 kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* cache,
                     int32_t* topk, int32_t* scores, unsigned char* ws, const WsLayout& w,
                     uint32_t* st, cudaStream_t s) {
+    if (cache->capacity > kMaxTopkCapacity) return KVC_ERR_CAPACITY;
     TopkArgs a;
     a.idx_q = idx_q;
     a.idx_k = cache->idx_k;
@@ -184,8 +190,9 @@ kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* c
     a.di = c.idx_dim;
     a.topk_idx = topk;
     a.scores = scores ? scores : reinterpret_cast<int32_t*>(ws + w.scores);
-    a.hist = reinterpret_cast<int32_t*>(ws + w.hist);
-    a.cand_count = a.hist + (size_t)cache->batch * kBins;
+    a.counters = reinterpret_cast<int32_t*>(ws + w.counters);
+    a.thr = reinterpret_cast<int32_t*>(ws + w.thr);
+    a.tile_count = reinterpret_cast<int32_t*>(ws + w.tile_count);
     a.cands = reinterpret_cast<unsigned long long*>(ws + w.cands);
     a.status = st;
     return launch_index_topk(a, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;

@@ -12,8 +12,18 @@ namespace kvc {
 
 // Indexer histogram: 2048 bins over the biased int8 x int8 score range.
 constexpr int kBins = 2048;
-// Candidates per sequence kept for the in-shared-memory top-K finish.
-constexpr int kMaxCand = 4096;
+// Top-K selection: scores are cut into tiles of kSelTile entries; each tile
+// keeps its candidate keys (in index order) in its own slot of the candidate
+// array.  A sequence holds at most kMaxSelTiles tiles (8,388,608 entries).
+constexpr int kSelTile = 2048;
+constexpr int kMaxSelTiles = 4096;
+constexpr long long kMaxTopkCapacity = (long long)kSelTile * kMaxSelTiles;
+// Candidates of the threshold bin kept for the in-shared-memory finish.
+constexpr int kMaxTies = 4096;
+__host__ __device__ inline int sel_tiles(int capacity) { return (capacity + kSelTile - 1) / kSelTile; }
+// Per-call counters of the top-K: histograms [B][kBins], finished scan CTAs
+// [B] and finished select CTAs [B], adjacent so one memset clears them.
+inline size_t topk_counter_words(int batch) { return (size_t)batch * (kBins + 2); }
 // Upper bound on the number of key splits of one attention problem.
 constexpr int kMaxSplit = 16;
 // Keys per attention chunk.
@@ -73,9 +83,10 @@ struct TopkArgs {
     int batch, capacity, topk, di;
     int32_t* topk_idx;     // [B][K]
     int32_t* scores;       // [B][cap] (user buffer or workspace)
-    int32_t* hist;         // [B][kBins] (zeroed by the launcher)
-    int32_t* cand_count;   // [B]        (zeroed by the launcher)
-    unsigned long long* cands;  // [B][kMaxCand]
+    int32_t* counters;     // topk_counter_words(B) ints, zeroed by the launcher
+    int32_t* thr;          // [B][2] threshold bin, entries above it (written by the scan)
+    int32_t* tile_count;   // [B][sel_tiles(cap)] candidates per tile
+    unsigned long long* cands;  // [B][sel_tiles(cap) * kSelTile]
     uint32_t* status;
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);

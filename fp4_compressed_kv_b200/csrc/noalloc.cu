@@ -9,7 +9,7 @@
 // per-sequence histograms and counters, the candidate lists -- lives in the
 // file-scope array below, sized for at most kNoAllocMaxBatch sequences and
 // kNoAllocMaxRows = batch x capacity entries.  Every GPU that loads the library
-// holds the array (about 6.5 MiB) until the process exits.
+// holds the array (about 8 MiB) until the process exits.
 #include <mutex>
 
 #include "kvc_internal.cuh"
@@ -18,11 +18,15 @@ namespace kvc {
 namespace {
 
 constexpr int kNoAllocMaxBatch = 64;
-constexpr long long kNoAllocMaxRows = 1ll << 20;
+constexpr long long kNoAllocMaxRows = 1ll << 19;
+// tiles of the top-K selection over the whole batch: each sequence rounds up
+constexpr size_t kMaxTiles = (size_t)(kNoAllocMaxRows / kSelTile) + kNoAllocMaxBatch;
 constexpr size_t kScoresBytes = (size_t)kNoAllocMaxRows * 4;
-constexpr size_t kHistBytes = ((size_t)kNoAllocMaxBatch * (kBins + 1) * 4 + 255) / 256 * 256;
-constexpr size_t kCandBytes = (size_t)kNoAllocMaxBatch * kMaxCand * 8;
-constexpr size_t kScratchBytes = kScoresBytes + kHistBytes + kCandBytes;
+constexpr size_t kCounterBytes = ((size_t)kNoAllocMaxBatch * (kBins + 2) * 4 + 255) / 256 * 256;
+constexpr size_t kThrBytes = 512;
+constexpr size_t kTileCountBytes = (kMaxTiles * 4 + 255) / 256 * 256;
+constexpr size_t kCandBytes = kMaxTiles * kSelTile * 8;
+constexpr size_t kScratchBytes = kScoresBytes + kCounterBytes + kThrBytes + kTileCountBytes + kCandBytes;
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kScratchBytes];
 
@@ -87,9 +91,14 @@ extern "C" kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t
     a.di = cfg->idx_dim;
     a.topk_idx = topk_idx;
     a.scores = scores ? scores : reinterpret_cast<int32_t*>(ws);
-    a.hist = reinterpret_cast<int32_t*>(ws + kScoresBytes);  // cleared on the stream by the launcher
-    a.cand_count = a.hist + (size_t)cache->batch * kBins;
-    a.cands = reinterpret_cast<unsigned long long*>(ws + kScoresBytes + kHistBytes);
+    unsigned char* p = ws + kScoresBytes;
+    a.counters = reinterpret_cast<int32_t*>(p);  // cleared on the stream by the launcher
+    p += kCounterBytes;
+    a.thr = reinterpret_cast<int32_t*>(p);
+    p += kThrBytes;
+    a.tile_count = reinterpret_cast<int32_t*>(p);
+    p += kTileCountBytes;
+    a.cands = reinterpret_cast<unsigned long long*>(p);
     a.status = dev_status;
     return launch_index_topk(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVC_OK
                                                                                  : KVC_ERR_CUDA;

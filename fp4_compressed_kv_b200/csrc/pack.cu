@@ -8,70 +8,79 @@
 // group gets a scale, elements stored relative to it) and 3.2 (a learned key
 // compressor maps several tokens to one entry).
 //
-// Design (B200): one warp per entry, a pure HBM stream.  Lane l owns the
-// 8-channel chunks c = l, l+32, ...; each chunk of each token is one 16-byte
-// (bf16) or two 16-byte (fp32) coalesced loads, and each chunk's eight codes
-// leave as one 4-byte store, so a warp writes 128 contiguous bytes per step.
-// The group maximum is a xor-shuffle over the G/8 lanes of a group.
+// Design (B200): a pure HBM stream.  A team of 8 lanes owns one entry (4
+// entries per warp, 32 per CTA); lane l of a team owns the 8-channel chunks
+// c = l, l+8, ..., so for the 576-channel MLA entry every lane holds 9 chunks
+// and no lane idles.  Each chunk of each token is one 16-byte load and the 8
+// lanes of a team read 128 contiguous bytes; the raw bf16 chunks stay packed in
+// registers between the two passes.  A chunk's eight codes leave as one 4-byte
+// store (a team writes 32 contiguous bytes per pass).  Group maxima are xor
+// shuffles inside the team (G <= 64) or a shared-memory reduction (G > 64).
 //
-// Bit-exactness: the gate logit difference is accumulated in fp64 in a fixed
-// order -- lane l sums its chunks in increasing order with one fma per
-// channel, then a xor butterfly over offsets 16..1 -- and the pair weight
-// w0 = 1 / (1 + exp(-delta)) uses the exp below (Cody-Waite reduction with a
-// 32-bit head of ln 2, degree-13 Taylor polynomial in Horner form, exact
-// power-of-two scaling), so every implementation of this order produces the
-// same fp32 entry and therefore the same codes.
+// Bit-exactness: the gate logit difference is accumulated in fp32 in a fixed
+// order -- lane l sums its chunks in increasing order, one fmaf per channel
+// after an fp32 subtraction, then a xor tree over offsets 4, 2, 1 -- and the
+// pair weight w0 = 1 / (1 + exp(-delta)) uses the exp below (Cody-Waite
+// reduction with a 16-bit head of ln 2, degree-7 Taylor polynomial in Horner
+// form, exact power-of-two scaling), so every implementation of this order
+// produces the same fp32 entry and therefore the same codes.
 #include "kvc_internal.cuh"
 
 namespace kvc {
 namespace {
 
-constexpr double kLn2Hi = 0x1.62e42feep-1;
-constexpr double kLn2Lo = 0x1.a39ef35793c76p-33;
-constexpr double kInvLn2 = 0x1.71547652b82fep+0;
+constexpr float kLn2HiF = 0x1.62e4p-1f;
+constexpr float kLn2LoF = 0x1.7f7d1cp-20f;
+constexpr float kInvLn2F = 0x1.715476p+0f;
 
-__device__ __forceinline__ double exp_cody_waite(double x) {
+__device__ __forceinline__ float exp_cody_waite(float x) {
     if (x != x) return x;
-    if (x > 709.0) return __longlong_as_double(0x7ff0000000000000LL);
-    if (x < -708.0) return 0.0;
-    const double n = rint(__dmul_rn(x, kInvLn2));
-    double r = __fma_rn(-n, kLn2Hi, x);
-    r = __fma_rn(-n, kLn2Lo, r);
-    // 1/k! for k = 13 .. 0
-    double p = 0x1.6124613a86d09p-33;
-    p = __fma_rn(p, r, 0x1.1eed8eff8d898p-29);
-    p = __fma_rn(p, r, 0x1.ae64567f544e4p-26);
-    p = __fma_rn(p, r, 0x1.27e4fb7789f5cp-22);
-    p = __fma_rn(p, r, 0x1.71de3a556c734p-19);
-    p = __fma_rn(p, r, 0x1.a01a01a01a01ap-16);
-    p = __fma_rn(p, r, 0x1.a01a01a01a01ap-13);
-    p = __fma_rn(p, r, 0x1.6c16c16c16c17p-10);
-    p = __fma_rn(p, r, 0x1.1111111111111p-7);
-    p = __fma_rn(p, r, 0x1.5555555555555p-5);
-    p = __fma_rn(p, r, 0x1.5555555555555p-3);
-    p = __fma_rn(p, r, 0x1.0p-1);
-    p = __fma_rn(p, r, 1.0);
-    p = __fma_rn(p, r, 1.0);
-    const long long bits = ((long long)n + 1023) << 52;
-    return __dmul_rn(p, __longlong_as_double(bits));
+    if (x > 88.0f) return __int_as_float(0x7f800000);
+    if (x < -87.0f) return 0.0f;
+    const float n = rintf(__fmul_rn(x, kInvLn2F));
+    float r = __fmaf_rn(-n, kLn2HiF, x);
+    r = __fmaf_rn(-n, kLn2LoF, r);
+    // 1/k! for k = 7 .. 0
+    float p = 0x1.a01a02p-13f;
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);
+    p = __fmaf_rn(p, r, 0x1.0p-1f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    return __fmul_rn(p, __int_as_float(((int)n + 127) << 23));
 }
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float v[8]) {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+// Raw token chunk (8 channels) kept in registers between the passes.
+template <typename T>
+struct Chunk;
+template <>
+struct Chunk<__nv_bfloat16> {
+    uint4 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+        v = __ldcs(reinterpret_cast<const uint4*>(p));
     }
-}
-
-__device__ __forceinline__ void load8(const float* p, float v[8]) {
-    const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
+    __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ float get(int t) const {
+        const uint32_t w = t < 2 ? v.x : t < 4 ? v.y : t < 6 ? v.z : v.w;
+        return (t & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
+    }
+};
+template <>
+struct Chunk<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = __ldcs(reinterpret_cast<const float4*>(p));
+        b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float get(int t) const {
+        const float4& q = t < 4 ? a : b;
+        const int u = t & 3;
+        return u == 0 ? q.x : u == 1 ? q.y : u == 2 ? q.z : q.w;
+    }
+};
 
 __device__ __forceinline__ void load8_gate(const float* p, float v[8]) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(p));
@@ -80,120 +89,152 @@ __device__ __forceinline__ void load8_gate(const float* p, float v[8]) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-constexpr int kWarps = 8;
-constexpr int kTailBytes = 528;  // >= 1024/8 groups x 4 bytes + padding
+constexpr int kThreads = 256;
+constexpr int kTeams = kThreads / 8;  // entries per CTA
+constexpr int kTailBytes = 528;       // >= 128 groups x 4 bytes, padded
+constexpr int kMaxChunks = 128;       // D <= 1024
 
-// MAXJ: chunks per lane (D <= 256 * MAXJ).
+// MAXJ: chunks per lane (D <= 64 * MAXJ).
 template <typename T, int MAXJ>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kThreads)
 pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
-    __shared__ __align__(16) uint8_t tail_smem[kWarps][kTailBytes];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const long long e = (long long)blockIdx.x * kWarps + wid;
+    __shared__ __align__(16) uint8_t tail_smem[kTeams][kTailBytes];
+    __shared__ float cmax_smem[kTeams][kMaxChunks];  // only for groups wider than a team pass
+    const int lane = threadIdx.x & 31;
+    const int team = threadIdx.x >> 3, l = threadIdx.x & 7;
+    const long long e = (long long)blockIdx.x * kTeams + team;
     const int half = a.n_new >> 1;
-    if (e >= (long long)a.batch * half) return;
-    const int b = (int)(e / half), i = (int)(e % half);
-    const int base = a.n_entries[b];
-    if (base < 0 || base + half > a.capacity) {
-        if (lane == 0 && i == 0) set_status(a.status, KVC_DEV_CAPACITY);
-        return;
+    const bool in_range = e < (long long)a.batch * half;
+    int b = 0, i = 0, base = 0;
+    bool valid = false;
+    if (in_range) {
+        b = (int)(e / half);
+        i = (int)(e % half);
+        base = a.n_entries[b];
+        valid = base >= 0 && base + half <= a.capacity;
+        if (!valid && i == 0 && l == 0) set_status(a.status, KVC_DEV_CAPACITY);
     }
-    const long long pos = (long long)base + i;
     const int D = sh.D, nchunk = D >> 3;
+    const long long pos = (long long)base + i;
     const T* k0p = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 2 * i) * D;
     const T* k1p = k0p + D;
 
-    float k0[MAXJ][8], k1[MAXJ][8];
+    Chunk<T> k0[MAXJ], k1[MAXJ];
 #pragma unroll
     for (int j = 0; j < MAXJ; ++j) {
-        const int c = lane + 32 * j;
-        if (c < nchunk) {
-            load8(k0p + 8 * c, k0[j]);
-            load8(k1p + 8 * c, k1[j]);
+        const int c = l + 8 * j;
+        if (valid && c < nchunk) {
+            k0[j].load(k0p + 8 * c);
+            k1[j].load(k1p + 8 * c);
         } else {
-#pragma unroll
-            for (int t = 0; t < 8; ++t) k0[j][t] = k1[j][t] = 0.f;
+            k0[j].zero();
+            k1[j].zero();
         }
     }
 
-    // gate logit difference, fixed order
-    double acc = 0.0;
+    // gate logit difference, fixed order (all lanes take part in the shuffles)
+    float acc = 0.f;
 #pragma unroll
     for (int j = 0; j < MAXJ; ++j) {
-        const int c = lane + 32 * j;
-        if (c < nchunk) {
+        const int c = l + 8 * j;
+        if (valid && c < nchunk) {
             float g[8];
             load8_gate(a.gate + 8 * c, g);
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-                acc = __fma_rn((double)g[t], __dsub_rn((double)k0[j][t], (double)k1[j][t]), acc);
+                acc = __fmaf_rn(g[t], __fsub_rn(k0[j].get(t), k1[j].get(t)), acc);
         }
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1)
-        acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
-    const double w0 = __ddiv_rn(1.0, __dadd_rn(1.0, exp_cody_waite(-acc)));
-    const double w1 = __dsub_rn(1.0, w0);
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
+    const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-acc)));
+    const float w1 = __fsub_rn(1.0f, w0);
 
     uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
-    uint8_t* tail = tail_smem[wid];
+    uint8_t* tail = tail_smem[team];
     const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
-    for (int t = lane * 4; t < tail_len; t += 128) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
-    __syncwarp();
+    for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
 
+    // entry values and lane-local chunk maxima
     bool bad = false;
+    float cmax[MAXJ];
 #pragma unroll
     for (int j = 0; j < MAXJ; ++j) {
-        const int c = lane + 32 * j;
-        const bool active = c < nchunk;
-        float x[8];
-        float amax = 0.f;
+        const int c = l + 8 * j;
+        const bool active = valid && c < nchunk;
+        float m = 0.f;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            float v = __double2float_rn(
-                __fma_rn(w0, (double)k0[j][t], __dmul_rn(w1, (double)k1[j][t])));
-            if (!isfinite(v)) {
-                if (active) bad = true;
-                v = 0.f;
-            }
-            x[t] = v;
-            amax = fmaxf(amax, fabsf(v));
+            const float v = __fmaf_rn(w0, k0[j].get(t), __fmul_rn(w1, k1[j].get(t)));
+            if (isfinite(v)) m = fmaxf(m, fabsf(v));
+            else if (active) bad = true;
         }
-        for (int o = 1; o < sh.lpg; o <<= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        float s = __fdiv_rn(amax, 6.0f);
+        cmax[j] = m;
+    }
+    // group maxima
+    const int lpg = sh.lpg;
+    if (lpg <= 8) {
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j)
+            for (int o = 1; o < lpg; o <<= 1)
+                cmax[j] = fmaxf(cmax[j], __shfl_xor_sync(0xffffffffu, cmax[j], o));
+    } else {
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j)
+            if (l + 8 * j < kMaxChunks) cmax_smem[team][l + 8 * j] = cmax[j];
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) {
+            const int c = l + 8 * j;
+            if (c < nchunk) {
+                const int g0 = c / lpg * lpg;
+                float m = 0.f;
+                for (int u = g0; u < min(g0 + lpg, nchunk); ++u) m = fmaxf(m, cmax_smem[team][u]);
+                cmax[j] = m;
+            }
+        }
+    }
+    __syncwarp();
+
+    // scales and codes
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = l + 8 * j;
+        if (!(valid && c < nchunk)) continue;
+        float s = __fdiv_rn(cmax[j], 6.0f);
         uint32_t sbyte = 0;
         if (ue4m3) {
             sbyte = e4m3_from_f32(s);
             s = e4m3_to_f32(sbyte);
         }
-        if (active) {
-            float v[8];
+        float v[8];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const float q = s > 0.f ? __fdiv_rn(x[t], s) : 0.f;
-                v[t] = fminf(fmaxf(q, -6.f), 6.f);
-            }
-            *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
-            if (c % sh.lpg == 0) {
-                const int gi = c / sh.lpg;
-                if (ue4m3)
-                    tail[gi] = (uint8_t)sbyte;
-                else
-                    *reinterpret_cast<float*>(tail + 4 * gi) = s;
-            }
+        for (int t = 0; t < 8; ++t) {
+            float x = __fmaf_rn(w0, k0[j].get(t), __fmul_rn(w1, k1[j].get(t)));
+            if (!isfinite(x)) x = 0.f;
+            const float q = s > 0.f ? __fdiv_rn(x, s) : 0.f;
+            v[t] = fminf(fmaxf(q, -6.f), 6.f);
+        }
+        *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
+        if (c % lpg == 0) {
+            const int gi = c / lpg;
+            if (ue4m3)
+                tail[gi] = (uint8_t)sbyte;
+            else
+                *reinterpret_cast<float*>(tail + 4 * gi) = s;
         }
     }
     __syncwarp();
-    for (int t = lane * 4; t < tail_len; t += 128)
-        *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
-            *reinterpret_cast<const uint32_t*>(tail + t);
-
-    // indexer key append: Di bytes as 16-byte pieces, one per lane
-    if (lane < (di >> 4)) {
-        const uint4 v = __ldcs(
-            reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di) + lane);
-        *(reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di) + lane) = v;
+    if (valid) {
+        for (int t = l * 4; t < tail_len; t += 32)
+            *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
+                *reinterpret_cast<const uint32_t*>(tail + t);
+        // indexer key append: Di bytes as 16-byte pieces
+        const uint4* src =
+            reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di);
+        uint4* dst = reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di);
+        for (int p = l; p < (di >> 4); p += 8) dst[p] = __ldcs(src + p);
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
@@ -209,15 +250,17 @@ template <typename T>
 cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
                           cudaStream_t s) {
     const long long entries = (long long)a.batch * (a.n_new / 2);
-    const unsigned grid = (unsigned)((entries + kWarps - 1) / kWarps);
-    const int maxj = (sh.D / 8 + 31) / 32;
+    const unsigned grid = (unsigned)((entries + kTeams - 1) / kTeams);
+    const int maxj = (sh.D / 8 + 7) / 8;
     trace_before("pack", s);
-    switch (maxj) {
-        case 1: pack_kernel<T, 1><<<grid, kWarps * 32, 0, s>>>(a, sh, ue4m3, di); break;
-        case 2: pack_kernel<T, 2><<<grid, kWarps * 32, 0, s>>>(a, sh, ue4m3, di); break;
-        case 3: pack_kernel<T, 3><<<grid, kWarps * 32, 0, s>>>(a, sh, ue4m3, di); break;
-        default: pack_kernel<T, 4><<<grid, kWarps * 32, 0, s>>>(a, sh, ue4m3, di); break;
-    }
+    if (maxj <= 2)
+        pack_kernel<T, 2><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+    else if (maxj <= 4)
+        pack_kernel<T, 4><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+    else if (maxj <= 9)
+        pack_kernel<T, 9><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+    else
+        pack_kernel<T, 16><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
     trace_after(s);
     return cudaGetLastError();
 }

@@ -138,7 +138,8 @@ kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,
  *           visible score (positions past n_entries are not written).
  * ws        device workspace of at least kvc_workspace_bytes(cfg, batch,
  *           capacity) bytes, 256-byte aligned; its contents need no
- *           initialisation and are scratch after the call.               */
+ *           initialisation and are scratch after the call.
+ * capacity must not exceed 8,388,608 entries (KVC_ERR_CAPACITY).         */
 kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
                           const kvc_cache* cache, int32_t* topk_idx,
                           int32_t* scores, void* ws, size_t ws_bytes,
@@ -151,9 +152,9 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
  * pages have no counterpart of this call; it computes exactly what
  * kvc_index_topk computes (same kernels, same results).
  * Its scratch (scores, histograms, counters, candidate lists) is a fixed
- * array inside the library, about 6.5 MiB, held on every GPU that loads the
+ * array inside the library, about 8 MiB, held on every GPU that loads the
  * library until the process exits.  Limits: batch <= 64 and
- * batch * capacity <= 1,048,576 entries; larger problems return
+ * batch * capacity <= 524,288 entries; larger problems return
  * KVC_ERR_CAPACITY before anything is enqueued.  The call allocates nothing.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
@@ -216,7 +217,7 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * max_launches launches are recorded).  kvc_trace_kernel, called after the
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
- * "pack", "pack_commit", "index_scan", "topk_collect", "topk_finalize",
+ * "pack", "pack_commit", "index_scan", "topk_select", "attn_tc05",
  * "attn_mma", "attn_simt", "attn_merge", "fp4_codec".                      */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);

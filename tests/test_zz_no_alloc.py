@@ -67,7 +67,7 @@ def test_noalloc_heavy_ties_and_limits(kvc):
         assert torch.equal(tk, ref)
         assert torch.equal(tk[0], torch.arange(w.topk, dtype=torch.int32, device="cuda"))
     # beyond the fixed scratch: rejected before any work, with KVC_ERR_CAPACITY
-    big_cfg, big, _ = _cache(kvc, w.scaled(batch=1), [(1 << 20) + 16], seed=7)
+    big_cfg, big, _ = _cache(kvc, w.scaled(batch=1), [(1 << 19) + 16], seed=7)
     with pytest.raises(kvc.KvcError) as e:
         kvc.index_topk_noalloc(big_cfg, q, big, torch.empty(1, w.topk, dtype=torch.int32,
                                                              device="cuda"))
