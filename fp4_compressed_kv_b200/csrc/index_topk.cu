@@ -9,7 +9,8 @@
 // indices in ascending order, padded with -1.
 //
 // Design (B200): the scan is a pure HBM stream of 128-byte int8 rows.
-//  1. index_scan: a grid of CTAs tiles every sequence's visible entries;
+//  1. index_scan: one wave of CTAs (4 per SM) splits the batch's rows into
+//     equal contiguous slices (a slice may span two sequences);
 //     Di/16 lanes share a row, each loading 16 bytes (coalesced 512-byte warp
 //     loads, 8 rows in flight per lane), dp4a + xor-shuffle reduce to the
 //     score.  Each score is stored (4 bytes beside the 128 read) and counted
@@ -96,27 +97,14 @@ __device__ void find_threshold(const int* s_hist, int K, int* t_out, int* above_
     __syncthreads();
 }
 
+// Scans rows [start, end) of sequence b into the shared histogram and the
+// score array (the histogram must be zero on entry).
 template <int DI>
-__global__ void __launch_bounds__(kThreads)
-index_scan_kernel(TopkArgs a, int tile, int bias, int shift) {
-    __shared__ __align__(16) int hist[kBins];
-    __shared__ int sh_warp[kThreads / 32];
-    __shared__ int s_last, s_t, s_above;
+__device__ __forceinline__ void scan_rows(const TopkArgs& a, int b, int start, int end, int bias,
+                                          int shift, int* hist) {
     constexpr int TPR = DI / 16;   // lanes per row
     constexpr int RPW = 32 / TPR;  // rows per warp step
     constexpr int UNROLL = 8;
-    const int b = blockIdx.y;
-    const int n = a.n_entries[b];
-    if (n < 0 || n > a.capacity) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, KVC_DEV_BAD_LENGTH);
-        return;
-    }
-    const int start = blockIdx.x * tile;
-    if (start >= n) return;
-    const int end = min(start + tile, n);
-    for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
-    __syncthreads();
-
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane % TPR, rloc = lane / TPR;
     const int4 qv = __ldg(reinterpret_cast<const int4*>(a.idx_q + (size_t)b * DI) + sub);
@@ -148,29 +136,60 @@ index_scan_kernel(TopkArgs a, int tile, int bias, int shift) {
             }
         }
     }
-    __syncthreads();
-    int32_t* gh = a.counters + (size_t)b * kBins;
-    for (int i = threadIdx.x; i < kBins; i += kThreads)
-        if (hist[i]) atomicAdd(&gh[i], hist[i]);
-    if (n <= a.topk) return;  // everything is selected; no threshold needed
+}
 
-    // the last scan CTA of this sequence derives the threshold
-    __threadfence();
-    __syncthreads();
-    const int nctas = (n + tile - 1) / tile;
-    if (threadIdx.x == 0)
-        s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) == nctas - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int i = threadIdx.x * 4; i < kBins; i += kThreads * 4)
-        *reinterpret_cast<int4*>(hist + i) = __ldcg(reinterpret_cast<const int4*>(gh + i));
-    if (threadIdx.x == 0) s_t = s_above = 0;
-    __syncthreads();
-    find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
-    if (threadIdx.x == 0) {
-        a.thr[2 * b] = s_t;
-        a.thr[2 * b + 1] = s_above;
+// Grid of exactly (CTAs per SM x SMs) CTAs; CTA c scans the rows
+// [c*per, (c+1)*per) of the batch laid end to end (sequence b owns rows
+// [b*capacity, b*capacity + n_entries[b])), so every CTA streams the same
+// number of bytes whatever the lengths, in one wave.
+template <int DI>
+__global__ void __launch_bounds__(kThreads, 4)
+index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
+    __shared__ __align__(16) int hist[kBins];
+    __shared__ int sh_warp[kThreads / 32];
+    __shared__ int s_last, s_t, s_above;
+    const long long cap = a.capacity;
+    const long long lo = (long long)blockIdx.x * per;
+    const long long hi = min(lo + per, (long long)a.batch * cap);
+    if (lo >= hi) return;
+    for (int b = (int)(lo / cap); b <= (int)((hi - 1) / cap); ++b) {
+        const int n = a.n_entries[b];
+        if (n < 0 || n > a.capacity) {
+            if (threadIdx.x == 0) set_status(a.status, KVC_DEV_BAD_LENGTH);
+            continue;
+        }
+        const long long base = (long long)b * cap;
+        const int start = (int)(max(lo, base) - base);
+        const int end = (int)min(min(hi, base + cap) - base, (long long)n);
+        if (start >= end) continue;  // this CTA holds none of b's visible rows
+        __syncthreads();
+        for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
+        __syncthreads();
+        scan_rows<DI>(a, b, start, end, bias, shift, hist);
+        __syncthreads();
+        int32_t* gh = a.counters + (size_t)b * kBins;
+        for (int i = threadIdx.x; i < kBins; i += kThreads)
+            if (hist[i]) atomicAdd(&gh[i], hist[i]);
+        if (n <= a.topk) continue;  // everything is selected; no threshold needed
+        // the last CTA holding rows of b derives b's threshold
+        const long long first = base / per, last = (base + n - 1) / per;
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) ==
+                     (int)(last - first);
+        __syncthreads();
+        if (!s_last) continue;
+        __threadfence();
+        for (int i = threadIdx.x * 4; i < kBins; i += kThreads * 4)
+            *reinterpret_cast<int4*>(hist + i) = __ldcg(reinterpret_cast<const int4*>(gh + i));
+        if (threadIdx.x == 0) s_t = s_above = 0;
+        __syncthreads();
+        find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
+        if (threadIdx.x == 0) {
+            a.thr[2 * b] = s_t;
+            a.thr[2 * b + 1] = s_above;
+        }
     }
 }
 
@@ -371,9 +390,9 @@ topk_select_kernel(TopkArgs a, int bias, int shift) {
 }
 
 template <int DI>
-cudaError_t launch_scan(const TopkArgs& a, int tile, int bias, int shift, cudaStream_t s) {
-    dim3 grid((a.capacity + tile - 1) / tile, a.batch);
-    index_scan_kernel<DI><<<grid, kThreads, 0, s>>>(a, tile, bias, shift);
+cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, int shift,
+                        cudaStream_t s) {
+    index_scan_kernel<DI><<<ctas, kThreads, 0, s>>>(a, per, bias, shift);
     return cudaGetLastError();
 }
 
@@ -386,25 +405,27 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     cudaError_t err =
         cudaMemsetAsync(a.counters, 0, topk_counter_words(a.batch) * sizeof(int32_t), s);
     if (err != cudaSuccess) return err;
-    // scan tile: aim for about 4 CTAs per SM over the whole batch
+    // one wave: 4 CTAs per SM (64 registers x 256 threads), equal row slices
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long rows = (long long)a.batch * a.capacity;
-    long long tile = (rows + 4 * 148 - 1) / (4 * 148);
-    tile = (tile + 255) / 256 * 256;
-    if (tile < 256) tile = 256;
-    if (tile > 16384) tile = 16384;
+    int ctas = 4 * sms;
+    long long per = (rows + ctas - 1) / ctas;
+    per = (per + 255) / 256 * 256;
+    if (per < 256) per = 256;
+    ctas = (int)((rows + per - 1) / per);
     trace_before("index_scan", s);
     switch (a.di) {
-        case 16: err = launch_scan<16>(a, (int)tile, bias, shift, s); break;
-        case 32: err = launch_scan<32>(a, (int)tile, bias, shift, s); break;
-        case 64: err = launch_scan<64>(a, (int)tile, bias, shift, s); break;
-        case 128: err = launch_scan<128>(a, (int)tile, bias, shift, s); break;
-        default: err = launch_scan<256>(a, (int)tile, bias, shift, s); break;
+        case 16: err = launch_scan<16>(a, ctas, per, bias, shift, s); break;
+        case 32: err = launch_scan<32>(a, ctas, per, bias, shift, s); break;
+        case 64: err = launch_scan<64>(a, ctas, per, bias, shift, s); break;
+        case 128: err = launch_scan<128>(a, ctas, per, bias, shift, s); break;
+        default: err = launch_scan<256>(a, ctas, per, bias, shift, s); break;
     }
     trace_after(s);
     if (err != cudaSuccess) return err;
     static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         err = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kSelSmem);

@@ -239,6 +239,119 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
 
+// Small appends (decode: one pair per sequence): one warp per entry so the
+// work of a few dozen entries spreads over many SMs.  Lanes 0-7 form the gate
+// team in exactly the order above (lane l sums chunks l, l+8, ... then the
+// xor tree over 4, 2, 1 inside the team); all 32 lanes then quantise, lane l
+// owning chunks l, l+32, l+64.  Same arithmetic, same bits as pack_kernel.
+constexpr int kSmallWarps = 4;
+
+template <typename T, int MAXJ>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
+    __shared__ __align__(16) uint8_t tail_smem[kSmallWarps][kTailBytes];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const long long e = (long long)blockIdx.x * kSmallWarps + wid;
+    const int half = a.n_new >> 1;
+    if (e >= (long long)a.batch * half) return;  // whole warp
+    const int b = (int)(e / half), i = (int)(e % half);
+    const int base = a.n_entries[b];
+    if (base < 0 || base + half > a.capacity) {
+        if (i == 0 && lane == 0) set_status(a.status, KVC_DEV_CAPACITY);
+        return;
+    }
+    const int D = sh.D, nchunk = D >> 3;
+    const long long pos = (long long)base + i;
+    const T* k0p = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 2 * i) * D;
+    const T* k1p = k0p + D;
+
+    float acc = 0.f;
+    if (lane < 8) {
+        for (int c = lane; c < nchunk; c += 8) {
+            Chunk<T> x0, x1;
+            x0.load(k0p + 8 * c);
+            x1.load(k1p + 8 * c);
+            float g[8];
+            load8_gate(a.gate + 8 * c, g);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                acc = __fmaf_rn(g[t], __fsub_rn(x0.get(t), x1.get(t)), acc);
+        }
+    }
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
+    const float delta = __shfl_sync(0xffffffffu, acc, 0);
+    const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-delta)));
+    const float w1 = __fsub_rn(1.0f, w0);
+
+    uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
+    uint8_t* tail = tail_smem[wid];
+    const int tail_len = sh.rb - sh.code_bytes;
+    for (int t = lane * 4; t < tail_len; t += 128) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
+    __syncwarp();
+
+    bool bad = false;
+    const int lpg = sh.lpg;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        const bool active = c < nchunk;
+        Chunk<T> x0, x1;
+        if (active) {
+            x0.load(k0p + 8 * c);
+            x1.load(k1p + 8 * c);
+        } else {
+            x0.zero();
+            x1.zero();
+        }
+        float x[8];
+        float m = 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float v = __fmaf_rn(w0, x0.get(t), __fmul_rn(w1, x1.get(t)));
+            if (!isfinite(v)) {
+                if (active) bad = true;
+                v = 0.f;
+            }
+            x[t] = v;
+            m = fmaxf(m, fabsf(v));
+        }
+        for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (!active) continue;
+        float s = __fdiv_rn(m, 6.0f);
+        uint32_t sbyte = 0;
+        if (ue4m3) {
+            sbyte = e4m3_from_f32(s);
+            s = e4m3_to_f32(sbyte);
+        }
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const float q = s > 0.f ? __fdiv_rn(x[t], s) : 0.f;
+            v[t] = fminf(fmaxf(q, -6.f), 6.f);
+        }
+        *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
+        if (c % lpg == 0) {
+            const int gi = c / lpg;
+            if (ue4m3)
+                tail[gi] = (uint8_t)sbyte;
+            else
+                *reinterpret_cast<float*>(tail + 4 * gi) = s;
+        }
+    }
+    __syncwarp();
+    for (int t = lane * 4; t < tail_len; t += 128)
+        *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
+            *reinterpret_cast<const uint32_t*>(tail + t);
+    if (lane < (di >> 4)) {
+        const uint4 v = __ldcs(
+            reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di) + lane);
+        *(reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di) + lane) = v;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
+}
+
 __global__ void pack_commit_kernel(int32_t* n_entries, int batch, int half, int capacity) {
     for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
         const int n = n_entries[b];
@@ -250,6 +363,21 @@ template <typename T>
 cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
                           cudaStream_t s) {
     const long long entries = (long long)a.batch * (a.n_new / 2);
+    if (entries <= 4096) {  // latency-bound append: a warp per entry
+        const unsigned grid = (unsigned)((entries + kSmallWarps - 1) / kSmallWarps);
+        const int maxj = (sh.D / 8 + 31) / 32;
+        trace_before("pack", s);
+        if (maxj <= 1)
+            pack_small_kernel<T, 1><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+        else if (maxj <= 2)
+            pack_small_kernel<T, 2><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+        else if (maxj <= 3)
+            pack_small_kernel<T, 3><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+        else
+            pack_small_kernel<T, 4><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+        trace_after(s);
+        return cudaGetLastError();
+    }
     const unsigned grid = (unsigned)((entries + kTeams - 1) / kTeams);
     const int maxj = (sh.D / 8 + 7) / 8;
     trace_before("pack", s);

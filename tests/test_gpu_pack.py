@@ -105,3 +105,20 @@ def test_codecs_match_oracle(kvc):
     kvc.e4m3_encode(torch.from_numpy(ys).cuda(), out)
     want = np.array([oracle.e4m3_encode(float(y)) for y in ys])
     assert np.array_equal(out.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("name,batch,context", [("batch32x128k", 2, 2 * 4200),
+                                                 ("mla32k", 1, 2 * 300)])
+def test_pack_team_and_warp_variants(kvc, name, batch, context):
+    """Large appends take the 8-lanes-per-entry kernel, small ones the
+    warp-per-entry kernel; both must give the oracle's bytes."""
+    w = synth.WORKLOADS[name].scaled(batch=batch, context=context)
+    inp = synth.make_inputs(w)
+    rec, ic, n, _ = oracle_pack(w, inp["tokens"], inp["gate"], inp["idx_k"])
+    cache, st = _gpu_pack(kvc, w, inp["tokens"].cuda(), inp["gate"].cuda(), inp["idx_k"].cuda())
+    assert st == 0 and cache.n_entries.cpu().tolist() == n.tolist()
+    assert np.array_equal(cache.records.cpu().numpy(), rec)
+    # one pair at a time (the decode append) gives the same bytes as one append
+    cache2, _ = _gpu_pack(kvc, w, inp["tokens"][:, :64].cuda().contiguous(), inp["gate"].cuda(),
+                          inp["idx_k"][:, :32].cuda().contiguous(), capacity=w.entries, chunks=2)
+    assert np.array_equal(cache2.records.cpu().numpy()[:, :32], rec[:, :32])
