@@ -10,13 +10,8 @@
 // softmax runs jointly over the selected entries and the window keys.
 //
 // Kernels
-//  attn_mma   bf16 path for 64 heads x 576 (512 latent) entries.  A CTA owns a
-//             contiguous range of 64-key chunks of one sequence.  Per chunk the
-//             selected records (16-byte aligned rows) and window rows are
-//             gathered into shared memory with cp.async, records are
-//             dequantised in registers to bf16 (exact for UE4M3 scales), then
-//             S = Q K^T and O += P V run on the tensor cores with fp32
-//             accumulation and an online softmax in the log2 domain.
+//  attn_tc05  (attn_tc05.cu) tensor-core path for 64 heads x 576 (512 latent)
+//             bf16 entries.
 //  attn_simt  generic fp32 / bf16 path for other shapes (one warp per head).
 //  attn_merge combines the per-split (max, sum, O) partials by log-sum-exp.
 #include "kvc_internal.cuh"
@@ -214,288 +209,6 @@ attn_merge_kernel(AttnArgs a, int H, int Dv, int nsplit) {
     if (tid == 0 && a.lse) a.lse[(size_t)b * H + h] = s_lse;
 }
 
-// ----------------------------------------------------------------------------
-// tensor-core path (bf16, 64 heads, 576-channel entries, 512-channel values)
-namespace tc {
-constexpr int H = 64, D = 576, DV = 512, CK = kChunk;
-constexpr int QS = D + 8;    // shared row stride in elements (1168 B: ldmatrix conflict-free)
-constexpr int PS = CK + 8;   // 144 B
-constexpr int RAW = 384;     // bytes reserved per gathered record
-constexpr int kThreadsTC = 256;
-constexpr size_t kOffQ = 0;
-constexpr size_t kOffK = kOffQ + (size_t)H * QS * 2;
-constexpr size_t kOffP = kOffK + (size_t)CK * QS * 2;
-constexpr size_t kOffRaw = kOffP + (size_t)H * PS * 2;
-constexpr size_t kOffKind = kOffRaw + (size_t)CK * RAW;
-constexpr size_t kOffMax = kOffKind + CK * 4;
-constexpr size_t kOffSum = kOffMax + 2 * H * 4;
-constexpr size_t kSmem = kOffSum + 2 * H * 4;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;\n" ::: "memory");
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
-        "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-__global__ void __launch_bounds__(kThreadsTC, 1)
-attn_mma_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int chunks_per_split,
-                int nsplit, int ue4m3) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + kOffQ);
-    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + kOffK);
-    __nv_bfloat16* sP = reinterpret_cast<__nv_bfloat16*>(smem + kOffP);
-    unsigned char* sRaw = smem + kOffRaw;
-    int* sKind = reinterpret_cast<int*>(smem + kOffKind);
-    float* sMax = reinterpret_cast<float*>(smem + kOffMax);
-    float* sSum = reinterpret_cast<float*>(smem + kOffSum);
-
-    const int b = blockIdx.y, split = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int hg = warp & 3, kh = warp >> 2;  // head group (16 rows); key half / value half
-    const int n = a.n_entries[b];
-    const bool len_ok = n >= 0 && n <= a.capacity;
-    const int total = K + a.window_len;
-    const int c0 = split * chunks_per_split;
-    const int c1 = min(c0 + chunks_per_split, (total + CK - 1) / CK);
-    const int rb = sh.rb, pieces = rb >> 4;
-
-    // Q: 64 rows x 72 16-byte pieces
-    {
-        const unsigned char* qg =
-            static_cast<const unsigned char*>(a.q) + (size_t)b * H * D * 2;
-        for (int p = tid; p < H * (D / 8); p += kThreadsTC) {
-            const int r = p / (D / 8), c = p - r * (D / 8);
-            cp_async16(smem_u32(sQ + r * QS + c * 8), qg + (size_t)r * D * 2 + c * 16);
-        }
-    }
-
-    float o[32][4];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-    const int r0 = hg * 16 + (lane >> 2);  // rows r0 and r0 + 8
-
-    const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), p_base = smem_u32(sP);
-
-    for (int c = c0; c < c1; ++c) {
-        if (tid < CK) {
-            const int j = c * CK + tid;
-            sKind[tid] = (j < total && len_ok) ? slot_kind(a, b, j, K, n) : -1;
-        }
-        __syncthreads();
-        // gather records into sRaw, window rows straight into sK, zero empty rows
-        for (int p = tid; p < CK * pieces; p += kThreadsTC) {
-            const int s = p / pieces, pc = p - s * pieces;
-            const int k = sKind[s];
-            if (k >= 0)
-                cp_async16(smem_u32(sRaw + s * RAW + pc * 16),
-                           a.records + ((size_t)b * a.capacity + k) * rb + pc * 16);
-        }
-        for (int p = tid; p < CK * (D / 8); p += kThreadsTC) {
-            const int s = p / (D / 8), pc = p - s * (D / 8);
-            const int k = sKind[s];
-            if (k <= -2) {
-                const int t = -2 - k;
-                cp_async16(smem_u32(sK + s * QS + pc * 8),
-                           static_cast<const unsigned char*>(a.window) +
-                               (((size_t)b * a.window_stride + t) * D) * 2 + pc * 16);
-            } else if (k == -1) {
-                *reinterpret_cast<uint4*>(sK + s * QS + pc * 8) = make_uint4(0, 0, 0, 0);
-            }
-        }
-        cp_async_wait_all();
-        __syncthreads();
-        // dequantise records: (slot, 8-channel chunk) per item
-        for (int p = tid; p < CK * (D / 8); p += kThreadsTC) {
-            const int s = p / (D / 8), pc = p - s * (D / 8);
-            if (sKind[s] < 0) continue;
-            const unsigned char* rec = sRaw + s * RAW;
-            const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + pc * 4);
-            const int g = pc / sh.lpg;
-            const float sc = ue4m3 ? e4m3_to_f32(rec[sh.code_bytes + g])
-                                   : reinterpret_cast<const float*>(rec + sh.code_bytes)[g];
-            uint4 v;
-            v.x = pack_bf16(e2m1_value(codes & 15u) * sc, e2m1_value((codes >> 4) & 15u) * sc);
-            v.y = pack_bf16(e2m1_value((codes >> 8) & 15u) * sc, e2m1_value((codes >> 12) & 15u) * sc);
-            v.z = pack_bf16(e2m1_value((codes >> 16) & 15u) * sc, e2m1_value((codes >> 20) & 15u) * sc);
-            v.w = pack_bf16(e2m1_value((codes >> 24) & 15u) * sc, e2m1_value(codes >> 28) * sc);
-            *reinterpret_cast<uint4*>(sK + s * QS + pc * 8) = v;
-        }
-        __syncthreads();
-
-        // S[16 rows of group hg][32 keys of half kh] = Q K^T
-        float sacc[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
-#pragma unroll 4
-        for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t af[4];
-            ldsm_x4(af, q_base + ((hg * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * QS + ks * 16 +
-                                  (lane >> 4) * 8) * 2);
-#pragma unroll
-            for (int pr = 0; pr < 2; ++pr) {
-                uint32_t bf[4];
-                const int key0 = kh * 32 + pr * 16;
-                ldsm_x4(bf, k_base + ((key0 + (lane & 7) + (lane >> 4) * 8) * QS + ks * 16 +
-                                      ((lane >> 3) & 1) * 8) * 2);
-                mma16816(sacc[2 * pr], af, bf[0], bf[1]);
-                mma16816(sacc[2 * pr + 1], af, bf[2], bf[3]);
-            }
-        }
-        // scale, mask, chunk row max
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = kh * 32 + nt * 8 + 2 * (lane & 3) + (e & 1);
-                float x = sacc[nt][e] * scale_log2;
-                if (sKind[key] == -1) x = -INFINITY;
-                sacc[nt][e] = x;
-                mx[e >> 1] = fmaxf(mx[e >> 1], x);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
-        }
-        if ((lane & 3) == 0) {
-            sMax[kh * H + r0] = mx[0];
-            sMax[kh * H + r0 + 8] = mx[1];
-        }
-        __syncthreads();
-        float alpha[2], mnew[2], rs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = r0 + 8 * i;
-            const float mc = fmaxf(sMax[r], sMax[H + r]);
-            mnew[i] = fmaxf(m_run[i], mc);
-            alpha[i] = mnew[i] == -INFINITY ? 1.f : exp2f(m_run[i] - mnew[i]);
-        }
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            float p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float mm = mnew[e >> 1];
-                p[e] = mm == -INFINITY ? 0.f : exp2f(sacc[nt][e] - mm);
-                rs[e >> 1] += p[e];
-            }
-            const int col = kh * 32 + nt * 8 + 2 * (lane & 3);
-            *reinterpret_cast<uint32_t*>(sP + r0 * PS + col) = pack_bf16(p[0], p[1]);
-            *reinterpret_cast<uint32_t*>(sP + (r0 + 8) * PS + col) = pack_bf16(p[2], p[3]);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            rs[i] += __shfl_xor_sync(0xffffffffu, rs[i], 1);
-            rs[i] += __shfl_xor_sync(0xffffffffu, rs[i], 2);
-        }
-        if ((lane & 3) == 0) {
-            sSum[kh * H + r0] = rs[0];
-            sSum[kh * H + r0 + 8] = rs[1];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = r0 + 8 * i;
-            l_run[i] = l_run[i] * alpha[i] + sSum[r] + sSum[H + r];
-            m_run[i] = mnew[i];
-        }
-        // O[16 rows][256 values of half kh] = O * alpha + P V
-#pragma unroll
-        for (int nt = 0; nt < 32; ++nt) {
-            o[nt][0] *= alpha[0];
-            o[nt][1] *= alpha[0];
-            o[nt][2] *= alpha[1];
-            o[nt][3] *= alpha[1];
-        }
-#pragma unroll
-        for (int kk = 0; kk < CK / 16; ++kk) {
-            uint32_t af[4];
-            ldsm_x4(af, p_base + ((hg * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * PS + kk * 16 +
-                                  (lane >> 4) * 8) * 2);
-#pragma unroll
-            for (int np = 0; np < 16; ++np) {
-                uint32_t bf[4];
-                const int col0 = kh * 256 + np * 16;
-                ldsm_x4_t(bf, k_base + ((kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * QS + col0 +
-                                        (lane >> 4) * 8) * 2);
-                mma16816(o[2 * np], af, bf[0], bf[1]);
-                mma16816(o[2 * np + 1], af, bf[2], bf[3]);
-            }
-        }
-        __syncthreads();
-    }
-    cp_async_wait_all();  // a split without chunks still drains the Q copies
-
-    // epilogue
-    const int h0 = r0, h1 = r0 + 8;
-    if (nsplit == 1) {
-        const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
-        const float inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 32; ++nt) {
-            const int col = kh * 256 + nt * 8 + 2 * (lane & 3);
-            *reinterpret_cast<float2*>(a.out + ((size_t)b * H + h0) * DV + col) =
-                make_float2(o[nt][0] * inv0, o[nt][1] * inv0);
-            *reinterpret_cast<float2*>(a.out + ((size_t)b * H + h1) * DV + col) =
-                make_float2(o[nt][2] * inv1, o[nt][3] * inv1);
-        }
-        if (kh == 0 && (lane & 3) == 0 && a.lse) {
-            a.lse[(size_t)b * H + h0] = l_run[0] > 0.f ? (m_run[0] + __log2f(l_run[0])) * kLn2 : -INFINITY;
-            a.lse[(size_t)b * H + h1] = l_run[1] > 0.f ? (m_run[1] + __log2f(l_run[1])) * kLn2 : -INFINITY;
-        }
-    } else {
-        const size_t row0 = ((size_t)b * H + h0) * kMaxSplit + split;
-        const size_t row1 = ((size_t)b * H + h1) * kMaxSplit + split;
-#pragma unroll
-        for (int nt = 0; nt < 32; ++nt) {
-            const int col = kh * 256 + nt * 8 + 2 * (lane & 3);
-            *reinterpret_cast<float2*>(a.part_o + row0 * DV + col) = make_float2(o[nt][0], o[nt][1]);
-            *reinterpret_cast<float2*>(a.part_o + row1 * DV + col) = make_float2(o[nt][2], o[nt][3]);
-        }
-        if (kh == 0 && (lane & 3) == 0) {
-            a.part_ml[row0 * 2] = m_run[0];
-            a.part_ml[row0 * 2 + 1] = l_run[0];
-            a.part_ml[row1 * 2] = m_run[1];
-            a.part_ml[row1 * 2 + 1] = l_run[1];
-        }
-    }
-}
-}  // namespace tc
-
-bool tc_supported(const kvc_config& c, const Shape& sh) {
-    return c.act_dtype == KVC_BF16 && c.n_heads == tc::H && sh.D == tc::D && sh.Dv == tc::DV &&
-           sh.rb <= tc::RAW;
-}
-
 }  // namespace
 
 bool tc05_supported(const kvc_config& c, const Shape& sh);
@@ -517,25 +230,6 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
     if (tc05_supported(c, sh)) {
         nsplit = launch_attention_tc05(c, sh, a, s);
         if (nsplit < 0) return cudaErrorLaunchFailure;
-    } else if (tc_supported(c, sh)) {
-        const int nchunks = (total + tc::CK - 1) / tc::CK;
-        int want = sms / a.batch;
-        if (want < 1) want = 1;
-        if (want > kMaxSplit) want = kMaxSplit;
-        if (want > nchunks) want = nchunks;
-        const int cps = nchunks == 0 ? 1 : (nchunks + want - 1) / want;
-        nsplit = nchunks == 0 ? 1 : (nchunks + cps - 1) / cps;
-        static bool attr_set[64] = {};
-        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-            err = cudaFuncSetAttribute(tc::attn_mma_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmem);
-            if (err != cudaSuccess) return err;
-            attr_set[dev] = true;
-        }
-        trace_before("attn_mma", s);
-        tc::attn_mma_kernel<<<dim3(nsplit, a.batch), tc::kThreadsTC, tc::kSmem, s>>>(
-            a, sh, K, scale_log2, cps, nsplit, ue4m3);
-        trace_after(s);
     } else {
         const int nchunks = (total + kSimtChunk - 1) / kSimtChunk;
         const int hblocks = (c.n_heads + 7) / 8;
@@ -555,6 +249,10 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
                      : cudaFuncSetAttribute(attn_simt_kernel<float>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             kSimtChunk * 1024 * 4);
+            if (err == cudaSuccess)
+                err = ti ? prefer_shared(attn_simt_kernel<__nv_bfloat16>)
+                         : prefer_shared(attn_simt_kernel<float>);
+            if (err == cudaSuccess) err = prefer_shared(attn_merge_kernel);
             if (err != cudaSuccess) return err;
             attr_set2[dev][ti] = true;
         }

@@ -288,7 +288,9 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         }
         mma_commit(smem_u32(&bars[0]));
     }
-    bool ok = __syncthreads_and(mbar_wait(smem_u32(&bars[0]), 0)) != 0;
+    // warp 0 polls the barrier; the other warps wait in the block barrier
+    bool ok = warp == 0 ? mbar_wait(smem_u32(&bars[0]), 0) : true;
+    ok = __syncthreads_and(ok) != 0;
     tc_fence_after();
 
     // ---- 4. softmax: warps 0-1, one thread per head row of S
@@ -341,8 +343,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                          kk > 0);
         mma_commit(smem_u32(&bars[1]));
     }
-    bool ok2 = false;
-    if (ok) ok2 = mbar_wait(smem_u32(&bars[1]), 0);
+    bool ok2 = ok;
+    if (ok && warp == 0) ok2 = mbar_wait(smem_u32(&bars[1]), 0);
     const bool ok_s = ok;
     ok = __syncthreads_and(ok2) != 0;
     tc_fence_after();
@@ -419,7 +421,8 @@ int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& 
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(tc05::attn_tc05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc05::SMEM_BYTES) != cudaSuccess)
+                                 (int)tc05::SMEM_BYTES) != cudaSuccess ||
+            prefer_shared(tc05::attn_tc05_kernel) != cudaSuccess)
             return -1;
         attr_set[dev] = true;
     }

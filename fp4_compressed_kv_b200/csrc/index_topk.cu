@@ -9,26 +9,28 @@
 // indices in ascending order, padded with -1.
 //
 // Design (B200): the scan is a pure HBM stream of 128-byte int8 rows.
-//  1. index_scan: one wave of CTAs (4 per SM) splits the batch's rows into
-//     equal contiguous slices (a slice may span two sequences);
-//     Di/16 lanes share a row, each loading 16 bytes (coalesced 512-byte warp
-//     loads, 8 rows in flight per lane), dp4a + xor-shuffle reduce to the
+//  1. index_scan: one wave of CTAs (2 per SM) splits the batch's rows into
+//     equal contiguous slices (a slice may span two sequences).  Thread 0 of
+//     each CTA streams blocks of 256 rows into a 3-stage shared-memory ring
+//     with bulk copies (mbarrier byte counts); each thread takes one row's
+//     dot product (lane-rotated 16-byte reads, 4 dp4a accumulators) to the
 //     score.  Each score is stored (4 bytes beside the 128 read) and counted
 //     in a 2048-bin shared-memory histogram of its biased value; the CTA adds
 //     its non-zero bins to the sequence's histogram.  The last scan CTA of a
 //     sequence (a fenced counter; nobody waits) derives the threshold bin t
 //     (the highest bin whose suffix count reaches K) and the count above it.
-//  2. topk_select: a CTA per tile of 2,048 scores compacts the (score, index)
-//     keys of its entries in bins >= t, in index order, into the tile's own
-//     slot (block prefix sum; typically a few dozen per tile).  The last CTA
-//     of a sequence to finish completes the selection without sorting the
-//     output: the r = K - above best keys of bin t (a bitonic sort of the few
-//     tie candidates) give the cut-off key k*, every candidate with key >= k*
-//     is selected, and a prefix sum over the tiles places the winners -- the
-//     tiles are in index order, so the output is too.  If more than kMaxTies
+//  2. topk_collect: a CTA per tile of 8,192 scores compacts the (score,
+//     index) keys of its entries in bins >= t, in index order, into the
+//     tile's own slot (block prefix sum).
+//  3. topk_finish: a CTA per sequence completes the selection without
+//     sorting the output: it stages every
+//     candidate key in shared memory in index order (one round of parallel
+//     loads), takes the r = K - above best keys of bin t (a bitonic sort of the
+//     few tie candidates) as the cut-off key k*, and a block prefix sum over
+//     the candidates with key >= k* places the winners in index order.  If more than kMaxTies
 //     entries share bin t, an exact slower path finds the threshold score and
 //     the index cut-off with a second histogram and compacts the scores.
-// No CTA waits on another: the two launches are stream-ordered.
+// No CTA waits on another: the launches are stream-ordered.
 #include "kvc_internal.cuh"
 
 namespace kvc {
@@ -97,99 +99,200 @@ __device__ void find_threshold(const int* s_hist, int K, int* t_out, int* above_
     __syncthreads();
 }
 
-// Scans rows [start, end) of sequence b into the shared histogram and the
-// score array (the histogram must be zero on entry).
-template <int DI>
-__device__ __forceinline__ void scan_rows(const TopkArgs& a, int b, int start, int end, int bias,
-                                          int shift, int* hist) {
-    constexpr int TPR = DI / 16;   // lanes per row
-    constexpr int RPW = 32 / TPR;  // rows per warp step
-    constexpr int UNROLL = 8;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int sub = lane % TPR, rloc = lane / TPR;
-    const int4 qv = __ldg(reinterpret_cast<const int4*>(a.idx_q + (size_t)b * DI) + sub);
-    const int8_t* kb = a.idx_k + (size_t)b * a.capacity * DI;
-    int32_t* sc = a.scores + (size_t)b * a.capacity;
-    constexpr int kStep = (kThreads / 32) * RPW;  // rows per CTA step
-    for (int r0 = start + warp * RPW; r0 < end; r0 += kStep * UNROLL) {
-        int4 kv[UNROLL];
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int row = r0 + u * kStep + rloc;
-            if (row < end)
-                kv[u] = __ldcs(reinterpret_cast<const int4*>(kb + (size_t)row * DI) + sub);
-            else
-                kv[u] = make_int4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            int s = __dp4a(kv[u].x, qv.x, 0);
-            s = __dp4a(kv[u].y, qv.y, s);
-            s = __dp4a(kv[u].z, qv.z, s);
-            s = __dp4a(kv[u].w, qv.w, s);
-#pragma unroll
-            for (int o = 1; o < TPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            const int row = r0 + u * kStep + rloc;
-            if (sub == 0 && row < end) {
-                sc[row] = s;
-                atomicAdd(&hist[score_bin(s, bias, shift)], 1);
-            }
-        }
+// ---- bulk-copy pipeline helpers (non-multicast bulk copies into this CTA's
+// own shared memory; every wait bounded by a 2-second clock)
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = now_ns();
+    for (uint32_t i = 0;; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if ((i & 255) == 255 && now_ns() - t0 > 2000000000ull) return false;
     }
 }
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
 
-// Grid of exactly (CTAs per SM x SMs) CTAs; CTA c scans the rows
-// [c*per, (c+1)*per) of the batch laid end to end (sequence b owns rows
-// [b*capacity, b*capacity + n_entries[b])), so every CTA streams the same
-// number of bytes whatever the lengths, in one wave.
+// Cursor over this CTA's rows, chunked per sequence: rows [row, end) of
+// sequence b are visible; chunks hold at most `rows` rows.
+struct ScanCursor {
+    int b, row, end;
+};
+__device__ __forceinline__ bool cursor_seek(const TopkArgs& a, long long lo, long long hi,
+                                            ScanCursor& c, int b_from) {
+    const long long cap = a.capacity;
+    for (int b = b_from; b <= (int)((hi - 1) / cap); ++b) {
+        const int n = a.n_entries[b];
+        if (n < 0 || n > a.capacity) continue;
+        const long long base = (long long)b * cap;
+        const int start = (int)(max(lo, base) - base);
+        const int end = (int)min(min(hi, base + cap) - base, (long long)n);
+        if (start < end) {
+            c.b = b;
+            c.row = start;
+            c.end = end;
+            return true;
+        }
+    }
+    return false;
+}
+
+constexpr int kScanStages = 3;
+constexpr int kStageRows = kThreads;  // one row per thread per stage
+
+// Grid of (2 CTAs per SM x SMs) CTAs; CTA c scans the rows [c*per, (c+1)*per)
+// of the batch laid end to end (sequence b owns rows [b*capacity,
+// b*capacity + n_entries[b])), so every CTA streams the same number of bytes
+// whatever the lengths.  Thread 0 keeps kScanStages blocks of 256 rows in
+// flight with bulk copies into a shared-memory ring; each thread then takes
+// the dot product of one row, reading its 16-byte pieces in a lane-rotated
+// order so that a warp's reads spread over all banks.
 template <int DI>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, 2)
 index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
+    extern __shared__ __align__(128) unsigned char ring[];  // kScanStages x 256 rows
     __shared__ __align__(16) int hist[kBins];
+    __shared__ __align__(16) int4 qs[DI / 16];
+    __shared__ __align__(8) uint64_t full[kScanStages];
     __shared__ int sh_warp[kThreads / 32];
     __shared__ int s_last, s_t, s_above;
+    constexpr int PIECES = DI / 16;               // 16-byte pieces per row
+    constexpr int STAGE = kStageRows * DI;        // bytes per stage
+    const int tid = threadIdx.x;
     const long long cap = a.capacity;
     const long long lo = (long long)blockIdx.x * per;
     const long long hi = min(lo + per, (long long)a.batch * cap);
     if (lo >= hi) return;
-    for (int b = (int)(lo / cap); b <= (int)((hi - 1) / cap); ++b) {
+    // flag invalid lengths once (the cursor skips those sequences)
+    if (tid == 0)
+        for (int b = (int)(lo / cap); b <= (int)((hi - 1) / cap); ++b) {
+            const int n = a.n_entries[b];
+            if (n < 0 || n > a.capacity) set_status(a.status, KVC_DEV_BAD_LENGTH);
+        }
+    ScanCursor cc;  // consumer cursor (all threads)
+    if (!cursor_seek(a, lo, hi, cc, (int)(lo / cap))) return;
+    if (tid == 0) {
+        for (int s = 0; s < kScanStages; ++s)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
+    if (tid < PIECES) qs[tid] = __ldg(reinterpret_cast<const int4*>(a.idx_q + (size_t)cc.b * DI) + tid);
+    __syncthreads();
+    // producer (thread 0): issue the first kScanStages chunks
+    ScanCursor pc = cc;
+    bool pmore = true;
+    if (tid == 0) {
+        for (int s = 0; s < kScanStages && pmore; ++s) {
+            const int rows = min(kStageRows, pc.end - pc.row);
+            bulk_load(smem_addr(ring + s * STAGE),
+                      a.idx_k + ((size_t)pc.b * cap + pc.row) * DI, (uint32_t)rows * DI,
+                      smem_addr(&full[s]));
+            pc.row += rows;
+            if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
+        }
+    }
+    uint32_t phase = 0;  // bit s = parity to wait for on stage s
+    bool ok = true;
+    for (int chunk = 0;; ++chunk) {
+        const int s = chunk % kScanStages;
+        const int rows = min(kStageRows, cc.end - cc.row);
+        bool got = (tid >> 5) == 0 ? bar_wait(smem_addr(&full[s]), (phase >> s) & 1u) : true;
+        if (__syncthreads_and(got) == 0) {
+            ok = false;
+            break;
+        }
+        phase ^= 1u << s;
+        if (tid < rows) {
+            const unsigned char* row = ring + s * STAGE + tid * DI;
+            int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int c = 0; c < PIECES; ++c) {
+                const int p = (c + tid) % PIECES;
+                const int4 kv = *reinterpret_cast<const int4*>(row + p * 16);
+                const int4 q = qs[p];
+                acc[c & 3] = __dp4a(kv.x, q.x, acc[c & 3]);
+                acc[c & 3] = __dp4a(kv.y, q.y, acc[c & 3]);
+                acc[c & 3] = __dp4a(kv.z, q.z, acc[c & 3]);
+                acc[c & 3] = __dp4a(kv.w, q.w, acc[c & 3]);
+            }
+            const int v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            a.scores[(size_t)cc.b * cap + cc.row + tid] = v;
+            atomicAdd(&hist[score_bin(v, bias, shift)], 1);
+        }
+        __syncthreads();  // stage s is free again
+        if (tid == 0 && pmore) {
+            const int prow = min(kStageRows, pc.end - pc.row);
+            bulk_load(smem_addr(ring + s * STAGE),
+                      a.idx_k + ((size_t)pc.b * cap + pc.row) * DI, (uint32_t)prow * DI,
+                      smem_addr(&full[s]));
+            pc.row += prow;
+            if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
+        }
+        cc.row += rows;
+        if (cc.row < cc.end) continue;
+        // ---- sequence cc.b done in this CTA: flush, maybe derive its threshold
+        const int b = cc.b;
         const int n = a.n_entries[b];
-        if (n < 0 || n > a.capacity) {
-            if (threadIdx.x == 0) set_status(a.status, KVC_DEV_BAD_LENGTH);
-            continue;
-        }
-        const long long base = (long long)b * cap;
-        const int start = (int)(max(lo, base) - base);
-        const int end = (int)min(min(hi, base + cap) - base, (long long)n);
-        if (start >= end) continue;  // this CTA holds none of b's visible rows
-        __syncthreads();
-        for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
-        __syncthreads();
-        scan_rows<DI>(a, b, start, end, bias, shift, hist);
-        __syncthreads();
         int32_t* gh = a.counters + (size_t)b * kBins;
-        for (int i = threadIdx.x; i < kBins; i += kThreads)
+        for (int i = tid; i < kBins; i += kThreads)
             if (hist[i]) atomicAdd(&gh[i], hist[i]);
-        if (n <= a.topk) continue;  // everything is selected; no threshold needed
-        // the last CTA holding rows of b derives b's threshold
-        const long long first = base / per, last = (base + n - 1) / per;
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0)
-            s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) ==
-                     (int)(last - first);
-        __syncthreads();
-        if (!s_last) continue;
-        __threadfence();
-        for (int i = threadIdx.x * 4; i < kBins; i += kThreads * 4)
-            *reinterpret_cast<int4*>(hist + i) = __ldcg(reinterpret_cast<const int4*>(gh + i));
-        if (threadIdx.x == 0) s_t = s_above = 0;
-        __syncthreads();
-        find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
-        if (threadIdx.x == 0) {
-            a.thr[2 * b] = s_t;
-            a.thr[2 * b + 1] = s_above;
+        if (n > a.topk) {
+            const long long base = (long long)b * cap;
+            const long long first = base / per, last = (base + n - 1) / per;
+            __threadfence();
+            __syncthreads();
+            if (tid == 0)
+                s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) ==
+                         (int)(last - first);
+            __syncthreads();
+            if (s_last) {
+                __threadfence();
+                for (int i = tid * 4; i < kBins; i += kThreads * 4)
+                    *reinterpret_cast<int4*>(hist + i) =
+                        __ldcg(reinterpret_cast<const int4*>(gh + i));
+                if (tid == 0) s_t = s_above = 0;
+                __syncthreads();
+                find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
+                if (tid == 0) {
+                    a.thr[2 * b] = s_t;
+                    a.thr[2 * b + 1] = s_above;
+                }
+            }
         }
+        __syncthreads();
+        for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
+        if (!cursor_seek(a, lo, hi, cc, b + 1)) break;
+        if (tid < PIECES)
+            qs[tid] = __ldg(reinterpret_cast<const int4*>(a.idx_q + (size_t)cc.b * DI) + tid);
+        __syncthreads();
+    }
+    if (!ok && tid == 0) {
+        // a bounded wait gave up: flag it and let the copies still in flight land
+        set_status(a.status, KVC_DEV_TIMEOUT);
+        for (int s = 0; s < kScanStages; ++s) bar_wait(smem_addr(&full[s]), (phase >> s) & 1u);
     }
 }
 
@@ -215,135 +318,192 @@ __device__ void block_bitonic(Key* k, int p, bool desc) {
     }
 }
 
-constexpr size_t kSelSmem = (size_t)kMaxTies * 8 + (size_t)kMaxSelTiles * 4 * 2;
+// Candidate keys of one sequence staged in shared memory for the finish.
+constexpr int kStageKeys = 6144;
+constexpr size_t kFinishSmem =
+    (size_t)kStageKeys * 8 + (size_t)kMaxTies * 8 + (size_t)kMaxSelTiles * 4 * 2;
 
 __global__ void __launch_bounds__(kThreads)
-topk_select_kernel(TopkArgs a, int bias, int shift) {
+topk_collect_kernel(TopkArgs a, int bias, int shift) {
+    __shared__ int sh_warp[kThreads / 32];
+    constexpr int PER = kSelTile / kThreads;  // scores per thread
+    const int b = blockIdx.y, K = a.topk, tid = threadIdx.x;
+    const int n = a.n_entries[b];
+    if (n < 0 || n > a.capacity || n <= K) return;
+    const int ntiles = (n + kSelTile - 1) / kSelTile;
+    const int tile = blockIdx.x;
+    if (tile >= ntiles) return;
+    const int t = __ldcg(a.thr + 2 * b);
+    const int32_t* sc = a.scores + (size_t)b * a.capacity;
+    const int ctiles = sel_tiles(a.capacity);
+    unsigned long long* cand = a.cands + ((size_t)b * ctiles + tile) * kSelTile;
+    // compact this tile's candidates (bins >= t) in index order
+    int v[PER];
+    const int j0 = tile * kSelTile + tid * PER;
+    if (j0 + PER <= n && ((reinterpret_cast<uintptr_t>(sc + j0) & 15) == 0)) {
+#pragma unroll
+        for (int u = 0; u < PER / 4; ++u) {
+            const int4 x = __ldcg(reinterpret_cast<const int4*>(sc + j0) + u);
+            v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) v[u] = (j0 + u < n) ? __ldcg(sc + j0 + u) : 0;
+    }
+    unsigned take = 0;
+#pragma unroll
+    for (int u = 0; u < PER; ++u)
+        if (j0 + u < n && score_bin(v[u], bias, shift) >= t) take |= 1u << u;
+    int pos;
+    const int total = block_excl_scan(__popc(take), &pos, sh_warp);
+#pragma unroll
+    for (int u = 0; u < PER; ++u)
+        if (take & (1u << u)) cand[pos++] = make_key(v[u], j0 + u, bias);
+    if (tid == 0) a.tile_count[(size_t)b * ctiles + tile] = total;
+}
+
+// One CTA per sequence finishes the selection from the tiles' candidates.
+__global__ void __launch_bounds__(kThreads)
+topk_finish_kernel(TopkArgs a, int bias, int shift) {
     extern __shared__ __align__(16) unsigned char smem[];
-    unsigned long long* ties = reinterpret_cast<unsigned long long*>(smem);  // kMaxTies
+    unsigned long long* stage = reinterpret_cast<unsigned long long*>(smem);  // kStageKeys
+    unsigned long long* ties = stage + kStageKeys;                            // kMaxTies
     int* cnt = reinterpret_cast<int*>(ties + kMaxTies);                       // per tile
     int* off = cnt + kMaxSelTiles;                                            // per tile
     __shared__ int sh_warp[kThreads / 32];
-    __shared__ int s_last, s_nt, s_low, s_gt;
+    __shared__ int s_nt, s_low, s_gt;
     __shared__ unsigned long long s_kstar;
-    const int b = blockIdx.y, K = a.topk, tid = threadIdx.x;
+    const int b = blockIdx.x, K = a.topk, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int n = a.n_entries[b];
     int32_t* out = a.topk_idx + (size_t)b * K;
     if (n < 0 || n > a.capacity) {
-        if (blockIdx.x == 0)
-            for (int i = tid; i < K; i += kThreads) out[i] = -1;
+        for (int i = tid; i < K; i += kThreads) out[i] = -1;
         return;
     }
     if (n <= K) {
-        if (blockIdx.x == 0)
-            for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
+        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
     const int ntiles = (n + kSelTile - 1) / kSelTile;
-    const int tile = blockIdx.x;
-    if (tile >= ntiles) return;
     const int t = __ldcg(a.thr + 2 * b), above = __ldcg(a.thr + 2 * b + 1);
     const int32_t* sc = a.scores + (size_t)b * a.capacity;
     const int ctiles = sel_tiles(a.capacity);
-    unsigned long long* cand = a.cands + ((size_t)b * ctiles + tile) * kSelTile;
-
-    // ---- compact this tile's candidates (bins >= t) in index order
-    {
-        int v[8];
-        const int j0 = tile * kSelTile + tid * 8;
-        if (j0 + 8 <= n && ((reinterpret_cast<uintptr_t>(sc + j0) & 15) == 0)) {
-            const int4 x0 = __ldcg(reinterpret_cast<const int4*>(sc + j0));
-            const int4 x1 = __ldcg(reinterpret_cast<const int4*>(sc + j0) + 1);
-            v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-            v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-        } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = (j0 + u < n) ? __ldcg(sc + j0 + u) : 0;
-        }
-        unsigned take = 0;
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (j0 + u < n && score_bin(v[u], bias, shift) >= t) take |= 1u << u;
-        int pos;
-        const int total = block_excl_scan(__popc(take), &pos, sh_warp);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (take & (1u << u)) cand[pos++] = make_key(v[u], j0 + u, bias);
-        if (tid == 0) a.tile_count[(size_t)b * ctiles + tile] = total;
-    }
-    // ---- the last CTA of this sequence to finish completes the selection
-    __threadfence();
-    __syncthreads();
-    if (tid == 0)
-        s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + a.batch + b, 1) == ntiles - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-
     const unsigned long long* cb = a.cands + (size_t)b * ctiles * kSelTile;
-    for (int i = tid; i < ntiles; i += kThreads) cnt[i] = __ldcg(a.tile_count + (size_t)b * ctiles + i);
+    // tile counts and their exclusive prefix
+    int M = 0;
+    for (int base = 0; base < ntiles; base += kThreads) {
+        const int i = base + tid;
+        const int c = i < ntiles ? __ldcg(a.tile_count + (size_t)b * ctiles + i) : 0;
+        int ex;
+        const int tot = block_excl_scan(c, &ex, sh_warp);
+        if (i < ntiles) {
+            cnt[i] = c;
+            off[i] = M + ex;
+        }
+        M += tot;
+    }
     if (tid == 0) s_nt = 0;
     __syncthreads();
-    // the tie candidates: keys of bin t (a warp per tile)
-    const int r = K - above;
-    for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
-        const unsigned long long* ct = cb + (size_t)ti * kSelTile;
-        for (int i = lane; i < cnt[ti]; i += 32) {
-            const unsigned long long k = __ldcg(ct + i);
+    const int r = K - above;  // entries to take from bin t
+    if (M <= kStageKeys) {
+        // every candidate key, in index order, with one round of parallel loads
+        for (int p = tid; p < M; p += kThreads) {
+            int lo = 0, hi = ntiles - 1;  // last tile with off <= p
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (off[mid] <= p) lo = mid; else hi = mid - 1;
+            }
+            const unsigned long long k = __ldcg(cb + (size_t)lo * kSelTile + (p - off[lo]));
+            stage[p] = k;
             if ((int)((k >> 32) >> shift) == t) {
-                const int p = atomicAdd(&s_nt, 1);
-                if (p < kMaxTies) ties[p] = k;
+                const int q = atomicAdd(&s_nt, 1);
+                if (q < kMaxTies) ties[q] = k;
             }
         }
-    }
-    __syncthreads();
-    const int nt = s_nt;
-    if (nt <= kMaxTies) {
-        int p2 = 1;
-        while (p2 < nt) p2 <<= 1;
-        for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;  // sorts last
         __syncthreads();
-        block_bitonic(ties, p2, true);
-        if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;  // r-th best of bin t
-        __syncthreads();
-        const unsigned long long kstar = s_kstar;
-        // winners per tile, prefix over tiles, then write in index order
-        for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
-            const unsigned long long* ct = cb + (size_t)ti * kSelTile;
-            int c = 0;
-            for (int i = lane; i < cnt[ti]; i += 32) c += __ldcg(ct + i) >= kstar;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-            if (lane == 0) off[ti] = c;
-        }
-        __syncthreads();
-        int run = 0;
-        for (int base = 0; base < ntiles; base += kThreads) {
-            const int i = base + tid;
-            const int c = i < ntiles ? off[i] : 0;
-            int ex;
-            const int tot = block_excl_scan(c, &ex, sh_warp);
-            if (i < ntiles) off[i] = run + ex;
-            run += tot;
+        const int nt = s_nt;
+        if (nt <= kMaxTies) {
+            int p2 = 1;
+            while (p2 < nt) p2 <<= 1;
+            for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;  // sorts last
             __syncthreads();
+            block_bitonic(ties, p2, true);
+            if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;
+            __syncthreads();
+            const unsigned long long kstar = s_kstar;
+            int run = 0;
+            for (int base = 0; base < M; base += kThreads) {
+                const int p = base + tid;
+                const bool sel = p < M && stage[p] >= kstar;
+                int ex;
+                const int tot = block_excl_scan(sel ? 1 : 0, &ex, sh_warp);
+                if (sel && run + ex < K) out[run + ex] = key_index(stage[p]);
+                run += tot;
+            }
+            for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
+            return;
         }
+    } else {
+        // too many candidates to stage: the tie keys straight from the tiles
         for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
             const unsigned long long* ct = cb + (size_t)ti * kSelTile;
-            int o = off[ti];
-            for (int i0 = 0; i0 < cnt[ti]; i0 += 32) {
-                const int i = i0 + lane;
-                const unsigned long long k = i < cnt[ti] ? __ldcg(ct + i) : 0ull;
-                const bool sel = i < cnt[ti] && k >= kstar;
-                const unsigned m = __ballot_sync(0xffffffffu, sel);
-                const int p = o + __popc(m & ((1u << lane) - 1u));
-                if (sel && p < K) out[p] = key_index(k);
-                o += __popc(m);
+            for (int i = lane; i < cnt[ti]; i += 32) {
+                const unsigned long long k = __ldcg(ct + i);
+                if ((int)((k >> 32) >> shift) == t) {
+                    const int q = atomicAdd(&s_nt, 1);
+                    if (q < kMaxTies) ties[q] = k;
+                }
             }
         }
         __syncthreads();
-        for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
-        return;
+        const int nt = s_nt;
+        if (nt <= kMaxTies) {
+            int p2 = 1;
+            while (p2 < nt) p2 <<= 1;
+            for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;
+            __syncthreads();
+            block_bitonic(ties, p2, true);
+            if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;
+            __syncthreads();
+            const unsigned long long kstar = s_kstar;
+            // winners per tile, prefix over tiles, then write in index order
+            for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
+                const unsigned long long* ct = cb + (size_t)ti * kSelTile;
+                int c = 0;
+                for (int i = lane; i < cnt[ti]; i += 32) c += __ldcg(ct + i) >= kstar;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+                if (lane == 0) off[ti] = c;
+            }
+            __syncthreads();
+            int run = 0;
+            for (int base = 0; base < ntiles; base += kThreads) {
+                const int i = base + tid;
+                const int c = i < ntiles ? off[i] : 0;
+                int ex;
+                const int tot = block_excl_scan(c, &ex, sh_warp);
+                if (i < ntiles) off[i] = run + ex;
+                run += tot;
+                __syncthreads();
+            }
+            for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
+                const unsigned long long* ct = cb + (size_t)ti * kSelTile;
+                int o = off[ti];
+                for (int i0 = 0; i0 < cnt[ti]; i0 += 32) {
+                    const int i = i0 + lane;
+                    const unsigned long long k = i < cnt[ti] ? __ldcg(ct + i) : 0ull;
+                    const bool sel = i < cnt[ti] && k >= kstar;
+                    const unsigned m = __ballot_sync(0xffffffffu, sel);
+                    const int p = o + __popc(m & ((1u << lane) - 1u));
+                    if (sel && p < K) out[p] = key_index(k);
+                    o += __popc(m);
+                }
+            }
+            __syncthreads();
+            for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
+            return;
+        }
     }
 
     // Heavy ties: exact threshold score inside bin t from a second histogram
@@ -392,7 +552,19 @@ topk_select_kernel(TopkArgs a, int bias, int shift) {
 template <int DI>
 cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, int shift,
                         cudaStream_t s) {
-    index_scan_kernel<DI><<<ctas, kThreads, 0, s>>>(a, per, bias, shift);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(
+            index_scan_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            kScanStages * kStageRows * DI);
+        if (e == cudaSuccess) e = prefer_shared(index_scan_kernel<DI>);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    index_scan_kernel<DI><<<ctas, kThreads, kScanStages * kStageRows * DI, s>>>(a, per, bias,
+                                                                                shift);
     return cudaGetLastError();
 }
 
@@ -405,12 +577,13 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     cudaError_t err =
         cudaMemsetAsync(a.counters, 0, topk_counter_words(a.batch) * sizeof(int32_t), s);
     if (err != cudaSuccess) return err;
-    // one wave: 4 CTAs per SM (64 registers x 256 threads), equal row slices
+    // one wave: 2 CTAs per SM (96 KB ring + 8 KB histogram each for Di = 128),
+    // equal row slices
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long rows = (long long)a.batch * a.capacity;
-    int ctas = 4 * sms;
+    int ctas = (a.di >= 256 ? 1 : 2) * sms;
     long long per = (rows + ctas - 1) / ctas;
     per = (per + 255) / 256 * 256;
     if (per < 256) per = 256;
@@ -425,16 +598,22 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     }
     trace_after(s);
     if (err != cudaSuccess) return err;
+    dim3 grid(sel_tiles(a.capacity), a.batch);
+    trace_before("topk_collect", s);
+    topk_collect_kernel<<<grid, kThreads, 0, s>>>(a, bias, shift);
+    trace_after(s);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     static bool attr_set[64] = {};
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        err = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kSelSmem);
+        err = cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kFinishSmem);
+        if (err == cudaSuccess) err = prefer_shared(topk_finish_kernel);
+        if (err == cudaSuccess) err = prefer_shared(topk_collect_kernel);
         if (err != cudaSuccess) return err;
         attr_set[dev] = true;
     }
-    dim3 grid(sel_tiles(a.capacity), a.batch);
-    trace_before("topk_select", s);
-    topk_select_kernel<<<grid, kThreads, kSelSmem, s>>>(a, bias, shift);
+    trace_before("topk_finish", s);
+    topk_finish_kernel<<<a.batch, kThreads, kFinishSmem, s>>>(a, bias, shift);
     trace_after(s);
     return cudaGetLastError();
 }

@@ -15,8 +15,8 @@ constexpr int kBins = 2048;
 // Top-K selection: scores are cut into tiles of kSelTile entries; each tile
 // keeps its candidate keys (in index order) in its own slot of the candidate
 // array.  A sequence holds at most kMaxSelTiles tiles (8,388,608 entries).
-constexpr int kSelTile = 2048;
-constexpr int kMaxSelTiles = 4096;
+constexpr int kSelTile = 8192;
+constexpr int kMaxSelTiles = 1024;
 constexpr long long kMaxTopkCapacity = (long long)kSelTile * kMaxSelTiles;
 // Candidates of the threshold bin kept for the in-shared-memory finish.
 constexpr int kMaxTies = 4096;
@@ -109,6 +109,15 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
 
 cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3,
                              cudaStream_t s);
+
+// All library kernels ask for the largest shared-memory carve-out, so that
+// consecutive kernels of a step never make the SM reconfigure L1/shared.
+// Called once per kernel and device, before the first launch.
+template <typename F>
+inline cudaError_t prefer_shared(F* kernel) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared);
+}
 
 // ------------------------------------------------------------------ device helpers
 #ifdef __CUDACC__

@@ -9,7 +9,7 @@
 // per-sequence histograms and counters, the candidate lists -- lives in the
 // file-scope array below, sized for at most kNoAllocMaxBatch sequences and
 // kNoAllocMaxRows = batch x capacity entries.  Every GPU that loads the library
-// holds the array (about 8 MiB) until the process exits.
+// holds the array (about 10.5 MiB) until the process exits.
 #include <mutex>
 
 #include "kvc_internal.cuh"

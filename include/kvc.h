@@ -152,7 +152,7 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
  * pages have no counterpart of this call; it computes exactly what
  * kvc_index_topk computes (same kernels, same results).
  * Its scratch (scores, histograms, counters, candidate lists) is a fixed
- * array inside the library, about 8 MiB, held on every GPU that loads the
+ * array inside the library, about 10.5 MiB, held on every GPU that loads the
  * library until the process exits.  Limits: batch <= 64 and
  * batch * capacity <= 524,288 entries; larger problems return
  * KVC_ERR_CAPACITY before anything is enqueued.  The call allocates nothing.
@@ -217,8 +217,8 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * max_launches launches are recorded).  kvc_trace_kernel, called after the
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
- * "pack", "pack_commit", "index_scan", "topk_select", "attn_tc05",
- * "attn_mma", "attn_simt", "attn_merge", "fp4_codec".                      */
+ * "pack", "pack_commit", "index_scan", "topk_collect", "topk_finish", "attn_tc05",
+ * "attn_simt", "attn_merge", "fp4_codec".                      */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);
 kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);
