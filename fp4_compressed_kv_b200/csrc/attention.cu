@@ -188,21 +188,16 @@ attn_merge_kernel(AttnArgs a, int H, int Dv, int nsplit) {
     __syncthreads();
     const float inv = s_inv;
     for (int d = tid * 4; d < Dv; d += 128 * 4) {
-        float4 v[kMaxSplit];
-#pragma unroll
-        for (int s = 0; s < kMaxSplit; ++s)
-            if (s < nsplit)
-                v[s] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (row0 + s) * Dv + d));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int s = 0; s < kMaxSplit; ++s)
-            if (s < nsplit) {
-                const float w = s_w[s];
-                acc.x = fmaf(w, v[s].x, acc.x);
-                acc.y = fmaf(w, v[s].y, acc.y);
-                acc.z = fmaf(w, v[s].z, acc.z);
-                acc.w = fmaf(w, v[s].w, acc.w);
-            }
+#pragma unroll 4
+        for (int s = 0; s < nsplit; ++s) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (row0 + s) * Dv + d));
+            const float w = s_w[s];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
         *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h) * Dv + d) =
             make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
@@ -249,10 +244,6 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
                      : cudaFuncSetAttribute(attn_simt_kernel<float>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             kSimtChunk * 1024 * 4);
-            if (err == cudaSuccess)
-                err = ti ? prefer_shared(attn_simt_kernel<__nv_bfloat16>)
-                         : prefer_shared(attn_simt_kernel<float>);
-            if (err == cudaSuccess) err = prefer_shared(attn_merge_kernel);
             if (err != cudaSuccess) return err;
             attr_set2[dev][ti] = true;
         }

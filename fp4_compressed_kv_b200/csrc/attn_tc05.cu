@@ -43,7 +43,7 @@ constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
 constexpr uint32_t OFF_RAW = OFF_K + K_BYTES;   // P (16 KB) reuses this after dequant
 constexpr uint32_t OFF_P = OFF_RAW;
 constexpr uint32_t OFF_MISC = OFF_RAW + RAW_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 3072 + 1024;  // + misc + table + alignment slack
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;  // + misc + table + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0, O_COL = 128;
 
@@ -146,8 +146,37 @@ __device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c16) {
     return (r >> 3) * 1024u + (r & 7u) * 128u + ((c16 ^ (r & 7u)) << 4);
 }
 
+// 32 lanes x 16 consecutive columns
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// The reference maximum of a head only moves when a chunk's maximum passes it
+// by more than this (log2 units): probabilities stay <= 2^8 in bf16 and the
+// accumulated O^T is rescaled in tensor memory only on such a jump.
+constexpr float kRescaleSlack = 8.0f;
+
 __global__ void __launch_bounds__(NT, 1)
-attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int ue4m3) {
+attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int cps, int ue4m3) {
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -156,11 +185,14 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sP = base + OFF_P;
     unsigned char* raw = smem + OFF_RAW;
     int* kind = reinterpret_cast<int*>(smem + OFF_MISC);                 // [CK]
-    float* mrow = reinterpret_cast<float*>(smem + OFF_MISC + 512);       // [H]
-    float* lrow = mrow + H;                                              // [H]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_MISC + 1536);  // S done, O done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 1600);
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 2048);  // [256] bf16x2
+    float* mref = reinterpret_cast<float*>(smem + OFF_MISC + 512);       // [H] reference max
+    float* lrun = mref + H;                                              // [H] running sum
+    float* fac = lrun + H;                                               // [H] rescale factor
+    float* part = fac + H;                                               // [2][H] half max/sum
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_MISC + 2048);  // S done, O done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 2112);
+    int* flags = reinterpret_cast<int*>(smem + OFF_MISC + 2176);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 3072);  // [256] bf16x2
 
     const int b = blockIdx.y, split = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -168,6 +200,7 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
     const bool len_ok = n >= 0 && n <= a.capacity;
     const int total = K + a.window_len;
     const int rb = sh.rb;
+    const int c0 = split * cps, c1 = min(c0 + cps, (total + CK - 1) / CK);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
@@ -180,178 +213,241 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         mbar_init(smem_u32(&bars[1]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
-    if (tid < CK) {
-        const int j = split * CK + tid;
-        int k = -1;
-        if (j < total && len_ok) {
-            if (j < K) {
-                const int idx = a.topk_idx[(size_t)b * K + j];
-                if (idx >= 0 && idx < n)
-                    k = idx;
-                else if (idx != -1)
-                    set_status(a.status, KVC_DEV_BAD_INDEX);
-            } else {
-                k = -2 - (j - K);  // window row
-            }
-        }
-        kind[tid] = k;
+    if (tid < H) {
+        mref[tid] = -INFINITY;
+        lrun[tid] = 0.f;
     }
-    {  // code-pair table: byte -> (E2M1(low nibble), E2M1(high nibble)) as bf16x2
-        lut[tid] = pack_bf16(e2m1_value(tid & 15u), e2m1_value(tid >> 4));
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    // ---- 1. gathers: Q (swizzled), records (raw rows), window rows (swizzled)
+    // code-pair table: byte -> (E2M1(low nibble), E2M1(high nibble)) as bf16x2
+    lut[tid] = pack_bf16(e2m1_value(tid & 15u), e2m1_value(tid >> 4));
+    // Q (64 x 576) once, 128B-swizzled K-major
     {
         const unsigned char* qg = static_cast<const unsigned char*>(a.q) + (size_t)b * H * D * 2;
         for (int p = tid; p < H * (D / 8); p += NT) {
             const int h = p / (D / 8), c = p - h * (D / 8);
             cp_async16(sQ + (c >> 3) * 8192u + swz(h, c & 7), qg + (size_t)h * D * 2 + c * 16);
         }
-        const int pieces = rb >> 4;
-        for (int p = tid; p < CK * pieces; p += NT) {
-            const int s = p / pieces, pc = p - s * pieces;
-            const int k = kind[s];
-            if (k >= 0)
-                cp_async16(smem_u32(raw + s * RAW_STRIDE + pc * 16),
-                           a.records + ((size_t)b * a.capacity + k) * rb + pc * 16);
-        }
-        for (int p = tid; p < CK * (D / 8); p += NT) {
-            const int s = p / (D / 8), c = p - s * (D / 8);
-            const int k = kind[s];
-            const uint32_t dst = sK + (c >> 3) * K_ATOM + swz(s, c & 7);
-            if (k <= -2) {
-                const int t = -2 - k;
-                cp_async16(dst, static_cast<const unsigned char*>(a.window) +
-                                    ((size_t)b * a.window_stride + t) * D * 2 + c * 16);
-            } else if (k == -1) {
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(0u), "r"(0u),
-                             "r"(0u), "r"(0u));
-            }
-        }
-        cp_async_wait_all();
     }
-    __syncthreads();
-
-    // ---- 2. dequantise records into the swizzled K tile.  UE4M3 scales: a
-    // byte of two codes -> bf16x2 table entry, times the bf16x2 scale (the
-    // products have at most 6 significant bits, so the bf16 multiply is exact).
-    if (ue4m3) {
-        for (int p = tid; p < CK * (D / 8); p += NT) {
-            const int s = p / (D / 8), c = p - s * (D / 8);
-            if (kind[s] < 0) continue;
-            const unsigned char* rec = raw + s * RAW_STRIDE;
-            const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + c * 4);
-            const float sc = e4m3_to_f32(rec[sh.code_bytes + c / sh.lpg]);
-            const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc, sc);
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t e = lut[(codes >> (8 * k)) & 0xFFu];
-                const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e), s2);
-                w[k] = *reinterpret_cast<const uint32_t*>(&v);
-            }
-            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
-                             sK + (c >> 3) * K_ATOM + swz(s, c & 7)),
-                         "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
-        }
-    } else {
-        for (int p = tid; p < CK * (D / 8); p += NT) {
-            const int s = p / (D / 8), c = p - s * (D / 8);
-            if (kind[s] < 0) continue;
-            const unsigned char* rec = raw + s * RAW_STRIDE;
-            const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + c * 4);
-            const float sc = reinterpret_cast<const float*>(rec + sh.code_bytes)[c / sh.lpg];
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                w[k] = pack_bf16(e2m1_value((codes >> (8 * k)) & 15u) * sc,
-                                 e2m1_value((codes >> (8 * k + 4)) & 15u) * sc);
-            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
-                             sK + (c >> 3) * K_ATOM + swz(s, c & 7)),
-                         "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
-        }
-    }
-    fence_async_smem();
-    __syncthreads();
-
-    // ---- 3. S = Q K^T (one thread issues)
-    if (tid == 0) {
-        tc_fence_after();
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t at = ks >> 2, koff = (ks & 3) * 32;
-            mma_bf16(tmem + S_COL, sdesc(sQ + at * 8192u + koff, 16, 1024),
-                     sdesc(sK + at * K_ATOM + koff, 16, 1024), kIdescQK, ks > 0);
-        }
-        mma_commit(smem_u32(&bars[0]));
-    }
-    // warp 0 polls the barrier; the other warps wait in the block barrier
-    bool ok = warp == 0 ? mbar_wait(smem_u32(&bars[0]), 0) : true;
-    ok = __syncthreads_and(ok) != 0;
-    tc_fence_after();
-
-    // ---- 4. softmax: warps 0-1, one thread per head row of S
-    if (ok && warp < 2) {
-        const int h = warp * 32 + lane;
-        float sv[CK];
-#pragma unroll
-        for (int c0 = 0; c0 < CK; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + S_COL + c0, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[c0 + i] = __uint_as_float(r[i]);
-        }
-        float m = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < CK; ++j) {
-            const float x = kind[j] == -1 ? -INFINITY : sv[j] * scale_log2;
-            sv[j] = x;
-            m = fmaxf(m, x);
-        }
-        float l = 0.f;
-#pragma unroll
-        for (int cj = 0; cj < CK / 8; ++cj) {
-            float p[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                p[u] = m == -INFINITY ? 0.f : exp2f(sv[cj * 8 + u] - m);
-                l += p[u];
-            }
-            const uint32_t dst = sP + (cj >> 3) * 8192u + swz(h, cj & 7);
-            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst),
-                         "r"(pack_bf16(p[0], p[1])), "r"(pack_bf16(p[2], p[3])),
-                         "r"(pack_bf16(p[4], p[5])), "r"(pack_bf16(p[6], p[7])));
-        }
-        mrow[h] = m;
-        lrow[h] = l;
-    }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
-
-    // ---- 5. O^T = V^T P^T (one thread issues); V^T = latent atoms of the K tile
-    if (ok && tid == 0) {
-        tc_fence_after();
-        for (int mt = 0; mt < DV / 128; ++mt)
-            for (int kk = 0; kk < CK / 16; ++kk)
-                mma_bf16(tmem + O_COL + 64 * mt,
-                         sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
-                         sdesc(sP + (kk >> 2) * 8192u + (kk & 3) * 32u, 16, 1024), kIdescPV,
-                         kk > 0);
-        mma_commit(smem_u32(&bars[1]));
-    }
-    bool ok2 = ok;
-    if (ok && warp == 0) ok2 = mbar_wait(smem_u32(&bars[1]), 0);
-    const bool ok_s = ok;
-    ok = __syncthreads_and(ok2) != 0;
     tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    for (int c = c0; c < c1 && ok; ++c) {
+        const int it = c - c0;
+        // ---- slot kinds of this chunk
+        if (tid < CK) {
+            const int j = c * CK + tid;
+            int k = -1;
+            if (j < total && len_ok) {
+                if (j < K) {
+                    const int idx = a.topk_idx[(size_t)b * K + j];
+                    if (idx >= 0 && idx < n)
+                        k = idx;
+                    else if (idx != -1)
+                        set_status(a.status, KVC_DEV_BAD_INDEX);
+                } else {
+                    k = -2 - (j - K);  // window row
+                }
+            }
+            kind[tid] = k;
+        }
+        __syncthreads();
+        // ---- 1. gathers: records (raw rows), window rows (swizzled) and zero rows
+        {
+            const int pieces = rb >> 4;
+            for (int p = tid; p < CK * pieces; p += NT) {
+                const int s = p / pieces, pc = p - s * pieces;
+                const int k = kind[s];
+                if (k >= 0)
+                    cp_async16(smem_u32(raw + s * RAW_STRIDE + pc * 16),
+                               a.records + ((size_t)b * a.capacity + k) * rb + pc * 16);
+            }
+            for (int p = tid; p < CK * (D / 8); p += NT) {
+                const int s = p / (D / 8), cc = p - s * (D / 8);
+                const int k = kind[s];
+                const uint32_t dst = sK + (cc >> 3) * K_ATOM + swz(s, cc & 7);
+                if (k <= -2) {
+                    const int t = -2 - k;
+                    cp_async16(dst, static_cast<const unsigned char*>(a.window) +
+                                        ((size_t)b * a.window_stride + t) * D * 2 + cc * 16);
+                } else if (k == -1) {
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(0u),
+                                 "r"(0u), "r"(0u), "r"(0u));
+                }
+            }
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        // ---- 2. dequantise records into the swizzled K tile.  UE4M3 scales, groups
+        // of >= 32: 32 channels per item, a byte of two codes -> bf16x2 table
+        // entry times the bf16x2 scale (the products have at most 6 significant
+        // bits, so the bf16 multiply is exact).
+        if (ue4m3 && sh.lpg >= 4) {
+            for (int p = tid; p < CK * (D / 32); p += NT) {
+                const int s = p / (D / 32), i4 = p - s * (D / 32);
+                if (kind[s] < 0) continue;
+                const unsigned char* rec = raw + s * RAW_STRIDE;
+                const uint4 codes = *reinterpret_cast<const uint4*>(rec + i4 * 16);
+                const float sc = e4m3_to_f32(rec[sh.code_bytes + (4 * i4) / sh.lpg]);
+                const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc, sc);
+                const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+                const uint32_t row = sK + (i4 >> 1) * K_ATOM;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t e = lut[(cw[u] >> (8 * k)) & 0xFFu];
+                        const __nv_bfloat162 v =
+                            __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e), s2);
+                        w[k] = *reinterpret_cast<const uint32_t*>(&v);
+                    }
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                                     row + swz(s, 4 * (i4 & 1) + u)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+                }
+            }
+        } else {
+            for (int p = tid; p < CK * (D / 8); p += NT) {
+                const int s = p / (D / 8), cc = p - s * (D / 8);
+                if (kind[s] < 0) continue;
+                const unsigned char* rec = raw + s * RAW_STRIDE;
+                const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + cc * 4);
+                const int g = cc / sh.lpg;
+                const float sc = ue4m3 ? e4m3_to_f32(rec[sh.code_bytes + g])
+                                       : reinterpret_cast<const float*>(rec + sh.code_bytes)[g];
+                uint32_t w[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    w[k] = pack_bf16(e2m1_value((codes >> (8 * k)) & 15u) * sc,
+                                     e2m1_value((codes >> (8 * k + 4)) & 15u) * sc);
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                                 sK + (cc >> 3) * K_ATOM + swz(s, cc & 7)),
+                             "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+            }
+        }
+        fence_async_smem();
+        __syncthreads();
+
+        // ---- 3. S = Q K^T (one thread issues)
+        if (tid == 0) {
+            tc_fence_after();
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t at = ks >> 2, koff = (ks & 3) * 32;
+                mma_bf16(tmem + S_COL, sdesc(sQ + at * 8192u + koff, 16, 1024),
+                         sdesc(sK + at * K_ATOM + koff, 16, 1024), kIdescQK, ks > 0);
+            }
+            mma_commit(smem_u32(&bars[0]));
+        }
+        // warp 0 polls the barrier; the other warps wait in the block barrier
+        bool got = warp == 0 ? mbar_wait(smem_u32(&bars[0]), it & 1) : true;
+        ok = __syncthreads_and(got) != 0;
+        tc_fence_after();
+        if (!ok) break;
+
+        // ---- 4. softmax: warps 0,1 take columns [0, 48) and warps 4,5 columns
+        // [48, 96) of the head rows (TMEM lanes 0..63)
+        const bool sm_warp = (warp & 3) < 2;
+        const int h = (warp & 3) * 32 + lane, half = warp >> 2;
+        float sv[CK / 2];
+        if (sm_warp) {
+            const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL + half * (CK / 2);
+            uint32_t r32[32];
+            uint32_t r16[16];
+            tmem_ld32(ta, r32);
+            tmem_ld16(ta + 32, r16);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r32[i]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sv[32 + i] = __uint_as_float(r16[i]);
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int j = 0; j < CK / 2; ++j) {
+                const float x = kind[half * (CK / 2) + j] == -1 ? -INFINITY : sv[j] * scale_log2;
+                sv[j] = x;
+                m4[j & 3] = fmaxf(m4[j & 3], x);
+            }
+            part[half * H + h] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+        __syncthreads();
+        if (sm_warp) {
+            const float mc = fmaxf(part[h], part[H + h]);
+            const float mo = mref[h];
+            // move the reference only on a large jump (or the first keys)
+            const float mn = (mo == -INFINITY || mc > mo + kRescaleSlack) ? mc : mo;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int cj = 0; cj < CK / 16; ++cj) {
+                float pv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    pv[u] = mn == -INFINITY ? 0.f : exp2f(sv[cj * 8 + u] - mn);
+                    l4[u & 3] += pv[u];
+                }
+                const int kc = half * (CK / 16) + cj;  // 8-key chunk index in the P row
+                const uint32_t dst = sP + (kc >> 3) * 8192u + swz(h, kc & 7);
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst),
+                             "r"(pack_bf16(pv[0], pv[1])), "r"(pack_bf16(pv[2], pv[3])),
+                             "r"(pack_bf16(pv[4], pv[5])), "r"(pack_bf16(pv[6], pv[7])));
+            }
+            __syncwarp();
+            sv[0] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            if (half == 0) fac[h] = mn;  // the new reference, published below
+        }
+        __syncthreads();
+        if (sm_warp) part[half * H + h] = sv[0];
+        if (tid == 0) flags[0] = 0;
+        __syncthreads();
+        if (tid < H) {
+            const float mo = mref[tid], mn = fac[tid];
+            const float f = mo == -INFINITY ? 0.f : exp2f(mo - mn);  // 1 when unchanged
+            lrun[tid] = lrun[tid] * f + part[tid] + part[H + tid];
+            mref[tid] = mn;
+            fac[tid] = f;
+            if (it > 0 && f != 1.f) flags[0] = 1;
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- rare: a head's reference moved after O^T holds earlier chunks
+        if (flags[0]) {
+            tc_fence_after();
+            const int g = warp & 3;
+            for (int t = 0; t < 2; ++t) {
+                const int mt = (warp >> 2) * 2 + t;
+                for (int h0 = 0; h0 < H; h0 += 32) {
+                    const uint32_t ta = tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0;
+                    uint32_t r[32];
+                    tmem_ld32(ta, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(__uint_as_float(r[i]) * fac[h0 + i]);
+                    tmem_st32(ta, r);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+        }
+        // ---- 5. O^T += V^T P^T (one thread issues); V^T = latent atoms of the K tile
+        if (tid == 0) {
+            tc_fence_after();
+            for (int mt = 0; mt < DV / 128; ++mt)
+                for (int kk = 0; kk < CK / 16; ++kk)
+                    mma_bf16(tmem + O_COL + 64 * mt,
+                             sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
+                             sdesc(sP + (kk >> 2) * 8192u + (kk & 3) * 32u, 16, 1024), kIdescPV,
+                             (it > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(smem_u32(&bars[1]));
+        }
+        got = warp == 0 ? mbar_wait(smem_u32(&bars[1]), it & 1) : true;
+        ok = __syncthreads_and(got) != 0;  // the K tile and P are free again
+        tc_fence_after();
+    }
 
     // ---- 6. epilogue: thread = one latent channel, 64 heads from TMEM
-    if (ok) {
-        const int g = warp & 3;                 // TMEM lanes 32g .. 32g+31
+    if (ok && c0 < c1) {
+        const int g = warp & 3;  // TMEM lanes 32g .. 32g+31
         for (int t = 0; t < 2; ++t) {
             const int mt = (warp >> 2) * 2 + t;
             const int d = mt * 128 + g * 32 + lane;
@@ -361,7 +457,7 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                 if (nsplit == 1) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float l = lrow[h0 + i];
+                        const float l = lrun[h0 + i];
                         a.out[((size_t)b * H + h0 + i) * DV + d] =
                             l > 0.f ? __uint_as_float(r[i]) / l : 0.f;
                     }
@@ -374,25 +470,25 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
             }
         }
         if (tid < H) {
-            const float m = mrow[tid], l = lrow[tid];
+            const float m = mref[tid], l = lrun[tid];
             if (nsplit == 1) {
-                if (a.lse) a.lse[(size_t)b * H + tid] = l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f
-                                                                : -INFINITY;
+                if (a.lse)
+                    a.lse[(size_t)b * H + tid] =
+                        l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
             } else {
                 const size_t row = ((size_t)b * H + tid) * kMaxSplit + split;
                 a.part_ml[row * 2] = m;
                 a.part_ml[row * 2 + 1] = l;
             }
         }
-    } else {
-        // a bounded wait gave up: flag it, give the MMAs that were issued one
-        // more bounded wait, then free the tensor memory
-        if (tid == 0) {
-            set_status(a.status, KVC_DEV_TIMEOUT);
-            mbar_wait(smem_u32(&bars[0]), 0);
-            if (ok_s) mbar_wait(smem_u32(&bars[1]), 0);
-        }
+    } else if (!ok && tid == 0) {
+        // a bounded wait gave up: flag it, give the issued MMAs one more bounded
+        // wait each, then free the tensor memory
+        set_status(a.status, KVC_DEV_TIMEOUT);
+        mbar_wait(smem_u32(&bars[0]), 0);
+        mbar_wait(smem_u32(&bars[1]), 0);
     }
+    cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -414,21 +510,23 @@ bool tc05_supported(const kvc_config& c, const Shape& sh) {
 int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                           cudaStream_t s) {
     const int total = c.topk + a.window_len;
-    const int nsplit = (total + tc05::CK - 1) / tc05::CK;
+    const int nchunks = (total + tc05::CK - 1) / tc05::CK;
+    // two chunks per CTA: one wave at the batched workload, fewer partials
+    const int cps = nchunks <= 1 ? 1 : 2 + (nchunks - 1) / (2 * kMaxSplit);
+    const int nsplit = nchunks == 0 ? 1 : (nchunks + cps - 1) / cps;
     if (nsplit > kMaxSplit) return -1;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(tc05::attn_tc05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc05::SMEM_BYTES) != cudaSuccess ||
-            prefer_shared(tc05::attn_tc05_kernel) != cudaSuccess)
+                                 (int)tc05::SMEM_BYTES) != cudaSuccess)
             return -1;
         attr_set[dev] = true;
     }
     trace_before("attn_tc05", s);
     tc05::attn_tc05_kernel<<<dim3(nsplit, a.batch), tc05::NT, tc05::SMEM_BYTES, s>>>(
-        a, sh, c.topk, c.sm_scale * 1.4426950408889634f, nsplit,
+        a, sh, c.topk, c.sm_scale * 1.4426950408889634f, nsplit, cps,
         c.scale_fmt == KVC_SCALE_UE4M3);
     trace_after(s);
     return cudaGetLastError() == cudaSuccess ? nsplit : -1;

@@ -319,6 +319,37 @@ __device__ void block_bitonic(Key* k, int p, bool desc) {
 }
 
 // Candidate keys of one sequence staged in shared memory for the finish.
+// One warp sorts up to 64 keys descending (lane l holds positions l and l+32;
+// padding must be 0).  Ascending bitonic network on ~key, shuffles only.
+__device__ __forceinline__ void warp_sort64_desc(unsigned long long& x0, unsigned long long& x1,
+                                                 int lane) {
+    x0 = ~x0;
+    x1 = ~x1;
+#pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j == 32) {  // partner is the lane's other element; k == 64: ascending
+                const unsigned long long lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
+                x0 = lo;
+                x1 = hi;
+            } else {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    unsigned long long& x = r ? x1 : x0;
+                    const int e = lane + 32 * r;
+                    const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+                    const bool asc = (e & k) == 0;
+                    const bool keep_min = ((e & j) == 0) == asc;
+                    x = keep_min ? (x < y ? x : y) : (x < y ? y : x);
+                }
+            }
+        }
+    }
+    x0 = ~x0;
+    x1 = ~x1;
+}
+
 constexpr int kStageKeys = 6144;
 constexpr size_t kFinishSmem =
     (size_t)kStageKeys * 8 + (size_t)kMaxTies * 8 + (size_t)kMaxSelTiles * 4 * 2;
@@ -424,12 +455,24 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
         __syncthreads();
         const int nt = s_nt;
         if (nt <= kMaxTies) {
-            int p2 = 1;
-            while (p2 < nt) p2 <<= 1;
-            for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;  // sorts last
-            __syncthreads();
-            block_bitonic(ties, p2, true);
-            if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;
+            if (nt <= 64) {  // the common case: one warp, no block barriers
+                if (warp == 0) {
+                    unsigned long long x0 = lane < nt ? ties[lane] : 0ull;
+                    unsigned long long x1 = lane + 32 < nt ? ties[lane + 32] : 0ull;
+                    warp_sort64_desc(x0, x1, lane);
+                    const int want = r - 1;  // r-th best key of bin t
+                    const unsigned long long k =
+                        __shfl_sync(0xffffffffu, want < 32 ? x0 : x1, want & 31);
+                    if (lane == 0) s_kstar = (r >= 1 && r <= nt) ? k : ~0ull;
+                }
+            } else {
+                int p2 = 1;
+                while (p2 < nt) p2 <<= 1;
+                for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;  // sorts last
+                __syncthreads();
+                block_bitonic(ties, p2, true);
+                if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;
+            }
             __syncthreads();
             const unsigned long long kstar = s_kstar;
             int run = 0;
@@ -559,7 +602,6 @@ cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, in
         cudaError_t e = cudaFuncSetAttribute(
             index_scan_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
             kScanStages * kStageRows * DI);
-        if (e == cudaSuccess) e = prefer_shared(index_scan_kernel<DI>);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -607,8 +649,6 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         err = cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kFinishSmem);
-        if (err == cudaSuccess) err = prefer_shared(topk_finish_kernel);
-        if (err == cudaSuccess) err = prefer_shared(topk_collect_kernel);
         if (err != cudaSuccess) return err;
         attr_set[dev] = true;
     }

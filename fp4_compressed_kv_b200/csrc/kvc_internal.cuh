@@ -110,15 +110,6 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
 cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3,
                              cudaStream_t s);
 
-// All library kernels ask for the largest shared-memory carve-out, so that
-// consecutive kernels of a step never make the SM reconfigure L1/shared.
-// Called once per kernel and device, before the first launch.
-template <typename F>
-inline cudaError_t prefer_shared(F* kernel) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                (int)cudaSharedmemCarveoutMaxShared);
-}
-
 // ------------------------------------------------------------------ device helpers
 #ifdef __CUDACC__
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t bit) {

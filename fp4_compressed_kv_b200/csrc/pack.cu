@@ -360,26 +360,8 @@ __global__ void pack_commit_kernel(int32_t* n_entries, int batch, int half, int 
 }
 
 template <typename T>
-cudaError_t pack_attrs() {
-    static bool done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || done[dev]) return cudaSuccess;
-    cudaError_t e = cudaSuccess;
-    for (cudaError_t r : {prefer_shared(pack_kernel<T, 2>), prefer_shared(pack_kernel<T, 4>),
-                          prefer_shared(pack_kernel<T, 9>), prefer_shared(pack_kernel<T, 16>),
-                          prefer_shared(pack_small_kernel<T, 1>), prefer_shared(pack_small_kernel<T, 2>),
-                          prefer_shared(pack_small_kernel<T, 3>), prefer_shared(pack_small_kernel<T, 4>),
-                          prefer_shared(pack_commit_kernel)})
-        if (r != cudaSuccess) e = r;
-    if (e == cudaSuccess) done[dev] = true;
-    return e;
-}
-
-template <typename T>
 cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
                           cudaStream_t s) {
-    if (const cudaError_t e = pack_attrs<T>(); e != cudaSuccess) return e;
     const long long entries = (long long)a.batch * (a.n_new / 2);
     if (entries <= 4096) {  // latency-bound append: a warp per entry
         const unsigned grid = (unsigned)((entries + kSmallWarps - 1) / kSmallWarps);

@@ -113,3 +113,22 @@ def test_attention_batch_splits(kvc):
     assert st == 0
     assert_attn_close(out, ref, "batch")
     assert np.max(np.abs(lse - ref_lse)) < 2e-3 * np.abs(ref_lse).max()
+
+
+def test_attention_online_rescale(kvc):
+    """Window keys along head 0's query: their logits exceed the earlier chunks'
+    maximum by far more than the lazy-rescale slack, so the running output in
+    tensor memory must be rescaled; other heads see ordinary logits."""
+    w = synth.WORKLOADS["mla32k"].scaled(context=2 * 1200)
+    inp, rec, ic, n, cfg, cache = _setup(kvc, w)
+    ocfg = oracle_cfg(w)
+    tk = oracle.index_topk(ocfg, inp["idx_q"][0].numpy(), ic, n)
+    q = inp["q"][0]
+    win = inp["windows"][0].clone()
+    win[0, : w.window // 2] = (q[0, 0].float() * 3).to(torch.bfloat16)
+    out, lse, st = _attn(kvc, cfg, cache, q, torch.from_numpy(tk), win, w.window)
+    ref, ref_lse, _ = oracle.sparse_decode(ocfg, f32(q), rec, n, tk, f32(win), w.window)
+    assert st == 0
+    assert ref_lse[0, 0] / np.log(2) > 60  # head 0's maximum jumped by > 8 (log2)
+    assert_attn_close(out, ref, "rescale")
+    assert np.max(np.abs(lse - ref_lse)) < 2e-3 * np.abs(ref_lse).max()
