@@ -81,6 +81,7 @@ attn_simt_kernel(AttnArgs a, Shape sh, int H, int K, float scale_log2, int chunk
                  int nsplit, int ue4m3) {
     extern __shared__ __align__(16) float keys[];  // [kSimtChunk][D]
     __shared__ int kind[kSimtChunk];
+    pdl_wait();
     const int b = blockIdx.z, split = blockIdx.x;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int h = blockIdx.y * 8 + w;
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(128)
 attn_merge_kernel(AttnArgs a, int H, int Dv, int nsplit) {
     __shared__ float s_w[kMaxSplit];
     __shared__ float s_inv, s_lse;
+    pdl_wait();
     const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const size_t row0 = ((size_t)b * H + h) * kMaxSplit;
     if (tid < 32) {
@@ -250,19 +252,19 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
         dim3 grid(nsplit, hblocks, a.batch);
         trace_before("attn_simt", s);
         if (ti)
-            attn_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a, sh, c.n_heads, K, scale_log2,
-                                                                    cps, nsplit, ue4m3);
+            err = launch_pdl(attn_simt_kernel<__nv_bfloat16>, grid, 256, smem, s, a, sh, c.n_heads,
+                             K, scale_log2, cps, nsplit, ue4m3);
         else
-            attn_simt_kernel<float><<<grid, 256, smem, s>>>(a, sh, c.n_heads, K, scale_log2, cps,
-                                                            nsplit, ue4m3);
+            err = launch_pdl(attn_simt_kernel<float>, grid, 256, smem, s, a, sh, c.n_heads, K,
+                             scale_log2, cps, nsplit, ue4m3);
         trace_after(s);
+        if (err != cudaSuccess) return err;
     }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (nsplit > 1) {
         trace_before("attn_merge", s);
-        attn_merge_kernel<<<dim3(c.n_heads, a.batch), 128, 0, s>>>(a, c.n_heads, sh.Dv, nsplit);
+        err = launch_pdl(attn_merge_kernel, dim3(c.n_heads, a.batch), 128, 0, s, a, c.n_heads, sh.Dv,
+                         nsplit);
         trace_after(s);
-        err = cudaGetLastError();
     }
     return err;
 }

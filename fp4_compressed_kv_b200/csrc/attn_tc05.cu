@@ -196,8 +196,6 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
 
     const int b = blockIdx.y, split = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = a.n_entries[b];
-    const bool len_ok = n >= 0 && n <= a.capacity;
     const int total = K + a.window_len;
     const int rb = sh.rb;
     const int c0 = split * cps, c1 = min(c0 + cps, (total + CK - 1) / CK);
@@ -219,6 +217,9 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
     }
     // code-pair table: byte -> (E2M1(low nibble), E2M1(high nibble)) as bf16x2
     lut[tid] = pack_bf16(e2m1_value(tid & 15u), e2m1_value(tid >> 4));
+    pdl_wait();  // everything above was local set-up
+    const int n = a.n_entries[b];
+    const bool len_ok = n >= 0 && n <= a.capacity;
     // Q (64 x 576) once, 128B-swizzled K-major
     {
         const unsigned char* qg = static_cast<const unsigned char*>(a.q) + (size_t)b * H * D * 2;
@@ -445,6 +446,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         tc_fence_after();
     }
 
+    pdl_trigger();  // only the epilogue is left: let the merge be scheduled
+
     // ---- 6. epilogue: thread = one latent channel, 64 heads from TMEM
     if (ok && c0 < c1) {
         const int g = warp & 3;  // TMEM lanes 32g .. 32g+31
@@ -525,11 +528,12 @@ int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& 
         attr_set[dev] = true;
     }
     trace_before("attn_tc05", s);
-    tc05::attn_tc05_kernel<<<dim3(nsplit, a.batch), tc05::NT, tc05::SMEM_BYTES, s>>>(
-        a, sh, c.topk, c.sm_scale * 1.4426950408889634f, nsplit, cps,
-        c.scale_fmt == KVC_SCALE_UE4M3);
+    const cudaError_t e = launch_pdl(tc05::attn_tc05_kernel, dim3(nsplit, a.batch), tc05::NT,
+                                     tc05::SMEM_BYTES, s, a, sh, c.topk,
+                                     c.sm_scale * 1.4426950408889634f, nsplit, cps,
+                                     (int)(c.scale_fmt == KVC_SCALE_UE4M3));
     trace_after(s);
-    return cudaGetLastError() == cudaSuccess ? nsplit : -1;
+    return e == cudaSuccess ? nsplit : -1;
 }
 
 }  // namespace kvc

@@ -185,6 +185,14 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
     const long long lo = (long long)blockIdx.x * per;
     const long long hi = min(lo + per, (long long)a.batch * cap);
     if (lo >= hi) return;
+    // local set-up first, then wait for the previous kernel (the lengths)
+    if (tid == 0) {
+        for (int s = 0; s < kScanStages; ++s)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
+    pdl_wait();
     // flag invalid lengths once (the cursor skips those sequences)
     if (tid == 0)
         for (int b = (int)(lo / cap); b <= (int)((hi - 1) / cap); ++b) {
@@ -193,12 +201,6 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
         }
     ScanCursor cc;  // consumer cursor (all threads)
     if (!cursor_seek(a, lo, hi, cc, (int)(lo / cap))) return;
-    if (tid == 0) {
-        for (int s = 0; s < kScanStages; ++s)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
-        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    }
-    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
     if (tid < PIECES) qs[tid] = __ldg(reinterpret_cast<const int4*>(a.idx_q + (size_t)cc.b * DI) + tid);
     __syncthreads();
     // producer (thread 0): issue the first kScanStages chunks
@@ -289,6 +291,7 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
             qs[tid] = __ldg(reinterpret_cast<const int4*>(a.idx_q + (size_t)cc.b * DI) + tid);
         __syncthreads();
     }
+    pdl_trigger();  // this CTA's rows are done: let the collect kernel be scheduled
     if (!ok && tid == 0) {
         // a bounded wait gave up: flag it and let the copies still in flight land
         set_status(a.status, KVC_DEV_TIMEOUT);
@@ -356,6 +359,7 @@ constexpr size_t kFinishSmem =
 
 __global__ void __launch_bounds__(kThreads)
 topk_collect_kernel(TopkArgs a, int bias, int shift) {
+    pdl_wait();
     __shared__ int sh_warp[kThreads / 32];
     constexpr int PER = kSelTile / kThreads;  // scores per thread
     const int b = blockIdx.y, K = a.topk, tid = threadIdx.x;
@@ -404,6 +408,7 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
     __shared__ int sh_warp[kThreads / 32];
     __shared__ int s_nt, s_low, s_gt;
     __shared__ unsigned long long s_kstar;
+    pdl_wait();
     const int b = blockIdx.x, K = a.topk, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int n = a.n_entries[b];
@@ -592,6 +597,13 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
     for (int i = taken + tid; i < K; i += kThreads) out[i] = -1;
 }
 
+// Clears the per-call counters (a kernel, so the launch chain stays kernel to
+// kernel).
+__global__ void zero_counters_kernel(int32_t* p, int n) {
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
+}
+
 template <int DI>
 cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, int shift,
                         cudaStream_t s) {
@@ -605,9 +617,8 @@ cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, in
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    index_scan_kernel<DI><<<ctas, kThreads, kScanStages * kStageRows * DI, s>>>(a, per, bias,
-                                                                                shift);
-    return cudaGetLastError();
+    return launch_pdl(index_scan_kernel<DI>, ctas, kThreads, (size_t)kScanStages * kStageRows * DI,
+                      s, a, per, bias, shift);
 }
 
 }  // namespace
@@ -616,8 +627,11 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     if (a.batch == 0) return cudaSuccess;
     const int bias = score_bias(a.di), shift = score_shift(a.di);
     // zero the histograms and the finished-CTA counters (adjacent in the workspace)
-    cudaError_t err =
-        cudaMemsetAsync(a.counters, 0, topk_counter_words(a.batch) * sizeof(int32_t), s);
+    const int words = (int)topk_counter_words(a.batch);
+    trace_before("topk_zero", s);
+    cudaError_t err = launch_pdl(zero_counters_kernel, (words + 1023) / 1024, 256, 0, s,
+                                 a.counters, words);
+    trace_after(s);
     if (err != cudaSuccess) return err;
     // one wave: 2 CTAs per SM (96 KB ring + 8 KB histogram each for Di = 128),
     // equal row slices
@@ -642,9 +656,9 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     dim3 grid(sel_tiles(a.capacity), a.batch);
     trace_before("topk_collect", s);
-    topk_collect_kernel<<<grid, kThreads, 0, s>>>(a, bias, shift);
+    err = launch_pdl(topk_collect_kernel, grid, kThreads, 0, s, a, bias, shift);
     trace_after(s);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (err != cudaSuccess) return err;
     static bool attr_set[64] = {};
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         err = cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -653,9 +667,9 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
         attr_set[dev] = true;
     }
     trace_before("topk_finish", s);
-    topk_finish_kernel<<<a.batch, kThreads, kFinishSmem, s>>>(a, bias, shift);
+    err = launch_pdl(topk_finish_kernel, a.batch, kThreads, kFinishSmem, s, a, bias, shift);
     trace_after(s);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace kvc

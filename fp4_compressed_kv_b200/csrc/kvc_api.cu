@@ -90,6 +90,7 @@ void trace_after(cudaStream_t s) {
 namespace {
 __global__ void codec_kernel(const float* __restrict__ x, int64_t n, uint8_t* __restrict__ out,
                              int e4m3) {
+    pdl_wait();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float v = x[i];
@@ -110,13 +111,22 @@ cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3, 
     int64_t blocks = (n + 255) / 256;
     if (blocks > 4096) blocks = 4096;
     trace_before("fp4_codec", s);
-    codec_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, n, out, e4m3);
+    const cudaError_t e = launch_pdl(codec_kernel, (unsigned)blocks, 256, 0, s, x, n, out, e4m3);
     trace_after(s);
-    return cudaGetLastError();
+    return e;
+}
+
+namespace {
+// Copies a Reuse layer's borrowed top-K rows (a kernel, so the launch chain
+// of a layer group stays kernel to kernel).
+__global__ void copy_topk_kernel(const int32_t* __restrict__ src, int32_t* __restrict__ dst,
+                                 int n) {
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        dst[i] = src[i];
 }
 
 // ------------------------------------------------------------------ workspace
-namespace {
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -353,9 +363,13 @@ kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers, const int32
             if (st != KVC_OK) return st;
             head = l;
         } else {
-            if (cudaMemcpyAsync(tk, topk + (size_t)head * B * K, B * K * 4, cudaMemcpyDeviceToDevice,
-                                s) != cudaSuccess)
-                return KVC_ERR_CUDA;
+            const int cnt = (int)(B * K);
+            trace_before("copy_topk", s);
+            const cudaError_t e = launch_pdl(copy_topk_kernel, (cnt + 1023) / 1024, 256, 0, s,
+                                             static_cast<const int32_t*>(topk + (size_t)head * B * K),
+                                             tk, cnt);
+            trace_after(s);
+            if (e != cudaSuccess) return KVC_ERR_CUDA;
         }
         st = run_attn(*cfg, sh, static_cast<const unsigned char*>(q) + l * q_stride, cache, tk,
                       windows ? static_cast<const unsigned char*>(windows) + l * w_stride : nullptr,

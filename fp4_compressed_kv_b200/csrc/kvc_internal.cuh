@@ -110,8 +110,39 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
 cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3,
                              cudaStream_t s);
 
+// Every library kernel is launched with programmatic stream serialization:
+// the long kernels signal griddepcontrol.launch_dependents once their main
+// loop is done, so the next kernel's CTAs are scheduled while they drain; each
+// kernel does only local set-up (shared memory, tensor memory, barriers)
+// before waiting for its predecessor with griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------------ device helpers
 #ifdef __CUDACC__
+// Lets the next kernel on the stream be scheduled (it still waits for this
+// one to complete before it reads anything this one writes).
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;\n");
+}
+// Waits until the previous kernel on the stream has completed and its writes
+// are visible (returns at once when it was not launched as a dependent).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t bit) {
     if (st) atomicOr(st, bit);
 }

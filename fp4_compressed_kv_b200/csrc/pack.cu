@@ -62,6 +62,12 @@ struct Chunk<__nv_bfloat16> {
         v = __ldcs(reinterpret_cast<const uint4*>(p));
     }
     __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void load_shared(const __nv_bfloat16* p) {
+        v = *reinterpret_cast<const uint4*>(p);
+    }
+    __device__ __forceinline__ void store_shared(__nv_bfloat16* p) const {
+        *reinterpret_cast<uint4*>(p) = v;
+    }
     __device__ __forceinline__ float get(int t) const {
         const uint32_t w = t < 2 ? v.x : t < 4 ? v.y : t < 6 ? v.z : v.w;
         return (t & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
@@ -75,6 +81,14 @@ struct Chunk<float> {
         b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
     }
     __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void load_shared(const float* p) {
+        a = reinterpret_cast<const float4*>(p)[0];
+        b = reinterpret_cast<const float4*>(p)[1];
+    }
+    __device__ __forceinline__ void store_shared(float* p) const {
+        reinterpret_cast<float4*>(p)[0] = a;
+        reinterpret_cast<float4*>(p)[1] = b;
+    }
     __device__ __forceinline__ float get(int t) const {
         const float4& q = t < 4 ? a : b;
         const int u = t & 3;
@@ -89,6 +103,26 @@ __device__ __forceinline__ void load8_gate(const float* p, float v[8]) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+// E2M1 rounding input fl(x / s), given r = 1/s rounded.  x * r lies within
+// about 2 fp32 ulps of the correctly rounded quotient (two roundings of
+// 2^-24 relative each, quotients below 8), so both round to the same E2M1
+// code unless x * r sits within a few ulps of one of the grid's rounding
+// midpoints {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5}.  The map below sends every
+// midpoint to k + 1/2; near one of them the quotient is divided out exactly.
+__device__ __forceinline__ float e2m1_input(float x, float s, float r) {
+    const float q = __fmul_rn(x, r);
+    const float a = fabsf(q);
+    const float u = a < 2.f ? a + a : (a < 4.f ? a : 0.5f * a);
+    return fabsf(u - floorf(u) - 0.5f) < 1.0e-5f ? __fdiv_rn(x, s) : q;
+}
+
+// fl(x / s) for the E2M1 code (0 when s is 0); r = 1/s rounded, `fast` when r
+// is finite.
+__device__ __forceinline__ float e2m1_quotient(float x, float s, float r, bool fast) {
+    if (!(s > 0.f)) return 0.f;
+    return fast ? e2m1_input(x, s, r) : __fdiv_rn(x, s);
+}
+
 constexpr int kThreads = 256;
 constexpr int kTeams = kThreads / 8;  // entries per CTA
 constexpr int kTailBytes = 528;       // >= 128 groups x 4 bytes, padded
@@ -98,6 +132,7 @@ constexpr int kMaxChunks = 128;       // D <= 1024
 template <typename T, int MAXJ>
 __global__ void __launch_bounds__(kThreads)
 pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
+    pdl_wait();
     __shared__ __align__(16) uint8_t tail_smem[kTeams][kTailBytes];
     __shared__ float cmax_smem[kTeams][kMaxChunks];  // only for groups wider than a team pass
     const int lane = threadIdx.x & 31;
@@ -208,12 +243,14 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
             sbyte = e4m3_from_f32(s);
             s = e4m3_to_f32(sbyte);
         }
+        const float r = __frcp_rn(s);
+        const bool fast = r < 3.0e38f;
         float v[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             float x = __fmaf_rn(w0, k0[j].get(t), __fmul_rn(w1, k1[j].get(t)));
             if (!isfinite(x)) x = 0.f;
-            const float q = s > 0.f ? __fdiv_rn(x, s) : 0.f;
+            const float q = e2m1_quotient(x, s, r, fast);
             v[t] = fminf(fmaxf(q, -6.f), 6.f);
         }
         *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
@@ -240,16 +277,26 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
 }
 
 // Small appends (decode: one pair per sequence): one warp per entry so the
-// work of a few dozen entries spreads over many SMs.  Lanes 0-7 form the gate
-// team in exactly the order above (lane l sums chunks l, l+8, ... then the
-// xor tree over 4, 2, 1 inside the team); all 32 lanes then quantise, lane l
-// owning chunks l, l+32, l+64.  Same arithmetic, same bits as pack_kernel.
+// work of a few dozen entries spreads over many SMs.  The whole warp first
+// stages the token pair and the gate in shared memory (one round trip to
+// HBM); lanes 0-7 then form the gate team in exactly the order above (lane l
+// sums chunks l, l+8, ... then the xor tree over 4, 2, 1 inside the team), and
+// all 32 lanes quantise from registers, lane l owning chunks l, l+32, l+64.
+// Same arithmetic, same bits as pack_kernel.  With one pair per sequence the
+// warp also commits the sequence's new length (no other warp touches it).
 constexpr int kSmallWarps = 4;
+
+template <typename T>
+__host__ __device__ constexpr size_t small_stage_bytes(int D) {
+    return (size_t)D * (2 * sizeof(T) + sizeof(float));  // k0, k1, gate
+}
 
 template <typename T, int MAXJ>
 __global__ void __launch_bounds__(kSmallWarps * 32)
 pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
+    extern __shared__ __align__(16) unsigned char stage_smem[];
     __shared__ __align__(16) uint8_t tail_smem[kSmallWarps][kTailBytes];
+    pdl_wait();
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long e = (long long)blockIdx.x * kSmallWarps + wid;
     const int half = a.n_new >> 1;
@@ -264,18 +311,47 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     const long long pos = (long long)base + i;
     const T* k0p = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 2 * i) * D;
     const T* k1p = k0p + D;
+    T* s0 = reinterpret_cast<T*>(stage_smem + wid * small_stage_bytes<T>(D));
+    T* s1 = s0 + D;
+    float* sg = reinterpret_cast<float*>(s1 + D);
+
+    // every load of the entry in flight at once
+    Chunk<T> x0[MAXJ], x1[MAXJ];
+    float4 g0[MAXJ], g1[MAXJ];
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nchunk) {
+            x0[j].load(k0p + 8 * c);
+            x1[j].load(k1p + 8 * c);
+            g0[j] = __ldg(reinterpret_cast<const float4*>(a.gate + 8 * c));
+            g1[j] = __ldg(reinterpret_cast<const float4*>(a.gate + 8 * c) + 1);
+        } else {
+            x0[j].zero();
+            x1[j].zero();
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nchunk) {
+            x0[j].store_shared(s0 + 8 * c);
+            x1[j].store_shared(s1 + 8 * c);
+            reinterpret_cast<float4*>(sg + 8 * c)[0] = g0[j];
+            reinterpret_cast<float4*>(sg + 8 * c)[1] = g1[j];
+        }
+    }
+    __syncwarp();
 
     float acc = 0.f;
     if (lane < 8) {
         for (int c = lane; c < nchunk; c += 8) {
-            Chunk<T> x0, x1;
-            x0.load(k0p + 8 * c);
-            x1.load(k1p + 8 * c);
-            float g[8];
-            load8_gate(a.gate + 8 * c, g);
+            Chunk<T> y0, y1;
+            y0.load_shared(s0 + 8 * c);
+            y1.load_shared(s1 + 8 * c);
 #pragma unroll
             for (int t = 0; t < 8; ++t)
-                acc = __fmaf_rn(g[t], __fsub_rn(x0.get(t), x1.get(t)), acc);
+                acc = __fmaf_rn(sg[8 * c + t], __fsub_rn(y0.get(t), y1.get(t)), acc);
         }
     }
     acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
@@ -297,19 +373,11 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     for (int j = 0; j < MAXJ; ++j) {
         const int c = lane + 32 * j;
         const bool active = c < nchunk;
-        Chunk<T> x0, x1;
-        if (active) {
-            x0.load(k0p + 8 * c);
-            x1.load(k1p + 8 * c);
-        } else {
-            x0.zero();
-            x1.zero();
-        }
         float x[8];
         float m = 0.f;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            float v = __fmaf_rn(w0, x0.get(t), __fmul_rn(w1, x1.get(t)));
+            float v = __fmaf_rn(w0, x0[j].get(t), __fmul_rn(w1, x1[j].get(t)));
             if (!isfinite(v)) {
                 if (active) bad = true;
                 v = 0.f;
@@ -325,10 +393,12 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
             sbyte = e4m3_from_f32(s);
             s = e4m3_to_f32(sbyte);
         }
+        const float r = __frcp_rn(s);
+        const bool fast = r < 3.0e38f;
         float v[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            const float q = s > 0.f ? __fdiv_rn(x[t], s) : 0.f;
+            const float q = e2m1_quotient(x[t], s, r, fast);
             v[t] = fminf(fmaxf(q, -6.f), 6.f);
         }
         *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
@@ -350,47 +420,63 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
         *(reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di) + lane) = v;
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
+    if (half == 1 && lane == 0) a.n_entries[b] = base + 1;
 }
 
 __global__ void pack_commit_kernel(int32_t* n_entries, int batch, int half, int capacity) {
+    pdl_wait();
     for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
         const int n = n_entries[b];
         if (n >= 0 && n + half <= capacity) n_entries[b] = n + half;
     }
 }
 
+template <typename T, int MAXJ>
+cudaError_t launch_small(unsigned grid, size_t smem, cudaStream_t s, const PackArgs& a,
+                         const Shape& sh, int ue4m3, int di) {
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            pack_small_kernel<T, MAXJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(pack_small_kernel<T, MAXJ>, grid, kSmallWarps * 32, smem, s, a, sh, ue4m3,
+                      di);
+}
+
 template <typename T>
 cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
                           cudaStream_t s) {
     const long long entries = (long long)a.batch * (a.n_new / 2);
+    cudaError_t err;
     if (entries <= 4096) {  // latency-bound append: a warp per entry
         const unsigned grid = (unsigned)((entries + kSmallWarps - 1) / kSmallWarps);
         const int maxj = (sh.D / 8 + 31) / 32;
+        const size_t smem = kSmallWarps * small_stage_bytes<T>(sh.D);
         trace_before("pack", s);
         if (maxj <= 1)
-            pack_small_kernel<T, 1><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+            err = launch_small<T, 1>(grid, smem, s, a, sh, ue4m3, di);
         else if (maxj <= 2)
-            pack_small_kernel<T, 2><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+            err = launch_small<T, 2>(grid, smem, s, a, sh, ue4m3, di);
         else if (maxj <= 3)
-            pack_small_kernel<T, 3><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+            err = launch_small<T, 3>(grid, smem, s, a, sh, ue4m3, di);
         else
-            pack_small_kernel<T, 4><<<grid, kSmallWarps * 32, 0, s>>>(a, sh, ue4m3, di);
+            err = launch_small<T, 4>(grid, smem, s, a, sh, ue4m3, di);
         trace_after(s);
-        return cudaGetLastError();
+        return err;
     }
     const unsigned grid = (unsigned)((entries + kTeams - 1) / kTeams);
     const int maxj = (sh.D / 8 + 7) / 8;
     trace_before("pack", s);
     if (maxj <= 2)
-        pack_kernel<T, 2><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+        err = launch_pdl(pack_kernel<T, 2>, grid, kThreads, 0, s, a, sh, ue4m3, di);
     else if (maxj <= 4)
-        pack_kernel<T, 4><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+        err = launch_pdl(pack_kernel<T, 4>, grid, kThreads, 0, s, a, sh, ue4m3, di);
     else if (maxj <= 9)
-        pack_kernel<T, 9><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+        err = launch_pdl(pack_kernel<T, 9>, grid, kThreads, 0, s, a, sh, ue4m3, di);
     else
-        pack_kernel<T, 16><<<grid, kThreads, 0, s>>>(a, sh, ue4m3, di);
+        err = launch_pdl(pack_kernel<T, 16>, grid, kThreads, 0, s, a, sh, ue4m3, di);
     trace_after(s);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace
@@ -404,11 +490,12 @@ cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
                           ? launch_pack_t<__nv_bfloat16>(sh, a, ue, c.idx_dim, s)
                           : launch_pack_t<float>(sh, a, ue, c.idx_dim, s);
     if (err != cudaSuccess) return err;
+    if (half == 1 && a.batch <= 4096) return cudaSuccess;  // committed by the append kernel
     trace_before("pack_commit", s);
-    pack_commit_kernel<<<(a.batch + 255) / 256, 256, 0, s>>>(a.n_entries, a.batch, half,
-                                                             a.capacity);
+    err = launch_pdl(pack_commit_kernel, (a.batch + 255) / 256, 256, 0, s, a.n_entries, a.batch,
+                     half, a.capacity);
     trace_after(s);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace kvc

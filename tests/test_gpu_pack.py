@@ -122,3 +122,52 @@ def test_pack_team_and_warp_variants(kvc, name, batch, context):
     cache2, _ = _gpu_pack(kvc, w, inp["tokens"][:, :64].cuda().contiguous(), inp["gate"].cuda(),
                           inp["idx_k"][:, :32].cuda().contiguous(), capacity=w.entries, chunks=2)
     assert np.array_equal(cache2.records.cpu().numpy()[:, :32], rec[:, :32])
+
+
+def _midpoint_tokens(w, batch, pairs, seed):
+    """Token pairs (k, k) whose entries land on and next to the E2M1 rounding
+    midpoints: each group holds 6*s (so the group scale is s exactly), then
+    s times midpoints {0.25, ..., 5}, grid points, and their nearest neighbours
+    in the token dtype.  With a zero gate both weights are 1/2 and the entry is
+    k exactly, so x / s falls on a midpoint or a unit in the last place away."""
+    rng = np.random.default_rng(seed)
+    dt = w.torch_dtype
+    D = w.dim
+    # midpoints and grid points below the group maximum 6 (which sets s)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0])
+    scales = np.array([1.0, 0.75, 0.125, 3.0, 0.009765625])  # exact in E4M3, fp32 and bf16
+    ent = np.empty((batch, pairs, D), np.float32)
+    for b in range(batch):
+        s = scales[rng.integers(0, len(scales), pairs)][:, None]
+        v = torch.from_numpy((rng.choice(mids, (pairs, D)) * s).astype(np.float32)).to(dt)
+        step = rng.integers(-1, 2, (pairs, D))  # -1, 0, +1 units in the last place
+        up = torch.nextafter(v, torch.full_like(v, np.inf))
+        dn = torch.nextafter(v, torch.full_like(v, -np.inf))
+        v = torch.where(torch.from_numpy(step == 1), up, torch.where(torch.from_numpy(step == -1),
+                                                                     dn, v))
+        v = v.float().numpy() * rng.choice([-1.0, 1.0], (pairs, D))
+        for g0 in list(range(0, w.latent, w.group)) + list(range(w.latent, D, w.group)):
+            v[:, g0] = 6.0 * s[:, 0]
+        ent[b] = v
+    tok = torch.from_numpy(np.repeat(ent, 2, axis=1)).to(dt)
+    return tok
+
+
+@pytest.mark.parametrize("name,pairs", [("tiny", 300), ("tiny", 4100), ("mla32k", 200),
+                                        ("mla32k", 2100)])
+def test_pack_rounding_midpoints(kvc, name, pairs):
+    """Both append kernels (warp per entry, 8 lanes per entry) against the
+    oracle's exact division on quotients at and beside the rounding midpoints."""
+    w = synth.WORKLOADS[name]
+    batch = 2
+    tok = _midpoint_tokens(w, batch, pairs, seed=7)
+    assert torch.equal(tok[:, 0::2], tok[:, 1::2])
+    gate = torch.zeros(w.dim, dtype=torch.float32)
+    idx = torch.zeros(batch, pairs, w.idx_dim, dtype=torch.int8)
+    rec, ic, n, ost = oracle_pack(w, tok, gate, idx)
+    assert ost == 0
+    cache, st = _gpu_pack(kvc, w, tok.cuda(), gate.cuda(), idx.cuda())
+    assert st == 0
+    got = cache.records.cpu().numpy()
+    diff = np.argwhere(got != rec)
+    assert diff.size == 0, f"{len(diff)} bytes differ, first {diff[:5].tolist()}"
