@@ -51,7 +51,55 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--hier", type=int, default=0,
+                   help="hierarchical indexer: blocks kept (0 = off; the pages use 2048 of 8)")
+    p.add_argument("--hier-block", type=int, default=8)
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the hierarchical-indexer side measurement")
     return p.parse_args()
+
+
+def time_group(w, steps, warmup, hier_blocks, hier_block, dev):
+    """Device ms per decode step of workload w's layer group (no pack), K
+    steps in one CUDA graph; the CSA2 group and the 1M stack with and without
+    the hierarchical indexer."""
+    import torch
+    from fp4_compressed_kv_b200 import kvc, synth
+    cfg = kvc.config_for(w)
+    inp = synth.make_inputs(w, dev)
+    cache = kvc.Cache(cfg, w.batch, w.entries, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    kvc.pack(cfg, inp["tokens"], inp["gate"], inp["idx_k"], cache, status=st)
+    del inp["tokens"]
+    L, B, H = w.layers, w.batch, w.heads
+    out = torch.empty(L, B, H, w.latent, device=dev)
+    lse = torch.empty(L, B, H, device=dev)
+    tk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
+    ws = kvc.workspace(cfg, B, w.entries, device=dev, hier_blocks=hier_blocks,
+                       hier_block=hier_block)
+
+    def step():
+        kvc.layer_group_step(cfg, list(w.modes), inp["q"], inp["idx_q"], inp["windows"],
+                             w.window, cache, out, tk, ws, lse=lse, status=st,
+                             hier_blocks=hier_blocks, hier_block=hier_block)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(steps):
+            step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    return ms
 
 
 # ----------------------------------------------------------------------------- bytes
@@ -271,7 +319,7 @@ def run_ours(args):
     torch.cuda.empty_cache()
     gate = inp["gate"]
     q, idx_q, windows = inp["q"], inp["idx_q"], inp["windows"]
-    ws = kvc.workspace(cfg, B, cap, device=dev)
+    ws = kvc.workspace(cfg, B, cap, device=dev, hier_blocks=args.hier, hier_block=args.hier_block)
     out = torch.empty(L, B, H, w.latent, device=dev)
     lse = torch.empty(L, B, H, device=dev)
     topk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
@@ -284,7 +332,8 @@ def run_ours(args):
     def step(s):
         kvc.pack(cfg, pair_tok[s], gate, pair_idx[s], cache, status=status)
         kvc.layer_group_step(cfg, modes, q, idx_q, windows, w.window, cache, out, topk, ws,
-                             lse=lse, status=status)
+                             lse=lse, status=status, hier_blocks=args.hier,
+                             hier_block=args.hier_block)
 
     for s in range(args.warmup):
         step(s)
@@ -417,7 +466,8 @@ def run_ours(args):
             didx.copy_(hidx, non_blocking=True)
             kvc.pack(cfg, dtok, gate, didx, cache, status=status)
             kvc.layer_group_step(cfg, modes, dq, diq, windows, w.window, cache, out, topk, ws,
-                                 lse=lse, status=status)
+                                 lse=lse, status=status, hier_blocks=args.hier,
+                                 hier_block=args.hier_block)
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
 
@@ -439,6 +489,22 @@ def run_ours(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(te_ms / reps, 4)}
 
+    # ---- the hierarchical indexer (2048 blocks of 8) on the CSA2 group and the
+    # 1M-token stack, against the plain group step (device time per step)
+    extra = None
+    if not args.no_extra and world == 1 and args.hier == 0:
+        torch.cuda.empty_cache()
+        extra = {}
+        for name in ("csa2group", "stack1m"):
+            wx = synth.WORKLOADS[name]
+            plain = time_group(wx, 10, 3, 0, 8, dev)
+            hier = time_group(wx, 10, 3, 2048, 8, dev)
+            extra[name] = {"ms_per_step_plain": round(plain, 4), "ms_per_step_hier": round(hier, 4),
+                           "query_tokens_per_s_plain": round(wx.batch / (plain * 1e-3), 1),
+                           "query_tokens_per_s_hier": round(wx.batch / (hier * 1e-3), 1),
+                           "hier": "2048 blocks of 8 entries"}
+            torch.cuda.empty_cache()
+
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -458,6 +524,8 @@ def run_ours(args):
                    "heads": H, "latent": w.latent, "rope": w.rope, "group": w.group,
                    "scale": "ue4m3" if w.scale_fmt == 1 else "f32", "topk": w.topk,
                    "window": w.window, "idx_dim": w.idx_dim, "parallelism": f"dp{world}",
+                   "hier_indexer": (f"{args.hier} blocks of {args.hier_block}" if args.hier
+                                    else "off"),
                    "l2": "inputs larger than L2 (indexer scan reads %.0f MB per step)"
                          % (B * scan_bytes(w, N0) * heads_layers / 1e6),
                    "timing": "K steps in one CUDA graph, CUDA events, max over ranks; "
@@ -475,6 +543,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk,
+        "hier_indexer": extra,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

@@ -36,7 +36,7 @@ constexpr int KGRP = CK / 8;                    // 12 groups of 8 keys
 constexpr uint32_t Q_BYTES = NATOM * 8 * 1024;  // 64 rows: 8 row groups per atom
 constexpr uint32_t K_ATOM = KGRP * 1024;        // one channel atom of the K tile
 constexpr uint32_t K_BYTES = NATOM * K_ATOM;
-constexpr uint32_t RAW_STRIDE = 320;            // record bytes reserved per key
+constexpr uint32_t RAW_STRIDE = 368;            // record bytes reserved per key (G >= 8)
 constexpr uint32_t RAW_BYTES = CK * RAW_STRIDE;
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
@@ -280,22 +280,28 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
             cp_async_wait_all();
         }
         __syncthreads();
-        // ---- 2. dequantise records into the swizzled K tile.  UE4M3 scales, groups
-        // of >= 32: 32 channels per item, a byte of two codes -> bf16x2 table
-        // entry times the bf16x2 scale (the products have at most 6 significant
-        // bits, so the bf16 multiply is exact).
-        if (ue4m3 && sh.lpg >= 4) {
+        // ---- 2. dequantise records into the swizzled K tile.  UE4M3 scales: 32
+        // channels per item, a byte of two codes -> bf16x2 table entry times
+        // the bf16x2 scale of its group (the products have at most 6
+        // significant bits, so the bf16 multiply is exact).  Groups of >= 32
+        // share one scale per item; groups of 8 or 16 take one per 8 channels.
+        if (ue4m3) {
+            const int lpg = sh.lpg;
             for (int p = tid; p < CK * (D / 32); p += NT) {
                 const int s = p / (D / 32), i4 = p - s * (D / 32);
                 if (kind[s] < 0) continue;
                 const unsigned char* rec = raw + s * RAW_STRIDE;
                 const uint4 codes = *reinterpret_cast<const uint4*>(rec + i4 * 16);
-                const float sc = e4m3_to_f32(rec[sh.code_bytes + (4 * i4) / sh.lpg]);
-                const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc, sc);
+                const float sc = e4m3_to_f32(rec[sh.code_bytes + (4 * i4) / lpg]);
+                __nv_bfloat162 s2 = __floats2bfloat162_rn(sc, sc);
                 const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
                 const uint32_t row = sK + (i4 >> 1) * K_ATOM;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
+                    if (lpg < 4 && u > 0) {
+                        const float su = e4m3_to_f32(rec[sh.code_bytes + (4 * i4 + u) / lpg]);
+                        s2 = __floats2bfloat162_rn(su, su);
+                    }
                     uint32_t w[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {

@@ -124,15 +124,59 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
         if ((i & 255) == 255 && now_ns() - t0 > 2000000000ull) return false;
     }
 }
+// The indexer rows are read once per scan: bulk copies carry an L2
+// evict-first policy so the stream does not push the scores, candidates and
+// attention records out of L2.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1], %2, [%3], %4;\n" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+        : "memory");
+}
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
                  : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
+    bulk_copy(dst, src, bytes, bar, evict_first_policy());
+}
+
+// Rows [row, row + rows) of sequence b into shared memory at dst, completing
+// on mbarrier bar: one bulk copy, or in pool mode one per run of rows inside
+// a pool block (the pool's rows are whole blocks of consecutive entries).
+__device__ __forceinline__ void load_rows(const TopkArgs& a, int b, int row, int rows, int di,
+                                          uint32_t dst, uint32_t bar) {
+    const int8_t* base = a.idx_k + (size_t)b * a.idx_capacity * di;
+    if (!a.pool_blocks) {
+        bulk_load(dst, base + (size_t)row * di, (uint32_t)rows * di, bar);
+        return;
+    }
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar),
+                 "r"((uint32_t)rows * di)
+                 : "memory");
+    const int32_t* blocks = a.pool_blocks + (size_t)b * a.pool_keep;
+    const uint64_t pol = evict_first_policy();
+    for (int r = row; r < row + rows;) {
+        const int blk = r / a.pool_block, off = r - blk * a.pool_block;
+        const int len = min(a.pool_block - off, row + rows - r);
+        const long long e = (long long)blocks[blk] * a.pool_block + off;
+        bulk_copy(dst + (uint32_t)(r - row) * di, base + e * di, (uint32_t)len * di, bar, pol);
+        r += len;
+    }
+}
+
+// Top-K output index of row p of sequence b: the entry itself, or in pool
+// mode the pool row's entry.
+__device__ __forceinline__ int out_index(const TopkArgs& a, int b, int p) {
+    if (!a.pool_blocks) return p;
+    const int blk = p / a.pool_block;
+    return a.pool_blocks[(size_t)b * a.pool_keep + blk] * a.pool_block + (p - blk * a.pool_block);
 }
 
 // Cursor over this CTA's rows, chunked per sequence: rows [row, end) of
@@ -209,8 +253,7 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
     if (tid == 0) {
         for (int s = 0; s < kScanStages && pmore; ++s) {
             const int rows = min(kStageRows, pc.end - pc.row);
-            bulk_load(smem_addr(ring + s * STAGE),
-                      a.idx_k + ((size_t)pc.b * cap + pc.row) * DI, (uint32_t)rows * DI,
+            load_rows(a, pc.b, pc.row, rows, DI, smem_addr(ring + s * STAGE),
                       smem_addr(&full[s]));
             pc.row += rows;
             if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
@@ -247,8 +290,7 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
         __syncthreads();  // stage s is free again
         if (tid == 0 && pmore) {
             const int prow = min(kStageRows, pc.end - pc.row);
-            bulk_load(smem_addr(ring + s * STAGE),
-                      a.idx_k + ((size_t)pc.b * cap + pc.row) * DI, (uint32_t)prow * DI,
+            load_rows(a, pc.b, pc.row, prow, DI, smem_addr(ring + s * STAGE),
                       smem_addr(&full[s]));
             pc.row += prow;
             if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
@@ -359,10 +401,12 @@ constexpr size_t kFinishSmem =
 
 __global__ void __launch_bounds__(kThreads)
 topk_collect_kernel(TopkArgs a, int bias, int shift) {
-    pdl_wait();
     __shared__ int sh_warp[kThreads / 32];
-    constexpr int PER = kSelTile / kThreads;  // scores per thread
+    constexpr int PER = kSelTile / kThreads;     // scores per thread (32)
+    constexpr int WROWS = kSelTile / (kThreads / 32);  // rows per warp (1024)
+    pdl_wait();
     const int b = blockIdx.y, K = a.topk, tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
     const int n = a.n_entries[b];
     if (n < 0 || n > a.capacity || n <= K) return;
     const int ntiles = (n + kSelTile - 1) / kSelTile;
@@ -372,28 +416,35 @@ topk_collect_kernel(TopkArgs a, int bias, int shift) {
     const int32_t* sc = a.scores + (size_t)b * a.capacity;
     const int ctiles = sel_tiles(a.capacity);
     unsigned long long* cand = a.cands + ((size_t)b * ctiles + tile) * kSelTile;
-    // compact this tile's candidates (bins >= t) in index order
+    // warp w owns rows [w*1024, (w+1)*1024) of the tile; lane l reads rows
+    // i*32 + l, so every load of the warp is one contiguous 128-byte line
+    const int r0 = tile * kSelTile + warp * WROWS + lane;
     int v[PER];
-    const int j0 = tile * kSelTile + tid * PER;
-    if (j0 + PER <= n && ((reinterpret_cast<uintptr_t>(sc + j0) & 15) == 0)) {
 #pragma unroll
-        for (int u = 0; u < PER / 4; ++u) {
-            const int4 x = __ldcg(reinterpret_cast<const int4*>(sc + j0) + u);
-            v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
-        }
-    } else {
-#pragma unroll
-        for (int u = 0; u < PER; ++u) v[u] = (j0 + u < n) ? __ldcg(sc + j0 + u) : 0;
-    }
+    for (int i = 0; i < PER; ++i) v[i] = (r0 + 32 * i < n) ? __ldcg(sc + r0 + 32 * i) : 0;
     unsigned take = 0;
 #pragma unroll
-    for (int u = 0; u < PER; ++u)
-        if (j0 + u < n && score_bin(v[u], bias, shift) >= t) take |= 1u << u;
-    int pos;
-    const int total = block_excl_scan(__popc(take), &pos, sh_warp);
+    for (int i = 0; i < PER; ++i)
+        if (r0 + 32 * i < n && score_bin(v[i], bias, shift) >= t) take |= 1u << i;
+    int wc = __popc(take);
 #pragma unroll
-    for (int u = 0; u < PER; ++u)
-        if (take & (1u << u)) cand[pos++] = make_key(v[u], j0 + u, bias);
+    for (int o = 16; o >= 1; o >>= 1) wc += __shfl_xor_sync(0xffffffffu, wc, o);
+    if (lane == 0) sh_warp[warp] = wc;
+    __syncthreads();
+    int base = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        base += w < warp ? sh_warp[w] : 0;
+        total += sh_warp[w];
+    }
+    // compact in index order: row-major over (i, lane) inside the warp
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const unsigned m = __ballot_sync(0xffffffffu, (take >> i) & 1u);
+        if ((take >> i) & 1u) cand[base + __popc(m & lt)] = make_key(v[i], r0 + 32 * i, bias);
+        base += __popc(m);
+    }
     if (tid == 0) a.tile_count[(size_t)b * ctiles + tile] = total;
 }
 
@@ -418,7 +469,7 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
         return;
     }
     if (n <= K) {
-        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
+        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? out_index(a, b, i) : -1;
         return;
     }
     const int ntiles = (n + kSelTile - 1) / kSelTile;
@@ -443,15 +494,20 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
     __syncthreads();
     const int r = K - above;  // entries to take from bin t
     if (M <= kStageKeys) {
-        // every candidate key, in index order, with one round of parallel loads
+        // every candidate key, in index order: all loads in flight at once,
+        // then the keys of bin t gathered from shared memory
+#pragma unroll 4
         for (int p = tid; p < M; p += kThreads) {
             int lo = 0, hi = ntiles - 1;  // last tile with off <= p
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
                 if (off[mid] <= p) lo = mid; else hi = mid - 1;
             }
-            const unsigned long long k = __ldcg(cb + (size_t)lo * kSelTile + (p - off[lo]));
-            stage[p] = k;
+            stage[p] = __ldcg(cb + (size_t)lo * kSelTile + (p - off[lo]));
+        }
+        __syncthreads();
+        for (int p = tid; p < M; p += kThreads) {
+            const unsigned long long k = stage[p];
             if ((int)((k >> 32) >> shift) == t) {
                 const int q = atomicAdd(&s_nt, 1);
                 if (q < kMaxTies) ties[q] = k;
@@ -486,7 +542,7 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
                 const bool sel = p < M && stage[p] >= kstar;
                 int ex;
                 const int tot = block_excl_scan(sel ? 1 : 0, &ex, sh_warp);
-                if (sel && run + ex < K) out[run + ex] = key_index(stage[p]);
+                if (sel && run + ex < K) out[run + ex] = out_index(a, b, key_index(stage[p]));
                 run += tot;
             }
             for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
@@ -544,7 +600,7 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
                     const bool sel = i < cnt[ti] && k >= kstar;
                     const unsigned m = __ballot_sync(0xffffffffu, sel);
                     const int p = o + __popc(m & ((1u << lane) - 1u));
-                    if (sel && p < K) out[p] = key_index(k);
+                    if (sel && p < K) out[p] = out_index(a, b, key_index(k));
                     o += __popc(m);
                 }
             }
@@ -590,7 +646,7 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
         const int take = (j < n) && (s > thr || (is_eq && eq_seen + eq_before < need_eq));
         int pos_before;
         const int take_total = block_excl_scan(take, &pos_before, sh_warp);
-        if (take && taken + pos_before < K) out[taken + pos_before] = j;
+        if (take && taken + pos_before < K) out[taken + pos_before] = out_index(a, b, j);
         taken += take_total;
         eq_seen += eq_total;
     }
@@ -602,6 +658,80 @@ topk_finish_kernel(TopkArgs a, int bias, int shift) {
 __global__ void zero_counters_kernel(int32_t* p, int n) {
     pdl_wait();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
+}
+
+// ---- hierarchical indexer, block stage
+constexpr int kBlkPerThread = 8;
+constexpr int kBlkPerCta = kThreads * kBlkPerThread;
+
+// Block scores of one tile of kBlkPerCta blocks of a sequence: the highest
+// visible entry score of each block, counted in the sequence's histogram; the
+// last CTA of the sequence derives the threshold bin of the best `keep`.
+__global__ void __launch_bounds__(kThreads)
+block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
+    __shared__ int hist[kBins];
+    __shared__ int sh_warp[kThreads / 32];
+    __shared__ int s_last, s_t, s_above;
+    pdl_wait();
+    const int b = blockIdx.y, tid = threadIdx.x;
+    const int n0 = h.n_entries[b];
+    const int n = (n0 >= 0 && n0 <= h.capacity) ? n0 : 0;
+    const int nb = (n + h.block - 1) / h.block;
+    if (blockIdx.x == 0 && tid == 0) h.nblk[b] = nb;
+    const int ntiles = (nb + kBlkPerCta - 1) / kBlkPerCta;
+    if ((int)blockIdx.x >= ntiles) return;
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    const int32_t* sc = h.scores + (size_t)b * h.capacity;
+    int32_t* bs = h.bscore + (size_t)b * cap_blk;
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+        const int j = blockIdx.x * kBlkPerCta + u * kThreads + tid;
+        if (j < nb) {
+            const int e0 = j * h.block, e1 = min(n, e0 + h.block);
+            int m = __ldcg(sc + e0);
+            for (int e = e0 + 1; e < e1; ++e) m = max(m, __ldcg(sc + e));
+            bs[j] = m;
+            atomicAdd(&hist[score_bin(m, bias, shift)], 1);
+        }
+    }
+    __syncthreads();
+    int32_t* gh = h.counters + (size_t)b * kBins;
+    for (int i = tid; i < kBins; i += kThreads)
+        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+    if (nb <= h.keep) return;  // every block is kept: no threshold needed
+    __threadfence();
+    __syncthreads();
+    if (tid == 0)
+        s_last = atomicAdd(h.counters + (size_t)h.batch * kBins + b, 1) == ntiles - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = __ldcg(gh + i);
+    if (tid == 0) s_t = s_above = 0;
+    __syncthreads();
+    find_threshold(hist, h.keep, &s_t, &s_above, sh_warp);
+    if (tid == 0) {
+        h.thr[2 * b] = s_t;
+        h.thr[2 * b + 1] = s_above;
+    }
+}
+
+// Pool length of each sequence: whole kept blocks, the last block of the
+// sequence counting only its visible entries.
+__global__ void pool_len_kernel(HierArgs h) {
+    pdl_wait();
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= h.batch) return;
+    const int n0 = h.n_entries[b];
+    const int n = (n0 >= 0 && n0 <= h.capacity) ? n0 : 0;
+    const int nb = (n + h.block - 1) / h.block;
+    const int32_t* blocks = h.pool_blocks + (size_t)b * h.keep;
+    int k = 0;
+    while (k < h.keep && blocks[k] >= 0) ++k;
+    int len = k * h.block;
+    if (k > 0 && blocks[k - 1] == nb - 1) len -= nb * h.block - n;
+    h.pool_n[b] = len;
 }
 
 template <int DI>
@@ -621,17 +751,74 @@ cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, in
                       s, a, per, bias, shift);
 }
 
+cudaError_t launch_select(const TopkArgs& a, int bias, int shift, cudaStream_t s) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    dim3 grid(sel_tiles(a.capacity), a.batch);
+    trace_before("topk_collect", s);
+    cudaError_t err = launch_pdl(topk_collect_kernel, grid, kThreads, 0, s, a, bias, shift);
+    trace_after(s);
+    if (err != cudaSuccess) return err;
+    static bool attr_set[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        err = cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kFinishSmem);
+        if (err != cudaSuccess) return err;
+        attr_set[dev] = true;
+    }
+    trace_before("topk_finish", s);
+    err = launch_pdl(topk_finish_kernel, a.batch, kThreads, kFinishSmem, s, a, bias, shift);
+    trace_after(s);
+    return err;
+}
+
+cudaError_t launch_zero(int32_t* p, int words, cudaStream_t s) {
+    trace_before("topk_zero", s);
+    const cudaError_t err = launch_pdl(zero_counters_kernel, (words + 1023) / 1024, 256, 0, s, p,
+                                       words);
+    trace_after(s);
+    return err;
+}
+
 }  // namespace
+
+cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
+    if (h.batch == 0) return cudaSuccess;
+    const int bias = score_bias(h.di), shift = score_shift(h.di);
+    const int cap_blk = (h.capacity + h.block - 1) / h.block;
+    cudaError_t err = launch_zero(h.counters, (int)topk_counter_words(h.batch), s);
+    if (err != cudaSuccess) return err;
+    trace_before("block_max", s);
+    err = launch_pdl(block_max_kernel, dim3((cap_blk + kBlkPerCta - 1) / kBlkPerCta, h.batch),
+                     kThreads, 0, s, h, cap_blk, bias, shift);
+    trace_after(s);
+    if (err != cudaSuccess) return err;
+    TopkArgs a = {};
+    a.n_entries = h.nblk;
+    a.batch = h.batch;
+    a.capacity = cap_blk;
+    a.idx_capacity = cap_blk;
+    a.topk = h.keep;
+    a.di = h.di;
+    a.topk_idx = h.pool_blocks;
+    a.scores = h.bscore;
+    a.counters = h.counters;
+    a.thr = h.thr;
+    a.tile_count = h.tile_count;
+    a.cands = h.cands;
+    a.status = h.status;
+    if ((err = launch_select(a, bias, shift, s)) != cudaSuccess) return err;
+    trace_before("pool_len", s);
+    err = launch_pdl(pool_len_kernel, (h.batch + 127) / 128, 128, 0, s, h);
+    trace_after(s);
+    return err;
+}
 
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     if (a.batch == 0) return cudaSuccess;
     const int bias = score_bias(a.di), shift = score_shift(a.di);
     // zero the histograms and the finished-CTA counters (adjacent in the workspace)
-    const int words = (int)topk_counter_words(a.batch);
-    trace_before("topk_zero", s);
-    cudaError_t err = launch_pdl(zero_counters_kernel, (words + 1023) / 1024, 256, 0, s,
-                                 a.counters, words);
-    trace_after(s);
+    cudaError_t err = launch_zero(a.counters, (int)topk_counter_words(a.batch), s);
     if (err != cudaSuccess) return err;
     // one wave: 2 CTAs per SM (96 KB ring + 8 KB histogram each for Di = 128),
     // equal row slices
@@ -654,22 +841,7 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     }
     trace_after(s);
     if (err != cudaSuccess) return err;
-    dim3 grid(sel_tiles(a.capacity), a.batch);
-    trace_before("topk_collect", s);
-    err = launch_pdl(topk_collect_kernel, grid, kThreads, 0, s, a, bias, shift);
-    trace_after(s);
-    if (err != cudaSuccess) return err;
-    static bool attr_set[64] = {};
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        err = cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kFinishSmem);
-        if (err != cudaSuccess) return err;
-        attr_set[dev] = true;
-    }
-    trace_before("topk_finish", s);
-    err = launch_pdl(topk_finish_kernel, a.batch, kThreads, kFinishSmem, s, a, bias, shift);
-    trace_after(s);
-    return err;
+    return launch_select(a, bias, shift, s);
 }
 
 }  // namespace kvc

@@ -2,6 +2,7 @@
 // layout, CSA2 layer-group orchestration, tracing and the format codecs.
 // Every entry point validates on the host and then only enqueues kernels on
 // the caller's stream; nothing here allocates device memory or synchronises.
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -131,10 +132,14 @@ constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t scores, counters, thr, tile_count, cands, part_o, part_ml, total;
+    size_t scores, counters, thr, tile_count, cands, part_o, part_ml;
+    size_t bscore, nblk, pool_blocks, pool_n;  // hierarchical indexer (0 when off)
+    size_t total;
 };
-WsLayout ws_layout(const kvc_config& c, const Shape& sh, int batch, int cap) {
-    WsLayout w;
+// hier_blocks > 0 adds the hierarchical indexer's block scores and pool.
+WsLayout ws_layout(const kvc_config& c, const Shape& sh, int batch, int cap,
+                   int hier_blocks = 0, int hier_block = 0) {
+    WsLayout w = {};
     size_t off = 0;
     const size_t tiles = (size_t)batch * sel_tiles(cap);
     w.scores = off;
@@ -151,6 +156,17 @@ WsLayout ws_layout(const kvc_config& c, const Shape& sh, int batch, int cap) {
     off = up(off + (size_t)batch * c.n_heads * kMaxSplit * sh.Dv * 4);
     w.part_ml = off;
     off = up(off + (size_t)batch * c.n_heads * kMaxSplit * 2 * 4);
+    if (hier_blocks > 0) {
+        const size_t cap_blk = ((size_t)cap + hier_block - 1) / hier_block;
+        w.bscore = off;
+        off = up(off + (size_t)batch * cap_blk * 4);
+        w.nblk = off;
+        off = up(off + (size_t)batch * 4);
+        w.pool_blocks = off;
+        off = up(off + (size_t)batch * hier_blocks * 4);
+        w.pool_n = off;
+        off = up(off + (size_t)batch * 4);
+    }
     w.total = off;
     return w;
 }
@@ -180,8 +196,8 @@ kvc_status check_cache(const kvc_cache* cache, const Shape& sh) {
 }
 
 kvc_status check_ws(void* ws, size_t ws_bytes, const kvc_config& c, const Shape& sh, int batch,
-                    int cap, WsLayout* w) {
-    *w = ws_layout(c, sh, batch, cap);
+                    int cap, WsLayout* w, int hier_blocks = 0, int hier_block = 0) {
+    *w = ws_layout(c, sh, batch, cap, hier_blocks, hier_block);
     if (!ws || !aligned(ws, kAlign) || ws_bytes < w->total) return KVC_ERR_WORKSPACE;
     return KVC_OK;
 }
@@ -190,12 +206,13 @@ kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* c
                     int32_t* topk, int32_t* scores, unsigned char* ws, const WsLayout& w,
                     uint32_t* st, cudaStream_t s) {
     if (cache->capacity > kMaxTopkCapacity) return KVC_ERR_CAPACITY;
-    TopkArgs a;
+    TopkArgs a = {};
     a.idx_q = idx_q;
     a.idx_k = cache->idx_k;
     a.n_entries = cache->n_entries;
     a.batch = cache->batch;
     a.capacity = cache->capacity;
+    a.idx_capacity = cache->capacity;
     a.topk = c.topk;
     a.di = c.idx_dim;
     a.topk_idx = topk;
@@ -205,6 +222,56 @@ kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* c
     a.tile_count = reinterpret_cast<int32_t*>(ws + w.tile_count);
     a.cands = reinterpret_cast<unsigned long long*>(ws + w.cands);
     a.status = st;
+    return launch_index_topk(a, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+// Hierarchical indexer: the block pool of a Full layer (its scores are in
+// the workspace after run_topk).
+kvc_status run_block_pool(const kvc_config& c, const kvc_cache* cache, int keep, int block,
+                          unsigned char* ws, const WsLayout& w, uint32_t* st, cudaStream_t s) {
+    HierArgs h = {};
+    h.scores = reinterpret_cast<const int32_t*>(ws + w.scores);
+    h.n_entries = cache->n_entries;
+    h.batch = cache->batch;
+    h.capacity = cache->capacity;
+    h.block = block;
+    h.keep = keep;
+    h.di = c.idx_dim;
+    h.bscore = reinterpret_cast<int32_t*>(ws + w.bscore);
+    h.nblk = reinterpret_cast<int32_t*>(ws + w.nblk);
+    h.pool_blocks = reinterpret_cast<int32_t*>(ws + w.pool_blocks);
+    h.pool_n = reinterpret_cast<int32_t*>(ws + w.pool_n);
+    h.counters = reinterpret_cast<int32_t*>(ws + w.counters);
+    h.thr = reinterpret_cast<int32_t*>(ws + w.thr);
+    h.tile_count = reinterpret_cast<int32_t*>(ws + w.tile_count);
+    h.cands = reinterpret_cast<unsigned long long*>(ws + w.cands);
+    h.status = st;
+    return launch_block_pool(h, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+// A Reindex layer over the pool: its indexer query scores the pool's rows only.
+kvc_status run_pool_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* cache,
+                         int keep, int block, int32_t* topk, unsigned char* ws,
+                         const WsLayout& w, uint32_t* st, cudaStream_t s) {
+    TopkArgs a = {};
+    a.idx_q = idx_q;
+    a.idx_k = cache->idx_k;
+    a.n_entries = reinterpret_cast<const int32_t*>(ws + w.pool_n);
+    a.batch = cache->batch;
+    a.capacity = (int)std::min<long long>((long long)keep * block, cache->capacity);
+    a.idx_capacity = cache->capacity;
+    a.topk = c.topk;
+    a.di = c.idx_dim;
+    a.topk_idx = topk;
+    a.scores = reinterpret_cast<int32_t*>(ws + w.scores);
+    a.counters = reinterpret_cast<int32_t*>(ws + w.counters);
+    a.thr = reinterpret_cast<int32_t*>(ws + w.thr);
+    a.tile_count = reinterpret_cast<int32_t*>(ws + w.tile_count);
+    a.cands = reinterpret_cast<unsigned long long*>(ws + w.cands);
+    a.status = st;
+    a.pool_blocks = reinterpret_cast<const int32_t*>(ws + w.pool_blocks);
+    a.pool_keep = keep;
+    a.pool_block = block;
     return launch_index_topk(a, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
@@ -254,6 +321,19 @@ size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity) {
     Shape sh;
     if (!derive_shape(cfg, &sh) || batch < 0 || capacity < 0) return 0;
     return ws_layout(*cfg, sh, batch, capacity).total;
+}
+
+static bool hier_ok(int hier_blocks, int hier_block) {
+    return hier_blocks == 0 ||
+           (hier_blocks > 0 && hier_blocks <= 65536 && hier_block >= 1 && hier_block <= 256);
+}
+
+size_t kvc_workspace_bytes_hier(const kvc_config* cfg, int batch, int capacity, int hier_blocks,
+                                int hier_block) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh) || batch < 0 || capacity < 0 || !hier_ok(hier_blocks, hier_block))
+        return 0;
+    return ws_layout(*cfg, sh, batch, capacity, hier_blocks, hier_block).total;
 }
 
 kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new, const float* gate,
@@ -327,8 +407,19 @@ kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers, const int32
                                 int window_len, const kvc_cache* cache, float* out, float* lse,
                                 int32_t* topk, void* ws, size_t ws_bytes, uint32_t* dev_status,
                                 void* stream) {
+    return kvc_layer_group_step_hier(cfg, 0, 0, n_layers, modes, q, idx_q, windows, window_len,
+                                     cache, out, lse, topk, ws, ws_bytes, dev_status, stream);
+}
+
+kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int hier_block,
+                                     int n_layers, const int32_t* modes, const void* q,
+                                     const int8_t* idx_q, const void* windows, int window_len,
+                                     const kvc_cache* cache, float* out, float* lse,
+                                     int32_t* topk, void* ws, size_t ws_bytes,
+                                     uint32_t* dev_status, void* stream) {
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    if (!hier_ok(hier_blocks, hier_block)) return KVC_ERR_INVALID;
     kvc_status st = check_cache(cache, sh);
     if (st != KVC_OK) return st;
     if (n_layers < 1 || !modes) return KVC_ERR_INVALID;
@@ -347,19 +438,34 @@ kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers, const int32
     const size_t w_stride = B * (size_t)cfg->window * sh.D * sh.act_bytes;
     if (q_stride % 16 || (w_stride % 16) || (B * cfg->idx_dim) % 16) return KVC_ERR_INVALID;
     WsLayout w;
-    if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w, hier_blocks,
+                       hier_block)) != KVC_OK)
+        return st;
     if (!device_ok()) return KVC_ERR_DEVICE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     unsigned char* wsb = static_cast<unsigned char*>(ws);
     const size_t K = (size_t)cfg->topk;
     int head = -1;
+    bool have_pool = false;
     for (int l = 0; l < n_layers; ++l) {
         int32_t* tk = topk + (size_t)l * B * K;
-        if (modes[l] == KVC_FULL || modes[l] == KVC_REINDEX) {
+        const int8_t* iq = idx_q + (size_t)l * B * cfg->idx_dim;
+        if (modes[l] == KVC_FULL || (modes[l] == KVC_REINDEX && !have_pool)) {
             // Full scores its stored cache; Reindex rescores the same stored
             // (Full layer's) cache with its own indexer query.
-            st = run_topk(*cfg, idx_q + (size_t)l * B * cfg->idx_dim, cache, tk, nullptr, wsb, w,
-                          dev_status, s);
+            st = run_topk(*cfg, iq, cache, tk, nullptr, wsb, w, dev_status, s);
+            if (st != KVC_OK) return st;
+            if (hier_blocks > 0 && modes[l] == KVC_FULL) {
+                // hierarchical indexer: later Reindex layers score only the
+                // pool of this layer's best blocks
+                st = run_block_pool(*cfg, cache, hier_blocks, hier_block, wsb, w, dev_status, s);
+                if (st != KVC_OK) return st;
+                have_pool = true;
+            }
+            head = l;
+        } else if (modes[l] == KVC_REINDEX) {
+            st = run_pool_topk(*cfg, iq, cache, hier_blocks, hier_block, tk, wsb, w, dev_status,
+                               s);
             if (st != KVC_OK) return st;
             head = l;
         } else {

@@ -88,8 +88,37 @@ struct TopkArgs {
     int32_t* tile_count;   // [B][sel_tiles(cap)] candidates per tile
     unsigned long long* cands;  // [B][sel_tiles(cap) * kSelTile]
     uint32_t* status;
+    int idx_capacity;      // row stride (entries) of idx_k per sequence
+    // Pool mode (hierarchical indexer): when pool_blocks is set, row r of
+    // sequence b is entry pool_blocks[b][r / pool_block] * pool_block +
+    // r % pool_block of idx_k; capacity and n_entries then describe the pool
+    // and the top-K is written as entry indices.
+    const int32_t* pool_blocks;  // [B][pool_keep] ascending, or null
+    int pool_keep, pool_block;
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
+
+// Hierarchical indexer, block stage: from a Full layer's entry scores
+// ([B][capacity]), the blocks of `block` consecutive entries are scored by
+// their best entry and the best `keep` blocks of every sequence are written
+// ascending to pool_blocks [B][keep] (-1 padded); pool_n [B] receives the
+// number of pool entries.  Scratch regions as in TopkArgs, sized for
+// ceil(capacity / block) block scores.
+struct HierArgs {
+    const int32_t* scores;     // [B][capacity] entry scores
+    const int32_t* n_entries;  // [B]
+    int batch, capacity, block, keep, di;
+    int32_t* bscore;           // [B][ceil(capacity / block)]
+    int32_t* nblk;             // [B]
+    int32_t* pool_blocks;      // [B][keep]
+    int32_t* pool_n;           // [B]
+    int32_t* counters;         // topk_counter_words(B)
+    int32_t* thr;              // [B][2]
+    int32_t* tile_count;       // [B][sel_tiles(ceil(capacity / block))]
+    unsigned long long* cands; // [B][sel_tiles(...) * kSelTile]
+    uint32_t* status;
+};
+cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s);
 
 struct AttnArgs {
     const void* q;          // [B][H][D]

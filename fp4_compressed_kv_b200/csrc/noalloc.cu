@@ -81,12 +81,13 @@ extern "C" kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t
     unsigned char* ws = nullptr;
     kvc_status st = scratch_for_current_device(&ws);
     if (st != KVC_OK) return st;
-    TopkArgs a;
+    TopkArgs a = {};
     a.idx_q = idx_q;
     a.idx_k = cache->idx_k;
     a.n_entries = cache->n_entries;
     a.batch = cache->batch;
     a.capacity = cache->capacity;
+    a.idx_capacity = cache->capacity;
     a.topk = cfg->topk;
     a.di = cfg->idx_dim;
     a.topk_idx = topk_idx;

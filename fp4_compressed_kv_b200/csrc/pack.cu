@@ -103,24 +103,31 @@ __device__ __forceinline__ void load8_gate(const float* p, float v[8]) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// E2M1 rounding input fl(x / s), given r = 1/s rounded.  x * r lies within
-// about 2 fp32 ulps of the correctly rounded quotient (two roundings of
-// 2^-24 relative each, quotients below 8), so both round to the same E2M1
-// code unless x * r sits within a few ulps of one of the grid's rounding
-// midpoints {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5}.  The map below sends every
-// midpoint to k + 1/2; near one of them the quotient is divided out exactly.
-__device__ __forceinline__ float e2m1_input(float x, float s, float r) {
-    const float q = __fmul_rn(x, r);
-    const float a = fabsf(q);
-    const float u = a < 2.f ? a + a : (a < 4.f ? a : 0.5f * a);
-    return fabsf(u - floorf(u) - 0.5f) < 1.0e-5f ? __fdiv_rn(x, s) : q;
-}
-
-// fl(x / s) for the E2M1 code (0 when s is 0); r = 1/s rounded, `fast` when r
-// is finite.
-__device__ __forceinline__ float e2m1_quotient(float x, float s, float r, bool fast) {
-    if (!(s > 0.f)) return 0.f;
-    return fast ? e2m1_input(x, s, r) : __fdiv_rn(x, s);
+// Eight E2M1 codes of fl(x[t] / s) (s > 0, x finite) without a division per
+// element.  With r = 1/s rounded, x * r(1 - 2^-20) and x * r(1 + 2^-20)
+// (each product rounded) bracket the correctly rounded quotient: the few
+// roundings move them by a handful of 2^-24 relative units, far less than
+// the 2^-20 offset.  Rounding to the E2M1 grid is monotone, so when both
+// brackets give the same codes the quotient gives them too; otherwise (a
+// quotient within 2^-20 of a rounding midpoint, or r not finite) the eight
+// quotients are divided out exactly.
+__device__ __forceinline__ uint32_t e2m1x8_quotient(const float x[8], float s) {
+    const float r = __frcp_rn(s);
+    if (r < 3.0e38f) {
+        const float rl = __fmul_rn(r, 1.0f - 0x1p-20f), rh = __fmul_rn(r, 1.0f + 0x1p-20f);
+        float lo[8], hi[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            lo[t] = __fmul_rn(x[t], rl);
+            hi[t] = __fmul_rn(x[t], rh);
+        }
+        const uint32_t cl = e2m1x8_from_f32(lo);
+        if (cl == e2m1x8_from_f32(hi)) return cl;
+    }
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = fminf(fmaxf(__fdiv_rn(x[t], s), -6.f), 6.f);
+    return e2m1x8_from_f32(v);
 }
 
 constexpr int kThreads = 256;
@@ -130,7 +137,7 @@ constexpr int kMaxChunks = 128;       // D <= 1024
 
 // MAXJ: chunks per lane (D <= 64 * MAXJ).
 template <typename T, int MAXJ>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (MAXJ <= 4 || (sizeof(T) == 2 && MAXJ <= 9)) ? 2 : 1)
 pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     pdl_wait();
     __shared__ __align__(16) uint8_t tail_smem[kTeams][kTailBytes];
@@ -191,9 +198,11 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
     for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
 
-    // entry values and lane-local chunk maxima
+    // entry values (replacing the token chunks in registers) and lane-local
+    // chunk maxima; non-finite values are flagged and coded as 0
     bool bad = false;
     float cmax[MAXJ];
+    float x[MAXJ][8];
 #pragma unroll
     for (int j = 0; j < MAXJ; ++j) {
         const int c = l + 8 * j;
@@ -201,9 +210,13 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
         float m = 0.f;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            const float v = __fmaf_rn(w0, k0[j].get(t), __fmul_rn(w1, k1[j].get(t)));
-            if (isfinite(v)) m = fmaxf(m, fabsf(v));
-            else if (active) bad = true;
+            float v = __fmaf_rn(w0, k0[j].get(t), __fmul_rn(w1, k1[j].get(t)));
+            if (!isfinite(v)) {
+                if (active) bad = true;
+                v = 0.f;
+            }
+            x[j][t] = v;
+            m = fmaxf(m, fabsf(v));
         }
         cmax[j] = m;
     }
@@ -243,17 +256,7 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
             sbyte = e4m3_from_f32(s);
             s = e4m3_to_f32(sbyte);
         }
-        const float r = __frcp_rn(s);
-        const bool fast = r < 3.0e38f;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            float x = __fmaf_rn(w0, k0[j].get(t), __fmul_rn(w1, k1[j].get(t)));
-            if (!isfinite(x)) x = 0.f;
-            const float q = e2m1_quotient(x, s, r, fast);
-            v[t] = fminf(fmaxf(q, -6.f), 6.f);
-        }
-        *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
+        *reinterpret_cast<uint32_t*>(rec + 4 * c) = s > 0.f ? e2m1x8_quotient(x[j], s) : 0u;
         if (c % lpg == 0) {
             const int gi = c / lpg;
             if (ue4m3)
@@ -316,6 +319,10 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     float* sg = reinterpret_cast<float*>(s1 + D);
 
     // every load of the entry in flight at once
+    uint4 ik = make_uint4(0, 0, 0, 0);
+    if (lane < (di >> 4))
+        ik = __ldcs(reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di) +
+                    lane);
     Chunk<T> x0[MAXJ], x1[MAXJ];
     float4 g0[MAXJ], g1[MAXJ];
 #pragma unroll
@@ -393,15 +400,7 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
             sbyte = e4m3_from_f32(s);
             s = e4m3_to_f32(sbyte);
         }
-        const float r = __frcp_rn(s);
-        const bool fast = r < 3.0e38f;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const float q = e2m1_quotient(x[t], s, r, fast);
-            v[t] = fminf(fmaxf(q, -6.f), 6.f);
-        }
-        *reinterpret_cast<uint32_t*>(rec + 4 * c) = e2m1x8_from_f32(v);
+        *reinterpret_cast<uint32_t*>(rec + 4 * c) = s > 0.f ? e2m1x8_quotient(x, s) : 0u;
         if (c % lpg == 0) {
             const int gi = c / lpg;
             if (ue4m3)
@@ -414,11 +413,8 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     for (int t = lane * 4; t < tail_len; t += 128)
         *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
             *reinterpret_cast<const uint32_t*>(tail + t);
-    if (lane < (di >> 4)) {
-        const uint4 v = __ldcs(
-            reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di) + lane);
-        *(reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di) + lane) = v;
-    }
+    if (lane < (di >> 4))
+        *(reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di) + lane) = ik;
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
     if (half == 1 && lane == 0) a.n_entries[b] = base + 1;
 }

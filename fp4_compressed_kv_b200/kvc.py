@@ -63,6 +63,9 @@ def _lib():
             "kvc_index_topk_noalloc": (S, [P, P, P, P, P, P, P]),
             "kvc_sparse_decode_attn": (S, [P, P, P, P, P, I, P, P, P, Z, P, P]),
             "kvc_layer_group_step": (S, [P, I, P, P, P, P, I, P, P, P, P, P, Z, P, P]),
+            "kvc_workspace_bytes_hier": (Z, [P, I, I, I, I]),
+            "kvc_layer_group_step_hier": (S, [P, I, I, I, P, P, P, P, I, P, P, P, P, P, Z, P,
+                                              P]),
             "kvc_e2m1_encode": (S, [P, C.c_int64, P, P]),
             "kvc_e4m3_encode": (S, [P, C.c_int64, P, P]),
             "kvc_trace_begin": (S, [I]),
@@ -146,8 +149,17 @@ class Cache:
                            self.n_entries.data_ptr(), self.batch, self.capacity)
 
 
-def workspace(cfg: Config, batch: int, capacity: int, device="cuda") -> torch.Tensor:
-    n = workspace_bytes(cfg, batch, capacity)
+def workspace(cfg: Config, batch: int, capacity: int, device="cuda", hier_blocks: int = 0,
+              hier_block: int = 8) -> torch.Tensor:
+    """Workspace for the calls on `batch` x `capacity` (and, with hier_blocks
+    > 0, for the hierarchical group step)."""
+    if hier_blocks:
+        n = int(_lib().kvc_workspace_bytes_hier(C.byref(cfg), batch, capacity, hier_blocks,
+                                                 hier_block))
+    else:
+        n = workspace_bytes(cfg, batch, capacity)
+    if n == 0:
+        raise KvcError("invalid workspace request")
     return torch.empty(n + 256, dtype=torch.uint8, device=device)
 
 
@@ -192,10 +204,18 @@ def sparse_decode_attn(cfg, q, cache: Cache, topk, window, window_len, out, ws, 
 
 
 def layer_group_step(cfg, modes, q, idx_q, windows, window_len, cache: Cache, out, topk, ws,
-                     lse=None, status=None, stream=None):
+                     lse=None, status=None, stream=None, hier_blocks=0, hier_block=8):
+    """One decode step through a CSA2 layer group; hier_blocks > 0 turns on
+    the hierarchical indexer (the workspace must have been sized for it)."""
     modes_arr = (C.c_int32 * len(modes))(*modes)
     p, n = _ws(ws)
     cs = cache.struct()
+    if hier_blocks:
+        _check("kvc_layer_group_step_hier", _lib().kvc_layer_group_step_hier(
+            C.byref(cfg), int(hier_blocks), int(hier_block), len(modes), modes_arr, _ptr(q),
+            _ptr(idx_q), _ptr(windows), int(window_len), C.byref(cs), _ptr(out), _ptr(lse),
+            _ptr(topk), p, n, _ptr(status), _stream(stream)))
+        return
     _check("kvc_layer_group_step", _lib().kvc_layer_group_step(
         C.byref(cfg), len(modes), modes_arr, _ptr(q), _ptr(idx_q), _ptr(windows), int(window_len),
         C.byref(cs), _ptr(out), _ptr(lse), _ptr(topk), p, n, _ptr(status), _stream(stream)))

@@ -204,6 +204,31 @@ kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers,
                                 size_t ws_bytes, uint32_t* dev_status,
                                 void* stream);
 
+/* The layer group step with the hierarchical sparse indexer ([A] part 4
+ * "层级稀疏索引器：后面的层只在候选池里找"): every Full layer, after its own
+ * top-K, cuts its scored entries into blocks of `hier_block` consecutive
+ * entries (8 on the page), scores each block by its best entry and keeps the
+ * best `hier_blocks` blocks (2048 on the page; ties to the lower block,
+ * written ascending); every later Reindex layer of the call scores only that
+ * pool (16,384 entries on the page) with its own indexer query and keeps its
+ * top-K among them (ties to the lower entry index).  A Reindex layer before
+ * any Full layer scores the whole cache.  The last block of a sequence may be
+ * short.  hier_blocks = 0 is kvc_layer_group_step; otherwise
+ * 1 <= hier_blocks <= 65536 and 1 <= hier_block <= 256 (else
+ * KVC_ERR_INVALID).  ws must hold kvc_workspace_bytes_hier(cfg, batch,
+ * capacity, hier_blocks, hier_block) bytes; all other arguments as in
+ * kvc_layer_group_step.                                                     */
+size_t kvc_workspace_bytes_hier(const kvc_config* cfg, int batch, int capacity,
+                                int hier_blocks, int hier_block);
+kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks,
+                                     int hier_block, int n_layers,
+                                     const int32_t* modes, const void* q,
+                                     const int8_t* idx_q, const void* windows,
+                                     int window_len, const kvc_cache* cache,
+                                     float* out, float* lse, int32_t* topk,
+                                     void* ws, size_t ws_bytes,
+                                     uint32_t* dev_status, void* stream);
+
 /* E2M1 / E4M3 codecs as the pack kernel applies them (format utilities).
  * kvc_e2m1_encode: x [n] fp32 -> codes [n] uint8 (0..15), round to nearest
  * even on the grid {0, 0.5, 1, 1.5, 2, 3, 4, 6}, saturating, -0 stored as 0.
@@ -218,8 +243,8 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
  * "pack", "pack_commit", "topk_zero", "index_scan", "topk_collect",
- * "topk_finish", "copy_topk", "attn_tc05", "attn_simt", "attn_merge",
- * "fp4_codec".                                                             */
+ * "topk_finish", "block_max", "pool_len", "copy_topk", "attn_tc05",
+ * "attn_simt", "attn_merge", "fp4_codec".                                                             */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);
 kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);

@@ -87,6 +87,10 @@ def lib():
             "orc_bytes_resident": (C.c_uint64, [P, C.c_int64, C.c_int, C.c_int, C.c_int]),
             "orc_group_step": (C.c_int, [P, C.c_int, P, C.c_int, P, P, P, C.c_int, P, P,
                                          C.c_int, P, P, P, P, P]),
+            "orc_group_step_hier": (C.c_int, [P, C.c_int, P, C.c_int, P, P, P, C.c_int, P, P,
+                                              C.c_int, P, C.c_int, C.c_int, P, P, P, P]),
+            "orc_block_pool": (C.c_int, [P, C.c_int, C.c_int, C.c_int, P, P]),
+            "orc_pool_topk": (C.c_int, [P, P, C.c_int, P, C.c_int, C.c_int, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(_lib, name)
@@ -246,8 +250,25 @@ def sparse_decode(cfg: Cfg, q, records, n_entries, topk_idx, window, window_len)
     return out, lse, int(st[0])
 
 
+def block_pool(scores, block, keep):
+    """Hierarchical indexer pool of one sequence's scores: (blocks, pool)."""
+    scores = _c(scores, np.int32)
+    blocks = np.empty(keep, np.int32)
+    pool = np.empty(keep * block, np.int32)
+    n = lib().orc_block_pool(_p(scores), scores.size, block, keep, _p(blocks), _p(pool))
+    return blocks, pool[:n].copy()
+
+
+def pool_topk(q, keys, pool, k):
+    """Top-K of one sequence over the pool's entries only."""
+    q, keys, pool = _c(q, np.int8), _c(keys, np.int8), _c(pool, np.int32)
+    out = np.empty(k, np.int32)
+    lib().orc_pool_topk(_p(q), _p(keys), keys.shape[1], _p(pool), pool.size, k, _p(out))
+    return out
+
+
 def group_step(cfg: Cfg, modes, q, idx_q, windows, window_len, records, idx_cache,
-               n_entries):
+               n_entries, hier_keep=0, hier_block=8):
     modes = np.ascontiguousarray(modes, dtype=np.int32)
     q, windows = _c(q, np.float32), _c(windows, np.float32)
     idx_q = _c(idx_q, np.int8)
@@ -259,9 +280,10 @@ def group_step(cfg: Cfg, modes, q, idx_q, windows, window_len, records, idx_cach
     lse = np.empty((L, B, cfg.n_heads), np.float64)
     tk = np.empty((L, B, cfg.topk), np.int32)
     st = np.zeros(1, np.uint32)
-    rc = lib().orc_group_step(C.byref(cfg), L, _p(modes), B, _p(q), _p(idx_q), _p(windows),
-                              int(window_len), _p(records), _p(idx_cache), cap, _p(n_entries),
-                              _p(out), _p(lse), _p(tk), _p(st))
+    rc = lib().orc_group_step_hier(C.byref(cfg), L, _p(modes), B, _p(q), _p(idx_q),
+                                   _p(windows), int(window_len), _p(records), _p(idx_cache),
+                                   cap, _p(n_entries), int(hier_keep), int(hier_block),
+                                   _p(out), _p(lse), _p(tk), _p(st))
     if rc:
         raise ValueError(f"orc_group_step failed: {rc}")
     return out, lse, tk, int(st[0])

@@ -398,6 +398,59 @@ int orc_index_topk(const orc_cfg* c, int B, const int8_t* idx_q,
 }
 
 /* ------------------------------------------------------------------ */
+/* Hierarchical sparse indexer ([P2] part 4 "层级稀疏索引器：后面的层只在候选池
+ * 里找"): after the first Full layer has scored every entry, the entries are
+ * cut into blocks of `block` consecutive entries, each block scored by the
+ * highest score inside it; the best `keep` blocks (2048 of 8 on the page)
+ * form the candidate pool (16,384 entries) that later Reindex layers score
+ * instead of the whole context.
+ * Readings: the last block may be short (its visible entries only); blocks
+ * are ranked like entries, (block score descending, block index ascending);
+ * fewer than `keep` blocks means all of them.
+ * blocks_out [keep]: chosen block indices ascending, -1 padded;
+ * pool_out [keep * block]: their entries, ascending.  Returns the pool size. */
+int orc_block_pool(const int32_t* scores, int n, int block, int keep,
+                   int32_t* blocks_out, int32_t* pool_out) {
+    int nb = (n + block - 1) / block;
+    int32_t* bs = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nb > 0 ? nb : 1));
+    for (int i = 0; i < nb; ++i) {
+        int32_t m = scores[(size_t)i * block];
+        for (int j = i * block + 1; j < n && j < (i + 1) * block; ++j)
+            if (scores[j] > m) m = scores[j];
+        bs[i] = m;
+    }
+    int kept = orc_topk(bs, nb, keep, blocks_out);
+    int pn = 0;
+    for (int i = 0; i < kept; ++i)
+        for (int j = blocks_out[i] * block; j < n && j < (blocks_out[i] + 1) * block; ++j)
+            pool_out[pn++] = j;
+    free(bs);
+    return pn;
+}
+
+/* A Reindex layer over the pool: its own indexer query scores only the
+ * pool's entries; top-K among them by (score descending, entry index
+ * ascending), written ascending, -1 padded.  Returns the number kept.     */
+int orc_pool_topk(const int8_t* q, const int8_t* keys, int di, const int32_t* pool,
+                  int pool_n, int k, int32_t* out) {
+    orc_scored* v = (orc_scored*)malloc(sizeof(orc_scored) * (size_t)(pool_n > 0 ? pool_n : 1));
+    for (int p = 0; p < pool_n; ++p) {
+        int32_t s = 0;
+        for (int d = 0; d < di; ++d)
+            s += (int32_t)q[d] * (int32_t)keys[(size_t)pool[p] * di + d];
+        v[p].score = s;
+        v[p].idx = pool[p];
+    }
+    qsort(v, (size_t)pool_n, sizeof(orc_scored), orc_by_score_desc_idx_asc);
+    int kept = pool_n < k ? pool_n : k;
+    for (int i = 0; i < kept; ++i) out[i] = v[i].idx;
+    qsort(out, (size_t)kept, sizeof(int32_t), orc_int_asc);
+    for (int i = kept; i < k; ++i) out[i] = -1;
+    free(v);
+    return kept;
+}
+
+/* ------------------------------------------------------------------ */
 /* R5: decode attention for one query token, all heads, in fp64 ([P2]
  * breakthrough 2: heads share one 512+64 latent entry, values are the
  * latent; breakthrough 4: window + top-512 global branch).
@@ -481,35 +534,74 @@ int orc_sparse_decode(const orc_cfg* c, int B, const float* q,
  * read the one stored cache (the Full layer's).  Arrays are layer-major:
  * q [L][B][H][D], idx_q [L][B][Di], windows [L][B][W][D],
  * out [L][B][H][Dv], lse [L][B][H], topk [L][B][K].                     */
+/* hier_keep > 0 turns on the hierarchical indexer: every Full layer also
+ * builds the block pool from its scores, and every Reindex layer after a
+ * Full layer of the same call scores only that pool.                      */
+int orc_group_step_hier(const orc_cfg* c, int n_layers, const int* modes, int B,
+                        const float* q, const int8_t* idx_q, const float* windows,
+                        int window_len, const uint8_t* records,
+                        const int8_t* idx_cache, int cap, const int32_t* n_entries,
+                        int hier_keep, int hier_block,
+                        double* out, double* lse, int32_t* topk, uint32_t* status) {
+    int D = c->latent_dim + c->rope_dim, Dv = c->latent_dim, H = c->n_heads;
+    int K = c->topk, Di = c->idx_dim;
+    if (n_layers < 1 || modes[0] == ORC_MODE_REUSE) return ORC_ERR_INVALID;
+    if (hier_keep < 0 || (hier_keep > 0 && hier_block < 1)) return ORC_ERR_INVALID;
+    size_t pool_cap = (size_t)(hier_keep > 0 ? hier_keep : 1) * (size_t)(hier_block > 0 ? hier_block : 1);
+    int32_t* pool = (int32_t*)malloc(sizeof(int32_t) * (size_t)B * pool_cap);
+    int32_t* pool_n = (int32_t*)calloc((size_t)B, sizeof(int32_t));
+    int32_t* blocks = (int32_t*)malloc(sizeof(int32_t) * (size_t)(hier_keep > 0 ? hier_keep : 1));
+    int32_t* sc = (int32_t*)malloc(sizeof(int32_t) * (size_t)(cap > 0 ? cap : 1));
+    int have_pool = 0, rc = ORC_OK;
+    int head = -1;
+    for (int l = 0; l < n_layers && rc == ORC_OK; ++l) {
+        int32_t* tk = topk + (size_t)l * B * K;
+        const int8_t* ql = idx_q + (size_t)l * B * Di;
+        if (modes[l] == ORC_MODE_FULL || (modes[l] == ORC_MODE_REINDEX && !have_pool)) {
+            for (int b = 0; b < B && rc == ORC_OK; ++b) {
+                int n = n_entries[b];
+                if (n < 0 || n > cap) {
+                    rc = ORC_ERR_CAPACITY;
+                    break;
+                }
+                orc_index_scores(ql + (size_t)b * Di, idx_cache + (size_t)b * cap * Di, n, Di, sc);
+                orc_topk(sc, n, K, tk + (size_t)b * K);
+                if (hier_keep > 0 && modes[l] == ORC_MODE_FULL)
+                    pool_n[b] = orc_block_pool(sc, n, hier_block, hier_keep, blocks,
+                                               pool + (size_t)b * pool_cap);
+            }
+            if (hier_keep > 0 && modes[l] == ORC_MODE_FULL) have_pool = 1;
+            head = l;
+        } else if (modes[l] == ORC_MODE_REINDEX) {
+            for (int b = 0; b < B; ++b)
+                orc_pool_topk(ql + (size_t)b * Di, idx_cache + (size_t)b * cap * Di, Di,
+                              pool + (size_t)b * pool_cap, pool_n[b], K, tk + (size_t)b * K);
+            head = l;
+        } else if (modes[l] == ORC_MODE_REUSE) {
+            memcpy(tk, topk + (size_t)head * B * K, sizeof(int32_t) * (size_t)B * K);
+        } else {
+            rc = ORC_ERR_INVALID;
+            break;
+        }
+        if (rc == ORC_OK)
+            rc = orc_sparse_decode(c, B, q + (size_t)l * B * H * D, records, cap, n_entries, tk,
+                                   windows + (size_t)l * B * c->window * D, window_len,
+                                   out + (size_t)l * B * H * Dv, lse + (size_t)l * B * H, status);
+    }
+    free(pool);
+    free(pool_n);
+    free(blocks);
+    free(sc);
+    return rc;
+}
+
 int orc_group_step(const orc_cfg* c, int n_layers, const int* modes, int B,
                    const float* q, const int8_t* idx_q, const float* windows,
                    int window_len, const uint8_t* records,
                    const int8_t* idx_cache, int cap, const int32_t* n_entries,
                    double* out, double* lse, int32_t* topk, uint32_t* status) {
-    int D = c->latent_dim + c->rope_dim, Dv = c->latent_dim, H = c->n_heads;
-    int K = c->topk;
-    if (n_layers < 1 || modes[0] == ORC_MODE_REUSE) return ORC_ERR_INVALID;
-    int head = -1;
-    for (int l = 0; l < n_layers; ++l) {
-        int32_t* tk = topk + (size_t)l * B * K;
-        if (modes[l] == ORC_MODE_FULL || modes[l] == ORC_MODE_REINDEX) {
-            int rc = orc_index_topk(c, B, idx_q + (size_t)l * B * c->idx_dim,
-                                    idx_cache, cap, n_entries, tk, NULL);
-            if (rc) return rc;
-            head = l;
-        } else if (modes[l] == ORC_MODE_REUSE) {
-            memcpy(tk, topk + (size_t)head * B * K, sizeof(int32_t) * (size_t)B * K);
-        } else {
-            return ORC_ERR_INVALID;
-        }
-        int rc = orc_sparse_decode(c, B, q + (size_t)l * B * H * D, records, cap,
-                                   n_entries, tk,
-                                   windows + (size_t)l * B * c->window * D,
-                                   window_len, out + (size_t)l * B * H * Dv,
-                                   lse + (size_t)l * B * H, status);
-        if (rc) return rc;
-    }
-    return ORC_OK;
+    return orc_group_step_hier(c, n_layers, modes, B, q, idx_q, windows, window_len, records,
+                               idx_cache, cap, n_entries, 0, 0, out, lse, topk, status);
 }
 
 /* ------------------------------------------------------------------ */

@@ -95,3 +95,23 @@ def test_no_device_fails_loudly(lib):
     rc = so.kvc_pack(C.byref(cfg), C.c_void_p(16), 2, C.c_void_p(16), C.c_void_p(16),
                      C.byref(cache), None, None)
     assert rc == 6  # KVC_ERR_DEVICE: nothing was enqueued
+
+
+def test_hier_workspace_and_validation(lib):
+    so = lib.lib()
+    w = synth.WORKLOADS["stack1m"]
+    cfg = lib.config_for(w)
+    plain = so.kvc_workspace_bytes(C.byref(cfg), 1, w.entries)
+    hier = so.kvc_workspace_bytes_hier(C.byref(cfg), 1, w.entries, 2048, 8)
+    # block scores (4 B per 8 entries) + pool blocks + lengths, each 256-aligned
+    assert plain + (w.entries // 8) * 4 <= hier <= plain + (w.entries // 8) * 4 + 2048 * 4 + 1024
+    assert so.kvc_workspace_bytes_hier(C.byref(cfg), 1, w.entries, 0, 0) == plain
+    assert so.kvc_workspace_bytes_hier(C.byref(cfg), 1, w.entries, 2048, 0) == 0
+    assert so.kvc_workspace_bytes_hier(C.byref(cfg), 1, w.entries, -1, 8) == 0
+    cache = lib.CacheStruct(16, 16, 16, 1, 8)
+    modes = (C.c_int32 * 2)(0, 1)
+    for blocks, block in ((2048, 0), (70000, 8), (16, 300)):
+        assert so.kvc_layer_group_step_hier(
+            C.byref(cfg), blocks, block, 2, modes, C.c_void_p(16), C.c_void_p(16),
+            C.c_void_p(16), 32, C.byref(cache), C.c_void_p(16), None, C.c_void_p(16),
+            C.c_void_p(256), 1 << 30, None, None) == 1

@@ -108,3 +108,20 @@ def test_topk_workspace_validation(kvc):
     with pytest.raises(kvc.KvcError) as e:
         kvc.index_topk(cfg, torch.zeros(1, 32, dtype=torch.int8, device="cuda"), cache, tk, small)
     assert e.value.status == 7
+
+
+def test_topk_scan_slices_span_sequences(kvc):
+    """400 short sequences: each scan CTA's row slice covers parts of two or
+    more sequences, so candidate segments start mid-slice and mid-sequence;
+    lengths are ragged on both sides of K."""
+    w = synth.WORKLOADS["mla32k"].scaled(batch=400, context=2 * 600)
+    inp = synth.make_inputs(w, with_tokens=False)
+    rng = np.random.default_rng(3)
+    n = rng.integers(300, 601, 400).astype(np.int32)
+    n[:3] = [600, 512, 513]
+    tk, sc, st = _run(kvc, w, inp["idx_k"], inp["idx_q"][0], n, 600)
+    otk, osc = _oracle(w, inp["idx_k"], inp["idx_q"][0], n, 600)
+    assert st == 0
+    for b in range(400):
+        assert np.array_equal(sc[b, : n[b]], osc[b, : n[b]]), b
+    topk_set_equal(tk, otk)
