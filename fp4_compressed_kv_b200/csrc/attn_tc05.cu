@@ -25,6 +25,8 @@
 //     attn_merge combines the chunks of a sequence by log-sum-exp.
 // Every wait on an mbarrier is bounded by a 2-second clock; on expiry the CTA
 // sets KVC_DEV_TIMEOUT, frees its tensor memory and returns.
+#include <algorithm>
+
 #include "kvc_internal.cuh"
 
 namespace kvc {
@@ -44,6 +46,9 @@ constexpr uint32_t OFF_RAW = OFF_K + K_BYTES;   // P (16 KB) reuses this after d
 constexpr uint32_t OFF_P = OFF_RAW;
 constexpr uint32_t OFF_MISC = OFF_RAW + RAW_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;  // + misc + table + alignment slack
+// Cluster epilogue scratch over Q, K and the raw rows: this split's O
+// [H][DV] fp32, then the splits' (m, l) of the heads this CTA combines.
+static_assert((uint32_t)H * DV * 4 + 2 * 8 * H * 4 <= OFF_MISC, "epilogue scratch below misc");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0, O_COL = 128;
 
@@ -65,6 +70,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+// every group but the most recent one complete
+__device__ __forceinline__ void cp_async_wait_prior() {
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;\n" ::: "memory");
@@ -175,8 +187,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // accumulated O^T is rescaled in tensor memory only on such a jump.
 constexpr float kRescaleSlack = 8.0f;
 
+// The CTAs of one cluster (the splits of one sequence) meet here; every
+// thread of every CTA of the cluster executes it the same number of times.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::
+                     : "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
+    float4 v;
+    asm("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float ld_peer_f32(uint32_t addr) {
+    float v;
+    asm("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr));
+    return v;
+}
+
 __global__ void __launch_bounds__(NT, 1)
-attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int cps, int ue4m3) {
+attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int cps, int ue4m3,
+                 int cluster) {
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -253,8 +291,10 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
             }
             kind[tid] = k;
         }
-        __syncthreads();
-        // ---- 1. gathers: records (raw rows), window rows (swizzled) and zero rows
+        // any window or empty slot in this chunk?
+        const int other_rows = __syncthreads_or(tid < CK && kind[tid < CK ? tid : 0] < 0);
+        // ---- 1. gathers: records (raw rows) as one group of copies, then window
+        // rows (swizzled) and zero rows, which only the QK product needs
         {
             const int pieces = rb >> 4;
             for (int p = tid; p < CK * pieces; p += NT) {
@@ -264,7 +304,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                     cp_async16(smem_u32(raw + s * RAW_STRIDE + pc * 16),
                                a.records + ((size_t)b * a.capacity + k) * rb + pc * 16);
             }
-            for (int p = tid; p < CK * (D / 8); p += NT) {
+            cp_async_commit();
+            for (int p = tid; other_rows && p < CK * (D / 8); p += NT) {
                 const int s = p / (D / 8), cc = p - s * (D / 8);
                 const int k = kind[s];
                 const uint32_t dst = sK + (cc >> 3) * K_ATOM + swz(s, cc & 7);
@@ -277,7 +318,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                                  "r"(0u), "r"(0u), "r"(0u));
                 }
             }
-            cp_async_wait_all();
+            cp_async_commit();
+            cp_async_wait_prior();  // this thread's record copies have landed
         }
         __syncthreads();
         // ---- 2. dequantise records into the swizzled K tile.  UE4M3 scales: 32
@@ -286,33 +328,48 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         // significant bits, so the bf16 multiply is exact).  Groups of >= 32
         // share one scale per item; groups of 8 or 16 take one per 8 channels.
         if (ue4m3) {
+            // two items per pass, all their shared-memory loads issued first
             const int lpg = sh.lpg;
-            for (int p = tid; p < CK * (D / 32); p += NT) {
-                const int s = p / (D / 32), i4 = p - s * (D / 32);
-                if (kind[s] < 0) continue;
-                const unsigned char* rec = raw + s * RAW_STRIDE;
-                const uint4 codes = *reinterpret_cast<const uint4*>(rec + i4 * 16);
-                const float sc = e4m3_to_f32(rec[sh.code_bytes + (4 * i4) / lpg]);
-                __nv_bfloat162 s2 = __floats2bfloat162_rn(sc, sc);
-                const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-                const uint32_t row = sK + (i4 >> 1) * K_ATOM;
+            constexpr int NI = CK * (D / 32);
+            for (int p0 = tid; p0 < NI; p0 += 2 * NT) {
+                uint4 codes[2];
+                float sc[2][4];
+                int sk[2], ik[2];
+                bool act[2];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (lpg < 4 && u > 0) {
-                        const float su = e4m3_to_f32(rec[sh.code_bytes + (4 * i4 + u) / lpg]);
-                        s2 = __floats2bfloat162_rn(su, su);
-                    }
-                    uint32_t w[4];
+                for (int q = 0; q < 2; ++q) {
+                    const int p = p0 + q * NT;
+                    sk[q] = p / (D / 32);
+                    ik[q] = p - sk[q] * (D / 32);
+                    act[q] = p < NI && kind[sk[q]] >= 0;
+                    if (act[q]) {
+                        const unsigned char* rec = raw + sk[q] * RAW_STRIDE;
+                        codes[q] = *reinterpret_cast<const uint4*>(rec + ik[q] * 16);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t e = lut[(cw[u] >> (8 * k)) & 0xFFu];
-                        const __nv_bfloat162 v =
-                            __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e), s2);
-                        w[k] = *reinterpret_cast<const uint32_t*>(&v);
+                        for (int u = 0; u < 4; ++u)
+                            sc[q][u] = e4m3_to_f32(rec[sh.code_bytes + (4 * ik[q] + (lpg < 4 ? u : 0)) / lpg]);
                     }
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
-                                     row + swz(s, 4 * (i4 & 1) + u)),
-                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    if (!act[q]) continue;
+                    const uint32_t cw[4] = {codes[q].x, codes[q].y, codes[q].z, codes[q].w};
+                    const uint32_t row = sK + (ik[q] >> 1) * K_ATOM;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc[q][u], sc[q][u]);
+                        uint32_t w[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t e = lut[(cw[u] >> (8 * k)) & 0xFFu];
+                            const __nv_bfloat162 v =
+                                __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e), s2);
+                            w[k] = *reinterpret_cast<const uint32_t*>(&v);
+                        }
+                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                                         row + swz(sk[q], 4 * (ik[q] & 1) + u)),
+                                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+                    }
                 }
             }
         } else {
@@ -334,6 +391,7 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                              "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
             }
         }
+        cp_async_wait_all();  // the window rows too
         fence_async_smem();
         __syncthreads();
 
@@ -452,10 +510,94 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         tc_fence_after();
     }
 
-    pdl_trigger();  // only the epilogue is left: let the merge be scheduled
+    pdl_trigger();  // only the epilogue is left: let the next kernel be scheduled
 
-    // ---- 6. epilogue: thread = one latent channel, 64 heads from TMEM
-    if (ok && c0 < c1) {
+    if (cluster) {
+        // ---- 6'. the nsplit CTAs of this sequence form one cluster: each puts
+        // its unnormalised O (64 heads x 512 channels, fp32) in its own shared
+        // memory over the free Q and K tiles, then CTA r combines heads
+        // [r*hpc, (r+1)*hpc) from every split through distributed shared
+        // memory, all loads of an item issued before any is used.
+        float* xo = reinterpret_cast<float*>(smem + OFF_Q);
+        float* pm = reinterpret_cast<float*>(smem + OFF_Q + H * DV * 4);  // [nsplit][H]
+        float* pl = pm + 8 * H;                                            // [nsplit][H]
+        const bool mine = ok && c0 < c1;
+        if (mine) {
+            const int g = warp & 3;
+            for (int t = 0; t < 2; ++t) {
+                const int mt = (warp >> 2) * 2 + t;
+                const int d = mt * 128 + g * 32 + lane;
+                for (int h0 = 0; h0 < H; h0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) xo[(h0 + i) * DV + d] = __uint_as_float(r[i]);
+                }
+            }
+        }
+        if (!mine && tid < H) {  // nothing (or nothing valid) from this split
+            mref[tid] = -INFINITY;
+            lrun[tid] = 0.f;
+        }
+        cluster_sync();  // every split's O, m and l are in place
+        const int hpc = (H + nsplit - 1) / nsplit;
+        const int h_lo = split * hpc, h_hi = min(H, h_lo + hpc), nh = h_hi - h_lo;
+        for (int i = tid; i < nsplit * nh; i += NT) {  // the splits' (m, l) of my heads
+            const int s2 = i / nh, h = h_lo + (i - s2 * nh);
+            pm[s2 * H + h] = ld_peer_f32(peer_addr(smem_u32(mref + h), s2));
+            pl[s2 * H + h] = ld_peer_f32(peer_addr(smem_u32(lrun + h), s2));
+        }
+        __syncthreads();
+        float* wts = part;  // [nh][nsplit] weights; fac[] = 1 / L
+        if (tid < nh) {
+            const int h = h_lo + tid;
+            float M = -INFINITY;
+            for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, pm[s2 * H + h]);
+            float L = 0.f;
+            for (int s2 = 0; s2 < nsplit; ++s2) {
+                const float m = pm[s2 * H + h];
+                const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
+                wts[tid * nsplit + s2] = w;
+                L += w * pl[s2 * H + h];
+            }
+            fac[tid] = L > 0.f ? 1.f / L : 0.f;
+            if (a.lse)
+                a.lse[(size_t)b * H + h] = L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f
+                                                   : -INFINITY;
+        }
+        __syncthreads();
+        const uint32_t xo_local = smem_u32(xo);
+        for (int it2 = tid; it2 < nh * (DV / 4); it2 += NT) {
+            const int hh = it2 / (DV / 4), d4 = it2 - hh * (DV / 4);
+            const uint32_t off = (uint32_t)(((h_lo + hh) * DV + 4 * d4) * 4);
+            float4 v[8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+                if (s2 < nsplit && wts[hh * nsplit + s2] != 0.f)
+                    v[s2] = ld_peer_f4(peer_addr(xo_local, s2) + off);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                if (s2 >= nsplit) break;
+                const float w = wts[hh * nsplit + s2];
+                if (w == 0.f) continue;
+                acc.x = fmaf(w, v[s2].x, acc.x);
+                acc.y = fmaf(w, v[s2].y, acc.y);
+                acc.z = fmaf(w, v[s2].z, acc.z);
+                acc.w = fmaf(w, v[s2].w, acc.w);
+            }
+            const float inv = fac[hh];
+            *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h_lo + hh) * DV + 4 * d4) =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        }
+        cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+        if (!ok && tid == 0) {
+            set_status(a.status, KVC_DEV_TIMEOUT);
+            mbar_wait(smem_u32(&bars[0]), 0);
+            mbar_wait(smem_u32(&bars[1]), 0);
+        }
+    } else if (ok && c0 < c1) {
+        // ---- 6. epilogue: thread = one latent channel, 64 heads from TMEM
         const int g = warp & 3;  // TMEM lanes 32g .. 32g+31
         for (int t = 0; t < 2; ++t) {
             const int mt = (warp >> 2) * 2 + t;
@@ -514,32 +656,58 @@ bool tc05_supported(const kvc_config& c, const Shape& sh) {
            sh.Dv == tc05::DV && sh.rb <= (int)tc05::RAW_STRIDE;
 }
 
-// Launches the chunks of every sequence; returns the number of splits (chunks)
-// so the caller merges them, or a negative value on a launch error.
+// Launches the chunks of every sequence; returns the number of partial
+// results the caller still has to merge (1 when the kernel wrote the final
+// output itself), or a negative value on a launch error.
 int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                           cudaStream_t s) {
     const int total = c.topk + a.window_len;
     const int nchunks = (total + tc05::CK - 1) / tc05::CK;
-    // two chunks per CTA: one wave at the batched workload, fewer partials
-    const int cps = nchunks <= 1 ? 1 : 2 + (nchunks - 1) / (2 * kMaxSplit);
-    const int nsplit = nchunks == 0 ? 1 : (nchunks + cps - 1) / cps;
-    if (nsplit > kMaxSplit) return -1;
     static bool attr_set[64] = {};
+    static int sm_count[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
+    int sms = 148;
+    if (dev >= 0 && dev < 64) {
+        if (!sm_count[dev]) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+        sms = sm_count[dev];
+    }
+    // chunks per CTA: as few as keep every (sequence, split) CTA in one wave
+    // (one CTA per SM), and at most kMaxSplit splits
+    int cps = (int)(((long long)a.batch * nchunks + sms - 1) / sms);
+    cps = std::max(cps, (nchunks + kMaxSplit - 1) / kMaxSplit);
+    cps = std::max(cps, 1);
+    const int nsplit = nchunks == 0 ? 1 : (nchunks + cps - 1) / cps;
+    if (nsplit > kMaxSplit) return -1;
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(tc05::attn_tc05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tc05::SMEM_BYTES) != cudaSuccess)
             return -1;
         attr_set[dev] = true;
     }
+    // the splits of one sequence merge inside a cluster when they fit one
+    const int cluster = (nsplit > 1 && nsplit <= 8) ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nsplit, a.batch);
+    cfg.blockDim = dim3(tc05::NT);
+    cfg.dynamicSmemBytes = tc05::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster ? nsplit : 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     trace_before("attn_tc05", s);
-    const cudaError_t e = launch_pdl(tc05::attn_tc05_kernel, dim3(nsplit, a.batch), tc05::NT,
-                                     tc05::SMEM_BYTES, s, a, sh, c.topk,
-                                     c.sm_scale * 1.4426950408889634f, nsplit, cps,
-                                     (int)(c.scale_fmt == KVC_SCALE_UE4M3));
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, tc05::attn_tc05_kernel, a, sh, c.topk,
+                                             c.sm_scale * 1.4426950408889634f, nsplit, cps,
+                                             (int)(c.scale_fmt == KVC_SCALE_UE4M3), cluster);
     trace_after(s);
-    return e == cudaSuccess ? nsplit : -1;
+    if (e != cudaSuccess) return -1;
+    return cluster ? 1 : nsplit;  // a merged cluster needs no merge kernel
 }
 
 }  // namespace kvc

@@ -132,3 +132,20 @@ def test_attention_online_rescale(kvc):
     assert ref_lse[0, 0] / np.log(2) > 60  # head 0's maximum jumped by > 8 (log2)
     assert_attn_close(out, ref, "rescale")
     assert np.max(np.abs(lse - ref_lse)) < 2e-3 * np.abs(ref_lse).max()
+
+
+@pytest.mark.parametrize("topk", [192, 1024, 2048])
+def test_attention_split_counts(kvc, topk):
+    """Key counts that give 4 splits per sequence (merged inside a thread-block
+    cluster) and 12 splits of one and of two chunks each (more than a cluster
+    holds: merged by the separate merge kernel)."""
+    w = synth.WORKLOADS["mla32k"].scaled(context=2 * 5000, topk=topk, batch=3)
+    inp, rec, ic, n, cfg, cache = _setup(kvc, w)
+    ocfg = oracle_cfg(w)
+    tk = oracle.index_topk(ocfg, inp["idx_q"][0].numpy(), ic, n)
+    q, win = inp["q"][0], inp["windows"][0]
+    out, lse, st = _attn(kvc, cfg, cache, q, torch.from_numpy(tk), win, w.window)
+    ref, ref_lse, _ = oracle.sparse_decode(ocfg, f32(q), rec, n, tk, f32(win), w.window)
+    assert st == 0
+    assert_attn_close(out, ref, f"topk={topk}")
+    assert np.max(np.abs(lse - ref_lse)) < 2e-3 * np.abs(ref_lse).max()
