@@ -37,7 +37,7 @@ METRIC = "sparse FP4-KV decode query-tokens/s; achieved HBM GB/s vs 8 TB/s"
 UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNELS = ("pack", "pack_commit", "topk_zero", "index_scan", "topk_select", "block_max",
-           "pool_len", "copy_topk", "attn_tc05", "attn_simt", "attn_merge")
+           "copy_topk", "attn_tc05", "attn_simt", "attn_merge")
 
 
 def parse():

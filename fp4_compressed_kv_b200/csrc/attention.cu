@@ -206,6 +206,15 @@ attn_merge_kernel(AttnArgs a, int H, int Dv, int nsplit) {
     if (tid == 0 && a.lse) a.lse[(size_t)b * H + h] = s_lse;
 }
 
+// A Reuse layer's copy of its head's top-K (the tensor-core kernel writes it
+// itself while it reads the indices).
+__global__ void copy_topk_kernel(const int32_t* __restrict__ src, int32_t* __restrict__ dst,
+                                 int n) {
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        dst[i] = src[i];
+}
+
 }  // namespace
 
 bool tc05_supported(const kvc_config& c, const Shape& sh);
@@ -222,7 +231,7 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
     cudaGetDevice(&dev);
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t err;
+    cudaError_t err = cudaSuccess;
     int nsplit;
     if (tc05_supported(c, sh)) {
         nsplit = launch_attention_tc05(c, sh, a, s);
@@ -259,6 +268,14 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
                              scale_log2, cps, nsplit, ue4m3);
         trace_after(s);
         if (err != cudaSuccess) return err;
+        if (a.topk_copy) {
+            const int cnt = a.batch * K;
+            trace_before("copy_topk", s);
+            err = launch_pdl(copy_topk_kernel, (cnt + 1023) / 1024, 256, 0, s, a.topk_idx,
+                             a.topk_copy, cnt);
+            trace_after(s);
+            if (err != cudaSuccess) return err;
+        }
     }
     if (nsplit > 1) {
         trace_before("attn_merge", s);

@@ -8,24 +8,32 @@
 // window), part 4 "P4 main KV" (FP4 is dequantised before attention).  One
 // softmax runs jointly over the selected entries and the window keys.
 //
-// One CTA (256 threads) owns one chunk of 96 keys of one sequence:
-//  1. cp.async gathers the 96 selected records (16-byte rows) and window rows;
-//     Q (64 x 576 bf16) lands in a 128B-swizzled K-major tile.
-//  2. Records are dequantised in registers (E2M1 x scale, exact in bf16 for
-//     UE4M3 scales) into the K tile, 128B-swizzled K-major: 9 atoms of 64
-//     channels x 96 keys.
+// One CTA (256 threads) owns one to a few chunks of 96 keys of one sequence;
+// the operands are f16 (exact for every dequantised entry and for bf16
+// queries and window rows in the f16 range):
+//  1. Q (64 x 576) is converted from bf16 once into a 128B-swizzled K-major
+//     tile.  Per chunk, cp.async gathers the selected records (16-byte
+//     rows) as one group and the window rows as a second group.
+//  2. Records are dequantised by the hardware E2M1 -> f16x2 conversion times
+//     the f16x2 group scale (exact: at most 6 significant bits) into the K
+//     tile, 128B-swizzled K-major: 9 atoms of 64 channels x 96 keys, while the
+//     window rows land; those are then converted to f16 in place.
 //  3. One thread issues S = Q K^T: 36 tcgen05.mma (M=128, N=96, K=16) into
 //     TMEM; rows 64..127 of the A operand read the next atom (don't-care rows).
-//  4. Warps 0-1 read their head's S row from TMEM (one thread per head), take
-//     max / exp2 / sum in fp32 and write P (bf16) 128B-swizzled K-major.
-//  5. One thread issues O^T = V^T P^T: the K tile's latent atoms read as an
+//  4. Four warps read the head rows of S from TMEM, take max / exp2 / sum in
+//     fp32 against a lazily moved reference and write P (f16) 128B-swizzled.
+//  5. One thread issues O^T += V^T P^T: the K tile's latent atoms read as an
 //     MN-major operand (no second copy), 4 x 6 tcgen05.mma (M=128 channels,
 //     N=64 heads, K=16 keys) into TMEM.
-//  6. All warps read O^T from TMEM and store the chunk's partial (m, l, O);
-//     attn_merge combines the chunks of a sequence by log-sum-exp.
+//  6. The splits of a sequence (at most 8) form a thread-block cluster: each
+//     stores its unnormalised O and (m, l) (they stay in L2), one cluster
+//     barrier orders the stores, and CTA r combines heads [r*64/n,
+//     (r+1)*64/n) from all of them.  With more splits the partials go to
+//     attn_merge.
 // Every wait on an mbarrier is bounded by a 2-second clock; on expiry the CTA
 // sets KVC_DEV_TIMEOUT, frees its tensor memory and returns.
 #include <algorithm>
+#include <cuda_fp16.h>
 
 #include "kvc_internal.cuh"
 
@@ -46,16 +54,12 @@ constexpr uint32_t OFF_RAW = OFF_K + K_BYTES;   // P (16 KB) reuses this after d
 constexpr uint32_t OFF_P = OFF_RAW;
 constexpr uint32_t OFF_MISC = OFF_RAW + RAW_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;  // + misc + table + alignment slack
-// Cluster epilogue scratch over Q, K and the raw rows: this split's O
-// [H][DV] fp32, then the splits' (m, l) of the heads this CTA combines.
-static_assert((uint32_t)H * DV * 4 + 2 * 8 * H * 4 <= OFF_MISC, "epilogue scratch below misc");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0, O_COL = 128;
 
-// instruction descriptors (kind::f16): D f32, A and B bf16, M = 128
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(CK >> 3) << 17) |
-                              ((uint32_t)(128 >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) /* A MN-major */ |
+// instruction descriptors (kind::f16): D f32, A and B f16 (type code 0), M = 128
+constexpr uint32_t kIdescQK = (1u << 4) | ((uint32_t)(CK >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 15) /* A MN-major */ |
                               ((uint32_t)(H >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -141,15 +145,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
 
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-    const uint32_t m = c & 7u;  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6
-    const float mag =
-        m < 4u ? 0.5f * (float)m : (float)(1u << (m >> 1)) * (1.0f + 0.5f * (m & 1u)) * 0.5f;
-    return (c & 8u) ? -mag : mag;
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&v);
+}
+// two bf16 (low half first) -> two f16; exact for |x| in [2^-14, 65504]
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// eight E2M1 codes (channel 2i in the low nibble of byte i) -> four f16x2
+// words, each times the f16x2 scale s2 (a code times a UE4M3 scale has at
+// most 6 significant bits and stays in the f16 range: the product is exact)
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t codes, __half2 s2, uint32_t (&w)[4]) {
+    uint32_t r[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(codes));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&r[k]), s2);
+        w[k] = *reinterpret_cast<const uint32_t*>(&v);
+    }
 }
 
 // byte offset of 16-byte chunk `c16` of row `r` inside a 128B-swizzled block
@@ -193,25 +214,6 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::
                      : "memory");
 }
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
-    float4 v;
-    asm("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];\n"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ float ld_peer_f32(uint32_t addr) {
-    float v;
-    asm("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr));
-    return v;
-}
-
 __global__ void __launch_bounds__(NT, 1)
 attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int cps, int ue4m3,
                  int cluster) {
@@ -230,7 +232,6 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_MISC + 2048);  // S done, O done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 2112);
     int* flags = reinterpret_cast<int*>(smem + OFF_MISC + 2176);
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + OFF_MISC + 3072);  // [256] bf16x2
 
     const int b = blockIdx.y, split = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -253,18 +254,23 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         mref[tid] = -INFINITY;
         lrun[tid] = 0.f;
     }
-    // code-pair table: byte -> (E2M1(low nibble), E2M1(high nibble)) as bf16x2
-    lut[tid] = pack_bf16(e2m1_value(tid & 15u), e2m1_value(tid >> 4));
     pdl_wait();  // everything above was local set-up
     const int n = a.n_entries[b];
     const bool len_ok = n >= 0 && n <= a.capacity;
-    // Q (64 x 576) once, 128B-swizzled K-major
+    // Q (64 x 576) once, converted to f16, 128B-swizzled K-major
     {
-        const unsigned char* qg = static_cast<const unsigned char*>(a.q) + (size_t)b * H * D * 2;
+        const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(a.q) +
+                                                         (size_t)b * H * D * 2);
+#pragma unroll 6
         for (int p = tid; p < H * (D / 8); p += NT) {
             const int h = p / (D / 8), c = p - h * (D / 8);
-            cp_async16(sQ + (c >> 3) * 8192u + swz(h, c & 7), qg + (size_t)h * D * 2 + c * 16);
+            const uint4 v = __ldg(qg + p);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                             sQ + (c >> 3) * 8192u + swz(h, c & 7)),
+                         "r"(bf16x2_to_f16x2(v.x)), "r"(bf16x2_to_f16x2(v.y)),
+                         "r"(bf16x2_to_f16x2(v.z)), "r"(bf16x2_to_f16x2(v.w)));
         }
+        fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -277,6 +283,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         // ---- slot kinds of this chunk
         if (tid < CK) {
             const int j = c * CK + tid;
+            if (a.topk_copy && j < K)  // a Reuse layer's own copy of its head's top-K
+                a.topk_copy[(size_t)b * K + j] = a.topk_idx[(size_t)b * K + j];
             int k = -1;
             if (j < total && len_ok) {
                 if (j < K) {
@@ -327,71 +335,50 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         // the bf16x2 scale of its group (the products have at most 6
         // significant bits, so the bf16 multiply is exact).  Groups of >= 32
         // share one scale per item; groups of 8 or 16 take one per 8 channels.
-        if (ue4m3) {
-            // two items per pass, all their shared-memory loads issued first
+        {
+            // 32 channels per item: one 16-byte load of codes, a scale per group
+            // (per 8 channels for groups of 8 or 16), hardware E2M1 -> f16x2
+            // conversion times the f16x2 scale, four 16-byte stores
             const int lpg = sh.lpg;
             constexpr int NI = CK * (D / 32);
-            for (int p0 = tid; p0 < NI; p0 += 2 * NT) {
-                uint4 codes[2];
-                float sc[2][4];
-                int sk[2], ik[2];
-                bool act[2];
+#pragma unroll 2
+            for (int p = tid; p < NI; p += NT) {
+                const int sk = p / (D / 32), ik = p - sk * (D / 32);
+                if (kind[sk] < 0) continue;
+                const unsigned char* rec = raw + sk * RAW_STRIDE;
+                const uint4 codes = *reinterpret_cast<const uint4*>(rec + ik * 16);
+                const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
+                const uint32_t row = sK + (ik >> 1) * K_ATOM;
+                const float s0 = e4m3_to_f32(rec[sh.code_bytes + (4 * ik) / lpg]);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int p = p0 + q * NT;
-                    sk[q] = p / (D / 32);
-                    ik[q] = p - sk[q] * (D / 32);
-                    act[q] = p < NI && kind[sk[q]] >= 0;
-                    if (act[q]) {
-                        const unsigned char* rec = raw + sk[q] * RAW_STRIDE;
-                        codes[q] = *reinterpret_cast<const uint4*>(rec + ik[q] * 16);
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            sc[q][u] = e4m3_to_f32(rec[sh.code_bytes + (4 * ik[q] + (lpg < 4 ? u : 0)) / lpg]);
-                    }
+                for (int u = 0; u < 4; ++u) {
+                    const float su =
+                        lpg >= 4 ? s0 : e4m3_to_f32(rec[sh.code_bytes + (4 * ik + u) / lpg]);
+                    uint32_t w[4];
+                    e2m1x8_to_f16(cw[u], __floats2half2_rn(su, su), w);
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                                     row + swz(sk, 4 * (ik & 1) + u)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
                 }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    if (!act[q]) continue;
-                    const uint32_t cw[4] = {codes[q].x, codes[q].y, codes[q].z, codes[q].w};
-                    const uint32_t row = sK + (ik[q] >> 1) * K_ATOM;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc[q][u], sc[q][u]);
-                        uint32_t w[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t e = lut[(cw[u] >> (8 * k)) & 0xFFu];
-                            const __nv_bfloat162 v =
-                                __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e), s2);
-                            w[k] = *reinterpret_cast<const uint32_t*>(&v);
-                        }
-                        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
-                                         row + swz(sk[q], 4 * (ik[q] & 1) + u)),
-                                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
-                    }
-                }
-            }
-        } else {
-            for (int p = tid; p < CK * (D / 8); p += NT) {
-                const int s = p / (D / 8), cc = p - s * (D / 8);
-                if (kind[s] < 0) continue;
-                const unsigned char* rec = raw + s * RAW_STRIDE;
-                const uint32_t codes = *reinterpret_cast<const uint32_t*>(rec + cc * 4);
-                const int g = cc / sh.lpg;
-                const float sc = ue4m3 ? e4m3_to_f32(rec[sh.code_bytes + g])
-                                       : reinterpret_cast<const float*>(rec + sh.code_bytes)[g];
-                uint32_t w[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    w[k] = pack_bf16(e2m1_value((codes >> (8 * k)) & 15u) * sc,
-                                     e2m1_value((codes >> (8 * k + 4)) & 15u) * sc);
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
-                                 sK + (cc >> 3) * K_ATOM + swz(s, cc & 7)),
-                             "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
             }
         }
         cp_async_wait_all();  // the window rows too
+        if (other_rows) {
+            __syncthreads();  // every thread's window copies have landed
+            // window rows arrived as bf16: convert them in place to f16
+            for (int p = tid; p < CK * (D / 8); p += NT) {
+                const int s = p / (D / 8), cc = p - s * (D / 8);
+                if (kind[s] > -2) continue;
+                const uint32_t addr = sK + (cc >> 3) * K_ATOM + swz(s, cc & 7);
+                uint32_t v0, v1, v2, v3;
+                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                             : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                             : "r"(addr));
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr),
+                             "r"(bf16x2_to_f16x2(v0)), "r"(bf16x2_to_f16x2(v1)),
+                             "r"(bf16x2_to_f16x2(v2)), "r"(bf16x2_to_f16x2(v3)));
+            }
+        }
         fence_async_smem();
         __syncthreads();
 
@@ -453,8 +440,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                 const int kc = half * (CK / 16) + cj;  // 8-key chunk index in the P row
                 const uint32_t dst = sP + (kc >> 3) * 8192u + swz(h, kc & 7);
                 asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst),
-                             "r"(pack_bf16(pv[0], pv[1])), "r"(pack_bf16(pv[2], pv[3])),
-                             "r"(pack_bf16(pv[4], pv[5])), "r"(pack_bf16(pv[6], pv[7])));
+                             "r"(pack_f16(pv[0], pv[1])), "r"(pack_f16(pv[2], pv[3])),
+                             "r"(pack_f16(pv[4], pv[5])), "r"(pack_f16(pv[6], pv[7])));
             }
             __syncwarp();
             sv[0] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
@@ -513,15 +500,13 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
     pdl_trigger();  // only the epilogue is left: let the next kernel be scheduled
 
     if (cluster) {
-        // ---- 6'. the nsplit CTAs of this sequence form one cluster: each puts
-        // its unnormalised O (64 heads x 512 channels, fp32) in its own shared
-        // memory over the free Q and K tiles, then CTA r combines heads
-        // [r*hpc, (r+1)*hpc) from every split through distributed shared
-        // memory, all loads of an item issued before any is used.
-        float* xo = reinterpret_cast<float*>(smem + OFF_Q);
-        float* pm = reinterpret_cast<float*>(smem + OFF_Q + H * DV * 4);  // [nsplit][H]
-        float* pl = pm + 8 * H;                                            // [nsplit][H]
+        // ---- 6'. the nsplit CTAs of this sequence form one cluster.  Each
+        // stores its unnormalised O and (m, l) to the partial buffers (they
+        // stay in L2), the cluster barrier orders those stores before every
+        // CTA's loads, then CTA r combines heads [r*hpc, (r+1)*hpc) from all
+        // splits and writes the final rows: no separate merge launch.
         const bool mine = ok && c0 < c1;
+        const size_t prow0 = (size_t)b * H * kMaxSplit;  // row (b, h, split) = prow0 + h*kMaxSplit + split
         if (mine) {
             const int g = warp & 3;
             for (int t = 0; t < 2; ++t) {
@@ -531,34 +516,39 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                     uint32_t r[32];
                     tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) xo[(h0 + i) * DV + d] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 32; ++i)
+                        __stcg(a.part_o + (prow0 + (size_t)(h0 + i) * kMaxSplit + split) * DV + d,
+                               __uint_as_float(r[i]));
                 }
             }
         }
-        if (!mine && tid < H) {  // nothing (or nothing valid) from this split
-            mref[tid] = -INFINITY;
-            lrun[tid] = 0.f;
+        if (tid < H) {  // nothing (or nothing valid) from this split: weight 0
+            const size_t row = prow0 + (size_t)tid * kMaxSplit + split;
+            __stcg(a.part_ml + row * 2, mine ? mref[tid] : -INFINITY);
+            __stcg(a.part_ml + row * 2 + 1, mine ? lrun[tid] : 0.f);
         }
-        cluster_sync();  // every split's O, m and l are in place
+        cluster_sync();  // every split's partial is stored
         const int hpc = (H + nsplit - 1) / nsplit;
         const int h_lo = split * hpc, h_hi = min(H, h_lo + hpc), nh = h_hi - h_lo;
-        for (int i = tid; i < nsplit * nh; i += NT) {  // the splits' (m, l) of my heads
-            const int s2 = i / nh, h = h_lo + (i - s2 * nh);
-            pm[s2 * H + h] = ld_peer_f32(peer_addr(smem_u32(mref + h), s2));
-            pl[s2 * H + h] = ld_peer_f32(peer_addr(smem_u32(lrun + h), s2));
-        }
-        __syncthreads();
         float* wts = part;  // [nh][nsplit] weights; fac[] = 1 / L
         if (tid < nh) {
             const int h = h_lo + tid;
+            const size_t row = prow0 + (size_t)h * kMaxSplit;
+            float m[8], l[8];
             float M = -INFINITY;
-            for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, pm[s2 * H + h]);
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                m[s2] = s2 < nsplit ? __ldcg(a.part_ml + (row + s2) * 2) : -INFINITY;
+                l[s2] = s2 < nsplit ? __ldcg(a.part_ml + (row + s2) * 2 + 1) : 0.f;
+                M = fmaxf(M, m[s2]);
+            }
             float L = 0.f;
-            for (int s2 = 0; s2 < nsplit; ++s2) {
-                const float m = pm[s2 * H + h];
-                const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                if (s2 >= nsplit) break;
+                const float w = (M == -INFINITY || m[s2] == -INFINITY) ? 0.f : exp2f(m[s2] - M);
                 wts[tid * nsplit + s2] = w;
-                L += w * pl[s2 * H + h];
+                L += w * l[s2];
             }
             fac[tid] = L > 0.f ? 1.f / L : 0.f;
             if (a.lse)
@@ -566,31 +556,43 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                                                    : -INFINITY;
         }
         __syncthreads();
-        const uint32_t xo_local = smem_u32(xo);
-        for (int it2 = tid; it2 < nh * (DV / 4); it2 += NT) {
-            const int hh = it2 / (DV / 4), d4 = it2 - hh * (DV / 4);
-            const uint32_t off = (uint32_t)(((h_lo + hh) * DV + 4 * d4) * 4);
-            float4 v[8];
+        // four items per pass: up to 4 x nsplit 16-byte L2 loads in flight
+        constexpr int UNR = 4;
+        for (int base = tid; base < nh * (DV / 4); base += UNR * NT) {
+            float4 v[UNR][8];
 #pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2)
-                if (s2 < nsplit && wts[hh * nsplit + s2] != 0.f)
-                    v[s2] = ld_peer_f4(peer_addr(xo_local, s2) + off);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int u = 0; u < UNR; ++u) {
+                const int it2 = base + u * NT;
+                if (it2 >= nh * (DV / 4)) continue;
+                const int hh = it2 / (DV / 4), d4 = it2 - hh * (DV / 4);
+                const float4* src = reinterpret_cast<const float4*>(
+                    a.part_o + (prow0 + (size_t)(h_lo + hh) * kMaxSplit) * DV + 4 * d4);
 #pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) {
-                if (s2 >= nsplit) break;
-                const float w = wts[hh * nsplit + s2];
-                if (w == 0.f) continue;
-                acc.x = fmaf(w, v[s2].x, acc.x);
-                acc.y = fmaf(w, v[s2].y, acc.y);
-                acc.z = fmaf(w, v[s2].z, acc.z);
-                acc.w = fmaf(w, v[s2].w, acc.w);
+                for (int s2 = 0; s2 < 8; ++s2)
+                    if (s2 < nsplit && wts[hh * nsplit + s2] != 0.f)
+                        v[u][s2] = __ldcg(src + (size_t)s2 * (DV / 4));
             }
-            const float inv = fac[hh];
-            *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h_lo + hh) * DV + 4 * d4) =
-                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int it2 = base + u * NT;
+                if (it2 >= nh * (DV / 4)) continue;
+                const int hh = it2 / (DV / 4), d4 = it2 - hh * (DV / 4);
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int s2 = 0; s2 < 8; ++s2) {
+                    if (s2 >= nsplit) break;
+                    const float w = wts[hh * nsplit + s2];
+                    if (w == 0.f) continue;
+                    acc.x = fmaf(w, v[u][s2].x, acc.x);
+                    acc.y = fmaf(w, v[u][s2].y, acc.y);
+                    acc.z = fmaf(w, v[u][s2].z, acc.z);
+                    acc.w = fmaf(w, v[u][s2].w, acc.w);
+                }
+                const float inv = fac[hh];
+                *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h_lo + hh) * DV + 4 * d4) =
+                    make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            }
         }
-        cluster_sync();  // no CTA leaves while a peer may still read its shared memory
         if (!ok && tid == 0) {
             set_status(a.status, KVC_DEV_TIMEOUT);
             mbar_wait(smem_u32(&bars[0]), 0);
@@ -652,8 +654,8 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
 }  // namespace tc05
 
 bool tc05_supported(const kvc_config& c, const Shape& sh) {
-    return c.act_dtype == KVC_BF16 && c.n_heads == tc05::H && sh.D == tc05::D &&
-           sh.Dv == tc05::DV && sh.rb <= (int)tc05::RAW_STRIDE;
+    return c.act_dtype == KVC_BF16 && c.scale_fmt == KVC_SCALE_UE4M3 && c.n_heads == tc05::H &&
+           sh.D == tc05::D && sh.Dv == tc05::DV && sh.rb <= (int)tc05::RAW_STRIDE;
 }
 
 // Launches the chunks of every sequence; returns the number of partial

@@ -410,8 +410,29 @@ constexpr size_t kFinishSmem =
     (size_t)kStageKeys * 8 + (size_t)kMaxTies * 8 + (size_t)kMaxSelTiles * 4 * 2;
 
 // One CTA per sequence finishes the selection from the tiles' candidates.
+__device__ void finish_body(const TopkArgs& a, int b, int bias, int shift, unsigned char* smem);
+
+// Finishes sequence b; in the hierarchical block stage also derives the pool
+// length (whole kept blocks, the sequence's last block counting only its
+// visible entries).
 __device__ void finish_sequence(const TopkArgs& a, int b, int bias, int shift,
                                 unsigned char* smem) {
+    finish_body(a, b, bias, shift, smem);
+    if (!a.pool_len_out) return;
+    __syncthreads();  // this CTA's output writes are visible to its threads
+    if (threadIdx.x == 0) {
+        const int nb = a.n_entries[b];  // blocks of the sequence
+        const int n0 = a.pool_src_n[b];
+        const int n = (n0 >= 0 && n0 <= a.pool_src_cap) ? n0 : 0;
+        const int kept = (nb >= 0 && nb <= a.capacity) ? min(a.topk, nb) : 0;
+        int len = kept * a.pool_src_block;
+        if (kept > 0 && __ldcg(a.topk_idx + (size_t)b * a.topk + kept - 1) == nb - 1)
+            len -= nb * a.pool_src_block - n;
+        a.pool_len_out[b] = len;
+    }
+}
+
+__device__ void finish_body(const TopkArgs& a, int b, int bias, int shift, unsigned char* smem) {
     unsigned long long* stage = reinterpret_cast<unsigned long long*>(smem);  // kStageKeys
     unsigned long long* ties = stage + kStageKeys;                            // kMaxTies
     int* cnt = reinterpret_cast<int*>(ties + kMaxTies);                       // per tile
@@ -683,7 +704,7 @@ __global__ void zero_counters_kernel(int32_t* p, int n) {
 }
 
 // ---- hierarchical indexer, block stage
-constexpr int kBlkPerThread = 8;
+constexpr int kBlkPerThread = 4;
 constexpr int kBlkPerCta = kThreads * kBlkPerThread;
 
 // Block scores of one tile of kBlkPerCta blocks of a sequence: the highest
@@ -703,21 +724,41 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
     const int ntiles = (nb + kBlkPerCta - 1) / kBlkPerCta;
     if ((int)blockIdx.x >= ntiles) return;
     for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
-    __syncthreads();
     const int32_t* sc = h.scores + (size_t)b * h.capacity;
     int32_t* bs = h.bscore + (size_t)b * cap_blk;
+    if (h.block <= 8) {  // every load of the thread's blocks in flight at once
+        int v[kBlkPerThread][8];
 #pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-        const int j = blockIdx.x * kBlkPerCta + u * kThreads + tid;
-        if (j < nb) {
+        for (int u = 0; u < kBlkPerThread; ++u) {
+            const int j = blockIdx.x * kBlkPerCta + u * kThreads + tid;
+            const int e0 = j * h.block, e1 = j < nb ? min(n, e0 + h.block) : e0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[u][q] = e0 + q < e1 ? __ldcg(sc + e0 + q) : INT_MIN;
+        }
+        __syncthreads();  // histogram zeroed
+#pragma unroll
+        for (int u = 0; u < kBlkPerThread; ++u) {
+            const int j = blockIdx.x * kBlkPerCta + u * kThreads + tid;
+            if (j >= nb) continue;
+            int m = v[u][0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q) m = max(m, v[u][q]);
+            bs[j] = m;
+            atomicAdd(&hist[score_bin(m, bias, shift)], 1);
+        }
+    } else {
+        __syncthreads();
+        for (int u = 0; u < kBlkPerThread; ++u) {
+            const int j = blockIdx.x * kBlkPerCta + u * kThreads + tid;
+            if (j >= nb) continue;
             const int e0 = j * h.block, e1 = min(n, e0 + h.block);
             int m = INT_MIN;
-            for (int e = e0; e < e1; e += 8) {  // eight loads in flight per pass
-                int v[8];
+            for (int e = e0; e < e1; e += 8) {
+                int w[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = e + u < e1 ? __ldcg(sc + e + u) : INT_MIN;
+                for (int q = 0; q < 8; ++q) w[q] = e + q < e1 ? __ldcg(sc + e + q) : INT_MIN;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) m = max(m, v[u]);
+                for (int q = 0; q < 8; ++q) m = max(m, w[q]);
             }
             bs[j] = m;
             atomicAdd(&hist[score_bin(m, bias, shift)], 1);
@@ -743,22 +784,6 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
         h.thr[2 * b] = s_t;
         h.thr[2 * b + 1] = s_above;
     }
-}
-
-// Pool length of each sequence: whole kept blocks, the last block of the
-// sequence counting only its visible entries.
-__global__ void pool_len_kernel(HierArgs h) {
-    pdl_wait();
-    const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= h.batch) return;
-    const int n0 = h.n_entries[b];
-    const int n = (n0 >= 0 && n0 <= h.capacity) ? n0 : 0;
-    const int nb = (n + h.block - 1) / h.block;
-    const int32_t* blocks = h.pool_blocks + (size_t)b * h.keep;
-    const int k = min(h.keep, nb);  // the selection keeps min(keep, blocks) blocks
-    int len = k * h.block;
-    if (k > 0 && blocks[k - 1] == nb - 1) len -= nb * h.block - n;
-    h.pool_n[b] = len;
 }
 
 template <int DI>
@@ -831,11 +856,11 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
     a.tile_count = h.tile_count;
     a.cands = h.cands;
     a.status = h.status;
-    if ((err = launch_select(a, bias, shift, s)) != cudaSuccess) return err;
-    trace_before("pool_len", s);
-    err = launch_pdl(pool_len_kernel, (h.batch + 127) / 128, 128, 0, s, h);
-    trace_after(s);
-    return err;
+    a.pool_len_out = h.pool_n;
+    a.pool_src_n = h.n_entries;
+    a.pool_src_cap = h.capacity;
+    a.pool_src_block = h.block;
+    return launch_select(a, bias, shift, s);
 }
 
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {

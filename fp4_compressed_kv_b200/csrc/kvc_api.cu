@@ -118,15 +118,6 @@ cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3, 
 }
 
 namespace {
-// Copies a Reuse layer's borrowed top-K rows (a kernel, so the launch chain
-// of a layer group stays kernel to kernel).
-__global__ void copy_topk_kernel(const int32_t* __restrict__ src, int32_t* __restrict__ dst,
-                                 int n) {
-    pdl_wait();
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
-        dst[i] = src[i];
-}
-
 // ------------------------------------------------------------------ workspace
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -278,8 +269,9 @@ kvc_status run_pool_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cac
 kvc_status run_attn(const kvc_config& c, const Shape& sh, const void* q, const kvc_cache* cache,
                     const int32_t* topk, const void* window, int window_len, float* out,
                     float* lse, unsigned char* ws, const WsLayout& w, uint32_t* st,
-                    cudaStream_t s) {
-    AttnArgs a;
+                    cudaStream_t s, int32_t* topk_copy = nullptr) {
+    AttnArgs a = {};
+    a.topk_copy = topk_copy;
     a.q = q;
     a.records = static_cast<const uint8_t*>(cache->records);
     a.n_entries = cache->n_entries;
@@ -468,19 +460,15 @@ kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int
                                s);
             if (st != KVC_OK) return st;
             head = l;
-        } else {
-            const int cnt = (int)(B * K);
-            trace_before("copy_topk", s);
-            const cudaError_t e = launch_pdl(copy_topk_kernel, (cnt + 1023) / 1024, 256, 0, s,
-                                             static_cast<const int32_t*>(topk + (size_t)head * B * K),
-                                             tk, cnt);
-            trace_after(s);
-            if (e != cudaSuccess) return KVC_ERR_CUDA;
         }
-        st = run_attn(*cfg, sh, static_cast<const unsigned char*>(q) + l * q_stride, cache, tk,
+        // a Reuse layer attends over its head's top-K; the attention launch
+        // also writes the layer's own copy of those indices
+        const bool reuse = modes[l] == KVC_REUSE;
+        st = run_attn(*cfg, sh, static_cast<const unsigned char*>(q) + l * q_stride, cache,
+                      reuse ? topk + (size_t)head * B * K : tk,
                       windows ? static_cast<const unsigned char*>(windows) + l * w_stride : nullptr,
                       window_len, out + (size_t)l * B * H * sh.Dv, lse ? lse + (size_t)l * B * H : nullptr,
-                      wsb, w, dev_status, s);
+                      wsb, w, dev_status, s, reuse ? tk : nullptr);
         if (st != KVC_OK) return st;
     }
     return KVC_OK;

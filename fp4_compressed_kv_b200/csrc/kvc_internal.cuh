@@ -95,6 +95,12 @@ struct TopkArgs {
     // and the top-K is written as entry indices.
     const int32_t* pool_blocks;  // [B][pool_keep] ascending, or null
     int pool_keep, pool_block;
+    // Block stage of the hierarchical indexer (selecting blocks): when set,
+    // the finish also writes each sequence's pool length, from the entries
+    // pool_src_n (capacity pool_src_cap) cut into blocks of pool_src_block.
+    int32_t* pool_len_out;
+    const int32_t* pool_src_n;
+    int pool_src_cap, pool_src_block;
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
 
@@ -132,6 +138,7 @@ struct AttnArgs {
     float* part_o;          // [B][H][kMaxSplit][Dv]
     float* part_ml;         // [B][H][kMaxSplit][2]
     uint32_t* status;
+    int32_t* topk_copy;     // [B][K]: receives a copy of topk_idx (a Reuse layer's), or null
 };
 cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                              cudaStream_t s);

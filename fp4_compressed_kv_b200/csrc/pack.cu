@@ -61,6 +61,9 @@ struct Chunk<__nv_bfloat16> {
     __device__ __forceinline__ void load(const __nv_bfloat16* p) {
         v = __ldcs(reinterpret_cast<const uint4*>(p));
     }
+    __device__ __forceinline__ void load_cached(const __nv_bfloat16* p) {
+        v = __ldg(reinterpret_cast<const uint4*>(p));
+    }
     __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
     __device__ __forceinline__ void load_shared(const __nv_bfloat16* p) {
         v = *reinterpret_cast<const uint4*>(p);
@@ -79,6 +82,10 @@ struct Chunk<float> {
     __device__ __forceinline__ void load(const float* p) {
         a = __ldcs(reinterpret_cast<const float4*>(p));
         b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void load_cached(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
     }
     __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
     __device__ __forceinline__ void load_shared(const float* p) {
@@ -279,6 +286,122 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
 
+// Streaming form of pack_kernel for groups of at most 64 channels (a group's
+// chunks then sit in the team's lanes at the same chunk step): the same
+// arithmetic in the same order, but no token chunk is held across the whole
+// entry.  Pass 1 streams the chunks for the gate; pass 2 reloads each chunk
+// (from L1/L2), forms the entry values, takes the group maximum across the
+// team and quantises it right away.  The register footprint drops to a
+// fraction of pack_kernel's, so several times more warps hide the latency.
+template <typename T, int MAXJ>
+__global__ void __launch_bounds__(kThreads, 5)
+pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
+    pdl_wait();
+    __shared__ __align__(16) uint8_t tail_smem[kTeams][kTailBytes];
+    const int lane = threadIdx.x & 31;
+    const int team = threadIdx.x >> 3, l = threadIdx.x & 7;
+    const long long e = (long long)blockIdx.x * kTeams + team;
+    const int half = a.n_new >> 1;
+    const bool in_range = e < (long long)a.batch * half;
+    int b = 0, i = 0, base = 0;
+    bool valid = false;
+    if (in_range) {
+        b = (int)(e / half);
+        i = (int)(e % half);
+        base = a.n_entries[b];
+        valid = base >= 0 && base + half <= a.capacity;
+        if (!valid && i == 0 && l == 0) set_status(a.status, KVC_DEV_CAPACITY);
+    }
+    const int D = sh.D, nchunk = D >> 3;
+    const long long pos = (long long)base + i;
+    const T* k0p = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 2 * i) * D;
+    const T* k1p = k0p + D;
+
+    // pass 1: gate logit difference, fixed order (lane l: chunks l, l+8, ...)
+    float acc = 0.f;
+#pragma unroll 3
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = l + 8 * j;
+        if (valid && c < nchunk) {
+            Chunk<T> x0, x1;
+            x0.load_cached(k0p + 8 * c);
+            x1.load_cached(k1p + 8 * c);
+            float g[8];
+            load8_gate(a.gate + 8 * c, g);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                acc = __fmaf_rn(g[t], __fsub_rn(x0.get(t), x1.get(t)), acc);
+        }
+    }
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
+    const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-acc)));
+    const float w1 = __fsub_rn(1.0f, w0);
+
+    uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
+    uint8_t* tail = tail_smem[team];
+    const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
+    for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
+    __syncwarp();
+
+    // pass 2: entry values, group maxima (xor over the group's lanes), codes
+    bool bad = false;
+    const int lpg = sh.lpg;
+#pragma unroll 2
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = l + 8 * j;
+        const bool active = valid && c < nchunk;
+        Chunk<T> x0, x1;
+        if (active) {
+            x0.load_cached(k0p + 8 * c);
+            x1.load_cached(k1p + 8 * c);
+        } else {
+            x0.zero();
+            x1.zero();
+        }
+        float x[8];
+        float m = 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float v = __fmaf_rn(w0, x0.get(t), __fmul_rn(w1, x1.get(t)));
+            if (!isfinite(v)) {
+                if (active) bad = true;
+                v = 0.f;
+            }
+            x[t] = v;
+            m = fmaxf(m, fabsf(v));
+        }
+        for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (!active) continue;
+        float sc = __fdiv_rn(m, 6.0f);
+        uint32_t sbyte = 0;
+        if (ue4m3) {
+            sbyte = e4m3_from_f32(sc);
+            sc = e4m3_to_f32(sbyte);
+        }
+        *reinterpret_cast<uint32_t*>(rec + 4 * c) = sc > 0.f ? e2m1x8_quotient(x, sc) : 0u;
+        if (c % lpg == 0) {
+            const int gi = c / lpg;
+            if (ue4m3)
+                tail[gi] = (uint8_t)sbyte;
+            else
+                *reinterpret_cast<float*>(tail + 4 * gi) = sc;
+        }
+    }
+    __syncwarp();
+    if (valid) {
+        for (int t = l * 4; t < tail_len; t += 32)
+            *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
+                *reinterpret_cast<const uint32_t*>(tail + t);
+        const uint4* src =
+            reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di);
+        uint4* dst = reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di);
+        for (int p = l; p < (di >> 4); p += 8) dst[p] = __ldcs(src + p);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
+}
+
 // Small appends (decode: one pair per sequence): one warp per entry so the
 // work of a few dozen entries spreads over many SMs.  The whole warp first
 // stages the token pair and the gate in shared memory (one round trip to
@@ -463,6 +586,18 @@ cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
     const unsigned grid = (unsigned)((entries + kTeams - 1) / kTeams);
     const int maxj = (sh.D / 8 + 7) / 8;
     trace_before("pack", s);
+    if (sh.lpg <= 8) {  // groups within one chunk step: the streaming kernel
+        if (maxj <= 2)
+            err = launch_pdl(pack_stream_kernel<T, 2>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+        else if (maxj <= 4)
+            err = launch_pdl(pack_stream_kernel<T, 4>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+        else if (maxj <= 9)
+            err = launch_pdl(pack_stream_kernel<T, 9>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+        else
+            err = launch_pdl(pack_stream_kernel<T, 16>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+        trace_after(s);
+        return err;
+    }
     if (maxj <= 2)
         err = launch_pdl(pack_kernel<T, 2>, grid, kThreads, 0, s, a, sh, ue4m3, di);
     else if (maxj <= 4)

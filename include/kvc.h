@@ -243,8 +243,8 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
  * "pack", "pack_commit", "topk_zero", "index_scan", "topk_select",
- * "block_max", "pool_len", "copy_topk", "attn_tc05", "attn_simt",
- * "attn_merge", "fp4_codec".                                                             */
+ * "block_max", "copy_topk", "attn_tc05", "attn_simt", "attn_merge",
+ * "fp4_codec".                                                             */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);
 kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);
