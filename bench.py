@@ -212,6 +212,49 @@ def traffic_for(kernel):
     return kv
 
 
+def time_scoring(w, steps, warmup, batched, dev):
+    """Device ms to score and select every Full/Reindex layer of workload w
+    (their indexer queries known up front): one batched tensor-core pass, or
+    one scan per layer."""
+    import torch
+    from fp4_compressed_kv_b200 import kvc, synth
+    cfg = kvc.config_for(w)
+    heads = [i for i, m in enumerate(w.modes) if m != synth.REUSE]
+    g = synth.generator(dev, w.seed)
+    cache = kvc.Cache(cfg, w.batch, w.entries, device=dev)
+    cache.idx_k.copy_(torch.randint(-127, 128, cache.idx_k.shape, generator=g, device=dev,
+                                    dtype=torch.int8))
+    cache.n_entries.fill_(w.entries)
+    q = torch.randint(-127, 128, (len(heads), w.batch, w.idx_dim), generator=g, device=dev,
+                      dtype=torch.int8)
+    tk = torch.empty(len(heads), w.batch, w.topk, dtype=torch.int32, device=dev)
+    if batched:
+        ws = kvc.workspace_batched(cfg, len(heads), w.batch, w.entries, device=dev)
+
+        def step():
+            kvc.index_topk_batched(cfg, q, cache, tk, ws)
+    else:
+        ws = kvc.workspace(cfg, w.batch, w.entries, device=dev)
+
+        def step():
+            for i in range(len(heads)):
+                kvc.index_topk(cfg, q[i], cache, tk[i], ws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(steps):
+            step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del gr
+    return e0.elapsed_time(e1) / steps
+
+
 # ----------------------------------------------------------------------------- oracle leg
 def oracle_decode_sample(w, seconds, seed_shift=0):
     """Time the CPU oracle on single-sequence decode steps of workload w.
@@ -504,6 +547,15 @@ def run_ours(args):
                            "query_tokens_per_s_hier": round(wx.batch / (hier * 1e-3), 1),
                            "hier": "2048 blocks of 8 entries"}
             torch.cuda.empty_cache()
+        # every scoring layer's indexer query in one tensor-core pass, against
+        # one scan per layer (a schedule where all queries are known up front)
+        for name in ("csa2group", "stack1m"):
+            wx = synth.WORKLOADS[name]
+            one = time_scoring(wx, 10, 3, False, dev)
+            bat = time_scoring(wx, 10, 3, True, dev)
+            extra[name].update({"scoring_ms_per_layer_scans": round(one, 4),
+                                "scoring_ms_batched_tensor_core": round(bat, 4)})
+            torch.cuda.empty_cache()
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
@@ -543,7 +595,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk,
-        "hier_indexer": extra,
+        "next_rows": extra,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

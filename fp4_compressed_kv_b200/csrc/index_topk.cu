@@ -33,6 +33,7 @@
 //     compacts the scores.
 // No CTA waits on another: the launches are stream-ordered and the last-CTA
 // hand-offs are counters that nobody polls.
+#include <algorithm>
 #include <climits>
 
 #include "kvc_internal.cuh"
@@ -786,6 +787,232 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
     }
 }
 
+// ---- batched scoring on the tensor cores: several indexer queries of the
+// same sequence against each 128-row tile of its indexer keys in one
+// tcgen05.mma kind::i8 (M = 128 rows, N = 16 padded queries, K = 128 int8 as
+// 4 steps of 32), accumulators in tensor memory.  The rows stream in as
+// plain bulk copies and are re-laid into the 128-byte-swizzled K-major
+// operand tile in shared memory; each thread then owns one row's scores.
+namespace tcs {
+constexpr int NT = 128;           // thread t <-> tensor-memory lane t <-> row t of the tile
+constexpr int ROWS = 128;         // rows per tile (MMA M)
+constexpr int DI = 128;           // indexer width: one 128-byte swizzle row
+constexpr int NQP = 16;           // MMA N (queries, padded)
+constexpr int TILE = ROWS * DI;   // 16 KB
+constexpr int MAX_STAGES = 8;
+constexpr uint32_t TMEM_COLS = 32;
+// D s32 (2 << 4), A and B s8 (1 << 7, 1 << 10), both K-major, N = 16, M = 128
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NQP >> 3) << 17) |
+                            ((uint32_t)(ROWS >> 4) << 24);
+
+__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c16) {
+    return (r >> 3) * 1024u + (r & 7u) * 128u + ((c16 ^ (r & 7u)) << 4);
+}
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {  // SW128 K-major, SBO 1024
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(16 >> 4) << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ void mma_i8(uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(ad), "l"(bd), "r"(kIdesc), "r"(acc));
+}
+}  // namespace tcs
+
+__global__ void __launch_bounds__(tcs::NT, 2)
+index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int stages) {
+    using namespace tcs;
+    extern __shared__ __align__(1024) unsigned char tsm[];
+    const TopkArgs& a = ba.q[0];
+    const int nq = ba.nq;
+    // 1024-aligned layout: A tile, B tile, raw ring, histograms [nq][kBins]
+    const uint32_t base0 = smem_addr(tsm);
+    const uint32_t pad = ((base0 + 1023u) & ~1023u) - base0;
+    unsigned char* sm = tsm + pad;
+    const uint32_t sA = smem_addr(sm), sB = sA + TILE;
+    unsigned char* ring = sm + TILE + 2048;
+    int* hist = reinterpret_cast<int*>(ring + (size_t)stages * TILE);
+    __shared__ __align__(8) uint64_t full[MAX_STAGES];
+    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int sh_warp[NT / 32];
+    __shared__ int s_last, s_t, s_above;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const long long cap = a.capacity;
+    const long long lo = (long long)blockIdx.x * per;
+    const long long hi = min(lo + per, (long long)a.batch * cap);
+    if (lo >= hi) return;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_addr(&tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    if (tid == 0) {
+        for (int st = 0; st < stages; ++st)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[st])));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&mma_bar)));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    for (int i = tid; i < nq * kBins; i += NT) hist[i] = 0;
+    pdl_wait();
+    if (tid == 0)
+        for (int b = (int)(lo / cap); b <= (int)((hi - 1) / cap); ++b) {
+            const int n = a.n_entries[b];
+            if (n < 0 || n > a.capacity) set_status(a.status, KVC_DEV_BAD_LENGTH);
+        }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t tmem = tmem_slot;
+    bool ok = true;
+    uint32_t phase = 0, mma_phase = 0;
+    ScanCursor cc;
+    const bool any = cursor_seek(a, lo, hi, cc, (int)(lo / cap));
+    if (any) {
+        ScanCursor pc = cc;
+        bool pmore = true;
+        auto issue = [&](int st) {  // thread 0: the next tile of rows into raw stage st
+            const int rows = min(ROWS, pc.end - pc.row);
+            bulk_load(smem_addr(ring + (size_t)st * TILE),
+                      a.idx_k + ((size_t)pc.b * a.idx_capacity + pc.row) * DI, (uint32_t)rows * DI,
+                      smem_addr(&full[st]));
+            pc.row += rows;
+            if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
+        };
+        if (tid == 0)
+            for (int st = 0; st < stages && pmore; ++st) issue(st);
+        int qb = -1;  // sequence whose queries are in the B tile
+        for (int tile = 0;; ++tile) {
+            const int st = tile % stages;
+            const int rows = min(ROWS, cc.end - cc.row);
+            if (cc.b != qb) {  // this sequence's queries, zero-padded, into B
+                qb = cc.b;
+                for (int p = tid; p < NQP * (DI / 16); p += NT) {
+                    const int q = p / (DI / 16), c16 = p - q * (DI / 16);
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (q < nq)
+                        v = __ldg(reinterpret_cast<const uint4*>(ba.q[q].idx_q + (size_t)qb * DI) + c16);
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(sB + swz(q, c16)),
+                                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+                }
+            }
+            const bool got = warp == 0 ? bar_wait(smem_addr(&full[st]), (phase >> st) & 1u) : true;
+            if (__syncthreads_and(got) == 0) {
+                ok = false;
+                break;
+            }
+            phase ^= 1u << st;
+            // re-lay row tid of the raw stage into the swizzled A tile
+            {
+                const unsigned char* src = ring + (size_t)st * TILE + tid * DI;
+#pragma unroll
+                for (int c = 0; c < DI / 16; ++c) {
+                    const int c16 = (c + tid) & 7;
+                    const uint4 v = *reinterpret_cast<const uint4*>(src + c16 * 16);
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(sA + swz(tid, c16)),
+                                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+            __syncthreads();  // A and B ready; raw stage st free again
+            if (tid == 0) {
+                if (pmore) issue(st);
+                asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll
+                for (int ks = 0; ks < DI / 32; ++ks)
+                    mma_i8(tmem, sdesc(sA + ks * 32), sdesc(sB + ks * 32), ks > 0 ? 1u : 0u);
+                asm volatile(
+                    "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                        smem_addr(&mma_bar))
+                    : "memory");
+            }
+            const bool done = warp == 0 ? bar_wait(smem_addr(&mma_bar), mma_phase) : true;
+            mma_phase ^= 1u;
+            if (__syncthreads_and(done) == 0) {
+                ok = false;
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+            uint32_t r[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+                "%13,%14,%15}, [%16];\n"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                  "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                  "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                : "r"(tmem + ((uint32_t)(warp * 32) << 16)));
+            asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+            if (tid < rows) {
+                const size_t row = (size_t)cc.b * cap + cc.row + tid;
+#pragma unroll
+                for (int q = 0; q < kMaxBatchQ; ++q)
+                    if (q < nq) {
+                        const int v = (int)r[q];
+                        ba.q[q].scores[row] = v;
+                        atomicAdd(&hist[q * kBins + score_bin(v, bias, shift)], 1);
+                    }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+            __syncthreads();  // the accumulator and the A tile are free again
+            cc.row += rows;
+            if (cc.row < cc.end) continue;
+            // ---- sequence cc.b done in this CTA: flush, maybe derive thresholds
+            const int b = cc.b;
+            const int n = a.n_entries[b];
+            for (int q = 0; q < nq; ++q) {
+                int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
+                for (int i = tid; i < kBins; i += NT)
+                    if (hist[q * kBins + i]) atomicAdd(&gh[i], hist[q * kBins + i]);
+            }
+            if (n > a.topk) {
+                const long long sbase = (long long)b * cap;
+                const long long first = sbase / per, last = (sbase + n - 1) / per;
+                __threadfence();
+                __syncthreads();
+                if (tid == 0)
+                    s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) ==
+                             (int)(last - first);
+                __syncthreads();
+                if (s_last) {
+                    __threadfence();
+                    for (int q = 0; q < nq; ++q) {
+                        const int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
+                        int* h = hist + q * kBins;
+                        for (int i = tid; i < kBins; i += NT) h[i] = __ldcg(gh + i);
+                        if (tid == 0) s_t = s_above = 0;
+                        __syncthreads();
+                        find_threshold(h, a.topk, &s_t, &s_above, sh_warp);
+                        if (tid == 0) {
+                            ba.q[q].thr[2 * b] = s_t;
+                            ba.q[q].thr[2 * b + 1] = s_above;
+                        }
+                        __syncthreads();
+                    }
+                }
+            }
+            __syncthreads();
+            for (int i = tid; i < nq * kBins; i += NT) hist[i] = 0;
+            if (!cursor_seek(a, lo, hi, cc, b + 1)) break;
+            __syncthreads();
+        }
+    }
+    if (!ok && tid == 0) {
+        set_status(a.status, KVC_DEV_TIMEOUT);
+        for (int st = 0; st < stages; ++st) bar_wait(smem_addr(&full[st]), (phase >> st) & 1u);
+        bar_wait(smem_addr(&mma_bar), mma_phase);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                     "r"(TMEM_COLS));
+    }
+}
+
 template <int DI>
 cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, int shift,
                         cudaStream_t s) {
@@ -861,6 +1088,54 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
     a.pool_src_cap = h.capacity;
     a.pool_src_block = h.block;
     return launch_select(a, bias, shift, s);
+}
+
+cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s) {
+    const TopkArgs& a = ba.q[0];
+    if (a.batch == 0 || ba.nq == 0) return cudaSuccess;
+    if (a.di != tcs::DI || ba.nq > kMaxBatchQ) return cudaErrorInvalidValue;
+    const int bias = score_bias(a.di), shift = score_shift(a.di);
+    cudaError_t err;
+    for (int q = 0; q < ba.nq; ++q)
+        if ((err = launch_zero(ba.q[q].counters, (int)topk_counter_words(a.batch), s)) !=
+            cudaSuccess)
+            return err;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // two CTAs per SM when at least two 16 KB stages fit in half an SM's shared
+    // memory beside the tiles and histograms (their per-tile round trips
+    // overlap), else one CTA with as many stages as fit
+    const size_t fixed = 1024 + tcs::TILE + 2048 + (size_t)ba.nq * kBins * 4;
+    int per_sm = 2;
+    size_t budget = 112 * 1024;
+    if ((budget - fixed) / tcs::TILE < 2) {
+        per_sm = 1;
+        budget = 200 * 1024;
+    }
+    int stages = (int)((budget - fixed) / tcs::TILE);
+    stages = std::max(2, std::min(stages, tcs::MAX_STAGES));
+    const size_t smem = fixed + (size_t)stages * tcs::TILE;
+    static bool attr_set[64] = {};
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        err = cudaFuncSetAttribute(index_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   200 * 1024 + 2048);
+        if (err != cudaSuccess) return err;
+        attr_set[dev] = true;
+    }
+    const long long rows = (long long)a.batch * a.capacity;
+    int ctas = per_sm * sms;
+    long long per = (rows + ctas - 1) / ctas;
+    per = (per + tcs::ROWS - 1) / tcs::ROWS * tcs::ROWS;
+    if (per < tcs::ROWS) per = tcs::ROWS;
+    ctas = (int)((rows + per - 1) / per);
+    trace_before("index_scan_tc", s);
+    err = launch_pdl(index_scan_tc_kernel, ctas, tcs::NT, smem, s, ba, per, bias, shift, stages);
+    trace_after(s);
+    if (err != cudaSuccess) return err;
+    for (int q = 0; q < ba.nq; ++q)
+        if ((err = launch_select(ba.q[q], bias, shift, s)) != cudaSuccess) return err;
+    return cudaSuccess;
 }
 
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {

@@ -186,6 +186,28 @@ kvc_status check_cache(const kvc_cache* cache, const Shape& sh) {
     return KVC_OK;
 }
 
+// Batched scoring: one block per query holding that query's scores, counters,
+// thresholds and candidates (the same regions as the single-query layout).
+struct BatchWs {
+    size_t scores, counters, thr, tile_count, cands, block;
+};
+BatchWs batch_ws_layout(int batch, int cap) {
+    BatchWs w = {};
+    size_t off = 0;
+    w.scores = off;
+    off = up(off + (size_t)batch * cap * 4);
+    w.counters = off;
+    off = up(off + topk_counter_words(batch) * 4);
+    w.thr = off;
+    off = up(off + (size_t)batch * 2 * 4);
+    w.tile_count = off;
+    off = up(off + (size_t)batch * sel_tiles(cap) * 4);
+    w.cands = off;
+    off = up(off + (size_t)batch * sel_tiles(cap) * kSelTile * 8);
+    w.block = off;
+    return w;
+}
+
 kvc_status check_ws(void* ws, size_t ws_bytes, const kvc_config& c, const Shape& sh, int batch,
                     int cap, WsLayout* w, int hier_blocks = 0, int hier_block = 0) {
     *w = ws_layout(c, sh, batch, cap, hier_blocks, hier_block);
@@ -472,6 +494,57 @@ kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int
         if (st != KVC_OK) return st;
     }
     return KVC_OK;
+}
+
+size_t kvc_workspace_bytes_batched(const kvc_config* cfg, int nq, int batch, int capacity) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh) || nq < 1 || nq > kMaxBatchQ || batch < 0 || capacity < 0)
+        return 0;
+    return (size_t)nq * batch_ws_layout(batch, capacity).block;
+}
+
+kvc_status kvc_index_topk_batched(const kvc_config* cfg, int nq, const int8_t* idx_q,
+                                  const kvc_cache* cache, int32_t* topk_idx, void* ws,
+                                  size_t ws_bytes, uint32_t* dev_status, void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    if (nq < 1 || nq > kMaxBatchQ) return KVC_ERR_INVALID;
+    if (cfg->idx_dim != 128) return KVC_ERR_UNSUPPORTED;
+    kvc_status st = check_cache(cache, sh);
+    if (st != KVC_OK) return st;
+    if (cache->batch == 0) return KVC_OK;
+    if (!idx_q || !topk_idx || !aligned(idx_q, 16) || !aligned(topk_idx, 4))
+        return KVC_ERR_INVALID;
+    if (cache->capacity > kMaxTopkCapacity) return KVC_ERR_CAPACITY;
+    const BatchWs w = batch_ws_layout(cache->batch, cache->capacity);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < (size_t)nq * w.block) return KVC_ERR_WORKSPACE;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    unsigned char* wsb = static_cast<unsigned char*>(ws);
+    BatchTopkArgs ba = {};
+    ba.nq = nq;
+    const size_t B = (size_t)cache->batch, K = (size_t)cfg->topk;
+    for (int q = 0; q < nq; ++q) {
+        TopkArgs& a = ba.q[q];
+        unsigned char* blk = wsb + (size_t)q * w.block;
+        a.idx_q = idx_q + (size_t)q * B * cfg->idx_dim;
+        a.idx_k = cache->idx_k;
+        a.n_entries = cache->n_entries;
+        a.batch = cache->batch;
+        a.capacity = cache->capacity;
+        a.idx_capacity = cache->capacity;
+        a.topk = cfg->topk;
+        a.di = cfg->idx_dim;
+        a.topk_idx = topk_idx + (size_t)q * B * K;
+        a.scores = reinterpret_cast<int32_t*>(blk + w.scores);
+        a.counters = reinterpret_cast<int32_t*>(blk + w.counters);
+        a.thr = reinterpret_cast<int32_t*>(blk + w.thr);
+        a.tile_count = reinterpret_cast<int32_t*>(blk + w.tile_count);
+        a.cands = reinterpret_cast<unsigned long long*>(blk + w.cands);
+        a.status = dev_status;
+    }
+    return launch_index_topk_batched(ba, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KVC_OK
+               : KVC_ERR_CUDA;
 }
 
 kvc_status kvc_e2m1_encode(const float* x, int64_t n, uint8_t* codes, void* stream) {

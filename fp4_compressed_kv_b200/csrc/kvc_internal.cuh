@@ -104,6 +104,17 @@ struct TopkArgs {
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
 
+// Several indexer queries per sequence scored in one pass over the shared
+// indexer cache on the tensor cores (kind::i8), then one selection per query.
+// All queries share idx_k / n_entries / batch / capacity / topk / di (= 128);
+// each has its own idx_q, output and scratch.
+constexpr int kMaxBatchQ = 8;
+struct BatchTopkArgs {
+    TopkArgs q[kMaxBatchQ];
+    int nq;
+};
+cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s);
+
 // Hierarchical indexer, block stage: from a Full layer's entry scores
 // ([B][capacity]), the blocks of `block` consecutive entries are scored by
 // their best entry and the best `keep` blocks of every sequence are written

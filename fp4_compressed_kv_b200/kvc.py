@@ -64,6 +64,8 @@ def _lib():
             "kvc_sparse_decode_attn": (S, [P, P, P, P, P, I, P, P, P, Z, P, P]),
             "kvc_layer_group_step": (S, [P, I, P, P, P, P, I, P, P, P, P, P, Z, P, P]),
             "kvc_workspace_bytes_hier": (Z, [P, I, I, I, I]),
+            "kvc_workspace_bytes_batched": (Z, [P, I, I, I]),
+            "kvc_index_topk_batched": (S, [P, I, P, P, P, P, Z, P, P]),
             "kvc_layer_group_step_hier": (S, [P, I, I, I, P, P, P, P, I, P, P, P, P, P, Z, P,
                                               P]),
             "kvc_e2m1_encode": (S, [P, C.c_int64, P, P]),
@@ -168,6 +170,25 @@ def _ws(ws):
     base = ws.data_ptr()
     off = (-base) % 256
     return C.c_void_p(base + off), ws.numel() - off
+
+
+def workspace_batched(cfg: Config, nq: int, batch: int, capacity: int,
+                      device="cuda") -> torch.Tensor:
+    """Workspace for index_topk_batched with nq queries per sequence."""
+    n = int(_lib().kvc_workspace_bytes_batched(C.byref(cfg), nq, batch, capacity))
+    if n == 0:
+        raise KvcError("invalid batched workspace request")
+    return torch.empty(n + 256, dtype=torch.uint8, device=device)
+
+
+def index_topk_batched(cfg, idx_q, cache: Cache, topk_out, ws, status=None, stream=None):
+    """idx_q [nq][B][Di] int8 -> topk_out [nq][B][K]: every query against the
+    cache in one tensor-core pass."""
+    p, n = _ws(ws)
+    cs = cache.struct()
+    _check("kvc_index_topk_batched", _lib().kvc_index_topk_batched(
+        C.byref(cfg), idx_q.shape[0], _ptr(idx_q), C.byref(cs), _ptr(topk_out), p, n,
+        _ptr(status), _stream(stream)))
 
 
 def pack(cfg, tokens, gate, idx_k_new, cache: Cache, status=None, stream=None):

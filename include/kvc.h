@@ -167,6 +167,26 @@ kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t* idx_q,
                                   int32_t* scores, uint32_t* dev_status,
                                   void* stream);
 
+/* Several indexer queries per sequence scored in one pass over the cache
+ * (the lightweight indexer of [A] breakthrough 4 for all the Full and
+ * Reindex layers of a CSA2 stack at once, part 4 "CSA2：三种模式").  Valid
+ * only where every query is known before the pass (a verification or prefill
+ * schedule, or a stack whose indexer queries do not depend on earlier
+ * layers); it computes exactly what nq calls of kvc_index_topk compute.  The
+ * scores are one tensor-core product per 128-row tile (int8 x int8 -> int32,
+ * tcgen05 kind::i8 with the queries as the N = 16 side), read once from HBM.
+ * idx_q     [nq][batch][idx_dim] int8, 1 <= nq <= 8; idx_dim must be 128
+ *           (else KVC_ERR_UNSUPPORTED).
+ * topk_idx  [nq][batch][topk] int32, as kvc_index_topk's output per query.
+ * ws        kvc_workspace_bytes_batched(cfg, nq, batch, capacity) bytes,
+ *           256-byte aligned; scratch.                                     */
+size_t kvc_workspace_bytes_batched(const kvc_config* cfg, int nq, int batch,
+                                   int capacity);
+kvc_status kvc_index_topk_batched(const kvc_config* cfg, int nq,
+                                  const int8_t* idx_q, const kvc_cache* cache,
+                                  int32_t* topk_idx, void* ws, size_t ws_bytes,
+                                  uint32_t* dev_status, void* stream);
+
 /* Sparse decode attention (A6-A10; [A] breakthrough 2 and 4, "P4 main KV").
  * q         [batch][n_heads][D] act_dtype queries (already in latent space).
  * topk_idx  [batch][topk] int32 selected entries; -1 entries are skipped, any
@@ -242,9 +262,9 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * max_launches launches are recorded).  kvc_trace_kernel, called after the
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
- * "pack", "pack_commit", "topk_zero", "index_scan", "topk_select",
- * "block_max", "copy_topk", "attn_tc05", "attn_simt", "attn_merge",
- * "fp4_codec".                                                             */
+ * "pack", "pack_commit", "topk_zero", "index_scan", "index_scan_tc",
+ * "topk_select", "block_max", "copy_topk", "attn_tc05", "attn_simt",
+ * "attn_merge", "fp4_codec".                                                             */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);
 kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);

@@ -115,3 +115,19 @@ def test_hier_workspace_and_validation(lib):
             C.byref(cfg), blocks, block, 2, modes, C.c_void_p(16), C.c_void_p(16),
             C.c_void_p(16), 32, C.byref(cache), C.c_void_p(16), None, C.c_void_p(16),
             C.c_void_p(256), 1 << 30, None, None) == 1
+
+
+def test_batched_workspace_and_validation(lib):
+    so = lib.lib()
+    w = synth.WORKLOADS["stack1m"]
+    cfg = lib.config_for(w)
+    one = so.kvc_workspace_bytes_batched(C.byref(cfg), 1, 1, w.entries)
+    assert one > 0 and so.kvc_workspace_bytes_batched(C.byref(cfg), 5, 1, w.entries) == 5 * one
+    assert so.kvc_workspace_bytes_batched(C.byref(cfg), 0, 1, w.entries) == 0
+    assert so.kvc_workspace_bytes_batched(C.byref(cfg), 9, 1, w.entries) == 0
+    cache = lib.CacheStruct(16, 16, 16, 1, 8)
+    tiny = lib.config_for(synth.WORKLOADS["tiny"])  # idx_dim 32: not supported
+    assert so.kvc_index_topk_batched(C.byref(tiny), 2, C.c_void_p(16), C.byref(cache),
+                                     C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 4
+    assert so.kvc_index_topk_batched(C.byref(cfg), 9, C.c_void_p(16), C.byref(cache),
+                                     C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 1
