@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse FP4-KV decode query-tokens/s; achieved HBM GB/s vs 8 TB/s"
 UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNELS = ("pack", "pack_commit", "topk_zero", "index_scan", "topk_select", "block_max",
+KERNELS = ("pack", "pack_commit", "index_scan", "index_scan_tc", "topk_select", "block_max",
            "copy_topk", "attn_tc05", "attn_simt", "attn_merge")
 
 

@@ -312,9 +312,9 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
         const int b = cc.b;
         const int n = a.n_entries[b];
         int32_t* gh = a.counters + (size_t)b * kBins;
-        for (int i = tid; i < kBins; i += kThreads)
-            if (hist[i]) atomicAdd(&gh[i], hist[i]);
         if (n > a.topk) {
+            for (int i = tid; i < kBins; i += kThreads)
+                if (hist[i]) atomicAdd(&gh[i], hist[i]);
             const long long base = (long long)b * cap;
             const long long first = base / per, last = (base + n - 1) / per;
             __threadfence();
@@ -325,10 +325,16 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
             __syncthreads();
             if (s_last) {
                 __threadfence();
-                for (int i = tid * 4; i < kBins; i += kThreads * 4)
+                for (int i = tid * 4; i < kBins; i += kThreads * 4) {
                     *reinterpret_cast<int4*>(hist + i) =
                         __ldcg(reinterpret_cast<const int4*>(gh + i));
-                if (tid == 0) s_t = s_above = 0;
+                    // the counters are left zeroed for the next call
+                    *reinterpret_cast<int4*>(gh + i) = make_int4(0, 0, 0, 0);
+                }
+                if (tid == 0) {
+                    a.counters[(size_t)a.batch * kBins + b] = 0;
+                    s_t = s_above = 0;
+                }
                 __syncthreads();
                 find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
                 if (tid == 0) {
@@ -694,15 +700,10 @@ topk_select_kernel(TopkArgs a, int bias, int shift) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    if (tid == 0) a.counters[(size_t)a.batch * (kBins + 1) + b] = 0;  // zeroed for the next call
     finish_sequence(a, b, bias, shift, fsmem);
 }
 
-// Clears the per-call counters (a kernel, so the launch chain stays kernel to
-// kernel).
-__global__ void zero_counters_kernel(int32_t* p, int n) {
-    pdl_wait();
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
-}
 
 // ---- hierarchical indexer, block stage
 constexpr int kBlkPerThread = 4;
@@ -766,10 +767,10 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
         }
     }
     __syncthreads();
+    if (nb <= h.keep) return;  // every block is kept: no threshold needed
     int32_t* gh = h.counters + (size_t)b * kBins;
     for (int i = tid; i < kBins; i += kThreads)
         if (hist[i]) atomicAdd(&gh[i], hist[i]);
-    if (nb <= h.keep) return;  // every block is kept: no threshold needed
     __threadfence();
     __syncthreads();
     if (tid == 0)
@@ -777,8 +778,14 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int i = tid; i < kBins; i += kThreads) hist[i] = __ldcg(gh + i);
-    if (tid == 0) s_t = s_above = 0;
+    for (int i = tid; i < kBins; i += kThreads) {
+        hist[i] = __ldcg(gh + i);
+        gh[i] = 0;  // left zeroed for the next call
+    }
+    if (tid == 0) {
+        h.counters[(size_t)h.batch * kBins + b] = 0;
+        s_t = s_above = 0;
+    }
     __syncthreads();
     find_threshold(hist, h.keep, &s_t, &s_above, sh_warp);
     if (tid == 0) {
@@ -962,12 +969,12 @@ index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int s
             // ---- sequence cc.b done in this CTA: flush, maybe derive thresholds
             const int b = cc.b;
             const int n = a.n_entries[b];
-            for (int q = 0; q < nq; ++q) {
-                int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
-                for (int i = tid; i < kBins; i += NT)
-                    if (hist[q * kBins + i]) atomicAdd(&gh[i], hist[q * kBins + i]);
-            }
             if (n > a.topk) {
+                for (int q = 0; q < nq; ++q) {
+                    int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
+                    for (int i = tid; i < kBins; i += NT)
+                        if (hist[q * kBins + i]) atomicAdd(&gh[i], hist[q * kBins + i]);
+                }
                 const long long sbase = (long long)b * cap;
                 const long long first = sbase / per, last = (sbase + n - 1) / per;
                 __threadfence();
@@ -978,10 +985,14 @@ index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int s
                 __syncthreads();
                 if (s_last) {
                     __threadfence();
+                    if (tid == 0) a.counters[(size_t)a.batch * kBins + b] = 0;
                     for (int q = 0; q < nq; ++q) {
-                        const int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
+                        int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
                         int* h = hist + q * kBins;
-                        for (int i = tid; i < kBins; i += NT) h[i] = __ldcg(gh + i);
+                        for (int i = tid; i < kBins; i += NT) {
+                            h[i] = __ldcg(gh + i);
+                            gh[i] = 0;  // left zeroed for the next call
+                        }
                         if (tid == 0) s_t = s_above = 0;
                         __syncthreads();
                         find_threshold(h, a.topk, &s_t, &s_above, sh_warp);
@@ -1048,13 +1059,6 @@ cudaError_t launch_select(const TopkArgs& a, int bias, int shift, cudaStream_t s
     return err;
 }
 
-cudaError_t launch_zero(int32_t* p, int words, cudaStream_t s) {
-    trace_before("topk_zero", s);
-    const cudaError_t err = launch_pdl(zero_counters_kernel, (words + 1023) / 1024, 256, 0, s, p,
-                                       words);
-    trace_after(s);
-    return err;
-}
 
 }  // namespace
 
@@ -1062,8 +1066,7 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
     if (h.batch == 0) return cudaSuccess;
     const int bias = score_bias(h.di), shift = score_shift(h.di);
     const int cap_blk = (h.capacity + h.block - 1) / h.block;
-    cudaError_t err = launch_zero(h.counters, (int)topk_counter_words(h.batch), s);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
     trace_before("block_max", s);
     err = launch_pdl(block_max_kernel, dim3((cap_blk + kBlkPerCta - 1) / kBlkPerCta, h.batch),
                      kThreads, 0, s, h, cap_blk, bias, shift);
@@ -1096,10 +1099,6 @@ cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s) {
     if (a.di != tcs::DI || ba.nq > kMaxBatchQ) return cudaErrorInvalidValue;
     const int bias = score_bias(a.di), shift = score_shift(a.di);
     cudaError_t err;
-    for (int q = 0; q < ba.nq; ++q)
-        if ((err = launch_zero(ba.q[q].counters, (int)topk_counter_words(a.batch), s)) !=
-            cudaSuccess)
-            return err;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1141,9 +1140,7 @@ cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s) {
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     if (a.batch == 0) return cudaSuccess;
     const int bias = score_bias(a.di), shift = score_shift(a.di);
-    // zero the histograms and the finished-CTA counters (adjacent in the workspace)
-    cudaError_t err = launch_zero(a.counters, (int)topk_counter_words(a.batch), s);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
     // one wave: 3 CTAs per SM (64 KB ring + 8 KB histogram each for Di = 128;
     // measured faster than 2 CTAs with 3 stages or 1 CTA with 6), equal row
     // slices

@@ -162,7 +162,7 @@ def workspace(cfg: Config, batch: int, capacity: int, device="cuda", hier_blocks
         n = workspace_bytes(cfg, batch, capacity)
     if n == 0:
         raise KvcError("invalid workspace request")
-    return torch.empty(n + 256, dtype=torch.uint8, device=device)
+    return torch.zeros(n + 256, dtype=torch.uint8, device=device)  # zero-filled before first use
 
 
 def _ws(ws):
@@ -178,7 +178,7 @@ def workspace_batched(cfg: Config, nq: int, batch: int, capacity: int,
     n = int(_lib().kvc_workspace_bytes_batched(C.byref(cfg), nq, batch, capacity))
     if n == 0:
         raise KvcError("invalid batched workspace request")
-    return torch.empty(n + 256, dtype=torch.uint8, device=device)
+    return torch.zeros(n + 256, dtype=torch.uint8, device=device)  # zero-filled before first use
 
 
 def index_topk_batched(cfg, idx_q, cache: Cache, topk_out, ws, status=None, stream=None):

@@ -108,7 +108,13 @@ size_t kvc_bytes_resident(const kvc_config* cfg, int64_t entries, int n_layers,
                           int padded);
 
 /* Device workspace needed by kvc_index_topk, kvc_sparse_decode_attn and
- * kvc_layer_group_step for `batch` sequences of up to `capacity` entries. */
+ * kvc_layer_group_step for `batch` sequences of up to `capacity` entries.
+ * Every workspace (this one, the hierarchical and the batched ones) must be
+ * zero-filled before its first use (for example with cudaMemset): the top-K
+ * counters in it start at zero, and every call leaves them at zero again, so
+ * no call spends a launch clearing them.  After a call that set
+ * KVC_DEV_TIMEOUT in the status word, zero the workspace again.  Nothing
+ * else in it needs initialisation.                                         */
 size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity);
 
 /* Append n_new raw tokens per sequence (A1-A3 of the hot path).
@@ -137,8 +143,8 @@ kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,
  * scores    [batch][capacity] int32 out, or NULL; when given it receives every
  *           visible score (positions past n_entries are not written).
  * ws        device workspace of at least kvc_workspace_bytes(cfg, batch,
- *           capacity) bytes, 256-byte aligned; its contents need no
- *           initialisation and are scratch after the call.
+ *           capacity) bytes, 256-byte aligned, zero-filled before its first
+ *           use (see kvc_workspace_bytes).
  * capacity must not exceed 8,388,608 entries (KVC_ERR_CAPACITY).         */
 kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
                           const kvc_cache* cache, int32_t* topk_idx,
@@ -158,10 +164,11 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
  * KVC_ERR_CAPACITY before anything is enqueued.  The call allocates nothing.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  Every call shares the one array and it keeps the last call's
- * contents: the parts that must start at zero are cleared on `stream` by each
- * call, but calls whose work overlaps on the GPU (different streams, or
- * different host threads on one device) race on it.                      */
+ * capture.  Every call shares the one array: its counters start at zero
+ * (a static array) and every call leaves them at zero, but calls whose work
+ * overlaps on the GPU (different streams, or different host threads on one
+ * device) race on it, and after a call that set KVC_DEV_TIMEOUT the array
+ * stays unusable until the process exits.                                */
 kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t* idx_q,
                                   const kvc_cache* cache, int32_t* topk_idx,
                                   int32_t* scores, uint32_t* dev_status,
@@ -179,7 +186,7 @@ kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t* idx_q,
  *           (else KVC_ERR_UNSUPPORTED).
  * topk_idx  [nq][batch][topk] int32, as kvc_index_topk's output per query.
  * ws        kvc_workspace_bytes_batched(cfg, nq, batch, capacity) bytes,
- *           256-byte aligned; scratch.                                     */
+ *           256-byte aligned, zero-filled before its first use.           */
 size_t kvc_workspace_bytes_batched(const kvc_config* cfg, int nq, int batch,
                                    int capacity);
 kvc_status kvc_index_topk_batched(const kvc_config* cfg, int nq,
@@ -262,7 +269,7 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * max_launches launches are recorded).  kvc_trace_kernel, called after the
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
- * "pack", "pack_commit", "topk_zero", "index_scan", "index_scan_tc",
+ * "pack", "pack_commit", "index_scan", "index_scan_tc",
  * "topk_select", "block_max", "copy_topk", "attn_tc05", "attn_simt",
  * "attn_merge", "fp4_codec".                                                             */
 kvc_status kvc_trace_begin(int max_launches);

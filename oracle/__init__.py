@@ -90,6 +90,8 @@ def lib():
             "orc_group_step_hier": (C.c_int, [P, C.c_int, P, C.c_int, P, P, P, C.c_int, P, P,
                                               C.c_int, P, C.c_int, C.c_int, P, P, P, P]),
             "orc_block_pool": (C.c_int, [P, C.c_int, C.c_int, C.c_int, P, P]),
+            "orc_window_fp8": (C.c_int, [P, C.c_int, P, P]),
+            "orc_window_fp8_dequant": (None, [P, C.c_float, C.c_int, P]),
             "orc_pool_topk": (C.c_int, [P, P, C.c_int, P, C.c_int, C.c_int, P]),
         }
         for name, (res, args) in sig.items():
@@ -248,6 +250,34 @@ def sparse_decode(cfg: Cfg, q, records, n_entries, topk_idx, window, window_len)
     if rc:
         raise ValueError(f"orc_sparse_decode failed: {rc}")
     return out, lse, int(st[0])
+
+
+def window_fp8(rows):
+    """FP8 window rows [..][D] fp32 -> (codes uint8 [..][D], scales fp32 [..], bad rows)."""
+    rows = _c(rows, np.float32)
+    D = rows.shape[-1]
+    flat = rows.reshape(-1, D)
+    codes = np.zeros(flat.shape, np.uint8)
+    scales = np.zeros(flat.shape[0], np.float32)
+    bad = 0
+    for i in range(flat.shape[0]):
+        sc = C.c_float(0.0)
+        bad |= lib().orc_window_fp8(_p(flat[i]), D, _p(codes[i]), C.byref(sc))
+        scales[i] = sc.value
+    return codes.reshape(rows.shape), scales.reshape(rows.shape[:-1]), bad
+
+
+def window_fp8_dequant(codes, scales):
+    """Decoded FP8 window rows, fp32."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.float32)
+    D = codes.shape[-1]
+    flat = codes.reshape(-1, D)
+    sf = scales.reshape(-1)
+    out = np.empty(flat.shape, np.float32)
+    for i in range(flat.shape[0]):
+        lib().orc_window_fp8_dequant(_p(flat[i]), float(sf[i]), D, _p(out[i]))
+    return out.reshape(codes.shape)
 
 
 def block_pool(scores, block, keep):

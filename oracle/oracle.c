@@ -169,6 +169,44 @@ int orc_e4m3_encode(float v) {
 }
 
 /* ------------------------------------------------------------------ */
+/* FP8 window rows ([P2] part 4 "P4 main KV": the SWA KV stays FP8; the
+ * pages give no scale layout).  Reading: one fp32 scale per row,
+ * s = absmax / 448 over the row's finite values (IEEE RN), each element
+ * coded as signed E4M3 of x / s rounded to nearest even and saturating at
+ * 448; a magnitude of zero is stored as +0; non-finite elements are coded 0
+ * and reported.  Returns 1 if the row held a non-finite value.            */
+int orc_window_fp8(const float* row, int D, uint8_t* codes, float* scale) {
+    float amax = 0.0f;
+    int bad = 0;
+    for (int d = 0; d < D; ++d) {
+        if (!isfinite(row[d])) {
+            bad = 1;
+            continue;
+        }
+        float a = fabsf(row[d]);
+        if (a > amax) amax = a;
+    }
+    float s = amax / 448.0f;
+    *scale = s;
+    for (int d = 0; d < D; ++d) {
+        float x = row[d];
+        int c = 0;
+        if (isfinite(x) && s > 0.0f) {
+            float v = x / s;
+            int mag = orc_e4m3_encode(fabsf(v));
+            c = mag == 0 ? 0 : ((v < 0.0f ? 0x80 : 0) | mag);
+        }
+        codes[d] = (uint8_t)c;
+    }
+    return bad;
+}
+
+/* Decoded FP8 window row: E4M3(code) x scale, in fp32.                 */
+void orc_window_fp8_dequant(const uint8_t* codes, float scale, int D, float* out) {
+    for (int d = 0; d < D; ++d) out[d] = orc_e4m3_value(codes[d]) * scale;
+}
+
+/* ------------------------------------------------------------------ */
 /* R3 grouping and the record layout.                                 */
 int orc_n_groups(int latent, int rope, int group) {
     return (latent + group - 1) / group + (rope + group - 1) / group;

@@ -125,3 +125,26 @@ def test_topk_scan_slices_span_sequences(kvc):
     for b in range(400):
         assert np.array_equal(sc[b, : n[b]], osc[b, : n[b]]), b
     topk_set_equal(tk, otk)
+
+
+def test_workspace_reused_across_calls(kvc):
+    """The workspace is zero-filled once; every call leaves its counters at zero,
+    so calls of different lengths and queries on one workspace stay exact."""
+    w = synth.WORKLOADS["csa2group"].scaled(batch=4, context=2 * 20000)
+    cfg = kvc.config_for(w)
+    g = torch.Generator().manual_seed(21)
+    idx_k = torch.randint(-127, 128, (4, 20000, 128), generator=g, dtype=torch.int8)
+    cache = kvc.Cache(cfg, 4, 20000)
+    cache.idx_k.copy_(idx_k.cuda())
+    ws = kvc.workspace(cfg, 4, 20000)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for rnd, n in enumerate([[20000, 9000, 300, 513], [511, 20000, 20000, 8192],
+                             [20000, 20000, 20000, 20000], [1, 0, 600, 19999]]):
+        q = torch.randint(-127, 128, (4, 128), generator=g, dtype=torch.int8)
+        cache.n_entries.copy_(torch.as_tensor(n, dtype=torch.int32))
+        tk = torch.empty(4, w.topk, dtype=torch.int32, device="cuda")
+        kvc.index_topk(cfg, q.cuda(), cache, tk, ws, status=st)
+        torch.cuda.synchronize()
+        want = _oracle(w, idx_k, q, n, 20000)[0]
+        assert st.item() == 0, rnd
+        topk_set_equal(tk.cpu().numpy(), want)
