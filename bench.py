@@ -255,6 +255,50 @@ def time_scoring(w, steps, warmup, batched, dev):
     return e0.elapsed_time(e1) / steps
 
 
+def time_attention_window(w, steps, warmup, fp8, dev):
+    """Device ms of one attention call of workload w's shape (every sequence,
+    one layer) with the window in bf16 or in FP8."""
+    import torch
+    from fp4_compressed_kv_b200 import kvc, synth
+    wx = w.scaled(context=2 * 4096)
+    cfg = kvc.config_for(wx)
+    g = synth.generator(dev, 17)
+    B, N = wx.batch, wx.entries
+    cache = kvc.Cache(cfg, B, N, device=dev)
+    gate = (torch.randn(wx.dim, generator=g, device=dev) / wx.dim ** 0.5).float()
+    nt = synth.make_new_tokens(wx, 2 * N, dev)
+    kvc.pack(cfg, nt["tokens"], gate, nt["idx_k"], cache)
+    tk = torch.sort(torch.stack([torch.randperm(N, generator=g, device=dev)[: wx.topk]
+                                 for _ in range(B)]), 1).values.int().contiguous()
+    q = torch.randn(B, wx.heads, wx.dim, generator=g, device=dev).to(wx.torch_dtype)
+    win = torch.randn(B, wx.window, wx.dim, generator=g, device=dev).to(wx.torch_dtype)
+    codes = torch.empty(win.shape, dtype=torch.uint8, device=dev)
+    scales = torch.empty(win.shape[:-1], dtype=torch.float32, device=dev)
+    kvc.pack_window_fp8(cfg, win, codes, scales)
+    out = torch.empty(B, wx.heads, wx.latent, device=dev)
+    ws = kvc.workspace(cfg, B, N, device=dev)
+
+    def step():
+        if fp8:
+            kvc.sparse_decode_attn_fp8win(cfg, q, cache, tk, codes, scales, wx.window, out, ws)
+        else:
+            kvc.sparse_decode_attn(cfg, q, cache, tk, win, wx.window, out, ws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(steps):
+            step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del gr
+    return e0.elapsed_time(e1) / steps
+
+
 # ----------------------------------------------------------------------------- oracle leg
 def oracle_decode_sample(w, seconds, seed_shift=0):
     """Time the CPU oracle on single-sequence decode steps of workload w.
@@ -556,6 +600,12 @@ def run_ours(args):
             extra[name].update({"scoring_ms_per_layer_scans": round(one, 4),
                                 "scoring_ms_batched_tensor_core": round(bat, 4)})
             torch.cuda.empty_cache()
+        # the attention of this workload with the window in bf16 and in FP8
+        extra["fp8_window"] = {
+            "workload": w0.name,
+            "attention_ms_bf16_window": round(time_attention_window(w0, 20, 3, False, dev), 4),
+            "attention_ms_fp8_window": round(time_attention_window(w0, 20, 3, True, dev), 4)}
+        torch.cuda.empty_cache()
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None

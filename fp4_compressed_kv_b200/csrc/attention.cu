@@ -120,8 +120,9 @@ attn_simt_kernel(AttnArgs a, Shape sh, int H, int K, float scale_log2, int chunk
                           : reinterpret_cast<const float*>(rec + sh.code_bytes)[g];
                 v = e2m1_value(code) * sc;
             } else if (k <= -2) {
-                const int t = -2 - k;
-                v = to_f32(static_cast<const T*>(a.window)[((size_t)b * a.window_stride + t) * D + d]);
+                const size_t row = (size_t)b * a.window_stride + (-2 - k);
+                v = a.win_fp8 ? e4m3s_to_f32(a.win_fp8[row * D + d]) * a.win_scale[row]
+                              : to_f32(static_cast<const T*>(a.window)[row * D + d]);
             }
             keys[p] = v;
         }

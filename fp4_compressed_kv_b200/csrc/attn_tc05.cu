@@ -318,6 +318,7 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                 const int k = kind[s];
                 const uint32_t dst = sK + (cc >> 3) * K_ATOM + swz(s, cc & 7);
                 if (k <= -2) {
+                    if (a.win_fp8) continue;  // FP8 rows are decoded after the dequantisation
                     const int t = -2 - k;
                     cp_async16(dst, static_cast<const unsigned char*>(a.window) +
                                         ((size_t)b * a.window_stride + t) * D * 2 + cc * 16);
@@ -363,7 +364,42 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
             }
         }
         cp_async_wait_all();  // the window rows too
-        if (other_rows) {
+        if (other_rows && a.win_fp8) {
+            // FP8 window rows: 16 codes per load, E4M3 -> f16x2 in hardware,
+            // times the row's scale in fp32, two 16-byte pieces of the K tile
+            for (int p = tid; p < CK * (D / 16); p += NT) {
+                const int s = p / (D / 16), c16 = p - s * (D / 16);
+                const int k = kind[s];
+                if (k > -2) continue;
+                const size_t row = (size_t)b * a.window_stride + (-2 - k);
+                const uint4 cw = __ldg(reinterpret_cast<const uint4*>(a.win_fp8 + row * D) + c16);
+                const float sc = __ldg(a.win_scale + row);
+                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint32_t o[8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t h0, h1;
+                    asm("{\n\t.reg .b16 lo, hi;\n\t"
+                        "mov.b32 {lo, hi}, %2;\n\t"
+                        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+                        "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+                        : "=r"(h0), "=r"(h1)
+                        : "r"(words[u]));
+                    const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+                    const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+                    o[2 * u] = pack_f16(f0.x * sc, f0.y * sc);
+                    o[2 * u + 1] = pack_f16(f1.x * sc, f1.y * sc);
+                }
+#pragma unroll
+                for (int hpc = 0; hpc < 2; ++hpc) {
+                    const int cc = 2 * c16 + hpc;
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(
+                                     sK + (cc >> 3) * K_ATOM + swz(s, cc & 7)),
+                                 "r"(o[4 * hpc]), "r"(o[4 * hpc + 1]), "r"(o[4 * hpc + 2]),
+                                 "r"(o[4 * hpc + 3]));
+                }
+            }
+        } else if (other_rows) {
             __syncthreads();  // every thread's window copies have landed
             // window rows arrived as bf16: convert them in place to f16
             for (int p = tid; p < CK * (D / 8); p += NT) {

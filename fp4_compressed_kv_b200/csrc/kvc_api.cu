@@ -291,9 +291,12 @@ kvc_status run_pool_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cac
 kvc_status run_attn(const kvc_config& c, const Shape& sh, const void* q, const kvc_cache* cache,
                     const int32_t* topk, const void* window, int window_len, float* out,
                     float* lse, unsigned char* ws, const WsLayout& w, uint32_t* st,
-                    cudaStream_t s, int32_t* topk_copy = nullptr) {
+                    cudaStream_t s, int32_t* topk_copy = nullptr,
+                    const uint8_t* win_fp8 = nullptr, const float* win_scale = nullptr) {
     AttnArgs a = {};
     a.topk_copy = topk_copy;
+    a.win_fp8 = win_fp8;
+    a.win_scale = win_scale;
     a.q = q;
     a.records = static_cast<const uint8_t*>(cache->records);
     a.n_entries = cache->n_entries;
@@ -414,6 +417,48 @@ kvc_status kvc_sparse_decode_attn(const kvc_config* cfg, const void* q, const kv
     if (!device_ok()) return KVC_ERR_DEVICE;
     return run_attn(*cfg, sh, q, cache, topk_idx, window, window_len, out, lse,
                     static_cast<unsigned char*>(ws), w, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+kvc_status kvc_sparse_decode_attn_fp8win(const kvc_config* cfg, const void* q,
+                                         const kvc_cache* cache, const int32_t* topk_idx,
+                                         const uint8_t* win_codes, const float* win_scales,
+                                         int window_len, float* out, float* lse, void* ws,
+                                         size_t ws_bytes, uint32_t* dev_status, void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    kvc_status st = check_cache(cache, sh);
+    if (st != KVC_OK) return st;
+    if (cache->batch == 0) return KVC_OK;
+    if (window_len < 0 || window_len > cfg->window) return KVC_ERR_INVALID;
+    if (!q || !topk_idx || !out || (window_len > 0 && (!win_codes || !win_scales)))
+        return KVC_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(topk_idx, 4) ||
+        (win_codes && !aligned(win_codes, 16)) || (win_scales && !aligned(win_scales, 4)) ||
+        (lse && !aligned(lse, 4)) || sh.D % 16)
+        return KVC_ERR_INVALID;
+    WsLayout w;
+    if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    // a non-null code pointer selects the FP8 window in the kernels
+    const uint8_t* codes = window_len > 0 ? win_codes : nullptr;
+    return run_attn(*cfg, sh, q, cache, topk_idx, nullptr, window_len, out, lse,
+                    static_cast<unsigned char*>(ws), w, dev_status,
+                    static_cast<cudaStream_t>(stream), nullptr, codes, win_scales);
+}
+
+kvc_status kvc_pack_window_fp8(const kvc_config* cfg, const void* rows, int64_t n_rows,
+                               uint8_t* codes, float* scales, uint32_t* dev_status,
+                               void* stream) {
+    Shape sh;
+    if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    if (n_rows < 0 || (n_rows > 0 && (!rows || !codes || !scales))) return KVC_ERR_INVALID;
+    if (n_rows == 0) return KVC_OK;
+    if (!aligned(rows, 16) || !aligned(codes, 8) || !aligned(scales, 4)) return KVC_ERR_INVALID;
+    if (!device_ok()) return KVC_ERR_DEVICE;
+    return launch_window_fp8(*cfg, sh, rows, n_rows, codes, scales, dev_status,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KVC_OK
+               : KVC_ERR_CUDA;
 }
 
 kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers, const int32_t* modes,

@@ -150,9 +150,18 @@ struct AttnArgs {
     float* part_ml;         // [B][H][kMaxSplit][2]
     uint32_t* status;
     int32_t* topk_copy;     // [B][K]: receives a copy of topk_idx (a Reuse layer's), or null
+    // FP8 window: when set, the window rows are signed E4M3 codes
+    // [B][W][D] with one fp32 scale per row [B][W] (window is then unused)
+    const uint8_t* win_fp8;
+    const float* win_scale;
 };
 cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                              cudaStream_t s);
+
+// FP8 window rows: rows [n][D] act_dtype -> codes [n][D] signed E4M3, one
+// fp32 scale per row (absmax / 448).
+cudaError_t launch_window_fp8(const kvc_config& c, const Shape& sh, const void* rows, long long n,
+                              uint8_t* codes, float* scales, uint32_t* status, cudaStream_t s);
 
 cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3,
                              cudaStream_t s);
@@ -207,6 +216,22 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
     const uint32_t e = (b >> 3) & 15u, m = b & 7u;
     if (e == 0) return (float)m * 0x1.0p-9f;
     return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Signed E4M3 decode (exact).
+__device__ __forceinline__ float e4m3s_to_f32(uint32_t b) {
+    const float v = e4m3_to_f32(b & 0x7Fu);
+    return (b & 0x80u) ? -v : v;
+}
+// Four fp32 values -> four signed E4M3 bytes (value t in byte t), round to
+// nearest even, saturating; codes of magnitude 0 lose their sign.
+__device__ __forceinline__ uint32_t e4m3x4_from_f32(float a0, float a1, float a2, float a3) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(a1), "f"(a0));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(a3), "f"(a2));
+    const uint32_t w = (uint32_t)lo | ((uint32_t)hi << 16);
+    const uint32_t nonzero = ((w & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) & 0x80808080u;
+    return w & (0x7F7F7F7Fu | nonzero);
 }
 
 // Eight fp32 values already in [-6, 6] -> eight E2M1 codes in one word,

@@ -610,6 +610,99 @@ cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
     return err;
 }
 
+// ---- FP8 window rows: a warp per row.  s = absmax / 448 over the finite
+// elements; codes = E4M3 of x / s, by the same bracket of two reciprocal
+// products as the E2M1 codes (rounding to E4M3 is monotone too), with an
+// exact division where the brackets disagree.
+constexpr int kWinWarps = 4;
+template <typename T, int MAXC>
+__global__ void __launch_bounds__(kWinWarps * 32)
+window_fp8_kernel(const T* __restrict__ rows, long long n, int D, uint8_t* __restrict__ codes,
+                  float* __restrict__ scales, uint32_t* status) {
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const long long r = (long long)blockIdx.x * kWinWarps + (threadIdx.x >> 5);
+    if (r >= n) return;
+    const int nchunk = D >> 3;
+    const T* src = rows + r * D;
+    float x[MAXC][8];
+    float amax = 0.f;
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const int c = lane + 32 * j;
+        Chunk<T> v;
+        if (c < nchunk) v.load_cached(src + 8 * c); else v.zero();
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float e = v.get(t);
+            if (!isfinite(e)) {
+                if (c < nchunk) bad = true;
+                e = 0.f;
+            }
+            x[j][t] = e;
+            amax = fmaxf(amax, fabsf(e));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = __fdiv_rn(amax, 448.0f);
+    const float rc = __frcp_rn(sc);
+    const bool fast = sc > 0.f && rc < 3.0e38f;
+    const float rl = __fmul_rn(rc, 1.0f - 0x1p-20f), rh = __fmul_rn(rc, 1.0f + 0x1p-20f);
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const int c = lane + 32 * j;
+        if (c >= nchunk) continue;
+        uint32_t w[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float* e = x[j] + 4 * h;
+            uint32_t code = 0;
+            if (sc > 0.f) {
+                bool done = false;
+                if (fast) {
+                    const uint32_t cl = e4m3x4_from_f32(__fmul_rn(e[0], rl), __fmul_rn(e[1], rl),
+                                                        __fmul_rn(e[2], rl), __fmul_rn(e[3], rl));
+                    const uint32_t ch = e4m3x4_from_f32(__fmul_rn(e[0], rh), __fmul_rn(e[1], rh),
+                                                        __fmul_rn(e[2], rh), __fmul_rn(e[3], rh));
+                    if (cl == ch) {
+                        code = cl;
+                        done = true;
+                    }
+                }
+                if (!done)
+                    code = e4m3x4_from_f32(__fdiv_rn(e[0], sc), __fdiv_rn(e[1], sc),
+                                           __fdiv_rn(e[2], sc), __fdiv_rn(e[3], sc));
+            }
+            w[h] = code;
+        }
+        *reinterpret_cast<uint2*>(codes + r * D + 8 * c) = make_uint2(w[0], w[1]);
+    }
+    if (lane == 0) scales[r] = sc;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, KVC_DEV_NONFINITE);
+}
+
+template <typename T>
+cudaError_t launch_window_t(const void* rows, long long n, int D, uint8_t* codes, float* scales,
+                            uint32_t* status, cudaStream_t s) {
+    const unsigned grid = (unsigned)((n + kWinWarps - 1) / kWinWarps);
+    const int maxc = (D / 8 + 31) / 32;
+    const T* r = static_cast<const T*>(rows);
+    trace_before("window_fp8", s);
+    cudaError_t err;
+    if (maxc <= 1)
+        err = launch_pdl(window_fp8_kernel<T, 1>, grid, kWinWarps * 32, 0, s, r, n, D, codes, scales, status);
+    else if (maxc <= 2)
+        err = launch_pdl(window_fp8_kernel<T, 2>, grid, kWinWarps * 32, 0, s, r, n, D, codes, scales, status);
+    else if (maxc <= 3)
+        err = launch_pdl(window_fp8_kernel<T, 3>, grid, kWinWarps * 32, 0, s, r, n, D, codes, scales, status);
+    else
+        err = launch_pdl(window_fp8_kernel<T, 4>, grid, kWinWarps * 32, 0, s, r, n, D, codes, scales, status);
+    trace_after(s);
+    return err;
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
@@ -627,6 +720,14 @@ cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
                      half, a.capacity);
     trace_after(s);
     return err;
+}
+
+cudaError_t launch_window_fp8(const kvc_config& c, const Shape& sh, const void* rows, long long n,
+                              uint8_t* codes, float* scales, uint32_t* status, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    return c.act_dtype == KVC_BF16
+               ? launch_window_t<__nv_bfloat16>(rows, n, sh.D, codes, scales, status, s)
+               : launch_window_t<float>(rows, n, sh.D, codes, scales, status, s);
 }
 
 }  // namespace kvc

@@ -65,6 +65,8 @@ def _lib():
             "kvc_layer_group_step": (S, [P, I, P, P, P, P, I, P, P, P, P, P, Z, P, P]),
             "kvc_workspace_bytes_hier": (Z, [P, I, I, I, I]),
             "kvc_workspace_bytes_batched": (Z, [P, I, I, I]),
+            "kvc_pack_window_fp8": (S, [P, P, C.c_int64, P, P, P, P]),
+            "kvc_sparse_decode_attn_fp8win": (S, [P, P, P, P, P, P, I, P, P, P, Z, P, P]),
             "kvc_index_topk_batched": (S, [P, I, P, P, P, P, Z, P, P]),
             "kvc_layer_group_step_hier": (S, [P, I, I, I, P, P, P, P, I, P, P, P, P, P, Z, P,
                                               P]),
@@ -170,6 +172,22 @@ def _ws(ws):
     base = ws.data_ptr()
     off = (-base) % 256
     return C.c_void_p(base + off), ws.numel() - off
+
+
+def pack_window_fp8(cfg, rows, codes, scales, status=None, stream=None):
+    """rows [..][D] -> codes [..][D] uint8 (signed E4M3), scales [..] fp32."""
+    n = rows.numel() // rows.shape[-1]
+    _check("kvc_pack_window_fp8", _lib().kvc_pack_window_fp8(
+        C.byref(cfg), _ptr(rows), n, _ptr(codes), _ptr(scales), _ptr(status), _stream(stream)))
+
+
+def sparse_decode_attn_fp8win(cfg, q, cache: Cache, topk_idx, win_codes, win_scales, window_len,
+                              out, ws, lse=None, status=None, stream=None):
+    p, n = _ws(ws)
+    cs = cache.struct()
+    _check("kvc_sparse_decode_attn_fp8win", _lib().kvc_sparse_decode_attn_fp8win(
+        C.byref(cfg), _ptr(q), C.byref(cs), _ptr(topk_idx), _ptr(win_codes), _ptr(win_scales),
+        int(window_len), _ptr(out), _ptr(lse), p, n, _ptr(status), _stream(stream)))
 
 
 def workspace_batched(cfg: Config, nq: int, batch: int, capacity: int,

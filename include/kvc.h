@@ -212,6 +212,30 @@ kvc_status kvc_sparse_decode_attn(const kvc_config* cfg, const void* q,
                                   float* lse, void* ws, size_t ws_bytes,
                                   uint32_t* dev_status, void* stream);
 
+/* FP8 window rows ([A] part 4 "P4 main KV": the sliding-window KV stays in
+ * FP8; the pages give no scale layout, so this build keeps one fp32 scale
+ * per row).  rows [n_rows][D] act_dtype -> codes [n_rows][D] signed E4M3
+ * bytes and scales [n_rows] fp32 = absmax / 448 over the row's finite
+ * elements; each code is x / scale rounded to nearest even, saturating at
+ * 448, a magnitude of zero stored as +0; non-finite elements are coded 0 and
+ * set KVC_DEV_NONFINITE.  rows 16-byte, codes 8-byte aligned.             */
+kvc_status kvc_pack_window_fp8(const kvc_config* cfg, const void* rows,
+                               int64_t n_rows, uint8_t* codes, float* scales,
+                               uint32_t* dev_status, void* stream);
+
+/* kvc_sparse_decode_attn with the window in FP8: win_codes [batch][window][D]
+ * signed E4M3 (16-byte aligned), win_scales [batch][window] fp32, as written
+ * by kvc_pack_window_fp8; each window key is E4M3(code) x scale.  D must be
+ * a multiple of 16.  Everything else as kvc_sparse_decode_attn.           */
+kvc_status kvc_sparse_decode_attn_fp8win(const kvc_config* cfg, const void* q,
+                                         const kvc_cache* cache,
+                                         const int32_t* topk_idx,
+                                         const uint8_t* win_codes,
+                                         const float* win_scales, int window_len,
+                                         float* out, float* lse, void* ws,
+                                         size_t ws_bytes, uint32_t* dev_status,
+                                         void* stream);
+
 /* One decode step through a CSA2 layer group (A11; [A] part 4 "CSA2：三种模式，
  * 40 层只存 4 份"): layers run in order on `stream`.
  *  Full    -- indexer top-K with its own idx_q over `cache`, then attention;
@@ -269,7 +293,7 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * max_launches launches are recorded).  kvc_trace_kernel, called after the
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
- * "pack", "pack_commit", "index_scan", "index_scan_tc",
+ * "pack", "pack_commit", "window_fp8", "index_scan", "index_scan_tc",
  * "topk_select", "block_max", "copy_topk", "attn_tc05", "attn_simt",
  * "attn_merge", "fp4_codec".                                                             */
 kvc_status kvc_trace_begin(int max_launches);
