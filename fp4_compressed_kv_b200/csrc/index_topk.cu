@@ -19,90 +19,18 @@
 //     its non-zero bins to the sequence's histogram.  The last scan CTA of a
 //     sequence (a fenced counter; nobody waits) derives the threshold bin t
 //     (the highest bin whose suffix count reaches K) and the count above it.
-//  2. topk_select: a CTA per tile of 8,192 scores compacts the (score,
-//     index) keys of its entries in bins >= t, in index order, into the
-//     tile's own slot (a warp per 1,024 scores, ballot prefix sums).  The
-//     sequence's last tile CTA (a fenced counter) then completes the
-//     selection without sorting the output: it stages every candidate key in
-//     shared memory in index order (one round of parallel loads), takes the
-//     r = K - above best keys of bin t (a bitonic sort of the few tie
-//     candidates) as the cut-off key k*, and a block prefix sum over the
-//     candidates with key >= k* places the winners in index order.  If more
-//     than kMaxTies entries share bin t, an exact slower path finds the
-//     threshold score and the index cut-off with a second histogram and
-//     compacts the scores.
+//  2. topk_select (topk_select.cu) takes the K best keys from the stored
+//     scores and the threshold bins.
 // No CTA waits on another: the launches are stream-ordered and the last-CTA
 // hand-offs are counters that nobody polls.
 #include <algorithm>
 #include <climits>
 
-#include "kvc_internal.cuh"
+#include "topk_common.cuh"
 
 namespace kvc {
 namespace {
 
-constexpr int kThreads = 256;
-
-__device__ __forceinline__ int score_bin(int s, int bias, int shift) {
-    return (s + bias) >> shift;
-}
-
-__device__ __forceinline__ unsigned long long make_key(int s, int idx, int bias) {
-    return ((unsigned long long)(uint32_t)(s + bias) << 32) | (uint32_t)(~(uint32_t)idx);
-}
-__device__ __forceinline__ int key_index(unsigned long long k) {
-    return (int)(~(uint32_t)(k & 0xffffffffull));
-}
-
-// Block-wide exclusive prefix sum of one int per thread; returns the block total.
-__device__ int block_excl_scan(int v, int* excl, int* sh_warp) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += u;
-    }
-    __syncthreads();
-    if (lane == 31) sh_warp[w] = x;
-    __syncthreads();
-    int pre = 0, total = 0;
-    for (int i = 0; i < nw; ++i) {
-        if (i < w) pre += sh_warp[i];
-        total += sh_warp[i];
-    }
-    *excl = pre + x - v;
-    return total;
-}
-
-// Block-wide: threshold bin t = the highest bin whose suffix count >= K, and
-// the count of entries in bins above t, from a histogram already staged in
-// shared memory.  Requires total >= K.  blockDim.x must divide kBins.
-__device__ void find_threshold(const int* s_hist, int K, int* t_out, int* above_out,
-                               int* sh_warp) {
-    const int nt = blockDim.x, tid = threadIdx.x;
-    const int per = kBins / nt;
-    // thread tid covers bins [kBins - (tid+1)*per, kBins - tid*per): thread 0 the top
-    const int hi = kBins - tid * per, lo = hi - per;
-    int local = 0;
-    for (int b = lo; b < hi; ++b) local += s_hist[b];
-    int excl;
-    // prefix over threads in order: thread 0 holds the top bins
-    block_excl_scan(local, &excl, sh_warp);
-    const int incl = excl + local;
-    if (excl < K && incl >= K) {
-        int run = excl;
-        for (int b = hi - 1; b >= lo; --b) {
-            if (run + s_hist[b] >= K) {
-                *t_out = b;
-                *above_out = run;
-                break;
-            }
-            run += s_hist[b];
-        }
-    }
-    __syncthreads();
-}
 
 // ---- bulk-copy pipeline helpers (non-multicast bulk copies into this CTA's
 // own shared memory; every wait bounded by a 2-second clock)
@@ -181,13 +109,6 @@ __device__ __forceinline__ void load_rows(const TopkArgs& a, int b, int row, int
     }
 }
 
-// Top-K output index of row p of sequence b: the entry itself, or in pool
-// mode the pool row's entry.
-__device__ __forceinline__ int out_index(const TopkArgs& a, int b, int p) {
-    if (!a.pool_blocks) return p;
-    const int blk = p / a.pool_block;
-    return a.pool_blocks[(size_t)b * a.pool_keep + blk] * a.pool_block + (p - blk * a.pool_block);
-}
 
 // Cursor over this CTA's rows, chunked per sequence: rows [row, end) of
 // sequence b are visible; chunks hold at most `rows` rows.
@@ -358,351 +279,6 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
     }
 }
 
-// In-place block bitonic sort of p (a power of two) keys; descending when
-// `desc`.  Every thread of the block must call it.
-template <typename Key>
-__device__ void block_bitonic(Key* k, int p, bool desc) {
-    for (int size = 2; size <= p; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = threadIdx.x; i < p; i += blockDim.x) {
-                const int j = i ^ stride;
-                if (j > i) {
-                    const bool up = ((i & size) == 0) != desc;  // ascending run
-                    const Key x = k[i], y = k[j];
-                    if ((x > y) == up) {
-                        k[i] = y;
-                        k[j] = x;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
-}
-
-// Candidate keys of one sequence staged in shared memory for the finish.
-// One warp sorts up to 64 keys descending (lane l holds positions l and l+32;
-// padding must be 0).  Ascending bitonic network on ~key, shuffles only.
-__device__ __forceinline__ void warp_sort64_desc(unsigned long long& x0, unsigned long long& x1,
-                                                 int lane) {
-    x0 = ~x0;
-    x1 = ~x1;
-#pragma unroll
-    for (int k = 2; k <= 64; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            if (j == 32) {  // partner is the lane's other element; k == 64: ascending
-                const unsigned long long lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
-                x0 = lo;
-                x1 = hi;
-            } else {
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    unsigned long long& x = r ? x1 : x0;
-                    const int e = lane + 32 * r;
-                    const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
-                    const bool asc = (e & k) == 0;
-                    const bool keep_min = ((e & j) == 0) == asc;
-                    x = keep_min ? (x < y ? x : y) : (x < y ? y : x);
-                }
-            }
-        }
-    }
-    x0 = ~x0;
-    x1 = ~x1;
-}
-
-constexpr int kStageKeys = 6144;
-constexpr size_t kFinishSmem =
-    (size_t)kStageKeys * 8 + (size_t)kMaxTies * 8 + (size_t)kMaxSelTiles * 4 * 2;
-
-// One CTA per sequence finishes the selection from the tiles' candidates.
-__device__ void finish_body(const TopkArgs& a, int b, int bias, int shift, unsigned char* smem);
-
-// Finishes sequence b; in the hierarchical block stage also derives the pool
-// length (whole kept blocks, the sequence's last block counting only its
-// visible entries).
-__device__ void finish_sequence(const TopkArgs& a, int b, int bias, int shift,
-                                unsigned char* smem) {
-    finish_body(a, b, bias, shift, smem);
-    if (!a.pool_len_out) return;
-    __syncthreads();  // this CTA's output writes are visible to its threads
-    if (threadIdx.x == 0) {
-        const int nb = a.n_entries[b];  // blocks of the sequence
-        const int n0 = a.pool_src_n[b];
-        const int n = (n0 >= 0 && n0 <= a.pool_src_cap) ? n0 : 0;
-        const int kept = (nb >= 0 && nb <= a.capacity) ? min(a.topk, nb) : 0;
-        int len = kept * a.pool_src_block;
-        if (kept > 0 && __ldcg(a.topk_idx + (size_t)b * a.topk + kept - 1) == nb - 1)
-            len -= nb * a.pool_src_block - n;
-        a.pool_len_out[b] = len;
-    }
-}
-
-__device__ void finish_body(const TopkArgs& a, int b, int bias, int shift, unsigned char* smem) {
-    unsigned long long* stage = reinterpret_cast<unsigned long long*>(smem);  // kStageKeys
-    unsigned long long* ties = stage + kStageKeys;                            // kMaxTies
-    int* cnt = reinterpret_cast<int*>(ties + kMaxTies);                       // per tile
-    int* off = cnt + kMaxSelTiles;                                            // per tile
-    __shared__ int sh_warp[kThreads / 32];
-    __shared__ int s_nt, s_low, s_gt;
-    __shared__ unsigned long long s_kstar;
-    const int K = a.topk, tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    const int n = a.n_entries[b];
-    int32_t* out = a.topk_idx + (size_t)b * K;
-    if (n < 0 || n > a.capacity) {
-        for (int i = tid; i < K; i += kThreads) out[i] = -1;
-        return;
-    }
-    if (n <= K) {
-        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? out_index(a, b, i) : -1;
-        return;
-    }
-    const int ntiles = (n + kSelTile - 1) / kSelTile;
-    const int t = __ldcg(a.thr + 2 * b), above = __ldcg(a.thr + 2 * b + 1);
-    const int32_t* sc = a.scores + (size_t)b * a.capacity;
-    const int ctiles = sel_tiles(a.capacity);
-    const unsigned long long* cb = a.cands + (size_t)b * ctiles * kSelTile;
-    // tile counts and their exclusive prefix
-    int M = 0;
-    for (int base = 0; base < ntiles; base += kThreads) {
-        const int i = base + tid;
-        const int c = i < ntiles ? __ldcg(a.tile_count + (size_t)b * ctiles + i) : 0;
-        int ex;
-        const int tot = block_excl_scan(c, &ex, sh_warp);
-        if (i < ntiles) {
-            cnt[i] = c;
-            off[i] = M + ex;
-        }
-        M += tot;
-    }
-    if (tid == 0) s_nt = 0;
-    __syncthreads();
-    const int r = K - above;  // entries to take from bin t
-    if (M <= kStageKeys) {
-        // every candidate key, in index order: all loads in flight at once,
-        // then the keys of bin t gathered from shared memory
-#pragma unroll 4
-        for (int p = tid; p < M; p += kThreads) {
-            int lo = 0, hi = ntiles - 1;  // last tile with off <= p
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (off[mid] <= p) lo = mid; else hi = mid - 1;
-            }
-            stage[p] = __ldcg(cb + (size_t)lo * kSelTile + (p - off[lo]));
-        }
-        __syncthreads();
-        for (int p = tid; p < M; p += kThreads) {
-            const unsigned long long k = stage[p];
-            if ((int)((k >> 32) >> shift) == t) {
-                const int q = atomicAdd(&s_nt, 1);
-                if (q < kMaxTies) ties[q] = k;
-            }
-        }
-        __syncthreads();
-        const int nt = s_nt;
-        if (nt <= kMaxTies) {
-            if (nt <= 64) {  // the common case: one warp, no block barriers
-                if (warp == 0) {
-                    unsigned long long x0 = lane < nt ? ties[lane] : 0ull;
-                    unsigned long long x1 = lane + 32 < nt ? ties[lane + 32] : 0ull;
-                    warp_sort64_desc(x0, x1, lane);
-                    const int want = r - 1;  // r-th best key of bin t
-                    const unsigned long long k =
-                        __shfl_sync(0xffffffffu, want < 32 ? x0 : x1, want & 31);
-                    if (lane == 0) s_kstar = (r >= 1 && r <= nt) ? k : ~0ull;
-                }
-            } else {
-                int p2 = 1;
-                while (p2 < nt) p2 <<= 1;
-                for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;  // sorts last
-                __syncthreads();
-                block_bitonic(ties, p2, true);
-                if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;
-            }
-            __syncthreads();
-            const unsigned long long kstar = s_kstar;
-            int run = 0;
-            for (int base = 0; base < M; base += kThreads) {
-                const int p = base + tid;
-                const bool sel = p < M && stage[p] >= kstar;
-                int ex;
-                const int tot = block_excl_scan(sel ? 1 : 0, &ex, sh_warp);
-                if (sel && run + ex < K) out[run + ex] = out_index(a, b, key_index(stage[p]));
-                run += tot;
-            }
-            for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
-            return;
-        }
-    } else {
-        // too many candidates to stage: the tie keys straight from the tiles
-        for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
-            const unsigned long long* ct = cb + (size_t)ti * kSelTile;
-            for (int i = lane; i < cnt[ti]; i += 32) {
-                const unsigned long long k = __ldcg(ct + i);
-                if ((int)((k >> 32) >> shift) == t) {
-                    const int q = atomicAdd(&s_nt, 1);
-                    if (q < kMaxTies) ties[q] = k;
-                }
-            }
-        }
-        __syncthreads();
-        const int nt = s_nt;
-        if (nt <= kMaxTies) {
-            int p2 = 1;
-            while (p2 < nt) p2 <<= 1;
-            for (int i = nt + tid; i < p2; i += kThreads) ties[i] = 0ull;
-            __syncthreads();
-            block_bitonic(ties, p2, true);
-            if (tid == 0) s_kstar = (r >= 1 && r <= nt) ? ties[r - 1] : ~0ull;
-            __syncthreads();
-            const unsigned long long kstar = s_kstar;
-            // winners per tile, prefix over tiles, then write in index order
-            for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
-                const unsigned long long* ct = cb + (size_t)ti * kSelTile;
-                int c = 0;
-                for (int i = lane; i < cnt[ti]; i += 32) c += __ldcg(ct + i) >= kstar;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-                if (lane == 0) off[ti] = c;
-            }
-            __syncthreads();
-            int run = 0;
-            for (int base = 0; base < ntiles; base += kThreads) {
-                const int i = base + tid;
-                const int c = i < ntiles ? off[i] : 0;
-                int ex;
-                const int tot = block_excl_scan(c, &ex, sh_warp);
-                if (i < ntiles) off[i] = run + ex;
-                run += tot;
-                __syncthreads();
-            }
-            for (int ti = warp; ti < ntiles; ti += kThreads / 32) {
-                const unsigned long long* ct = cb + (size_t)ti * kSelTile;
-                int o = off[ti];
-                for (int i0 = 0; i0 < cnt[ti]; i0 += 32) {
-                    const int i = i0 + lane;
-                    const unsigned long long k = i < cnt[ti] ? __ldcg(ct + i) : 0ull;
-                    const bool sel = i < cnt[ti] && k >= kstar;
-                    const unsigned m = __ballot_sync(0xffffffffu, sel);
-                    const int p = o + __popc(m & ((1u << lane) - 1u));
-                    if (sel && p < K) out[p] = out_index(a, b, key_index(k));
-                    o += __popc(m);
-                }
-            }
-            __syncthreads();
-            for (int i = run + tid; i < K; i += kThreads) out[i] = -1;  // only if inconsistent
-            return;
-        }
-    }
-
-    // Heavy ties: exact threshold score inside bin t from a second histogram
-    // over the low `shift` bits (<= 4096 bins), then an index-order pass.
-    int* h2 = reinterpret_cast<int*>(smem);
-    const int nb2 = 1 << shift;
-    for (int i = tid; i < nb2; i += kThreads) h2[i] = 0;
-    __syncthreads();
-    for (int j = tid; j < n; j += kThreads) {
-        const int v = __ldcg(sc + j) + bias;
-        if ((v >> shift) == t) atomicAdd(&h2[v & (nb2 - 1)], 1);
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int run = 0, low = 0;
-        for (int i = nb2 - 1; i >= 0; --i) {
-            if (run + h2[i] >= r) {
-                low = i;
-                break;
-            }
-            run += h2[i];
-        }
-        s_low = low;  // threshold score = (t << shift | low) - bias
-        s_gt = run;   // entries of bin t above the threshold score
-    }
-    __syncthreads();
-    const int thr = ((t << shift) | s_low) - bias;
-    const int need_eq = r - s_gt;  // entries equal to thr to take, lowest index first
-    int taken = 0, eq_seen = 0;
-    for (int base = 0; base < n; base += kThreads) {
-        const int j = base + tid;
-        const int s = j < n ? __ldcg(sc + j) : INT32_MIN;
-        const int is_eq = (j < n && s == thr) ? 1 : 0;
-        int eq_before;
-        const int eq_total = block_excl_scan(is_eq, &eq_before, sh_warp);
-        const int take = (j < n) && (s > thr || (is_eq && eq_seen + eq_before < need_eq));
-        int pos_before;
-        const int take_total = block_excl_scan(take, &pos_before, sh_warp);
-        if (take && taken + pos_before < K) out[taken + pos_before] = out_index(a, b, j);
-        taken += take_total;
-        eq_seen += eq_total;
-    }
-    for (int i = taken + tid; i < K; i += kThreads) out[i] = -1;
-}
-
-__global__ void __launch_bounds__(kThreads)
-topk_select_kernel(TopkArgs a, int bias, int shift) {
-    extern __shared__ __align__(16) unsigned char fsmem[];
-    __shared__ int sh_warp[kThreads / 32];
-    __shared__ int s_last;
-    constexpr int PER = kSelTile / kThreads;     // scores per thread (32)
-    constexpr int WROWS = kSelTile / (kThreads / 32);  // rows per warp (1024)
-    pdl_wait();
-    const int b = blockIdx.y, K = a.topk, tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    const int n = a.n_entries[b];
-    if (n < 0 || n > a.capacity || n <= K) {  // nothing to select: all or nothing
-        if (blockIdx.x == 0) finish_sequence(a, b, bias, shift, fsmem);
-        return;
-    }
-    const int ntiles = (n + kSelTile - 1) / kSelTile;
-    const int tile = blockIdx.x;
-    if (tile >= ntiles) return;
-    const int t = __ldcg(a.thr + 2 * b);
-    const int32_t* sc = a.scores + (size_t)b * a.capacity;
-    const int ctiles = sel_tiles(a.capacity);
-    unsigned long long* cand = a.cands + ((size_t)b * ctiles + tile) * kSelTile;
-    // warp w owns rows [w*1024, (w+1)*1024) of the tile; lane l reads rows
-    // i*32 + l, so every load of the warp is one contiguous 128-byte line
-    const int r0 = tile * kSelTile + warp * WROWS + lane;
-    int v[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) v[i] = (r0 + 32 * i < n) ? __ldcg(sc + r0 + 32 * i) : 0;
-    unsigned take = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-        if (r0 + 32 * i < n && score_bin(v[i], bias, shift) >= t) take |= 1u << i;
-    int wc = __popc(take);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) wc += __shfl_xor_sync(0xffffffffu, wc, o);
-    if (lane == 0) sh_warp[warp] = wc;
-    __syncthreads();
-    int base = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) {
-        base += w < warp ? sh_warp[w] : 0;
-        total += sh_warp[w];
-    }
-    // compact in index order: row-major over (i, lane) inside the warp
-    const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const unsigned m = __ballot_sync(0xffffffffu, (take >> i) & 1u);
-        if ((take >> i) & 1u) cand[base + __popc(m & lt)] = make_key(v[i], r0 + 32 * i, bias);
-        base += __popc(m);
-    }
-    if (tid == 0) a.tile_count[(size_t)b * ctiles + tile] = total;
-    // the sequence's last tile CTA (a fenced counter; nobody waits) finishes it
-    __threadfence();
-    __syncthreads();
-    if (tid == 0)
-        s_last = atomicAdd(a.counters + (size_t)a.batch * (kBins + 1) + b, 1) == ntiles - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (tid == 0) a.counters[(size_t)a.batch * (kBins + 1) + b] = 0;  // zeroed for the next call
-    finish_sequence(a, b, bias, shift, fsmem);
-}
 
 
 // ---- hierarchical indexer, block stage
@@ -1041,24 +617,6 @@ cudaError_t launch_scan(const TopkArgs& a, int ctas, long long per, int bias, in
                       s, a, per, bias, shift);
 }
 
-cudaError_t launch_select(const TopkArgs& a, int bias, int shift, cudaStream_t s) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    static bool attr_set[64] = {};
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(
-            topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinishSmem);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
-    dim3 grid(sel_tiles(a.capacity), a.batch);
-    trace_before("topk_select", s);
-    const cudaError_t err =
-        launch_pdl(topk_select_kernel, grid, kThreads, kFinishSmem, s, a, bias, shift);
-    trace_after(s);
-    return err;
-}
-
 
 }  // namespace
 
@@ -1066,12 +624,14 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
     if (h.batch == 0) return cudaSuccess;
     const int bias = score_bias(h.di), shift = score_shift(h.di);
     const int cap_blk = (h.capacity + h.block - 1) / h.block;
-    cudaError_t err;
-    trace_before("block_max", s);
-    err = launch_pdl(block_max_kernel, dim3((cap_blk + kBlkPerCta - 1) / kBlkPerCta, h.batch),
-                     kThreads, 0, s, h, cap_blk, bias, shift);
-    trace_after(s);
-    if (err != cudaSuccess) return err;
+    if (cap_blk > 0) {
+        trace_before("block_max", s);
+        const cudaError_t err =
+            launch_pdl(block_max_kernel, dim3((cap_blk + kBlkPerCta - 1) / kBlkPerCta, h.batch),
+                       kThreads, 0, s, h, cap_blk, bias, shift);
+        trace_after(s);
+        if (err != cudaSuccess) return err;
+    }
     TopkArgs a = {};
     a.n_entries = h.nblk;
     a.batch = h.batch;
@@ -1128,10 +688,12 @@ cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s) {
     per = (per + tcs::ROWS - 1) / tcs::ROWS * tcs::ROWS;
     if (per < tcs::ROWS) per = tcs::ROWS;
     ctas = (int)((rows + per - 1) / per);
-    trace_before("index_scan_tc", s);
-    err = launch_pdl(index_scan_tc_kernel, ctas, tcs::NT, smem, s, ba, per, bias, shift, stages);
-    trace_after(s);
-    if (err != cudaSuccess) return err;
+    if (rows > 0) {
+        trace_before("index_scan_tc", s);
+        err = launch_pdl(index_scan_tc_kernel, ctas, tcs::NT, smem, s, ba, per, bias, shift, stages);
+        trace_after(s);
+        if (err != cudaSuccess) return err;
+    }
     for (int q = 0; q < ba.nq; ++q)
         if ((err = launch_select(ba.q[q], bias, shift, s)) != cudaSuccess) return err;
     return cudaSuccess;
@@ -1153,16 +715,18 @@ cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
     per = (per + 255) / 256 * 256;
     if (per < 256) per = 256;
     ctas = (int)((rows + per - 1) / per);
-    trace_before("index_scan", s);
-    switch (a.di) {
-        case 16: err = launch_scan<16>(a, ctas, per, bias, shift, s); break;
-        case 32: err = launch_scan<32>(a, ctas, per, bias, shift, s); break;
-        case 64: err = launch_scan<64>(a, ctas, per, bias, shift, s); break;
-        case 128: err = launch_scan<128>(a, ctas, per, bias, shift, s); break;
-        default: err = launch_scan<256>(a, ctas, per, bias, shift, s); break;
+    if (rows > 0) {  // (no rows at all: the selection alone writes the -1 padding)
+        trace_before("index_scan", s);
+        switch (a.di) {
+            case 16: err = launch_scan<16>(a, ctas, per, bias, shift, s); break;
+            case 32: err = launch_scan<32>(a, ctas, per, bias, shift, s); break;
+            case 64: err = launch_scan<64>(a, ctas, per, bias, shift, s); break;
+            case 128: err = launch_scan<128>(a, ctas, per, bias, shift, s); break;
+            default: err = launch_scan<256>(a, ctas, per, bias, shift, s); break;
+        }
+        trace_after(s);
+        if (err != cudaSuccess) return err;
     }
-    trace_after(s);
-    if (err != cudaSuccess) return err;
     return launch_select(a, bias, shift, s);
 }
 

@@ -103,6 +103,8 @@ struct TopkArgs {
     int pool_src_cap, pool_src_block;
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
+// The selection alone, from scores and threshold bins already in the scratch.
+cudaError_t launch_select(const TopkArgs& a, int bias, int shift, cudaStream_t s);
 
 // Several indexer queries per sequence scored in one pass over the shared
 // indexer cache on the tensor cores (kind::i8), then one selection per query.

@@ -148,3 +148,67 @@ def test_workspace_reused_across_calls(kvc):
         want = _oracle(w, idx_k, q, n, 20000)[0]
         assert st.item() == 0, rnd
         topk_set_equal(tk.cpu().numpy(), want)
+
+
+def _rows_with_sums(sums, di=128):
+    """int8 rows whose elements add up to the given sums (|sum| <= 127 * di)."""
+    sums = np.asarray(sums, np.int64)
+    base = np.floor_divide(sums, di)
+    rem = sums - base * di
+    rows = np.repeat(base[:, None], di, 1)
+    rows += (np.arange(di)[None, :] < rem[:, None])
+    assert np.all(rows.sum(1) == sums) and np.abs(rows).max() <= 127
+    return torch.from_numpy(rows.astype(np.int8))
+
+
+@pytest.mark.parametrize("ties", [100, 1000, 6000])
+@pytest.mark.parametrize("cap", [20000, 9 * 8192, 9 * 16384])
+def test_topk_tie_counts(kvc, ties, cap):
+    """A chosen number of entries in the threshold bin, spread over every
+    tile: up to 128 (one warp sorts them), up to 4096 (a block sorts them),
+    more (the second-histogram pass).  A capacity of at most 8 tiles of
+    8,192 or of 16,384 scores selects inside one cluster per sequence, a
+    larger one through the sequence's last tile CTA."""
+    w = synth.WORKLOADS["mla32k"].scaled(context=2 * 20000)
+    N, K = 20000, w.topk
+    rng = np.random.default_rng(ties)
+    pos = rng.permutation(N)
+    sums = np.full(N, -5000, np.int64)
+    sums[pos[:400]] = 8000 + np.arange(400)              # above the threshold bin
+    sums[pos[400:400 + ties]] = 5000 + rng.integers(0, 4, ties)  # the threshold bin
+    idx_k = _rows_with_sums(sums).unsqueeze(0)
+    idx_q = torch.full((1, 128), 127, dtype=torch.int8)
+    tk, sc, st = _run(kvc, w, idx_k, idx_q, [N], cap)
+    otk, osc = _oracle(w, idx_k, idx_q, [N], cap)
+    assert st == 0 and np.array_equal(sc[:, :N], osc[:, :N])
+    topk_set_equal(tk, otk)
+    assert np.array_equal(tk, otk)  # ascending, exactly K (no -1)
+    assert np.all(tk >= 0) and tk.shape[1] == K
+
+
+@pytest.mark.parametrize("cap", [8192 * 8, 8192 * 8 + 1, 16384 * 8, 16384 * 8 + 1])
+def test_topk_cluster_tile_boundaries(kvc, cap):
+    """Capacities at the edges of the selection layouts (8 tiles of 8,192,
+    8 tiles of 16,384, beyond).  The winners crowd into the last 4,200
+    entries (the most recent score highest): 200 distinct high scores and
+    4,000 equal ones in the threshold bin, so one tile holds more candidate
+    keys than its shared-memory buffer (they spill to global memory) and a
+    block sorts the ties."""
+    w = synth.WORKLOADS["mla32k"].scaled(batch=2, context=2 * 4096)
+    g = torch.Generator().manual_seed(cap % 1000)
+    n = [cap, cap - 1000]
+    idx_q = torch.randint(-127, 128, (2, 128), generator=g, dtype=torch.int8)
+    idx_k = torch.randint(-127, 128, (2, cap, 128), generator=g, dtype=torch.int8)
+    for b in range(2):
+        q16 = idx_q[b].to(torch.int16)
+        lo = n[b] - 4200
+        idx_k[b, lo:n[b]] = (q16 // 2).to(torch.int8)  # equal scores, about |q|^2 / 2
+        hi = (q16 * 3 // 4).to(torch.int8).repeat(200, 1)
+        hi[:, :8] = torch.randint(-127, 128, (200, 8), generator=g, dtype=torch.int8)
+        idx_k[b, lo:n[b]:21] = hi                        # 200 rows above them
+    tk, sc, st = _run(kvc, w, idx_k, idx_q, n, cap)
+    otk, osc = _oracle(w, idx_k, idx_q, n, cap)
+    assert st == 0
+    for b in range(2):
+        assert np.array_equal(sc[b, : n[b]], osc[b, : n[b]])
+    topk_set_equal(tk, otk)
