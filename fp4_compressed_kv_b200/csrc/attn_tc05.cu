@@ -254,11 +254,9 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
         mref[tid] = -INFINITY;
         lrun[tid] = 0.f;
     }
-    pdl_wait();  // everything above was local set-up
-    const int n = a.n_entries[b];
-    const bool len_ok = n >= 0 && n <= a.capacity;
-    // Q (64 x 576) once, converted to f16, 128B-swizzled K-major
-    {
+    // Q (64 x 576) once, converted to f16, 128B-swizzled K-major: before the
+    // wait when no kernel launched since the caller wrote q writes it
+    auto load_q = [&]() {
         const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(a.q) +
                                                          (size_t)b * H * D * 2);
 #pragma unroll 6
@@ -271,7 +269,12 @@ attn_tc05_kernel(AttnArgs a, Shape sh, int K, float scale_log2, int nsplit, int 
                          "r"(bf16x2_to_f16x2(v.z)), "r"(bf16x2_to_f16x2(v.w)));
         }
         fence_async_smem();
-    }
+    };
+    if (a.q_ready) load_q();
+    pdl_wait();  // everything above was local set-up or reads of inputs
+    const int n = a.n_entries[b];
+    const bool len_ok = n >= 0 && n <= a.capacity;
+    if (!a.q_ready) load_q();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

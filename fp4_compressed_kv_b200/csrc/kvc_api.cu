@@ -292,8 +292,10 @@ kvc_status run_attn(const kvc_config& c, const Shape& sh, const void* q, const k
                     const int32_t* topk, const void* window, int window_len, float* out,
                     float* lse, unsigned char* ws, const WsLayout& w, uint32_t* st,
                     cudaStream_t s, int32_t* topk_copy = nullptr,
-                    const uint8_t* win_fp8 = nullptr, const float* win_scale = nullptr) {
+                    const uint8_t* win_fp8 = nullptr, const float* win_scale = nullptr,
+                    bool q_ready = false) {
     AttnArgs a = {};
+    a.q_ready = q_ready ? 1 : 0;
     a.topk_copy = topk_copy;
     a.win_fp8 = win_fp8;
     a.win_scale = win_scale;
@@ -535,7 +537,8 @@ kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int
                       reuse ? topk + (size_t)head * B * K : tk,
                       windows ? static_cast<const unsigned char*>(windows) + l * w_stride : nullptr,
                       window_len, out + (size_t)l * B * H * sh.Dv, lse ? lse + (size_t)l * B * H : nullptr,
-                      wsb, w, dev_status, s, reuse ? tk : nullptr);
+                      wsb, w, dev_status, s, reuse ? tk : nullptr, nullptr, nullptr,
+                      /*q_ready=*/true);  // only this step's own kernels ran since the call
         if (st != KVC_OK) return st;
     }
     return KVC_OK;

@@ -156,6 +156,10 @@ struct AttnArgs {
     // [B][W][D] with one fp32 scale per row [B][W] (window is then unused)
     const uint8_t* win_fp8;
     const float* win_scale;
+    // set when nothing launched between the caller's last write of q and
+    // this call writes q (a layer-group step): q is then read while the
+    // previous kernel still drains, before griddepcontrol.wait
+    int q_ready;
 };
 cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                              cudaStream_t s);
@@ -170,9 +174,13 @@ cudaError_t launch_fp4_codec(const float* x, int64_t n, uint8_t* out, int e4m3,
 
 // Every library kernel is launched with programmatic stream serialization:
 // the long kernels signal griddepcontrol.launch_dependents once their main
-// loop is done, so the next kernel's CTAs are scheduled while they drain; each
-// kernel does only local set-up (shared memory, tensor memory, barriers)
-// before waiting for its predecessor with griddepcontrol.wait.
+// loop is done, the pack of a few tokens as it starts, so the next kernel's
+// CTAs are scheduled while they run or drain (the selection does not: the
+// attention's clusters are placed best on SMs freed all at once);
+// each kernel does only local set-up (shared memory, tensor memory,
+// barriers, and inputs no library kernel writes) before waiting for its
+// predecessor with griddepcontrol.wait, which returns once the predecessor
+// -- and so every kernel before it -- has completed.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args... args) {

@@ -422,6 +422,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
 pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     extern __shared__ __align__(16) unsigned char stage_smem[];
     __shared__ __align__(16) uint8_t tail_smem[kSmallWarps][kTailBytes];
+    pdl_trigger();  // a short kernel: the next one may be scheduled at once
     pdl_wait();
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long e = (long long)blockIdx.x * kSmallWarps + wid;

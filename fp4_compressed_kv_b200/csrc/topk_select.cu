@@ -537,14 +537,27 @@ topk_select_cluster_kernel(TopkArgs a, int bias, int shift) {
             const int pos = base + __popc(m & lt);
             if (spill) gslot[pos] = key;
             else cand[pos] = key;
-            if (score_bin(v[i], bias, shift) == t) {
-                const int q = atomicAdd(&s_nt, 1);
-                if (q < kTieSlots) ties[q] = key;  // staged; sent below in one round
-            }
         }
         base += __popc(m);
     }
     if (spill) __threadfence();
+    __syncthreads();
+    // this tile's keys of bin t, staged (any order) to be sent below in one
+    // round: one shared-memory atomic per warp and pass
+    {
+        const unsigned long long* mine = spill ? gslot : cand;
+        for (int p0 = 0; p0 < total; p0 += kThreads) {
+            const int p = p0 + tid;
+            const unsigned long long key = p < total ? mine[p] : 0ull;
+            const bool tie = p < total && (int)((key >> 32) >> shift) == t;
+            const unsigned m = __ballot_sync(0xffffffffu, tie);
+            int q0 = 0;
+            if (lane == 0 && m) q0 = atomicAdd(&s_nt, __popc(m));
+            q0 = __shfl_sync(0xffffffffu, q0, 0);
+            const int q = q0 + __popc(m & lt);
+            if (tie && q < kTieSlots) ties[q] = key;
+        }
+    }
     __syncthreads();
     {  // this tile's counts and ties into every CTA (one store per thread)
         const int nt = s_nt, sent = min(nt, kTieSlots);
