@@ -423,26 +423,22 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     extern __shared__ __align__(16) unsigned char stage_smem[];
     __shared__ __align__(16) uint8_t tail_smem[kSmallWarps][kTailBytes];
     pdl_trigger();  // a short kernel: the next one may be scheduled at once
-    pdl_wait();
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long e = (long long)blockIdx.x * kSmallWarps + wid;
     const int half = a.n_new >> 1;
     if (e >= (long long)a.batch * half) return;  // whole warp
     const int b = (int)(e / half), i = (int)(e % half);
-    const int base = a.n_entries[b];
-    if (base < 0 || base + half > a.capacity) {
-        if (i == 0 && lane == 0) set_status(a.status, KVC_DEV_CAPACITY);
-        return;
-    }
     const int D = sh.D, nchunk = D >> 3;
-    const long long pos = (long long)base + i;
     const T* k0p = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 2 * i) * D;
     const T* k1p = k0p + D;
     T* s0 = reinterpret_cast<T*>(stage_smem + wid * small_stage_bytes<T>(D));
     T* s1 = s0 + D;
     float* sg = reinterpret_cast<float*>(s1 + D);
 
-    // every load of the entry in flight at once
+    // The entry is formed before waiting for the previous kernel: the token
+    // pair, gate and indexer row are inputs no library kernel writes; only
+    // the sequence's length and the cache stores wait.  Every load in flight
+    // at once.
     uint4 ik = make_uint4(0, 0, 0, 0);
     if (lane < (di >> 4))
         ik = __ldcs(reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di) +
@@ -492,7 +488,6 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-delta)));
     const float w1 = __fsub_rn(1.0f, w0);
 
-    uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
     uint8_t* tail = tail_smem[wid];
     const int tail_len = sh.rb - sh.code_bytes;
     for (int t = lane * 4; t < tail_len; t += 128) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
@@ -500,6 +495,7 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
 
     bool bad = false;
     const int lpg = sh.lpg;
+    uint32_t code[MAXJ];  // the 8 codes of chunk lane + 32 j
 #pragma unroll
     for (int j = 0; j < MAXJ; ++j) {
         const int c = lane + 32 * j;
@@ -517,6 +513,7 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
             m = fmaxf(m, fabsf(v));
         }
         for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        code[j] = 0u;
         if (!active) continue;
         float s = __fdiv_rn(m, 6.0f);
         uint32_t sbyte = 0;
@@ -524,7 +521,7 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
             sbyte = e4m3_from_f32(s);
             s = e4m3_to_f32(sbyte);
         }
-        *reinterpret_cast<uint32_t*>(rec + 4 * c) = s > 0.f ? e2m1x8_quotient(x, s) : 0u;
+        code[j] = s > 0.f ? e2m1x8_quotient(x, s) : 0u;
         if (c % lpg == 0) {
             const int gi = c / lpg;
             if (ue4m3)
@@ -534,6 +531,20 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
         }
     }
     __syncwarp();
+
+    pdl_wait();  // the previous kernel is done: the length and the cache
+    const int base = a.n_entries[b];
+    if (base < 0 || base + half > a.capacity) {
+        if (i == 0 && lane == 0) set_status(a.status, KVC_DEV_CAPACITY);
+        return;
+    }
+    const long long pos = (long long)base + i;
+    uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nchunk) *reinterpret_cast<uint32_t*>(rec + 4 * c) = code[j];
+    }
     for (int t = lane * 4; t < tail_len; t += 128)
         *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
             *reinterpret_cast<const uint32_t*>(tail + t);

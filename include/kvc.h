@@ -30,6 +30,14 @@
  *    synchronises.  Kernels never trap, and every wait inside a kernel is
  *    bounded: when a bound is hit the kernel sets KVC_DEV_TIMEOUT and returns.
  *  - Records and token/query/window rows must start on 16-byte boundaries.
+ *  - Kernels are launched as programmatic dependents of the kernel before
+ *    them on the stream and wait for it to complete (griddepcontrol.wait)
+ *    before reading anything a kernel may have written.  One exception:
+ *    kvc_pack reads its tokens, gate and idx_k_new before that wait, while
+ *    the previous kernel may still be finishing.  Ordinary kernels (which
+ *    never execute griddepcontrol.launch_dependents) have completed before
+ *    it starts, so this needs nothing; a caller's kernel that does signal
+ *    launch_dependents must do so after its last write of those inputs.
  */
 #ifndef KVC_H
 #define KVC_H
