@@ -60,18 +60,24 @@ def parse():
 
 
 def time_group(w, steps, warmup, hier_blocks, hier_block, dev):
-    """Device ms per decode step of workload w's layer group (no pack), K
+    """Device ms per decode step of workload w's layer groups (no pack), K
     steps in one CUDA graph; the CSA2 group and the 1M stack with and without
-    the hierarchical indexer."""
+    the hierarchical indexer, the 18-layer encoder stack (3 groups, each with
+    its own cache)."""
     import torch
     from fp4_compressed_kv_b200 import kvc, synth
     cfg = kvc.config_for(w)
-    inp = synth.make_inputs(w, dev)
-    cache = kvc.Cache(cfg, w.batch, w.entries, device=dev)
-    st = torch.zeros(1, dtype=torch.int32, device=dev)
-    kvc.pack(cfg, inp["tokens"], inp["gate"], inp["idx_k"], cache, status=st)
-    del inp["tokens"]
     L, B, H = w.layers, w.batch, w.heads
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    groups = []
+    for gi in range(w.groups):
+        inp = synth.make_inputs(w.scaled(seed=w.seed + 100 * gi), dev)
+        cache = kvc.Cache(cfg, w.batch, w.entries, device=dev)
+        kvc.pack(cfg, inp["tokens"], inp["gate"], inp["idx_k"], cache, status=st)
+        del inp["tokens"]
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        groups.append((inp, cache))
     out = torch.empty(L, B, H, w.latent, device=dev)
     lse = torch.empty(L, B, H, device=dev)
     tk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
@@ -79,9 +85,10 @@ def time_group(w, steps, warmup, hier_blocks, hier_block, dev):
                        hier_block=hier_block)
 
     def step():
-        kvc.layer_group_step(cfg, list(w.modes), inp["q"], inp["idx_q"], inp["windows"],
-                             w.window, cache, out, tk, ws, lse=lse, status=st,
-                             hier_blocks=hier_blocks, hier_block=hier_block)
+        for inp, cache in groups:
+            kvc.layer_group_step(cfg, list(w.modes), inp["q"], inp["idx_q"], inp["windows"],
+                                 w.window, cache, out, tk, ws, lse=lse, status=st,
+                                 hier_blocks=hier_blocks, hier_block=hier_block)
 
     for _ in range(warmup):
         step()
@@ -613,6 +620,15 @@ def run_ours(args):
             extra[name].update({"scoring_ms_per_layer_scans": round(one, 4),
                                 "scoring_ms_batched_tensor_core": round(bat, 4)})
             torch.cuda.empty_cache()
+        # the 18-layer encoder stack at 1M tokens: 3 groups (Full + 5 Reuse),
+        # each with its own cache
+        wx = synth.WORKLOADS["encoder1m"]
+        enc = time_group(wx, 10, 3, 0, 8, dev)
+        extra["encoder1m"] = {"ms_per_step": round(enc, 4),
+                              "query_tokens_per_s": round(wx.batch / (enc * 1e-3), 1),
+                              "layers": wx.groups * wx.layers,
+                              "groups": "3 x (Full + 5 Reuse), own cache each"}
+        torch.cuda.empty_cache()
         # the attention of this workload with the window in bf16 and in FP8
         extra["fp8_window"] = {
             "workload": w0.name,

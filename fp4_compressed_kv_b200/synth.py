@@ -40,6 +40,7 @@ class Workload:
     tail_factor: float
     seed: int
     pack_new: int = 0     # new raw tokens per sequence for the pack benchmark
+    groups: int = 1       # independent layer groups, each with its own cache and `modes`
 
     @property
     def dim(self) -> int:
@@ -51,6 +52,7 @@ class Workload:
 
     @property
     def layers(self) -> int:
+        """Layers of one group (every group has the same modes)."""
         return len(self.modes)
 
     @property
@@ -66,6 +68,7 @@ class Workload:
 
 
 _STACK20 = (FULL, REUSE, REUSE, REUSE) + (REINDEX, REUSE, REUSE, REUSE) * 4
+_ENC6 = (FULL,) + (REUSE,) * 5
 
 WORKLOADS = {
     # tiny single layer, fp32 everything, fp32 scales
@@ -83,6 +86,11 @@ WORKLOADS = {
     # 1M-token sequence through the 20-layer decoder stack
     "stack1m": Workload("stack1m", 1, 1_000_000, 512, 64, 32, SCALE_UE4M3, 128, 512, 128,
                         64, "bf16", _STACK20, 6, 10.0, 4),
+    # 1M-token sequence through the 18-layer encoder stack: 3 groups of one
+    # Full and five Reuse layers, each group with its own cache, groups of 16
+    # channels per scale
+    "encoder1m": Workload("encoder1m", 1, 1_000_000, 512, 64, 16, SCALE_UE4M3, 128, 512,
+                          128, 64, "bf16", _ENC6, 6, 10.0, 5, groups=3),
 }
 
 

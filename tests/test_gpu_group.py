@@ -70,3 +70,15 @@ def test_group_rejects_reuse_first(kvc):
                              torch.zeros(2, 1, 8, 64, device="cuda"),
                              torch.zeros(2, 1, 64, dtype=torch.int32, device="cuda"),
                              kvc.workspace(cfg, 1, 16))
+
+
+def test_encoder_groups_reduced(kvc):
+    """The encoder stack's layout ("DeepSeek V1 到 V4.1-Flash ..." part 4, CSA2):
+    3 groups of one Full and five Reuse layers, each group with its own cache
+    and inputs, groups of 16 channels per scale; every Reuse layer attends over
+    its group's Full selection."""
+    base = synth.WORKLOADS["encoder1m"]
+    assert base.groups == 3 and base.modes == (0, 2, 2, 2, 2, 2) and base.group == 16
+    for gi in range(base.groups):
+        w, tk = _group(kvc, base.scaled(seed=base.seed + 100 * gi), context=2 * 4000)
+        assert all(np.array_equal(tk[l], tk[0]) for l in range(1, w.layers))

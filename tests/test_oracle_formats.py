@@ -69,6 +69,29 @@ def test_group_counts_and_record_sizes(orc):
     assert [orc.record_bytes(c, True) for c in (c2, c3, c1)] == [320, 304, 64]
 
 
+def test_pages_entry_bytes_and_encoder_accounting(orc):
+    """The pages' estimate of the bytes a token occupies ("DeepSeek V1 到
+    V4.1-Flash ...", "890 字节是怎么算出来的"): an FP4 main-KV entry of 512
+    latent channels with one FP8 scale per 16 channels is 512 x 0.5 + 32 =
+    288 B, which is this format's record with no RoPE channels.  With the
+    RoPE channels the record holds 576 codes and 36 scales; the encoder's 3
+    caches (one per group, 2 tokens per entry) and the decoder's one cache
+    then hold (3 x 6-layer + 20-layer) bytes as below."""
+    page = orc.make_cfg(512, 0, 16, orc.SCALE_UE4M3, 128, 512, 128, 64, 1.0)
+    assert orc.record_bytes(page, False) == 512 // 2 + 512 // 16 == 288
+    enc = orc.make_cfg(512, 64, 16, orc.SCALE_UE4M3, 128, 512, 128, 64, 1.0)
+    assert orc.record_bytes(enc, False) == 576 // 2 + 576 // 16 == 324
+    dec = orc.make_cfg(512, 64, 32, orc.SCALE_UE4M3, 128, 512, 128, 64, 1.0)
+    entries = 500_000  # 1M tokens, 2 per entry
+    window = 128 * 576 * 2  # one bf16 window per layer
+    enc_b = orc.bytes_resident(enc, entries, 6, 2, padded=False)
+    dec_b = orc.bytes_resident(dec, entries, 20, 2, padded=False)
+    assert enc_b == entries * (324 + 128) + 6 * window
+    assert dec_b == entries * (306 + 128) + 20 * window
+    per_token = (3 * enc_b + dec_b) / 1_000_000
+    assert 900 < per_token < 901  # int8 indexer keys, RoPE channels included
+
+
 def test_bytes_resident_stack1m(orc):
     c = orc.make_cfg(512, 64, 32, orc.SCALE_UE4M3, 128, 512, 128, 64, 1.0)
     # 500,000 x 306 + 500,000 x 128 + 20 layers x 128 x 576 x 2
