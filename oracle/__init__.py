@@ -44,15 +44,17 @@ def build(force: bool = False) -> str:
 class Cfg(C.Structure):
     _fields_ = [("latent_dim", C.c_int), ("rope_dim", C.c_int), ("group", C.c_int),
                 ("scale_fmt", C.c_int), ("idx_dim", C.c_int), ("topk", C.c_int),
-                ("window", C.c_int), ("n_heads", C.c_int), ("sm_scale", C.c_double)]
+                ("window", C.c_int), ("n_heads", C.c_int), ("sm_scale", C.c_double),
+                ("ratio", C.c_int)]
 
 
 def make_cfg(latent_dim, rope_dim, group, scale_fmt, idx_dim, topk, window, n_heads,
-             sm_scale) -> Cfg:
-    if group <= 0 or latent_dim <= 0 or rope_dim < 0:
+             sm_scale, ratio=2) -> Cfg:
+    """ratio: raw tokens per entry, 2 or 4."""
+    if group <= 0 or latent_dim <= 0 or rope_dim < 0 or ratio not in (2, 4):
         raise ValueError("bad dims")
     return Cfg(latent_dim, rope_dim, group, scale_fmt, idx_dim, topk, window, n_heads,
-               float(sm_scale))
+               float(sm_scale), ratio)
 
 
 _lib = None
@@ -74,6 +76,8 @@ def lib():
             "orc_record_bytes": (C.c_int, [P, C.c_int]),
             "orc_gate_delta": (C.c_float, [P, P, P, C.c_int]),
             "orc_compress_pair": (None, [P, P, P, C.c_int, P]),
+            "orc_gate_logit": (C.c_float, [P, P, C.c_int]),
+            "orc_compress_group4": (None, [P, P, P, P, P, C.c_int, P]),
             "orc_quantize_entry": (C.c_int, [P, P, P]),
             "orc_dequantize_entry": (None, [P, P, P]),
             "orc_pack": (C.c_int, [P, C.c_int, C.c_int, P, P, P, C.c_int, P, P, P, P]),
@@ -158,6 +162,20 @@ def compress_pair(k0, k1, g) -> np.ndarray:
     k0, k1, g = _c(k0, np.float32), _c(k1, np.float32), _c(g, np.float32)
     e = np.empty_like(k0)
     lib().orc_compress_pair(_p(k0), _p(k1), _p(g), k0.size, _p(e))
+    return e
+
+
+def gate_logit(k, g) -> float:
+    k, g = _c(k, np.float32), _c(g, np.float32)
+    return lib().orc_gate_logit(_p(k), _p(g), k.size)
+
+
+def compress_group4(ks, g) -> np.ndarray:
+    """One entry from four tokens ks [4][D] (the 4:1 ratio)."""
+    ks = [_c(k, np.float32) for k in ks]
+    g = _c(g, np.float32)
+    e = np.empty_like(ks[0])
+    lib().orc_compress_group4(*[_p(k) for k in ks], _p(g), ks[0].size, _p(e))
     return e
 
 

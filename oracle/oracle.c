@@ -34,6 +34,10 @@
  *     decoded scale and rounded to nearest-even onto the E2M1 grid.
  *  R5 attention: one joint softmax over the selected entries and the window
  *     tokens; values are the first Dv (latent) channels of each key.
+ *  R6 4:1 compression ([P1] 4.3 lists a CSA2 compression ratio of 2x or 4x):
+ *     four consecutive tokens form one entry, weighted by the softmax of their
+ *     four gate logits, each logit summed in the order of R1; see
+ *     orc_compress_group4.
  *
  * Compile with -ffp-contract=off: every fused multiply-add below is an
  * explicit fma() call and nothing else may be contracted.
@@ -68,6 +72,7 @@ typedef struct {
     int window;      /* W                                                 */
     int n_heads;     /* H                                                 */
     double sm_scale; /* softmax scale applied to q.k                      */
+    int ratio;       /* raw tokens per entry: 2 (0 also means 2) or 4     */
 } orc_cfg;
 
 /* ------------------------------------------------------------------ */
@@ -275,6 +280,48 @@ void orc_compress_pair(const float* k0, const float* k1, const float* g, int D,
     for (int d = 0; d < D; ++d) e[d] = fmaf(w0, k0[d], w1 * k1[d]);
 }
 
+/* R6: the 4:1 compression of four consecutive tokens (the ratio 4 of [P1]
+ * 4.3; the pages give the 2:1 rule only, this is its plainest extension).
+ * logit_t = g . k_t, each summed like delta in R1: 8 partial sums over the
+ * 8-channel chunks (chunk c to partial c mod 8, chunks and channels in
+ * increasing order, one fmaf per term), combined by a xor tree over 4, 2, 1.
+ * M = max_t logit_t; e_t = exp(logit_t - M) (R2, fp32 subtraction first);
+ * S = ((e_0 + e_1) + e_2) + e_3; w_t = e_t / S;
+ * entry_d = fmaf(w0, k0_d, fmaf(w1, k1_d, fmaf(w2, k2_d, w3 * k3_d))). */
+float orc_gate_logit(const float* k, const float* g, int D) {
+    float acc[8];
+    for (int l = 0; l < 8; ++l) acc[l] = 0.0f;
+    for (int c = 0; c * 8 < D; ++c) {
+        int l = c % 8;
+        for (int t = 0; t < 8 && 8 * c + t < D; ++t) {
+            int d = 8 * c + t;
+            acc[l] = fmaf(g[d], k[d], acc[l]);
+        }
+    }
+    for (int off = 4; off >= 1; off >>= 1) {
+        float nxt[8];
+        for (int l = 0; l < 8; ++l) nxt[l] = acc[l] + acc[l ^ off];
+        memcpy(acc, nxt, sizeof acc);
+    }
+    return acc[0];
+}
+
+void orc_compress_group4(const float* k0, const float* k1, const float* k2, const float* k3,
+                         const float* g, int D, float* e) {
+    const float* k[4] = {k0, k1, k2, k3};
+    float lg[4], ex[4], w[4];
+    float m = -INFINITY;
+    for (int t = 0; t < 4; ++t) {
+        lg[t] = orc_gate_logit(k[t], g, D);
+        if (lg[t] > m) m = lg[t];
+    }
+    for (int t = 0; t < 4; ++t) ex[t] = orc_expf(lg[t] - m);
+    float sum = ((ex[0] + ex[1]) + ex[2]) + ex[3];
+    for (int t = 0; t < 4; ++t) w[t] = ex[t] / sum;
+    for (int d = 0; d < D; ++d)
+        e[d] = fmaf(w[0], k0[d], fmaf(w[1], k1[d], fmaf(w[2], k2[d], w[3] * k3[d])));
+}
+
 /* ------------------------------------------------------------------ */
 /* R4: FP4 group quantisation of one entry into one record ([P1] 3.1;
  * [P2] "P4 main KV").  Returns the number of non-finite inputs, which are
@@ -333,34 +380,38 @@ void orc_dequantize_entry(const orc_cfg* c, const uint8_t* rec, float* x) {
 }
 
 /* ------------------------------------------------------------------ */
-/* Pack: append n_new/2 compressed entries per sequence, with their
- * indexer keys, at position n_entries[b]; then advance n_entries[b].
- * tokens [B][n_new][D] fp32 (bf16 inputs widened exactly by the caller),
- * idxk_new [B][n_new/2][Di], records [B][cap][record_bytes(padded)],
- * idx_cache [B][cap][Di].                                               */
+/* Pack: append n_new/r compressed entries per sequence (r = the ratio, 2
+ * or 4), with their indexer keys, at position n_entries[b]; then advance
+ * n_entries[b].  tokens [B][n_new][D] fp32 (bf16 inputs widened exactly by
+ * the caller), idxk_new [B][n_new/r][Di], records [B][cap][record_bytes
+ * (padded)], idx_cache [B][cap][Di].                                     */
 int orc_pack(const orc_cfg* c, int B, int n_new, const float* tokens,
              const float* g, const int8_t* idxk_new, int cap, uint8_t* records,
              int8_t* idx_cache, int32_t* n_entries, uint32_t* status) {
     int D = c->latent_dim + c->rope_dim;
     int rb = orc_record_bytes(c, 1);
-    int half = n_new / 2;
-    if (n_new < 0 || (n_new & 1)) return ORC_ERR_INVALID;
+    int r = c->ratio == 0 ? 2 : c->ratio;
+    if (r != 2 && r != 4) return ORC_ERR_INVALID;
+    if (n_new < 0 || n_new % r) return ORC_ERR_INVALID;
+    int per = n_new / r;
     for (int b = 0; b < B; ++b)
-        if (n_entries[b] < 0 || n_entries[b] + half > cap) return ORC_ERR_CAPACITY;
+        if (n_entries[b] < 0 || n_entries[b] + per > cap) return ORC_ERR_CAPACITY;
     float* e = (float*)malloc(sizeof(float) * (size_t)D);
     for (int b = 0; b < B; ++b) {
-        for (int i = 0; i < half; ++i) {
-            const float* k0 = tokens + ((size_t)b * n_new + 2 * i) * D;
-            const float* k1 = k0 + D;
+        for (int i = 0; i < per; ++i) {
+            const float* k0 = tokens + ((size_t)b * n_new + (size_t)r * i) * D;
             int64_t pos = n_entries[b] + i;
-            orc_compress_pair(k0, k1, g, D, e);
+            if (r == 2)
+                orc_compress_pair(k0, k0 + D, g, D, e);
+            else
+                orc_compress_group4(k0, k0 + D, k0 + 2 * D, k0 + 3 * D, g, D, e);
             if (orc_quantize_entry(c, e, records + ((size_t)b * cap + pos) * rb))
                 *status |= ORC_ST_NONFINITE;
             memcpy(idx_cache + ((size_t)b * cap + pos) * c->idx_dim,
-                   idxk_new + ((size_t)b * half + i) * c->idx_dim,
+                   idxk_new + ((size_t)b * per + i) * c->idx_dim,
                    (size_t)c->idx_dim);
         }
-        n_entries[b] += half;
+        n_entries[b] += per;
     }
     free(e);
     return ORC_OK;
