@@ -28,6 +28,7 @@ bool derive_shape(const kvc_config* c, Shape* s) {
     if (c->n_heads < 1 || c->n_heads > 256) return false;
     if (!(c->sm_scale > 0.f) || !(c->sm_scale < 1e30f)) return false;
     if (c->act_dtype != KVC_F32 && c->act_dtype != KVC_BF16) return false;
+    if (c->ratio != 0 && c->ratio != 2 && c->ratio != 4) return false;
     s->D = D;
     s->Dv = c->latent_dim;
     s->G = G;
@@ -362,9 +363,10 @@ kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new, const 
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     kvc_status st = check_cache(cache, sh);
     if (st != KVC_OK) return st;
-    if (n_new < 0 || (n_new & 1)) return KVC_ERR_INVALID;
+    const int r = cfg->ratio == 4 ? 4 : 2;
+    if (n_new < 0 || n_new % r) return KVC_ERR_INVALID;
     if (n_new == 0 || cache->batch == 0) return KVC_OK;
-    if (n_new / 2 > cache->capacity) return KVC_ERR_CAPACITY;
+    if (n_new / r > cache->capacity) return KVC_ERR_CAPACITY;
     if (!tokens || !gate || !idx_k_new) return KVC_ERR_INVALID;
     if (!aligned(tokens, 16) || !aligned(gate, 16) || !aligned(idx_k_new, 16)) return KVC_ERR_INVALID;
     if (!device_ok()) return KVC_ERR_DEVICE;

@@ -554,6 +554,166 @@ pack_small_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     if (half == 1 && lane == 0) a.n_entries[b] = base + 1;
 }
 
+// 4:1 compression (the ratio 4 of [B] 4.3): four consecutive tokens form one
+// entry, weighted by the softmax of their four gate logits.  One warp per
+// entry, as for the decode append: the warp stages the four tokens and the
+// gate in shared memory (one round trip), lanes 0-7 form the four logits
+// each in the order of the pair's gate (lane l sums chunks l, l+8, ... then
+// the xor tree over 4, 2, 1), every lane takes the weights
+// (w_t = exp(logit_t - max) / S, S summed left to right) and quantises its
+// chunks from registers: entry = fma(w0, k0, fma(w1, k1, fma(w2, k2, w3 k3))).
+// The entry is formed before the wait for the previous kernel, as in the
+// decode append; one entry per sequence also commits the new length.
+template <typename T>
+__host__ __device__ constexpr size_t group4_stage_bytes(int D) {
+    return (size_t)D * (4 * sizeof(T) + sizeof(float));  // k0..k3, gate
+}
+
+template <typename T, int MAXJ>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+pack_group4_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
+    extern __shared__ __align__(16) unsigned char stage_smem[];
+    __shared__ __align__(16) uint8_t tail_smem[kSmallWarps][kTailBytes];
+    pdl_trigger();  // a short kernel: the next one may be scheduled at once
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const long long e = (long long)blockIdx.x * kSmallWarps + wid;
+    const int per = a.n_new >> 2;
+    if (e >= (long long)a.batch * per) return;  // whole warp
+    const int b = (int)(e / per), i = (int)(e % per);
+    const int D = sh.D, nchunk = D >> 3;
+    const T* kp = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 4 * i) * D;
+    T* st = reinterpret_cast<T*>(stage_smem + wid * group4_stage_bytes<T>(D));  // [4][D]
+    float* sg = reinterpret_cast<float*>(st + 4 * D);
+
+    uint4 ik = make_uint4(0, 0, 0, 0);
+    if (lane < (di >> 4))
+        ik = __ldcs(reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * per + i) * di) +
+                    lane);
+    Chunk<T> x[4][MAXJ];
+    float4 g0[MAXJ], g1[MAXJ];
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nchunk) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) x[t][j].load(kp + (long long)t * D + 8 * c);
+            g0[j] = __ldg(reinterpret_cast<const float4*>(a.gate + 8 * c));
+            g1[j] = __ldg(reinterpret_cast<const float4*>(a.gate + 8 * c) + 1);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) x[t][j].zero();
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nchunk) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) x[t][j].store_shared(st + t * D + 8 * c);
+            reinterpret_cast<float4*>(sg + 8 * c)[0] = g0[j];
+            reinterpret_cast<float4*>(sg + 8 * c)[1] = g1[j];
+        }
+    }
+    __syncwarp();
+
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (lane < 8) {
+        for (int c = lane; c < nchunk; c += 8) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                Chunk<T> y;
+                y.load_shared(st + t * D + 8 * c);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[t] = __fmaf_rn(sg[8 * c + u], y.get(u), acc[t]);
+            }
+        }
+    }
+    float lg[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float v = acc[t];
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 2));
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 1));
+        lg[t] = __shfl_sync(0xffffffffu, v, 0);
+    }
+    const float mx = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+    float ex[4], w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) ex[t] = exp_cody_waite(__fsub_rn(lg[t], mx));
+    const float sum = __fadd_rn(__fadd_rn(__fadd_rn(ex[0], ex[1]), ex[2]), ex[3]);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) w[t] = __fdiv_rn(ex[t], sum);
+
+    uint8_t* tail = tail_smem[wid];
+    const int tail_len = sh.rb - sh.code_bytes;
+    for (int t = lane * 4; t < tail_len; t += 128) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
+    __syncwarp();
+
+    bool bad = false;
+    const int lpg = sh.lpg;
+    uint32_t code[MAXJ];
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        const bool active = c < nchunk;
+        float xv[8];
+        float m = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float v = __fmaf_rn(w[0], x[0][j].get(u),
+                                __fmaf_rn(w[1], x[1][j].get(u),
+                                          __fmaf_rn(w[2], x[2][j].get(u),
+                                                    __fmul_rn(w[3], x[3][j].get(u)))));
+            if (!isfinite(v)) {
+                if (active) bad = true;
+                v = 0.f;
+            }
+            xv[u] = v;
+            m = fmaxf(m, fabsf(v));
+        }
+        for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        code[j] = 0u;
+        if (!active) continue;
+        float sc = __fdiv_rn(m, 6.0f);
+        uint32_t sbyte = 0;
+        if (ue4m3) {
+            sbyte = e4m3_from_f32(sc);
+            sc = e4m3_to_f32(sbyte);
+        }
+        code[j] = sc > 0.f ? e2m1x8_quotient(xv, sc) : 0u;
+        if (c % lpg == 0) {
+            const int gi = c / lpg;
+            if (ue4m3)
+                tail[gi] = (uint8_t)sbyte;
+            else
+                *reinterpret_cast<float*>(tail + 4 * gi) = sc;
+        }
+    }
+    __syncwarp();
+
+    pdl_wait();  // the previous kernel is done: the length and the cache
+    const int base = a.n_entries[b];
+    if (base < 0 || base + per > a.capacity) {
+        if (i == 0 && lane == 0) set_status(a.status, KVC_DEV_CAPACITY);
+        return;
+    }
+    const long long pos = (long long)base + i;
+    uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int c = lane + 32 * j;
+        if (c < nchunk) *reinterpret_cast<uint32_t*>(rec + 4 * c) = code[j];
+    }
+    for (int t = lane * 4; t < tail_len; t += 128)
+        *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
+            *reinterpret_cast<const uint32_t*>(tail + t);
+    if (lane < (di >> 4))
+        *(reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di) + lane) = ik;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
+    if (per == 1 && lane == 0) a.n_entries[b] = base + 1;
+}
+
 __global__ void pack_commit_kernel(int32_t* n_entries, int batch, int half, int capacity) {
     pdl_wait();
     for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
@@ -572,6 +732,40 @@ cudaError_t launch_small(unsigned grid, size_t smem, cudaStream_t s, const PackA
     }
     return launch_pdl(pack_small_kernel<T, MAXJ>, grid, kSmallWarps * 32, smem, s, a, sh, ue4m3,
                       di);
+}
+
+template <typename T, int MAXJ>
+cudaError_t launch_group4(unsigned grid, size_t smem, cudaStream_t s, const PackArgs& a,
+                          const Shape& sh, int ue4m3, int di) {
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            pack_group4_kernel<T, MAXJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(pack_group4_kernel<T, MAXJ>, grid, kSmallWarps * 32, smem, s, a, sh, ue4m3,
+                      di);
+}
+
+// 4:1 appends: a warp per entry at every size
+template <typename T>
+cudaError_t launch_pack4_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
+                           cudaStream_t s) {
+    const long long entries = (long long)a.batch * (a.n_new / 4);
+    const unsigned grid = (unsigned)((entries + kSmallWarps - 1) / kSmallWarps);
+    const int maxj = (sh.D / 8 + 31) / 32;
+    const size_t smem = kSmallWarps * group4_stage_bytes<T>(sh.D);
+    trace_before("pack", s);
+    cudaError_t err;
+    if (maxj <= 1)
+        err = launch_group4<T, 1>(grid, smem, s, a, sh, ue4m3, di);
+    else if (maxj <= 2)
+        err = launch_group4<T, 2>(grid, smem, s, a, sh, ue4m3, di);
+    else if (maxj <= 3)
+        err = launch_group4<T, 3>(grid, smem, s, a, sh, ue4m3, di);
+    else
+        err = launch_group4<T, 4>(grid, smem, s, a, sh, ue4m3, di);
+    trace_after(s);
+    return err;
 }
 
 template <typename T>
@@ -719,14 +913,20 @@ cudaError_t launch_window_t(const void* rows, long long n, int D, uint8_t* codes
 
 cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
                         cudaStream_t s) {
-    const int half = a.n_new / 2;
+    const bool four = c.ratio == 4;
+    const int half = a.n_new / (four ? 4 : 2);  // entries per sequence
     if (half == 0 || a.batch == 0) return cudaSuccess;
     const int ue = c.scale_fmt == KVC_SCALE_UE4M3;
-    cudaError_t err = c.act_dtype == KVC_BF16
-                          ? launch_pack_t<__nv_bfloat16>(sh, a, ue, c.idx_dim, s)
-                          : launch_pack_t<float>(sh, a, ue, c.idx_dim, s);
+    cudaError_t err;
+    if (four)
+        err = c.act_dtype == KVC_BF16 ? launch_pack4_t<__nv_bfloat16>(sh, a, ue, c.idx_dim, s)
+                                      : launch_pack4_t<float>(sh, a, ue, c.idx_dim, s);
+    else
+        err = c.act_dtype == KVC_BF16 ? launch_pack_t<__nv_bfloat16>(sh, a, ue, c.idx_dim, s)
+                                      : launch_pack_t<float>(sh, a, ue, c.idx_dim, s);
     if (err != cudaSuccess) return err;
-    if (half == 1 && a.batch <= 4096) return cudaSuccess;  // committed by the append kernel
+    // one entry per sequence: committed by the append kernel
+    if (half == 1 && (four || a.batch <= 4096)) return cudaSuccess;
     trace_before("pack_commit", s);
     err = launch_pdl(pack_commit_kernel, (a.batch + 255) / 256, 256, 0, s, a.n_entries, a.batch,
                      half, a.capacity);

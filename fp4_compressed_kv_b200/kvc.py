@@ -34,7 +34,7 @@ class Config(C.Structure):
     _fields_ = [("latent_dim", C.c_int32), ("rope_dim", C.c_int32), ("group", C.c_int32),
                 ("scale_fmt", C.c_int32), ("idx_dim", C.c_int32), ("topk", C.c_int32),
                 ("window", C.c_int32), ("n_heads", C.c_int32), ("sm_scale", C.c_float),
-                ("act_dtype", C.c_int32)]
+                ("act_dtype", C.c_int32), ("ratio", C.c_int32)]
 
 
 class CacheStruct(C.Structure):
@@ -113,15 +113,16 @@ def _stream(stream):
 
 
 def make_config(latent_dim, rope_dim, group, scale_fmt, idx_dim, topk, window, n_heads, sm_scale,
-                act_dtype) -> Config:
+                act_dtype, ratio=2) -> Config:
+    """ratio: raw tokens per entry, 2 or 4."""
     return Config(latent_dim, rope_dim, group, scale_fmt, idx_dim, topk, window, n_heads,
-                  float(sm_scale), act_dtype)
+                  float(sm_scale), act_dtype, ratio)
 
 
 def config_for(w) -> Config:
     """kvc_config of a synth.Workload."""
     return make_config(w.latent, w.rope, w.group, w.scale_fmt, w.idx_dim, w.topk, w.window,
-                       w.heads, w.sm_scale, F32 if w.act == "f32" else BF16)
+                       w.heads, w.sm_scale, F32 if w.act == "f32" else BF16, w.ratio)
 
 
 def record_bytes(cfg: Config) -> int:

@@ -41,6 +41,7 @@ class Workload:
     seed: int
     pack_new: int = 0     # new raw tokens per sequence for the pack benchmark
     groups: int = 1       # independent layer groups, each with its own cache and `modes`
+    ratio: int = 2        # raw tokens per entry (2 or 4)
 
     @property
     def dim(self) -> int:
@@ -48,7 +49,7 @@ class Workload:
 
     @property
     def entries(self) -> int:
-        return self.context // 2
+        return self.context // self.ratio
 
     @property
     def layers(self) -> int:
@@ -117,7 +118,7 @@ def make_inputs(w: Workload, device="cpu", *, with_tokens: bool = True) -> dict:
 
     tokens   [B][T][D]     raw keys of the context (compressed 2:1 into the cache)
     gate     [D]  fp32     compression gate, N(0, 1/D)
-    idx_k    [B][N][Di]    int8 indexer keys of the N = T/2 entries, U[-127, 127]
+    idx_k    [B][N][Di]    int8 indexer keys of the N = T/ratio entries, U[-127, 127]
     idx_q    [L][B][Di]    int8 indexer queries, one per layer
     q        [L][B][H][D]  query heads (already absorbed into the latent space)
     windows  [L][B][W][D]  per-layer sliding-window keys; layer 0 holds the last
@@ -146,6 +147,6 @@ def make_new_tokens(w: Workload, n_new: int, device="cpu", seed_offset: int = 7)
     """Fresh raw tokens (and their indexer keys) to append with pack."""
     gen = generator(device, w.seed * 1000 + seed_offset)
     tokens = _keys(w, (w.batch, n_new), gen, device)
-    idx_k = torch.randint(-127, 128, (w.batch, n_new // 2, w.idx_dim), generator=gen,
+    idx_k = torch.randint(-127, 128, (w.batch, n_new // w.ratio, w.idx_dim), generator=gen,
                           device=device, dtype=torch.int8)
     return {"tokens": tokens, "idx_k": idx_k}

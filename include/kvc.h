@@ -88,6 +88,7 @@ typedef struct {
     int32_t idx_dim, topk, window, n_heads;
     float sm_scale;
     int32_t act_dtype;
+    int32_t ratio;  /* raw tokens per entry: 2 (0 also means 2) or 4 */
 } kvc_config;
 
 /* One stored cache (the Full layer's).  Caller-owned device buffers:
@@ -126,15 +127,16 @@ size_t kvc_bytes_resident(const kvc_config* cfg, int64_t entries, int n_layers,
 size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity);
 
 /* Append n_new raw tokens per sequence (A1-A3 of the hot path).
- * tokens    [batch][n_new][D] act_dtype; n_new even: token pairs (2i, 2i+1) are
- *           compressed into one entry ([A] breakthrough 4 "CSA 把每 2 个 token
- *           的 KV 压成 1 条"; [B] 3.2).  The pair's weights are the softmax of
- *           the two gate logits g.k; the weighted sum is quantised per group
- *           to E2M1 with scale absmax/6 ([B] 3.1; [A] "P4 main KV").
+ * tokens    [batch][n_new][D] act_dtype; n_new a multiple of r = cfg->ratio:
+ *           tokens r i .. r i + r - 1 are compressed into entry i ([A]
+ *           breakthrough 4 "CSA 把每 2 个 token 的 KV 压成 1 条"; [B] 3.2; the
+ *           ratio 4 of [B] 4.3).  The tokens' weights are the softmax of their
+ *           gate logits g.k; the weighted sum is quantised per group to E2M1
+ *           with scale absmax/6 ([B] 3.1; [A] "P4 main KV").
  * gate      [D] fp32 gate vector g.
- * idx_k_new [batch][n_new/2][idx_dim] int8 indexer keys of the new entries.
- * Entries are written at positions n_entries[b] .. n_entries[b]+n_new/2-1 and
- * n_entries[b] then advances by n_new/2.  If that would pass the capacity the
+ * idx_k_new [batch][n_new/r][idx_dim] int8 indexer keys of the new entries.
+ * Entries are written at positions n_entries[b] .. n_entries[b]+n_new/r-1 and
+ * n_entries[b] then advances by n_new/r.  If that would pass the capacity the
  * sequence is left unchanged and KVC_DEV_CAPACITY is set.  NaN/Inf channels are
  * coded 0, left out of the group maximum, and set KVC_DEV_NONFINITE.         */
 kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,

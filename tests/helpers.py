@@ -14,7 +14,7 @@ ATTN_RTOL = 2e-3
 
 def oracle_cfg(w: synth.Workload) -> oracle.Cfg:
     return oracle.make_cfg(w.latent, w.rope, w.group, w.scale_fmt, w.idx_dim, w.topk, w.window,
-                           w.heads, w.sm_scale)
+                           w.heads, w.sm_scale, w.ratio)
 
 
 def f32(t: torch.Tensor) -> np.ndarray:
@@ -26,7 +26,7 @@ def oracle_pack(w: synth.Workload, tokens, gate, idx_k, capacity=None):
     """Oracle cache of the raw tokens: (records, idx_cache, n_entries, status)."""
     cfg = oracle_cfg(w)
     B, T = tokens.shape[0], tokens.shape[1]
-    cap = capacity or T // 2
+    cap = capacity or T // w.ratio
     rec = np.zeros((B, cap, oracle.record_bytes(cfg)), np.uint8)
     ic = np.zeros((B, cap, w.idx_dim), np.int8)
     n = np.zeros(B, np.int32)

@@ -44,7 +44,7 @@ def test_sizes_match_oracle(lib, orc):
     for name, w in synth.WORKLOADS.items():
         cfg = lib.config_for(w)
         ocfg = orc.make_cfg(w.latent, w.rope, w.group, w.scale_fmt, w.idx_dim, w.topk, w.window,
-                            w.heads, w.sm_scale)
+                            w.heads, w.sm_scale, w.ratio)
         assert lib.record_bytes(cfg) == orc.record_bytes(ocfg, True), name
         for padded in (False, True):
             assert lib.bytes_resident(cfg, w.entries, w.layers, padded) == \
@@ -58,7 +58,7 @@ def test_invalid_configs_rejected(lib):
     base = synth.WORKLOADS["mla32k"]
     for field, value in [("group", 48), ("group", 1024), ("latent_dim", 500), ("idx_dim", 100),
                          ("topk", 0), ("topk", 5000), ("scale_fmt", 3), ("act_dtype", 7),
-                         ("sm_scale", 0.0), ("n_heads", 0)]:
+                         ("sm_scale", 0.0), ("n_heads", 0), ("ratio", 3), ("ratio", 8)]:
         cfg = lib.config_for(base)
         setattr(cfg, field, value)
         assert lib.record_bytes(cfg) == 0, field
@@ -71,6 +71,11 @@ def test_host_validation_before_device(lib):
     cache = lib.CacheStruct(16, 16, 16, 1, 8)  # fake aligned addresses: never dereferenced
     # odd n_new is invalid whatever the device
     assert so.kvc_pack(C.byref(cfg), C.c_void_p(16), 3, C.c_void_p(16), C.c_void_p(16),
+                       C.byref(cache), None, None) == 1
+    # at the 4:1 ratio n_new must be a multiple of 4
+    cfg4 = lib.config_for(synth.WORKLOADS["tiny"].scaled(ratio=4))
+    assert lib.record_bytes(cfg4) == lib.record_bytes(cfg)
+    assert so.kvc_pack(C.byref(cfg4), C.c_void_p(16), 6, C.c_void_p(16), C.c_void_p(16),
                        C.byref(cache), None, None) == 1
     # misaligned tokens
     assert so.kvc_pack(C.byref(cfg), C.c_void_p(17), 2, C.c_void_p(16), C.c_void_p(16),
