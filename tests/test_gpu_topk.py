@@ -161,14 +161,15 @@ def _rows_with_sums(sums, di=128):
     return torch.from_numpy(rows.astype(np.int8))
 
 
-@pytest.mark.parametrize("ties", [100, 1000, 6000])
+@pytest.mark.parametrize("ties", [100, 128, 129, 1000, 4096, 4097, 6000])
 @pytest.mark.parametrize("cap", [20000, 9 * 8192, 9 * 16384])
 def test_topk_tie_counts(kvc, ties, cap):
     """A chosen number of entries in the threshold bin, spread over every
-    tile: up to 128 (one warp sorts them), up to 4096 (a block sorts them),
-    more (the second-histogram pass).  A capacity of at most 8 tiles of
-    8,192 or of 16,384 scores selects inside one cluster per sequence, a
-    larger one through the sequence's last tile CTA."""
+    tile, on both sides of each path's limit: up to 128 (every CTA ranks
+    them), up to 4096 (a block sorts them), more (the second-histogram
+    pass).  A capacity of at most 8 tiles of 8,192 or of 16,384 scores
+    selects inside one cluster per sequence, a larger one through the
+    sequence's last tile CTA."""
     w = synth.WORKLOADS["mla32k"].scaled(context=2 * 20000)
     N, K = 20000, w.topk
     rng = np.random.default_rng(ties)
