@@ -202,22 +202,27 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
             break;
         }
         phase ^= 1u << s;
+        // rows of up to 128 bytes: this thread's row into registers, and the
+        // stage goes back to the producer before the dot product is formed
+        // (wider rows keep the products between the loads and the release)
+        constexpr int HELD = PIECES <= 8 ? PIECES : 1;
+        int4 kv[HELD];
+        int acc[4] = {0, 0, 0, 0};
         if (tid < rows) {
             const unsigned char* row = ring + s * STAGE + tid * DI;
-            int acc[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int c = 0; c < PIECES; ++c) {
-                const int p = (c + tid) % PIECES;
-                const int4 kv = *reinterpret_cast<const int4*>(row + p * 16);
-                const int4 q = qs[p];
-                acc[c & 3] = __dp4a(kv.x, q.x, acc[c & 3]);
-                acc[c & 3] = __dp4a(kv.y, q.y, acc[c & 3]);
-                acc[c & 3] = __dp4a(kv.z, q.z, acc[c & 3]);
-                acc[c & 3] = __dp4a(kv.w, q.w, acc[c & 3]);
+                const int4 x = *reinterpret_cast<const int4*>(row + ((c + tid) % PIECES) * 16);
+                if constexpr (PIECES <= 8) {
+                    kv[c] = x;
+                } else {
+                    const int4 q = qs[(c + tid) % PIECES];
+                    acc[c & 3] = __dp4a(x.x, q.x, acc[c & 3]);
+                    acc[c & 3] = __dp4a(x.y, q.y, acc[c & 3]);
+                    acc[c & 3] = __dp4a(x.z, q.z, acc[c & 3]);
+                    acc[c & 3] = __dp4a(x.w, q.w, acc[c & 3]);
+                }
             }
-            const int v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-            a.scores[(size_t)cc.b * cap + cc.row + tid] = v;
-            atomicAdd(&hist[score_bin(v, bias, shift)], 1);
         }
         __syncthreads();  // stage s is free again
         if (tid < 32 && pmore) {
@@ -227,9 +232,25 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
             pc.row += prow;
             if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
         }
+        if (tid < rows) {
+            if constexpr (PIECES <= 8) {
+#pragma unroll
+                for (int c = 0; c < PIECES; ++c) {
+                    const int4 q = qs[(c + tid) % PIECES];
+                    acc[c & 3] = __dp4a(kv[c].x, q.x, acc[c & 3]);
+                    acc[c & 3] = __dp4a(kv[c].y, q.y, acc[c & 3]);
+                    acc[c & 3] = __dp4a(kv[c].z, q.z, acc[c & 3]);
+                    acc[c & 3] = __dp4a(kv[c].w, q.w, acc[c & 3]);
+                }
+            }
+            const int v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            a.scores[(size_t)cc.b * cap + cc.row + tid] = v;
+            atomicAdd(&hist[score_bin(v, bias, shift)], 1);
+        }
         cc.row += rows;
         if (cc.row < cc.end) continue;
         // ---- sequence cc.b done in this CTA: flush, maybe derive its threshold
+        __syncthreads();  // every count of the last stage is in the histogram
         const int b = cc.b;
         const int n = a.n_entries[b];
         int32_t* gh = a.counters + (size_t)b * kBins;
