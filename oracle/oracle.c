@@ -39,6 +39,14 @@
  *     four gate logits, each logit summed in the order of R1; see
  *     orc_compress_group4.
  *
+ * Pins: every function is checked by the not-gpu tests against what the
+ * pages or the mathematics fix (printed values, closed forms, brute force,
+ * library routines).  orc_compress_pair and orc_compress_group4 are pinned
+ * only by invariants (identical tokens, zero gate, a dominant token,
+ * convexity, fp64 softmax weights); their exact fp32 operation order is a
+ * reading (R1, R6), so beyond those invariants they are "parity unpinned"
+ * by the pages, and the GPU is held to them by following the same order.
+ *
  * Compile with -ffp-contract=off: every fused multiply-add below is an
  * explicit fma() call and nothing else may be contracted.
  */
