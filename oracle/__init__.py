@@ -77,6 +77,9 @@ def lib():
             "orc_gate_delta": (C.c_float, [P, P, P, C.c_int]),
             "orc_compress_pair": (None, [P, P, P, C.c_int, P]),
             "orc_gate_logit": (C.c_float, [P, P, C.c_int]),
+            "orc_idx_fp4_score": (C.c_int64, [P, P, C.c_int]),
+            "orc_topk64": (C.c_int, [P, C.c_int, C.c_int, P]),
+            "orc_index_topk_fp4": (C.c_int, [P, C.c_int, P, P, C.c_int, P, P, P]),
             "orc_compress_group4": (None, [P, P, P, P, P, C.c_int, P]),
             "orc_quantize_entry": (C.c_int, [P, P, P]),
             "orc_dequantize_entry": (None, [P, P, P]),
@@ -236,6 +239,51 @@ def index_topk(cfg: Cfg, idx_q, idx_cache, n_entries, want_scores=False):
                               _p(tk), _p(sc) if sc is not None else None)
     if rc:
         raise ValueError(f"orc_index_topk failed: {rc}")
+    return (tk, sc) if want_scores else tk
+
+
+def idx_fp4_cfg(cfg: Cfg) -> Cfg:
+    """The quantisation configuration of FP4 indexer keys (R18): Di channels,
+    no RoPE, groups of 16, UE4M3 scales."""
+    return make_cfg(cfg.idx_dim, 0, 16, SCALE_UE4M3, cfg.idx_dim, cfg.topk, cfg.window,
+                    cfg.n_heads, cfg.sm_scale)
+
+
+def idx_fp4_quantize(cfg: Cfg, keys) -> np.ndarray:
+    """FP4 indexer rows [n][Di/2 + Di/16] of float keys [n][Di]."""
+    keys = _c(keys, np.float32)
+    qc = idx_fp4_cfg(cfg)
+    rb = record_bytes(qc, False)
+    out = np.empty((keys.shape[0], rb), np.uint8)
+    for j in range(keys.shape[0]):
+        out[j] = quantize_entry(qc, keys[j])[0][:rb]
+    return out
+
+
+def idx_fp4_score(q, row, di) -> int:
+    """Exact score times 2^10 of int8 query q against one FP4 indexer row."""
+    q, row = _c(q, np.int8), _c(row, np.uint8)
+    return int(lib().orc_idx_fp4_score(_p(q), _p(row), int(di)))
+
+
+def topk64(scores, k) -> np.ndarray:
+    scores = _c(scores, np.int64)
+    out = np.empty(k, np.int32)
+    lib().orc_topk64(_p(scores), scores.size, k, _p(out))
+    return out
+
+
+def index_topk_fp4(cfg: Cfg, idx_q, keys, n_entries, want_scores=False):
+    """Top-K over FP4 indexer rows keys [B][cap][Di/2 + Di/16]."""
+    idx_q, keys = _c(idx_q, np.int8), _c(keys, np.uint8)
+    n_entries = _c(n_entries, np.int32)
+    B, cap, _ = keys.shape
+    tk = np.empty((B, cfg.topk), np.int32)
+    sc = np.zeros((B, cap), np.int64) if want_scores else None
+    rc = lib().orc_index_topk_fp4(C.byref(cfg), B, _p(idx_q), _p(keys), cap, _p(n_entries),
+                                  _p(tk), _p(sc) if sc is not None else None)
+    if rc:
+        raise ValueError(f"orc_index_topk_fp4 failed: {rc}")
     return (tk, sc) if want_scores else tk
 
 

@@ -34,6 +34,9 @@
  *     decoded scale and rounded to nearest-even onto the E2M1 grid.
  *  R5 attention: one joint softmax over the selected entries and the window
  *     tokens; values are the first Dv (latent) channels of each key.
+ *  R18 FP4 indexer keys: quantised like a main-KV entry (no RoPE, groups of
+ *     16, UE4M3), scored exactly against the int8 query (see
+ *     orc_idx_fp4_score).
  *  R6 4:1 compression ([P1] 4.3 lists a CSA2 compression ratio of 2x or 4x):
  *     four consecutive tokens form one entry, weighted by the softmax of their
  *     four gate logits, each logit summed in the order of R1; see
@@ -489,6 +492,84 @@ int orc_index_topk(const orc_cfg* c, int B, const int8_t* idx_q,
                          idx_cache + (size_t)b * cap * c->idx_dim, n, c->idx_dim, s);
         if (scores_out) memcpy(scores_out + (size_t)b * cap, s, sizeof(int32_t) * (size_t)n);
         orc_topk(s, n, c->topk, topk + (size_t)b * c->topk);
+    }
+    free(s);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* R18: FP4 indexer keys ([P2] "890 字节是怎么算出来的": an FP4 indexer K is
+ * 128 dims x 0.5 B plus 8 scales = 72 B).  A key row is quantised exactly
+ * like a main-KV entry of Di latent channels, no RoPE channels, groups of 16
+ * and UE4M3 scales (orc_quantize_entry with that configuration): Di/2 code
+ * bytes, then Di/16 scale bytes.  Its score against the int8 query is the
+ * exact value of q . dequant(k): per group, the integer sum of q_d times
+ * twice the E2M1 value (an integer in -12..12), times the scale times 2^9
+ * (an integer: every UE4M3 value is a multiple of 2^-9), summed over the
+ * groups -- the score times 2^10, exact in int64 (|.| < 2^36 for Di = 128),
+ * so the top-K over these scores is as exact as over int8 keys.          */
+int64_t orc_idx_fp4_score(const int8_t* q, const uint8_t* rec, int di) {
+    int64_t total = 0;
+    for (int g = 0; g < di / 16; ++g) {
+        int64_t part = 0;
+        for (int d = 16 * g; d < 16 * g + 16; ++d) {
+            int code = (d & 1) ? (rec[d / 2] >> 4) : (rec[d / 2] & 15);
+            int twice = (int)lrint(2.0 * (double)orc_e2m1_value(code));  /* exact */
+            part += (int64_t)q[d] * twice;
+        }
+        int64_t s9 = (int64_t)llrint((double)orc_e4m3_value(rec[di / 2 + g]) * 512.0);
+        total += part * s9;
+    }
+    return total;
+}
+
+/* Top-K over int64 scores, (score descending, index ascending); the same
+ * output form as orc_topk.                                               */
+typedef struct {
+    int64_t score;
+    int32_t idx;
+} orc_scored64;
+
+static int orc_by_score64_desc_idx_asc(const void* pa, const void* pb) {
+    const orc_scored64* a = (const orc_scored64*)pa;
+    const orc_scored64* b = (const orc_scored64*)pb;
+    if (a->score != b->score) return (a->score > b->score) ? -1 : 1;
+    return (a->idx < b->idx) ? -1 : (a->idx > b->idx);
+}
+
+int orc_topk64(const int64_t* scores, int n, int k, int32_t* out) {
+    orc_scored64* v = (orc_scored64*)malloc(sizeof(orc_scored64) * (size_t)(n > 0 ? n : 1));
+    for (int j = 0; j < n; ++j) {
+        v[j].score = scores[j];
+        v[j].idx = j;
+    }
+    qsort(v, (size_t)n, sizeof(orc_scored64), orc_by_score64_desc_idx_asc);
+    int kept = n < k ? n : k;
+    for (int i = 0; i < kept; ++i) out[i] = v[i].idx;
+    qsort(out, (size_t)kept, sizeof(int32_t), orc_int_asc);
+    for (int i = kept; i < k; ++i) out[i] = -1;
+    free(v);
+    return kept;
+}
+
+/* Indexer top-K over FP4 keys: idx_q [B][Di] int8, keys [B][cap][Di/2 +
+ * Di/16] (R18 rows), scores_out [B][cap] int64 (times 2^10) or NULL.     */
+int orc_index_topk_fp4(const orc_cfg* c, int B, const int8_t* idx_q, const uint8_t* keys,
+                       int cap, const int32_t* n_entries, int32_t* topk, int64_t* scores_out) {
+    int di = c->idx_dim, row = di / 2 + di / 16;
+    if (di % 16) return ORC_ERR_INVALID;
+    int64_t* s = (int64_t*)malloc(sizeof(int64_t) * (size_t)(cap > 0 ? cap : 1));
+    for (int b = 0; b < B; ++b) {
+        int n = n_entries[b];
+        if (n < 0 || n > cap) {
+            free(s);
+            return ORC_ERR_CAPACITY;
+        }
+        for (int j = 0; j < n; ++j)
+            s[j] = orc_idx_fp4_score(idx_q + (size_t)b * di,
+                                     keys + ((size_t)b * cap + j) * row, di);
+        if (scores_out) memcpy(scores_out + (size_t)b * cap, s, sizeof(int64_t) * (size_t)n);
+        orc_topk64(s, n, c->topk, topk + (size_t)b * c->topk);
     }
     free(s);
     return ORC_OK;
