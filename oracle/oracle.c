@@ -37,7 +37,7 @@
  *  R18 FP4 indexer keys: quantised like a main-KV entry (no RoPE, groups of
  *     16, UE4M3), scored exactly against the int8 query (see
  *     orc_idx_fp4_score).
- *  R6 4:1 compression ([P1] 4.3 lists a CSA2 compression ratio of 2x or 4x):
+ *  R17 4:1 compression ([P1] 4.3 lists a CSA2 compression ratio of 2x or 4x):
  *     four consecutive tokens form one entry, weighted by the softmax of their
  *     four gate logits, each logit summed in the order of R1; see
  *     orc_compress_group4.
@@ -47,7 +47,7 @@
  * library routines).  orc_compress_pair and orc_compress_group4 are pinned
  * only by invariants (identical tokens, zero gate, a dominant token,
  * convexity, fp64 softmax weights); their exact fp32 operation order is a
- * reading (R1, R6), so beyond those invariants they are "parity unpinned"
+ * reading (R1, R17), so beyond those invariants they are "parity unpinned"
  * by the pages, and the GPU is held to them by following the same order.
  *
  * Compile with -ffp-contract=off: every fused multiply-add below is an
@@ -291,7 +291,7 @@ void orc_compress_pair(const float* k0, const float* k1, const float* g, int D,
     for (int d = 0; d < D; ++d) e[d] = fmaf(w0, k0[d], w1 * k1[d]);
 }
 
-/* R6: the 4:1 compression of four consecutive tokens (the ratio 4 of [P1]
+/* R17: the 4:1 compression of four consecutive tokens (the ratio 4 of [P1]
  * 4.3; the pages give the 2:1 rule only, this is its plainest extension).
  * logit_t = g . k_t, each summed like delta in R1: 8 partial sums over the
  * 8-channel chunks (chunk c to partial c mod 8, chunks and channels in
