@@ -29,6 +29,7 @@ bool derive_shape(const kvc_config* c, Shape* s) {
     if (!(c->sm_scale > 0.f) || !(c->sm_scale < 1e30f)) return false;
     if (c->act_dtype != KVC_F32 && c->act_dtype != KVC_BF16) return false;
     if (c->ratio != 0 && c->ratio != 2 && c->ratio != 4) return false;
+    if (c->idx_fmt != 0 && c->idx_fmt != 1) return false;
     s->D = D;
     s->Dv = c->latent_dim;
     s->G = G;
@@ -39,6 +40,8 @@ bool derive_shape(const kvc_config* c, Shape* s) {
     s->rec_unpadded = s->code_bytes + s->n_groups * s->scale_bytes;
     s->rb = (s->rec_unpadded + 15) / 16 * 16;
     s->act_bytes = c->act_dtype == KVC_BF16 ? 2 : 4;
+    s->idx_fmt = c->idx_fmt;
+    s->idx_rb = c->idx_fmt == 1 ? di / 2 + di / 16 : di;
     return true;
 }
 
@@ -220,6 +223,7 @@ kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* c
                     int32_t* topk, int32_t* scores, unsigned char* ws, const WsLayout& w,
                     uint32_t* st, cudaStream_t s) {
     if (cache->capacity > kMaxTopkCapacity) return KVC_ERR_CAPACITY;
+    if (c.idx_fmt == 1 && scores) return KVC_ERR_UNSUPPORTED;
     TopkArgs a = {};
     a.idx_q = idx_q;
     a.idx_k = cache->idx_k;
@@ -236,6 +240,13 @@ kvc_status run_topk(const kvc_config& c, const int8_t* idx_q, const kvc_cache* c
     a.tile_count = reinterpret_cast<int32_t*>(ws + w.tile_count);
     a.cands = reinterpret_cast<unsigned long long*>(ws + w.cands);
     a.status = st;
+    if (c.idx_fmt == 1) {  // exact 64-bit scores in the candidate region (unused here)
+        const int rb = c.idx_dim / 2 + c.idx_dim / 16;
+        return launch_index_topk_fp4(a, rb, reinterpret_cast<long long*>(ws + w.cands), s) ==
+                       cudaSuccess
+                   ? KVC_OK
+                   : KVC_ERR_CUDA;
+    }
     return launch_index_topk(a, s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
@@ -329,11 +340,16 @@ size_t kvc_record_bytes(const kvc_config* cfg) {
     return derive_shape(cfg, &sh) ? (size_t)sh.rb : 0;
 }
 
+size_t kvc_idx_row_bytes(const kvc_config* cfg) {
+    Shape sh;
+    return derive_shape(cfg, &sh) ? (size_t)sh.idx_rb : 0;
+}
+
 size_t kvc_bytes_resident(const kvc_config* cfg, int64_t entries, int n_layers, int padded) {
     Shape sh;
     if (!derive_shape(cfg, &sh) || entries < 0 || n_layers < 0) return 0;
     const int64_t rec = padded ? sh.rb : sh.rec_unpadded;
-    return (size_t)(entries * rec + entries * cfg->idx_dim +
+    return (size_t)(entries * rec + entries * sh.idx_rb +
                     (int64_t)n_layers * cfg->window * sh.D * sh.act_bytes);
 }
 
@@ -395,6 +411,7 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q, const kvc_
     if (cache->batch == 0) return KVC_OK;
     if (!idx_q || !topk_idx || !aligned(idx_q, 16) || !aligned(topk_idx, 4)) return KVC_ERR_INVALID;
     if (scores && !aligned(scores, 4)) return KVC_ERR_INVALID;
+    if (scores && sh.idx_fmt == 1) return KVC_ERR_UNSUPPORTED;  // FP4 keys: 64-bit scores
     WsLayout w;
     if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
     if (!device_ok()) return KVC_ERR_DEVICE;
@@ -483,6 +500,7 @@ kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     if (!hier_ok(hier_blocks, hier_block)) return KVC_ERR_INVALID;
+    if (hier_blocks > 0 && sh.idx_fmt != 0) return KVC_ERR_UNSUPPORTED;
     kvc_status st = check_cache(cache, sh);
     if (st != KVC_OK) return st;
     if (n_layers < 1 || !modes) return KVC_ERR_INVALID;
@@ -559,7 +577,7 @@ kvc_status kvc_index_topk_batched(const kvc_config* cfg, int nq, const int8_t* i
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     if (nq < 1 || nq > kMaxBatchQ) return KVC_ERR_INVALID;
-    if (cfg->idx_dim != 128) return KVC_ERR_UNSUPPORTED;
+    if (cfg->idx_dim != 128 || sh.idx_fmt != 0) return KVC_ERR_UNSUPPORTED;
     kvc_status st = check_cache(cache, sh);
     if (st != KVC_OK) return st;
     if (cache->batch == 0) return KVC_OK;

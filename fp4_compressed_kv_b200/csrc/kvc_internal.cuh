@@ -43,6 +43,8 @@ struct Shape {
     int rec_unpadded;
     int rb;         // record stride (padded to 16)
     int act_bytes;  // 2 (bf16) or 4 (fp32)
+    int idx_fmt;    // 0 int8 indexer rows, 1 FP4 indexer rows
+    int idx_rb;     // bytes of one indexer row
 };
 
 bool derive_shape(const kvc_config* c, Shape* s);
@@ -103,6 +105,10 @@ struct TopkArgs {
     int pool_src_cap, pool_src_block;
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
+// FP4 indexer keys: exact 64-bit scores (scores64 [B][capacity]) and the
+// top-K by a radix selection; idx_k rows of idx_rb bytes.
+cudaError_t launch_index_topk_fp4(const TopkArgs& a, int idx_rb, long long* scores64,
+                                  cudaStream_t s);
 // The selection alone, from scores and threshold bins already in the scratch.
 cudaError_t launch_select(const TopkArgs& a, int bias, int shift, cudaStream_t s);
 

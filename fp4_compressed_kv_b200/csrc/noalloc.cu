@@ -67,6 +67,7 @@ extern "C" kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t
                                              void* stream) {
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
+    if (sh.idx_fmt != 0) return KVC_ERR_UNSUPPORTED;
     if (!cache || !cache->records || !cache->idx_k || !cache->n_entries) return KVC_ERR_INVALID;
     if (cache->batch < 0 || cache->capacity < 0) return KVC_ERR_INVALID;
     if (!aligned_to(cache->idx_k, 16) || !aligned_to(cache->n_entries, 4)) return KVC_ERR_INVALID;

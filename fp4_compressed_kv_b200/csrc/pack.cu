@@ -909,6 +909,60 @@ cudaError_t launch_window_t(const void* rows, long long n, int D, uint8_t* codes
     return err;
 }
 
+__device__ __forceinline__ float key_f32(float v) { return v; }
+__device__ __forceinline__ float key_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// FP4 indexer keys (idx_fmt = 1): the new entries' keys quantised like a
+// record of idx_dim channels with groups of 16 and UE4M3 scales (absmax / 6,
+// round to nearest even; the same scale and quotient steps as the records).
+// A thread per group of 16 channels; the rows are written at the entries'
+// positions before the pack kernel that follows on the stream advances the
+// lengths.  Row: idx_dim/2 code bytes (channel 2c in the low nibble of byte
+// c), then idx_dim/16 scale bytes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+idx_fp4_pack_kernel(const T* __restrict__ keys, int per, int batch, int di, int capacity,
+                    const int32_t* __restrict__ n_entries, uint8_t* __restrict__ rows,
+                    uint32_t* status) {
+    pdl_trigger();  // a short kernel: the next one may be scheduled at once
+    pdl_wait();
+    const int ng = di / 16;
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= (long long)batch * per * ng) return;
+    const int g = (int)(t % ng);
+    const long long e = t / ng;
+    const int b = (int)(e / per), i = (int)(e % per);
+    const int base = n_entries[b];
+    if (base < 0 || base + per > capacity) return;  // the pack kernel flags it
+    const T* k = keys + ((long long)b * per + i) * di + 16 * g;
+    float x[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) x[u] = key_f32(k[u]);
+    bool bad = false;
+    float m = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        if (!isfinite(x[u])) {
+            bad = true;
+            x[u] = 0.f;
+        }
+        m = fmaxf(m, fabsf(x[u]));
+    }
+    float sc = __fdiv_rn(m, 6.0f);
+    const uint32_t sbyte = e4m3_from_f32(sc);
+    sc = e4m3_to_f32(sbyte);
+    const uint32_t c0 = sc > 0.f ? e2m1x8_quotient(x, sc) : 0u;
+    const uint32_t c1 = sc > 0.f ? e2m1x8_quotient(x + 8, sc) : 0u;
+    uint8_t* row = rows + ((long long)b * capacity + base + i) * (di / 2 + di / 16);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // byte stores: a row need not be 4-byte aligned
+        row[8 * g + u] = (uint8_t)(c0 >> (8 * u));
+        row[8 * g + 4 + u] = (uint8_t)(c1 >> (8 * u));
+    }
+    row[di / 2 + g] = (uint8_t)sbyte;
+    if (bad) set_status(status, KVC_DEV_NONFINITE);
+}
+
 }  // namespace
 
 cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
@@ -918,12 +972,30 @@ cudaError_t launch_pack(const kvc_config& c, const Shape& sh, const PackArgs& a,
     if (half == 0 || a.batch == 0) return cudaSuccess;
     const int ue = c.scale_fmt == KVC_SCALE_UE4M3;
     cudaError_t err;
+    int di_copy = c.idx_dim;  // int8 keys are copied by the pack kernel itself
+    if (c.idx_fmt == 1) {     // FP4 keys: quantised first, at the entries' positions
+        di_copy = 0;
+        const long long groups = (long long)a.batch * half * (c.idx_dim / 16);
+        const unsigned grid = (unsigned)((groups + 255) / 256);
+        trace_before("pack_idx", s);
+        err = c.act_dtype == KVC_BF16
+                  ? launch_pdl(idx_fp4_pack_kernel<__nv_bfloat16>, grid, 256, 0, s,
+                               reinterpret_cast<const __nv_bfloat16*>(a.idx_k_new), half, a.batch,
+                               c.idx_dim, a.capacity, a.n_entries,
+                               reinterpret_cast<uint8_t*>(a.idx_k), a.status)
+                  : launch_pdl(idx_fp4_pack_kernel<float>, grid, 256, 0, s,
+                               reinterpret_cast<const float*>(a.idx_k_new), half, a.batch,
+                               c.idx_dim, a.capacity, a.n_entries,
+                               reinterpret_cast<uint8_t*>(a.idx_k), a.status);
+        trace_after(s);
+        if (err != cudaSuccess) return err;
+    }
     if (four)
-        err = c.act_dtype == KVC_BF16 ? launch_pack4_t<__nv_bfloat16>(sh, a, ue, c.idx_dim, s)
-                                      : launch_pack4_t<float>(sh, a, ue, c.idx_dim, s);
+        err = c.act_dtype == KVC_BF16 ? launch_pack4_t<__nv_bfloat16>(sh, a, ue, di_copy, s)
+                                      : launch_pack4_t<float>(sh, a, ue, di_copy, s);
     else
-        err = c.act_dtype == KVC_BF16 ? launch_pack_t<__nv_bfloat16>(sh, a, ue, c.idx_dim, s)
-                                      : launch_pack_t<float>(sh, a, ue, c.idx_dim, s);
+        err = c.act_dtype == KVC_BF16 ? launch_pack_t<__nv_bfloat16>(sh, a, ue, di_copy, s)
+                                      : launch_pack_t<float>(sh, a, ue, di_copy, s);
     if (err != cudaSuccess) return err;
     // one entry per sequence: committed by the append kernel
     if (half == 1 && (four || a.batch <= 4096)) return cudaSuccess;

@@ -34,7 +34,7 @@ class Config(C.Structure):
     _fields_ = [("latent_dim", C.c_int32), ("rope_dim", C.c_int32), ("group", C.c_int32),
                 ("scale_fmt", C.c_int32), ("idx_dim", C.c_int32), ("topk", C.c_int32),
                 ("window", C.c_int32), ("n_heads", C.c_int32), ("sm_scale", C.c_float),
-                ("act_dtype", C.c_int32), ("ratio", C.c_int32)]
+                ("act_dtype", C.c_int32), ("ratio", C.c_int32), ("idx_fmt", C.c_int32)]
 
 
 class CacheStruct(C.Structure):
@@ -56,6 +56,7 @@ def _lib():
         S = C.c_int  # kvc_status
         sig = {
             "kvc_record_bytes": (Z, [P]),
+            "kvc_idx_row_bytes": (Z, [P]),
             "kvc_bytes_resident": (Z, [P, C.c_int64, I, I]),
             "kvc_workspace_bytes": (Z, [P, I, I]),
             "kvc_pack": (S, [P, P, I, P, P, P, P, P]),
@@ -113,20 +114,26 @@ def _stream(stream):
 
 
 def make_config(latent_dim, rope_dim, group, scale_fmt, idx_dim, topk, window, n_heads, sm_scale,
-                act_dtype, ratio=2) -> Config:
-    """ratio: raw tokens per entry, 2 or 4."""
+                act_dtype, ratio=2, idx_fmt=0) -> Config:
+    """ratio: raw tokens per entry, 2 or 4; idx_fmt: indexer keys as int8 (0)
+    or FP4 rows (1)."""
     return Config(latent_dim, rope_dim, group, scale_fmt, idx_dim, topk, window, n_heads,
-                  float(sm_scale), act_dtype, ratio)
+                  float(sm_scale), act_dtype, ratio, idx_fmt)
 
 
 def config_for(w) -> Config:
     """kvc_config of a synth.Workload."""
     return make_config(w.latent, w.rope, w.group, w.scale_fmt, w.idx_dim, w.topk, w.window,
-                       w.heads, w.sm_scale, F32 if w.act == "f32" else BF16, w.ratio)
+                       w.heads, w.sm_scale, F32 if w.act == "f32" else BF16, w.ratio,
+                       w.idx_fmt)
 
 
 def record_bytes(cfg: Config) -> int:
     return int(_lib().kvc_record_bytes(C.byref(cfg)))
+
+
+def idx_row_bytes(cfg: Config) -> int:
+    return int(_lib().kvc_idx_row_bytes(C.byref(cfg)))
 
 
 def bytes_resident(cfg: Config, entries: int, n_layers: int, padded: bool) -> int:
@@ -146,7 +153,12 @@ class Cache:
             raise ValueError("invalid kvc config")
         self.cfg, self.batch, self.capacity = cfg, batch, capacity
         self.records = torch.zeros(batch, capacity, rb, dtype=torch.uint8, device=device)
-        self.idx_k = torch.zeros(batch, capacity, cfg.idx_dim, dtype=torch.int8, device=device)
+        if cfg.idx_fmt == 1:  # FP4 rows of idx_dim/2 + idx_dim/16 bytes
+            self.idx_k = torch.zeros(batch, capacity, idx_row_bytes(cfg), dtype=torch.uint8,
+                                     device=device)
+        else:
+            self.idx_k = torch.zeros(batch, capacity, cfg.idx_dim, dtype=torch.int8,
+                                     device=device)
         self.n_entries = torch.zeros(batch, dtype=torch.int32, device=device)
 
     def struct(self) -> CacheStruct:

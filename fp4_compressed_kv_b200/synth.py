@@ -42,6 +42,7 @@ class Workload:
     pack_new: int = 0     # new raw tokens per sequence for the pack benchmark
     groups: int = 1       # independent layer groups, each with its own cache and `modes`
     ratio: int = 2        # raw tokens per entry (2 or 4)
+    idx_fmt: int = 0      # indexer keys: 0 int8, 1 FP4 rows
 
     @property
     def dim(self) -> int:

@@ -88,7 +88,12 @@ typedef struct {
     int32_t idx_dim, topk, window, n_heads;
     float sm_scale;
     int32_t act_dtype;
-    int32_t ratio;  /* raw tokens per entry: 2 (0 also means 2) or 4 */
+    int32_t ratio;   /* raw tokens per entry: 2 (0 also means 2) or 4 */
+    int32_t idx_fmt; /* indexer keys: 0 = int8 rows of idx_dim bytes; 1 = FP4 rows of
+                        idx_dim/2 E2M1 code bytes (channel 2c in the low nibble of
+                        byte c) then idx_dim/16 UE4M3 scales, one per 16 channels
+                        -- the 72-byte indexer K of [A] "890 字节是怎么算出来的" at
+                        128 channels */
 } kvc_config;
 
 /* One stored cache (the Full layer's).  Caller-owned device buffers:
@@ -96,7 +101,8 @@ typedef struct {
  *             Record = [D/2 bytes of E2M1 codes, channel 2c in the low nibble of
  *             byte c][one scale per group, in group order: 1 byte UE4M3 or 4
  *             bytes fp32][zero padding to a multiple of 16 bytes]
- *  idx_k      [batch][capacity][idx_dim] int8 indexer keys
+ *  idx_k      [batch][capacity][kvc_idx_row_bytes(cfg)] indexer keys (int8
+ *             values, or FP4 rows when cfg->idx_fmt = 1)
  *  n_entries  [batch] int32, entries stored per sequence (visible to the
  *             indexer: entries 0 .. n_entries-1)                            */
 typedef struct {
@@ -108,6 +114,10 @@ typedef struct {
 
 /* Bytes of one record (with padding) = the record stride. 0 if cfg invalid. */
 size_t kvc_record_bytes(const kvc_config* cfg);
+
+/* Bytes of one indexer row in the cache: idx_dim (int8 keys) or idx_dim/2 +
+ * idx_dim/16 (FP4 keys, idx_fmt = 1).  0 if cfg invalid. */
+size_t kvc_idx_row_bytes(const kvc_config* cfg);
 
 /* Bytes resident per sequence for `entries` stored entries and `n_layers`
  * layers each holding its own window of W raw keys (record bytes with or
@@ -134,7 +144,10 @@ size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity);
  *           gate logits g.k; the weighted sum is quantised per group to E2M1
  *           with scale absmax/6 ([B] 3.1; [A] "P4 main KV").
  * gate      [D] fp32 gate vector g.
- * idx_k_new [batch][n_new/r][idx_dim] int8 indexer keys of the new entries.
+ * idx_k_new [batch][n_new/r][idx_dim] indexer keys of the new entries: int8
+ *           (idx_fmt = 0), or act_dtype values (idx_fmt = 1) quantised to FP4
+ *           rows like a record of idx_dim channels with groups of 16 and UE4M3
+ *           scales (absmax/6, round to nearest even).
  * Entries are written at positions n_entries[b] .. n_entries[b]+n_new/r-1 and
  * n_entries[b] then advances by n_new/r.  If that would pass the capacity the
  * sequence is left unchanged and KVC_DEV_CAPACITY is set.  NaN/Inf channels are
@@ -155,7 +168,11 @@ kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,
  * ws        device workspace of at least kvc_workspace_bytes(cfg, batch,
  *           capacity) bytes, 256-byte aligned, zero-filled before its first
  *           use (see kvc_workspace_bytes).
- * capacity must not exceed 8,388,608 entries (KVC_ERR_CAPACITY).         */
+ * capacity must not exceed 8,388,608 entries (KVC_ERR_CAPACITY).
+ * FP4 indexer keys (idx_fmt = 1): the score of an entry is the exact value of
+ * idx_q . dequant(k) (an integer multiple of 2^-10, held in 64 bits), the
+ * selection as above; `scores` must be NULL (KVC_ERR_UNSUPPORTED).  The
+ * hierarchical, batched and fixed-scratch variants take int8 keys only.         */
 kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
                           const kvc_cache* cache, int32_t* topk_idx,
                           int32_t* scores, void* ws, size_t ws_bytes,
@@ -303,9 +320,10 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * max_launches launches are recorded).  kvc_trace_kernel, called after the
  * traced work has completed, returns the number of recorded launches of the
  * kernel named `name` and their summed device time in milliseconds.  Names:
- * "pack", "pack_commit", "window_fp8", "index_scan", "index_scan_tc",
- * "topk_select", "block_max", "copy_topk", "attn_tc05", "attn_simt",
- * "attn_merge", "fp4_codec".                                                             */
+ * "pack", "pack_idx", "pack_commit", "window_fp8", "index_scan",
+ * "index_scan_tc", "index_scan_fp4", "topk_select", "topk_select_fp4",
+ * "block_max", "copy_topk", "attn_tc05", "attn_simt", "attn_merge",
+ * "fp4_codec".                                                             */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);
 kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);

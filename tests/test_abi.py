@@ -58,7 +58,8 @@ def test_invalid_configs_rejected(lib):
     base = synth.WORKLOADS["mla32k"]
     for field, value in [("group", 48), ("group", 1024), ("latent_dim", 500), ("idx_dim", 100),
                          ("topk", 0), ("topk", 5000), ("scale_fmt", 3), ("act_dtype", 7),
-                         ("sm_scale", 0.0), ("n_heads", 0), ("ratio", 3), ("ratio", 8)]:
+                         ("sm_scale", 0.0), ("n_heads", 0), ("ratio", 3), ("ratio", 8),
+                         ("idx_fmt", 2), ("idx_fmt", -1)]:
         cfg = lib.config_for(base)
         setattr(cfg, field, value)
         assert lib.record_bytes(cfg) == 0, field
@@ -136,3 +137,31 @@ def test_batched_workspace_and_validation(lib):
                                      C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 4
     assert so.kvc_index_topk_batched(C.byref(cfg), 9, C.c_void_p(16), C.byref(cache),
                                      C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 1
+
+
+def test_fp4_indexer_rows_and_rejections(lib):
+    """FP4 indexer keys: 72-byte rows at 128 channels (idx_dim/2 + idx_dim/16),
+    counted in the bytes resident; the hierarchical, batched and fixed-scratch
+    variants refuse them before touching the device."""
+    so = lib.lib()
+    w = synth.WORKLOADS["mla32k"]
+    c8, c4 = lib.config_for(w), lib.config_for(w.scaled(idx_fmt=1))
+    assert lib.idx_row_bytes(c8) == 128 and lib.idx_row_bytes(c4) == 72
+    assert lib.record_bytes(c4) == lib.record_bytes(c8)
+    assert lib.bytes_resident(c8, 1000, 0, False) - lib.bytes_resident(c4, 1000, 0, False) == \
+        1000 * (128 - 72)
+    for di, rb in ((16, 9), (32, 18), (64, 36), (256, 144)):
+        assert lib.idx_row_bytes(lib.config_for(w.scaled(idx_fmt=1, idx_dim=di))) == rb
+    cache = lib.CacheStruct(16, 16, 16, 1, 8)
+    assert so.kvc_index_topk_noalloc(C.byref(c4), C.c_void_p(16), C.byref(cache),
+                                     C.c_void_p(16), None, None, None) == 4
+    assert so.kvc_index_topk_batched(C.byref(c4), 2, C.c_void_p(16), C.byref(cache),
+                                     C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 4
+    modes = (C.c_int32 * 1)(0)
+    assert so.kvc_layer_group_step_hier(C.byref(c4), 2048, 8, 1, modes, C.c_void_p(16),
+                                        C.c_void_p(16), C.c_void_p(16), 32, C.byref(cache),
+                                        C.c_void_p(16), None, C.c_void_p(16), C.c_void_p(256),
+                                        1 << 30, None, None) == 4
+    # the exact scores are 64-bit: no int32 score output for FP4 keys
+    assert so.kvc_index_topk(C.byref(c4), C.c_void_p(16), C.byref(cache), C.c_void_p(16),
+                             C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 4

@@ -1,0 +1,111 @@
+"""GPU FP4 indexer keys (idx_fmt = 1; the pages' 72-byte indexer K, "DeepSeek
+V1 到 V4.1-Flash ...", "890 字节是怎么算出来的") vs the oracle: the pack writes
+the key rows bit for bit as the oracle quantises them; the exact 64-bit
+scores give bit-exact top-K sets (ragged lengths, K >= N, forced ties); a
+layer-group step over FP4 keys matches the oracle's selection and attention."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_compressed_kv_b200 import synth
+from helpers import assert_attn_close, f32, oracle_cfg, oracle_pack
+
+pytestmark = pytest.mark.gpu
+
+
+def _keys(B, N, di, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(B, N, di, generator=g) * scale).to(torch.bfloat16)
+
+
+def _packed(kvc, w, keys, chunks):
+    """GPU cache of workload w's tokens with FP4 indexer rows from `keys`."""
+    inp = synth.make_inputs(w)
+    cfg = kvc.config_for(w)
+    B, T = inp["tokens"].shape[:2]
+    N = T // 2
+    cache = kvc.Cache(cfg, B, N)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok, gate, kd = inp["tokens"].cuda(), inp["gate"].cuda(), keys.cuda()
+    for t0 in range(0, T, chunks):
+        kvc.pack(cfg, tok[:, t0:t0 + chunks].contiguous(), gate,
+                 kd[:, t0 // 2:(t0 + chunks) // 2].contiguous(), cache, status=st)
+    torch.cuda.synchronize()
+    return inp, cfg, cache, int(st.item())
+
+
+def _oracle_rows(w, keys):
+    ocfg = oracle_cfg(w)
+    return np.stack([oracle.idx_fp4_quantize(ocfg, f32(keys[b])) for b in range(keys.shape[0])])
+
+
+@pytest.mark.parametrize("chunks", [2, 3000])
+def test_pack_writes_fp4_key_rows(kvc, chunks):
+    w = synth.WORKLOADS["mla32k"].scaled(batch=2, context=2 * 1500, idx_fmt=1)
+    keys = _keys(2, 1500, 128, 3, scale=5.0)
+    inp, cfg, cache, st = _packed(kvc, w, keys, chunks)
+    assert st == 0 and kvc.idx_row_bytes(cfg) == 72
+    assert cache.n_entries.cpu().tolist() == [1500, 1500]
+    assert np.array_equal(cache.idx_k.cpu().numpy(), _oracle_rows(w, keys))
+    rec, _, _, _ = oracle_pack(w, inp["tokens"], inp["gate"], torch.zeros(2, 1500, 128,
+                                                                          dtype=torch.int8))
+    assert np.array_equal(cache.records.cpu().numpy(), rec)
+
+
+def test_topk_over_fp4_keys(kvc):
+    w = synth.WORKLOADS["mla32k"].scaled(batch=4, context=2 * 3000, idx_fmt=1)
+    keys = _keys(4, 3000, 128, 5)
+    keys[1, 1000:1400] = keys[1, 17]   # 401 equal rows: ties to the lower index
+    keys[2] = keys[2, 0]               # every row equal
+    inp, cfg, cache, st = _packed(kvc, w, keys, 6000)
+    assert st == 0
+    n = [3000, 2999, 2500, 400]        # ragged; the last below K
+    cache.n_entries.copy_(torch.tensor(n, dtype=torch.int32))
+    q = torch.randint(-128, 128, (4, 128), generator=torch.Generator().manual_seed(8),
+                      dtype=torch.int8)
+    tk = torch.empty(4, w.topk, dtype=torch.int32, device="cuda")
+    ws = kvc.workspace(cfg, 4, cache.capacity)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvc.index_topk(cfg, q.cuda(), cache, tk, ws, status=st2)
+    torch.cuda.synchronize()
+    rows = _oracle_rows(w, keys)       # the oracle's own rows, equal to the GPU's
+    assert np.array_equal(cache.idx_k.cpu().numpy(), rows)
+    otk = oracle.index_topk_fp4(oracle_cfg(w), q.numpy(), rows, np.array(n, np.int32))
+    assert int(st2.item()) == 0
+    assert np.array_equal(tk.cpu().numpy(), otk)
+    assert tk[2].cpu().tolist() == list(range(w.topk))
+    assert tk[3].cpu().tolist()[:400] == list(range(400)) and (tk[3, 400:] == -1).all()
+
+
+def test_group_step_over_fp4_keys(kvc):
+    w = synth.WORKLOADS["csa2group"].scaled(batch=2, context=2 * 2500, idx_fmt=1)
+    keys = _keys(2, 2500, 128, 11, scale=3.0)
+    inp, cfg, cache, st = _packed(kvc, w, keys, 5000)
+    assert st == 0
+    L, B, H = w.layers, w.batch, w.heads
+    out = torch.empty(L, B, H, w.latent, device="cuda")
+    lse = torch.empty(L, B, H, device="cuda")
+    tk = torch.empty(L, B, w.topk, dtype=torch.int32, device="cuda")
+    ws = kvc.workspace(cfg, B, cache.capacity)
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvc.layer_group_step(cfg, list(w.modes), inp["q"].cuda(), inp["idx_q"].cuda(),
+                         inp["windows"].cuda(), w.window, cache, out, tk, ws, lse=lse, status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0
+    ocfg = oracle_cfg(w)
+    # the oracle's own cache (records from its pack, rows from its quantiser)
+    recs, _, n, _ = oracle_pack(w, inp["tokens"], inp["gate"],
+                                torch.zeros(2, 2500, 128, dtype=torch.int8))
+    rows = _oracle_rows(w, keys)
+    assert np.array_equal(cache.records.cpu().numpy(), recs)
+    assert np.array_equal(cache.idx_k.cpu().numpy(), rows)
+    head = None
+    for l, m in enumerate(w.modes):
+        if m != synth.REUSE:
+            head = oracle.index_topk_fp4(ocfg, inp["idx_q"][l].numpy(), rows, n)
+        assert np.array_equal(tk[l].cpu().numpy(), head), l
+        ref, _, ost = oracle.sparse_decode(ocfg, f32(inp["q"][l]), recs, n, head,
+                                           f32(inp["windows"][l]), w.window)
+        assert ost == 0
+        assert_attn_close(out[l].cpu().numpy(), ref, f"fp4 keys layer {l}")
