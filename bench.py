@@ -110,6 +110,54 @@ def time_group(w, steps, warmup, hier_blocks, hier_block, dev):
     return ms
 
 
+def time_index_fp4(w, steps, warmup, dev):
+    """Device ms of one top-K call of workload w's shape with FP4 indexer keys
+    (72-byte rows: seeded random E2M1 codes, UE4M3 scales between 2^-8 and 2^1)
+    against the same call with int8 keys (random values)."""
+    import torch
+    from fp4_compressed_kv_b200 import kvc, synth
+    g = synth.generator(dev, w.seed + 7)
+    res = {}
+    for fmt in (0, 1):
+        cfg = kvc.config_for(w.scaled(idx_fmt=fmt))
+        cache = kvc.Cache(cfg, w.batch, w.entries, device=dev)
+        if fmt == 1:
+            half = w.idx_dim // 2
+            cache.idx_k[..., :half] = torch.randint(0, 256, cache.idx_k[..., :half].shape,
+                                                    generator=g, device=dev, dtype=torch.uint8)
+            cache.idx_k[..., half:] = torch.randint(0x20, 0x40, cache.idx_k[..., half:].shape,
+                                                    generator=g, device=dev, dtype=torch.uint8)
+        else:
+            cache.idx_k.copy_(torch.randint(-127, 128, cache.idx_k.shape, generator=g,
+                                            device=dev, dtype=torch.int8))
+        cache.n_entries.fill_(w.entries)
+        q = torch.randint(-127, 128, (w.batch, w.idx_dim), generator=g, device=dev,
+                          dtype=torch.int8)
+        tk = torch.empty(w.batch, w.topk, dtype=torch.int32, device=dev)
+        ws = kvc.workspace(cfg, w.batch, w.entries, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(warmup):
+            kvc.index_topk(cfg, q, cache, tk, ws, status=st)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for _ in range(steps):
+                kvc.index_topk(cfg, q, cache, tk, ws, status=st)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gr.replay()  # untimed first launch (uploads the graph)
+        torch.cuda.synchronize()
+        e0.record()
+        gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del gr
+        assert st.item() == 0, st.item()
+        res["fp4_keys" if fmt else "int8_keys"] = round(e0.elapsed_time(e1) / steps, 4)
+        del cache, ws
+        torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- bytes
 def record_unpadded(w):
     n_groups = -(-w.latent // w.group) + -(-w.rope // w.group)
@@ -670,6 +718,17 @@ def run_ours(args):
             "attention_ms_bf16_window": round(time_attention_window(w0, 20, 3, False, dev), 4),
             "attention_ms_fp8_window": round(time_attention_window(w0, 20, 3, True, dev), 4)}
         torch.cuda.empty_cache()
+        # the top-K call with FP4 indexer keys (72-byte rows) against int8 keys;
+        # last, and recorded as an error string if it fails
+        try:
+            extra["fp4_indexer_keys"] = {"workload": w0.name,
+                                         "index_topk_ms": time_index_fp4(w0, 20, 3, dev),
+                                         "row_bytes": {"int8_keys": w0.idx_dim,
+                                                       "fp4_keys": w0.idx_dim // 2 +
+                                                       w0.idx_dim // 16}}
+            torch.cuda.empty_cache()
+        except Exception as e:  # a side measurement must not cost the headline line
+            extra["fp4_indexer_keys"] = {"error": str(e)[:200]}
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
