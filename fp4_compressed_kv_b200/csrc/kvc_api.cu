@@ -412,6 +412,7 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q, const kvc_
     if (!idx_q || !topk_idx || !aligned(idx_q, 16) || !aligned(topk_idx, 4)) return KVC_ERR_INVALID;
     if (scores && !aligned(scores, 4)) return KVC_ERR_INVALID;
     if (scores && sh.idx_fmt == 1) return KVC_ERR_UNSUPPORTED;  // FP4 keys: 64-bit scores
+    if (cache->capacity > kMaxTopkCapacity) return KVC_ERR_CAPACITY;
     WsLayout w;
     if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w)) != KVC_OK) return st;
     if (!device_ok()) return KVC_ERR_DEVICE;
@@ -518,6 +519,7 @@ kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int
     const size_t q_stride = B * H * sh.D * sh.act_bytes;
     const size_t w_stride = B * (size_t)cfg->window * sh.D * sh.act_bytes;
     if (q_stride % 16 || (w_stride % 16) || (B * cfg->idx_dim) % 16) return KVC_ERR_INVALID;
+    if (cache->capacity > kMaxTopkCapacity) return KVC_ERR_CAPACITY;
     WsLayout w;
     if ((st = check_ws(ws, ws_bytes, *cfg, sh, cache->batch, cache->capacity, &w, hier_blocks,
                        hier_block)) != KVC_OK)

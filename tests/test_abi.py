@@ -177,3 +177,17 @@ def test_workspace_holds_fp4_scores(lib):
         n8, n4 = lib.workspace_bytes(c8, B, cap), lib.workspace_bytes(c4, B, cap)
         assert n8 == n4 > 0
         assert n4 >= B * cap * (4 + 8)
+
+
+def test_capacity_limit_on_the_host(lib):
+    """The top-K and the group step refuse capacities past 8,388,608 entries
+    before looking for a device."""
+    so = lib.lib()
+    cfg = lib.config_for(synth.WORKLOADS["tiny"])
+    big = lib.CacheStruct(16, 16, 16, 1, 8_388_609)
+    assert so.kvc_index_topk(C.byref(cfg), C.c_void_p(16), C.byref(big), C.c_void_p(16), None,
+                             C.c_void_p(256), 1 << 62, None, None) == 2
+    modes = (C.c_int32 * 1)(0)
+    assert so.kvc_layer_group_step(C.byref(cfg), 1, modes, C.c_void_p(16), C.c_void_p(16),
+                                   C.c_void_p(16), 32, C.byref(big), C.c_void_p(16), None,
+                                   C.c_void_p(16), C.c_void_p(256), 1 << 62, None, None) == 2
