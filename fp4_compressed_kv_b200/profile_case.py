@@ -1,10 +1,12 @@
 """Run one hot-path call a few times on synthetic inputs, for profilers.
 
-    python -m fp4_compressed_kv_b200.profile_case --kernel scan|attn|pack|step \
+    python -m fp4_compressed_kv_b200.profile_case --kernel scan|scan_fp4|attn|pack|step \
         [--config NAME] [--batch B] [--entries N] [--iters 3]
 
 scan  kvc_index_topk over B sequences of N int8 indexer rows (the indexer
-      scan, collect and finalize kernels), inputs from the workload's shapes.
+      scan and selection kernels), inputs from the workload's shapes.
+scan_fp4  the same over FP4 indexer rows (72 bytes at 128 channels: random
+      codes, UE4M3 scales between 2^-8 and 2^1).
 attn  kvc_sparse_decode_attn: B sequences, each with a cache of N packed
       entries, a top-K drawn uniformly from them and a full window.
 pack  kvc_pack of the workload's pack case (pack_new raw tokens per sequence,
@@ -24,7 +26,7 @@ from fp4_compressed_kv_b200 import build, kvc, synth
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("--kernel", required=True, choices=["scan", "attn", "pack", "step"])
+    p.add_argument("--kernel", required=True, choices=["scan", "scan_fp4", "attn", "pack", "step"])
     p.add_argument("--config", default="batch32x128k")
     p.add_argument("--batch", type=int, default=0)
     p.add_argument("--entries", type=int, default=0)
@@ -41,14 +43,23 @@ def main():
     g = synth.generator(dev, w.seed)
     B, N = w.batch, w.entries
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    if a.kernel in ("scan", "step", "attn"):
+    if a.kernel == "scan_fp4":  # FP4 indexer keys: random codes, scales 2^-8 .. 2^1
+        cfg = kvc.config_for(w.scaled(idx_fmt=1))
+    if a.kernel in ("scan", "scan_fp4", "step", "attn"):
         cache = kvc.Cache(cfg, B, N + a.iters + 8, device=dev)
         ws = kvc.workspace(cfg, B, cache.capacity, device=dev)
     if a.kernel in ("scan", "step"):
         cache.idx_k[:, :N] = torch.randint(-127, 128, (B, N, w.idx_dim), generator=g, device=dev,
                                            dtype=torch.int8)
         cache.n_entries.fill_(N)
-    if a.kernel == "scan":
+    if a.kernel == "scan_fp4":
+        half = w.idx_dim // 2
+        cache.idx_k[:, :N, :half] = torch.randint(0, 256, (B, N, half), generator=g, device=dev,
+                                                  dtype=torch.uint8)
+        cache.idx_k[:, :N, half:] = torch.randint(0x20, 0x40, (B, N, w.idx_dim // 16),
+                                                  generator=g, device=dev, dtype=torch.uint8)
+        cache.n_entries.fill_(N)
+    if a.kernel in ("scan", "scan_fp4"):
         q = torch.randint(-127, 128, (B, w.idx_dim), generator=g, device=dev, dtype=torch.int8)
         tk = torch.empty(B, w.topk, dtype=torch.int32, device=dev)
         for _ in range(a.iters):
