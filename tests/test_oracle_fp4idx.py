@@ -99,3 +99,15 @@ def test_topk_brute_force_with_ties():
         order = sorted(range(n[b]), key=lambda j: (-s[j], j))[:K]
         assert tk[b].tolist() == sorted(order)
     assert tk[1].tolist() == list(range(K))
+
+
+@pytest.mark.parametrize("n,k", [(0, 8), (5, 8), (1000, 64), (3000, 512)])
+def test_topk64_brute_force(n, k):
+    """The 64-bit selection: scores beyond 32 bits, many ties, K >= N."""
+    rng = np.random.default_rng(n + k)
+    s = rng.integers(-(1 << 36), 1 << 36, n)
+    if n > 10:
+        s[rng.choice(n, n // 3, replace=False)] = s[0]  # a third of them tie
+    got = orc.topk64(s.astype(np.int64), k)
+    order = sorted(range(n), key=lambda j: (-int(s[j]), j))[:k]
+    assert got.tolist() == sorted(order) + [-1] * (k - min(k, n))
