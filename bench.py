@@ -61,9 +61,8 @@ def parse():
 
 def time_group(w, steps, warmup, hier_blocks, hier_block, dev):
     """Device ms per decode step of workload w's layer groups (no pack), K
-    steps in one CUDA graph; the CSA2 group and the 1M stack with and without
-    the hierarchical indexer, the 18-layer encoder stack (3 groups, each with
-    its own cache)."""
+    steps in one CUDA graph, a new query set per step: the 18-layer encoder
+    stack (3 groups, each with its own cache)."""
     import torch
     from fp4_compressed_kv_b200 import kvc, synth
     cfg = kvc.config_for(w)
@@ -83,20 +82,24 @@ def time_group(w, steps, warmup, hier_blocks, hier_block, dev):
     tk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
     ws = kvc.workspace(cfg, B, w.entries, device=dev, hier_blocks=hier_blocks,
                        hier_block=hier_block)
+    # a new query set per step and group
+    sets = [synth.make_step_inputs(w.scaled(seed=w.seed + 100 * gi), warmup + steps, dev)
+            for gi in range(w.groups)]
 
-    def step():
-        for inp, cache in groups:
-            kvc.layer_group_step(cfg, list(w.modes), inp["q"], inp["idx_q"], inp["windows"],
+    def step(s):
+        for gi, (inp, cache) in enumerate(groups):
+            x = sets[gi][s]
+            kvc.layer_group_step(cfg, list(w.modes), x["q"], x["idx_q"], x["windows"],
                                  w.window, cache, out, tk, ws, lse=lse, status=st,
                                  hier_blocks=hier_blocks, hier_block=hier_block)
 
-    for _ in range(warmup):
-        step()
+    for s in range(warmup):
+        step(s)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        for _ in range(steps):
-            step()
+        for s in range(warmup, warmup + steps):
+            step(s)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     g.replay()  # untimed first launch (uploads the graph)
     torch.cuda.synchronize()
@@ -318,7 +321,7 @@ def time_attention_window(w, steps, warmup, fp8, dev):
     one layer) with the window in bf16 or in FP8."""
     import torch
     from fp4_compressed_kv_b200 import kvc, synth
-    wx = w.scaled(context=2 * 4096)
+    wx = w.scaled(context=2 * 32768)  # 32 x 32768 records: 318 MB, beyond L2
     cfg = kvc.config_for(wx)
     g = synth.generator(dev, 17)
     B, N = wx.batch, wx.entries
@@ -326,28 +329,33 @@ def time_attention_window(w, steps, warmup, fp8, dev):
     gate = (torch.randn(wx.dim, generator=g, device=dev) / wx.dim ** 0.5).float()
     nt = synth.make_new_tokens(wx, 2 * N, dev)
     kvc.pack(cfg, nt["tokens"], gate, nt["idx_k"], cache)
-    tk = torch.sort(torch.stack([torch.randperm(N, generator=g, device=dev)[: wx.topk]
-                                 for _ in range(B)]), 1).values.int().contiguous()
-    q = torch.randn(B, wx.heads, wx.dim, generator=g, device=dev).to(wx.torch_dtype)
-    win = torch.randn(B, wx.window, wx.dim, generator=g, device=dev).to(wx.torch_dtype)
-    codes = torch.empty(win.shape, dtype=torch.uint8, device=dev)
-    scales = torch.empty(win.shape[:-1], dtype=torch.float32, device=dev)
-    kvc.pack_window_fp8(cfg, win, codes, scales)
+    del nt
     out = torch.empty(B, wx.heads, wx.latent, device=dev)
     ws = kvc.workspace(cfg, B, N, device=dev)
+    sets = []
+    for _ in range(8):  # rotated: every call gathers a new selection
+        tk = torch.sort(torch.stack([torch.randperm(N, generator=g, device=dev)[: wx.topk]
+                                     for _ in range(B)]), 1).values.int().contiguous()
+        q = torch.randn(B, wx.heads, wx.dim, generator=g, device=dev).to(wx.torch_dtype)
+        win = torch.randn(B, wx.window, wx.dim, generator=g, device=dev).to(wx.torch_dtype)
+        codes = torch.empty(win.shape, dtype=torch.uint8, device=dev)
+        scales = torch.empty(win.shape[:-1], dtype=torch.float32, device=dev)
+        kvc.pack_window_fp8(cfg, win, codes, scales)
+        sets.append((tk, q, win, codes, scales))
 
-    def step():
+    def step(s):
+        tk, q, win, codes, scales = sets[s % len(sets)]
         if fp8:
             kvc.sparse_decode_attn_fp8win(cfg, q, cache, tk, codes, scales, wx.window, out, ws)
         else:
             kvc.sparse_decode_attn(cfg, q, cache, tk, win, wx.window, out, ws)
-    for _ in range(warmup):
-        step()
+    for s in range(warmup):
+        step(s)
     torch.cuda.synchronize()
     gr = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gr):
-        for _ in range(steps):
-            step()
+        for s in range(steps):
+            step(s)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gr.replay()  # untimed first launch (uploads the graph)
     torch.cuda.synchronize()
@@ -432,6 +440,171 @@ def oracle_decode_sample(w, seconds, seed_shift=0):
 
 
 # ----------------------------------------------------------------------------- ours
+def measure_decode(w, steps, warmup, dev, stream, hier=0, hier_block=8, clocks_gpu=None):
+    """Decode steps of workload w on this rank: the context is packed on the
+    device (untimed), then K steps -- each packs the token pair completed at
+    that step and runs the layer group on that step's own queries, indexer
+    queries and windows -- are captured into one CUDA graph and replayed
+    once between barriers (CUDA events on the launching stream, max over
+    ranks).  A second capture of the same steps with an event pair around
+    every library launch gives per-kernel durations.  Returns the numbers
+    and the state the end-to-end leg reuses."""
+    import torch
+
+    from fp4_compressed_kv_b200 import kvc, synth
+    from fp4_compressed_kv_b200 import dist as kd
+    cfg = kvc.config_for(w)
+    B, L, H = w.batch, w.layers, w.heads
+    N0 = w.entries
+    cap = N0 + warmup + steps + 64
+    inp = synth.make_inputs(w, dev)
+    cache = kvc.Cache(cfg, B, cap, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kvc.pack(cfg, inp["tokens"], inp["gate"], inp["idx_k"], cache, status=status)
+    torch.cuda.synchronize()
+    del inp["tokens"], inp["idx_k"]
+    torch.cuda.empty_cache()
+    gate = inp["gate"]
+    nsteps = warmup + steps
+    # every step decodes new queries (so a new top-K set) and new windows
+    sets = synth.make_step_inputs(w, nsteps, dev)
+    ws = kvc.workspace(cfg, B, cap, device=dev, hier_blocks=hier, hier_block=hier_block)
+    out = torch.empty(L, B, H, w.latent, device=dev)
+    lse = torch.empty(L, B, H, device=dev)
+    topk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
+    newp = synth.make_new_tokens(w, 2 * nsteps, dev)
+    pair_tok = [newp["tokens"][:, 2 * s:2 * s + 2].contiguous() for s in range(nsteps)]
+    pair_idx = [newp["idx_k"][:, s:s + 1].contiguous() for s in range(nsteps)]
+    modes = list(w.modes)
+
+    def step(s):
+        x = sets[s]
+        kvc.pack(cfg, pair_tok[s], gate, pair_idx[s], cache, status=status)
+        kvc.layer_group_step(cfg, modes, x["q"], x["idx_q"], x["windows"], w.window, cache, out,
+                             topk, ws, lse=lse, status=status, hier_blocks=hier,
+                             hier_block=hier_block)
+
+    for s in range(warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    # ---- capture the K timed steps into one graph and replay it once
+    launches0 = kvc.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(warmup, nsteps):
+            step(s)
+    launches = kvc.launch_count() - launches0
+    n_before = cache.n_entries.clone()
+    # one untimed replay first (the graph's first launch also uploads it);
+    # the timed replay then starts again from the same context lengths
+    graph.replay()
+    torch.cuda.synchronize()
+    cache.n_entries.copy_(n_before)
+
+    clocks = Clocks(clocks_gpu, enabled=clocks_gpu is not None)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kd.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kd.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    assert status.item() == 0, f"device status {status.item()}"
+    n_after = cache.n_entries.clone()
+    assert torch.all(n_after - n_before == steps)
+    del graph
+    ms_max = kd.max_over_ranks(ms, device=dev)
+
+    # ---- the same K steps again, from the same starting length, captured with
+    # a pair of event nodes around every library kernel: per-kernel durations
+    # (the event nodes themselves add time, so this replay is not the headline)
+    cache.n_entries.copy_(n_before)
+    kvc.trace_begin(16 * steps * max(1, L) + 16)
+    graph2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph2, stream=stream):
+        for s in range(warmup, nsteps):
+            step(s)
+    kvc.trace_end()
+    cache.n_entries.copy_(n_before)
+    graph2.replay()  # untimed: uploads the graph (its event nodes record again below)
+    torch.cuda.synchronize()
+    cache.n_entries.copy_(n_before)
+    kd.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    graph2.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms_traced = kd.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
+    del graph2
+
+    kernels = {}
+    for name in KERNELS:
+        cnt, tot = kvc.trace_kernel(name)
+        if cnt:
+            kernels[name] = {"launches": cnt, "ms_total": round(tot, 4),
+                             "us_avg": round(1e3 * tot / cnt, 2)}
+    n_mean = N0 + warmup + (steps + 1) / 2.0  # entries visible during the timed steps
+    return {"cfg": cfg, "cache": cache, "status": status, "ws": ws, "out": out, "lse": lse,
+            "topk": topk, "gate": gate, "sets": sets, "newp": newp, "n_before": n_before,
+            "ms_max": ms_max, "ms_traced": ms_traced, "kernels": kernels, "launches": launches,
+            "clocks": clk, "n_mean": n_mean}
+
+
+def kernel_bytes(w, n_mean):
+    """Algorithmic bytes per launch of the kernels whose work has a byte count."""
+    return {"index_scan": w.batch * scan_bytes(w, n_mean),
+            "attn_tc05": w.batch * attn_bytes(w),
+            "attn_simt": w.batch * attn_bytes(w),
+            "pack": w.batch * pack_bytes(w, 1)}
+
+
+def rooflines(w, m, peak, peak_kind):
+    """Per-kernel achieved GB/s and fraction of the peak, and the roofline
+    object of the dominant kernel (largest total time)."""
+    kernels = m["kernels"]
+    per_launch = kernel_bytes(w, m["n_mean"])
+    for name, k in kernels.items():
+        if name in per_launch:
+            gbs = per_launch[name] / (k["us_avg"] * 1e-6) / 1e9
+            k["gbs"] = round(gbs, 1)
+            k["frac"] = round(gbs / peak, 4)
+    dominant = max(kernels, key=lambda k: kernels[k]["ms_total"])
+    dom = kernels[dominant]
+    achieved = per_launch.get(dominant, 0) / (dom["us_avg"] * 1e-6) / 1e9
+    traffic = traffic_for(dominant)
+    return {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "bytes_per_launch": int(per_launch.get(dominant, 0)),
+            "traffic": (int(float(traffic["dram_bytes_per_launch"])) if traffic else None)}
+
+
+def workload_line(w, m, steps, world, peak, peak_kind):
+    """The measurement of one workload: throughput, step bandwidth, the
+    dominant kernel's roofline, per-kernel times and the bytes resident per
+    token of its cache."""
+    from fp4_compressed_kv_b200 import dist as kd
+    from fp4_compressed_kv_b200 import kvc
+    ms_step = m["ms_max"] / steps
+    sb = step_bytes(w, m["n_mean"])
+    step_gbs = sb / (ms_step * 1e-3) / 1e9
+    roof = rooflines(w, m, peak, peak_kind)
+    cfg = m["cfg"]
+    return {"value": round(kd.job_throughput(steps, w.batch, world, m["ms_max"]), 1),
+            "unit": UNIT, "ms_per_step": round(ms_step, 4),
+            "ms_per_step_traced": round(m["ms_traced"] / steps, 4),
+            "hbm_gbs_step": round(step_gbs, 1), "step_frac_of_peak": round(step_gbs / peak, 4),
+            "step_bytes": int(sb), "roofline": roof, "kernels": m["kernels"],
+            "bytes_resident_per_token": {
+                "unpadded": round(kvc.bytes_resident(cfg, w.entries, w.layers, False) / w.context, 2),
+                "padded": round(kvc.bytes_resident(cfg, w.entries, w.layers, True) / w.context, 2)}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -449,126 +622,19 @@ def run_ours(args):
 
     w0 = synth.WORKLOADS[args.config]
     w = kd.rank_workload(w0, rank)  # each rank decodes its own sequences
-    cfg = kvc.config_for(w)
-    B, L, H = w.batch, w.layers, w.heads
-    N0 = w.entries
-    cap = N0 + args.warmup + args.steps + 64
+    B, L = w.batch, w.layers
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
-
-    # ---- build the cache: pack the whole context on the device (untimed)
-    inp = synth.make_inputs(w, dev)
-    cache = kvc.Cache(cfg, B, cap, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    kvc.pack(cfg, inp["tokens"], inp["gate"], inp["idx_k"], cache, status=status)
-    torch.cuda.synchronize()
-    del inp["tokens"]
-    torch.cuda.empty_cache()
-    gate = inp["gate"]
-    q, idx_q, windows = inp["q"], inp["idx_q"], inp["windows"]
-    ws = kvc.workspace(cfg, B, cap, device=dev, hier_blocks=args.hier, hier_block=args.hier_block)
-    out = torch.empty(L, B, H, w.latent, device=dev)
-    lse = torch.empty(L, B, H, device=dev)
-    topk = torch.empty(L, B, w.topk, dtype=torch.int32, device=dev)
-    nsteps = args.warmup + args.steps
-    newp = synth.make_new_tokens(w, 2 * nsteps, dev)
-    pair_tok = [newp["tokens"][:, 2 * s:2 * s + 2].contiguous() for s in range(nsteps)]
-    pair_idx = [newp["idx_k"][:, s:s + 1].contiguous() for s in range(nsteps)]
-    modes = list(w.modes)
-
-    def step(s):
-        kvc.pack(cfg, pair_tok[s], gate, pair_idx[s], cache, status=status)
-        kvc.layer_group_step(cfg, modes, q, idx_q, windows, w.window, cache, out, topk, ws,
-                             lse=lse, status=status, hier_blocks=args.hier,
-                             hier_block=args.hier_block)
-
-    for s in range(args.warmup):
-        step(s)
-    torch.cuda.synchronize()
-
-    # ---- capture the K timed steps into one graph and replay it once
-    launches0 = kvc.launch_count()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for s in range(args.warmup, nsteps):
-            step(s)
-    launches = kvc.launch_count() - launches0
-    n_before = cache.n_entries.clone()
-    # one untimed replay first (the graph's first launch also uploads it);
-    # the timed replay then starts again from the same context lengths
-    graph.replay()
-    torch.cuda.synchronize()
-    cache.n_entries.copy_(n_before)
-
-    clocks = Clocks(local, enabled=not args.no_clocks)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    kd.barrier()
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    graph.replay()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    kd.barrier()
-    clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    assert status.item() == 0, f"device status {status.item()}"
-    n_after = cache.n_entries.clone()
-    assert torch.all(n_after - n_before == args.steps)
-    del graph
-
-    ms_max = kd.max_over_ranks(ms, device=dev)
-    value = kd.job_throughput(args.steps, B, world, ms_max)
-
-    # ---- the same K steps again, from the same starting length, captured with
-    # a pair of event nodes around every library kernel: per-kernel durations
-    # (the event nodes themselves add time, so this replay is not the headline)
-    cache.n_entries.copy_(n_before)
-    kvc.trace_begin(16 * args.steps + 16)
-    graph2 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph2, stream=stream):
-        for s in range(args.warmup, nsteps):
-            step(s)
-    kvc.trace_end()
-    cache.n_entries.copy_(n_before)
-    graph2.replay()  # untimed: uploads the graph (its event nodes record again below)
-    torch.cuda.synchronize()
-    cache.n_entries.copy_(n_before)
-    kd.barrier()
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    graph2.replay()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    ms_traced = kd.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
-    del graph2
-
-    # per-kernel device times from the event pairs of the traced replay
-    kernels = {}
-    for name in KERNELS:
-        cnt, tot = kvc.trace_kernel(name)
-        if cnt:
-            kernels[name] = {"launches": cnt, "ms_total": round(tot, 4),
-                             "us_avg": round(1e3 * tot / cnt, 2)}
-    n_mean = N0 + args.warmup + (args.steps + 1) / 2.0  # entries visible during the timed steps
-    heads_layers = sum(1 for m in modes if m != 2)
-    per_launch = {
-        "index_scan": B * scan_bytes(w, n_mean),
-        "attn_tc05": B * attn_bytes(w),
-        "attn_simt": B * attn_bytes(w),
-        "pack": B * pack_bytes(w, 1),
-    }
-    dominant = max(kernels, key=lambda k: kernels[k]["ms_total"])
     peak, peak_kind = peaks()
-    dom = kernels[dominant]
-    achieved = per_launch.get(dominant, 0) / (dom["us_avg"] * 1e-6) / 1e9
-    traffic = traffic_for(dominant)
-    roofline = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_kind} hbm_gbs",
-                "bytes_per_launch": int(per_launch.get(dominant, 0)),
-                "traffic": (int(float(traffic["dram_bytes_per_launch"])) if traffic else None)}
-    sb = step_bytes(w, n_mean)
-    step_gbs = sb / (ms_max / args.steps * 1e-3) / 1e9
+
+    m = measure_decode(w, args.steps, args.warmup, dev, stream, args.hier, args.hier_block,
+                       clocks_gpu=None if args.no_clocks else local)
+    cfg, cache, status, ws = m["cfg"], m["cache"], m["status"], m["ws"]
+    out, lse, topk, gate, n_before = m["out"], m["lse"], m["topk"], m["gate"], m["n_before"]
+    modes = list(w.modes)
+    line = workload_line(w, m, args.steps, world, peak, peak_kind)
+    value, ms_max, launches, clk = line["value"], m["ms_max"], m["launches"], m["clocks"]
+    heads_layers = sum(1 for x in modes if x != 2)
 
     # ---- pack throughput on fresh tokens (the batched workload's pack case)
     pack_info = None
@@ -601,48 +667,60 @@ def run_ours(args):
         del pk, pcache
 
     # ---- end to end through the public API with host buffers.  Every step
-    # uploads its inputs from pinned host memory and reads its result (the
-    # attention output and lse) back.  Within a step the queries (2.4 MB,
-    # needed only by the attention) travel on a copy stream while the pack,
-    # the scan and the selection run; the small inputs go up in one copy and
-    # the result comes back in one.  Steps stay serialised: a step starts
-    # after the previous one's result has been read back.
+    # uploads its own inputs (indexer queries, the completed token pair and
+    # its indexer key, the query heads: a new set each step) from pinned host
+    # memory and reads its result (the attention output and lse) back.
+    # Within a step the queries (needed only by the attention) travel on a
+    # copy stream while the pack, the scan and the selection run; the small
+    # inputs go up in one copy and the result comes back in one.  Steps stay
+    # serialised: a step starts after the previous one's result is read back.
     e2e = None
     if not args.no_e2e:
-        def staged(parts):
-            """One pinned host buffer and one device buffer holding the tensors
-            `parts` back to back (16-byte aligned); returns them and the views."""
+        def staged(parts, n_host=1):
+            """n_host pinned host buffers and one device buffer, each holding
+            tensors shaped like `parts` back to back (16-byte aligned); returns
+            them and their views."""
             sizes = [(t.numel() * t.element_size() + 15) // 16 * 16 for t in parts]
-            host = torch.empty(sum(sizes), dtype=torch.uint8).pin_memory()
-            devb = torch.empty(sum(sizes), dtype=torch.uint8, device=dev)
-            hv, dv, off = [], [], 0
-            for t, n in zip(parts, sizes):
-                nb = t.numel() * t.element_size()
-                hv.append(host[off:off + nb].view(t.dtype).view(t.shape))
-                dv.append(devb[off:off + nb].view(t.dtype).view(t.shape))
-                off += n
-            return host, devb, hv, dv
 
-        hin, din, (h_iq, h_tok, h_idx), (diq, dtok, didx) = staged(
-            [idx_q, newp["tokens"][:, :2], newp["idx_k"][:, :1]])
-        h_iq.copy_(idx_q)
-        h_tok.copy_(newp["tokens"][:, :2])
-        h_idx.copy_(newp["idx_k"][:, :1])
-        hq = q.cpu().pin_memory()
-        dq = torch.empty_like(q)
-        hres, dres, (h_out, h_lse), (d_out, d_lse) = staged([out, lse])
+            def views(buf):
+                v, off = [], 0
+                for t, n in zip(parts, sizes):
+                    nb = t.numel() * t.element_size()
+                    v.append(buf[off:off + nb].view(t.dtype).view(t.shape))
+                    off += n
+                return v
+            hosts = [torch.empty(sum(sizes), dtype=torch.uint8).pin_memory()
+                     for _ in range(n_host)]
+            devb = torch.empty(sum(sizes), dtype=torch.uint8, device=dev)
+            return hosts, devb, [views(h) for h in hosts], views(devb)
+
+        reps = args.steps
+        sets, newp = m["sets"], m["newp"]
+        nsteps = args.warmup + args.steps
+        step_ids = [args.warmup + (s % args.steps) for s in range(reps + 1)]
+        hins, din, hviews, (diq, dtok, didx) = staged(
+            [sets[0]["idx_q"], newp["tokens"][:, :2], newp["idx_k"][:, :1]], n_host=reps + 1)
+        hqs = []
+        for r, s in enumerate(step_ids):
+            h_iq, h_tok, h_idx = hviews[r]
+            h_iq.copy_(sets[s]["idx_q"])
+            h_tok.copy_(newp["tokens"][:, 2 * s:2 * s + 2])
+            h_idx.copy_(newp["idx_k"][:, s:s + 1])
+            hqs.append(sets[s]["q"].cpu().pin_memory())
+        dq = torch.empty_like(sets[0]["q"])
+        (hres,), dres, ((h_out, h_lse),), (d_out, d_lse) = staged([out, lse])
         copy_stream = torch.cuda.Stream(device=dev)
         q_ready = torch.cuda.Event()
         split = modes == [synth.FULL] and args.hier == 0
-        reps = args.steps
         cache.n_entries.copy_(n_before)
 
-        def e2e_step():
+        def e2e_step(r):
+            windows = sets[step_ids[r]]["windows"]  # the windows stay on the device
             copy_stream.wait_stream(stream)  # the previous step no longer reads dq
             with torch.cuda.stream(copy_stream):
-                dq.copy_(hq, non_blocking=True)
+                dq.copy_(hqs[r], non_blocking=True)
                 q_ready.record(copy_stream)
-            din.copy_(hin, non_blocking=True)
+            din.copy_(hins[r], non_blocking=True)
             kvc.pack(cfg, dtok, gate, didx, cache, status=status)
             if split:  # one Full layer: its scan and selection need no queries
                 kvc.index_topk(cfg, diq[0], cache, topk[0], ws, status=status)
@@ -656,44 +734,59 @@ def run_ours(args):
                                      hier_block=args.hier_block)
             hres.copy_(dres, non_blocking=True)
 
-        e2e_step()
+        e2e_step(reps)  # warm-up with the spare input set
         torch.cuda.synchronize()
         cache.n_entries.copy_(n_before)
         kd.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(reps):
-            e2e_step()
+        for r in range(reps):
+            e2e_step(r)
         e1.record(stream)
         torch.cuda.synchronize()
         te_ms = kd.max_over_ranks(e0.elapsed_time(e1), device=dev)
         assert status.item() == 0, f"device status {status.item()}"
-        h2d = sum(t.numel() * t.element_size() for t in (hq, h_iq, h_tok, h_idx))
+        h2d = (sum(t.numel() * t.element_size() for t in hviews[0])
+               + hqs[0].numel() * hqs[0].element_size())
         d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse))
         e2e = {"value": round(kd.job_throughput(reps, B, world, te_ms), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(te_ms / reps, 4),
+               "inputs": "a new query set uploaded every step",
                "api": ("kvc_pack, kvc_index_topk, kvc_sparse_decode_attn" if split else
                        "kvc_pack, kvc_layer_group_step"),
                "overlap": "query upload on a copy stream during pack, scan and selection"
                           if split else "none"}
+        del hins, hqs
 
-    # ---- the hierarchical indexer (2048 blocks of 8) on the CSA2 group and the
-    # 1M-token stack, against the plain group step (device time per step)
-    extra = None
+    # ---- the CSA2 group (8 x 256K, Full/Reindex/Reuse/Reuse) and the 1M-token
+    # 20-layer stack measured like the headline (pack + layer group, a new
+    # query set per step), and again with the hierarchical indexer (2048
+    # blocks of 8)
+    extra, workloads = None, None
     if not args.no_extra and world == 1 and args.hier == 0:
+        del m
         torch.cuda.empty_cache()
-        extra = {}
+        extra, workloads = {}, {}
         for name in ("csa2group", "stack1m"):
             wx = synth.WORKLOADS[name]
-            plain = time_group(wx, 10, 3, 0, 8, dev)
-            hier = time_group(wx, 10, 3, 2048, 8, dev)
-            extra[name] = {"ms_per_step_plain": round(plain, 4), "ms_per_step_hier": round(hier, 4),
-                           "query_tokens_per_s_plain": round(wx.batch / (plain * 1e-3), 1),
-                           "query_tokens_per_s_hier": round(wx.batch / (hier * 1e-3), 1),
-                           "hier": "2048 blocks of 8 entries"}
+            mx = measure_decode(wx, 10, 3, dev, stream)
+            lx = workload_line(wx, mx, 10, 1, peak, peak_kind)
+            lx["steps"], lx["warmup"] = 10, 3
+            lx["config"] = {"batch": wx.batch, "context_tokens": wx.context,
+                            "entries": wx.entries, "group": wx.group,
+                            "layers": [["Full", "Reindex", "Reuse"][x] for x in wx.modes]}
+            del mx
             torch.cuda.empty_cache()
+            mh = measure_decode(wx, 10, 3, dev, stream, 2048, 8)
+            lx["hier_indexer_2048x8"] = {
+                "value": round(kd.job_throughput(10, wx.batch, 1, mh["ms_max"]), 1),
+                "ms_per_step": round(mh["ms_max"] / 10, 4)}
+            del mh
+            torch.cuda.empty_cache()
+            workloads[name] = lx
+            extra[name] = {}
         # every scoring layer's indexer query in one tensor-core pass, against
         # one scan per layer (a schedule where all queries are known up front)
         for name in ("csa2group", "stack1m"):
@@ -741,33 +834,33 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_max / args.steps, 4),
-        "ms_per_step_traced": round(ms_traced / args.steps, 4), "higher_is_better": True,
+        "ms_per_step_traced": line["ms_per_step_traced"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.act == "bf16" else "f32",
         "data": "synthetic (seeded; no weights or datasets)",
         "config": {"workload": w.name, "batch_per_gpu": B, "context_tokens": w.context,
-                   "entries": N0, "layers": [["Full", "Reindex", "Reuse"][m] for m in modes],
-                   "heads": H, "latent": w.latent, "rope": w.rope, "group": w.group,
+                   "entries": w.entries, "layers": [["Full", "Reindex", "Reuse"][x] for x in modes],
+                   "heads": w.heads, "latent": w.latent, "rope": w.rope, "group": w.group,
                    "scale": "ue4m3" if w.scale_fmt == 1 else "f32", "topk": w.topk,
                    "window": w.window, "idx_dim": w.idx_dim, "parallelism": f"dp{world}",
                    "hier_indexer": (f"{args.hier} blocks of {args.hier_block}" if args.hier
                                     else "off"),
+                   "inputs": "a new set of queries, indexer queries and windows every step",
                    "l2": "inputs larger than L2 (indexer scan reads %.0f MB per step)"
-                         % (B * scan_bytes(w, N0) * heads_layers / 1e6),
+                         % (B * scan_bytes(w, w.entries) * heads_layers / 1e6),
                    "timing": "K steps in one CUDA graph, CUDA events, max over ranks; "
                              "per-kernel times from a second replay with event nodes"},
-        "hbm_gbs_step": round(step_gbs, 1),
-        "step_frac_of_peak": round(step_gbs / peak, 4),
-        "step_bytes": int(sb),
-        "roofline": roofline,
-        "kernels": kernels,
+        "hbm_gbs_step": line["hbm_gbs_step"],
+        "step_frac_of_peak": line["step_frac_of_peak"],
+        "step_bytes": line["step_bytes"],
+        "roofline": line["roofline"],
+        "kernels": line["kernels"],
         "pack": pack_info,
-        "bytes_resident_per_token": {
-            "unpadded": round(kvc.bytes_resident(cfg, N0, L, False) / w.context, 2),
-            "padded": round(kvc.bytes_resident(cfg, N0, L, True) / w.context, 2)},
+        "bytes_resident_per_token": line["bytes_resident_per_token"],
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clk,
+        "workloads": workloads,
         "next_rows": extra,
     }
     if rank == 0:

@@ -151,3 +151,23 @@ def make_new_tokens(w: Workload, n_new: int, device="cpu", seed_offset: int = 7)
     idx_k = torch.randint(-127, 128, (w.batch, n_new // w.ratio, w.idx_dim), generator=gen,
                           device=device, dtype=torch.int8)
     return {"tokens": tokens, "idx_k": idx_k}
+
+
+def make_step_inputs(w: Workload, n_steps: int, device="cpu", seed_offset: int = 13) -> list:
+    """Distinct per-step decode inputs: for each of n_steps steps a fresh
+    indexer query, query heads and window per layer (same shapes and
+    distributions as make_inputs).  A real decode step brings new queries and
+    so a new top-K selection every step; drawing them anew keeps a timed loop
+    from re-reading one step's gathered rows out of L2."""
+    gen = generator(device, w.seed * 1000 + seed_offset)
+    L, B, D = w.layers, w.batch, w.dim
+    sets = []
+    for _ in range(n_steps):
+        sets.append({
+            "idx_q": torch.randint(-127, 128, (L, B, w.idx_dim), generator=gen, device=device,
+                                   dtype=torch.int8),
+            "q": torch.randn(L, B, w.heads, D, generator=gen, device=device,
+                             dtype=torch.float32).to(w.torch_dtype),
+            "windows": _keys(w, (L, B, w.window), gen, device).contiguous(),
+        })
+    return sets

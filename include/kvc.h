@@ -139,7 +139,8 @@ size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity);
 /* Append n_new raw tokens per sequence (A1-A3 of the hot path).
  * tokens    [batch][n_new][D] act_dtype; n_new a multiple of r = cfg->ratio:
  *           tokens r i .. r i + r - 1 are compressed into entry i ([A]
- *           breakthrough 4 "CSA 把每 2 个 token 的 KV 压成 1 条"; [B] 3.2; the
+ *           breakthrough 4: the trained compressor merges every two tokens
+ *           into one cache entry; [B] 3.2; the
  *           ratio 4 of [B] 4.3).  The tokens' weights are the softmax of their
  *           gate logits g.k; the weighted sum is quantised per group to E2M1
  *           with scale absmax/6 ([B] 3.1; [A] "P4 main KV").
@@ -156,8 +157,8 @@ kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,
                     const float* gate, const int8_t* idx_k_new,
                     const kvc_cache* cache, uint32_t* dev_status, void* stream);
 
-/* Indexer scoring and exact top-K (A4-A5; [A] breakthrough 4 "用一个轻量索引器
- * 给所有历史 token 打分，只挑分数最高的 512 个"; part 4 "CSA2").
+/* Indexer scoring and exact top-K (A4-A5; [A] breakthrough 4: a light indexer
+ * scores every stored entry and the 512 best are attended; part 4 "CSA2").
  * idx_q     [batch][idx_dim] int8 indexer queries.
  * score_j = sum_d idx_q[d] * idx_k[j][d] in int32 over the visible entries.
  * topk_idx  [batch][topk] int32 out: the topk highest scores, ties to the lower

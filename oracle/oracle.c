@@ -22,8 +22,9 @@
  *  R1 gate: one D-vector g gives one logit per token; the pair's weights are
  *     the softmax of the two logits.  The pages fix no precision for this
  *     step; the quantised codes downstream depend on the exact fp32 entry, so
- *     it is evaluated in fp32 in a fixed order (8 partial sums over 8-channel
- *     chunks, then a xor tree), the precision and order the GPU kernel uses.
+ *     the specification fixes one: fp32, the channels dealt round-robin in
+ *     chunks of 8 to 8 running sums (chunk c to sum c mod 8), the 8 sums
+ *     combined pairwise at distances 4, 2, 1.
  *  R2 exp: written here in fp32 from the Cody-Waite argument reduction and a
  *     degree-7 Taylor polynomial (Horner form), so that the gate weight is the
  *     same bits on every implementation of this specification.
@@ -44,11 +45,15 @@
  *
  * Pins: every function is checked by the not-gpu tests against what the
  * pages or the mathematics fix (printed values, closed forms, brute force,
- * library routines).  orc_compress_pair and orc_compress_group4 are pinned
- * only by invariants (identical tokens, zero gate, a dominant token,
- * convexity, fp64 softmax weights); their exact fp32 operation order is a
- * reading (R1, R17), so beyond those invariants they are "parity unpinned"
- * by the pages, and the GPU is held to them by following the same order.
+ * library routines).  orc_compress_pair and orc_compress_group4 are pinned by
+ * invariants (identical tokens, zero gate, a dominant token, convexity) and
+ * by an fp64 evaluation of the compression that shares none of this order:
+ * every entry lies within a derived error bound of the exact softmax-weighted
+ * sum, and the packed records equal those of the fp64 entry rounded once to
+ * fp32 except for codes or scales whose quotient straddles a rounding
+ * midpoint within that bound (about 5e-7 of the codes).  Only the choice of
+ * the fp32 order itself (R1, R17) is a reading; the GPU follows the same one
+ * so that its records match the oracle's bit for bit.
  *
  * Compile with -ffp-contract=off: every fused multiply-add below is an
  * explicit fma() call and nothing else may be contracted.
@@ -254,8 +259,9 @@ static int orc_groups(const orc_cfg* c, int* start, int* len) {
 }
 
 /* ------------------------------------------------------------------ */
-/* R1: the 2:1 compression of a token pair ([P2] breakthrough 4 "CSA 把每 2
- * 个 token 的 KV 压成 1 条"; [P1] 3.2 "main key compressor").
+/* R1: the 2:1 compression of a token pair ([P2] breakthrough 4: a trained
+ * compressor turns every two tokens into one entry; [P1] 3.2: the key
+ * compressor of CSA2).
  * logit_t = g . k_t; (w0, w1) = softmax(logit_0, logit_1);
  * entry = w0 k_0 + w1 k_1, everything in fp32.
  * Fixed evaluation order: delta = logit_0 - logit_1 = sum_d g_d (k0_d - k1_d)
@@ -457,7 +463,7 @@ static int orc_int_asc(const void* pa, const void* pb) {
     return (a > b) - (a < b);
 }
 
-/* Top-K ([P2] breakthrough 4 "只挑分数最高的 512 个"): order all n
+/* Top-K ([P2] breakthrough 4: only the 512 best-scored entries are kept): order all n
  * entries by (score descending, index ascending), keep the first
  * min(k, n), write them sorted by index ascending and pad with -1.
  * Returns the number kept.                                              */
