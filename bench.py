@@ -37,7 +37,7 @@ METRIC = "sparse FP4-KV decode query-tokens/s; achieved HBM GB/s vs 8 TB/s"
 UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 KERNELS = ("pack", "pack_commit", "index_scan", "index_scan_tc", "topk_select", "block_max",
-           "copy_topk", "attn_tc05", "attn_simt", "attn_merge")
+           "copy_topk", "attn_t128", "attn_simt", "attn_merge")
 
 
 def parse():
@@ -558,7 +558,7 @@ def measure_decode(w, steps, warmup, dev, stream, hier=0, hier_block=8, clocks_g
 def kernel_bytes(w, n_mean):
     """Algorithmic bytes per launch of the kernels whose work has a byte count."""
     return {"index_scan": w.batch * scan_bytes(w, n_mean),
-            "attn_tc05": w.batch * attn_bytes(w),
+            "attn_t128": w.batch * attn_bytes(w),
             "attn_simt": w.batch * attn_bytes(w),
             "pack": w.batch * pack_bytes(w, 1)}
 

@@ -10,7 +10,7 @@
 // softmax runs jointly over the selected entries and the window keys.
 //
 // Kernels
-//  attn_tc05  (attn_tc05.cu) tensor-core path for 64 heads x 576 (512 latent)
+//  attn_t128  (attn_t128.cu) tensor-core path for 64 heads x 576 (512 latent)
 //             bf16 entries.
 //  attn_simt  generic fp32 / bf16 path for other shapes (one warp per head).
 //  attn_merge combines the per-split (max, sum, O) partials by log-sum-exp.
@@ -218,8 +218,8 @@ __global__ void copy_topk_kernel(const int32_t* __restrict__ src, int32_t* __res
 
 }  // namespace
 
-bool tc05_supported(const kvc_config& c, const Shape& sh);
-int launch_attention_tc05(const kvc_config& c, const Shape& sh, const AttnArgs& a, cudaStream_t s);
+bool t128_supported(const kvc_config& c, const Shape& sh);
+int launch_attention_t128(const kvc_config& c, const Shape& sh, const AttnArgs& a, cudaStream_t s);
 
 cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArgs& a,
                              cudaStream_t s) {
@@ -234,8 +234,8 @@ cudaError_t launch_attention(const kvc_config& c, const Shape& sh, const AttnArg
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaError_t err = cudaSuccess;
     int nsplit;
-    if (tc05_supported(c, sh)) {
-        nsplit = launch_attention_tc05(c, sh, a, s);
+    if (t128_supported(c, sh)) {
+        nsplit = launch_attention_t128(c, sh, a, s);
         if (nsplit < 0) return cudaErrorLaunchFailure;
     } else {
         const int nchunks = (total + kSimtChunk - 1) / kSimtChunk;

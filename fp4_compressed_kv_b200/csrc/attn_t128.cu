@@ -1,0 +1,872 @@
+// attn_t128.cu -- sparse decode attention on the 5th-generation tensor cores
+// for the MLA shape: 64 query heads sharing 576-channel entries (512 latent +
+// 64 RoPE), values = the latent channels.
+//
+// Method: "DeepSeek V1 到 V4.1-Flash，单 token 的 global KV 如何从 389,000 B
+// 压缩到 890 B的？" (acejoy.com) part 3 breakthrough 2 (every head reads the
+// same latent entry, up-projections absorbed), breakthrough 4 (the 512
+// selected entries plus a 128-token window), part 4 "P4 main KV" (FP4 is
+// dequantised before attention).  One softmax runs jointly over the selected
+// entries and the window keys.
+//
+// The key axis is the MMA's M dimension: a chunk of 128 keys against all 64
+// heads is one M = 128, N = 64 product, with no padding rows.
+//  1. A CTA owns either record chunks or the window chunk of one sequence.
+//     Record chunks run with f16 operands: every dequantised entry is exact in
+//     f16, and each head's query row is scaled by a power of two into the f16
+//     range (the softmax undoes it).  The window chunk runs with bf16
+//     operands: its query tile and key rows arrive by TMA (128B-swizzled
+//     boxes) without passing through registers.  FP8 window rows are decoded
+//     to their exact E4M3 values; each row's scale is applied to its logits
+//     and to its probabilities, not to the stored tile.
+//  2. A record chunk's keys are written into a 128B-swizzled K tile (9 atoms
+//     of 64 channels x 128 keys): the selected records are loaded into
+//     registers (16-byte loads, all in flight while the query tile is
+//     converted), their E2M1 codes converted in hardware and multiplied by
+//     the f16 group scale.  Thread = (key, half row): a warp's 16-byte stores
+//     cover 8 swizzle slots x 4 rows, the minimum 4 wavefronts.
+//  3. One thread issues S^T = K Q^T: 36 tcgen05.mma (M = 128 keys, N = 64
+//     heads, K = 16) into tensor memory.
+//  4. Warps 0-3 (thread = key = tensor-memory lane) read their key's 64
+//     scores, take each head's chunk maximum with warp max-reductions, move a
+//     head's reference only when its maximum passes it by more than 2^8 (the
+//     accumulated O^T is rescaled in tensor memory then), and write P^T (key
+//     rows of 64 heads) over the RoPE atom of the K tile, which the QK product
+//     no longer reads.  Row sums are column sums of that same rounded P^T.
+//  5. One thread issues O^T += V^T P^T: the latent atoms of the K tile read as
+//     an MN-major operand, 4 x 8 tcgen05.mma (M = 128 channels, N = 64 heads,
+//     K = 16 keys) into tensor memory.  A second record chunk's loads are in
+//     flight while this product runs.
+//  6. The CTAs of a sequence (at most 8) form a thread-block cluster: each
+//     stores its unnormalised O and (m, l) (they stay in L2), one cluster
+//     barrier orders the stores, and CTA r pulls the rows of heads
+//     [r*64/n, (r+1)*64/n) from every CTA into its freed K tile with bulk
+//     copies and combines them.  More CTAs per sequence: attn_merge.
+// Every wait on an mbarrier is bounded; on expiry the CTA sets
+// KVC_DEV_TIMEOUT, waits (bounded) for the copies and products it issued,
+// frees its tensor memory and returns.
+#include <algorithm>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <mutex>
+
+#include "kvc_internal.cuh"
+#include "tc05_common.cuh"
+
+namespace kvc {
+namespace t128 {
+
+using namespace tc;
+
+constexpr int H = 64, D = 576, DV = 512, CK = 128, NT = 256;
+constexpr int NATOM = D / 64;                        // 9 channel atoms of 64
+constexpr uint32_t Q_ATOM = H * 128;                 // 64 rows x 128 B
+constexpr uint32_t K_ATOM = CK * 128;                // 128 rows x 128 B
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + NATOM * Q_ATOM;   // 73,728
+constexpr uint32_t OFF_P = OFF_K + 8 * K_ATOM;       // the RoPE atom, P^T after QK
+constexpr uint32_t OFF_MISC = OFF_K + NATOM * K_ATOM;  // 221,184
+// misc: kidx[128] i32 | qs[64] | mref[64] | lrun[64] | fac[64] | wmax[4][64] |
+//       lpart[8][64] | ks[128] | bars[4] u64 | tmem slot | flags
+constexpr uint32_t M_KIDX = 0, M_QS = 512, M_MREF = 768, M_LRUN = 1024, M_FAC = 1280,
+                   M_WMAX = 1536, M_LPART = 2560, M_KS = 4608, M_BARS = 5120, M_TSLOT = 5152,
+                   M_FLAGS = 5168, MISC_BYTES = 5248;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL = 0, O_COL = 256;           // S^T: 64 cols; O^T: 4 tiles x 64 cols
+constexpr float kRescaleSlack = 8.0f;                // log2 units
+enum { BAR_S = 0, BAR_O = 1, BAR_Q = 2, BAR_W = 3 };
+
+// ---- TMA and bulk copies (non-multicast, into this CTA's shared memory)
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+// Q tile (64 heads x 576 channels, 9 boxes of 64 channels) of sequence b.
+__device__ __forceinline__ void tma_q(const CUtensorMap* map, uint32_t sQ, int b, uint32_t bar) {
+    mbar_expect_tx(bar, NATOM * Q_ATOM);
+    for (int at = 0; at < NATOM; ++at) tma_load_2d(sQ + at * Q_ATOM, map, 64 * at, b * H, bar);
+}
+
+// The query rows of a record CTA in registers: thread t holds head t/4,
+// channels [144 (t%4), +144) as 18 16-byte pieces.
+__device__ __forceinline__ void load_q_regs(const AttnArgs& a, int b, int tid, uint4 (&v)[18]) {
+    const int h = tid >> 2, qq = tid & 3;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(a.q) +
+                                                      ((size_t)b * H + h) * D * 2) + 18 * qq;
+#pragma unroll
+    for (int i = 0; i < 18; ++i) v[i] = __ldg(src + i);
+}
+// bf16 -> f16 with a per-head power of two that puts the row maximum in
+// [2^14, 2^15); the head's softmax multiplier qs[h] absorbs it.
+__device__ __forceinline__ void store_q_f16(const AttnArgs& a, const uint4 (&v)[18], float sm_log2,
+                                            uint32_t sQ, float* qs, int tid) {
+    const int h = tid >> 2, qq = tid & 3;
+    uint32_t amax = 0;  // max |x| as fp32 bits (integer order = float order)
+#pragma unroll
+    for (int i = 0; i < 18; ++i) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            amax = max(amax, (w[k] << 16) & 0x7FFFFFFFu);
+            amax = max(amax, w[k] & 0x7FFF0000u);
+        }
+    }
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    int k = 0;
+    if (amax >= 0x7F800000u) {
+        if (qq == 0) set_status(a.status, KVC_DEV_NONFINITE);
+    } else if (amax != 0) {
+        const int e = (int)(amax >> 23) - 127;  // floor(log2 amax) for normal values
+        k = min(max(e - 14, -60), 113);
+    }
+    const float mul = __uint_as_float((uint32_t)(127 - k) << 23);
+    if (qq == 0) qs[h] = sm_log2 * __uint_as_float((uint32_t)(127 + k) << 23);
+#pragma unroll
+    for (int i = 0; i < 18; ++i) {
+        const int c16 = 18 * qq + i;  // 16-byte chunk of the row: channels 8 c16 .. +7
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = pack_f16(__uint_as_float(w[j] << 16) * mul,
+                            __uint_as_float(w[j] & 0xFFFF0000u) * mul);
+        sts128(sQ + (c16 >> 3) * Q_ATOM + swz(h, c16 & 7), o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Scale byte index of 8-channel piece (item i, word u) for groups of G:
+// latent items 0..15, RoPE items 16..17 (groups restart at channel 512).
+template <int G>
+__device__ __host__ constexpr int scale_index(int i, int u) {
+    return i < 16 ? (32 * i + 8 * u) / G : 512 / G + (32 * (i - 16) + 8 * u) / G;
+}
+template <int G>
+constexpr int scale_vecs() {  // 16-byte loads covering the scale bytes
+    return (512 / G + (64 + G - 1) / G + 15) / 16;
+}
+
+// One record's half row (half 0: channels 0..287, half 1: 288..575) in
+// registers: 9 pieces of codes and the scale bytes.
+template <int G>
+struct RowRegs {
+    uint4 cw[9];
+    uint4 sv[scale_vecs<G>()];
+};
+template <int G>
+__device__ __forceinline__ void load_row(const uint8_t* rec, int half, RowRegs<G>& r) {
+#pragma unroll
+    for (int u = 0; u < 9; ++u) r.cw[u] = ldg_nc(rec + (9 * half + u) * 16);
+#pragma unroll
+    for (int u = 0; u < scale_vecs<G>(); ++u) r.sv[u] = ldg_nc(rec + 288 + 16 * u);
+}
+// ... dequantised into the K tile: codes times the f16 group scale, exact.
+template <int G, int HALF>
+__device__ __forceinline__ void store_row(const RowRegs<G>& r, uint32_t sK, int s) {
+    constexpr int NS = scale_vecs<G>();
+    uint32_t sb[4 * NS];
+#pragma unroll
+    for (int u = 0; u < NS; ++u) {
+        sb[4 * u] = r.sv[u].x;
+        sb[4 * u + 1] = r.sv[u].y;
+        sb[4 * u + 2] = r.sv[u].z;
+        sb[4 * u + 3] = r.sv[u].w;
+    }
+#pragma unroll
+    for (int u = 0; u < 9; ++u) {
+        const int i = 9 * HALF + u;  // 32-channel item
+        const uint32_t words[4] = {r.cw[u].x, r.cw[u].y, r.cw[u].z, r.cw[u].w};
+        const uint32_t row = sK + (uint32_t)(i >> 1) * K_ATOM;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int si = scale_index<G>(i, k);
+            const uint32_t byte = (sb[si >> 2] >> (8 * (si & 3))) & 0xFFu;
+            uint32_t w[4];
+            e2m1x8_scaled(words[k], ue4m3_f16x2(byte), w);
+            sts128(row + swz(s, 4 * (i & 1) + k), w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+__device__ __forceinline__ void zero_row_half(uint32_t sK, int s, int half) {
+#pragma unroll 1
+    for (int c16 = 36 * half; c16 < 36 * half + 36; ++c16)
+        sts128(sK + (uint32_t)(c16 >> 3) * K_ATOM + swz(s, c16 & 7), 0u, 0u, 0u, 0u);
+}
+
+template <int G>
+__global__ void __launch_bounds__(NT, 1)
+attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_w,
+                 AttnArgs a, Shape sh, int K, float sm_log2, int rsplit, int cpr, int nsplit,
+                 int cluster, unsigned long long wait_ns) {
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;  // 1024-byte alignment for the swizzle
+    unsigned char* smem = smem_raw + (base - raw_base);
+    const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sP = base + OFF_P;
+    unsigned char* misc = smem + OFF_MISC;
+    int* kidx = reinterpret_cast<int*>(misc + M_KIDX);
+    float* qs = reinterpret_cast<float*>(misc + M_QS);
+    float* mref = reinterpret_cast<float*>(misc + M_MREF);
+    float* lrun = reinterpret_cast<float*>(misc + M_LRUN);
+    float* fac = reinterpret_cast<float*>(misc + M_FAC);
+    int* wmax = reinterpret_cast<int*>(misc + M_WMAX);
+    float* lpart = reinterpret_cast<float*>(misc + M_LPART);
+    float* ks = reinterpret_cast<float*>(misc + M_KS);  // FP8 window: scale of each key row
+    uint64_t* bars = reinterpret_cast<uint64_t*>(misc + M_BARS);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + M_TSLOT);
+    int* flags = reinterpret_cast<int*>(misc + M_FLAGS);
+    const uint32_t bS = smem_u32(&bars[BAR_S]), bO = smem_u32(&bars[BAR_O]),
+                   bQ = smem_u32(&bars[BAR_Q]), bW = smem_u32(&bars[BAR_W]);
+
+    const int b = blockIdx.y, split = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int W = a.window_len;
+    const int rc = (K + CK - 1) / CK;
+    // this CTA's chunks: record chunks [c0, c1) or window chunk split - rsplit
+    const bool win = split >= rsplit;
+    const bool fp8 = win && a.win_fp8 != nullptr;
+    const int c0 = win ? split - rsplit : split * cpr;
+    const int c1 = win ? min(c0 + 1, (W + CK - 1) / CK) : min(c0 + cpr, rc);
+    const uint32_t idQK = idesc_f16(128, 64, win ? 1 : 0, 0, 0);
+    const uint32_t idPV = idesc_f16(128, 64, win ? 1 : 0, 1, 1);
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bars[i]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (tid < H) {
+        mref[tid] = -INFINITY;
+        lrun[tid] = 0.f;
+        if (win) qs[tid] = sm_log2;
+    }
+    __syncthreads();  // barriers initialised before any copy arrives on them
+    // The query tile: read before the wait when no kernel launched since the
+    // caller wrote q (inside a layer-group step), else after it.
+    uint4 qv[18];
+    if (a.q_ready) {
+        if (win) {
+            if (tid == 0) tma_q(&tm_q, sQ, b, bQ);
+        } else {
+            load_q_regs(a, b, tid, qv);
+        }
+    }
+    pdl_wait();
+    const int n = a.n_entries[b];
+    const bool len_ok = n >= 0 && n <= a.capacity;
+    if (!a.q_ready) {
+        if (win) {
+            if (tid == 0) tma_q(&tm_q, sQ, b, bQ);
+        } else {
+            load_q_regs(a, b, tid, qv);
+        }
+    }
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    int nqk = 0, npv = 0, nw = 0;  // commits / copies issued (for the cleanup waits)
+    const int s = tid & (CK - 1), half = tid >> 7;  // this thread's key and half row
+    // ---- slot table of chunk c: record index, window row, or -1 (masked)
+    auto slot_table = [&](int c) {
+        if (tid < CK) {
+            int k = -1;
+            if (!win) {
+                const int j = c * CK + tid;
+                if (j < K) {
+                    const int idx = a.topk_idx[(size_t)b * K + j];
+                    if (a.topk_copy) a.topk_copy[(size_t)b * K + j] = idx;
+                    if (len_ok && idx >= 0 && idx < n)
+                        k = idx;
+                    else if (idx != -1 && len_ok)
+                        set_status(a.status, KVC_DEV_BAD_INDEX);
+                }
+            } else {
+                const int r = c * CK + tid;
+                if (r < W) k = r;
+                if (fp8) ks[tid] = k >= 0 ? __ldg(a.win_scale + (size_t)b * a.window_stride + r) : 0.f;
+            }
+            kidx[tid] = k;
+        }
+        __syncthreads();
+        return kidx[s];
+    };
+    // ---- record rows into registers: in flight while the query tile is
+    // converted (first chunk) or while the previous chunk's PV runs
+    RowRegs<G> rr;
+    int k = -1;
+    if (c0 < c1) {
+        k = slot_table(c0);
+        if (!win && k >= 0) load_row<G>(a.records + ((size_t)b * a.capacity + k) * sh.rb, half, rr);
+    }
+    if (!win) store_q_f16(a, qv, sm_log2, sQ, qs, tid);
+
+    for (int c = c0; c < c1 && ok; ++c) {
+        const int it = c - c0;
+        if (it > 0) {
+            k = slot_table(c);
+            if (!win && k >= 0)
+                load_row<G>(a.records + ((size_t)b * a.capacity + k) * sh.rb, half, rr);
+        }
+        if (win && !fp8) {
+            // the window rows of this chunk by TMA: 9 boxes of 64 channels x 128 rows
+            if (tid == 0) {
+                mbar_expect_tx(bW, NATOM * K_ATOM);
+                for (int at = 0; at < NATOM; ++at)
+                    tma_load_2d(sK + at * K_ATOM, &tm_w, 64 * at, b * a.window_stride + c * CK, bW);
+            }
+            ++nw;
+        }
+        // ---- the K tile is free once the previous chunk's PV is done
+        if (it > 0) {
+            const bool got = warp == 0 ? mbar_wait(bO, (it - 1) & 1, wait_ns) : true;
+            ok = __syncthreads_and(got) != 0;
+            if (!ok) break;
+            tc_fence_after();
+        }
+        // ---- fill the K tile
+        if (!win) {
+            if (k < 0)
+                zero_row_half(sK, s, half);
+            else if (half == 0)
+                store_row<G, 0>(rr, sK, s);
+            else
+                store_row<G, 1>(rr, sK, s);
+        } else if (fp8) {
+            // signed E4M3 codes decoded exactly to bf16 (the row scale is
+            // applied to the logits and to the probabilities)
+            if (k < 0) {
+                zero_row_half(sK, s, half);
+            } else {
+                const uint8_t* src = a.win_fp8 + ((size_t)b * a.window_stride + k) * D + 288 * half;
+                uint4 v[18];
+#pragma unroll
+                for (int u = 0; u < 18; ++u) v[u] = ldg_nc(src + 16 * u);
+#pragma unroll
+                for (int u = 0; u < 18; ++u) {
+                    const uint32_t words[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t h0, h1;
+                        asm("{\n\t.reg .b16 lo, hi;\n\t"
+                            "mov.b32 {lo, hi}, %2;\n\t"
+                            "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+                            "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+                            : "=r"(h0), "=r"(h1)
+                            : "r"(words[q]));
+                        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+                        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+                        o[2 * q] = pack_bf16(f0.x, f0.y);  // exact: E4M3 has 4 significant bits
+                        o[2 * q + 1] = pack_bf16(f1.x, f1.y);
+                    }
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const int c16 = 36 * half + 2 * u + p;
+                        sts128(sK + (uint32_t)(c16 >> 3) * K_ATOM + swz(s, c16 & 7), o[4 * p],
+                               o[4 * p + 1], o[4 * p + 2], o[4 * p + 3]);
+                    }
+                }
+            }
+        } else {
+            // the TMA rows must have landed; masked rows are then zeroed (a
+            // box past the window reads other rows, or zeros past the tensor)
+            const bool got = warp == 0 ? mbar_wait(bW, (nw - 1) & 1, wait_ns) : true;
+            ok = __syncthreads_and(got) != 0;
+            if (!ok) break;
+            if (k < 0) zero_row_half(sK, s, half);
+        }
+        if (win && it == 0) {  // the query tile's TMA
+            const bool got = warp == 0 ? mbar_wait(bQ, 0, wait_ns) : true;
+            ok = __syncthreads_and(got) != 0;
+            if (!ok) break;
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- S^T = K Q^T (one thread issues)
+        if (tid == 0) {
+            tc_fence_after();
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t at = kk >> 2, koff = (kk & 3) * 32;
+                mma_f16(tmem + S_COL, sdesc(sK + at * K_ATOM + koff, 16, 1024),
+                        sdesc(sQ + at * Q_ATOM + koff, 16, 1024), idQK, kk > 0);
+            }
+            mma_commit(bS);
+        }
+        ++nqk;
+        {
+            const bool got = warp == 0 ? mbar_wait(bS, it & 1, wait_ns) : true;
+            ok = __syncthreads_and(got) != 0;
+        }
+        tc_fence_after();
+        if (!ok) break;
+
+        // ---- softmax, warps 0-3: thread = key = tensor-memory lane.  y is
+        // the raw logit (times the FP8 row scale); x = y * qs[h] in log2 units.
+        float y[64];
+        const float kf = fp8 ? ks[(warp & 3) * 32 + lane] : 1.f;
+        if (warp < 4) {
+            uint32_t r0[32], r1[32];
+            const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + S_COL;
+            tmem_ld32(ta, r0);
+            tmem_ld32(ta + 32, r1);
+            tmem_wait_ld();
+            const bool valid = k >= 0;
+#pragma unroll
+            for (int h = 0; h < 32; ++h) {
+                y[h] = valid ? __uint_as_float(r0[h]) * kf : -INFINITY;
+                y[32 + h] = valid ? __uint_as_float(r1[h]) * kf : -INFINITY;
+            }
+#pragma unroll
+            for (int h = 0; h < 64; ++h) {
+                const int m = __reduce_max_sync(0xffffffffu, f32_ord(y[h]));
+                if (lane == (h & 31)) wmax[warp * 64 + h] = m;
+            }
+        }
+        if (tid == 0) flags[0] = 0;
+        __syncthreads();
+        if (tid < H) {
+            float my = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) my = fmaxf(my, ord_f32(wmax[w * 64 + tid]));
+            const float mc = my * qs[tid];  // qs > 0
+            const float mo = mref[tid];
+            const float mn = (mo == -INFINITY || mc > mo + kRescaleSlack) ? mc : mo;
+            const float f = mo == -INFINITY ? 0.f : exp2f(mo - mn);  // 1 when unchanged
+            fac[tid] = f;
+            mref[tid] = mn;
+            if (it > 0 && f != 1.f) flags[0] = 1;
+        }
+        __syncthreads();
+        if (warp < 4) {
+            const int key = warp * 32 + lane;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int h = 8 * c8 + 2 * u;
+                    const float m0 = mref[h], m1 = mref[h + 1];
+                    float p0 = m0 == -INFINITY ? 0.f : exp2f(fmaf(y[h], qs[h], -m0));
+                    float p1 = m1 == -INFINITY ? 0.f : exp2f(fmaf(y[h + 1], qs[h + 1], -m1));
+                    if (fp8) {  // v = scale x E4M3 row: the scale moves onto p
+                        p0 *= kf;
+                        p1 *= kf;
+                    }
+                    w[u] = win ? pack_bf16(p0, p1) : pack_f16(p0, p1);
+                }
+                sts128(sP + swz(key, c8), w[0], w[1], w[2], w[3]);
+            }
+        }
+        __syncthreads();
+        // row sums of the rounded P^T (column sums over the chunk's keys):
+        // warp w adds keys [16 w, 16 w + 16) for the head pair of its lane
+        {
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+            for (int jj = 0; jj < 16; ++jj) {
+                const int j = 16 * warp + jj;
+                uint32_t v;
+                asm volatile("ld.shared.u32 %0, [%1];\n"
+                             : "=r"(v)
+                             : "r"(sP + swz(j, lane >> 2) + (lane & 3) * 4));
+                float2 f;
+                if (win) {
+                    f.x = __uint_as_float(v << 16);
+                    f.y = __uint_as_float(v & 0xFFFF0000u);
+                    if (fp8) {  // the stored value is p times the row scale
+                        const float sj = ks[j];
+                        const float inv = sj > 0.f ? 1.f / sj : 0.f;
+                        f.x *= inv;
+                        f.y *= inv;
+                    }
+                } else {
+                    f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+                }
+                s0 += f.x;
+                s1 += f.y;
+            }
+            lpart[warp * 64 + 2 * lane] = s0;
+            lpart[warp * 64 + 2 * lane + 1] = s1;
+        }
+        fence_async_smem();  // P^T stores before the PV product reads them
+        tc_fence_before();
+        __syncthreads();
+        if (tid < H) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) sum += lpart[w * 64 + tid];
+            lrun[tid] = lrun[tid] * fac[tid] + sum;
+        }
+        // ---- rare: a head's reference moved after O^T holds earlier chunks
+        if (flags[0]) {
+            tc_fence_after();
+            const int g = warp & 3;
+            for (int t = 0; t < 2; ++t) {
+                const int mt = (warp >> 2) * 2 + t;
+                for (int h0 = 0; h0 < H; h0 += 32) {
+                    const uint32_t ta = tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0;
+                    uint32_t r[32];
+                    tmem_ld32(ta, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(__uint_as_float(r[i]) * fac[h0 + i]);
+                    tmem_st32(ta, r);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+        }
+        // ---- O^T += V^T P^T (one thread issues)
+        if (tid == 0) {
+            tc_fence_after();
+            for (int mt = 0; mt < DV / 128; ++mt)
+                for (int kk = 0; kk < CK / 16; ++kk)
+                    mma_f16(tmem + O_COL + 64 * mt,
+                            sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
+                            sdesc(sP + kk * 2048u, K_ATOM, 1024), idPV, (it > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bO);
+        }
+        ++npv;
+    }
+    // the last chunk's PV must be complete before O^T is read
+    if (ok && c1 > c0) {
+        const bool got = warp == 0 ? mbar_wait(bO, (c1 - c0 - 1) & 1, wait_ns) : true;
+        ok = __syncthreads_and(got) != 0;
+        tc_fence_after();
+    }
+
+    pdl_trigger();  // only the epilogue is left: let the next kernel be scheduled
+
+    const bool mine = ok && c0 < c1;
+    if (cluster) {
+        // ---- the nsplit CTAs of this sequence form one cluster: each stores
+        // its unnormalised O and (m, l) (they stay in L2); after the cluster
+        // barrier CTA r pulls heads [r*hpc, (r+1)*hpc) of every CTA into its
+        // freed K tile with bulk copies and combines them
+        const size_t prow0 = (size_t)b * H * kMaxSplit;
+        if (mine) {
+            const int g = warp & 3;
+            for (int t = 0; t < 2; ++t) {
+                const int mt = (warp >> 2) * 2 + t;
+                const int d = mt * 128 + g * 32 + lane;
+                for (int h0 = 0; h0 < H; h0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        __stcg(a.part_o + (prow0 + (size_t)(h0 + i) * kMaxSplit + split) * DV + d,
+                               __uint_as_float(r[i]));
+                }
+            }
+        }
+        if (tid < H) {  // nothing (or nothing valid) from this CTA: weight 0
+            const size_t row = prow0 + (size_t)tid * kMaxSplit + split;
+            __stcg(a.part_ml + row * 2, mine ? mref[tid] : -INFINITY);
+            __stcg(a.part_ml + row * 2 + 1, mine ? lrun[tid] : 0.f);
+        }
+        // generic-proxy stores before the peers' bulk (async-proxy) reads
+        asm volatile("fence.proxy.async.global;\n" ::: "memory");
+        cluster_sync();  // every CTA's partial is stored
+        asm volatile("fence.proxy.async.global;\n" ::: "memory");
+        const int hpc = (H + nsplit - 1) / nsplit;
+        const int h_lo = split * hpc, h_hi = min(H, h_lo + hpc), nh = max(0, h_hi - h_lo);
+        float* wts = lpart;  // [nh][nsplit] weights (nh * nsplit <= 64 + 8)
+        // rows (head hh, split s2) land at sK + (hh * nsplit + s2) * 2 KB
+        // (at most 72 rows: 144 KB of the 147 KB tile)
+        if (tid == 0 && nh > 0) {
+            mbar_expect_tx(bW, (uint32_t)(nh * nsplit) * DV * 4);
+            for (int hh = 0; hh < nh; ++hh)
+                for (int s2 = 0; s2 < nsplit; ++s2)
+                    bulk_load(sK + (uint32_t)(hh * nsplit + s2) * DV * 4,
+                              a.part_o + (prow0 + (size_t)(h_lo + hh) * kMaxSplit + s2) * DV,
+                              DV * 4, bW);
+        }
+        if (tid < nh) {
+            const int h = h_lo + tid;
+            const size_t row = prow0 + (size_t)h * kMaxSplit;
+            float m[8], l[8];
+            float M = -INFINITY;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                m[s2] = s2 < nsplit ? __ldcg(a.part_ml + (row + s2) * 2) : -INFINITY;
+                l[s2] = s2 < nsplit ? __ldcg(a.part_ml + (row + s2) * 2 + 1) : 0.f;
+                M = fmaxf(M, m[s2]);
+            }
+            float L = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+                if (s2 >= nsplit) break;
+                const float w = (M == -INFINITY || m[s2] == -INFINITY) ? 0.f : exp2f(m[s2] - M);
+                wts[tid * nsplit + s2] = w;
+                L += w * l[s2];
+            }
+            fac[tid] = L > 0.f ? 1.f / L : 0.f;
+            if (a.lse)
+                a.lse[(size_t)b * H + h] = L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f
+                                                   : -INFINITY;
+        }
+        bool got = true;
+        if (nh > 0 && warp == 0) got = mbar_wait(bW, (uint32_t)nw & 1u, wait_ns);
+        if (nh > 0) ++nw;
+        const bool landed = __syncthreads_and(got) != 0;
+        if (!landed) ok = false;
+        const float* rows = reinterpret_cast<const float*>(smem + OFF_K);
+        for (int it2 = tid; landed && it2 < nh * (DV / 4); it2 += NT) {
+            const int hh = it2 / (DV / 4), d4 = it2 - hh * (DV / 4);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s2 = 0; s2 < nsplit; ++s2) {
+                const float w = wts[hh * nsplit + s2];
+                if (w == 0.f) continue;
+                const float4 v = reinterpret_cast<const float4*>(rows + (hh * nsplit + s2) * DV)[d4];
+                acc.x = fmaf(w, v.x, acc.x);
+                acc.y = fmaf(w, v.y, acc.y);
+                acc.z = fmaf(w, v.z, acc.z);
+                acc.w = fmaf(w, v.w, acc.w);
+            }
+            const float inv = fac[hh];
+            *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h_lo + hh) * DV + 4 * d4) =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        }
+    } else if (nsplit == 1 || mine) {
+        // ---- thread = one latent channel of a tile, 32 heads per load
+        const int g = warp & 3;
+        for (int t = 0; t < 2; ++t) {
+            const int mt = (warp >> 2) * 2 + t;
+            const int d = mt * 128 + g * 32 + lane;
+            for (int h0 = 0; h0 < H; h0 += 32) {
+                uint32_t r[32] = {};
+                if (mine) {
+                    tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
+                    tmem_wait_ld();
+                }
+                if (nsplit == 1) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float l = mine ? lrun[h0 + i] : 0.f;
+                        a.out[((size_t)b * H + h0 + i) * DV + d] =
+                            l > 0.f ? __uint_as_float(r[i]) / l : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        a.part_o[(((size_t)b * H + h0 + i) * kMaxSplit + split) * DV + d] =
+                            __uint_as_float(r[i]);
+                }
+            }
+        }
+    }
+    if (!cluster && tid < H) {
+        const float m = mine ? mref[tid] : -INFINITY, l = mine ? lrun[tid] : 0.f;
+        if (nsplit == 1) {
+            if (a.lse)
+                a.lse[(size_t)b * H + tid] =
+                    l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+        } else {
+            const size_t row = ((size_t)b * H + tid) * kMaxSplit + split;
+            a.part_ml[row * 2] = m;
+            a.part_ml[row * 2 + 1] = l;
+        }
+    }
+    if (!ok && tid == 0) {
+        // a bounded wait gave up: flag it, give the copies and products this
+        // CTA issued one more bounded wait each, then free the tensor memory
+        set_status(a.status, KVC_DEV_TIMEOUT);
+        if (nqk > 0) mbar_wait(bS, (nqk - 1) & 1, kCleanupWaitNs);
+        if (npv > 0) mbar_wait(bO, (npv - 1) & 1, kCleanupWaitNs);
+        if (nw > 0) mbar_wait(bW, (nw - 1) & 1, kCleanupWaitNs);
+        if (win) mbar_wait(bQ, 0, kCleanupWaitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                     "r"(TMEM_COLS));
+    }
+}
+
+}  // namespace t128
+
+bool t128_supported(const kvc_config& c, const Shape& sh) {
+    const bool g_ok = sh.G == 8 || sh.G == 16 || sh.G == 32 || sh.G == 64 || sh.G == 128;
+    return c.act_dtype == KVC_BF16 && c.scale_fmt == KVC_SCALE_UE4M3 && c.n_heads == t128::H &&
+           sh.D == t128::D && sh.Dv == t128::DV && g_ok;
+}
+
+namespace {
+unsigned long long g_wait_ns = 2000000000ull;  // bound on one device wait
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+// 2-D bf16 tensor [rows][576] (row stride 1152 B), boxes of 64 channels x
+// box_rows rows, 128-byte swizzle, zero fill past the end.
+bool encode_rows(CUtensorMap* m, const void* base, unsigned long long rows, unsigned box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)t128::D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)t128::D * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+unsigned long long device_wait_limit_ns() { return g_wait_ns; }
+void set_device_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns; }
+
+template <int G>
+static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const dim3& grid,
+                            int cluster_x, const AttnArgs& a, const Shape& sh, int K, float sm_log2,
+                            int rsplit, int cpr, int nsplit, int cluster, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(t128::attn_t128_kernel<G>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)t128::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(t128::NT);
+    cfg.dynamicSmemBytes = t128::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, t128::attn_t128_kernel<G>, tq, tw, a, sh, K, sm_log2, rsplit,
+                              cpr, nsplit, cluster, g_wait_ns);
+}
+
+// Clusters of `size` CTAs of this kernel that can be resident at once on the
+// current device (cached per device and size; 0 when the query fails).
+template <int G>
+static int max_clusters(int size) {
+    static int cache[64][9] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || size < 1 || size > 8) return 0;
+    if (cache[dev][size]) return cache[dev][size] > 0 ? cache[dev][size] : 0;
+    cudaFuncSetAttribute(t128::attn_t128_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)t128::SMEM_BYTES);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(size, 1);
+    cfg.blockDim = dim3(t128::NT);
+    cfg.dynamicSmemBytes = t128::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = size;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, t128::attn_t128_kernel<G>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cache[dev][size] = n > 0 ? n : -1;
+    return n > 0 ? n : 0;
+}
+
+template <int G>
+static int launch_t128_g(const kvc_config& c, const AttnArgs& a, const Shape& sh, cudaStream_t s) {
+    const int K = c.topk;
+    const int rc = (K + t128::CK - 1) / t128::CK;
+    const int wc = (a.window_len + t128::CK - 1) / t128::CK;
+    // one record chunk per CTA while the CTAs of a sequence fit one cluster
+    // and every sequence's cluster can be resident at once; else two or more
+    // chunks per record CTA (a chunk's loads overlap the previous one's
+    // products)
+    int cpr = 1;
+    while (rc > 0 && cpr < rc) {
+        const int ns = (rc + cpr - 1) / cpr + wc;
+        if (ns <= 8 && (ns == 1 || max_clusters<G>(ns) >= a.batch)) break;
+        ++cpr;
+    }
+    int rsplit = rc == 0 ? 0 : (rc + cpr - 1) / cpr;
+    int nsplit = rsplit + wc;
+    if (nsplit == 0) {  // nothing to attend: one CTA writes zeros and -inf
+        rsplit = 1;
+        nsplit = 1;
+    }
+    if (nsplit > kMaxSplit) return -1;
+    const int cluster = (nsplit > 1 && nsplit <= 8) ? 1 : 0;
+    CUtensorMap tq = {}, tw = {};
+    if (wc > 0) {  // the window chunk's query tile and (bf16) rows arrive by TMA
+        if (!encode_rows(&tq, a.q, (unsigned long long)a.batch * t128::H, t128::H)) return -1;
+        if (!a.win_fp8 &&
+            !encode_rows(&tw, a.window, (unsigned long long)a.batch * a.window_stride, t128::CK))
+            return -1;
+    }
+    const float sm_log2 = c.sm_scale * 1.4426950408889634f;
+    trace_before("attn_t128", s);
+    const cudaError_t e = launch_g<G>(tq, tw, dim3(nsplit, a.batch), cluster ? nsplit : 1, a, sh, K,
+                                      sm_log2, rsplit, cpr, nsplit, cluster, s);
+    trace_after(s);
+    if (e != cudaSuccess) return -1;
+    return cluster ? 1 : nsplit;
+}
+
+// Launches the chunks of every sequence; returns the number of partial
+// results the caller still has to merge (1 when the kernel wrote the final
+// output itself), or a negative value on a launch error.
+int launch_attention_t128(const kvc_config& c, const Shape& sh, const AttnArgs& a,
+                          cudaStream_t s) {
+    switch (sh.G) {
+        case 8: return launch_t128_g<8>(c, a, sh, s);
+        case 16: return launch_t128_g<16>(c, a, sh, s);
+        case 32: return launch_t128_g<32>(c, a, sh, s);
+        case 64: return launch_t128_g<64>(c, a, sh, s);
+        default: return launch_t128_g<128>(c, a, sh, s);
+    }
+}
+
+}  // namespace kvc

@@ -42,7 +42,19 @@ __device__ __forceinline__ uint64_t now_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+// limit_ns == 0: one non-blocking test of the phase (the timeout test hook)
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns == 0) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        return ok != 0;
+    }
     const uint64_t t0 = now_ns();
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
@@ -54,7 +66,7 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
             : "r"(bar), "r"(parity)
             : "memory");
         if (ok) return true;
-        if ((i & 255) == 255 && now_ns() - t0 > 2000000000ull) return false;
+        if ((i & 255) == 255 && now_ns() - t0 > limit_ns) return false;
     }
 }
 // The indexer rows are read once per scan: bulk copies carry an L2
@@ -196,7 +208,7 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
     for (int chunk = 0;; ++chunk) {
         const int s = chunk % kScanStages;
         const int rows = min(kStageRows, cc.end - cc.row);
-        bool got = (tid >> 5) == 0 ? bar_wait(smem_addr(&full[s]), (phase >> s) & 1u) : true;
+        bool got = (tid >> 5) == 0 ? bar_wait(smem_addr(&full[s]), (phase >> s) & 1u, a.wait_ns) : true;
         if (__syncthreads_and(got) == 0) {
             ok = false;
             break;
@@ -296,7 +308,8 @@ index_scan_kernel(TopkArgs a, long long per, int bias, int shift) {
     if (!ok && tid == 0) {
         // a bounded wait gave up: flag it and let the copies still in flight land
         set_status(a.status, KVC_DEV_TIMEOUT);
-        for (int s = 0; s < kScanStages; ++s) bar_wait(smem_addr(&full[s]), (phase >> s) & 1u);
+        for (int s = 0; s < kScanStages; ++s)
+            bar_wait(smem_addr(&full[s]), (phase >> s) & 1u, kCleanupWaitNs);
     }
 }
 
@@ -502,7 +515,8 @@ index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int s
                                  "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
                 }
             }
-            const bool got = warp == 0 ? bar_wait(smem_addr(&full[st]), (phase >> st) & 1u) : true;
+            const bool got =
+                warp == 0 ? bar_wait(smem_addr(&full[st]), (phase >> st) & 1u, a.wait_ns) : true;
             if (__syncthreads_and(got) == 0) {
                 ok = false;
                 break;
@@ -533,7 +547,7 @@ index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int s
                         smem_addr(&mma_bar))
                     : "memory");
             }
-            const bool done = warp == 0 ? bar_wait(smem_addr(&mma_bar), mma_phase) : true;
+            const bool done = warp == 0 ? bar_wait(smem_addr(&mma_bar), mma_phase, a.wait_ns) : true;
             mma_phase ^= 1u;
             if (__syncthreads_and(done) == 0) {
                 ok = false;
@@ -609,8 +623,9 @@ index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int s
     }
     if (!ok && tid == 0) {
         set_status(a.status, KVC_DEV_TIMEOUT);
-        for (int st = 0; st < stages; ++st) bar_wait(smem_addr(&full[st]), (phase >> st) & 1u);
-        bar_wait(smem_addr(&mma_bar), mma_phase);
+        for (int st = 0; st < stages; ++st)
+            bar_wait(smem_addr(&full[st]), (phase >> st) & 1u, kCleanupWaitNs);
+        bar_wait(smem_addr(&mma_bar), mma_phase, kCleanupWaitNs);
     }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
@@ -674,7 +689,9 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
     return launch_select(a, bias, shift, s);
 }
 
-cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s) {
+cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba0, cudaStream_t s) {
+    BatchTopkArgs ba = ba0;
+    for (int q = 0; q < kMaxBatchQ; ++q) ba.q[q].wait_ns = device_wait_limit_ns();
     const TopkArgs& a = ba.q[0];
     if (a.batch == 0 || ba.nq == 0) return cudaSuccess;
     if (a.di != tcs::DI || ba.nq > kMaxBatchQ) return cudaErrorInvalidValue;
@@ -720,7 +737,9 @@ cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba, cudaStream_t s) {
     return cudaSuccess;
 }
 
-cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s) {
+cudaError_t launch_index_topk(const TopkArgs& a0, cudaStream_t s) {
+    TopkArgs a = a0;
+    a.wait_ns = device_wait_limit_ns();
     if (a.batch == 0) return cudaSuccess;
     const int bias = score_bias(a.di), shift = score_shift(a.di);
     cudaError_t err;

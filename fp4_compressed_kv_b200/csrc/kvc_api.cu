@@ -9,6 +9,8 @@
 #include <vector>
 #include <atomic>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kvc_internal.cuh"
 
 namespace kvc {
@@ -331,6 +333,16 @@ kvc_status run_attn(const kvc_config& c, const Shape& sh, const void* q, const k
 
 }  // namespace kvc
 
+namespace kvc {
+// An NVTX range around every enqueuing entry point, so a profiler's timeline
+// shows each C-ABI call over the kernels it launched (free when no tool is
+// attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace kvc
+
 using namespace kvc;
 
 extern "C" {
@@ -375,6 +387,7 @@ size_t kvc_workspace_bytes_hier(const kvc_config* cfg, int batch, int capacity, 
 kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new, const float* gate,
                     const int8_t* idx_k_new, const kvc_cache* cache, uint32_t* dev_status,
                     void* stream) {
+    const NvtxRange nvtx_range("kvc_pack");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     kvc_status st = check_cache(cache, sh);
@@ -404,6 +417,7 @@ kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new, const 
 kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q, const kvc_cache* cache,
                           int32_t* topk_idx, int32_t* scores, void* ws, size_t ws_bytes,
                           uint32_t* dev_status, void* stream) {
+    const NvtxRange nvtx_range("kvc_index_topk");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     kvc_status st = check_cache(cache, sh);
@@ -424,6 +438,7 @@ kvc_status kvc_sparse_decode_attn(const kvc_config* cfg, const void* q, const kv
                                   const int32_t* topk_idx, const void* window, int window_len,
                                   float* out, float* lse, void* ws, size_t ws_bytes,
                                   uint32_t* dev_status, void* stream) {
+    const NvtxRange nvtx_range("kvc_sparse_decode_attn");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     kvc_status st = check_cache(cache, sh);
@@ -446,6 +461,7 @@ kvc_status kvc_sparse_decode_attn_fp8win(const kvc_config* cfg, const void* q,
                                          const uint8_t* win_codes, const float* win_scales,
                                          int window_len, float* out, float* lse, void* ws,
                                          size_t ws_bytes, uint32_t* dev_status, void* stream) {
+    const NvtxRange nvtx_range("kvc_sparse_decode_attn_fp8win");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     kvc_status st = check_cache(cache, sh);
@@ -471,6 +487,7 @@ kvc_status kvc_sparse_decode_attn_fp8win(const kvc_config* cfg, const void* q,
 kvc_status kvc_pack_window_fp8(const kvc_config* cfg, const void* rows, int64_t n_rows,
                                uint8_t* codes, float* scales, uint32_t* dev_status,
                                void* stream) {
+    const NvtxRange nvtx_range("kvc_pack_window_fp8");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     if (n_rows < 0 || (n_rows > 0 && (!rows || !codes || !scales))) return KVC_ERR_INVALID;
@@ -488,6 +505,7 @@ kvc_status kvc_layer_group_step(const kvc_config* cfg, int n_layers, const int32
                                 int window_len, const kvc_cache* cache, float* out, float* lse,
                                 int32_t* topk, void* ws, size_t ws_bytes, uint32_t* dev_status,
                                 void* stream) {
+    const NvtxRange nvtx_range("kvc_layer_group_step");
     return kvc_layer_group_step_hier(cfg, 0, 0, n_layers, modes, q, idx_q, windows, window_len,
                                      cache, out, lse, topk, ws, ws_bytes, dev_status, stream);
 }
@@ -498,6 +516,7 @@ kvc_status kvc_layer_group_step_hier(const kvc_config* cfg, int hier_blocks, int
                                      const kvc_cache* cache, float* out, float* lse,
                                      int32_t* topk, void* ws, size_t ws_bytes,
                                      uint32_t* dev_status, void* stream) {
+    const NvtxRange nvtx_range("kvc_layer_group_step_hier");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     if (!hier_ok(hier_blocks, hier_block)) return KVC_ERR_INVALID;
@@ -576,6 +595,7 @@ size_t kvc_workspace_bytes_batched(const kvc_config* cfg, int nq, int batch, int
 kvc_status kvc_index_topk_batched(const kvc_config* cfg, int nq, const int8_t* idx_q,
                                   const kvc_cache* cache, int32_t* topk_idx, void* ws,
                                   size_t ws_bytes, uint32_t* dev_status, void* stream) {
+    const NvtxRange nvtx_range("kvc_index_topk_batched");
     Shape sh;
     if (!derive_shape(cfg, &sh)) return KVC_ERR_INVALID;
     if (nq < 1 || nq > kMaxBatchQ) return KVC_ERR_INVALID;
@@ -618,6 +638,7 @@ kvc_status kvc_index_topk_batched(const kvc_config* cfg, int nq, const int8_t* i
 }
 
 kvc_status kvc_e2m1_encode(const float* x, int64_t n, uint8_t* codes, void* stream) {
+    const NvtxRange nvtx_range("kvc_e2m1_encode");
     if (n < 0 || (n > 0 && (!x || !codes))) return KVC_ERR_INVALID;
     if (n > 0 && !device_ok()) return KVC_ERR_DEVICE;
     return launch_fp4_codec(x, n, codes, 0, static_cast<cudaStream_t>(stream)) == cudaSuccess
@@ -626,6 +647,7 @@ kvc_status kvc_e2m1_encode(const float* x, int64_t n, uint8_t* codes, void* stre
 }
 
 kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stream) {
+    const NvtxRange nvtx_range("kvc_e4m3_encode");
     if (n < 0 || (n > 0 && (!x || !bytes))) return KVC_ERR_INVALID;
     if (n > 0 && !device_ok()) return KVC_ERR_DEVICE;
     return launch_fp4_codec(x, n, bytes, 1, static_cast<cudaStream_t>(stream)) == cudaSuccess
@@ -677,6 +699,11 @@ kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms) {
 }
 
 uint64_t kvc_launch_count(void) { return g_launches.load(); }
+
+kvc_status kvc_debug_set_wait_limit_ns(uint64_t ns) {
+    set_device_wait_limit_ns(ns);
+    return KVC_OK;
+}
 
 const char* kvc_status_string(kvc_status s) {
     switch (s) {

@@ -26,10 +26,6 @@ __host__ __device__ inline int sel_tiles(int capacity) { return (capacity + kSel
 inline size_t topk_counter_words(int batch) { return (size_t)batch * (kBins + 2); }
 // Upper bound on the number of key splits of one attention problem.
 constexpr int kMaxSplit = 16;
-// Keys per attention chunk.
-constexpr int kChunk = 64;
-// Bound on polls of an mbarrier or flag before a kernel gives up.
-constexpr uint32_t kSpinLimit = 1u << 24;
 
 // Shape facts derived once from a kvc_config.
 struct Shape {
@@ -64,6 +60,14 @@ inline int score_bias(int di) { return di * 127 * 128; }
 void trace_before(const char* name, cudaStream_t s);
 void trace_after(cudaStream_t s);
 
+// Bound on one device wait of a kernel launched from now on (nanoseconds of
+// %globaltimer; 2 s unless a test lowered it through
+// kvc_debug_set_wait_limit_ns).
+unsigned long long device_wait_limit_ns();
+void set_device_wait_limit_ns(unsigned long long ns);
+// Bound of the clean-up waits that follow a timeout (never lowered).
+constexpr unsigned long long kCleanupWaitNs = 2000000000ull;
+
 // ------------------------------------------------------------------ launchers
 struct PackArgs {
     const void* tokens;
@@ -85,7 +89,9 @@ struct TopkArgs {
     int batch, capacity, topk, di;
     int32_t* topk_idx;     // [B][K]
     int32_t* scores;       // [B][cap] (user buffer or workspace)
-    int32_t* counters;     // topk_counter_words(B) ints, zeroed by the launcher
+    int32_t* counters;     // topk_counter_words(B) ints: zero before the call (a zero-filled
+                           // workspace); the kernels' last CTAs leave them at zero again,
+                           // except after a timeout, which leaves them dirty
     int32_t* thr;          // [B][2] threshold bin, entries above it (written by the scan)
     int32_t* tile_count;   // [B][sel_tiles(cap)] candidates per tile
     unsigned long long* cands;  // [B][sel_tiles(cap) * kSelTile]
@@ -103,6 +109,9 @@ struct TopkArgs {
     int32_t* pool_len_out;
     const int32_t* pool_src_n;
     int pool_src_cap, pool_src_block;
+    // bound on one device wait (set by the launcher from the library's
+    // current limit; 0 = a single non-blocking poll, the timeout test hook)
+    unsigned long long wait_ns;
 };
 cudaError_t launch_index_topk(const TopkArgs& a, cudaStream_t s);
 // FP4 indexer keys: exact 64-bit scores (scores64 [B][capacity]) and the

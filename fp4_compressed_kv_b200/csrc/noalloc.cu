@@ -33,7 +33,10 @@ static __device__ __align__(256) unsigned char g_topk_scratch[kScratchBytes];
 // Device address of g_topk_scratch per device.  In host code the symbol's name
 // is only a host-side stand-in, so the address must come from
 // cudaGetSymbolAddress with that device current; it is looked up once per
-// device, on the first call made on it.
+// device, on the first call made on it, and kept for the life of the process.
+// Anything that destroys the device's primary context (cudaDeviceReset, a
+// framework tearing the context down) leaves that address dangling: the entry
+// point must not be called on that device afterwards.
 std::mutex g_mu;
 void* g_addr[64] = {};
 
@@ -94,7 +97,9 @@ extern "C" kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t
     a.topk_idx = topk_idx;
     a.scores = scores ? scores : reinterpret_cast<int32_t*>(ws);
     unsigned char* p = ws + kScoresBytes;
-    a.counters = reinterpret_cast<int32_t*>(p);  // cleared on the stream by the launcher
+    // zero when the library loads (a static array); the kernels' last CTAs
+    // leave them at zero after every call that did not time out
+    a.counters = reinterpret_cast<int32_t*>(p);
     p += kCounterBytes;
     a.thr = reinterpret_cast<int32_t*>(p);
     p += kThrBytes;

@@ -77,6 +77,7 @@ def _lib():
             "kvc_trace_end": (S, []),
             "kvc_trace_kernel": (S, [C.c_char_p, C.POINTER(C.c_int), C.POINTER(C.c_double)]),
             "kvc_launch_count": (C.c_uint64, []),
+            "kvc_debug_set_wait_limit_ns": (S, [C.c_uint64]),
             "kvc_status_string": (C.c_char_p, [I]),
             "kvc_version": (C.c_char_p, []),
         }
@@ -300,6 +301,12 @@ def trace_kernel(name: str):
 
 def launch_count() -> int:
     return int(_lib().kvc_launch_count())
+
+
+def debug_set_wait_limit_ns(ns: int):
+    """Test hook: bound of every in-kernel wait of later launches (0 = one
+    non-blocking poll; the library's default is 2_000_000_000)."""
+    _check("kvc_debug_set_wait_limit_ns", _lib().kvc_debug_set_wait_limit_ns(int(ns)))
 
 
 def version() -> str:

@@ -65,7 +65,8 @@ typedef enum { KVC_FULL = 0, KVC_REINDEX = 1, KVC_REUSE = 2 } kvc_mode;
 typedef enum { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
 
 /* device status bits */
-#define KVC_DEV_NONFINITE 0x1u  /* pack met a NaN/Inf channel (coded as 0)     */
+#define KVC_DEV_NONFINITE 0x1u  /* a NaN/Inf input: a pack channel (coded as 0)
+                                   or an attention query row                   */
 #define KVC_DEV_BAD_INDEX 0x2u  /* a top-K index outside [-1, n_entries)       */
 #define KVC_DEV_CAPACITY 0x4u   /* pack would pass the cache capacity          */
 #define KVC_DEV_TIMEOUT 0x8u    /* a bounded in-kernel wait gave up            */
@@ -196,7 +197,11 @@ kvc_status kvc_index_topk(const kvc_config* cfg, const int8_t* idx_q,
  * (a static array) and every call leaves them at zero, but calls whose work
  * overlaps on the GPU (different streams, or different host threads on one
  * device) race on it, and after a call that set KVC_DEV_TIMEOUT the array
- * stays unusable until the process exits.                                */
+ * stays unusable until the process exits.  The looked-up address is kept for
+ * the life of the process: after anything that destroys the device's primary
+ * context (cudaDeviceReset, a framework tearing the context down) it no
+ * longer points at the array, and this entry point must not be called on
+ * that device again.                                                     */
 kvc_status kvc_index_topk_noalloc(const kvc_config* cfg, const int8_t* idx_q,
                                   const kvc_cache* cache, int32_t* topk_idx,
                                   int32_t* scores, uint32_t* dev_status,
@@ -323,11 +328,25 @@ kvc_status kvc_e4m3_encode(const float* x, int64_t n, uint8_t* bytes, void* stre
  * kernel named `name` and their summed device time in milliseconds.  Names:
  * "pack", "pack_idx", "pack_commit", "window_fp8", "index_scan",
  * "index_scan_tc", "index_scan_fp4", "topk_select", "topk_select_fp4",
- * "block_max", "copy_topk", "attn_tc05", "attn_simt", "attn_merge",
- * "fp4_codec".                                                             */
+ * "block_max", "copy_topk", "attn_t128", "attn_simt", "attn_merge",
+ * "fp4_codec".  Every enqueuing entry point also opens an NVTX range named
+ * after itself for the duration of the call (a no-op without a profiler).  */
 kvc_status kvc_trace_begin(int max_launches);
 kvc_status kvc_trace_end(void);
 kvc_status kvc_trace_kernel(const char* name, int* launches, double* total_ms);
+
+/* TEST HOOK, not for production use.  Sets the bound on each in-kernel wait
+ * (mbarrier phases of the bulk-copy ring and of the tensor-core products) of
+ * every kernel enqueued after this call, in nanoseconds of %globaltimer; the
+ * library starts with 2,000,000,000 (2 s).  0 makes every such wait a single
+ * non-blocking poll, so a kernel reaches its timeout path at once: it sets
+ * KVC_DEV_TIMEOUT, waits (with the normal 2 s bound) for the copies and
+ * products it already issued, frees its tensor memory and returns normally.
+ * After such a call the top-K counters in the workspace are left dirty and
+ * the outputs are undefined: zero the workspace before the next call.  The
+ * value is read when a kernel is enqueued (a captured graph keeps the value
+ * it was captured with).  Not thread-safe with concurrent enqueues.        */
+kvc_status kvc_debug_set_wait_limit_ns(uint64_t ns);
 
 /* Number of kernels the library has enqueued since it was loaded. */
 uint64_t kvc_launch_count(void);

@@ -78,3 +78,29 @@ def test_noalloc_heavy_ties_and_limits(kvc):
                                                      device="cuda"), many,
                                torch.empty(65, w.topk, dtype=torch.int32, device="cuda"))
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("n_entries", [
+    [1 << 19],                                        # one sequence at the row limit
+    [8192 - 97 * (i % 7) for i in range(63)] + [8192],  # 64 ragged sequences, 2^19 rows
+])
+def test_noalloc_at_the_largest_accepted_shapes(kvc, n_entries):
+    """The fixed scratch is sized for batch x capacity <= 2^19 rows and at most
+    64 sequences; the shapes that fill it exactly must still equal
+    kvc_index_topk, on two calls in a row."""
+    w = synth.WORKLOADS["mla32k"]
+    cfg, cache, g = _cache(kvc, w.scaled(batch=len(n_entries)), n_entries, seed=9)
+    B, cap = cache.batch, cache.capacity
+    assert B * cap == 1 << 19
+    ws = kvc.workspace(cfg, B, cap)
+    for call in range(2):
+        q = torch.randint(-127, 128, (B, w.idx_dim), generator=g, device="cuda",
+                          dtype=torch.int8)
+        ref = torch.empty(B, w.topk, dtype=torch.int32, device="cuda")
+        kvc.index_topk(cfg, q, cache, ref, ws)
+        tk = torch.full((B, w.topk), -7, dtype=torch.int32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        kvc.index_topk_noalloc(cfg, q, cache, tk, status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        assert torch.equal(tk, ref), f"call {call}: top-K differs"
