@@ -439,6 +439,38 @@ def oracle_decode_sample(w, seconds, seed_shift=0):
     return steps, timed, desc
 
 
+def _oracle_worker(job):
+    """One spawned process: single-sequence oracle decode steps of workload
+    `name` for about `seconds` of timed work, on its own sequence draw."""
+    name, seconds, shift = job
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    import torch
+    torch.set_num_threads(1)
+    from fp4_compressed_kv_b200 import synth
+    steps, secs, _ = oracle_decode_sample(synth.WORKLOADS[name], seconds, seed_shift=shift)
+    return steps, secs
+
+
+def oracle_multicore(w, seconds, procs):
+    """The oracle on `procs` host cores at once: one spawned process per core,
+    each decoding its own sequences (the sequences of a batch are
+    independent), all running concurrently.  Returns the summed query-tokens/s
+    and the per-process results."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")  # CUDA is live in this process: never fork
+    with ctx.Pool(procs) as pool:
+        res = pool.map(_oracle_worker, [(w.name, seconds, 1 + i) for i in range(procs)])
+    rate = sum(s / t for s, t in res if t > 0)
+    return rate, res
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 # ----------------------------------------------------------------------------- ours
 def measure_decode(w, steps, warmup, dev, stream, hier=0, hier_block=8, clocks_gpu=None):
     """Decode steps of workload w on this rank: the context is packed on the
@@ -823,12 +855,26 @@ def run_ours(args):
         except Exception as e:  # a side measurement must not cost the headline line
             extra["fp4_indexer_keys"] = {"error": str(e)[:200]}
 
-    # ---- CPU oracle baseline (rank 0, N=1 only)
+    # ---- CPU oracle baseline (rank 0, N=1 only): one process per host core
+    # (up to 32), each decoding its own sequences concurrently, beside the
+    # single-core figure
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        steps_c, secs, desc = oracle_decode_sample(w0, args.cpu_seconds)
-        cpu = {"value": round(steps_c / secs, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": desc, "seconds": round(secs, 2)}
+        steps_c, secs, desc = oracle_decode_sample(w0, args.cpu_seconds / 2)
+        single = round(steps_c / secs, 3)
+        procs = max(1, min(32, host_cores()))
+        try:
+            rate, res = oracle_multicore(w0, args.cpu_seconds / 2, procs)
+            cpu = {"value": round(rate, 3), "unit": UNIT, "cores": procs, "kind": "oracle",
+                   "sample": (f"{sum(r[0] for r in res)} single-sequence decode steps of "
+                              f"{w0.name} on {procs} processes (one per core, its own "
+                              f"sequences; about {args.cpu_seconds / 2:.0f} s each), oracle C "
+                              f"code"),
+                   "host_cores": host_cores(),
+                   "single_core": {"value": single, "sample": desc}}
+        except Exception as e:  # the pool must not cost the headline line
+            cpu = {"value": single, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                   "multicore_error": str(e)[:200]}
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,

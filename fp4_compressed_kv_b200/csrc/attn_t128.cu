@@ -68,13 +68,13 @@ constexpr uint32_t OFF_K = OFF_Q + NATOM * Q_ATOM;   // 73,728
 constexpr uint32_t OFF_P = OFF_K + 8 * K_ATOM;       // the RoPE atom, P^T after QK
 constexpr uint32_t OFF_MISC = OFF_K + NATOM * K_ATOM;  // 221,184
 // misc: kidx[128] i32 | qs[64] | mref[64] | lrun[64] | fac[64] | wmax[4][64] |
-//       lpart[8][64] | ks[128] | bars[4] u64 | tmem slot | flags
+//       lpart[8][64] | ks[128] | bars[4] u64 | tmem slot | flags | ones (2 KB)
 constexpr uint32_t M_KIDX = 0, M_QS = 512, M_MREF = 768, M_LRUN = 1024, M_FAC = 1280,
                    M_WMAX = 1536, M_LPART = 2560, M_KS = 4608, M_BARS = 5120, M_TSLOT = 5152,
-                   M_FLAGS = 5168, MISC_BYTES = 5248;
+                   M_FLAGS = 5168, M_ONES = 5248, MISC_BYTES = 7296;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL = 0, O_COL = 256;           // S^T: 64 cols; O^T: 4 tiles x 64 cols
+constexpr uint32_t S_COL = 0, L_COL = 64, O_COL = 256;  // S^T, L^T: 64 cols; O^T: 4 x 64
 constexpr float kRescaleSlack = 8.0f;                // log2 units
 enum { BAR_S = 0, BAR_O = 1, BAR_Q = 2, BAR_W = 3 };
 
@@ -99,26 +99,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-// Q tile (64 heads x 576 channels, 9 boxes of 64 channels) of sequence b.
-__device__ __forceinline__ void tma_q(const CUtensorMap* map, uint32_t sQ, int b, uint32_t bar) {
-    mbar_expect_tx(bar, NATOM * Q_ATOM);
-    for (int at = 0; at < NATOM; ++at) tma_load_2d(sQ + at * Q_ATOM, map, 64 * at, b * H, bar);
-}
-
-// The query rows of a record CTA in registers: thread t holds head t/4,
-// channels [144 (t%4), +144) as 18 16-byte pieces.
-__device__ __forceinline__ void load_q_regs(const AttnArgs& a, int b, int tid, uint4 (&v)[18]) {
+// The query tile of a record CTA, landed by TMA as bf16, converted in place to
+// f16 with a per-head power of two that puts the row maximum in [2^14,
+// 2^15); the head's softmax multiplier qs[h] absorbs it.  Thread t: head t/4,
+// channels [144 (t%4), +144) as 18 16-byte pieces (the same swizzled
+// positions the TMA wrote; a warp's accesses take the minimum 4 wavefronts).
+__device__ __forceinline__ void convert_q_f16(const AttnArgs& a, float sm_log2, uint32_t sQ,
+                                              uint32_t q_atom, float* qs, int tid) {
     const int h = tid >> 2, qq = tid & 3;
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned char*>(a.q) +
-                                                      ((size_t)b * H + h) * D * 2) + 18 * qq;
+    uint4 v[18];
 #pragma unroll
-    for (int i = 0; i < 18; ++i) v[i] = __ldg(src + i);
-}
-// bf16 -> f16 with a per-head power of two that puts the row maximum in
-// [2^14, 2^15); the head's softmax multiplier qs[h] absorbs it.
-__device__ __forceinline__ void store_q_f16(const AttnArgs& a, const uint4 (&v)[18], float sm_log2,
-                                            uint32_t sQ, float* qs, int tid) {
-    const int h = tid >> 2, qq = tid & 3;
+    for (int i = 0; i < 18; ++i) {
+        const int c16 = 18 * qq + i;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                     : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w)
+                     : "r"(sQ + (c16 >> 3) * q_atom + swz(h, c16 & 7)));
+    }
     uint32_t amax = 0;  // max |x| as fp32 bits (integer order = float order)
 #pragma unroll
     for (int i = 0; i < 18; ++i) {
@@ -142,14 +138,14 @@ __device__ __forceinline__ void store_q_f16(const AttnArgs& a, const uint4 (&v)[
     if (qq == 0) qs[h] = sm_log2 * __uint_as_float((uint32_t)(127 + k) << 23);
 #pragma unroll
     for (int i = 0; i < 18; ++i) {
-        const int c16 = 18 * qq + i;  // 16-byte chunk of the row: channels 8 c16 .. +7
+        const int c16 = 18 * qq + i;
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
         uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             o[j] = pack_f16(__uint_as_float(w[j] << 16) * mul,
                             __uint_as_float(w[j] & 0xFFFF0000u) * mul);
-        sts128(sQ + (c16 >> 3) * Q_ATOM + swz(h, c16 & 7), o[0], o[1], o[2], o[3]);
+        sts128(sQ + (c16 >> 3) * q_atom + swz(h, c16 & 7), o[0], o[1], o[2], o[3]);
     }
 }
 
@@ -164,44 +160,73 @@ constexpr int scale_vecs() {  // 16-byte loads covering the scale bytes
     return (512 / G + (64 + G - 1) / G + 15) / 16;
 }
 
-// One record's half row (half 0: channels 0..287, half 1: 288..575) in
-// registers: 9 pieces of codes and the scale bytes.
+// Scale word (4 bytes at record offset 288 + 4 w) holding every scale of
+// 32-channel item i: for groups of 8..128 channels an item's scales share
+// one aligned word.
 template <int G>
-struct RowRegs {
-    uint4 cw[9];
-    uint4 sv[scale_vecs<G>()];
+__device__ __host__ constexpr int scale_word(int i) {
+    return scale_index<G>(i, 0) >> 2;
+}
+// A chunk's records, 8 threads per key: thread t = 8 q + sub takes keys
+// q, q + 32, q + 64, q + 96 and of each the 32-channel items sub, sub + 8
+// and (sub < 2) sub + 16 -- 16-byte loads where 8 adjacent lanes read 128
+// contiguous bytes of one record -- with the scale word of each item.
+struct RecRegs {
+    uint4 cw[4][3];
+    uint32_t sw[4][3];
 };
 template <int G>
-__device__ __forceinline__ void load_row(const uint8_t* rec, int half, RowRegs<G>& r) {
+__device__ __forceinline__ void load_records(const uint8_t* base, int rb, const int* kidx, int tid,
+                                             RecRegs& r) {
+    const int sub = tid & 7, q = tid >> 3;
 #pragma unroll
-    for (int u = 0; u < 9; ++u) r.cw[u] = ldg_nc(rec + (9 * half + u) * 16);
+    for (int p = 0; p < 4; ++p) {
+        const int k = kidx[q + 32 * p];
+        if (k < 0) continue;
+        const uint8_t* rec = base + (size_t)k * rb;
 #pragma unroll
-    for (int u = 0; u < scale_vecs<G>(); ++u) r.sv[u] = ldg_nc(rec + 288 + 16 * u);
-}
-// ... dequantised into the K tile: codes times the f16 group scale, exact.
-template <int G, int HALF>
-__device__ __forceinline__ void store_row(const RowRegs<G>& r, uint32_t sK, int s) {
-    constexpr int NS = scale_vecs<G>();
-    uint32_t sb[4 * NS];
-#pragma unroll
-    for (int u = 0; u < NS; ++u) {
-        sb[4 * u] = r.sv[u].x;
-        sb[4 * u + 1] = r.sv[u].y;
-        sb[4 * u + 2] = r.sv[u].z;
-        sb[4 * u + 3] = r.sv[u].w;
+        for (int u = 0; u < 3; ++u) {
+            const int i = sub + 8 * u;
+            if (u == 2 && sub >= 2) break;
+            r.cw[p][u] = ldg_nc(rec + 16 * i);
+            r.sw[p][u] = __ldg(reinterpret_cast<const uint32_t*>(rec + 288) + scale_word<G>(i));
+        }
     }
+}
+// ... dequantised into the K tile: codes times the f16 group scale (exact),
+// or zeros for a masked key.  Key j = q + 32 p has j & 7 = q & 7 and item i =
+// sub + 8 u has i & 1 = sub & 1, so a thread's 16-byte slots are fixed: only
+// the atom and the 4 KB row block move.  A warp's stores (4 keys x 8 items)
+// cover 8 swizzle slots x 4 atoms: the minimum 4 wavefronts.
+template <int G>
+__device__ __forceinline__ void store_records(const RecRegs& r, const int* kidx, uint32_t sK,
+                                              int tid) {
+    const int sub = tid & 7, q = tid >> 3;
+    const uint32_t x7 = q & 7;
+    const uint32_t base = sK + (uint32_t)(sub >> 1) * K_ATOM + (uint32_t)(q >> 3) * 1024u + x7 * 128u;
+    uint32_t slot[4];
 #pragma unroll
-    for (int u = 0; u < 9; ++u) {
-        const int i = 9 * HALF + u;  // 32-channel item
-        const uint32_t words[4] = {r.cw[u].x, r.cw[u].y, r.cw[u].z, r.cw[u].w};
-        const uint32_t row = sK + (uint32_t)(i >> 1) * K_ATOM;
+    for (int k = 0; k < 4; ++k) slot[k] = ((4u * (sub & 1) + k) ^ x7) << 4;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int si = scale_index<G>(i, k);
-            const uint32_t byte = (sb[si >> 2] >> (8 * (si & 3))) & 0xFFu;
-            uint32_t w[4];
-            e2m1x8_scaled(words[k], ue4m3_f16x2(byte), w);
-            sts128(row + swz(s, 4 * (i & 1) + k), w[0], w[1], w[2], w[3]);
+    for (int p = 0; p < 4; ++p) {
+        const bool live = kidx[q + 32 * p] >= 0;
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+            if (u == 2 && sub >= 2) break;
+            const int i = sub + 8 * u;
+            const uint32_t row = base + (uint32_t)(4 * u) * K_ATOM + (uint32_t)p * 4096u;
+            const uint32_t words[4] = {r.cw[p][u].x, r.cw[p][u].y, r.cw[p][u].z, r.cw[p][u].w};
+            const int s0 = scale_index<G>(i, 0) & 3;  // the item's first scale byte
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+                if (live) {
+                    const int sb = G >= 32 ? s0 : (s0 + (8 * k) / G);
+                    const uint32_t byte = (r.sw[p][u] >> (8 * sb)) & 0xFFu;
+                    e2m1x8_scaled(words[k], ue4m3_f16x2(byte), w);
+                }
+                sts128(row + slot[k], w[0], w[1], w[2], w[3]);
+            }
         }
     }
 }
@@ -211,11 +236,19 @@ __device__ __forceinline__ void zero_row_half(uint32_t sK, int s, int half) {
         sts128(sK + (uint32_t)(c16 >> 3) * K_ATOM + swz(s, c16 & 7), 0u, 0u, 0u, 0u);
 }
 
+// The all-ones A operand of the row-sum product (128 rows x 16 keys), in the
+// non-swizzled K-major layout: two 8x8 core matrices of 128 B along K, every
+// 8-row group reading the same two (stride 0).  L^T = ONES x P^T puts each
+// head's sum of its rounded weights in every lane of one tensor-memory tile.
+__device__ __forceinline__ uint64_t ones_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | (1ull << 46);
+}
+
 template <int G>
 __global__ void __launch_bounds__(NT, 1)
 attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_w,
                  AttnArgs a, Shape sh, int K, float sm_log2, int rsplit, int cpr, int nsplit,
-                 int cluster, unsigned long long wait_ns) {
+                 int cluster, int HG, unsigned long long wait_ns) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;  // 1024-byte alignment for the swizzle
@@ -233,20 +266,24 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(misc + M_BARS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + M_TSLOT);
     int* flags = reinterpret_cast<int*>(misc + M_FLAGS);
+    const uint32_t sOnes = base + OFF_MISC + M_ONES;
     const uint32_t bS = smem_u32(&bars[BAR_S]), bO = smem_u32(&bars[BAR_O]),
                    bQ = smem_u32(&bars[BAR_Q]), bW = smem_u32(&bars[BAR_W]);
 
-    const int b = blockIdx.y, split = blockIdx.x;
+    const int split = blockIdx.x, hg0 = blockIdx.y * HG, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = a.window_len;
     const int rc = (K + CK - 1) / CK;
+    const uint32_t q_atom = (uint32_t)HG * 128u;  // Q atoms of HG rows, packed
     // this CTA's chunks: record chunks [c0, c1) or window chunk split - rsplit
     const bool win = split >= rsplit;
     const bool fp8 = win && a.win_fp8 != nullptr;
+    const bool lmma = !fp8;  // row sums by the tensor core (FP8 rows: column sums)
     const int c0 = win ? split - rsplit : split * cpr;
     const int c1 = win ? min(c0 + 1, (W + CK - 1) / CK) : min(c0 + cpr, rc);
-    const uint32_t idQK = idesc_f16(128, 64, win ? 1 : 0, 0, 0);
+    const uint32_t idQK = idesc_f16(128, HG, win ? 1 : 0, 0, 0);
     const uint32_t idPV = idesc_f16(128, 64, win ? 1 : 0, 1, 1);
+    const uint32_t idL = idesc_f16(128, 64, win ? 1 : 0, 0, 1);
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
@@ -263,32 +300,30 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         lrun[tid] = 0.f;
         if (win) qs[tid] = sm_log2;
     }
-    __syncthreads();  // barriers initialised before any copy arrives on them
-    // The query tile: read before the wait when no kernel launched since the
-    // caller wrote q (inside a layer-group step), else after it.
-    uint4 qv[18];
-    if (a.q_ready) {
-        if (win) {
-            if (tid == 0) tma_q(&tm_q, sQ, b, bQ);
-        } else {
-            load_q_regs(a, b, tid, qv);
-        }
+    {  // the ones block (2 KB, read 256 B) of 1.0 in the chunk's operand type
+        const uint32_t one = win ? 0x3F803F80u : 0x3C003C00u;
+        asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(sOnes + 8 * tid), "r"(one));
     }
+    __syncthreads();  // barriers initialised before any copy arrives on them
+    // The query rows of this head group (bf16) by TMA: issued before the wait
+    // when no kernel launched since the caller wrote q (inside a layer-group
+    // step), else after it.  Record CTAs convert them in place.
+    auto tma_q = [&]() {
+        mbar_expect_tx(bQ, NATOM * q_atom);
+        for (int at = 0; at < NATOM; ++at)
+            tma_load_2d(sQ + at * q_atom, &tm_q, 64 * at, b * H + hg0, bQ);
+    };
+    if (a.q_ready && tid == 0) tma_q();
     pdl_wait();
     const int n = a.n_entries[b];
     const bool len_ok = n >= 0 && n <= a.capacity;
-    if (!a.q_ready) {
-        if (win) {
-            if (tid == 0) tma_q(&tm_q, sQ, b, bQ);
-        } else {
-            load_q_regs(a, b, tid, qv);
-        }
-    }
+    if (!a.q_ready && tid == 0) tma_q();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
     int nqk = 0, npv = 0, nw = 0;  // commits / copies issued (for the cleanup waits)
-    const int s = tid & (CK - 1), half = tid >> 7;  // this thread's key and half row
+    const int s = tid & (CK - 1), half = tid >> 7;  // key and half row (window paths)
+    const uint8_t* recs = a.records + (size_t)b * a.capacity * sh.rb;
     // ---- slot table of chunk c: record index, window row, or -1 (masked)
     auto slot_table = [&](int c) {
         if (tid < CK) {
@@ -297,10 +332,10 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int j = c * CK + tid;
                 if (j < K) {
                     const int idx = a.topk_idx[(size_t)b * K + j];
-                    if (a.topk_copy) a.topk_copy[(size_t)b * K + j] = idx;
+                    if (a.topk_copy && hg0 == 0) a.topk_copy[(size_t)b * K + j] = idx;
                     if (len_ok && idx >= 0 && idx < n)
                         k = idx;
-                    else if (idx != -1 && len_ok)
+                    else if (idx != -1 && len_ok && hg0 == 0)
                         set_status(a.status, KVC_DEV_BAD_INDEX);
                 }
             } else {
@@ -313,22 +348,26 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();
         return kidx[s];
     };
-    // ---- record rows into registers: in flight while the query tile is
-    // converted (first chunk) or while the previous chunk's PV runs
-    RowRegs<G> rr;
+    // ---- a record chunk's rows into registers: in flight while the query
+    // rows land and are converted (first chunk) or while the previous chunk's
+    // PV runs
+    RecRegs rr;
     int k = -1;
     if (c0 < c1) {
         k = slot_table(c0);
-        if (!win && k >= 0) load_row<G>(a.records + ((size_t)b * a.capacity + k) * sh.rb, half, rr);
+        if (!win) load_records<G>(recs, sh.rb, kidx, tid, rr);
     }
-    if (!win) store_q_f16(a, qv, sm_log2, sQ, qs, tid);
+    if (!win && c0 < c1) {
+        const bool got = warp == 0 ? mbar_wait(bQ, 0, wait_ns) : true;
+        ok = __syncthreads_and(got) != 0;
+        if (ok && tid < 4 * HG) convert_q_f16(a, sm_log2, sQ, q_atom, qs, tid);
+    }
 
     for (int c = c0; c < c1 && ok; ++c) {
         const int it = c - c0;
         if (it > 0) {
             k = slot_table(c);
-            if (!win && k >= 0)
-                load_row<G>(a.records + ((size_t)b * a.capacity + k) * sh.rb, half, rr);
+            if (!win) load_records<G>(recs, sh.rb, kidx, tid, rr);
         }
         if (win && !fp8) {
             // the window rows of this chunk by TMA: 9 boxes of 64 channels x 128 rows
@@ -348,12 +387,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // ---- fill the K tile
         if (!win) {
-            if (k < 0)
-                zero_row_half(sK, s, half);
-            else if (half == 0)
-                store_row<G, 0>(rr, sK, s);
-            else
-                store_row<G, 1>(rr, sK, s);
+            store_records<G>(rr, kidx, sK, tid);
         } else if (fp8) {
             // signed E4M3 codes decoded exactly to bf16 (the row scale is
             // applied to the logits and to the probabilities)
@@ -398,7 +432,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!ok) break;
             if (k < 0) zero_row_half(sK, s, half);
         }
-        if (win && it == 0) {  // the query tile's TMA
+        if (win && it == 0) {  // the query rows' TMA
             const bool got = warp == 0 ? mbar_wait(bQ, 0, wait_ns) : true;
             ok = __syncthreads_and(got) != 0;
             if (!ok) break;
@@ -413,7 +447,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t at = kk >> 2, koff = (kk & 3) * 32;
                 mma_f16(tmem + S_COL, sdesc(sK + at * K_ATOM + koff, 16, 1024),
-                        sdesc(sQ + at * Q_ATOM + koff, 16, 1024), idQK, kk > 0);
+                        sdesc(sQ + at * q_atom + koff, 16, 1024), idQK, kk > 0);
             }
             mma_commit(bS);
         }
@@ -427,88 +461,82 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
         // ---- softmax, warps 0-3: thread = key = tensor-memory lane.  y is
         // the raw logit (times the FP8 row scale); x = y * qs[h] in log2 units.
-        float y[64];
-        const float kf = fp8 ? ks[(warp & 3) * 32 + lane] : 1.f;
+        // The HG scores are read from tensor memory 8 at a time, twice
+        // (maxima, then weights), in rolled loops: each CTA runs this once.
+        const bool valid = k >= 0;
+        const float kf = fp8 ? ks[s] : 1.f;
+        const uint32_t ta_s = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL;
         if (warp < 4) {
-            uint32_t r0[32], r1[32];
-            const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + S_COL;
-            tmem_ld32(ta, r0);
-            tmem_ld32(ta + 32, r1);
-            tmem_wait_ld();
-            const bool valid = k >= 0;
+#pragma unroll 1
+            for (int h0 = 0; h0 < HG; h0 += 8) {
+                uint32_t r[8];
+                tmem_ld8(ta_s + h0, r);
+                tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < 32; ++h) {
-                y[h] = valid ? __uint_as_float(r0[h]) * kf : -INFINITY;
-                y[32 + h] = valid ? __uint_as_float(r1[h]) * kf : -INFINITY;
-            }
-#pragma unroll
-            for (int h = 0; h < 64; ++h) {
-                const int m = __reduce_max_sync(0xffffffffu, f32_ord(y[h]));
-                if (lane == (h & 31)) wmax[warp * 64 + h] = m;
+                for (int i = 0; i < 8; ++i) {
+                    const float y = valid ? __uint_as_float(r[i]) * kf : -INFINITY;
+                    const int m = __reduce_max_sync(0xffffffffu, f32_ord(y));
+                    if (lane == ((h0 + i) & 31)) wmax[warp * 64 + h0 + i] = m;
+                }
             }
         }
         if (tid == 0) flags[0] = 0;
         __syncthreads();
-        if (tid < H) {
+        if (tid < HG) {
             float my = -INFINITY;
 #pragma unroll
             for (int w = 0; w < 4; ++w) my = fmaxf(my, ord_f32(wmax[w * 64 + tid]));
             const float mc = my * qs[tid];  // qs > 0
             const float mo = mref[tid];
             const float mn = (mo == -INFINITY || mc > mo + kRescaleSlack) ? mc : mo;
-            const float f = mo == -INFINITY ? 0.f : exp2f(mo - mn);  // 1 when unchanged
+            const float f = mo == -INFINITY ? 0.f : ex2(mo - mn);  // 1 when unchanged
             fac[tid] = f;
             mref[tid] = mn;
             if (it > 0 && f != 1.f) flags[0] = 1;
         }
         __syncthreads();
         if (warp < 4) {
-            const int key = warp * 32 + lane;
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
+#pragma unroll 1
+            for (int c8 = 0; c8 < HG / 8; ++c8) {
+                uint32_t r[8];
+                tmem_ld8(ta_s + 8 * c8, r);
+                tmem_wait_ld();
                 uint32_t w[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int h = 8 * c8 + 2 * u;
                     const float m0 = mref[h], m1 = mref[h + 1];
-                    float p0 = m0 == -INFINITY ? 0.f : exp2f(fmaf(y[h], qs[h], -m0));
-                    float p1 = m1 == -INFINITY ? 0.f : exp2f(fmaf(y[h + 1], qs[h + 1], -m1));
+                    const float y0 = valid ? __uint_as_float(r[2 * u]) * kf : -INFINITY;
+                    const float y1 = valid ? __uint_as_float(r[2 * u + 1]) * kf : -INFINITY;
+                    float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, qs[h], -m0));
+                    float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, qs[h + 1], -m1));
                     if (fp8) {  // v = scale x E4M3 row: the scale moves onto p
                         p0 *= kf;
                         p1 *= kf;
                     }
                     w[u] = win ? pack_bf16(p0, p1) : pack_f16(p0, p1);
                 }
-                sts128(sP + swz(key, c8), w[0], w[1], w[2], w[3]);
+                sts128(sP + swz(s, c8), w[0], w[1], w[2], w[3]);
             }
         }
-        __syncthreads();
-        // row sums of the rounded P^T (column sums over the chunk's keys):
-        // warp w adds keys [16 w, 16 w + 16) for the head pair of its lane
-        {
+        if (!lmma) {
+            // FP8 rows: column sums of the rounded P^T divided by the row
+            // scale (warp w adds keys [16 w, 16 w + 16) for its lane's pair)
+            __syncthreads();
             float s0 = 0.f, s1 = 0.f;
+            if (2 * lane < HG) {
 #pragma unroll 4
-            for (int jj = 0; jj < 16; ++jj) {
-                const int j = 16 * warp + jj;
-                uint32_t v;
-                asm volatile("ld.shared.u32 %0, [%1];\n"
-                             : "=r"(v)
-                             : "r"(sP + swz(j, lane >> 2) + (lane & 3) * 4));
-                float2 f;
-                if (win) {
-                    f.x = __uint_as_float(v << 16);
-                    f.y = __uint_as_float(v & 0xFFFF0000u);
-                    if (fp8) {  // the stored value is p times the row scale
-                        const float sj = ks[j];
-                        const float inv = sj > 0.f ? 1.f / sj : 0.f;
-                        f.x *= inv;
-                        f.y *= inv;
-                    }
-                } else {
-                    f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = 16 * warp + jj;
+                    uint32_t v;
+                    asm volatile("ld.shared.u32 %0, [%1];\n"
+                                 : "=r"(v)
+                                 : "r"(sP + swz(j, lane >> 2) + (lane & 3) * 4));
+                    const float sj = ks[j];
+                    const float inv = sj > 0.f ? __frcp_rn(sj) : 0.f;
+                    s0 += __uint_as_float(v << 16) * inv;
+                    s1 += __uint_as_float(v & 0xFFFF0000u) * inv;
                 }
-                s0 += f.x;
-                s1 += f.y;
             }
             lpart[warp * 64 + 2 * lane] = s0;
             lpart[warp * 64 + 2 * lane + 1] = s1;
@@ -516,33 +544,35 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         fence_async_smem();  // P^T stores before the PV product reads them
         tc_fence_before();
         __syncthreads();
-        if (tid < H) {
+        if (!lmma && tid < HG) {
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) sum += lpart[w * 64 + tid];
             lrun[tid] = lrun[tid] * fac[tid] + sum;
         }
-        // ---- rare: a head's reference moved after O^T holds earlier chunks
+        // ---- rare: a head's reference moved after O^T (and L) hold earlier chunks
         if (flags[0]) {
             tc_fence_after();
             const int g = warp & 3;
-            for (int t = 0; t < 2; ++t) {
-                const int mt = (warp >> 2) * 2 + t;
-                for (int h0 = 0; h0 < H; h0 += 32) {
-                    const uint32_t ta = tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0;
+            for (int t = 0; t < 3; ++t) {
+                const int mt = (warp >> 2) * 3 + t;  // O^T tiles 0-3, L tile (4), spare (5)
+                if (mt > 4) break;
+                const uint32_t col = mt < 4 ? O_COL + 64 * mt : L_COL;
+                for (int h0 = 0; h0 < HG; h0 += 32) {
+                    const uint32_t ta = tmem + ((uint32_t)(g * 32) << 16) + col + h0;
                     uint32_t r[32];
                     tmem_ld32(ta, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        r[i] = __float_as_uint(__uint_as_float(r[i]) * fac[h0 + i]);
+                        if (h0 + i < HG) r[i] = __float_as_uint(__uint_as_float(r[i]) * fac[h0 + i]);
                     tmem_st32(ta, r);
                 }
             }
             tc_fence_before();
             __syncthreads();
         }
-        // ---- O^T += V^T P^T (one thread issues)
+        // ---- O^T += V^T P^T and L^T += ONES P^T (one thread issues)
         if (tid == 0) {
             tc_fence_after();
             for (int mt = 0; mt < DV / 128; ++mt)
@@ -550,6 +580,10 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_f16(tmem + O_COL + 64 * mt,
                             sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
                             sdesc(sP + kk * 2048u, K_ATOM, 1024), idPV, (it > 0 || kk > 0) ? 1u : 0u);
+            if (lmma)
+                for (int kk = 0; kk < CK / 16; ++kk)
+                    mma_f16(tmem + L_COL, ones_desc(sOnes), sdesc(sP + kk * 2048u, K_ATOM, 1024),
+                            idL, (it > 0 || kk > 0) ? 1u : 0u);
             mma_commit(bO);
         }
         ++npv;
@@ -559,58 +593,80 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool got = warp == 0 ? mbar_wait(bO, (c1 - c0 - 1) & 1, wait_ns) : true;
         ok = __syncthreads_and(got) != 0;
         tc_fence_after();
+        if (ok && lmma && warp == 0) {  // the row sums: every lane of the L tile holds them
+            for (int h0 = 0; h0 < HG; h0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + L_COL + h0, r);
+                tmem_wait_ld();
+                if (lane == 0)
+                    for (int i = 0; i < 32; ++i)
+                        if (h0 + i < HG) lrun[h0 + i] = __uint_as_float(r[i]);
+            }
+        }
+        __syncthreads();
     }
 
     pdl_trigger();  // only the epilogue is left: let the next kernel be scheduled
 
     const bool mine = ok && c0 < c1;
     if (cluster) {
-        // ---- the nsplit CTAs of this sequence form one cluster: each stores
-        // its unnormalised O and (m, l) (they stay in L2); after the cluster
-        // barrier CTA r pulls heads [r*hpc, (r+1)*hpc) of every CTA into its
-        // freed K tile with bulk copies and combines them
-        const size_t prow0 = (size_t)b * H * kMaxSplit;
+        // ---- the nsplit CTAs of this sequence and head group form one
+        // cluster.  Each writes its unnormalised O (HG heads x 512 channels,
+        // fp32) into its freed K tile and sends it to the partial buffer (rows
+        // [b][split][h], in L2) with bulk stores, plus (m, l) per head; after
+        // the cluster barrier CTA r pulls heads [r*hpc, (r+1)*hpc) of its group
+        // from every CTA back into its K tile and combines them.
+        float* po = a.part_o + (size_t)b * kMaxSplit * H * DV;
         if (mine) {
             const int g = warp & 3;
             for (int t = 0; t < 2; ++t) {
                 const int mt = (warp >> 2) * 2 + t;
-                const int d = mt * 128 + g * 32 + lane;
-                for (int h0 = 0; h0 < H; h0 += 32) {
+                const uint32_t d = mt * 128 + g * 32 + lane;
+                for (int h0 = 0; h0 < HG; h0 += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        __stcg(a.part_o + (prow0 + (size_t)(h0 + i) * kMaxSplit + split) * DV + d,
-                               __uint_as_float(r[i]));
+                        if (h0 + i < HG)
+                            asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(
+                                             sK + ((h0 + i) * DV + d) * 4),
+                                         "r"(r[i]));
                 }
             }
+            fence_async_smem();  // the rows before the bulk stores read them
         }
-        if (tid < H) {  // nothing (or nothing valid) from this CTA: weight 0
-            const size_t row = prow0 + (size_t)tid * kMaxSplit + split;
+        __syncthreads();
+        if (mine && tid == 0) {
+            for (int h = 0; h < HG; h += 8)  // 8 head rows (16 KB) per bulk store
+                asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(
+                                 po + ((size_t)split * H + hg0 + h) * DV),
+                             "r"(sK + (uint32_t)h * DV * 4), "r"(8 * DV * 4)
+                             : "memory");
+            asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;\n" ::: "memory");
+        }
+        if (tid < HG) {  // nothing (or nothing valid) from this CTA: weight 0
+            const size_t row = ((size_t)b * H + hg0 + tid) * kMaxSplit + split;
             __stcg(a.part_ml + row * 2, mine ? mref[tid] : -INFINITY);
             __stcg(a.part_ml + row * 2 + 1, mine ? lrun[tid] : 0.f);
         }
-        // generic-proxy stores before the peers' bulk (async-proxy) reads
         asm volatile("fence.proxy.async.global;\n" ::: "memory");
         cluster_sync();  // every CTA's partial is stored
         asm volatile("fence.proxy.async.global;\n" ::: "memory");
-        const int hpc = (H + nsplit - 1) / nsplit;
-        const int h_lo = split * hpc, h_hi = min(H, h_lo + hpc), nh = max(0, h_hi - h_lo);
+        const int hpc = (HG + nsplit - 1) / nsplit;
+        const int h_lo = hg0 + split * hpc, h_hi = min(hg0 + HG, h_lo + hpc);
+        const int nh = max(0, h_hi - h_lo);
         float* wts = lpart;  // [nh][nsplit] weights (nh * nsplit <= 64 + 8)
-        // rows (head hh, split s2) land at sK + (hh * nsplit + s2) * 2 KB
-        // (at most 72 rows: 144 KB of the 147 KB tile)
+        // source s2's rows land at sK + s2 * nh * 2 KB (at most 72 rows: 144 KB)
         if (tid == 0 && nh > 0) {
             mbar_expect_tx(bW, (uint32_t)(nh * nsplit) * DV * 4);
-            for (int hh = 0; hh < nh; ++hh)
-                for (int s2 = 0; s2 < nsplit; ++s2)
-                    bulk_load(sK + (uint32_t)(hh * nsplit + s2) * DV * 4,
-                              a.part_o + (prow0 + (size_t)(h_lo + hh) * kMaxSplit + s2) * DV,
-                              DV * 4, bW);
+            for (int s2 = 0; s2 < nsplit; ++s2)
+                bulk_load(sK + (uint32_t)(s2 * nh) * DV * 4, po + ((size_t)s2 * H + h_lo) * DV,
+                          (uint32_t)nh * DV * 4, bW);
         }
         if (tid < nh) {
             const int h = h_lo + tid;
-            const size_t row = prow0 + (size_t)h * kMaxSplit;
+            const size_t row = ((size_t)b * H + h) * kMaxSplit;
             float m[8], l[8];
             float M = -INFINITY;
 #pragma unroll
@@ -623,7 +679,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int s2 = 0; s2 < 8; ++s2) {
                 if (s2 >= nsplit) break;
-                const float w = (M == -INFINITY || m[s2] == -INFINITY) ? 0.f : exp2f(m[s2] - M);
+                const float w = (M == -INFINITY || m[s2] == -INFINITY) ? 0.f : ex2(m[s2] - M);
                 wts[tid * nsplit + s2] = w;
                 L += w * l[s2];
             }
@@ -644,7 +700,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int s2 = 0; s2 < nsplit; ++s2) {
                 const float w = wts[hh * nsplit + s2];
                 if (w == 0.f) continue;
-                const float4 v = reinterpret_cast<const float4*>(rows + (hh * nsplit + s2) * DV)[d4];
+                const float4 v = reinterpret_cast<const float4*>(rows + (s2 * nh + hh) * DV)[d4];
                 acc.x = fmaf(w, v.x, acc.x);
                 acc.y = fmaf(w, v.y, acc.y);
                 acc.z = fmaf(w, v.z, acc.z);
@@ -660,36 +716,35 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int t = 0; t < 2; ++t) {
             const int mt = (warp >> 2) * 2 + t;
             const int d = mt * 128 + g * 32 + lane;
-            for (int h0 = 0; h0 < H; h0 += 32) {
+            for (int h0 = 0; h0 < HG; h0 += 32) {
                 uint32_t r[32] = {};
                 if (mine) {
                     tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
                     tmem_wait_ld();
                 }
-                if (nsplit == 1) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 32; ++i) {
+                    if (h0 + i >= HG) break;
+                    const int h = hg0 + h0 + i;
+                    if (nsplit == 1) {
                         const float l = mine ? lrun[h0 + i] : 0.f;
-                        a.out[((size_t)b * H + h0 + i) * DV + d] =
-                            l > 0.f ? __uint_as_float(r[i]) / l : 0.f;
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        a.part_o[(((size_t)b * H + h0 + i) * kMaxSplit + split) * DV + d] =
+                        a.out[((size_t)b * H + h) * DV + d] = l > 0.f ? __uint_as_float(r[i]) / l : 0.f;
+                    } else {
+                        a.part_o[(((size_t)b * H + h) * kMaxSplit + split) * DV + d] =
                             __uint_as_float(r[i]);
+                    }
                 }
             }
         }
     }
-    if (!cluster && tid < H) {
+    if (!cluster && tid < HG) {
         const float m = mine ? mref[tid] : -INFINITY, l = mine ? lrun[tid] : 0.f;
+        const int h = hg0 + tid;
         if (nsplit == 1) {
             if (a.lse)
-                a.lse[(size_t)b * H + tid] =
-                    l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+                a.lse[(size_t)b * H + h] = l > 0.f ? (m + __log2f(l)) * 0.6931471805599453f : -INFINITY;
         } else {
-            const size_t row = ((size_t)b * H + tid) * kMaxSplit + split;
+            const size_t row = ((size_t)b * H + h) * kMaxSplit + split;
             a.part_ml[row * 2] = m;
             a.part_ml[row * 2 + 1] = l;
         }
@@ -701,8 +756,10 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (nqk > 0) mbar_wait(bS, (nqk - 1) & 1, kCleanupWaitNs);
         if (npv > 0) mbar_wait(bO, (npv - 1) & 1, kCleanupWaitNs);
         if (nw > 0) mbar_wait(bW, (nw - 1) & 1, kCleanupWaitNs);
-        if (win) mbar_wait(bQ, 0, kCleanupWaitNs);
     }
+    // the query rows' TMA must have landed before the CTA exits (a CTA with
+    // no chunk never waited for it)
+    if (tid == 0 && (!ok || c0 >= c1)) mbar_wait(bQ, 0, kCleanupWaitNs);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -756,7 +813,7 @@ void set_device_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns; }
 template <int G>
 static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const dim3& grid,
                             int cluster_x, const AttnArgs& a, const Shape& sh, int K, float sm_log2,
-                            int rsplit, int cpr, int nsplit, int cluster, cudaStream_t s) {
+                            int rsplit, int cpr, int nsplit, int cluster, int HG, cudaStream_t s) {
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -782,7 +839,7 @@ static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const 
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, t128::attn_t128_kernel<G>, tq, tw, a, sh, K, sm_log2, rsplit,
-                              cpr, nsplit, cluster, g_wait_ns);
+                              cpr, nsplit, cluster, HG, g_wait_ns);
 }
 
 // Clusters of `size` CTAs of this kernel that can be resident at once on the
@@ -821,35 +878,48 @@ static int launch_t128_g(const kvc_config& c, const AttnArgs& a, const Shape& sh
     const int K = c.topk;
     const int rc = (K + t128::CK - 1) / t128::CK;
     const int wc = (a.window_len + t128::CK - 1) / t128::CK;
-    // one record chunk per CTA while the CTAs of a sequence fit one cluster
-    // and every sequence's cluster can be resident at once; else two or more
-    // chunks per record CTA (a chunk's loads overlap the previous one's
-    // products)
-    int cpr = 1;
-    while (rc > 0 && cpr < rc) {
-        const int ns = (rc + cpr - 1) / cpr + wc;
-        if (ns <= 8 && (ns == 1 || max_clusters<G>(ns) >= a.batch)) break;
-        ++cpr;
+    // Work split: the key chunks of a sequence go to one cluster of CTAs (one
+    // record chunk each while that fits in 8, else cpr), and the 64 heads to
+    // 64 / HG such clusters.  Fewest chunks per CTA first, then the most
+    // clusters (smallest head group) that can all be resident at once;
+    // without one, the largest head group with the fewest chunks per CTA.
+    int cpr = 0, HG = 64;
+    for (int cp = 1; cp <= std::max(rc, 1) && !cpr; ++cp) {
+        const int ns = (rc + cp - 1) / cp + wc;
+        if (ns > 8) continue;
+        for (int hg = 16; hg <= 64; hg *= 2) {
+            const long long clusters = (long long)a.batch * (64 / hg);
+            if (ns == 1 || max_clusters<G>(ns) >= clusters) {
+                cpr = cp;
+                HG = hg;
+                break;
+            }
+        }
+    }
+    if (!cpr) {
+        cpr = 1;
+        while (rc > 0 && cpr < rc && (rc + cpr - 1) / cpr + wc > 8) ++cpr;
+        HG = 64;
     }
     int rsplit = rc == 0 ? 0 : (rc + cpr - 1) / cpr;
     int nsplit = rsplit + wc;
-    if (nsplit == 0) {  // nothing to attend: one CTA writes zeros and -inf
+    if (nsplit == 0) {  // nothing to attend: one CTA per head group writes zeros and -inf
         rsplit = 1;
         nsplit = 1;
     }
     if (nsplit > kMaxSplit) return -1;
     const int cluster = (nsplit > 1 && nsplit <= 8) ? 1 : 0;
+    // every CTA's query rows arrive by TMA (boxes of HG rows); so do bf16
+    // window rows
     CUtensorMap tq = {}, tw = {};
-    if (wc > 0) {  // the window chunk's query tile and (bf16) rows arrive by TMA
-        if (!encode_rows(&tq, a.q, (unsigned long long)a.batch * t128::H, t128::H)) return -1;
-        if (!a.win_fp8 &&
-            !encode_rows(&tw, a.window, (unsigned long long)a.batch * a.window_stride, t128::CK))
-            return -1;
-    }
+    if (!encode_rows(&tq, a.q, (unsigned long long)a.batch * t128::H, HG)) return -1;
+    if (wc > 0 && !a.win_fp8 &&
+        !encode_rows(&tw, a.window, (unsigned long long)a.batch * a.window_stride, t128::CK))
+        return -1;
     const float sm_log2 = c.sm_scale * 1.4426950408889634f;
     trace_before("attn_t128", s);
-    const cudaError_t e = launch_g<G>(tq, tw, dim3(nsplit, a.batch), cluster ? nsplit : 1, a, sh, K,
-                                      sm_log2, rsplit, cpr, nsplit, cluster, s);
+    const cudaError_t e = launch_g<G>(tq, tw, dim3(nsplit, 64 / HG, a.batch), cluster ? nsplit : 1,
+                                      a, sh, K, sm_log2, rsplit, cpr, nsplit, cluster, HG, s);
     trace_after(s);
     if (e != cudaSuccess) return -1;
     return cluster ? 1 : nsplit;
