@@ -468,12 +468,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t ta_s = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL;
         if (warp < 4) {
 #pragma unroll 1
-            for (int h0 = 0; h0 < HG; h0 += 8) {
-                uint32_t r[8];
-                tmem_ld8(ta_s + h0, r);
+            for (int h0 = 0; h0 < HG; h0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(ta_s + h0, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     const float y = valid ? __uint_as_float(r[i]) * kf : -INFINITY;
                     const int m = __reduce_max_sync(0xffffffffu, f32_ord(y));
                     if (lane == ((h0 + i) & 31)) wmax[warp * 64 + h0 + i] = m;
@@ -497,17 +497,21 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();
         if (warp < 4) {
 #pragma unroll 1
-            for (int c8 = 0; c8 < HG / 8; ++c8) {
-                uint32_t r[8];
-                tmem_ld8(ta_s + 8 * c8, r);
+            for (int c16 = 0; c16 < HG / 16; ++c16) {
+                uint32_t r[16];
+                tmem_ld16(ta_s + 16 * c16, r);
                 tmem_wait_ld();
+#pragma unroll
+              for (int half8 = 0; half8 < 2; ++half8) {
+                const int c8 = 2 * c16 + half8;
                 uint32_t w[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int h = 8 * c8 + 2 * u;
                     const float m0 = mref[h], m1 = mref[h + 1];
-                    const float y0 = valid ? __uint_as_float(r[2 * u]) * kf : -INFINITY;
-                    const float y1 = valid ? __uint_as_float(r[2 * u + 1]) * kf : -INFINITY;
+                    const float y0 = valid ? __uint_as_float(r[8 * half8 + 2 * u]) * kf : -INFINITY;
+                    const float y1 =
+                        valid ? __uint_as_float(r[8 * half8 + 2 * u + 1]) * kf : -INFINITY;
                     float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, qs[h], -m0));
                     float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, qs[h + 1], -m1));
                     if (fp8) {  // v = scale x E4M3 row: the scale moves onto p
@@ -517,6 +521,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     w[u] = win ? pack_bf16(p0, p1) : pack_f16(p0, p1);
                 }
                 sts128(sP + swz(s, c8), w[0], w[1], w[2], w[3]);
+              }
             }
         }
         if (!lmma) {
@@ -611,17 +616,43 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const bool mine = ok && c0 < c1;
     if (cluster) {
         // ---- the nsplit CTAs of this sequence and head group form one
-        // cluster.  Each writes its unnormalised O (HG heads x 512 channels,
-        // fp32) into its freed K tile and sends it to the partial buffer (rows
-        // [b][split][h], in L2) with bulk stores, plus (m, l) per head; after
-        // the cluster barrier CTA r pulls heads [r*hpc, (r+1)*hpc) of its group
-        // from every CTA back into its K tile and combines them.
-        float* po = a.part_o + (size_t)b * kMaxSplit * H * DV;
+        // cluster; CTA r owns heads [r*hpc, (r+1)*hpc) of the group.  Once
+        // every CTA's products are done (cluster barrier), each CTA stores its
+        // unnormalised O columns (from tensor memory, a lane per channel) and
+        // its (m, l) straight into the owners' shared memory -- rows [src][hh]
+        // of 2 KB in the owner's freed K tile -- and after a second cluster
+        // barrier every owner combines its rows locally and writes the output.
+        const int hpc = (HG + nsplit - 1) / nsplit;
+        const int h_lo = split * hpc, nh = max(0, min(HG, h_lo + hpc) - h_lo);
+        uint32_t* dst_off = reinterpret_cast<uint32_t*>(misc + M_KS);  // [HG] owner row addresses
+        float* mlx = lpart;                                            // [nsplit][nh][2]
+        float* wts = reinterpret_cast<float*>(wmax);                   // [nh][nsplit]
+        if (tid < HG) {
+            const int r = tid / hpc, hh = tid - r * hpc;
+            const int nh_r = min(hpc, HG - r * hpc);
+            uint32_t rk, rm;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rk) : "r"(sK), "r"(r));
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                         : "=r"(rm)
+                         : "r"(smem_u32(mlx)), "r"(r));
+            dst_off[tid] = rk + (uint32_t)(split * nh_r + hh) * DV * 4;
+            ks[64 + tid] = __uint_as_float(rm + (uint32_t)(split * nh_r + hh) * 8);
+        }
+        tc_fence_before();
+        cluster_sync();  // every CTA of the cluster is past its last product
+        tc_fence_after();
+        if (tid < HG) {
+            const float m = mine ? mref[tid] : -INFINITY, l = mine ? lrun[tid] : 0.f;
+            asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(
+                             __float_as_uint(ks[64 + tid])),
+                         "f"(m), "f"(l)
+                         : "memory");
+        }
         if (mine) {
             const int g = warp & 3;
             for (int t = 0; t < 2; ++t) {
                 const int mt = (warp >> 2) * 2 + t;
-                const uint32_t d = mt * 128 + g * 32 + lane;
+                const uint32_t d4 = (mt * 128 + g * 32 + lane) * 4;
                 for (int h0 = 0; h0 < HG; h0 += 32) {
                     uint32_t r[32];
                     tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
@@ -629,85 +660,44 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (h0 + i < HG)
-                            asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(
-                                             sK + ((h0 + i) * DV + d) * 4),
-                                         "r"(r[i]));
+                            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dst_off[h0 + i] + d4),
+                                         "r"(r[i])
+                                         : "memory");
                 }
             }
-            fence_async_smem();  // the rows before the bulk stores read them
         }
-        __syncthreads();
-        if (mine && tid == 0) {
-            for (int h = 0; h < HG; h += 8)  // 8 head rows (16 KB) per bulk store
-                asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(
-                                 po + ((size_t)split * H + hg0 + h) * DV),
-                             "r"(sK + (uint32_t)h * DV * 4), "r"(8 * DV * 4)
-                             : "memory");
-            asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;\n" ::: "memory");
-        }
-        if (tid < HG) {  // nothing (or nothing valid) from this CTA: weight 0
-            const size_t row = ((size_t)b * H + hg0 + tid) * kMaxSplit + split;
-            __stcg(a.part_ml + row * 2, mine ? mref[tid] : -INFINITY);
-            __stcg(a.part_ml + row * 2 + 1, mine ? lrun[tid] : 0.f);
-        }
-        asm volatile("fence.proxy.async.global;\n" ::: "memory");
-        cluster_sync();  // every CTA's partial is stored
-        asm volatile("fence.proxy.async.global;\n" ::: "memory");
-        const int hpc = (HG + nsplit - 1) / nsplit;
-        const int h_lo = hg0 + split * hpc, h_hi = min(hg0 + HG, h_lo + hpc);
-        const int nh = max(0, h_hi - h_lo);
-        float* wts = lpart;  // [nh][nsplit] weights (nh * nsplit <= 64 + 8)
-        // source s2's rows land at sK + s2 * nh * 2 KB (at most 72 rows: 144 KB)
-        if (tid == 0 && nh > 0) {
-            mbar_expect_tx(bW, (uint32_t)(nh * nsplit) * DV * 4);
-            for (int s2 = 0; s2 < nsplit; ++s2)
-                bulk_load(sK + (uint32_t)(s2 * nh) * DV * 4, po + ((size_t)s2 * H + h_lo) * DV,
-                          (uint32_t)nh * DV * 4, bW);
-        }
+        cluster_sync();  // every row and (m, l) has arrived
         if (tid < nh) {
-            const int h = h_lo + tid;
-            const size_t row = ((size_t)b * H + h) * kMaxSplit;
-            float m[8], l[8];
             float M = -INFINITY;
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) {
-                m[s2] = s2 < nsplit ? __ldcg(a.part_ml + (row + s2) * 2) : -INFINITY;
-                l[s2] = s2 < nsplit ? __ldcg(a.part_ml + (row + s2) * 2 + 1) : 0.f;
-                M = fmaxf(M, m[s2]);
-            }
+            for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, mlx[(s2 * nh + tid) * 2]);
             float L = 0.f;
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) {
-                if (s2 >= nsplit) break;
-                const float w = (M == -INFINITY || m[s2] == -INFINITY) ? 0.f : ex2(m[s2] - M);
+            for (int s2 = 0; s2 < nsplit; ++s2) {
+                const float m = mlx[(s2 * nh + tid) * 2], l = mlx[(s2 * nh + tid) * 2 + 1];
+                const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : ex2(m - M);
                 wts[tid * nsplit + s2] = w;
-                L += w * l[s2];
+                L += w * l;
             }
             fac[tid] = L > 0.f ? 1.f / L : 0.f;
             if (a.lse)
-                a.lse[(size_t)b * H + h] = L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f
-                                                   : -INFINITY;
+                a.lse[(size_t)b * H + hg0 + h_lo + tid] =
+                    L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f : -INFINITY;
         }
-        bool got = true;
-        if (nh > 0 && warp == 0) got = mbar_wait(bW, (uint32_t)nw & 1u, wait_ns);
-        if (nh > 0) ++nw;
-        const bool landed = __syncthreads_and(got) != 0;
-        if (!landed) ok = false;
+        __syncthreads();
         const float* rows = reinterpret_cast<const float*>(smem + OFF_K);
-        for (int it2 = tid; landed && it2 < nh * (DV / 4); it2 += NT) {
-            const int hh = it2 / (DV / 4), d4 = it2 - hh * (DV / 4);
+        for (int it2 = tid; it2 < nh * (DV / 4); it2 += NT) {
+            const int hh = it2 / (DV / 4), q4 = it2 - hh * (DV / 4);
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int s2 = 0; s2 < nsplit; ++s2) {
                 const float w = wts[hh * nsplit + s2];
                 if (w == 0.f) continue;
-                const float4 v = reinterpret_cast<const float4*>(rows + (s2 * nh + hh) * DV)[d4];
+                const float4 v = reinterpret_cast<const float4*>(rows + (s2 * nh + hh) * DV)[q4];
                 acc.x = fmaf(w, v.x, acc.x);
                 acc.y = fmaf(w, v.y, acc.y);
                 acc.z = fmaf(w, v.z, acc.z);
                 acc.w = fmaf(w, v.w, acc.w);
             }
             const float inv = fac[hh];
-            *reinterpret_cast<float4*>(a.out + ((size_t)b * H + h_lo + hh) * DV + 4 * d4) =
+            *reinterpret_cast<float4*>(a.out + ((size_t)b * H + hg0 + h_lo + hh) * DV + 4 * q4) =
                 make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         }
     } else if (nsplit == 1 || mine) {
