@@ -247,8 +247,9 @@ __device__ __forceinline__ uint64_t ones_desc(uint32_t saddr) {
 template <int G>
 __global__ void __launch_bounds__(NT, 1)
 attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_w,
-                 AttnArgs a, Shape sh, int K, float sm_log2, int rsplit, int cpr, int nsplit,
-                 int cluster, int HG, unsigned long long wait_ns) {
+                 const __grid_constant__ CUtensorMap tm_qw, AttnArgs a, Shape sh, int K,
+                 float sm_log2, int rsplit, int cpr, int nsplit, int cluster, int HG, int WH,
+                 unsigned long long wait_ns) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;  // 1024-byte alignment for the swizzle
@@ -593,9 +594,164 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         ++npv;
     }
-    // the last chunk's PV must be complete before O^T is read
+    // ---- folded window: with WH > 0 the window chunk has no CTA of its own;
+    // record CTA r also attends over the window rows for heads [r WH, r WH +
+    // WH) of its group (bf16 operands, the window-head query rows by TMA),
+    // updating those heads' running softmax and O^T in place.
+    int nq = 1;  // query-row copies issued on bQ
+    if (WH > 0 && !a.win_fp8 && ok && c0 < c1) {  // (the launcher folds bf16 windows only)
+        const int wh0 = split * WH;
+        const uint32_t qw_atom = (uint32_t)WH * 128u;
+        // the K tile, P^T and the query rows are free once the last PV is done
+        {
+            const bool got = warp == 0 ? mbar_wait(bO, (npv - 1) & 1, wait_ns) : true;
+            ok = __syncthreads_and(got) != 0;
+        }
+        tc_fence_after();
+        if (ok) {
+            if (tid < CK) kidx[tid] = tid < W ? tid : -1;
+            if (tid == 0) {
+                mbar_expect_tx(bW, NATOM * K_ATOM);
+                for (int at = 0; at < NATOM; ++at)
+                    tma_load_2d(sK + at * K_ATOM, &tm_w, 64 * at, b * a.window_stride, bW);
+                mbar_expect_tx(bQ, NATOM * qw_atom);
+                for (int at = 0; at < NATOM; ++at)
+                    tma_load_2d(sQ + at * qw_atom, &tm_qw, 64 * at, b * H + hg0 + wh0, bQ);
+            }
+            ++nw;
+            ++nq;
+            {  // the ones block in bf16 for the window's row sums
+                asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(sOnes + 8 * tid),
+                             "r"(0x3F803F80u));
+            }
+            const bool got = warp == 0 ? (mbar_wait(bW, 0, wait_ns) && mbar_wait(bQ, 1, wait_ns))
+                                       : true;
+            ok = __syncthreads_and(got) != 0;
+        }
+        if (ok) {
+            const int kw = kidx[s];
+            if (kw < 0) zero_row_half(sK, s, half);  // rows past the window
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t idQKw = idesc_f16(128, WH, 1, 0, 0);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t at = kk >> 2, koff = (kk & 3) * 32;
+                    mma_f16(tmem + S_COL, sdesc(sK + at * K_ATOM + koff, 16, 1024),
+                            sdesc(sQ + at * qw_atom + koff, 16, 1024), idQKw, kk > 0);
+                }
+                mma_commit(bS);
+            }
+            ++nqk;
+            const bool got = warp == 0 ? mbar_wait(bS, (nqk - 1) & 1, wait_ns) : true;
+            ok = __syncthreads_and(got) != 0;
+            tc_fence_after();
+            const bool valid = kw >= 0;
+            const uint32_t ta_s = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL;
+            if (ok && warp < 4) {
+#pragma unroll 1
+                for (int h0 = 0; h0 < WH; h0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(ta_s + h0, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float y = valid ? __uint_as_float(r[i]) : -INFINITY;
+                        const int m = __reduce_max_sync(0xffffffffu, f32_ord(y));
+                        if (lane == ((h0 + i) & 31)) wmax[warp * 64 + h0 + i] = m;
+                    }
+                }
+            }
+            if (tid == 0) flags[0] = 0;
+            __syncthreads();
+            if (ok && tid < HG) {
+                float f = 1.f;
+                if (tid >= wh0 && tid < wh0 + WH) {
+                    float my = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) my = fmaxf(my, ord_f32(wmax[w * 64 + tid - wh0]));
+                    const float mc = my * sm_log2;
+                    const float mo = mref[tid];
+                    const float mn = (mo == -INFINITY || mc > mo + kRescaleSlack) ? mc : mo;
+                    f = mo == -INFINITY ? 0.f : ex2(mo - mn);
+                    mref[tid] = mn;
+                    if (f != 1.f) flags[0] = 1;
+                }
+                fac[tid] = f;
+            }
+            __syncthreads();
+            if (ok && warp < 4) {
+                // P^T row of this key: the window heads' weights, zeros elsewhere
+#pragma unroll 1
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    const int h8 = 8 * c8;
+                    if (h8 >= wh0 && h8 < wh0 + WH) {
+                        uint32_t r[8];
+                        tmem_ld8(ta_s + (h8 - wh0), r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int h = h8 + 2 * u;
+                            const float m0 = mref[h], m1 = mref[h + 1];
+                            const float y0 = valid ? __uint_as_float(r[2 * u]) : -INFINITY;
+                            const float y1 = valid ? __uint_as_float(r[2 * u + 1]) : -INFINITY;
+                            const float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, sm_log2, -m0));
+                            const float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, sm_log2, -m1));
+                            w[u] = pack_bf16(p0, p1);
+                        }
+                    }
+                    sts128(sP + swz(s, c8), w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (ok && flags[0]) {  // window heads whose reference moved: rescale O^T and L
+                tc_fence_after();
+                const int g = warp & 3;
+                for (int t = 0; t < 3; ++t) {
+                    const int mt = (warp >> 2) * 3 + t;
+                    if (mt > 4) break;
+                    const uint32_t col = mt < 4 ? O_COL + 64 * mt : L_COL;
+                    for (int h0 = 0; h0 < HG; h0 += 32) {
+                        const uint32_t ta = tmem + ((uint32_t)(g * 32) << 16) + col + h0;
+                        uint32_t r[32];
+                        tmem_ld32(ta, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (h0 + i < HG)
+                                r[i] = __float_as_uint(__uint_as_float(r[i]) * fac[h0 + i]);
+                        tmem_st32(ta, r);
+                    }
+                }
+                tc_fence_before();
+                __syncthreads();
+            }
+            if (ok && tid == 0) {
+                tc_fence_after();
+                const uint32_t idPVw = idesc_f16(128, 64, 1, 1, 1);
+                const uint32_t idLw = idesc_f16(128, 64, 1, 0, 1);
+                for (int mt = 0; mt < DV / 128; ++mt)
+                    for (int kk = 0; kk < CK / 16; ++kk)
+                        mma_f16(tmem + O_COL + 64 * mt,
+                                sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
+                                sdesc(sP + kk * 2048u, K_ATOM, 1024), idPVw, 1u);
+                for (int kk = 0; kk < CK / 16; ++kk)
+                    mma_f16(tmem + L_COL, ones_desc(sOnes), sdesc(sP + kk * 2048u, K_ATOM, 1024),
+                            idLw, 1u);
+                mma_commit(bO);
+            }
+            if (ok) ++npv;
+        }
+    }
+
+    // the last PV must be complete before O^T is read
     if (ok && c1 > c0) {
-        const bool got = warp == 0 ? mbar_wait(bO, (c1 - c0 - 1) & 1, wait_ns) : true;
+        const bool got = warp == 0 ? mbar_wait(bO, (npv - 1) & 1, wait_ns) : true;
         ok = __syncthreads_and(got) != 0;
         tc_fence_after();
         if (ok && lmma && warp == 0) {  // the row sums: every lane of the L tile holds them
@@ -749,7 +905,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     // the query rows' TMA must have landed before the CTA exits (a CTA with
     // no chunk never waited for it)
-    if (tid == 0 && (!ok || c0 >= c1)) mbar_wait(bQ, 0, kCleanupWaitNs);
+    if (tid == 0 && (!ok || c0 >= c1)) mbar_wait(bQ, (nq - 1) & 1, kCleanupWaitNs);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -801,9 +957,10 @@ unsigned long long device_wait_limit_ns() { return g_wait_ns; }
 void set_device_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns; }
 
 template <int G>
-static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const dim3& grid,
-                            int cluster_x, const AttnArgs& a, const Shape& sh, int K, float sm_log2,
-                            int rsplit, int cpr, int nsplit, int cluster, int HG, cudaStream_t s) {
+static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& tqw,
+                            const dim3& grid, int cluster_x, const AttnArgs& a, const Shape& sh,
+                            int K, float sm_log2, int rsplit, int cpr, int nsplit, int cluster,
+                            int HG, int WH, cudaStream_t s) {
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -828,8 +985,8 @@ static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const 
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, t128::attn_t128_kernel<G>, tq, tw, a, sh, K, sm_log2, rsplit,
-                              cpr, nsplit, cluster, HG, g_wait_ns);
+    return cudaLaunchKernelEx(&cfg, t128::attn_t128_kernel<G>, tq, tw, tqw, a, sh, K, sm_log2,
+                              rsplit, cpr, nsplit, cluster, HG, WH, g_wait_ns);
 }
 
 // Clusters of `size` CTAs of this kernel that can be resident at once on the
@@ -891,8 +1048,25 @@ static int launch_t128_g(const kvc_config& c, const AttnArgs& a, const Shape& sh
         while (rc > 0 && cpr < rc && (rc + cpr - 1) / cpr + wc > 8) ++cpr;
         HG = 64;
     }
+    // When that split needs two or more record chunks per CTA, a window of
+    // one chunk can instead be folded into the record CTAs (each takes the
+    // window for HG / rc of the group's heads) if every sequence's cluster of
+    // rc CTAs can then be resident: one chunk and a window slice per CTA.
+    int WH = 0;
+    if (cpr > 1 && wc == 1 && rc >= 2 && rc <= 8 && !a.win_fp8) {  // bf16 window rows only
+        for (int hg = 16; hg <= 64; hg *= 2) {
+            if (hg % rc || (hg / rc) % 16) continue;
+            if (max_clusters<G>(rc) >= (long long)a.batch * (64 / hg)) {
+                cpr = 1;
+                HG = hg;
+                WH = hg / rc;
+                break;
+            }
+        }
+    }
+    const int wsplit = WH ? 0 : wc;  // window chunks with a CTA of their own
     int rsplit = rc == 0 ? 0 : (rc + cpr - 1) / cpr;
-    int nsplit = rsplit + wc;
+    int nsplit = rsplit + wsplit;
     if (nsplit == 0) {  // nothing to attend: one CTA per head group writes zeros and -inf
         rsplit = 1;
         nsplit = 1;
@@ -900,16 +1074,18 @@ static int launch_t128_g(const kvc_config& c, const AttnArgs& a, const Shape& sh
     if (nsplit > kMaxSplit) return -1;
     const int cluster = (nsplit > 1 && nsplit <= 8) ? 1 : 0;
     // every CTA's query rows arrive by TMA (boxes of HG rows); so do bf16
-    // window rows
-    CUtensorMap tq = {}, tw = {};
+    // window rows, and the folded window's query rows (boxes of WH rows)
+    CUtensorMap tq = {}, tw = {}, tqw = {};
     if (!encode_rows(&tq, a.q, (unsigned long long)a.batch * t128::H, HG)) return -1;
     if (wc > 0 && !a.win_fp8 &&
         !encode_rows(&tw, a.window, (unsigned long long)a.batch * a.window_stride, t128::CK))
         return -1;
+    if (WH && !encode_rows(&tqw, a.q, (unsigned long long)a.batch * t128::H, WH)) return -1;
     const float sm_log2 = c.sm_scale * 1.4426950408889634f;
     trace_before("attn_t128", s);
-    const cudaError_t e = launch_g<G>(tq, tw, dim3(nsplit, 64 / HG, a.batch), cluster ? nsplit : 1,
-                                      a, sh, K, sm_log2, rsplit, cpr, nsplit, cluster, HG, s);
+    const cudaError_t e = launch_g<G>(tq, tw, tqw, dim3(nsplit, 64 / HG, a.batch),
+                                      cluster ? nsplit : 1, a, sh, K, sm_log2, rsplit, cpr, nsplit,
+                                      cluster, HG, WH, s);
     trace_after(s);
     if (e != cudaSuccess) return -1;
     return cluster ? 1 : nsplit;

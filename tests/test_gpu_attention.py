@@ -136,9 +136,9 @@ def test_attention_online_rescale(kvc):
 
 @pytest.mark.parametrize("topk", [192, 1024, 2048])
 def test_attention_split_counts(kvc, topk):
-    """Key counts that give 4 splits per sequence (merged inside a thread-block
-    cluster) and 12 splits of one and of two chunks each (more than a cluster
-    holds: merged by the separate merge kernel)."""
+    """Key counts that give 2 record chunks and a window chunk per sequence,
+    and more record chunks than a cluster holds one per CTA (2 and 3 chunks
+    per CTA, merged inside the cluster)."""
     w = synth.WORKLOADS["mla32k"].scaled(context=2 * 5000, topk=topk, batch=3)
     inp, rec, ic, n, cfg, cache = _setup(kvc, w)
     ocfg = oracle_cfg(w)
@@ -148,4 +148,25 @@ def test_attention_split_counts(kvc, topk):
     ref, ref_lse, _ = oracle.sparse_decode(ocfg, f32(q), rec, n, tk, f32(win), w.window)
     assert st == 0
     assert_attn_close(out, ref, f"topk={topk}")
+    assert np.max(np.abs(lse - ref_lse)) < 2e-3 * np.abs(ref_lse).max()
+
+
+@pytest.mark.parametrize("window_len", [128, 100])
+def test_attention_wide_batch_folds_window(kvc, window_len):
+    """32 sequences: one CTA per record chunk plus a window CTA would not all
+    be resident as clusters, so each record CTA also takes the window for a
+    quarter of the heads (bf16, folded into its running softmax); ragged
+    lengths, padding, and a window shorter than its chunk."""
+    w = synth.WORKLOADS["mla32k"].scaled(batch=32, context=2 * 700)
+    inp, rec, ic, n, cfg, cache = _setup(kvc, w)
+    ocfg = oracle_cfg(w)
+    n2 = np.array([700 - 13 * (i % 9) for i in range(32)], np.int32)
+    cache.n_entries.copy_(torch.from_numpy(n2))
+    tk = oracle.index_topk(ocfg, inp["idx_q"][0].numpy(), ic, n2)
+    tk[3, 7:30] = -1
+    q, win = inp["q"][0], inp["windows"][0]
+    out, lse, st = _attn(kvc, cfg, cache, q, torch.from_numpy(tk), win, window_len)
+    ref, ref_lse, _ = oracle.sparse_decode(ocfg, f32(q), rec, n2, tk, f32(win), window_len)
+    assert st == 0
+    assert_attn_close(out, ref, f"wide batch, window {window_len}")
     assert np.max(np.abs(lse - ref_lse)) < 2e-3 * np.abs(ref_lse).max()
