@@ -247,8 +247,8 @@ __device__ __forceinline__ uint64_t ones_desc(uint32_t saddr) {
 template <int G>
 __global__ void __launch_bounds__(NT, 1)
 attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_w,
-                 const __grid_constant__ CUtensorMap tm_qw, AttnArgs a, Shape sh, int K,
-                 float sm_log2, int rsplit, int cpr, int nsplit, int cluster, int HG, int WH,
+                 const __grid_constant__ CUtensorMap tm_wr, AttnArgs a, Shape sh, int K,
+                 float sm_log2, int rsplit, int cpr, int nsplit, int cluster, int HG, int WR,
                  unsigned long long wait_ns) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -323,6 +323,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
     int nqk = 0, npv = 0, nw = 0;  // commits / copies issued (for the cleanup waits)
+    int nq = 1;                    // query-tile copies issued on bQ
     const int s = tid & (CK - 1), half = tid >> 7;  // key and half row (window paths)
     const uint8_t* recs = a.records + (size_t)b * a.capacity * sh.rb;
     // ---- slot table of chunk c: record index, window row, or -1 (masked)
@@ -459,6 +460,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         tc_fence_after();
         if (!ok) break;
+        // folded window: the last record product has read the f16 query tile;
+        // its bf16 original comes back by TMA while softmax and PV run
+        if (WR > 0 && !win && c == c1 - 1) {
+            if (tid == 0) tma_q();
+            nq = 2;
+        }
 
         // ---- softmax, warps 0-3: thread = key = tensor-memory lane.  y is
         // the raw logit (times the FP8 row scale); x = y * qs[h] in log2 units.
@@ -594,53 +601,53 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         ++npv;
     }
-    // ---- folded window: with WH > 0 the window chunk has no CTA of its own;
-    // record CTA r also attends over the window rows for heads [r WH, r WH +
-    // WH) of its group (bf16 operands, the window-head query rows by TMA),
-    // updating those heads' running softmax and O^T in place.
-    int nq = 1;  // query-row copies issued on bQ
-    if (WH > 0 && !a.win_fp8 && ok && c0 < c1) {  // (the launcher folds bf16 windows only)
-        const int wh0 = split * WH;
-        const uint32_t qw_atom = (uint32_t)WH * 128u;
-        // the K tile, P^T and the query rows are free once the last PV is done
-        {
+    // ---- folded window: with WR > 0 the window chunk has no CTA of its own;
+    // record CTA r also attends over window rows [r WR, r WR + WR) for every
+    // head of its group (bf16 operands), updating the running softmax and O^T
+    // in place.  The rows land by TMA as packed atoms of WR rows in the freed
+    // K tile (the product's A operand reads 128 rows from each atom start; the
+    // logits of rows past WR are masked), P^T after them.
+    if (WR > 0 && !win && !a.win_fp8 && ok && c0 < c1) {  // (bf16 window rows only)
+        const int r0 = split * WR;
+        const uint32_t w_atom = (uint32_t)WR * 128u;
+        const uint32_t sPw = sK + 9 * w_atom + 16384u;
+        {  // the K tile and P^T are free once the last record PV is done
             const bool got = warp == 0 ? mbar_wait(bO, (npv - 1) & 1, wait_ns) : true;
             ok = __syncthreads_and(got) != 0;
         }
         tc_fence_after();
         if (ok) {
-            if (tid < CK) kidx[tid] = tid < W ? tid : -1;
+            if (tid < CK) kidx[tid] = (tid < WR && r0 + tid < W) ? r0 + tid : -1;
             if (tid == 0) {
-                mbar_expect_tx(bW, NATOM * K_ATOM);
+                mbar_expect_tx(bW, NATOM * w_atom);
                 for (int at = 0; at < NATOM; ++at)
-                    tma_load_2d(sK + at * K_ATOM, &tm_w, 64 * at, b * a.window_stride, bW);
-                mbar_expect_tx(bQ, NATOM * qw_atom);
-                for (int at = 0; at < NATOM; ++at)
-                    tma_load_2d(sQ + at * qw_atom, &tm_qw, 64 * at, b * H + hg0 + wh0, bQ);
+                    tma_load_2d(sK + at * w_atom, &tm_wr, 64 * at, b * a.window_stride + r0, bW);
             }
             ++nw;
-            ++nq;
-            {  // the ones block in bf16 for the window's row sums
-                asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(sOnes + 8 * tid),
-                             "r"(0x3F803F80u));
-            }
-            const bool got = warp == 0 ? (mbar_wait(bW, 0, wait_ns) && mbar_wait(bQ, 1, wait_ns))
-                                       : true;
+            // the ones block in bf16 for the window's row sums
+            asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(sOnes + 8 * tid),
+                         "r"(0x3F803F80u));
+            const bool got =
+                warp == 0 ? (mbar_wait(bW, 0, wait_ns) && mbar_wait(bQ, 1, wait_ns)) : true;
             ok = __syncthreads_and(got) != 0;
         }
         if (ok) {
             const int kw = kidx[s];
-            if (kw < 0) zero_row_half(sK, s, half);  // rows past the window
+            if (s < WR && kw < 0) {  // rows past the window (read as other rows or zeros)
+#pragma unroll 1
+                for (int c16 = 36 * half; c16 < 36 * half + 36; ++c16)
+                    sts128(sK + (uint32_t)(c16 >> 3) * w_atom + swz(s, c16 & 7), 0u, 0u, 0u, 0u);
+            }
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
-                const uint32_t idQKw = idesc_f16(128, WH, 1, 0, 0);
+                const uint32_t idQKw = idesc_f16(128, HG, 1, 0, 0);
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t at = kk >> 2, koff = (kk & 3) * 32;
-                    mma_f16(tmem + S_COL, sdesc(sK + at * K_ATOM + koff, 16, 1024),
-                            sdesc(sQ + at * qw_atom + koff, 16, 1024), idQKw, kk > 0);
+                    mma_f16(tmem + S_COL, sdesc(sK + at * w_atom + koff, 16, 1024),
+                            sdesc(sQ + at * q_atom + koff, 16, 1024), idQKw, kk > 0);
                 }
                 mma_commit(bS);
             }
@@ -652,7 +659,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t ta_s = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL;
             if (ok && warp < 4) {
 #pragma unroll 1
-                for (int h0 = 0; h0 < WH; h0 += 16) {
+                for (int h0 = 0; h0 < HG; h0 += 16) {
                     uint32_t r[16];
                     tmem_ld16(ta_s + h0, r);
                     tmem_wait_ld();
@@ -667,49 +674,49 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (tid == 0) flags[0] = 0;
             __syncthreads();
             if (ok && tid < HG) {
-                float f = 1.f;
-                if (tid >= wh0 && tid < wh0 + WH) {
-                    float my = -INFINITY;
+                float my = -INFINITY;
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) my = fmaxf(my, ord_f32(wmax[w * 64 + tid - wh0]));
-                    const float mc = my * sm_log2;
-                    const float mo = mref[tid];
-                    const float mn = (mo == -INFINITY || mc > mo + kRescaleSlack) ? mc : mo;
-                    f = mo == -INFINITY ? 0.f : ex2(mo - mn);
-                    mref[tid] = mn;
-                    if (f != 1.f) flags[0] = 1;
-                }
+                for (int w = 0; w < 4; ++w) my = fmaxf(my, ord_f32(wmax[w * 64 + tid]));
+                const float mc = my * sm_log2;
+                const float mo = mref[tid];
+                const float mn = (mo == -INFINITY || mc > mo + kRescaleSlack) ? mc : mo;
+                const float f = mo == -INFINITY ? 0.f : ex2(mo - mn);
                 fac[tid] = f;
+                mref[tid] = mn;
+                if (f != 1.f) flags[0] = 1;
             }
             __syncthreads();
-            if (ok && warp < 4) {
-                // P^T row of this key: the window heads' weights, zeros elsewhere
+            // P^T rows of this CTA's window keys, by whole warps (the tensor-memory
+            // load is warp-collective; rows WR..31 come out as zeros, unread)
+            if (ok && warp < 4 && warp * 32 < WR) {
 #pragma unroll 1
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    uint32_t w[4] = {0u, 0u, 0u, 0u};
-                    const int h8 = 8 * c8;
-                    if (h8 >= wh0 && h8 < wh0 + WH) {
-                        uint32_t r[8];
-                        tmem_ld8(ta_s + (h8 - wh0), r);
-                        tmem_wait_ld();
+                for (int c16 = 0; c16 < HG / 16; ++c16) {
+                    uint32_t r[16];
+                    tmem_ld16(ta_s + 16 * c16, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int half8 = 0; half8 < 2; ++half8) {
+                        const int c8 = 2 * c16 + half8;
+                        uint32_t w[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const int h = h8 + 2 * u;
+                            const int h = 8 * c8 + 2 * u;
                             const float m0 = mref[h], m1 = mref[h + 1];
-                            const float y0 = valid ? __uint_as_float(r[2 * u]) : -INFINITY;
-                            const float y1 = valid ? __uint_as_float(r[2 * u + 1]) : -INFINITY;
+                            const float y0 = valid ? __uint_as_float(r[8 * half8 + 2 * u]) : -INFINITY;
+                            const float y1 =
+                                valid ? __uint_as_float(r[8 * half8 + 2 * u + 1]) : -INFINITY;
                             const float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, sm_log2, -m0));
                             const float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, sm_log2, -m1));
                             w[u] = pack_bf16(p0, p1);
                         }
+                        sts128(sPw + swz(s, c8), w[0], w[1], w[2], w[3]);
                     }
-                    sts128(sP + swz(s, c8), w[0], w[1], w[2], w[3]);
                 }
             }
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
-            if (ok && flags[0]) {  // window heads whose reference moved: rescale O^T and L
+            if (ok && flags[0]) {  // heads whose reference moved: rescale O^T and L
                 tc_fence_after();
                 const int g = warp & 3;
                 for (int t = 0; t < 3; ++t) {
@@ -736,12 +743,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint32_t idPVw = idesc_f16(128, 64, 1, 1, 1);
                 const uint32_t idLw = idesc_f16(128, 64, 1, 0, 1);
                 for (int mt = 0; mt < DV / 128; ++mt)
-                    for (int kk = 0; kk < CK / 16; ++kk)
+                    for (int kk = 0; kk < WR / 16; ++kk)
                         mma_f16(tmem + O_COL + 64 * mt,
-                                sdesc(sK + (2 * mt) * K_ATOM + kk * 2048u, K_ATOM, 1024),
-                                sdesc(sP + kk * 2048u, K_ATOM, 1024), idPVw, 1u);
-                for (int kk = 0; kk < CK / 16; ++kk)
-                    mma_f16(tmem + L_COL, ones_desc(sOnes), sdesc(sP + kk * 2048u, K_ATOM, 1024),
+                                sdesc(sK + (2 * mt) * w_atom + kk * 2048u, w_atom, 1024),
+                                sdesc(sPw + kk * 2048u, w_atom, 1024), idPVw, 1u);
+                for (int kk = 0; kk < WR / 16; ++kk)
+                    mma_f16(tmem + L_COL, ones_desc(sOnes), sdesc(sPw + kk * 2048u, w_atom, 1024),
                             idLw, 1u);
                 mma_commit(bO);
             }
@@ -957,10 +964,10 @@ unsigned long long device_wait_limit_ns() { return g_wait_ns; }
 void set_device_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns; }
 
 template <int G>
-static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& tqw,
+static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const CUtensorMap& twr,
                             const dim3& grid, int cluster_x, const AttnArgs& a, const Shape& sh,
                             int K, float sm_log2, int rsplit, int cpr, int nsplit, int cluster,
-                            int HG, int WH, cudaStream_t s) {
+                            int HG, int WR, cudaStream_t s) {
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -985,8 +992,8 @@ static cudaError_t launch_g(const CUtensorMap& tq, const CUtensorMap& tw, const 
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, t128::attn_t128_kernel<G>, tq, tw, tqw, a, sh, K, sm_log2,
-                              rsplit, cpr, nsplit, cluster, HG, WH, g_wait_ns);
+    return cudaLaunchKernelEx(&cfg, t128::attn_t128_kernel<G>, tq, tw, twr, a, sh, K, sm_log2,
+                              rsplit, cpr, nsplit, cluster, HG, WR, g_wait_ns);
 }
 
 // Clusters of `size` CTAs of this kernel that can be resident at once on the
@@ -1049,22 +1056,21 @@ static int launch_t128_g(const kvc_config& c, const AttnArgs& a, const Shape& sh
         HG = 64;
     }
     // When that split needs two or more record chunks per CTA, a window of
-    // one chunk can instead be folded into the record CTAs (each takes the
-    // window for HG / rc of the group's heads) if every sequence's cluster of
-    // rc CTAs can then be resident: one chunk and a window slice per CTA.
-    int WH = 0;
-    if (cpr > 1 && wc == 1 && rc >= 2 && rc <= 8 && !a.win_fp8) {  // bf16 window rows only
+    // one chunk can instead be folded into the record CTAs (each takes 128 /
+    // rc of the window rows, for all its heads) if every sequence's cluster
+    // of rc CTAs can then be resident: one chunk and a window slice per CTA.
+    int WR = 0;
+    if (cpr > 1 && wc == 1 && (rc == 2 || rc == 4 || rc == 8) && !a.win_fp8) {
         for (int hg = 16; hg <= 64; hg *= 2) {
-            if (hg % rc || (hg / rc) % 16) continue;
             if (max_clusters<G>(rc) >= (long long)a.batch * (64 / hg)) {
                 cpr = 1;
                 HG = hg;
-                WH = hg / rc;
+                WR = t128::CK / rc;
                 break;
             }
         }
     }
-    const int wsplit = WH ? 0 : wc;  // window chunks with a CTA of their own
+    const int wsplit = WR ? 0 : wc;  // window chunks with a CTA of their own
     int rsplit = rc == 0 ? 0 : (rc + cpr - 1) / cpr;
     int nsplit = rsplit + wsplit;
     if (nsplit == 0) {  // nothing to attend: one CTA per head group writes zeros and -inf
@@ -1074,18 +1080,19 @@ static int launch_t128_g(const kvc_config& c, const AttnArgs& a, const Shape& sh
     if (nsplit > kMaxSplit) return -1;
     const int cluster = (nsplit > 1 && nsplit <= 8) ? 1 : 0;
     // every CTA's query rows arrive by TMA (boxes of HG rows); so do bf16
-    // window rows, and the folded window's query rows (boxes of WH rows)
-    CUtensorMap tq = {}, tw = {}, tqw = {};
+    // window rows (boxes of a chunk, or of WR rows when folded)
+    CUtensorMap tq = {}, tw = {}, twr = {};
     if (!encode_rows(&tq, a.q, (unsigned long long)a.batch * t128::H, HG)) return -1;
     if (wc > 0 && !a.win_fp8 &&
         !encode_rows(&tw, a.window, (unsigned long long)a.batch * a.window_stride, t128::CK))
         return -1;
-    if (WH && !encode_rows(&tqw, a.q, (unsigned long long)a.batch * t128::H, WH)) return -1;
+    if (WR && !encode_rows(&twr, a.window, (unsigned long long)a.batch * a.window_stride, WR))
+        return -1;
     const float sm_log2 = c.sm_scale * 1.4426950408889634f;
     trace_before("attn_t128", s);
-    const cudaError_t e = launch_g<G>(tq, tw, tqw, dim3(nsplit, 64 / HG, a.batch),
+    const cudaError_t e = launch_g<G>(tq, tw, twr, dim3(nsplit, 64 / HG, a.batch),
                                       cluster ? nsplit : 1, a, sh, K, sm_log2, rsplit, cpr, nsplit,
-                                      cluster, HG, WH, s);
+                                      cluster, HG, WR, s);
     trace_after(s);
     if (e != cudaSuccess) return -1;
     return cluster ? 1 : nsplit;
