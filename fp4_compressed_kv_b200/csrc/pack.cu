@@ -68,6 +68,17 @@ struct Chunk<__nv_bfloat16> {
     __device__ __forceinline__ void load_shared(const __nv_bfloat16* p) {
         v = *reinterpret_cast<const uint4*>(p);
     }
+    // first read of a chunk (kept in L1 for the second pass) / its last read
+    __device__ __forceinline__ void load_keep(const __nv_bfloat16* p) {
+        asm volatile("ld.global.nc.L1::evict_last.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "l"(p));
+    }
+    __device__ __forceinline__ void load_last(const __nv_bfloat16* p) {
+        asm volatile("ld.global.nc.L1::evict_first.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "l"(p));
+    }
     __device__ __forceinline__ void store_shared(__nv_bfloat16* p) const {
         *reinterpret_cast<uint4*>(p) = v;
     }
@@ -75,6 +86,8 @@ struct Chunk<__nv_bfloat16> {
         const uint32_t w = t < 2 ? v.x : t < 4 ? v.y : t < 6 ? v.z : v.w;
         return (t & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
     }
+    // channels 2k, 2k + 1 as an fp32 pair (f2_* below)
+    __device__ __forceinline__ uint64_t pair(int k) const;
 };
 template <>
 struct Chunk<float> {
@@ -92,6 +105,22 @@ struct Chunk<float> {
         a = reinterpret_cast<const float4*>(p)[0];
         b = reinterpret_cast<const float4*>(p)[1];
     }
+    __device__ __forceinline__ void load_keep(const float* p) {
+        asm volatile("ld.global.nc.L1::evict_last.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(a.x), "=f"(a.y), "=f"(a.z), "=f"(a.w)
+                     : "l"(p));
+        asm volatile("ld.global.nc.L1::evict_last.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(b.x), "=f"(b.y), "=f"(b.z), "=f"(b.w)
+                     : "l"(p + 4));
+    }
+    __device__ __forceinline__ void load_last(const float* p) {
+        asm volatile("ld.global.nc.L1::evict_first.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(a.x), "=f"(a.y), "=f"(a.z), "=f"(a.w)
+                     : "l"(p));
+        asm volatile("ld.global.nc.L1::evict_first.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(b.x), "=f"(b.y), "=f"(b.z), "=f"(b.w)
+                     : "l"(p + 4));
+    }
     __device__ __forceinline__ void store_shared(float* p) const {
         reinterpret_cast<float4*>(p)[0] = a;
         reinterpret_cast<float4*>(p)[1] = b;
@@ -101,6 +130,7 @@ struct Chunk<float> {
         const int u = t & 3;
         return u == 0 ? q.x : u == 1 ? q.y : u == 2 ? q.z : q.w;
     }
+    __device__ __forceinline__ uint64_t pair(int k) const;
 };
 
 __device__ __forceinline__ void load8_gate(const float* p, float v[8]) {
@@ -135,6 +165,105 @@ __device__ __forceinline__ uint32_t e2m1x8_quotient(const float x[8], float s) {
 #pragma unroll
     for (int t = 0; t < 8; ++t) v[t] = fminf(fmaxf(__fdiv_rn(x[t], s), -6.f), 6.f);
     return e2m1x8_from_f32(v);
+}
+
+// ---- fp32 pairs: Blackwell's f32x2 instructions perform two IEEE
+// single-precision operations at once, each rounded exactly as its scalar
+// form, so pair arithmetic gives the bits of the scalar order it replaces.
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t p) { return __uint_as_float((uint32_t)p); }
+__device__ __forceinline__ float f2_hi(uint64_t p) { return __uint_as_float((uint32_t)(p >> 32)); }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t Chunk<__nv_bfloat16>::pair(int k) const {
+    const uint32_t w = k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+    return f2_make(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint64_t Chunk<float>::pair(int k) const {
+    return k == 0 ? f2_make(a.x, a.y) : k == 1 ? f2_make(a.z, a.w) : k == 2 ? f2_make(b.x, b.y)
+                                                                             : f2_make(b.z, b.w);
+}
+// max(|a|, |b|) in magnitude (the sign is that of neither), NaN if either is
+__device__ __forceinline__ float absmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// m / 6 correctly rounded (m >= 0 finite) without a division: the product by
+// c = RN(1/6) corrected once (q0 = m c; r = m - 6 q0, exact by one fma;
+// q = q0 + r c by a second), Markstein's correction step as used for division
+// by a constant known in advance (Brisebarre, Muller and Raina, 2004).  For
+// the divisor 6 it is correctly rounded for every m >= 2^-122 (all fp32
+// values checked); smaller m (subnormal quotients) are divided.
+__device__ __forceinline__ float div6_rn(float m) {
+    if (m < 0x1p-122f) return __fdiv_rn(m, 6.0f);
+    constexpr float c = 0x1.555556p-3f;
+    const float q0 = __fmul_rn(m, c);
+    const float r = __fmaf_rn(-q0, 6.0f, m);
+    return __fmaf_rn(r, c, q0);
+}
+
+// Eight E2M1 codes (raw: a zero keeps its sign) of four fp32 pairs in [-6, 6]
+// or saturating, element 2k + h (h = 0 low, 1 high half of pair k) in the
+// nibble of value 2k + h.
+__device__ __forceinline__ uint32_t e2m1x8_raw_f2(uint64_t p0, uint64_t p1, uint64_t p2,
+                                                  uint64_t p3) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .f32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+        "mov.b64 {l0, h0}, %1;\n\tmov.b64 {l1, h1}, %2;\n\t"
+        "mov.b64 {l2, h2}, %3;\n\tmov.b64 {l3, h3}, %4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, h0, l0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, h1, l1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, h2, l2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, h3, l3;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+    return w;
+}
+__device__ __forceinline__ uint32_t e2m1_clear_negzero(uint32_t w) {
+    const uint32_t mag = w & 0x77777777u;
+    const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;
+    return w & (0x77777777u | nonzero);
+}
+
+// e2m1x8_quotient for values held as four fp32 pairs, with the reciprocal and
+// its two brackets given (rl = RN(r (1 - 2^-20)), rh = RN(r (1 + 2^-20)),
+// r = RN(1 / s), s > 0 an E4M3 scale so r is finite): the same products,
+// two to an instruction, and the same exact fallback.
+__device__ __forceinline__ uint32_t e2m1x8_quotient_f2(const uint64_t v[4], float s, float rl,
+                                                       float rh) {
+    const uint64_t RL = f2_make(rl, rl), RH = f2_make(rh, rh);
+    const uint32_t cl =
+        e2m1x8_raw_f2(f2_mul(v[0], RL), f2_mul(v[1], RL), f2_mul(v[2], RL), f2_mul(v[3], RL));
+    const uint32_t ch =
+        e2m1x8_raw_f2(f2_mul(v[0], RH), f2_mul(v[1], RH), f2_mul(v[2], RH), f2_mul(v[3], RH));
+    if (cl == ch) return e2m1_clear_negzero(cl);
+    float q[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        q[2 * k] = fminf(fmaxf(__fdiv_rn(f2_lo(v[k]), s), -6.f), 6.f);
+        q[2 * k + 1] = fminf(fmaxf(__fdiv_rn(f2_hi(v[k]), s), -6.f), 6.f);
+    }
+    return e2m1x8_from_f32(q);
 }
 
 constexpr int kThreads = 256;
@@ -286,51 +415,73 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
 
-// Streaming form of pack_kernel for groups of at most 64 channels (a group's
-// chunks then sit in the team's lanes at the same chunk step): the same
-// arithmetic in the same order, but no token chunk is held across the whole
-// entry.  Pass 1 streams the chunks for the gate; pass 2 reloads each chunk
-// (from L1/L2), forms the entry values, takes the group maximum across the
-// team and quantises it right away.  The register footprint drops to a
-// fraction of pack_kernel's, so several times more warps hide the latency.
-template <typename T, int MAXJ>
+// Streaming form of pack_kernel for groups of at most 64 channels (LPG <= 8
+// chunks per group, so a group's chunks sit in the team's lanes at the same
+// chunk step): the same arithmetic in the same order, but no token chunk is
+// held across the whole entry.  Pass 1 streams the chunks for the gate (first
+// reads, kept in L1 by an evict-last hint); pass 2 reads each chunk again
+// (L1/L2, evict-first: its last use), forms the entry values, takes the group
+// maximum across the team and quantises it right away.  The small register
+// footprint keeps 40 warps per SM, which is what hides the two reads'
+// latency.  CTA (x, b) packs entries [32 x, 32 x + 32) of sequence b's
+// append, a team of 8 lanes per entry.
+//
+// Instruction count matters as much: the arithmetic runs on fp32 pairs
+// (f2_*), the group maximum propagates NaN so that one test per chunk replaces
+// a finiteness test per value (a warp that meets a non-finite value redoes
+// that chunk value by value), the scale m / 6 needs no division (div6_rn),
+// with E4M3 scales the reciprocal and its brackets come from a 128-entry table
+// (one per scale byte), and the group width LPG is a compile-time constant.
+template <typename T, int MAXJ, int LPG>
 __global__ void __launch_bounds__(kThreads, 5)
-pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
-    pdl_wait();
-    __shared__ __align__(16) uint8_t tail_smem[kTeams][kTailBytes];
-    const int lane = threadIdx.x & 31;
-    const int team = threadIdx.x >> 3, l = threadIdx.x & 7;
-    const long long e = (long long)blockIdx.x * kTeams + team;
-    const int half = a.n_new >> 1;
-    const bool in_range = e < (long long)a.batch * half;
-    int b = 0, i = 0, base = 0;
-    bool valid = false;
-    if (in_range) {
-        b = (int)(e / half);
-        i = (int)(e % half);
-        base = a.n_entries[b];
-        valid = base >= 0 && base + half <= a.capacity;
-        if (!valid && i == 0 && l == 0) set_status(a.status, KVC_DEV_CAPACITY);
-    }
+pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
+    extern __shared__ __align__(16) uint8_t dsm[];  // per-entry tails
+    __shared__ float tab_s[128], tab_rl[128], tab_rh[128];  // per E4M3 scale byte
+    const int tid = threadIdx.x, lane = tid & 31, team = tid >> 3, l = tid & 7;
+    const int b = blockIdx.y, half = a.n_new >> 1;
+    const int e0 = blockIdx.x * kTeams, ne = min(kTeams, half - e0);
+    const int i = e0 + team;  // this team's entry within the append
     const int D = sh.D, nchunk = D >> 3;
+    uint8_t* tail = dsm + team * tail_stride;
+    const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
+    if (ue4m3 && tid < 128) {
+        const float sv = e4m3_to_f32(tid);
+        const float r = __frcp_rn(sv);
+        tab_s[tid] = sv;
+        tab_rl[tid] = __fmul_rn(r, 1.0f - 0x1p-20f);
+        tab_rh[tid] = __fmul_rn(r, 1.0f + 0x1p-20f);
+    }
+    for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
+    __syncthreads();
+    pdl_wait();
+    const int base = a.n_entries[b];
+    if (!(base >= 0 && base + half <= a.capacity)) {  // the same for the whole CTA
+        if (blockIdx.x == 0 && tid == 0) set_status(a.status, KVC_DEV_CAPACITY);
+        return;
+    }
+    const bool valid = team < ne;
     const long long pos = (long long)base + i;
     const T* k0p = static_cast<const T*>(a.tokens) + ((long long)b * a.n_new + 2 * i) * D;
     const T* k1p = k0p + D;
+    const int jn = valid ? (nchunk - l + 7) / 8 : 0;  // chunks of this lane
 
     // pass 1: gate logit difference, fixed order (lane l: chunks l, l+8, ...)
     float acc = 0.f;
 #pragma unroll 3
     for (int j = 0; j < MAXJ; ++j) {
         const int c = l + 8 * j;
-        if (valid && c < nchunk) {
+        if (j < jn) {
             Chunk<T> x0, x1;
-            x0.load_cached(k0p + 8 * c);
-            x1.load_cached(k1p + 8 * c);
+            x0.load_keep(k0p + 8 * c);
+            x1.load_keep(k1p + 8 * c);
             float g[8];
             load8_gate(a.gate + 8 * c, g);
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
-                acc = __fmaf_rn(g[t], __fsub_rn(x0.get(t), x1.get(t)), acc);
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t d = f2_sub(x0.pair(k), x1.pair(k));
+                acc = __fmaf_rn(g[2 * k], f2_lo(d), acc);
+                acc = __fmaf_rn(g[2 * k + 1], f2_hi(d), acc);
+            }
         }
     }
     acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
@@ -338,51 +489,74 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
     const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-acc)));
     const float w1 = __fsub_rn(1.0f, w0);
-
+    const uint64_t W0 = f2_make(w0, w0), W1 = f2_make(w1, w1);
     uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
-    uint8_t* tail = tail_smem[team];
-    const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
-    for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
-    __syncwarp();
 
     // pass 2: entry values, group maxima (xor over the group's lanes), codes
     bool bad = false;
-    const int lpg = sh.lpg;
 #pragma unroll 2
     for (int j = 0; j < MAXJ; ++j) {
         const int c = l + 8 * j;
-        const bool active = valid && c < nchunk;
+        const bool active = j < jn;
         Chunk<T> x0, x1;
         if (active) {
-            x0.load_cached(k0p + 8 * c);
-            x1.load_cached(k1p + 8 * c);
+            x0.load_last(k0p + 8 * c);
+            x1.load_last(k1p + 8 * c);
         } else {
             x0.zero();
             x1.zero();
         }
-        float x[8];
-        float m = 0.f;
+        uint64_t v[4];  // v = w0 k0 + w1 k1, rounded as fmaf(w0, k0, w1 * k1)
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            float v = __fmaf_rn(w0, x0.get(t), __fmul_rn(w1, x1.get(t)));
-            if (!isfinite(v)) {
-                if (active) bad = true;
-                v = 0.f;
+        for (int k = 0; k < 4; ++k) v[k] = f2_fma(W0, x0.pair(k), f2_mul(W1, x1.pair(k)));
+        // the chunk's largest magnitude (a tree of pairwise maxima), then the group's
+        float m = absmax_nan(absmax_nan(absmax_nan(f2_lo(v[0]), f2_hi(v[0])),
+                                        absmax_nan(f2_lo(v[1]), f2_hi(v[1]))),
+                             absmax_nan(absmax_nan(f2_lo(v[2]), f2_hi(v[2])),
+                                        absmax_nan(f2_lo(v[3]), f2_hi(v[3]))));
+#pragma unroll
+        for (int o = 1; o < LPG; o <<= 1) m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+        m = fabsf(m);
+        if (__any_sync(0xffffffffu, !(m <= 3.0e38f))) {
+            // a NaN or inf somewhere in the warp: value by value, non-finite
+            // values coded as 0 (and reported)
+            m = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float lo = f2_lo(v[k]), hi = f2_hi(v[k]);
+                if (!isfinite(lo)) {
+                    if (active) bad = true;
+                    lo = 0.f;
+                }
+                if (!isfinite(hi)) {
+                    if (active) bad = true;
+                    hi = 0.f;
+                }
+                v[k] = f2_make(lo, hi);
+                m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
             }
-            x[t] = v;
-            m = fmaxf(m, fabsf(v));
+#pragma unroll
+            for (int o = 1; o < LPG; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         }
-        for (int o = 1; o < lpg; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (!active) continue;
-        float sc = __fdiv_rn(m, 6.0f);
-        uint32_t sbyte = 0;
+        const float sc = div6_rn(m);
+        uint32_t code, sbyte = 0;
         if (ue4m3) {
             sbyte = e4m3_from_f32(sc);
-            sc = e4m3_to_f32(sbyte);
+            const float sv = tab_s[sbyte];
+            code = sv > 0.f ? e2m1x8_quotient_f2(v, sv, tab_rl[sbyte], tab_rh[sbyte]) : 0u;
+        } else {
+            float x[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                x[2 * k] = f2_lo(v[k]);
+                x[2 * k + 1] = f2_hi(v[k]);
+            }
+            code = sc > 0.f ? e2m1x8_quotient(x, sc) : 0u;
         }
-        *reinterpret_cast<uint32_t*>(rec + 4 * c) = sc > 0.f ? e2m1x8_quotient(x, sc) : 0u;
-        if (c % lpg == 0) {
-            const int gi = c / lpg;
+        *reinterpret_cast<uint32_t*>(rec + 4 * c) = code;
+        if ((c & (LPG - 1)) == 0) {
+            const int gi = c / LPG;
             if (ue4m3)
                 tail[gi] = (uint8_t)sbyte;
             else
@@ -746,6 +920,24 @@ cudaError_t launch_group4(unsigned grid, size_t smem, cudaStream_t s, const Pack
                       di);
 }
 
+template <typename T, int MAXJ, int LPG>
+cudaError_t launch_stream(dim3 grid, cudaStream_t s, const PackArgs& a, const Shape& sh,
+                          int ue4m3, int di) {
+    const int tail_stride = ((sh.rb - sh.code_bytes) + 15) / 16 * 16;
+    return launch_pdl(pack_stream_kernel<T, MAXJ, LPG>, grid, kThreads,
+                      (size_t)kTeams * tail_stride, s, a, sh, ue4m3, di, tail_stride);
+}
+template <typename T, int MAXJ>
+cudaError_t launch_stream_j(dim3 grid, cudaStream_t s, const PackArgs& a, const Shape& sh,
+                            int ue4m3, int di) {
+    switch (sh.lpg) {
+        case 1: return launch_stream<T, MAXJ, 1>(grid, s, a, sh, ue4m3, di);
+        case 2: return launch_stream<T, MAXJ, 2>(grid, s, a, sh, ue4m3, di);
+        case 4: return launch_stream<T, MAXJ, 4>(grid, s, a, sh, ue4m3, di);
+        default: return launch_stream<T, MAXJ, 8>(grid, s, a, sh, ue4m3, di);
+    }
+}
+
 // 4:1 appends: a warp per entry at every size
 template <typename T>
 cudaError_t launch_pack4_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
@@ -793,14 +985,16 @@ cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
     const int maxj = (sh.D / 8 + 7) / 8;
     trace_before("pack", s);
     if (sh.lpg <= 8) {  // groups within one chunk step: the streaming kernel
+        const int half = a.n_new / 2;
+        const dim3 g2((unsigned)((half + kTeams - 1) / kTeams), (unsigned)a.batch);
         if (maxj <= 2)
-            err = launch_pdl(pack_stream_kernel<T, 2>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+            err = launch_stream_j<T, 2>(g2, s, a, sh, ue4m3, di);
         else if (maxj <= 4)
-            err = launch_pdl(pack_stream_kernel<T, 4>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+            err = launch_stream_j<T, 4>(g2, s, a, sh, ue4m3, di);
         else if (maxj <= 9)
-            err = launch_pdl(pack_stream_kernel<T, 9>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+            err = launch_stream_j<T, 9>(g2, s, a, sh, ue4m3, di);
         else
-            err = launch_pdl(pack_stream_kernel<T, 16>, grid, kThreads, 0, s, a, sh, ue4m3, di);
+            err = launch_stream_j<T, 16>(g2, s, a, sh, ue4m3, di);
         trace_after(s);
         return err;
     }

@@ -71,6 +71,48 @@ def test_pack_capacity_and_nonfinite_flags(kvc):
     assert cache.n_entries.item() == 32 and torch.equal(cache.records, before)
 
 
+@pytest.mark.parametrize("name", ["batch32x128k", "mla32k"])
+def test_pack_stream_nonfinite(kvc, name):
+    """Appends of more than 4096 entries take the streaming kernel, whose
+    group maxima propagate NaN and whose warps redo a chunk value by value
+    when they meet a non-finite value: a NaN (the whole entry's gate goes
+    NaN), +inf and -inf in different sequences and groups, against the oracle
+    byte for byte."""
+    w = synth.WORKLOADS[name].scaled(batch=3, context=2 * 3000)
+    inp = synth.make_inputs(w)
+    tok = inp["tokens"].clone()
+    tok[1, 100, 5] = float("nan")
+    tok[2, 2001, w.dim - 6] = float("inf")
+    tok[0, 4000, 300] = float("-inf")
+    rec, ic, n, ost = oracle_pack(w, tok, inp["gate"], inp["idx_k"])
+    cache, st = _gpu_pack(kvc, w, tok.cuda(), inp["gate"].cuda(), inp["idx_k"].cuda())
+    assert ost == oracle.ST_NONFINITE and st == kvc.DEV_NONFINITE
+    g = cache.records.cpu().numpy()
+    diff = np.argwhere(g != rec)
+    assert diff.size == 0, f"{len(diff)} bytes differ, first {diff[:5].tolist()}"
+    assert np.array_equal(cache.idx_k.cpu().numpy(), ic)
+
+
+def test_pack_rejects_tokens_not_16_byte_aligned(kvc):
+    """Token rows arrive by 16-byte loads and bulk copies: a start 2 bytes
+    past a 16-byte boundary is refused before any work (KVC_ERR_INVALID),
+    and the cache is untouched."""
+    w = synth.WORKLOADS["batch32x128k"].scaled(batch=2, context=2 * 2600)
+    inp = synth.make_inputs(w)
+    tok = inp["tokens"]
+    flat = torch.empty(tok.numel() + 8, dtype=tok.dtype, device="cuda")
+    shifted = flat[1:1 + tok.numel()].view(tok.shape)
+    shifted.copy_(tok.cuda())
+    assert shifted.data_ptr() % 16 == 2 and shifted.is_contiguous()
+    cfg = kvc.config_for(w)
+    cache = kvc.Cache(cfg, 2, 2600)
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.pack(cfg, shifted, inp["gate"].cuda(), inp["idx_k"].cuda(), cache)
+    assert e.value.status == 1  # KVC_ERR_INVALID
+    torch.cuda.synchronize()
+    assert cache.n_entries.cpu().tolist() == [0, 0]
+
+
 def test_pack_host_validation(kvc):
     w = synth.WORKLOADS["tiny"]
     cfg = kvc.config_for(w)
