@@ -11,15 +11,30 @@
 // integer for every UE4M3 value), summed over the groups -- the score times
 // 2^10, in 64 bits (|.| < 2^39 for di <= 256).  So the selection stays exact.
 //
-// A first, direct design:
-//  1. idx_fp4_scan: a thread per entry reads its row (byte loads: a row need
-//     not be 4-byte aligned) and the sequence's query, and writes the score.
-//  2. idx_fp4_select: a CTA of 1024 threads per sequence finds the K-th best
-//     score by a radix selection over the 40-bit value score + 2^39 (4 passes
-//     of 10 bits: a 1024-bin histogram of the entries that match the digits
-//     found so far, then a block prefix sum over the bins from the top), and
-//     one pass in index order takes the entries above that value and, lowest
-//     index first, as many equal to it as the K still need.
+// 128- and 256-channel keys (the fast path, the pages' 72-byte row and its
+// double):
+//  1. idx_fp4_scan_fast: CTA (x, b) scores 4096 rows of sequence b; a warp
+//     stages blocks of 32 rows with coalesced 8-byte loads (the next block's
+//     in flight) and each lane scores one row: byte permutes turn four codes
+//     into four signed twice-values for one dp4a with the query; the group sum
+//     times the scale's table value accumulates in 64 bits.  The row's 64-bit
+//     key (score, then index) is stored and its bin -- 16 per octave of |S| --
+//     counted; the sequence's last CTA derives the threshold bin.
+//  2. idx_fp4_select_tiles: per tile of 8192 keys, those of bins >= t go to
+//     candidate slots in index order.
+//  3. idx_fp4_select_finish: per sequence, the candidates in index order, the
+//     cut-off key among those of the threshold bin (ranked by counting, or
+//     sorted), and the winners' rows in index order; an exact radix selection
+//     over all keys when the candidates overflow.
+// Other widths (16, 32, 64 channels) take a direct design: a thread per entry
+// (byte loads) writes the score, then a CTA of 1024 threads per sequence finds
+// the K-th best score by a radix selection over the 40-bit value score + 2^39
+// (4 passes of 10 bits: a 1024-bin histogram of the entries that match the
+// digits found so far, then a block prefix sum over the bins from the top),
+// and one pass in index order takes the entries above that value and, lowest
+// index first, as many equal to it as the K still need.
+#include <algorithm>
+
 #include "topk_common.cuh"
 
 namespace kvc {
@@ -42,7 +57,7 @@ __device__ __forceinline__ long long ue4m3_times_512(int byte) {
 }
 
 __global__ void __launch_bounds__(256)
-idx_fp4_scan_kernel(const int8_t* __restrict__ q, const uint8_t* __restrict__ rows,
+idx_fp4_scan_direct_kernel(const int8_t* __restrict__ q, const uint8_t* __restrict__ rows,
                     const int32_t* __restrict__ n_entries, int batch, int capacity, int di,
                     int rb, long long* __restrict__ scores, uint32_t* status) {
     pdl_wait();
@@ -72,7 +87,7 @@ idx_fp4_scan_kernel(const int8_t* __restrict__ q, const uint8_t* __restrict__ ro
 }
 
 __global__ void __launch_bounds__(kSelThreads)
-idx_fp4_select_kernel(const long long* __restrict__ scores, const int32_t* __restrict__ n_entries,
+idx_fp4_select_direct_kernel(const long long* __restrict__ scores, const int32_t* __restrict__ n_entries,
                       int capacity, int K, int32_t* __restrict__ topk) {
     __shared__ int hist[kSelThreads];
     __shared__ int sh_warp[kSelThreads / 32];
@@ -140,6 +155,383 @@ idx_fp4_select_kernel(const long long* __restrict__ scores, const int32_t* __res
     for (int i = taken + tid; i < K; i += kSelThreads) out[i] = -1;  // only if inconsistent
 }
 
+// ======================================================================
+// Fast path (128- and 256-channel keys, rows of 72 / 144 bytes).
+//
+// Keys: the exact score S (the score times 2^10, |S| < 2^39) and the row j
+// pack into one 64-bit key, (S + 2^39) << 24 | (2^24 - 1 - j), so a larger key
+// is a better entry (score descending, index ascending) and no two are equal.
+// Bins: an 11-bit function of S that never decreases as S grows -- sign,
+// binary exponent of |S| and 4 bits below its leading one (16 bins per
+// octave) -- so the K best keys lie in the bins at or above the threshold bin
+// t of a 2048-bin histogram, and bin t holds a few hundred of them at most for
+// any spread-out score distribution.
+constexpr int kScanTile = 4096;        // rows per scan CTA: 8 warps x 16 blocks of 32
+constexpr int kFinishCap = kSelTile;  // candidates the finish stages in shared memory
+constexpr int kTileCands = kFp4TileCands;  // candidate slots per select tile
+constexpr long long kKeyBias = 1LL << 39;
+
+__device__ __forceinline__ int fp4_bin(long long S) {
+    // |S| truncated to fp32 (never rounds up, so the bin never decreases as
+    // |S| grows): its exponent and the 4 mantissa bits below the leading one;
+    // 0 for S = 0, 16 .. 639 otherwise (|S| < 2^39)
+    const uint32_t fb = __float_as_uint(__ll2float_rz(S < 0 ? -S : S));
+    const int v = max(0, (int)(fb >> 19) - (127 << 4) + 16);
+    return S < 0 ? 1023 - v : 1024 + v;
+}
+__device__ __forceinline__ unsigned long long fp4_key(long long S, int j) {
+    return ((unsigned long long)(S + kKeyBias) << 24) | (unsigned long long)(0xFFFFFFu - (uint32_t)j);
+}
+__device__ __forceinline__ long long key_score(unsigned long long k) {
+    return (long long)(k >> 24) - kKeyBias;
+}
+__device__ __forceinline__ int key_row(unsigned long long k) {
+    return (int)(0xFFFFFFu - (uint32_t)(k & 0xFFFFFFull));
+}
+
+// Four E2M1 codes (channel i in nibble i of the low 16 bits of x) as four
+// signed int8 twice-values (byte i) by byte permutes: the magnitude index
+// picks from a table of twice-magnitudes {0,1,2,3,4,6,8,12} and from its
+// negation, then each byte comes from one or the other by its sign bit.
+// (prmt.b32 in its default mode: bit 3 of a selector nibble would replicate
+// the byte's sign, so every selector here has it clear.)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ uint32_t e2m1x4_twice(uint32_t x) {
+    const uint32_t sel = x & 0x7777u;
+    const uint32_t pos = prmt(0x03020100u, 0x0C080604u, sel);
+    const uint32_t neg = prmt(0xFDFEFF00u, 0xF4F8FAFCu, sel);
+    return prmt(pos, neg, 0x3210u | ((x >> 1) & 0x4444u));
+}
+
+// idx_fp4_scan_fast: CTA (x, b) scores rows [4096 x, 4096 x + 4096) of
+// sequence b.  A warp takes blocks of 32 rows: coalesced 8-byte loads (the
+// next block's in flight during the arithmetic) into its shared-memory stage,
+// then lane l scores row l from there -- per group of 16 channels four dp4a of
+// decoded twice-values with the query (held in registers), times 2^9 times
+// the group's UE4M3 scale, summed in 64 bits.  It stores the row's key and
+// counts its bin; the sequence's last CTA (a fenced counter; nobody waits)
+// derives the threshold bin t and the count above it.
+template <int DI>
+__global__ void __launch_bounds__(kThreads, DI == 128 ? 5 : 2)
+idx_fp4_scan_fast(TopkArgs a, unsigned long long* __restrict__ keys) {
+    constexpr int RB = DI / 2 + DI / 16;  // row bytes
+    constexpr int RW = RB / 8;            // 8-byte words per row
+    constexpr int NG = DI / 16;           // channel groups (one code word each)
+    __shared__ __align__(16) unsigned long long stage[kThreads / 32][32 * RW];
+    __shared__ __align__(16) uint32_t qs[DI / 4];
+    __shared__ int s512[256];  // 2^9 times the value of each UE4M3 byte
+    __shared__ int hist[kBins];
+    __shared__ int sh_warp[kThreads / 32];
+    __shared__ int s_last, s_t, s_above;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.y, cap = a.capacity;
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
+    s512[tid] = (int)ue4m3_times_512(tid);  // kThreads = 256 bytes
+    pdl_wait();
+    const int n = a.n_entries[b];
+    if (n < 0 || n > cap) {
+        if (blockIdx.x == 0 && tid == 0) set_status(a.status, KVC_DEV_BAD_LENGTH);
+        return;
+    }
+    const int r0 = blockIdx.x * kScanTile;
+    if (r0 >= n) return;  // the sequence's CTAs are the first ceil(n / 4096)
+    const int rend = min(r0 + kScanTile, n);
+    if (tid < DI / 4) qs[tid] = __ldg(reinterpret_cast<const uint32_t*>(a.idx_q + (size_t)b * DI) + tid);
+    __syncthreads();  // histogram zeroed, tables and query staged
+    const unsigned long long* src =
+        reinterpret_cast<const unsigned long long*>(a.idx_k + (size_t)b * a.idx_capacity * RB);
+    unsigned long long pre[RW];
+    auto fetch = [&](int rb0) {  // rows [rb0, rb0 + 32): word k * 32 + lane of the block
+        if (rb0 + 32 <= rend) {
+#pragma unroll
+            for (int k = 0; k < RW; ++k) pre[k] = __ldcs(src + (size_t)rb0 * RW + k * 32 + lane);
+        } else {
+#pragma unroll
+            for (int k = 0; k < RW; ++k) {
+                const int w = k * 32 + lane;
+                pre[k] = rb0 + w / RW < rend ? __ldcs(src + (size_t)rb0 * RW + w) : 0ull;
+            }
+        }
+    };
+    unsigned long long* st = stage[warp];
+    int blk = r0 + 32 * warp;
+    if (blk < rend) fetch(blk);
+    for (; blk < rend; blk += 32 * (kThreads / 32)) {
+#pragma unroll
+        for (int k = 0; k < RW; ++k) st[k * 32 + lane] = pre[k];
+        __syncwarp();
+        if (blk + 256 < rend) fetch(blk + 256);
+        const int j = blk + lane;
+        if (j < rend) {
+            const uint2* row = reinterpret_cast<const uint2*>(st + lane * RW);
+            long long S = 0;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                const uint2 cw = row[g];
+                const uint4 qg = reinterpret_cast<const uint4*>(qs)[g];  // (broadcast)
+                int part = __dp4a((int)e2m1x4_twice(cw.x), (int)qg.x, 0);
+                part = __dp4a((int)e2m1x4_twice(cw.x >> 16), (int)qg.y, part);
+                part = __dp4a((int)e2m1x4_twice(cw.y), (int)qg.z, part);
+                part = __dp4a((int)e2m1x4_twice(cw.y >> 16), (int)qg.w, part);
+                const uint2 sw = row[NG + (g >> 3)];
+                const uint32_t sword = (g & 4) ? sw.y : sw.x;
+                S += (long long)part * s512[(sword >> (8 * (g & 3))) & 0xFFu];
+            }
+            keys[(size_t)b * cap + j] = fp4_key(S, j);
+            atomicAdd(&hist[fp4_bin(S)], 1);
+        }
+        __syncwarp();  // the stage is rewritten by the next block
+    }
+    __syncthreads();
+    if (n > a.topk) {
+        int32_t* gh = a.counters + (size_t)b * kBins;
+        for (int i = tid; i < kBins; i += kThreads)
+            if (hist[i]) atomicAdd(&gh[i], hist[i]);
+        __threadfence();
+        __syncthreads();
+        const int ntiles = (n + kScanTile - 1) / kScanTile;
+        if (tid == 0)
+            s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) == ntiles - 1;
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int i = tid; i < kBins; i += kThreads) {
+                hist[i] = __ldcg(gh + i);
+                gh[i] = 0;  // left zeroed for the next call
+            }
+            if (tid == 0) {
+                a.counters[(size_t)a.batch * kBins + b] = 0;
+                s_t = s_above = 0;
+            }
+            __syncthreads();
+            find_threshold(hist, a.topk, &s_t, &s_above, sh_warp);
+            if (tid == 0) {
+                a.thr[2 * b] = s_t;
+                a.thr[2 * b + 1] = s_above;
+            }
+        }
+    }
+    pdl_trigger();
+}
+
+// Descending bitonic sort of p (a power of two) keys in shared memory; every
+// thread of the block calls it.
+__device__ __forceinline__ void bitonic_desc(unsigned long long* k, int p) {
+    for (int size = 2; size <= p; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < p; i += blockDim.x) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const bool desc = (i & size) == 0;
+                    const unsigned long long x = k[i], y = k[j];
+                    if ((x < y) == desc) {
+                        k[i] = y;
+                        k[j] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// idx_fp4_select_tiles: CTA (x, b) takes tile x (8192 keys) of sequence b:
+// the keys of bins >= t go, in index order, to the tile's candidate slots (at
+// most kTileCands; a warp per 1024 keys, ballot prefix sums), and their count
+// (-1: too many) to tile_count.
+__global__ void __launch_bounds__(kThreads)
+idx_fp4_select_tiles(TopkArgs a, const unsigned long long* __restrict__ keys) {
+    extern __shared__ __align__(16) unsigned long long sk[];  // [kSelTile]
+    __shared__ int sh_warp[kThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.y, tile = blockIdx.x, cap = a.capacity, K = a.topk;
+    pdl_wait();
+    const int n = a.n_entries[b];
+    if (n < 0 || n > cap || n <= K) return;  // (the finish writes these outputs)
+    const int ntiles = (n + kSelTile - 1) / kSelTile;
+    if (tile >= ntiles) return;
+    const int t = a.thr[2 * b];
+    const unsigned long long* tk = keys + (size_t)b * cap + (size_t)tile * kSelTile;
+    const int tiles = sel_tiles(cap);
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(a.scores) +
+                               ((size_t)b * tiles + tile) * kTileCands;
+    const int tn = min(kSelTile, n - tile * kSelTile);
+    uint32_t take = 0;
+    for (int r0 = 0; r0 < 32; r0 += 16) {  // 16 loads in flight per lane
+        unsigned long long kv[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int i = warp * 1024 + (r0 + u) * 32 + lane;
+            kv[u] = i < tn ? __ldcg(tk + i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int i = warp * 1024 + (r0 + u) * 32 + lane;
+            if (i < tn) {
+                sk[i] = kv[u];
+                if (fp4_bin(key_score(kv[u])) >= t) take |= 1u << (r0 + u);
+            }
+        }
+    }
+    int cnt = 0;
+    for (int r = 0; r < 32; ++r) cnt += __popc(__ballot_sync(0xffffffffu, (take >> r) & 1u));
+    if (lane == 0) sh_warp[warp] = cnt;  // the warps' counts: offsets and total
+    __syncthreads();
+    int wbase = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        const int c = sh_warp[w];
+        wbase += w < warp ? c : 0;
+        total += c;
+    }
+    if (total <= kTileCands) {
+        const uint32_t lt = (1u << lane) - 1u;
+        int pos = wbase;
+        for (int r = 0; r < 32; ++r) {
+            const uint32_t bal = __ballot_sync(0xffffffffu, (take >> r) & 1u);
+            if ((take >> r) & 1u) cand[pos + __popc(bal & lt)] = sk[warp * 1024 + r * 32 + lane];
+            pos += __popc(bal);
+        }
+    }
+    if (tid == 0) a.tile_count[(size_t)b * tiles + tile] = total <= kTileCands ? total : -1;
+    pdl_trigger();
+}
+
+// idx_fp4_select_finish: CTA b gathers sequence b's candidates, tile by tile
+// (so in index order), into shared memory, finds the cut-off key k* -- the
+// (K - above)-th best of the candidates in bin t, by counting larger keys for
+// up to 1024 of them, else by a bitonic sort -- and writes the rows of the
+// keys >= k* in index order.  A tile with too many candidates, more than
+// kFinishCap in all or more than kMaxTies in bin t: the exact radix selection
+// over all the sequence's keys instead.
+__global__ void __launch_bounds__(kThreads)
+idx_fp4_select_finish(TopkArgs a, const unsigned long long* __restrict__ keys) {
+    extern __shared__ __align__(16) unsigned long long sk[];  // [kSelTile] | ties [kMaxTies]
+    unsigned long long* tie = sk + kSelTile;
+    __shared__ int sh_warp[kThreads / 32];
+    __shared__ int hist[256];
+    __shared__ int s_digit, s_above;
+    const int tid = threadIdx.x;
+    const int b = blockIdx.x, cap = a.capacity, K = a.topk;
+    pdl_wait();
+    const int n = a.n_entries[b];
+    int32_t* out = a.topk_idx + (size_t)b * K;
+    if (n < 0 || n > cap || n <= K) {  // a bad length: -1s; at most K entries: all of them
+        for (int i = tid; i < K; i += kThreads) out[i] = (n >= 0 && n <= cap && i < n) ? i : -1;
+        return;
+    }
+    const int ntiles = (n + kSelTile - 1) / kSelTile, tiles = sel_tiles(cap);
+    const int t = a.thr[2 * b], above = a.thr[2 * b + 1];
+    const unsigned long long* seq = keys + (size_t)b * cap;
+    const int32_t* tcnt = a.tile_count + (size_t)b * tiles;
+    int* cnt_s = reinterpret_cast<int*>(tie);  // tile counts, then offsets (ntiles <= 1024)
+    for (int i = tid; i < ntiles; i += kThreads) cnt_s[i] = __ldcg(tcnt + i);
+    __syncthreads();
+    int tot = 0;
+    bool exact = false;
+    for (int i = 0; i < ntiles; ++i) {
+        const int c = cnt_s[i];
+        exact |= c < 0;
+        tot += c;
+    }
+    unsigned long long kstar = 0;
+    exact |= tot > kFinishCap;
+    if (!exact) {
+        int off = 0;
+        const unsigned long long* sc =
+            reinterpret_cast<const unsigned long long*>(a.scores) + (size_t)b * tiles * kTileCands;
+        for (int i = 0; i < ntiles; ++i) {  // (independent loads: no global value steers them)
+            const int c = cnt_s[i];
+            for (int k = tid; k < c; k += kThreads) sk[off + k] = __ldcg(sc + (size_t)i * kTileCands + k);
+            off += c;
+        }
+        __syncthreads();  // (also: every thread has read the counts before tie[] is reused)
+        int m = 0;  // candidates of bin t, in index order, into tie[]
+        for (int base = 0; base < tot; base += kThreads) {
+            const int i = base + tid;
+            const int f = (i < tot && fp4_bin(key_score(sk[i])) == t) ? 1 : 0;
+            int ex;
+            const int ft = block_excl_scan(f, &ex, sh_warp);
+            if (f && m + ex < kMaxTies) tie[m + ex] = sk[i];
+            m += ft;
+        }
+        const int r = K - above;  // entries of bin t taken
+        exact = m > kMaxTies || r < 1 || r > m;
+        if (!exact && m <= 1024) {
+            // the key with exactly r - 1 larger ones among the m (distinct) keys
+            __syncthreads();
+            if (tid == 0) s_digit = 0;
+            __syncthreads();
+            for (int i = tid; i < m; i += kThreads) {
+                const unsigned long long x = tie[i];
+                int larger = 0;
+                for (int k = 0; k < m; ++k) larger += tie[k] > x;
+                if (larger == r - 1) {
+                    tie[kMaxTies - 1] = x;  // (m <= 1024: the slot is free)
+                    s_digit = 1;
+                }
+            }
+            __syncthreads();
+            kstar = tie[kMaxTies - 1];
+        } else if (!exact) {
+            int P = 1;
+            while (P < m) P <<= 1;
+            for (int i = m + tid; i < P; i += kThreads) tie[i] = 0ull;  // below every key
+            __syncthreads();
+            bitonic_desc(tie, P);
+            kstar = tie[r - 1];
+        }
+    }
+    // ---- exact path: the K-th largest of the n distinct keys by a radix
+    // selection over the 64 key bits, 8 at a time (a 256-bin histogram of the
+    // keys that match the digits found so far, then a prefix sum over the bins
+    // from the top)
+    if (exact) {
+        unsigned long long prefix = 0, mask = 0;
+        int remaining = K;
+        for (int p = 7; p >= 0; --p) {
+            const int shift = 8 * p;
+            hist[tid] = 0;
+            __syncthreads();
+            for (int j = tid; j < n; j += kThreads) {
+                const unsigned long long k = __ldcg(seq + j);
+                if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255], 1);
+            }
+            __syncthreads();
+            const int cnt = hist[255 - tid];  // thread t owns bin 255 - t: higher bins first
+            int excl;
+            block_excl_scan(cnt, &excl, sh_warp);
+            if (excl < remaining && remaining <= excl + cnt) {
+                s_digit = 255 - tid;
+                s_above = excl;
+            }
+            __syncthreads();
+            remaining -= s_above;
+            prefix |= (unsigned long long)s_digit << shift;
+            mask |= 255ull << shift;
+            __syncthreads();  // every thread has read the digit before the next pass
+        }
+        kstar = prefix;
+    }
+    // the winners, keys >= k*, in index order (a key's row is its index)
+    const unsigned long long* src = exact ? seq : sk;
+    const int len = exact ? n : tot;
+    int taken = 0;
+    for (int base = 0; base < len; base += kThreads) {
+        const int i = base + tid;
+        const unsigned long long k = i < len ? src[i] : 0ull;
+        const int w = (i < len && k >= kstar) ? 1 : 0;
+        int ex;
+        const int wt = block_excl_scan(w, &ex, sh_warp);
+        if (w && taken + ex < K) out[taken + ex] = key_row(k);
+        taken += wt;
+    }
+    for (int i = taken + tid; i < K; i += kThreads) out[i] = -1;
+}
 }  // namespace
 
 cudaError_t launch_index_topk_fp4(const TopkArgs& a, int idx_rb, long long* scores64,
@@ -147,16 +539,44 @@ cudaError_t launch_index_topk_fp4(const TopkArgs& a, int idx_rb, long long* scor
     if (a.batch == 0) return cudaSuccess;
     const long long rows = (long long)a.batch * a.capacity;
     cudaError_t err;
+    if (a.di == 128 || a.di == 256) {  // the fast path: keys and the threshold bins
+        unsigned long long* keys = reinterpret_cast<unsigned long long*>(scores64);
+        if (rows > 0) {
+            const dim3 g((unsigned)((a.capacity + kScanTile - 1) / kScanTile), (unsigned)a.batch);
+            trace_before("index_scan_fp4", s);
+            err = a.di == 128 ? launch_pdl(idx_fp4_scan_fast<128>, g, kThreads, 0, s, a, keys)
+                              : launch_pdl(idx_fp4_scan_fast<256>, g, kThreads, 0, s, a, keys);
+            trace_after(s);
+            if (err != cudaSuccess) return err;
+        }
+        const size_t smem_t = (size_t)kSelTile * sizeof(unsigned long long);
+        const size_t smem_f = (size_t)(kSelTile + kMaxTies) * sizeof(unsigned long long);
+        err = cudaFuncSetAttribute(idx_fp4_select_tiles,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
+        if (err != cudaSuccess) return err;
+        err = cudaFuncSetAttribute(idx_fp4_select_finish,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_f);
+        if (err != cudaSuccess) return err;
+        const dim3 g((unsigned)std::max(1, sel_tiles(a.capacity)), (unsigned)a.batch);
+        trace_before("topk_select_fp4", s);
+        err = launch_pdl(idx_fp4_select_tiles, g, kThreads, smem_t, s, a,
+                         static_cast<const unsigned long long*>(keys));
+        if (err == cudaSuccess)
+            err = launch_pdl(idx_fp4_select_finish, (unsigned)a.batch, kThreads, smem_f, s, a,
+                             static_cast<const unsigned long long*>(keys));
+        trace_after(s);
+        return err;
+    }
     if (rows > 0) {
         trace_before("index_scan_fp4", s);
-        err = launch_pdl(idx_fp4_scan_kernel, (unsigned)((rows + 255) / 256), 256, 0, s, a.idx_q,
-                         reinterpret_cast<const uint8_t*>(a.idx_k), a.n_entries, a.batch,
-                         a.capacity, a.di, idx_rb, scores64, a.status);
+        err = launch_pdl(idx_fp4_scan_direct_kernel, (unsigned)((rows + 255) / 256), 256, 0, s,
+                         a.idx_q, reinterpret_cast<const uint8_t*>(a.idx_k), a.n_entries,
+                         a.batch, a.capacity, a.di, idx_rb, scores64, a.status);
         trace_after(s);
         if (err != cudaSuccess) return err;
     }
     trace_before("topk_select_fp4", s);
-    err = launch_pdl(idx_fp4_select_kernel, (unsigned)a.batch, kSelThreads, 0, s,
+    err = launch_pdl(idx_fp4_select_direct_kernel, (unsigned)a.batch, kSelThreads, 0, s,
                      static_cast<const long long*>(scores64), a.n_entries, a.capacity, a.topk,
                      a.topk_idx);
     trace_after(s);

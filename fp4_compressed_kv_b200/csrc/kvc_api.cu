@@ -139,8 +139,8 @@ WsLayout ws_layout(const kvc_config& c, const Shape& sh, int batch, int cap,
     WsLayout w = {};
     size_t off = 0;
     const size_t tiles = (size_t)batch * sel_tiles(cap);
-    w.scores = off;
-    off = up(off + (size_t)batch * cap * 4);
+    w.scores = off;  // int32 scores, or the FP4 keys' candidate slots (as many bytes per tile)
+    off = up(off + (c.idx_fmt == 1 ? tiles * kFp4TileCands * 8 : (size_t)batch * cap * 4));
     w.counters = off;  // histograms [B][kBins], finished scan CTAs [B], finished select CTAs [B]
     off = up(off + topk_counter_words(batch) * 4);
     w.thr = off;

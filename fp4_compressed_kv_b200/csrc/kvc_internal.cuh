@@ -20,6 +20,9 @@ constexpr int kMaxSelTiles = 1024;
 constexpr long long kMaxTopkCapacity = (long long)kSelTile * kMaxSelTiles;
 // Candidates of the threshold bin kept for the in-shared-memory finish.
 constexpr int kMaxTies = 4096;
+// FP4 indexer keys: candidate slots (64-bit keys) per select tile, in the
+// workspace's score region (sized [B][sel_tiles(cap)][kFp4TileCands] keys).
+constexpr int kFp4TileCands = kSelTile / 2;
 __host__ __device__ inline int sel_tiles(int capacity) { return (capacity + kSelTile - 1) / kSelTile; }
 // Per-call counters of the top-K: histograms [B][kBins], finished scan CTAs
 // [B] and finished select CTAs [B], adjacent so one memset clears them.

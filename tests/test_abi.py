@@ -167,16 +167,19 @@ def test_fp4_indexer_rows_and_rejections(lib):
                              C.c_void_p(16), C.c_void_p(256), 1 << 30, None, None) == 4
 
 
-def test_workspace_holds_fp4_scores(lib):
-    """FP4 indexer keys keep their 64-bit scores in the workspace's candidate
-    region: the workspace is the same for both key formats and holds at least
-    the int32 scores plus 8 bytes per entry, at any capacity."""
+def test_workspace_holds_fp4_keys(lib):
+    """FP4 indexer keys keep one 64-bit key (exact score and index) per entry
+    in the workspace's candidate region and their selection candidates (half
+    a tile of keys per tile of 8192 entries) in its score region: the
+    workspace is at least the int8 one and at least B (8 cap + 8 x 4096 x
+    ceil(cap / 8192)) bytes, at any capacity."""
     w = synth.WORKLOADS["mla32k"]
     c8, c4 = lib.config_for(w), lib.config_for(w.scaled(idx_fmt=1))
     for B, cap in ((1, 1), (3, 1000), (32, 65600), (2, 131073), (1, 500_000)):
         n8, n4 = lib.workspace_bytes(c8, B, cap), lib.workspace_bytes(c4, B, cap)
-        assert n8 == n4 > 0
-        assert n4 >= B * cap * (4 + 8)
+        tiles = -(-cap // 8192)
+        assert n4 >= n8 > 0
+        assert n4 >= B * (8 * cap + 8 * 4096 * tiles)
 
 
 def test_capacity_limit_on_the_host(lib):

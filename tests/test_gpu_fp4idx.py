@@ -109,3 +109,50 @@ def test_group_step_over_fp4_keys(kvc):
                                            f32(inp["windows"][l]), w.window)
         assert ost == 0
         assert_attn_close(out[l].cpu().numpy(), ref, f"fp4 keys layer {l}")
+
+
+def _random_rows(B, N, di, seed, scale_lo=0x20, scale_hi=0x48):
+    """FP4 indexer rows with uniform random codes (every code, -0 included)
+    and UE4M3 scales drawn from [scale_lo, scale_hi)."""
+    g = np.random.default_rng(seed)
+    rows = np.empty((B, N, di // 2 + di // 16), np.uint8)
+    rows[:, :, :di // 2] = g.integers(0, 256, (B, N, di // 2))
+    rows[:, :, di // 2:] = g.integers(scale_lo, scale_hi, (B, N, di // 16))
+    return rows
+
+
+@pytest.mark.parametrize("di,N,case", [
+    (128, 20000, "all_equal"),   # bin t overflows the candidate slots: exact radix path
+    (128, 65536, "random"),      # full-size sequences: 16 scan tiles, 8 select tiles
+    (256, 9000, "tie_block"),    # 5000 equal rows: ties at the cut, fast path
+    (128, 9000, "wide_scales"),  # scales over the whole UE4M3 range (subnormal to 448)
+    (64, 5000, "random"),        # 64-channel rows: the direct kernels
+])
+def test_fp4_scan_and_select_paths(kvc, di, N, case):
+    """The FP4 key scan (tiled, log-scale threshold bins) and selection (tile
+    candidates, last-CTA finish, exact radix fallback) against the oracle's
+    exact top-K, bit for bit, on ragged lengths."""
+    B = 3
+    w = synth.WORKLOADS["mla32k"].scaled(batch=B, context=2 * N, idx_fmt=1, idx_dim=di)
+    cfg = kvc.config_for(w)
+    rows = (_random_rows(B, N, di, 21, 0x00, 0x7F) if case == "wide_scales"
+            else _random_rows(B, N, di, 21))
+    if case == "all_equal":
+        rows[0] = rows[0, 5]
+    if case == "tie_block":
+        rows[1, 2000:7000] = rows[1, 3]
+    cache = kvc.Cache(cfg, B, N)
+    cache.idx_k.copy_(torch.from_numpy(rows))
+    n = np.array([N, N - 77, N // 2 + 3], np.int32)
+    cache.n_entries.copy_(torch.from_numpy(n))
+    q = torch.randint(-128, 128, (B, di), generator=torch.Generator().manual_seed(9),
+                      dtype=torch.int8)
+    ws = kvc.workspace(cfg, B, N)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for call in range(2):  # twice: the counters must be left at zero
+        tk = torch.full((B, w.topk), -7, dtype=torch.int32, device="cuda")
+        kvc.index_topk(cfg, q.cuda(), cache, tk, ws, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        otk = oracle.index_topk_fp4(oracle_cfg(w), q.numpy(), rows, n)
+        assert np.array_equal(tk.cpu().numpy(), otk), f"call {call}"
