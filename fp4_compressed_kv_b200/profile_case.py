@@ -1,6 +1,7 @@
 """Run one hot-path call a few times on synthetic inputs, for profilers.
 
-    python -m fp4_compressed_kv_b200.profile_case --kernel scan|scan_fp4|attn|pack|step \
+    python -m fp4_compressed_kv_b200.profile_case \
+        --kernel scan|scan_fp4|attn|pack|step|hier|batched \
         [--config NAME] [--batch B] [--entries N] [--iters 3]
 
 scan  kvc_index_topk over B sequences of N int8 indexer rows (the indexer
@@ -12,6 +13,10 @@ attn  kvc_sparse_decode_attn: B sequences, each with a cache of N packed
 pack  kvc_pack of the workload's pack case (pack_new raw tokens per sequence,
       or 4096 when the workload has none).
 step  one decode step of the workload (pack of one pair + layer group).
+hier  the same step with the hierarchical indexer (2048 blocks of 8 kept):
+      block maxima, pool-mode scan and selection.
+batched  kvc_index_topk_batched: every Full/Reindex layer's query of the
+      workload against one cache in one tensor-core pass.
 Sizes default to the workload's; pass --batch/--entries to shrink a case so a
 profiler capture stays small (keep the streamed bytes above the 126 MB L2).
 """
@@ -26,7 +31,8 @@ from fp4_compressed_kv_b200 import build, kvc, synth
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("--kernel", required=True, choices=["scan", "scan_fp4", "attn", "pack", "step"])
+    p.add_argument("--kernel", required=True,
+                   choices=["scan", "scan_fp4", "attn", "pack", "step", "hier", "batched"])
     p.add_argument("--config", default="batch32x128k")
     p.add_argument("--batch", type=int, default=0)
     p.add_argument("--entries", type=int, default=0)
@@ -45,10 +51,11 @@ def main():
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     if a.kernel == "scan_fp4":  # FP4 indexer keys: random codes, scales 2^-8 .. 2^1
         cfg = kvc.config_for(w.scaled(idx_fmt=1))
-    if a.kernel in ("scan", "scan_fp4", "step", "attn"):
+    hier_blocks = 2048 if a.kernel == "hier" else 0
+    if a.kernel in ("scan", "scan_fp4", "step", "attn", "hier", "batched"):
         cache = kvc.Cache(cfg, B, N + a.iters + 8, device=dev)
-        ws = kvc.workspace(cfg, B, cache.capacity, device=dev)
-    if a.kernel in ("scan", "step"):
+        ws = kvc.workspace(cfg, B, cache.capacity, device=dev, hier_blocks=hier_blocks)
+    if a.kernel in ("scan", "step", "hier", "batched"):
         cache.idx_k[:, :N] = torch.randint(-127, 128, (B, N, w.idx_dim), generator=g, device=dev,
                                            dtype=torch.int8)
         cache.n_entries.fill_(N)
@@ -87,7 +94,15 @@ def main():
         for _ in range(a.iters):
             pc.n_entries.zero_()
             kvc.pack(cfg, nt["tokens"], gate, nt["idx_k"], pc, status=st)
-    else:  # step
+    elif a.kernel == "batched":
+        heads = [i for i, m in enumerate(w.modes) if m != synth.REUSE]
+        q = torch.randint(-127, 128, (len(heads), B, w.idx_dim), generator=g, device=dev,
+                          dtype=torch.int8)
+        tk = torch.empty(len(heads), B, w.topk, dtype=torch.int32, device=dev)
+        wsb = kvc.workspace_batched(cfg, len(heads), B, cache.capacity, device=dev)
+        for _ in range(a.iters):
+            kvc.index_topk_batched(cfg, q, cache, tk, wsb, status=st)
+    else:  # step, hier
         inp = synth.make_inputs(w, dev, with_tokens=False)
         L = w.layers
         nt = synth.make_new_tokens(w, 2, dev)
@@ -97,7 +112,8 @@ def main():
         for _ in range(a.iters):
             kvc.pack(cfg, nt["tokens"], inp["gate"], nt["idx_k"], cache, status=st)
             kvc.layer_group_step(cfg, list(w.modes), inp["q"], inp["idx_q"], inp["windows"],
-                                 w.window, cache, out, tk, ws, status=st)
+                                 w.window, cache, out, tk, ws, status=st,
+                                 hier_blocks=hier_blocks)
     torch.cuda.synchronize()
     assert st.item() == 0, st.item()
     print(f"profile_case {a.kernel} {w.name} B={B} N={N} iters={a.iters} ok")

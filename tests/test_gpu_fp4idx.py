@@ -124,7 +124,7 @@ def _random_rows(B, N, di, seed, scale_lo=0x20, scale_hi=0x48):
 @pytest.mark.parametrize("di,N,case", [
     (128, 20000, "all_equal"),   # bin t overflows the candidate slots: exact radix path
     (128, 65536, "random"),      # full-size sequences: 16 scan tiles, 8 select tiles
-    (256, 9000, "tie_block"),    # 5000 equal rows: ties at the cut, fast path
+    (256, 9000, "tie_block"),    # 2000 copies of the best row: the cut sorts ~2000 ties
     (128, 9000, "wide_scales"),  # scales over the whole UE4M3 range (subnormal to 448)
     (64, 5000, "random"),        # 64-channel rows: the direct kernels
 ])
@@ -139,14 +139,15 @@ def test_fp4_scan_and_select_paths(kvc, di, N, case):
             else _random_rows(B, N, di, 21))
     if case == "all_equal":
         rows[0] = rows[0, 5]
-    if case == "tie_block":
-        rows[1, 2000:7000] = rows[1, 3]
-    cache = kvc.Cache(cfg, B, N)
-    cache.idx_k.copy_(torch.from_numpy(rows))
     n = np.array([N, N - 77, N // 2 + 3], np.int32)
-    cache.n_entries.copy_(torch.from_numpy(n))
     q = torch.randint(-128, 128, (B, di), generator=torch.Generator().manual_seed(9),
                       dtype=torch.int8)
+    if case == "tie_block":  # the threshold bin then holds all 2000 copies
+        _, sc = oracle.index_topk_fp4(oracle_cfg(w), q.numpy(), rows, n, want_scores=True)
+        rows[1, 2000:4000] = rows[1, int(np.argmax(sc[1, :n[1]]))]
+    cache = kvc.Cache(cfg, B, N)
+    cache.idx_k.copy_(torch.from_numpy(rows))
+    cache.n_entries.copy_(torch.from_numpy(n))
     ws = kvc.workspace(cfg, B, N)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     for call in range(2):  # twice: the counters must be left at zero
