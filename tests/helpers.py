@@ -49,3 +49,31 @@ def assert_attn_close(out_gpu: np.ndarray, out_ref: np.ndarray, what=""):
 
 def topk_set_equal(a: np.ndarray, b: np.ndarray):
     assert np.array_equal(a, b), f"top-K differs at {np.argwhere(a != b)[:5].tolist()}"
+
+
+class Guarded:
+    """A device output buffer with canary regions on both sides: `t` is the
+    contiguous view handed to the library, the 4 KiB before and after it hold
+    a byte pattern that no kernel may touch.  `check()` raises if one changed,
+    naming the side and the first changed offset."""
+
+    GUARD = 4096
+    PATTERN = 0xA5
+
+    def __init__(self, shape, dtype, fill=None, device="cuda"):
+        shape = tuple(shape)
+        n = int(np.prod(shape)) if shape else 1
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        self._raw = torch.full((self.GUARD + nbytes + self.GUARD,), self.PATTERN,
+                               dtype=torch.uint8, device=device)
+        self.t = self._raw[self.GUARD:self.GUARD + nbytes].view(dtype).view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self):
+        if self._raw.is_cuda:
+            torch.cuda.synchronize()
+        for side, g in (("before", self._raw[:self.GUARD]), ("after", self._raw[-self.GUARD:])):
+            bad = torch.nonzero(g != self.PATTERN)
+            if bad.numel():
+                raise AssertionError(f"canary {side} the output changed at byte {int(bad[0])}")

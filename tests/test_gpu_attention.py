@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from fp4_compressed_kv_b200 import synth
-from helpers import assert_attn_close, f32, oracle_cfg, oracle_pack
+from helpers import Guarded, assert_attn_close, f32, oracle_cfg, oracle_pack
 
 pytestmark = pytest.mark.gpu
 
@@ -26,15 +26,17 @@ def _setup(kvc, w):
 
 
 def _attn(kvc, cfg, cache, q, tk, win, wl):
+    """One attention call into canary-guarded outputs (checked after it)."""
     B, H = q.shape[0], q.shape[1]
-    out = torch.full((B, H, cfg.latent_dim), float("nan"), device="cuda")
-    lse = torch.full((B, H), float("nan"), device="cuda")
+    out = Guarded((B, H, cfg.latent_dim), torch.float32, fill=float("nan"))
+    lse = Guarded((B, H), torch.float32, fill=float("nan"))
     ws = kvc.workspace(cfg, B, cache.capacity)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     kvc.sparse_decode_attn(cfg, q.cuda().contiguous(), cache, tk.cuda().contiguous(),
-                           win.cuda().contiguous(), wl, out, ws, lse=lse, status=st)
-    torch.cuda.synchronize()
-    return out.cpu().numpy(), lse.cpu().numpy(), int(st.item())
+                           win.cuda().contiguous(), wl, out.t, ws, lse=lse.t, status=st)
+    out.check()
+    lse.check()
+    return out.t.cpu().numpy(), lse.t.cpu().numpy(), int(st.item())
 
 
 @pytest.mark.parametrize("name", ["tiny", "mla32k"])

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from fp4_compressed_kv_b200 import synth
-from helpers import assert_attn_close, f32, oracle_cfg, oracle_pack
+from helpers import Guarded, assert_attn_close, f32, oracle_cfg, oracle_pack
 
 pytestmark = pytest.mark.gpu
 
@@ -22,14 +22,16 @@ def _group(kvc, w, context, batch=None):
     cache.idx_k.copy_(torch.from_numpy(ic))
     cache.n_entries.copy_(torch.from_numpy(n))
     L, B, H = w.layers, w.batch, w.heads
-    out = torch.full((L, B, H, w.latent), float("nan"), device="cuda")
-    lse = torch.empty(L, B, H, device="cuda")
-    tk = torch.empty(L, B, w.topk, dtype=torch.int32, device="cuda")
+    gout = Guarded((L, B, H, w.latent), torch.float32, fill=float("nan"))  # canaries around
+    glse = Guarded((L, B, H), torch.float32)                                # every output
+    gtk = Guarded((L, B, w.topk), torch.int32)
+    out, lse, tk = gout.t, glse.t, gtk.t
     ws = kvc.workspace(cfg, B, cache.capacity)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     kvc.layer_group_step(cfg, list(w.modes), inp["q"].cuda(), inp["idx_q"].cuda(),
                          inp["windows"].cuda(), w.window, cache, out, tk, ws, lse=lse, status=st)
-    torch.cuda.synchronize()
+    for g in (gout, glse, gtk):
+        g.check()
     ref, ref_lse, otk, ost = oracle.group_step(oracle_cfg(w), list(w.modes), f32(inp["q"]),
                                                inp["idx_q"].numpy(), f32(inp["windows"]), w.window,
                                                rec, ic, n)

@@ -6,21 +6,27 @@ import torch
 
 import oracle
 from fp4_compressed_kv_b200 import synth
-from helpers import f32, oracle_cfg, oracle_pack
+from helpers import Guarded, f32, oracle_cfg, oracle_pack
 
 pytestmark = pytest.mark.gpu
 
 
 def _gpu_pack(kvc, w, tokens, gate, idx_k, capacity=None, chunks=None):
+    """Pack into a cache whose record and indexer arrays sit between canary
+    regions (checked after the appends)."""
     cfg = kvc.config_for(w)
     B, T = tokens.shape[:2]
     cache = kvc.Cache(cfg, B, capacity or T // 2)
+    grec = Guarded(cache.records.shape, cache.records.dtype, fill=0)
+    gidx = Guarded(cache.idx_k.shape, cache.idx_k.dtype, fill=0)
+    cache.records, cache.idx_k = grec.t, gidx.t
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     step = chunks or T
     for t0 in range(0, T, step):
         kvc.pack(cfg, tokens[:, t0:t0 + step].contiguous(), gate,
                  idx_k[:, t0 // 2:(t0 + step) // 2].contiguous(), cache, status=st)
-    torch.cuda.synchronize()
+    grec.check()
+    gidx.check()
     return cache, int(st.item())
 
 

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from fp4_compressed_kv_b200 import synth
-from helpers import oracle_cfg, topk_set_equal
+from helpers import Guarded, oracle_cfg, topk_set_equal
 
 pytestmark = pytest.mark.gpu
 
@@ -18,13 +18,14 @@ def _run(kvc, w, idx_k, idx_q, n_entries, capacity):
     cache = kvc.Cache(cfg, B, capacity)
     cache.idx_k[:, : idx_k.shape[1]] = idx_k.cuda()
     cache.n_entries.copy_(torch.as_tensor(n_entries, dtype=torch.int32))
-    tk = torch.empty(B, w.topk, dtype=torch.int32, device="cuda")
-    sc = torch.zeros(B, capacity, dtype=torch.int32, device="cuda")
+    tk = Guarded((B, w.topk), torch.int32)  # canary-guarded outputs, checked after the call
+    sc = Guarded((B, capacity), torch.int32, fill=0)
     ws = kvc.workspace(cfg, B, capacity)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    kvc.index_topk(cfg, idx_q.cuda().contiguous(), cache, tk, ws, scores=sc, status=st)
-    torch.cuda.synchronize()
-    return tk.cpu().numpy(), sc.cpu().numpy(), int(st.item())
+    kvc.index_topk(cfg, idx_q.cuda().contiguous(), cache, tk.t, ws, scores=sc.t, status=st)
+    tk.check()
+    sc.check()
+    return tk.t.cpu().numpy(), sc.t.cpu().numpy(), int(st.item())
 
 
 def _oracle(w, idx_k, idx_q, n_entries, capacity):
