@@ -467,24 +467,26 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             nq = 2;
         }
 
-        // ---- softmax, warps 0-3: thread = key = tensor-memory lane.  y is
-        // the raw logit (times the FP8 row scale); x = y * qs[h] in log2 units.
-        // The HG scores are read from tensor memory 8 at a time, twice
-        // (maxima, then weights), in rolled loops: each CTA runs this once.
+        // ---- softmax, all 8 warps: thread = key = tensor-memory lane (warp w
+        // reads lane quadrant w & 3) and warp w takes head columns [c_lo,
+        // c_hi) = half (w >> 2) of the group, 8 at a time.  y is the raw logit
+        // (times the FP8 row scale); x = y * qs[h] in log2 units.  Scores are
+        // read twice (maxima, then weights), in rolled loops.
         const bool valid = k >= 0;
         const float kf = fp8 ? ks[s] : 1.f;
         const uint32_t ta_s = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL;
-        if (warp < 4) {
+        const int c8_lo = (warp >> 2) * (HG / 16), c8_hi = c8_lo + HG / 16;
+        {
 #pragma unroll 1
-            for (int h0 = 0; h0 < HG; h0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(ta_s + h0, r);
+            for (int c8 = c8_lo; c8 < c8_hi; ++c8) {
+                uint32_t r[8];
+                tmem_ld8(ta_s + 8 * c8, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     const float y = valid ? __uint_as_float(r[i]) * kf : -INFINITY;
                     const int m = __reduce_max_sync(0xffffffffu, f32_ord(y));
-                    if (lane == ((h0 + i) & 31)) wmax[warp * 64 + h0 + i] = m;
+                    if (lane == ((8 * c8 + i) & 31)) wmax[(warp & 3) * 64 + 8 * c8 + i] = m;
                 }
             }
         }
@@ -503,23 +505,19 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (it > 0 && f != 1.f) flags[0] = 1;
         }
         __syncthreads();
-        if (warp < 4) {
+        {
 #pragma unroll 1
-            for (int c16 = 0; c16 < HG / 16; ++c16) {
-                uint32_t r[16];
-                tmem_ld16(ta_s + 16 * c16, r);
+            for (int c8 = c8_lo; c8 < c8_hi; ++c8) {
+                uint32_t r[8];
+                tmem_ld8(ta_s + 8 * c8, r);
                 tmem_wait_ld();
-#pragma unroll
-              for (int half8 = 0; half8 < 2; ++half8) {
-                const int c8 = 2 * c16 + half8;
                 uint32_t w[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int h = 8 * c8 + 2 * u;
                     const float m0 = mref[h], m1 = mref[h + 1];
-                    const float y0 = valid ? __uint_as_float(r[8 * half8 + 2 * u]) * kf : -INFINITY;
-                    const float y1 =
-                        valid ? __uint_as_float(r[8 * half8 + 2 * u + 1]) * kf : -INFINITY;
+                    const float y0 = valid ? __uint_as_float(r[2 * u]) * kf : -INFINITY;
+                    const float y1 = valid ? __uint_as_float(r[2 * u + 1]) * kf : -INFINITY;
                     float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, qs[h], -m0));
                     float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, qs[h + 1], -m1));
                     if (fp8) {  // v = scale x E4M3 row: the scale moves onto p
@@ -529,7 +527,6 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     w[u] = win ? pack_bf16(p0, p1) : pack_f16(p0, p1);
                 }
                 sts128(sP + swz(s, c8), w[0], w[1], w[2], w[3]);
-              }
             }
         }
         if (!lmma) {
@@ -657,17 +654,21 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tc_fence_after();
             const bool valid = kw >= 0;
             const uint32_t ta_s = tmem + ((uint32_t)((warp & 3) * 32) << 16) + S_COL;
-            if (ok && warp < 4) {
+            // (heads split in halves between warps w and w + 4; quadrants
+            // without window rows report -inf maxima)
+            const bool rows_here = (warp & 3) * 32 < WR;
+            const int c8_lo = (warp >> 2) * (HG / 16), c8_hi = c8_lo + HG / 16;
+            if (ok) {
 #pragma unroll 1
-                for (int h0 = 0; h0 < HG; h0 += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(ta_s + h0, r);
+                for (int c8 = c8_lo; c8 < c8_hi; ++c8) {
+                    uint32_t r[8];
+                    tmem_ld8(ta_s + 8 * c8, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
+                    for (int i = 0; i < 8; ++i) {
                         const float y = valid ? __uint_as_float(r[i]) : -INFINITY;
                         const int m = __reduce_max_sync(0xffffffffu, f32_ord(y));
-                        if (lane == ((h0 + i) & 31)) wmax[warp * 64 + h0 + i] = m;
+                        if (lane == ((8 * c8 + i) & 31)) wmax[(warp & 3) * 64 + 8 * c8 + i] = m;
                     }
                 }
             }
@@ -687,30 +688,26 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             __syncthreads();
             // P^T rows of this CTA's window keys, by whole warps (the tensor-memory
-            // load is warp-collective; rows WR..31 come out as zeros, unread)
-            if (ok && warp < 4 && warp * 32 < WR) {
+            // load is warp-collective; rows WR..31 of a quadrant come out as
+            // zeros, unread)
+            if (ok && rows_here) {
 #pragma unroll 1
-                for (int c16 = 0; c16 < HG / 16; ++c16) {
-                    uint32_t r[16];
-                    tmem_ld16(ta_s + 16 * c16, r);
+                for (int c8 = c8_lo; c8 < c8_hi; ++c8) {
+                    uint32_t r[8];
+                    tmem_ld8(ta_s + 8 * c8, r);
                     tmem_wait_ld();
+                    uint32_t w[4];
 #pragma unroll
-                    for (int half8 = 0; half8 < 2; ++half8) {
-                        const int c8 = 2 * c16 + half8;
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int h = 8 * c8 + 2 * u;
-                            const float m0 = mref[h], m1 = mref[h + 1];
-                            const float y0 = valid ? __uint_as_float(r[8 * half8 + 2 * u]) : -INFINITY;
-                            const float y1 =
-                                valid ? __uint_as_float(r[8 * half8 + 2 * u + 1]) : -INFINITY;
-                            const float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, sm_log2, -m0));
-                            const float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, sm_log2, -m1));
-                            w[u] = pack_bf16(p0, p1);
-                        }
-                        sts128(sPw + swz(s, c8), w[0], w[1], w[2], w[3]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int h = 8 * c8 + 2 * u;
+                        const float m0 = mref[h], m1 = mref[h + 1];
+                        const float y0 = valid ? __uint_as_float(r[2 * u]) : -INFINITY;
+                        const float y1 = valid ? __uint_as_float(r[2 * u + 1]) : -INFINITY;
+                        const float p0 = m0 == -INFINITY ? 0.f : ex2(fmaf(y0, sm_log2, -m0));
+                        const float p1 = m1 == -INFINITY ? 0.f : ex2(fmaf(y1, sm_log2, -m1));
+                        w[u] = pack_bf16(p0, p1);
                     }
+                    sts128(sPw + swz(s, c8), w[0], w[1], w[2], w[3]);
                 }
             }
             fence_async_smem();
