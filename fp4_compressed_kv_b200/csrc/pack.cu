@@ -12,10 +12,15 @@
 // entries per warp, 32 per CTA); lane l of a team owns the 8-channel chunks
 // c = l, l+8, ..., so for the 576-channel MLA entry every lane holds 9 chunks
 // and no lane idles.  Each chunk of each token is one 16-byte load and the 8
-// lanes of a team read 128 contiguous bytes; the raw bf16 chunks stay packed in
-// registers between the two passes.  A chunk's eight codes leave as one 4-byte
-// store (a team writes 32 contiguous bytes per pass).  Group maxima are xor
-// shuffles inside the team (G <= 64) or a shared-memory reduction (G > 64).
+// lanes of a team read 128 contiguous bytes; a chunk's eight codes leave as one
+// 4-byte store (a team writes 32 contiguous bytes per chunk step).  Appends of
+// more than 4,096 entries with groups of at most 64 channels take the
+// streaming kernel (pack_stream_kernel: the chunks read twice, L1-resident
+// between the passes, arithmetic on fp32 pairs, no division); groups of 128
+// channels the register-held kernel (pack_kernel: the raw chunks kept packed in
+// registers between the passes, group maxima through shared memory); decode
+// appends a warp per entry (pack_small_kernel) and 4:1 appends likewise
+// (pack_group4_kernel).
 //
 // Bit-exactness: the gate logit difference is accumulated in fp32 in a fixed
 // order -- lane l sums its chunks in increasing order, one fmaf per channel
