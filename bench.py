@@ -748,11 +748,13 @@ def run_ours(args):
 
         def e2e_step(r):
             windows = sets[step_ids[r]]["windows"]  # the windows stay on the device
+            # the small inputs first: host-to-device copies run in order, and
+            # the pack, scan and selection need only these
+            din.copy_(hins[r], non_blocking=True)
             copy_stream.wait_stream(stream)  # the previous step no longer reads dq
             with torch.cuda.stream(copy_stream):
                 dq.copy_(hqs[r], non_blocking=True)
                 q_ready.record(copy_stream)
-            din.copy_(hins[r], non_blocking=True)
             kvc.pack(cfg, dtok, gate, didx, cache, status=status)
             if split:  # one Full layer: its scan and selection need no queries
                 kvc.index_topk(cfg, diq[0], cache, topk[0], ws, status=status)
@@ -766,7 +768,12 @@ def run_ours(args):
                                      hier_block=args.hier_block)
             hres.copy_(dres, non_blocking=True)
 
-        e2e_step(reps)  # warm-up with the spare input set
+        # warm-up: one pass over every step's pinned buffers (a first transfer
+        # from a pinned buffer runs at a fraction of the link rate; a serving
+        # loop reuses warm staging buffers), then the spare set
+        for r in range(reps + 1):
+            e2e_step(r)
+            cache.n_entries.copy_(n_before)
         torch.cuda.synchronize()
         cache.n_entries.copy_(n_before)
         kd.barrier()
@@ -785,10 +792,10 @@ def run_ours(args):
         e2e = {"value": round(kd.job_throughput(reps, B, world, te_ms), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(te_ms / reps, 4),
-               "inputs": "a new query set uploaded every step",
+               "inputs": "a new query set uploaded every step (each step's pinned buffer used once in the warm-up)",
                "api": ("kvc_pack, kvc_index_topk, kvc_sparse_decode_attn" if split else
                        "kvc_pack, kvc_layer_group_step"),
-               "overlap": "query upload on a copy stream during pack, scan and selection"
+               "overlap": "small inputs first, then the query upload on a copy stream during pack, scan and selection"
                           if split else "none"}
         del hins, hqs
 
