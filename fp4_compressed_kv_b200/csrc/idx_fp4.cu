@@ -15,8 +15,8 @@
 // double):
 //  1. idx_fp4_scan_fast: CTA (x, b) scores 4096 rows of sequence b; a warp
 //     stages blocks of 32 rows with coalesced 8-byte loads (the next block's
-//     in flight) and each lane scores one row: byte permutes turn four codes
-//     into four signed twice-values for one dp4a with the query; the group sum
+//     in flight) and each lane scores one row: byte permutes turn eight codes
+//     into eight signed twice-values for two dp4a with the query; the group sum
 //     times the scale's table value accumulates in 64 bits.  The row's 64-bit
 //     key (score, then index) is stored and its bin -- 16 per octave of |S| --
 //     counted; the sequence's last CTA derives the threshold bin.
@@ -189,22 +189,25 @@ __device__ __forceinline__ int key_row(unsigned long long k) {
     return (int)(0xFFFFFFu - (uint32_t)(k & 0xFFFFFFull));
 }
 
-// Four E2M1 codes (channel i in nibble i of the low 16 bits of x) as four
-// signed int8 twice-values (byte i) by byte permutes: the magnitude index
-// picks from a table of twice-magnitudes {0,1,2,3,4,6,8,12} and from its
-// negation, then each byte comes from one or the other by its sign bit.
-// (prmt.b32 in its default mode: bit 3 of a selector nibble would replicate
-// the byte's sign, so every selector here has it clear.)
+// Eight E2M1 codes (channel i in nibble i of w) as eight signed int8
+// twice-values, channels 0-3 in lo and 4-7 in hi, by byte permutes: the
+// magnitude index picks from a table of twice-magnitudes {0,1,2,3,4,6,8,12}
+// and from its negation, then each byte comes from one or the other by its
+// sign bit.  prmt.b32 in its default mode reads its selector from the low 16
+// bits (bit 3 of a nibble would replicate the byte's sign, so every selector
+// here has it clear); the high half's selectors are the shared masks shifted.
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
 }
-__device__ __forceinline__ uint32_t e2m1x4_twice(uint32_t x) {
-    const uint32_t sel = x & 0x7777u;
-    const uint32_t pos = prmt(0x03020100u, 0x0C080604u, sel);
-    const uint32_t neg = prmt(0xFDFEFF00u, 0xF4F8FAFCu, sel);
-    return prmt(pos, neg, 0x3210u | ((x >> 1) & 0x4444u));
+__device__ __forceinline__ void e2m1x8_twice(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t sel = w & 0x77777777u;                          // magnitude indexes
+    const uint32_t pick = ((w >> 1) & 0x44444444u) | 0x32103210u;  // byte i or byte 4 + i
+    const uint32_t sel_h = sel >> 16, pick_h = pick >> 16;
+    lo = prmt(prmt(0x03020100u, 0x0C080604u, sel), prmt(0xFDFEFF00u, 0xF4F8FAFCu, sel), pick);
+    hi = prmt(prmt(0x03020100u, 0x0C080604u, sel_h), prmt(0xFDFEFF00u, 0xF4F8FAFCu, sel_h),
+              pick_h);
 }
 
 // idx_fp4_scan_fast: CTA (x, b) scores rows [4096 x, 4096 x + 4096) of
@@ -273,10 +276,13 @@ idx_fp4_scan_fast(TopkArgs a, unsigned long long* __restrict__ keys) {
             for (int g = 0; g < NG; ++g) {
                 const uint2 cw = row[g];
                 const uint4 qg = reinterpret_cast<const uint4*>(qs)[g];  // (broadcast)
-                int part = __dp4a((int)e2m1x4_twice(cw.x), (int)qg.x, 0);
-                part = __dp4a((int)e2m1x4_twice(cw.x >> 16), (int)qg.y, part);
-                part = __dp4a((int)e2m1x4_twice(cw.y), (int)qg.z, part);
-                part = __dp4a((int)e2m1x4_twice(cw.y >> 16), (int)qg.w, part);
+                uint32_t c0, c1, c2, c3;
+                e2m1x8_twice(cw.x, c0, c1);
+                e2m1x8_twice(cw.y, c2, c3);
+                int part = __dp4a((int)c0, (int)qg.x, 0);
+                part = __dp4a((int)c1, (int)qg.y, part);
+                part = __dp4a((int)c2, (int)qg.z, part);
+                part = __dp4a((int)c3, (int)qg.w, part);
                 const uint2 sw = row[NG + (g >> 3)];
                 const uint32_t sword = (g & 4) ? sw.y : sw.x;
                 S += (long long)part * s512[(sword >> (8 * (g & 3))) & 0xFFu];

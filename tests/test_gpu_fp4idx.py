@@ -126,6 +126,7 @@ def _random_rows(B, N, di, seed, scale_lo=0x20, scale_hi=0x48):
     (128, 65536, "random"),      # full-size sequences: 16 scan tiles, 8 select tiles
     (256, 9000, "tie_block"),    # 2000 copies of the best row: the cut sorts ~2000 ties
     (128, 9000, "wide_scales"),  # scales over the whole UE4M3 range (subnormal to 448)
+    (128, 9001, "odd_rows"),     # 72-byte rows at odd positions; the buffer's last row read
     (64, 5000, "random"),        # 64-channel rows: the direct kernels
 ])
 def test_fp4_scan_and_select_paths(kvc, di, N, case):
@@ -140,6 +141,8 @@ def test_fp4_scan_and_select_paths(kvc, di, N, case):
     if case == "all_equal":
         rows[0] = rows[0, 5]
     n = np.array([N, N - 77, N // 2 + 3], np.int32)
+    if case == "odd_rows":  # sequence 1 starts at an odd row; sequence 2 fills its capacity
+        n = np.array([N - 77, N // 2 + 3, N], np.int32)
     q = torch.randint(-128, 128, (B, di), generator=torch.Generator().manual_seed(9),
                       dtype=torch.int8)
     if case == "tie_block":  # the threshold bin then holds all 2000 copies
