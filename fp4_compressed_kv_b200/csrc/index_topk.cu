@@ -25,6 +25,9 @@
 // hand-offs are counters that nobody polls.
 #include <algorithm>
 #include <climits>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <mutex>
 
 #include "topk_common.cuh"
 
@@ -55,7 +58,8 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint64_t
             : "memory");
         return ok != 0;
     }
-    const uint64_t t0 = now_ns();
+    // the clock is read only once the phase is found incomplete
+    uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
         asm volatile(
@@ -66,7 +70,8 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint64_t
             : "r"(bar), "r"(parity)
             : "memory");
         if (ok) return true;
-        if ((i & 255) == 255 && now_ns() - t0 > limit_ns) return false;
+        if (i == 0) t0 = now_ns();
+        else if ((i & 255) == 255 && now_ns() - t0 > limit_ns) return false;
     }
 }
 // The indexer rows are read once per scan: bulk copies carry an L2
@@ -407,17 +412,34 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
 // ---- batched scoring on the tensor cores: several indexer queries of the
 // same sequence against each 128-row tile of its indexer keys in one
 // tcgen05.mma kind::i8 (M = 128 rows, N = 16 padded queries, K = 128 int8 as
-// 4 steps of 32), accumulators in tensor memory.  The rows stream in as
-// plain bulk copies and are re-laid into the 128-byte-swizzled K-major
-// operand tile in shared memory; each thread then owns one row's scores.
+// 4 steps of 32), accumulators in tensor memory.  A 128-byte key row is one
+// 128-byte swizzle row, so a TMA tile load (128-byte swizzle) puts a tile in
+// shared memory already in the operand layout.  One CTA per SM runs a
+// warp-specialised pipeline over its slice of tiles, the stages linked by
+// mbarriers:
+//   warp 4 (loads): one TMA load per tile into a ring of NS stages, once the
+//     products of the tile NS back have released the stage;
+//   warp 5 (products): the queries of a new sequence into the B tile (after
+//     the earlier products are done), then a tile's four MMAs into one of
+//     NACC accumulators (once the epilogue has read it), committed twice: to
+//     the stage (free again) and to the accumulator (scores ready);
+//   warps 0-3 (epilogue, lane quadrant = warp): each thread one row: its nq
+//     scores from tensor memory, stored and counted in per-query histograms;
+//     at a sequence's end in this CTA the histograms are flushed and the
+//     sequence's last CTA derives each query's threshold (barriers among
+//     these 128 threads only).
+// Every wait is bounded; a wait that gives up sets KVC_DEV_TIMEOUT and an
+// abort flag the other warps see before their next wait.
 namespace tcs {
-constexpr int NT = 128;           // thread t <-> tensor-memory lane t <-> row t of the tile
+constexpr int NT = 192;
 constexpr int ROWS = 128;         // rows per tile (MMA M)
 constexpr int DI = 128;           // indexer width: one 128-byte swizzle row
 constexpr int NQP = 16;           // MMA N (queries, padded)
 constexpr int TILE = ROWS * DI;   // 16 KB
-constexpr int MAX_STAGES = 8;
-constexpr uint32_t TMEM_COLS = 32;
+constexpr int MAX_STAGES = 12;
+constexpr int NACC = 4;
+constexpr uint32_t TMEM_COLS = 64;  // NACC accumulators of 16 columns
+constexpr uint32_t kEpiBar = 1;     // named barrier of the epilogue warps
 // D s32 (2 << 4), A and B s8 (1 << 7, 1 << 10), both K-major, N = 16, M = 128
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NQP >> 3) << 17) |
                             ((uint32_t)(ROWS >> 4) << 24);
@@ -435,41 +457,131 @@ __device__ __forceinline__ void mma_i8(uint32_t d, uint64_t ad, uint64_t bd, uin
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
         "l"(ad), "l"(bd), "r"(kIdesc), "r"(acc));
 }
+__device__ __forceinline__ void commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void named_sync() {
+    asm volatile("bar.sync %0, 128;\n" ::"n"(kEpiBar) : "memory");
+}
+// true on every epilogue thread iff `v` is true on all 128 of them
+__device__ __forceinline__ bool epi_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(kEpiBar)
+        : "memory");
+    return r != 0;
+}
+// The tile's rows: 128 rows of the key tensor from (0, y) by TMA, 128-byte
+// swizzle, L2 evict-first (read once).
+__device__ __forceinline__ void tma_rows(uint32_t dst, const CUtensorMap* map, int y, uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar),
+                 "r"((uint32_t)TILE)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(bar), "l"(evict_first_policy())
+        : "memory");
+}
+// Threshold bin of a histogram in shared memory by the 128 epilogue threads
+// (thread e covers bins [kBins - 16 (e + 1), kBins - 16 e)); as find_threshold.
+__device__ __forceinline__ void epi_threshold(const int* s_hist, int K, int* t_out,
+                                              int* above_out, int* sh_warp, int e) {
+    const int hi = kBins - e * 16, lo = hi - 16;
+    int local = 0;
+    for (int b = lo; b < hi; ++b) local += s_hist[b];
+    const int lane = e & 31, w = e >> 5;
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += u;
+    }
+    if (lane == 31) sh_warp[w] = x;
+    named_sync();
+    int pre = 0;
+    for (int i = 0; i < w; ++i) pre += sh_warp[i];
+    const int excl = pre + x - local, incl = excl + local;
+    if (excl < K && incl >= K) {
+        int run = excl;
+        for (int b = hi - 1; b >= lo; --b) {
+            if (run + s_hist[b] >= K) {
+                *t_out = b;
+                *above_out = run;
+                break;
+            }
+            run += s_hist[b];
+        }
+    }
+    named_sync();
+}
+// A tile: rows [row, min(row + ROWS, end)) of sequence b, walked over this
+// CTA's slice of the batch laid end to end; `seq` counts the sequences entered.
+struct Tile {
+    int b, row, end, seq;
+};
+__device__ __forceinline__ bool tile_first(const TopkArgs& a, long long lo, long long hi, Tile& t) {
+    ScanCursor c;
+    if (!cursor_seek(a, lo, hi, c, (int)(lo / a.capacity))) return false;
+    t.b = c.b;
+    t.row = c.row;
+    t.end = c.end;
+    t.seq = 0;
+    return true;
+}
+__device__ __forceinline__ bool tile_next(const TopkArgs& a, long long lo, long long hi, Tile& t) {
+    t.row += min(ROWS, t.end - t.row);
+    if (t.row < t.end) return true;
+    ScanCursor c;
+    if (!cursor_seek(a, lo, hi, c, t.b + 1)) return false;
+    t.b = c.b;
+    t.row = c.row;
+    t.end = c.end;
+    ++t.seq;
+    return true;
+}
 }  // namespace tcs
 
-__global__ void __launch_bounds__(tcs::NT, 2)
-index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int stages) {
+__global__ void __launch_bounds__(tcs::NT, 1)
+index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba, long long per,
+                     int bias, int shift, int stages) {
     using namespace tcs;
     extern __shared__ __align__(1024) unsigned char tsm[];
     const TopkArgs& a = ba.q[0];
     const int nq = ba.nq;
-    // 1024-aligned layout: A tile, B tile, raw ring, histograms [nq][kBins]
+    // 1024-aligned layout: NS stages, the B tile, histograms [nq][kBins]
     const uint32_t base0 = smem_addr(tsm);
-    const uint32_t pad = ((base0 + 1023u) & ~1023u) - base0;
-    unsigned char* sm = tsm + pad;
-    const uint32_t sA = smem_addr(sm), sB = sA + TILE;
-    unsigned char* ring = sm + TILE + 2048;
-    int* hist = reinterpret_cast<int*>(ring + (size_t)stages * TILE);
-    __shared__ __align__(8) uint64_t full[MAX_STAGES];
-    __shared__ __align__(8) uint64_t mma_bar;
+    unsigned char* sm = tsm + (((base0 + 1023u) & ~1023u) - base0);
+    const uint32_t sA = smem_addr(sm), sB = sA + stages * TILE;
+    int* hist = reinterpret_cast<int*>(sm + (size_t)stages * TILE + 2048);
+    __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], done[NACC], read[NACC];
     __shared__ uint32_t tmem_slot;
-    __shared__ int sh_warp[NT / 32];
+    __shared__ int sh_warp[4];
     __shared__ int s_last, s_t, s_above;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    __shared__ volatile int s_abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long cap = a.capacity;
     const long long lo = (long long)blockIdx.x * per;
     const long long hi = min(lo + per, (long long)a.batch * cap);
     if (lo >= hi) return;
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
-                         smem_addr(&tmem_slot)),
-                     "r"(TMEM_COLS));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
-    }
     if (tid == 0) {
-        for (int st = 0; st < stages; ++st)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[st])));
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&mma_bar)));
+        for (int s = 0; s < stages; ++s) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&empty[s])));
+        }
+        for (int s = 0; s < NACC; ++s) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&done[s])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 4;\n" ::"r"(smem_addr(&read[s])));
+        }
+        s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     for (int i = tid; i < nq * kBins; i += NT) hist[i] = 0;
@@ -479,157 +591,192 @@ index_scan_tc_kernel(BatchTopkArgs ba, long long per, int bias, int shift, int s
             const int n = a.n_entries[b];
             if (n < 0 || n > a.capacity) set_status(a.status, KVC_DEV_BAD_LENGTH);
         }
+    Tile t0;
+    if (!tile_first(a, lo, hi, t0)) return;  // (the same for the whole CTA)
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_addr(&tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+    }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     const uint32_t tmem = tmem_slot;
-    bool ok = true;
-    uint32_t phase = 0, mma_phase = 0;
-    ScanCursor cc;
-    const bool any = cursor_seek(a, lo, hi, cc, (int)(lo / cap));
-    if (any) {
-        ScanCursor pc = cc;
-        bool pmore = true;
-        auto issue = [&](int st) {  // thread 0: the next tile of rows into raw stage st
-            const int rows = min(ROWS, pc.end - pc.row);
-            bulk_load(smem_addr(ring + (size_t)st * TILE),
-                      a.idx_k + ((size_t)pc.b * a.idx_capacity + pc.row) * DI, (uint32_t)rows * DI,
-                      smem_addr(&full[st]));
-            pc.row += rows;
-            if (pc.row >= pc.end) pmore = cursor_seek(a, lo, hi, pc, pc.b + 1);
-        };
-        if (tid == 0)
-            for (int st = 0; st < stages && pmore; ++st) issue(st);
-        int qb = -1;  // sequence whose queries are in the B tile
-        for (int tile = 0;; ++tile) {
-            const int st = tile % stages;
-            const int rows = min(ROWS, cc.end - cc.row);
-            if (cc.b != qb) {  // this sequence's queries, zero-padded, into B
-                qb = cc.b;
-                for (int p = tid; p < NQP * (DI / 16); p += NT) {
+    auto give_up = [&]() {
+        s_abort = 1;
+        set_status(a.status, KVC_DEV_TIMEOUT);
+    };
+    int issued = 0;  // (loads warp) tiles loaded
+    if (warp == 4) {
+        // ---- loads (each decision is the warp's: lanes agree by vote)
+        Tile t = t0;
+        for (int i = 0;; ++i) {
+            const int s = i % stages;
+            if (i >= stages) {
+                if (__any_sync(0xffffffffu, s_abort != 0)) break;
+                const bool got = bar_wait(smem_addr(&empty[s]), (uint32_t)(i / stages - 1) & 1u,
+                                          a.wait_ns);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) give_up();
+                    break;
+                }
+            }
+            if (lane == 0)
+                tma_rows(sA + s * TILE, &tm_k, (int)((long long)t.b * a.idx_capacity + t.row),
+                         smem_addr(&full[s]));
+            issued = i + 1;
+            if (!tile_next(a, lo, hi, t)) break;
+        }
+    } else if (warp == 5) {
+        // ---- products
+        Tile t = t0;
+        int built = -1, i = 0;
+        for (;; ++i) {
+            const int s = i % stages, c = i % NACC;
+            if (built != t.seq) {
+                // this sequence's queries, zero-padded, into B once every
+                // earlier product (in issue order) is done
+                if (i > 0) {
+                    const int pi = i - 1;
+                    const bool got = bar_wait(smem_addr(&done[pi % NACC]),
+                                              (uint32_t)(pi / NACC) & 1u, a.wait_ns);
+                    if (!__all_sync(0xffffffffu, got)) {
+                        if (lane == 0) give_up();
+                        break;
+                    }
+                }
+                for (int p = lane; p < NQP * (DI / 16); p += 32) {
                     const int q = p / (DI / 16), c16 = p - q * (DI / 16);
                     uint4 v = make_uint4(0, 0, 0, 0);
                     if (q < nq)
-                        v = __ldg(reinterpret_cast<const uint4*>(ba.q[q].idx_q + (size_t)qb * DI) + c16);
+                        v = __ldg(reinterpret_cast<const uint4*>(ba.q[q].idx_q + (size_t)t.b * DI) + c16);
                     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(sB + swz(q, c16)),
                                  "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
                 }
+                built = t.seq;
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
             }
-            const bool got =
-                warp == 0 ? bar_wait(smem_addr(&full[st]), (phase >> st) & 1u, a.wait_ns) : true;
-            if (__syncthreads_and(got) == 0) {
-                ok = false;
-                break;
-            }
-            phase ^= 1u << st;
-            // re-lay row tid of the raw stage into the swizzled A tile
-            {
-                const unsigned char* src = ring + (size_t)st * TILE + tid * DI;
-#pragma unroll
-                for (int c = 0; c < DI / 16; ++c) {
-                    const int c16 = (c + tid) & 7;
-                    const uint4 v = *reinterpret_cast<const uint4*>(src + c16 * 16);
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(sA + swz(tid, c16)),
-                                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
-                }
-            }
-            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-            asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-            __syncthreads();  // A and B ready; raw stage st free again
-            if (tid == 0) {
-                if (pmore) issue(st);
-                asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-#pragma unroll
-                for (int ks = 0; ks < DI / 32; ++ks)
-                    mma_i8(tmem, sdesc(sA + ks * 32), sdesc(sB + ks * 32), ks > 0 ? 1u : 0u);
-                asm volatile(
-                    "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                        smem_addr(&mma_bar))
-                    : "memory");
-            }
-            const bool done = warp == 0 ? bar_wait(smem_addr(&mma_bar), mma_phase, a.wait_ns) : true;
-            mma_phase ^= 1u;
-            if (__syncthreads_and(done) == 0) {
-                ok = false;
+            if (__any_sync(0xffffffffu, s_abort != 0)) break;
+            bool got = bar_wait(smem_addr(&full[s]), (uint32_t)(i / stages) & 1u, a.wait_ns);
+            if (got && i >= NACC)  // accumulator c: its last tile's scores have been read
+                got = bar_wait(smem_addr(&read[c]), (uint32_t)(i / NACC - 1) & 1u, a.wait_ns);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) give_up();
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-            uint32_t r[16];
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-                "%13,%14,%15}, [%16];\n"
-                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                  "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                  "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                : "r"(tmem + ((uint32_t)(warp * 32) << 16)));
+            if (lane == 0) {
+#pragma unroll
+                for (int ks = 0; ks < DI / 32; ++ks)
+                    mma_i8(tmem + (uint32_t)c * NQP, sdesc(sA + s * TILE + ks * 32),
+                           sdesc(sB + ks * 32), ks > 0 ? 1u : 0u);
+                commit(smem_addr(&empty[s]));
+                commit(smem_addr(&done[c]));
+            }
+            __syncwarp();
+            if (!tile_next(a, lo, hi, t)) {
+                ++i;
+                break;
+            }
+        }
+        // the products issued are done before the tensor memory is freed
+        if (lane == 0 && i > 0)
+            bar_wait(smem_addr(&done[(i - 1) % NACC]), (uint32_t)((i - 1) / NACC) & 1u,
+                     kCleanupWaitNs);
+        __syncwarp();
+    } else {
+        // ---- epilogue: rows warp * 32 + lane of every tile
+        const int e = tid, row = warp * 32 + lane;
+        Tile t = t0;
+        for (int i = 0;; ++i) {
+            const int c = i % NACC;
+            // the four warps decide together (they meet at barriers below)
+            const bool got = !s_abort && bar_wait(smem_addr(&done[c]),
+                                                  (uint32_t)(i / NACC) & 1u, a.wait_ns);
+            if (!epi_all(got)) {
+                if (e == 0 && !s_abort) give_up();
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+            uint32_t r[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                           "=r"(r[6]), "=r"(r[7])
+                         : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c * NQP));
             asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-            if (tid < rows) {
-                const size_t row = (size_t)cc.b * cap + cc.row + tid;
+            asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+            __syncwarp();
+            if (lane == 0) arrive(smem_addr(&read[c]));  // the accumulator is free
+            const int nrows = min(ROWS, t.end - t.row);
+            if (row < nrows) {
+                const size_t at = (size_t)t.b * cap + t.row + row;
 #pragma unroll
                 for (int q = 0; q < kMaxBatchQ; ++q)
                     if (q < nq) {
                         const int v = (int)r[q];
-                        ba.q[q].scores[row] = v;
+                        ba.q[q].scores[at] = v;
                         atomicAdd(&hist[q * kBins + score_bin(v, bias, shift)], 1);
                     }
             }
-            asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-            __syncthreads();  // the accumulator and the A tile are free again
-            cc.row += rows;
-            if (cc.row < cc.end) continue;
-            // ---- sequence cc.b done in this CTA: flush, maybe derive thresholds
-            const int b = cc.b;
-            const int n = a.n_entries[b];
-            if (n > a.topk) {
-                for (int q = 0; q < nq; ++q) {
-                    int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
-                    for (int i = tid; i < kBins; i += NT)
-                        if (hist[q * kBins + i]) atomicAdd(&gh[i], hist[q * kBins + i]);
-                }
-                const long long sbase = (long long)b * cap;
-                const long long first = sbase / per, last = (sbase + n - 1) / per;
-                __threadfence();
-                __syncthreads();
-                if (tid == 0)
-                    s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) ==
-                             (int)(last - first);
-                __syncthreads();
-                if (s_last) {
-                    __threadfence();
-                    if (tid == 0) a.counters[(size_t)a.batch * kBins + b] = 0;
+            if (t.row + nrows >= t.end) {
+                // ---- sequence t.b done in this CTA: flush, maybe derive thresholds
+                named_sync();  // every count of the sequence is in the histograms
+                const int b = t.b;
+                const int n = a.n_entries[b];
+                if (n > a.topk) {
                     for (int q = 0; q < nq; ++q) {
                         int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
-                        int* h = hist + q * kBins;
-                        for (int i = tid; i < kBins; i += NT) {
-                            h[i] = __ldcg(gh + i);
-                            gh[i] = 0;  // left zeroed for the next call
+                        for (int k = e; k < kBins; k += 128)
+                            if (hist[q * kBins + k]) atomicAdd(&gh[k], hist[q * kBins + k]);
+                    }
+                    const long long sbase = (long long)b * cap;
+                    const long long first = sbase / per, last = (sbase + n - 1) / per;
+                    __threadfence();
+                    named_sync();
+                    if (e == 0)
+                        s_last = atomicAdd(a.counters + (size_t)a.batch * kBins + b, 1) ==
+                                 (int)(last - first);
+                    named_sync();
+                    if (s_last) {
+                        __threadfence();
+                        if (e == 0) a.counters[(size_t)a.batch * kBins + b] = 0;
+                        for (int q = 0; q < nq; ++q) {
+                            int32_t* gh = ba.q[q].counters + (size_t)b * kBins;
+                            int* h = hist + q * kBins;
+                            for (int k = e; k < kBins; k += 128) {
+                                h[k] = __ldcg(gh + k);
+                                gh[k] = 0;  // left zeroed for the next call
+                            }
+                            if (e == 0) s_t = s_above = 0;
+                            named_sync();
+                            epi_threshold(h, a.topk, &s_t, &s_above, sh_warp, e);
+                            if (e == 0) {
+                                ba.q[q].thr[2 * b] = s_t;
+                                ba.q[q].thr[2 * b + 1] = s_above;
+                            }
+                            named_sync();
                         }
-                        if (tid == 0) s_t = s_above = 0;
-                        __syncthreads();
-                        find_threshold(h, a.topk, &s_t, &s_above, sh_warp);
-                        if (tid == 0) {
-                            ba.q[q].thr[2 * b] = s_t;
-                            ba.q[q].thr[2 * b + 1] = s_above;
-                        }
-                        __syncthreads();
                     }
                 }
+                named_sync();
+                for (int k = e; k < nq * kBins; k += 128) hist[k] = 0;
+                named_sync();
             }
-            __syncthreads();
-            for (int i = tid; i < nq * kBins; i += NT) hist[i] = 0;
-            if (!cursor_seek(a, lo, hi, cc, b + 1)) break;
-            __syncthreads();
+            if (!tile_next(a, lo, hi, t)) break;
         }
     }
-    if (!ok && tid == 0) {
-        set_status(a.status, KVC_DEV_TIMEOUT);
-        for (int st = 0; st < stages; ++st)
-            bar_wait(smem_addr(&full[st]), (phase >> st) & 1u, kCleanupWaitNs);
-        bar_wait(smem_addr(&mma_bar), mma_phase, kCleanupWaitNs);
-    }
+    pdl_trigger();
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 4 && lane == 0 && s_abort) {
+        // after a wait gave up: let the loads still in flight land before this
+        // CTA's shared memory is released
+        for (int k = max(0, issued - stages); k < issued; ++k)
+            bar_wait(smem_addr(&full[k % stages]), (uint32_t)(k / stages) & 1u, kCleanupWaitNs);
+    }
+    if (warp == 5) {
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
                      "r"(TMEM_COLS));
@@ -689,6 +836,29 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
     return launch_select(a, bias, shift, s);
 }
 
+// 2-D u8 tensor [rows][128] of indexer key rows (row stride 128 B), boxes of
+// 128 x 128 bytes, 128-byte swizzle, zero fill past the end.
+static bool encode_key_rows(CUtensorMap* m, const void* base, unsigned long long rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)tcs::DI, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)tcs::DI};
+    const cuuint32_t box[2] = {(cuuint32_t)tcs::DI, (cuuint32_t)tcs::ROWS};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba0, cudaStream_t s) {
     BatchTopkArgs ba = ba0;
     for (int q = 0; q < kMaxBatchQ; ++q) ba.q[q].wait_ns = device_wait_limit_ns();
@@ -700,35 +870,33 @@ cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba0, cudaStream_t s) 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // two CTAs per SM when at least two 16 KB stages fit in half an SM's shared
-    // memory beside the tiles and histograms (their per-tile round trips
-    // overlap), else one CTA with as many stages as fit
-    const size_t fixed = 1024 + tcs::TILE + 2048 + (size_t)ba.nq * kBins * 4;
-    int per_sm = 2;
-    size_t budget = 112 * 1024;
-    if ((budget - fixed) / tcs::TILE < 2) {
-        per_sm = 1;
-        budget = 200 * 1024;
-    }
+    // one CTA per SM: as many 16 KB stages as fit beside the query tile and
+    // the nq histograms
+    const size_t fixed = 1024 + 2048 + (size_t)ba.nq * kBins * 4;
+    const size_t budget = 224 * 1024;
     int stages = (int)((budget - fixed) / tcs::TILE);
     stages = std::max(2, std::min(stages, tcs::MAX_STAGES));
     const size_t smem = fixed + (size_t)stages * tcs::TILE;
     static bool attr_set[64] = {};
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         err = cudaFuncSetAttribute(index_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   200 * 1024 + 2048);
+                                   (int)budget);
         if (err != cudaSuccess) return err;
         attr_set[dev] = true;
     }
     const long long rows = (long long)a.batch * a.capacity;
-    int ctas = per_sm * sms;
+    int ctas = sms;
     long long per = (rows + ctas - 1) / ctas;
     per = (per + tcs::ROWS - 1) / tcs::ROWS * tcs::ROWS;
     if (per < tcs::ROWS) per = tcs::ROWS;
     ctas = (int)((rows + per - 1) / per);
     if (rows > 0) {
+        CUtensorMap tm;
+        if (!encode_key_rows(&tm, a.idx_k, (unsigned long long)a.batch * a.idx_capacity))
+            return cudaErrorInvalidValue;
         trace_before("index_scan_tc", s);
-        err = launch_pdl(index_scan_tc_kernel, ctas, tcs::NT, smem, s, ba, per, bias, shift, stages);
+        err = launch_pdl(index_scan_tc_kernel, ctas, tcs::NT, smem, s, tm, ba, per, bias, shift,
+                         stages);
         trace_after(s);
         if (err != cudaSuccess) return err;
     }

@@ -65,7 +65,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, uint64
             : "memory");
         return ok != 0;
     }
-    const uint64_t t0 = global_ns();
+    // the clock is read only once the phase is found incomplete
+    uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
         asm volatile(
@@ -76,7 +77,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, uint64
             : "r"(addr), "r"(parity)
             : "memory");
         if (ok) return true;
-        if ((i & 63) == 63 && global_ns() - t0 > limit_ns) return false;
+        if (i == 0) t0 = global_ns();
+        else if ((i & 63) == 63 && global_ns() - t0 > limit_ns) return false;
     }
 }
 // D (tensor memory) [+]= A (shared) x B (shared), kind::f16 operands.
