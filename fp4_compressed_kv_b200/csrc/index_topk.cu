@@ -414,16 +414,17 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
 // tcgen05.mma kind::i8 (M = 128 rows, N = 16 padded queries, K = 128 int8 as
 // 4 steps of 32), accumulators in tensor memory.  A 128-byte key row is one
 // 128-byte swizzle row, so a TMA tile load (128-byte swizzle) puts a tile in
-// shared memory already in the operand layout.  One CTA per SM runs a
+// shared memory already in the operand layout.  A stage holds 256 rows (two
+// products of 128), which halves the per-row cost of the waits and commits.  One CTA per SM runs a
 // warp-specialised pipeline over its slice of tiles, the stages linked by
 // mbarriers:
 //   warp 4 (loads): one TMA load per tile into a ring of NS stages, once the
 //     products of the tile NS back have released the stage;
 //   warp 5 (products): the queries of a new sequence into the B tile (after
-//     the earlier products are done), then a tile's four MMAs into one of
-//     NACC accumulators (once the epilogue has read it), committed twice: to
-//     the stage (free again) and to the accumulator (scores ready);
-//   warps 0-3 (epilogue, lane quadrant = warp): each thread one row: its nq
+//     the earlier products are done), then a tile's 2 x 4 MMAs into one of
+//     NPAIR accumulator pairs (once the epilogue has read it), committed
+//     twice: to the stage (free again) and to the pair (scores ready);
+//   warps 0-3 (epilogue, lane quadrant = warp): each thread two rows: their nq
 //     scores from tensor memory, stored and counted in per-query histograms;
 //     at a sequence's end in this CTA the histograms are flushed and the
 //     sequence's last CTA derives each query's threshold (barriers among
@@ -432,13 +433,17 @@ block_max_kernel(HierArgs h, int cap_blk, int bias, int shift) {
 // abort flag the other warps see before their next wait.
 namespace tcs {
 constexpr int NT = 192;
-constexpr int ROWS = 128;         // rows per tile (MMA M)
+constexpr int ROWS = 128;         // rows per product (MMA M)
+constexpr int PROD = 4;           // products per tile
+constexpr int TROWS = PROD * ROWS;  // rows per tile (stage)
+constexpr int BOX = 256;          // rows per TMA load
 constexpr int DI = 128;           // indexer width: one 128-byte swizzle row
 constexpr int NQP = 16;           // MMA N (queries, padded)
-constexpr int TILE = ROWS * DI;   // 16 KB
-constexpr int MAX_STAGES = 12;
-constexpr int NACC = 4;
-constexpr uint32_t TMEM_COLS = 64;  // NACC accumulators of 16 columns
+constexpr int HALF = ROWS * DI;   // 16 KB
+constexpr int TILE = TROWS * DI;  // 32 KB
+constexpr int MAX_STAGES = 6;
+constexpr int NPAIR = 2;
+constexpr uint32_t TMEM_COLS = NPAIR * PROD * 16;  // NPAIR sets of PROD accumulators of 16 columns
 constexpr uint32_t kEpiBar = 1;     // named barrier of the epilogue warps
 // D s32 (2 << 4), A and B s8 (1 << 7, 1 << 10), both K-major, N = 16, M = 128
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NQP >> 3) << 17) |
@@ -479,17 +484,20 @@ __device__ __forceinline__ bool epi_all(bool v) {
         : "memory");
     return r != 0;
 }
-// The tile's rows: 128 rows of the key tensor from (0, y) by TMA, 128-byte
+// The tile's rows: 256 rows of the key tensor from (0, y) by TMA, 128-byte
 // swizzle, L2 evict-first (read once).
 __device__ __forceinline__ void tma_rows(uint32_t dst, const CUtensorMap* map, int y, uint32_t bar) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar),
                  "r"((uint32_t)TILE)
                  : "memory");
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(bar), "l"(evict_first_policy())
-        : "memory");
+    const uint64_t pol = evict_first_policy();
+#pragma unroll
+    for (int k = 0; k < TROWS / BOX; ++k)
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(dst + k * BOX * DI),
+            "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y + k * BOX), "r"(bar), "l"(pol)
+            : "memory");
 }
 // Threshold bin of a histogram in shared memory by the 128 epilogue threads
 // (thread e covers bins [kBins - 16 (e + 1), kBins - 16 e)); as find_threshold.
@@ -523,7 +531,7 @@ __device__ __forceinline__ void epi_threshold(const int* s_hist, int K, int* t_o
     }
     named_sync();
 }
-// A tile: rows [row, min(row + ROWS, end)) of sequence b, walked over this
+// A tile: rows [row, min(row + TROWS, end)) of sequence b, walked over this
 // CTA's slice of the batch laid end to end; `seq` counts the sequences entered.
 struct Tile {
     int b, row, end, seq;
@@ -538,7 +546,7 @@ __device__ __forceinline__ bool tile_first(const TopkArgs& a, long long lo, long
     return true;
 }
 __device__ __forceinline__ bool tile_next(const TopkArgs& a, long long lo, long long hi, Tile& t) {
-    t.row += min(ROWS, t.end - t.row);
+    t.row += min(TROWS, t.end - t.row);
     if (t.row < t.end) return true;
     ScanCursor c;
     if (!cursor_seek(a, lo, hi, c, t.b + 1)) return false;
@@ -562,7 +570,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
     unsigned char* sm = tsm + (((base0 + 1023u) & ~1023u) - base0);
     const uint32_t sA = smem_addr(sm), sB = sA + stages * TILE;
     int* hist = reinterpret_cast<int*>(sm + (size_t)stages * TILE + 2048);
-    __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], done[NACC], read[NACC];
+    __shared__ __align__(8) uint64_t full[MAX_STAGES], empty[MAX_STAGES], done[NPAIR], read[NPAIR];
     __shared__ uint32_t tmem_slot;
     __shared__ int sh_warp[4];
     __shared__ int s_last, s_t, s_above;
@@ -577,7 +585,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&full[s])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&empty[s])));
         }
-        for (int s = 0; s < NACC; ++s) {
+        for (int s = 0; s < NPAIR; ++s) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(&done[s])));
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 4;\n" ::"r"(smem_addr(&read[s])));
         }
@@ -611,12 +619,12 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
     if (warp == 4) {
         // ---- loads (each decision is the warp's: lanes agree by vote)
         Tile t = t0;
+        int s = 0;
+        uint32_t ph = 1;  // lap L of the ring waits for empty phase L - 1 (parity flips per lap)
         for (int i = 0;; ++i) {
-            const int s = i % stages;
             if (i >= stages) {
                 if (__any_sync(0xffffffffu, s_abort != 0)) break;
-                const bool got = bar_wait(smem_addr(&empty[s]), (uint32_t)(i / stages - 1) & 1u,
-                                          a.wait_ns);
+                const bool got = bar_wait(smem_addr(&empty[s]), ph, a.wait_ns);
                 if (!__all_sync(0xffffffffu, got)) {
                     if (lane == 0) give_up();
                     break;
@@ -626,21 +634,26 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
                 tma_rows(sA + s * TILE, &tm_k, (int)((long long)t.b * a.idx_capacity + t.row),
                          smem_addr(&full[s]));
             issued = i + 1;
+            if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+            }
             if (!tile_next(a, lo, hi, t)) break;
         }
     } else if (warp == 5) {
         // ---- products
         Tile t = t0;
-        int built = -1, i = 0;
+        int built = -1, i = 0, s = 0;
+        uint32_t fph = 0;  // parity of the full phase of stage s
         for (;; ++i) {
-            const int s = i % stages, c = i % NACC;
+            const int c = i & (NPAIR - 1);
             if (built != t.seq) {
                 // this sequence's queries, zero-padded, into B once every
                 // earlier product (in issue order) is done
                 if (i > 0) {
                     const int pi = i - 1;
-                    const bool got = bar_wait(smem_addr(&done[pi % NACC]),
-                                              (uint32_t)(pi / NACC) & 1u, a.wait_ns);
+                    const bool got = bar_wait(smem_addr(&done[pi & (NPAIR - 1)]),
+                                              (uint32_t)(pi / NPAIR) & 1u, a.wait_ns);
                     if (!__all_sync(0xffffffffu, got)) {
                         if (lane == 0) give_up();
                         break;
@@ -659,23 +672,30 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
                 __syncwarp();
             }
             if (__any_sync(0xffffffffu, s_abort != 0)) break;
-            bool got = bar_wait(smem_addr(&full[s]), (uint32_t)(i / stages) & 1u, a.wait_ns);
-            if (got && i >= NACC)  // accumulator c: its last tile's scores have been read
-                got = bar_wait(smem_addr(&read[c]), (uint32_t)(i / NACC - 1) & 1u, a.wait_ns);
+            bool got = bar_wait(smem_addr(&full[s]), fph, a.wait_ns);
+            if (got && i >= NPAIR)  // pair c: its last tile's scores have been read
+                got = bar_wait(smem_addr(&read[c]), (uint32_t)(i / NPAIR - 1) & 1u, a.wait_ns);
             if (!__all_sync(0xffffffffu, got)) {
                 if (lane == 0) give_up();
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
             if (lane == 0) {
+                const uint64_t da = sdesc(sA + s * TILE), db = sdesc(sB);
 #pragma unroll
-                for (int ks = 0; ks < DI / 32; ++ks)
-                    mma_i8(tmem + (uint32_t)c * NQP, sdesc(sA + s * TILE + ks * 32),
-                           sdesc(sB + ks * 32), ks > 0 ? 1u : 0u);
+                for (int h = 0; h < PROD; ++h)
+#pragma unroll
+                    for (int ks = 0; ks < DI / 32; ++ks)  // (descriptor address field: bytes >> 4)
+                        mma_i8(tmem + (uint32_t)(PROD * c + h) * NQP,
+                               da + (h * HALF + ks * 32) / 16, db + ks * 2, ks > 0 ? 1u : 0u);
                 commit(smem_addr(&empty[s]));
                 commit(smem_addr(&done[c]));
             }
             __syncwarp();
+            if (++s == stages) {
+                s = 0;
+                fph ^= 1u;
+            }
             if (!tile_next(a, lo, hi, t)) {
                 ++i;
                 break;
@@ -683,7 +703,7 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
         }
         // the products issued are done before the tensor memory is freed
         if (lane == 0 && i > 0)
-            bar_wait(smem_addr(&done[(i - 1) % NACC]), (uint32_t)((i - 1) / NACC) & 1u,
+            bar_wait(smem_addr(&done[(i - 1) & (NPAIR - 1)]), (uint32_t)((i - 1) / NPAIR) & 1u,
                      kCleanupWaitNs);
         __syncwarp();
     } else {
@@ -691,35 +711,40 @@ index_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_k, BatchTopkArgs ba,
         const int e = tid, row = warp * 32 + lane;
         Tile t = t0;
         for (int i = 0;; ++i) {
-            const int c = i % NACC;
+            const int c = i & (NPAIR - 1);
             // the four warps decide together (they meet at barriers below)
             const bool got = !s_abort && bar_wait(smem_addr(&done[c]),
-                                                  (uint32_t)(i / NACC) & 1u, a.wait_ns);
+                                                  (uint32_t)(i / NPAIR) & 1u, a.wait_ns);
             if (!epi_all(got)) {
                 if (e == 0 && !s_abort) give_up();
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-            uint32_t r[8];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
-                         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                           "=r"(r[6]), "=r"(r[7])
-                         : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c * NQP));
+            uint32_t r[PROD][8];
+#pragma unroll
+            for (int h = 0; h < PROD; ++h)
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                    : "=r"(r[h][0]), "=r"(r[h][1]), "=r"(r[h][2]), "=r"(r[h][3]), "=r"(r[h][4]),
+                      "=r"(r[h][5]), "=r"(r[h][6]), "=r"(r[h][7])
+                    : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(PROD * c + h) * NQP));
             asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
             asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
             __syncwarp();
-            if (lane == 0) arrive(smem_addr(&read[c]));  // the accumulator is free
-            const int nrows = min(ROWS, t.end - t.row);
-            if (row < nrows) {
-                const size_t at = (size_t)t.b * cap + t.row + row;
+            if (lane == 0) arrive(smem_addr(&read[c]));  // the accumulator pair is free
+            const int nrows = min(TROWS, t.end - t.row);
 #pragma unroll
-                for (int q = 0; q < kMaxBatchQ; ++q)
-                    if (q < nq) {
-                        const int v = (int)r[q];
-                        ba.q[q].scores[at] = v;
-                        atomicAdd(&hist[q * kBins + score_bin(v, bias, shift)], 1);
-                    }
-            }
+            for (int h = 0; h < PROD; ++h)
+                if (h * ROWS + row < nrows) {
+                    const size_t at = (size_t)t.b * cap + t.row + h * ROWS + row;
+#pragma unroll
+                    for (int q = 0; q < kMaxBatchQ; ++q)
+                        if (q < nq) {
+                            const int v = (int)r[h][q];
+                            ba.q[q].scores[at] = v;
+                            atomicAdd(&hist[q * kBins + score_bin(v, bias, shift)], 1);
+                        }
+                }
             if (t.row + nrows >= t.end) {
                 // ---- sequence t.b done in this CTA: flush, maybe derive thresholds
                 named_sync();  // every count of the sequence is in the histograms
@@ -837,7 +862,7 @@ cudaError_t launch_block_pool(const HierArgs& h, cudaStream_t s) {
 }
 
 // 2-D u8 tensor [rows][128] of indexer key rows (row stride 128 B), boxes of
-// 128 x 128 bytes, 128-byte swizzle, zero fill past the end.
+// 256 rows x 128 bytes, 128-byte swizzle, zero fill past the end.
 static bool encode_key_rows(CUtensorMap* m, const void* base, unsigned long long rows) {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -852,7 +877,7 @@ static bool encode_key_rows(CUtensorMap* m, const void* base, unsigned long long
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)tcs::DI, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)tcs::DI};
-    const cuuint32_t box[2] = {(cuuint32_t)tcs::DI, (cuuint32_t)tcs::ROWS};
+    const cuuint32_t box[2] = {(cuuint32_t)tcs::DI, (cuuint32_t)tcs::BOX};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -887,8 +912,8 @@ cudaError_t launch_index_topk_batched(const BatchTopkArgs& ba0, cudaStream_t s) 
     const long long rows = (long long)a.batch * a.capacity;
     int ctas = sms;
     long long per = (rows + ctas - 1) / ctas;
-    per = (per + tcs::ROWS - 1) / tcs::ROWS * tcs::ROWS;
-    if (per < tcs::ROWS) per = tcs::ROWS;
+    per = (per + tcs::TROWS - 1) / tcs::TROWS * tcs::TROWS;
+    if (per < tcs::TROWS) per = tcs::TROWS;
     ctas = (int)((rows + per - 1) / per);
     if (rows > 0) {
         CUtensorMap tm;
