@@ -83,3 +83,37 @@ def test_batched_stack1m_scoring_layers(kvc):
     want = _oracle(w, inp["idx_k"], idx_q, [w.entries], w.entries)
     for q in range(len(heads)):
         topk_set_equal(tk[q], want[q])
+
+
+def test_batched_zero_wait_limit_times_out_then_recovers(kvc):
+    """Under a zero wait limit the pipeline's waits (tile landed, products
+    done, stage and accumulators released) give up at once: KVC_DEV_TIMEOUT,
+    a normal return with every warp out of the pipeline and the loads in
+    flight landed; after zeroing the workspace the next call is exact."""
+    w = synth.WORKLOADS["csa2group"].scaled(batch=3, context=2 * 20000)
+    g = torch.Generator().manual_seed(77)
+    idx_k = torch.randint(-127, 128, (3, 20000, 128), generator=g, dtype=torch.int8)
+    idx_q = torch.randint(-127, 128, (2, 3, 128), generator=g, dtype=torch.int8)
+    n = [20000, 11111, 600]
+    cfg = kvc.config_for(w)
+    cache = kvc.Cache(cfg, 3, 20000)
+    cache.idx_k.copy_(idx_k.cuda())
+    cache.n_entries.copy_(torch.as_tensor(n, dtype=torch.int32))
+    tk = torch.empty(2, 3, w.topk, dtype=torch.int32, device="cuda")
+    ws = kvc.workspace_batched(cfg, 2, 3, 20000)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvc.debug_set_wait_limit_ns(0)
+    try:
+        kvc.index_topk_batched(cfg, idx_q.cuda().contiguous(), cache, tk, ws, status=st)
+        torch.cuda.synchronize()
+    finally:
+        kvc.debug_set_wait_limit_ns(2_000_000_000)
+    assert int(st.item()) & 0x8, int(st.item())  # KVC_DEV_TIMEOUT
+    ws.zero_()
+    st.zero_()
+    kvc.index_topk_batched(cfg, idx_q.cuda().contiguous(), cache, tk, ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    want = _oracle(w, idx_k, idx_q, n, 20000)
+    for q in range(2):
+        topk_set_equal(tk.cpu().numpy()[q], want[q])
