@@ -846,16 +846,26 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float* rows = reinterpret_cast<const float*>(smem + OFF_K);
         for (int it2 = tid; it2 < nh * (DV / 4); it2 += NT) {
             const int hh = it2 / (DV / 4), q4 = it2 - hh * (DV / 4);
+            // every split's weight and row loaded at once (a cluster holds at
+            // most 8 CTAs); a split with weight 0 pushed no row: its value is
+            // selected away, never multiplied
+            float w[8];
+            float4 v[8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+                if (s2 < nsplit) {
+                    w[s2] = wts[hh * nsplit + s2];
+                    v[s2] = reinterpret_cast<const float4*>(rows + (s2 * nh + hh) * DV)[q4];
+                }
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s2 = 0; s2 < nsplit; ++s2) {
-                const float w = wts[hh * nsplit + s2];
-                if (w == 0.f) continue;
-                const float4 v = reinterpret_cast<const float4*>(rows + (s2 * nh + hh) * DV)[q4];
-                acc.x = fmaf(w, v.x, acc.x);
-                acc.y = fmaf(w, v.y, acc.y);
-                acc.z = fmaf(w, v.z, acc.z);
-                acc.w = fmaf(w, v.w, acc.w);
-            }
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+                if (s2 < nsplit && w[s2] != 0.f) {
+                    acc.x = fmaf(w[s2], v[s2].x, acc.x);
+                    acc.y = fmaf(w[s2], v[s2].y, acc.y);
+                    acc.z = fmaf(w[s2], v[s2].z, acc.z);
+                    acc.w = fmaf(w[s2], v[s2].w, acc.w);
+                }
             const float inv = fac[hh];
             *reinterpret_cast<float4*>(a.out + ((size_t)b * H + hg0 + h_lo + hh) * DV + 4 * q4) =
                 make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
