@@ -813,30 +813,45 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int t = 0; t < 2; ++t) {
                 const int mt = (warp >> 2) * 2 + t;
                 const uint32_t d4 = (mt * 128 + g * 32 + lane) * 4;
-                for (int h0 = 0; h0 < HG; h0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt + h0, r);
-                    tmem_wait_ld();
+                // both 32-head blocks of the tile loaded before one wait (HG <= 64)
+                uint32_t r[2][32];
+                const uint32_t ta = tmem + ((uint32_t)(g * 32) << 16) + O_COL + 64 * mt;
+                tmem_ld32(ta, r[0]);
+                if (HG > 32) tmem_ld32(ta + 32, r[1]);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (h0 + i < HG)
-                            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dst_off[h0 + i] + d4),
-                                         "r"(r[i])
-                                         : "memory");
-                }
+                for (int hb = 0; hb < 2; ++hb)
+                    if (hb * 32 < HG) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (hb * 32 + i < HG)
+                                asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(
+                                                 dst_off[hb * 32 + i] + d4),
+                                             "r"(r[hb][i])
+                                             : "memory");
+                    }
             }
         }
         cluster_sync();  // every row and (m, l) has arrived
         if (tid < nh) {
+            // every split's (m, l) loaded at once (at most 8 splits)
+            float2 ml[8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+                if (s2 < nsplit) ml[s2] = reinterpret_cast<const float2*>(mlx)[s2 * nh + tid];
             float M = -INFINITY;
-            for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, mlx[(s2 * nh + tid) * 2]);
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+                if (s2 < nsplit) M = fmaxf(M, ml[s2].x);
             float L = 0.f;
-            for (int s2 = 0; s2 < nsplit; ++s2) {
-                const float m = mlx[(s2 * nh + tid) * 2], l = mlx[(s2 * nh + tid) * 2 + 1];
-                const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : ex2(m - M);
-                wts[tid * nsplit + s2] = w;
-                L += w * l;
-            }
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+                if (s2 < nsplit) {
+                    const float m = ml[s2].x, l = ml[s2].y;
+                    const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : ex2(m - M);
+                    wts[tid * nsplit + s2] = w;
+                    L += w * l;
+                }
             fac[tid] = L > 0.f ? 1.f / L : 0.f;
             if (a.lse)
                 a.lse[(size_t)b * H + hg0 + h_lo + tid] =
@@ -844,6 +859,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         __syncthreads();
         const float* rows = reinterpret_cast<const float*>(smem + OFF_K);
+#pragma unroll 2
         for (int it2 = tid; it2 < nh * (DV / 4); it2 += NT) {
             const int hh = it2 / (DV / 4), q4 = it2 - hh * (DV / 4);
             // every split's weight and row loaded at once (a cluster holds at
