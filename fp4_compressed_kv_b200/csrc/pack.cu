@@ -30,6 +30,7 @@
 // form, exact power-of-two scaling), so every implementation of this order
 // produces the same fp32 entry and therefore the same codes.
 #include "kvc_internal.cuh"
+#include "tc05_common.cuh"
 
 namespace kvc {
 namespace {
@@ -420,6 +421,112 @@ pack_kernel(PackArgs a, Shape sh, int ue4m3, int di) {
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
 
+// One chunk of the gate logit difference, in the fixed order: for channels
+// 2k, 2k + 1 of the chunk, d = k0 - k1 (an fp32 pair subtraction), then one
+// fmaf per channel into the lane's running sum.
+template <typename T>
+__device__ __forceinline__ float gate_chunk(float acc, const Chunk<T>& x0, const Chunk<T>& x1,
+                                            const float (&g)[8]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint64_t d = f2_sub(x0.pair(k), x1.pair(k));
+        acc = __fmaf_rn(g[2 * k], f2_lo(d), acc);
+        acc = __fmaf_rn(g[2 * k + 1], f2_hi(d), acc);
+    }
+    return acc;
+}
+
+// The pair weights from the team's eight running sums (xor tree over 4, 2, 1).
+__device__ __forceinline__ void gate_weights(float acc, uint64_t& W0, uint64_t& W1) {
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
+    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
+    const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-acc)));
+    const float w1 = __fsub_rn(1.0f, w0);
+    W0 = f2_make(w0, w0);
+    W1 = f2_make(w1, w1);
+}
+
+// Pass 2 of one chunk step (chunk c of the lane's entry): the entry values
+// v = w0 k0 + w1 k1, the group maximum across the LPG lanes holding the
+// group's chunks, the scale and the eight codes.  Every lane of the warp
+// calls it (the maximum is a warp shuffle); only `active` lanes store: the
+// code word into the record, the scale (the group's first lane) into the
+// team's tail.  Inactive lanes must pass zero chunks.
+template <typename T, int LPG>
+__device__ __forceinline__ void quantise_chunk(const Chunk<T>& x0, const Chunk<T>& x1,
+                                               uint64_t W0, uint64_t W1, bool active, int c,
+                                               int ue4m3, const float* tab_s, const float* tab_rl,
+                                               const float* tab_rh, uint8_t* rec, uint8_t* tail,
+                                               bool& bad) {
+    uint64_t v[4];  // v = w0 k0 + w1 k1, rounded as fmaf(w0, k0, w1 * k1)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = f2_fma(W0, x0.pair(k), f2_mul(W1, x1.pair(k)));
+    // the chunk's largest magnitude (a tree of pairwise maxima), then the group's
+    float m = absmax_nan(absmax_nan(absmax_nan(f2_lo(v[0]), f2_hi(v[0])),
+                                    absmax_nan(f2_lo(v[1]), f2_hi(v[1]))),
+                         absmax_nan(absmax_nan(f2_lo(v[2]), f2_hi(v[2])),
+                                    absmax_nan(f2_lo(v[3]), f2_hi(v[3]))));
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
+    m = fabsf(m);
+    if (__any_sync(0xffffffffu, !(m <= 3.0e38f))) {
+        // a NaN or inf somewhere in the warp: value by value, non-finite
+        // values coded as 0 (and reported)
+        m = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float lo = f2_lo(v[k]), hi = f2_hi(v[k]);
+            if (!isfinite(lo)) {
+                if (active) bad = true;
+                lo = 0.f;
+            }
+            if (!isfinite(hi)) {
+                if (active) bad = true;
+                hi = 0.f;
+            }
+            v[k] = f2_make(lo, hi);
+            m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+        }
+#pragma unroll
+        for (int o = 1; o < LPG; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    if (!active) return;
+    const float sc = div6_rn(m);
+    uint32_t code, sbyte = 0;
+    if (ue4m3) {
+        sbyte = e4m3_from_f32(sc);
+        const float sv = tab_s[sbyte];
+        code = sv > 0.f ? e2m1x8_quotient_f2(v, sv, tab_rl[sbyte], tab_rh[sbyte]) : 0u;
+    } else {
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            x[2 * k] = f2_lo(v[k]);
+            x[2 * k + 1] = f2_hi(v[k]);
+        }
+        code = sc > 0.f ? e2m1x8_quotient(x, sc) : 0u;
+    }
+    *reinterpret_cast<uint32_t*>(rec + 4 * c) = code;
+    if ((c & (LPG - 1)) == 0) {
+        const int gi = c / LPG;
+        if (ue4m3)
+            tail[gi] = (uint8_t)sbyte;
+        else
+            *reinterpret_cast<float*>(tail + 4 * gi) = sc;
+    }
+}
+
+// Reciprocal brackets of the 128 UE4M3 scale values (entry i: scale byte i).
+__device__ __forceinline__ void fill_scale_tables(float* tab_s, float* tab_rl, float* tab_rh,
+                                                  int i) {
+    const float sv = e4m3_to_f32(i);
+    const float r = __frcp_rn(sv);
+    tab_s[i] = sv;
+    tab_rl[i] = __fmul_rn(r, 1.0f - 0x1p-20f);
+    tab_rh[i] = __fmul_rn(r, 1.0f + 0x1p-20f);
+}
+
 // Streaming form of pack_kernel for groups of at most 64 channels (LPG <= 8
 // chunks per group, so a group's chunks sit in the team's lanes at the same
 // chunk step): the same arithmetic in the same order, but no token chunk is
@@ -449,13 +556,7 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
     const int D = sh.D, nchunk = D >> 3;
     uint8_t* tail = dsm + team * tail_stride;
     const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
-    if (ue4m3 && tid < 128) {
-        const float sv = e4m3_to_f32(tid);
-        const float r = __frcp_rn(sv);
-        tab_s[tid] = sv;
-        tab_rl[tid] = __fmul_rn(r, 1.0f - 0x1p-20f);
-        tab_rh[tid] = __fmul_rn(r, 1.0f + 0x1p-20f);
-    }
+    if (ue4m3 && tid < 128) fill_scale_tables(tab_s, tab_rl, tab_rh, tid);
     for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
     __syncthreads();
     pdl_wait();
@@ -481,20 +582,11 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
             x1.load_keep(k1p + 8 * c);
             float g[8];
             load8_gate(a.gate + 8 * c, g);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t d = f2_sub(x0.pair(k), x1.pair(k));
-                acc = __fmaf_rn(g[2 * k], f2_lo(d), acc);
-                acc = __fmaf_rn(g[2 * k + 1], f2_hi(d), acc);
-            }
+            acc = gate_chunk(acc, x0, x1, g);
         }
     }
-    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 4));
-    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
-    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
-    const float w0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cody_waite(-acc)));
-    const float w1 = __fsub_rn(1.0f, w0);
-    const uint64_t W0 = f2_make(w0, w0), W1 = f2_make(w1, w1);
+    uint64_t W0, W1;
+    gate_weights(acc, W0, W1);
     uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
 
     // pass 2: entry values, group maxima (xor over the group's lanes), codes
@@ -511,62 +603,8 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
             x0.zero();
             x1.zero();
         }
-        uint64_t v[4];  // v = w0 k0 + w1 k1, rounded as fmaf(w0, k0, w1 * k1)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = f2_fma(W0, x0.pair(k), f2_mul(W1, x1.pair(k)));
-        // the chunk's largest magnitude (a tree of pairwise maxima), then the group's
-        float m = absmax_nan(absmax_nan(absmax_nan(f2_lo(v[0]), f2_hi(v[0])),
-                                        absmax_nan(f2_lo(v[1]), f2_hi(v[1]))),
-                             absmax_nan(absmax_nan(f2_lo(v[2]), f2_hi(v[2])),
-                                        absmax_nan(f2_lo(v[3]), f2_hi(v[3]))));
-#pragma unroll
-        for (int o = 1; o < LPG; o <<= 1) m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
-        m = fabsf(m);
-        if (__any_sync(0xffffffffu, !(m <= 3.0e38f))) {
-            // a NaN or inf somewhere in the warp: value by value, non-finite
-            // values coded as 0 (and reported)
-            m = 0.f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float lo = f2_lo(v[k]), hi = f2_hi(v[k]);
-                if (!isfinite(lo)) {
-                    if (active) bad = true;
-                    lo = 0.f;
-                }
-                if (!isfinite(hi)) {
-                    if (active) bad = true;
-                    hi = 0.f;
-                }
-                v[k] = f2_make(lo, hi);
-                m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
-            }
-#pragma unroll
-            for (int o = 1; o < LPG; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        }
-        if (!active) continue;
-        const float sc = div6_rn(m);
-        uint32_t code, sbyte = 0;
-        if (ue4m3) {
-            sbyte = e4m3_from_f32(sc);
-            const float sv = tab_s[sbyte];
-            code = sv > 0.f ? e2m1x8_quotient_f2(v, sv, tab_rl[sbyte], tab_rh[sbyte]) : 0u;
-        } else {
-            float x[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                x[2 * k] = f2_lo(v[k]);
-                x[2 * k + 1] = f2_hi(v[k]);
-            }
-            code = sc > 0.f ? e2m1x8_quotient(x, sc) : 0u;
-        }
-        *reinterpret_cast<uint32_t*>(rec + 4 * c) = code;
-        if ((c & (LPG - 1)) == 0) {
-            const int gi = c / LPG;
-            if (ue4m3)
-                tail[gi] = (uint8_t)sbyte;
-            else
-                *reinterpret_cast<float*>(tail + 4 * gi) = sc;
-        }
+        quantise_chunk<T, LPG>(x0, x1, W0, W1, active, c, ue4m3, tab_s, tab_rl, tab_rh, rec,
+                               tail, bad);
     }
     __syncwarp();
     if (valid) {
@@ -577,6 +615,203 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
             reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di);
         uint4* dst = reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di);
         for (int p = l; p < (di >> 4); p += 8) dst[p] = __ldcs(src + p);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
+}
+
+// Ring form of the streaming kernel for long appends of bf16 tokens (groups
+// of at most 64 channels): the same arithmetic in the same order, fed from
+// shared memory instead of L1/L2.  One persistent CTA per SM walks units of
+// kRingE consecutive entries of one sequence (unit u of the grid-stride
+// sequence u = blockIdx.x + k gridDim.x); a unit's token pairs are contiguous
+// in the token array, so one producer thread moves each unit with a single
+// bulk copy into a ring of shared-memory stages.  kRingGroups groups of
+// kRingE / 4 consumer warps take the units in turn (group k mod kRingGroups,
+// stage k mod stages), read every chunk twice from the stage -- the gate
+// pass and the quantisation pass -- and hand the stage back on its `empty`
+// barrier.  The second read of each chunk no longer goes out to L1/L2 (the
+// streaming kernel's latency).  The kernel is bound by instruction issue, so
+// the shared memory goes to the warps: at 576 channels the 12 stages of
+// 18 KB hold 11 groups' units (22 consumer warps) and one unit in flight;
+// measured on 32 x 4096 new tokens, 16 entries per unit in 4 groups (two
+// units in flight) took 56 us, 8 in 10 groups 54 us, 8 in 11 groups 51.6 us
+// (the streaming kernel 61.6 us).  Waits are bounded: a consumer or the
+// producer that gives up sets KVC_DEV_TIMEOUT and stops; the producer always
+// waits (up to 2 s) for its copies in flight before the CTA exits.
+constexpr int kRingE = 8;        // entries per unit (and per stage): 2 warps of 4 teams
+constexpr int kRingGroups = 11;  // consumer groups of kRingE / 4 warps (22 warps)
+constexpr int kRingConsumerWarps = kRingGroups * kRingE / 4;
+constexpr int kRingThreads = (kRingConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kRingMaxStages = 32;
+constexpr unsigned long long kRingDrainNs = 2000000000ull;
+
+__device__ __forceinline__ void ring_bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1], %2, [%3], %4;\n" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ void ring_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
+template <int MAXJ, int LPG>
+__global__ void __launch_bounds__(kRingThreads, 1)
+pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int stages,
+                 uint32_t stage_bytes, long long n_units, unsigned long long wait_ns) {
+    using T = __nv_bfloat16;
+    extern __shared__ __align__(128) uint8_t rsm[];  // stages | gate | team tails
+    __shared__ float tab_s[128], tab_rl[128], tab_rh[128];
+    __shared__ __align__(8) uint64_t full[kRingMaxStages], empty[kRingMaxStages];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int D = sh.D, nchunk = D >> 3, half = a.n_new >> 1;
+    const int units_per_seq = (half + kRingE - 1) / kRingE;
+    const uint32_t ring = tc::smem_u32(rsm);
+    float* gate_s = reinterpret_cast<float*>(rsm + (size_t)stages * stage_bytes);
+    uint8_t* tails = rsm + (size_t)stages * stage_bytes + (size_t)D * 4;
+    const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
+
+    if (ue4m3 && tid < 128) fill_scale_tables(tab_s, tab_rl, tab_rh, tid);
+    if (tid == 0) {
+        for (int st = 0; st < stages; ++st) {
+            tc::mbar_init(tc::smem_u32(&full[st]), 1);
+            tc::mbar_init(tc::smem_u32(&empty[st]), kRingE / 4);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    for (int t = tid * 4; t < kRingConsumerWarps * 4 * tail_stride; t += kRingThreads * 4)
+        *reinterpret_cast<uint32_t*>(tails + t) = 0u;
+    pdl_wait();
+    for (int t = tid; t < D / 4; t += kRingThreads)
+        reinterpret_cast<float4*>(gate_s)[t] = __ldg(reinterpret_cast<const float4*>(a.gate) + t);
+    __syncthreads();
+
+    if (warp == kRingConsumerWarps) {  // the producer
+        if (lane != 0) return;
+        const T* tokens = static_cast<const T*>(a.tokens);
+        long long k = 0;
+        for (;; ++k) {
+            const long long u = blockIdx.x + k * gridDim.x;
+            if (u >= n_units) break;
+            const int st = (int)(k % stages);
+            if (k >= stages &&
+                !tc::mbar_wait(tc::smem_u32(&empty[st]), (uint32_t)((k / stages - 1) & 1),
+                               wait_ns)) {
+                set_status(a.status, KVC_DEV_TIMEOUT);
+                break;
+            }
+            const int b = (int)(u / units_per_seq), e0 = (int)(u % units_per_seq) * kRingE;
+            const int ne = min(kRingE, half - e0);
+            ring_bulk_load(ring + (uint32_t)st * stage_bytes,
+                           tokens + ((long long)b * a.n_new + 2 * e0) * D,
+                           (uint32_t)(ne * 2 * D * (int)sizeof(T)), tc::smem_u32(&full[st]));
+        }
+        // copies still in flight must land before the CTA exits
+        for (long long j = k > stages ? k - stages : 0; j < k; ++j)
+            tc::mbar_wait(tc::smem_u32(&full[j % stages]), (uint32_t)((j / stages) & 1),
+                          kRingDrainNs);
+        return;
+    }
+
+    // consumers: warp wi of group grp; team `team` of the warp takes entry
+    // 4 wi + team of each of the group's units
+    const int grp = warp / (kRingE / 4), wi = warp % (kRingE / 4);
+    const int team = lane >> 3, l = lane & 7;
+    uint8_t* tail = tails + (warp * 4 + team) * tail_stride;
+    const int ei = wi * 4 + team;  // entry within the unit
+    bool bad = false;
+    for (long long k = grp;; k += kRingGroups) {
+        const long long u = blockIdx.x + k * gridDim.x;
+        if (u >= n_units) break;
+        const int st = (int)(k % stages);
+        const bool got = __all_sync(
+            0xffffffffu,
+            tc::mbar_wait(tc::smem_u32(&full[st]), (uint32_t)((k / stages) & 1), wait_ns));
+        if (!got) {
+            if (lane == 0) set_status(a.status, KVC_DEV_TIMEOUT);
+            break;
+        }
+        const int b = (int)(u / units_per_seq), e0 = (int)(u % units_per_seq) * kRingE;
+        const int ne = min(kRingE, half - e0);
+        const bool here = ei < ne;  // this team has an entry in the unit
+        const int i = e0 + ei;
+        // the sequence's length is first needed for the stores of pass 2: its
+        // load and the indexer key's are in flight during pass 1
+        const int base = a.n_entries[b];
+        uint4 ik[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        const uint4* isrc =
+            reinterpret_cast<const uint4*>(a.idx_k_new + ((long long)b * half + i) * di);
+        if (here) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                if (l + 8 * r < (di >> 4)) ik[r] = __ldcs(isrc + l + 8 * r);
+        }
+        const T* k0s = reinterpret_cast<const T*>(rsm + (size_t)st * stage_bytes) +
+                       (size_t)ei * 2 * D;
+        const T* k1s = k0s + D;
+        const int jn = here ? (nchunk - l + 7) / 8 : 0;  // chunks of this lane
+
+        // pass 1: gate logit difference, fixed order (lane l: chunks l, l+8, ...)
+        float acc = 0.f;
+#pragma unroll 3
+        for (int j = 0; j < MAXJ; ++j) {
+            const int c = l + 8 * j;
+            if (j < jn) {
+                Chunk<T> x0, x1;
+                x0.load_shared(k0s + 8 * c);
+                x1.load_shared(k1s + 8 * c);
+                float g[8];
+                const float4 ga = reinterpret_cast<const float4*>(gate_s + 8 * c)[0];
+                const float4 gb = reinterpret_cast<const float4*>(gate_s + 8 * c)[1];
+                g[0] = ga.x; g[1] = ga.y; g[2] = ga.z; g[3] = ga.w;
+                g[4] = gb.x; g[5] = gb.y; g[6] = gb.z; g[7] = gb.w;
+                acc = gate_chunk(acc, x0, x1, g);
+            }
+        }
+        uint64_t W0, W1;
+        gate_weights(acc, W0, W1);
+        const bool seq_ok = base >= 0 && base + half <= a.capacity;
+        if (!seq_ok && e0 == 0 && wi == 0 && lane == 0) set_status(a.status, KVC_DEV_CAPACITY);
+        const bool valid = seq_ok && here;
+        const long long pos = (long long)base + i;
+        uint8_t* rec = a.records + ((long long)b * a.capacity + pos) * sh.rb;
+
+        // pass 2: entry values, group maxima, codes (stored by valid teams)
+#pragma unroll 2
+        for (int j = 0; j < MAXJ; ++j) {
+            const int c = l + 8 * j;
+            const bool active = valid && j < jn;
+            Chunk<T> x0, x1;
+            if (j < jn) {
+                x0.load_shared(k0s + 8 * c);
+                x1.load_shared(k1s + 8 * c);
+            } else {
+                x0.zero();
+                x1.zero();
+            }
+            quantise_chunk<T, LPG>(x0, x1, W0, W1, active, c, ue4m3, tab_s, tab_rl, tab_rh, rec,
+                                   tail, bad);
+        }
+        __syncwarp();
+        if (lane == 0) ring_arrive(tc::smem_u32(&empty[st]));  // the stage is read
+        if (valid) {
+            for (int t = l * 4; t < tail_len; t += 32)
+                *reinterpret_cast<uint32_t*>(rec + sh.code_bytes + t) =
+                    *reinterpret_cast<const uint32_t*>(tail + t);
+            uint4* dst =
+                reinterpret_cast<uint4*>(a.idx_k + ((long long)b * a.capacity + pos) * di);
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                if (l + 8 * r < (di >> 4)) dst[l + 8 * r] = ik[r];
+        }
+        __syncwarp();  // the tail is read before the next unit writes it
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
@@ -943,6 +1178,69 @@ cudaError_t launch_stream_j(dim3 grid, cudaStream_t s, const PackArgs& a, const 
     }
 }
 
+// The ring kernel: one CTA per SM (fewer for short appends), as many stages
+// as fit beside the gate and the team tails (at least one more than the
+// consumer groups, else the streaming kernel runs).
+template <int MAXJ, int LPG>
+cudaError_t launch_ring(cudaStream_t s, const PackArgs& a, const Shape& sh, int ue4m3, int di,
+                        int stages, uint32_t stage_bytes, long long n_units, int sms,
+                        size_t smem) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        pack_ring_kernel<MAXJ, LPG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int tail_stride = ((sh.rb - sh.code_bytes) + 15) / 16 * 16;
+    const unsigned grid = (unsigned)(n_units < sms ? n_units : sms);
+    return launch_pdl(pack_ring_kernel<MAXJ, LPG>, grid, kRingThreads, smem, s, a, sh, ue4m3, di,
+                      tail_stride, stages, stage_bytes, n_units, device_wait_limit_ns());
+}
+
+// Ring plan for a bf16 append: stage count and dynamic shared memory, or
+// stages = 0 when the ring does not apply.
+struct RingPlan {
+    int stages = 0, sms = 0;
+    uint32_t stage_bytes = 0;
+    size_t smem = 0;
+};
+inline RingPlan ring_plan(const Shape& sh, const PackArgs& a, int di) {
+    RingPlan p;
+    const int D = sh.D;
+    if (D % 8 != 0 || D > 576 || D <= 128 || sh.lpg > 8 || di > 256 || di % 16 != 0) return p;
+    if (reinterpret_cast<uintptr_t>(a.tokens) % 16 != 0) return p;
+    int dev = 0, optin = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return p;
+    const int tail_stride = ((sh.rb - sh.code_bytes) + 15) / 16 * 16;
+    const size_t fixed = (size_t)D * 4 + (size_t)kRingConsumerWarps * 4 * tail_stride;
+    const uint32_t sb = (uint32_t)(kRingE * 2 * D * 2);
+    const long long room = (long long)optin - 2048 - (long long)fixed;  // static smem margin
+    int st = room > 0 ? (int)(room / sb) : 0;
+    if (st > kRingMaxStages) st = kRingMaxStages;
+    if (st < kRingGroups + 1) return p;
+    p.stages = st;
+    p.sms = sms;
+    p.stage_bytes = sb;
+    p.smem = fixed + (size_t)st * sb;
+    return p;
+}
+
+template <int MAXJ>
+cudaError_t launch_ring_j(cudaStream_t s, const PackArgs& a, const Shape& sh, int ue4m3, int di,
+                          const RingPlan& p, long long n_units) {
+    switch (sh.lpg) {
+        case 1: return launch_ring<MAXJ, 1>(s, a, sh, ue4m3, di, p.stages, p.stage_bytes, n_units,
+                                            p.sms, p.smem);
+        case 2: return launch_ring<MAXJ, 2>(s, a, sh, ue4m3, di, p.stages, p.stage_bytes, n_units,
+                                            p.sms, p.smem);
+        case 4: return launch_ring<MAXJ, 4>(s, a, sh, ue4m3, di, p.stages, p.stage_bytes, n_units,
+                                            p.sms, p.smem);
+        default: return launch_ring<MAXJ, 8>(s, a, sh, ue4m3, di, p.stages, p.stage_bytes,
+                                             n_units, p.sms, p.smem);
+    }
+}
+
 // 4:1 appends: a warp per entry at every size
 template <typename T>
 cudaError_t launch_pack4_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
@@ -989,6 +1287,17 @@ cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
     const unsigned grid = (unsigned)((entries + kTeams - 1) / kTeams);
     const int maxj = (sh.D / 8 + 7) / 8;
     trace_before("pack", s);
+    if (sh.lpg <= 8 && sizeof(T) == 2) {  // bf16 tokens: the ring kernel where it fits
+        const RingPlan p = ring_plan(sh, a, di);
+        if (p.stages > 0) {
+            const int half = a.n_new / 2;
+            const long long n_units = (long long)a.batch * ((half + kRingE - 1) / kRingE);
+            err = maxj <= 4 ? launch_ring_j<4>(s, a, sh, ue4m3, di, p, n_units)
+                            : launch_ring_j<9>(s, a, sh, ue4m3, di, p, n_units);
+            trace_after(s);
+            return err;
+        }
+    }
     if (sh.lpg <= 8) {  // groups within one chunk step: the streaming kernel
         const int half = a.n_new / 2;
         const dim3 g2((unsigned)((half + kTeams - 1) / kTeams), (unsigned)a.batch);

@@ -435,8 +435,8 @@ int orc_pack(const orc_cfg* c, int B, int n_new, const float* tokens,
 }
 
 /* ------------------------------------------------------------------ */
-/* Lightweight indexer ([P2] breakthrough 4 "用一个轻量索引器给所有历史
- * token 打分"): score_j = sum_d q_d k_{j,d}, int8 x int8 -> int32.       */
+/* Lightweight indexer ([P2] breakthrough 4: a small indexer scores every
+ * stored entry): score_j = sum_d q_d k_{j,d}, int8 x int8 -> int32.      */
 void orc_index_scores(const int8_t* q, const int8_t* keys, int n, int di,
                       int32_t* scores) {
     for (int j = 0; j < n; ++j) {

@@ -219,3 +219,51 @@ def test_pack_rounding_midpoints(kvc, name, pairs):
     got = cache.records.cpu().numpy()
     diff = np.argwhere(got != rec)
     assert diff.size == 0, f"{len(diff)} bytes differ, first {diff[:5].tolist()}"
+
+
+@pytest.mark.parametrize("group", [8, 16, 32, 64])
+def test_pack_ring_groups_ragged(kvc, group):
+    """Appends of more than 4096 bf16 entries run the ring kernel (units of 16
+    entries streamed through shared memory, one CTA per SM): every group width
+    it takes, four sequences whose appends are not a multiple of the unit, the
+    second append continuing a partly filled cache; byte for byte against the
+    oracle."""
+    w = synth.WORKLOADS["batch32x128k"].scaled(batch=4, context=2 * 2731, group=group)
+    inp = synth.make_inputs(w)
+    rec, ic, n, ost = oracle_pack(w, inp["tokens"], inp["gate"], inp["idx_k"])
+    assert ost == 0
+    cache, st = _gpu_pack(kvc, w, inp["tokens"].cuda(), inp["gate"].cuda(), inp["idx_k"].cuda(),
+                          chunks=2 * 1366)
+    assert st == 0
+    assert cache.n_entries.cpu().tolist() == n.tolist() == [2731] * 4
+    g = cache.records.cpu().numpy()
+    diff = np.argwhere(g != rec)
+    assert diff.size == 0, f"{len(diff)} bytes differ, first {diff[:5].tolist()}"
+    assert np.array_equal(cache.idx_k.cpu().numpy(), ic)
+
+
+def test_pack_ring_capacity(kvc):
+    """A long append that one sequence has no room for: that sequence is left
+    untouched and KVC_DEV_CAPACITY is set; the others are packed at their own
+    offsets exactly as the oracle packs them."""
+    w = synth.WORKLOADS["batch32x128k"].scaled(batch=3, context=2 * 2000)
+    inp = synth.make_inputs(w)
+    rec, ic, n, _ = oracle_pack(w, inp["tokens"], inp["gate"], inp["idx_k"])
+    cfg = kvc.config_for(w)
+    cache = kvc.Cache(cfg, 3, 2100)
+    grec = Guarded(cache.records.shape, cache.records.dtype, fill=0)
+    cache.records = grec.t
+    cache.n_entries.copy_(torch.tensor([0, 200, 50], dtype=torch.int32))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvc.pack(cfg, inp["tokens"].cuda(), inp["gate"].cuda(), inp["idx_k"].cuda(), cache, status=st)
+    torch.cuda.synchronize()
+    grec.check()
+    assert st.item() == kvc.DEV_CAPACITY
+    assert cache.n_entries.cpu().tolist() == [2000, 200, 2050]
+    g = cache.records.cpu().numpy()
+    assert not g[1].any()
+    assert np.array_equal(g[0, :2000], rec[0]) and not g[0, 2000:].any()
+    assert np.array_equal(g[2, 50:2050], rec[2]) and not g[2, :50].any()
+    gi = cache.idx_k.cpu().numpy()
+    assert np.array_equal(gi[0, :2000], ic[0]) and np.array_equal(gi[2, 50:2050], ic[2])
+    assert not gi[1].any()
