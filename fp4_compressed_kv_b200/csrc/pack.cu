@@ -669,7 +669,16 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
     using T = __nv_bfloat16;
     extern __shared__ __align__(128) uint8_t rsm[];  // stages | gate | team tails
     __shared__ float tab_s[128], tab_rl[128], tab_rh[128];
-    __shared__ __align__(8) uint64_t full[kRingMaxStages], empty[kRingMaxStages];
+    // full[f]: unit k's copy has landed, f = k % nfull (nfull = stages +
+    // kRingGroups); empty[k % stages]: unit k's stage has been read.  A stage
+    // carries the units of every group in turn, so a full barrier per stage
+    // could be tested by a group that never saw the stage's previous phase
+    // complete (mbarrier waits tell phases apart by parity only).  With one
+    // full barrier per unit index modulo stages + kRingGroups, the previous
+    // use of unit k's barrier is unit k - stages - kRingGroups, which was read
+    // before unit k - kRingGroups (the group's own previous unit) could be
+    // copied into its stage: every parity wait tests the phase it means.
+    __shared__ __align__(8) uint64_t full[kRingMaxStages + kRingGroups], empty[kRingMaxStages];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int D = sh.D, nchunk = D >> 3, half = a.n_new >> 1;
     const int units_per_seq = (half + kRingE - 1) / kRingE;
@@ -679,11 +688,10 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
     const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
 
     if (ue4m3 && tid < 128) fill_scale_tables(tab_s, tab_rl, tab_rh, tid);
+    const int nfull = stages + kRingGroups;
     if (tid == 0) {
-        for (int st = 0; st < stages; ++st) {
-            tc::mbar_init(tc::smem_u32(&full[st]), 1);
-            tc::mbar_init(tc::smem_u32(&empty[st]), kRingE / 4);
-        }
+        for (int f = 0; f < nfull; ++f) tc::mbar_init(tc::smem_u32(&full[f]), 1);
+        for (int st = 0; st < stages; ++st) tc::mbar_init(tc::smem_u32(&empty[st]), kRingE / 4);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     for (int t = tid * 4; t < kRingConsumerWarps * 4 * tail_stride; t += kRingThreads * 4)
@@ -697,6 +705,7 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
         if (lane != 0) return;
         const T* tokens = static_cast<const T*>(a.tokens);
         long long k = 0;
+        int f = 0;
         for (;; ++k) {
             const long long u = blockIdx.x + k * gridDim.x;
             if (u >= n_units) break;
@@ -711,11 +720,12 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
             const int ne = min(kRingE, half - e0);
             ring_bulk_load(ring + (uint32_t)st * stage_bytes,
                            tokens + ((long long)b * a.n_new + 2 * e0) * D,
-                           (uint32_t)(ne * 2 * D * (int)sizeof(T)), tc::smem_u32(&full[st]));
+                           (uint32_t)(ne * 2 * D * (int)sizeof(T)), tc::smem_u32(&full[f]));
+            if (++f == nfull) f = 0;
         }
         // copies still in flight must land before the CTA exits
         for (long long j = k > stages ? k - stages : 0; j < k; ++j)
-            tc::mbar_wait(tc::smem_u32(&full[j % stages]), (uint32_t)((j / stages) & 1),
+            tc::mbar_wait(tc::smem_u32(&full[(int)(j % nfull)]), (uint32_t)((j / nfull) & 1),
                           kRingDrainNs);
         return;
     }
@@ -727,13 +737,14 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
     uint8_t* tail = tails + (warp * 4 + team) * tail_stride;
     const int ei = wi * 4 + team;  // entry within the unit
     bool bad = false;
+    int f = grp, rf = 0;
     for (long long k = grp;; k += kRingGroups) {
         const long long u = blockIdx.x + k * gridDim.x;
         if (u >= n_units) break;
         const int st = (int)(k % stages);
         const bool got = __all_sync(
             0xffffffffu,
-            tc::mbar_wait(tc::smem_u32(&full[st]), (uint32_t)((k / stages) & 1), wait_ns));
+            tc::mbar_wait(tc::smem_u32(&full[f]), (uint32_t)(rf & 1), wait_ns));
         if (!got) {
             if (lane == 0) set_status(a.status, KVC_DEV_TIMEOUT);
             break;
@@ -812,6 +823,8 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
                 if (l + 8 * r < (di >> 4)) dst[l + 8 * r] = ik[r];
         }
         __syncwarp();  // the tail is read before the next unit writes it
+        f += kRingGroups;
+        if (f >= nfull) f -= nfull, ++rf;
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, KVC_DEV_NONFINITE);
 }
@@ -1215,7 +1228,7 @@ inline RingPlan ring_plan(const Shape& sh, const PackArgs& a, int di) {
     const int tail_stride = ((sh.rb - sh.code_bytes) + 15) / 16 * 16;
     const size_t fixed = (size_t)D * 4 + (size_t)kRingConsumerWarps * 4 * tail_stride;
     const uint32_t sb = (uint32_t)(kRingE * 2 * D * 2);
-    const long long room = (long long)optin - 2048 - (long long)fixed;  // static smem margin
+    const long long room = (long long)optin - 4096 - (long long)fixed;  // static smem margin
     int st = room > 0 ? (int)(room / sb) : 0;
     if (st > kRingMaxStages) st = kRingMaxStages;
     if (st < kRingGroups + 1) return p;
