@@ -153,7 +153,10 @@ size_t kvc_workspace_bytes(const kvc_config* cfg, int batch, int capacity);
  * Entries are written at positions n_entries[b] .. n_entries[b]+n_new/r-1 and
  * n_entries[b] then advances by n_new/r.  If that would pass the capacity the
  * sequence is left unchanged and KVC_DEV_CAPACITY is set.  NaN/Inf channels are
- * coded 0, left out of the group maximum, and set KVC_DEV_NONFINITE.         */
+ * coded 0, left out of the group maximum, and set KVC_DEV_NONFINITE.  Long
+ * bf16 appends stream the tokens through shared memory with bounded waits; if
+ * one gives up (KVC_DEV_TIMEOUT) n_entries still advances but some of the new
+ * entries may be unwritten: set n_entries back and append them again.        */
 kvc_status kvc_pack(const kvc_config* cfg, const void* tokens, int n_new,
                     const float* gate, const int8_t* idx_k_new,
                     const kvc_cache* cache, uint32_t* dev_status, void* stream);

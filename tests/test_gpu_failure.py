@@ -105,3 +105,36 @@ def test_attention_operand_range(kvc, where):
     assert_attn_close(o, ref, where)
     rl = np.asarray(ref_lse)
     assert np.max(np.abs(lse.cpu().numpy() - rl) / np.maximum(1.0, np.abs(rl))) < 2e-3
+
+
+def test_pack_ring_zero_wait_limit_times_out_then_recovers(kvc):
+    """A long bf16 append runs the pack ring (a producer thread, consumer warps
+    and stage barriers).  Under a zero wait limit its consumers and producer
+    give up at their first incomplete barrier: the call returns with
+    KVC_DEV_TIMEOUT, the copies already issued land before the CTAs exit, and
+    the next append (normal limit, fresh cache) equals the oracle byte for byte."""
+    # 8 x 375 units of 8 entries: more units per CTA than stages, so the
+    # producer waits on stages too
+    w = synth.WORKLOADS["batch32x128k"].scaled(batch=8, context=2 * 3000)
+    inp = synth.make_inputs(w)
+    cfg = kvc.config_for(w)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok, gate, idx = inp["tokens"].cuda(), inp["gate"].cuda(), inp["idx_k"].cuda()
+    spoiled = kvc.Cache(cfg, w.batch, w.entries)
+    kvc.debug_set_wait_limit_ns(0)
+    try:
+        kvc.pack(cfg, tok, gate, idx, spoiled, status=st)  # returns normally
+        torch.cuda.synchronize()  # and the kernel ends: no hang
+    finally:
+        kvc.debug_set_wait_limit_ns(2_000_000_000)
+    assert int(st.item()) & KVC_DEV_TIMEOUT, int(st.item())
+
+    st.zero_()
+    cache = kvc.Cache(cfg, w.batch, w.entries)
+    kvc.pack(cfg, tok, gate, idx, cache, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rec, ic, n, _ = oracle_pack(w, inp["tokens"], inp["gate"], inp["idx_k"])
+    assert np.array_equal(cache.records.cpu().numpy(), rec)
+    assert np.array_equal(cache.idx_k.cpu().numpy(), ic)
+    assert cache.n_entries.cpu().tolist() == n.tolist()
