@@ -882,6 +882,22 @@ def run_ours(args):
         except Exception as e:  # the pool must not cost the headline line
             cpu = {"value": single, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                    "multicore_error": str(e)[:200]}
+        # the same two oracle legs for the CSA2 group and the 1M-token stack
+        # (shorter samples: one 1M-token step takes about a second on one core)
+        for name in (workloads or {}):
+            wx = synth.WORKLOADS[name]
+            secs_x = args.cpu_seconds / 4
+            try:
+                sx, tx, dx = oracle_decode_sample(wx, secs_x)
+                rate_x, res_x = oracle_multicore(wx, secs_x, procs)
+                workloads[name]["cpu_baseline"] = {
+                    "value": round(rate_x, 3), "unit": UNIT, "cores": procs, "kind": "oracle",
+                    "sample": (f"{sum(r[0] for r in res_x)} single-sequence decode steps of "
+                               f"{wx.name} on {procs} processes (one per core, its own "
+                               f"sequences; about {secs_x:.0f} s each), oracle C code"),
+                    "single_core": {"value": round(sx / tx, 3), "sample": dx}}
+            except Exception as e:  # a side measurement must not cost the headline line
+                workloads[name]["cpu_baseline"] = {"error": str(e)[:200]}
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
