@@ -37,11 +37,13 @@
 //     an MN-major operand, 4 x 8 tcgen05.mma (M = 128 channels, N = 64 heads,
 //     K = 16 keys) into tensor memory.  A second record chunk's loads are in
 //     flight while this product runs.
-//  6. The CTAs of a sequence (at most 8) form a thread-block cluster: each
-//     stores its unnormalised O and (m, l) (they stay in L2), one cluster
-//     barrier orders the stores, and CTA r pulls the rows of heads
-//     [r*64/n, (r+1)*64/n) from every CTA into its freed K tile with bulk
-//     copies and combines them.  More CTAs per sequence: attn_merge.
+//  6. The CTAs of a sequence (at most 8) form a thread-block cluster; CTA r
+//     owns heads [r*HG/n, (r+1)*HG/n) of the group.  After a cluster barrier
+//     each CTA stores its unnormalised O columns (from tensor memory) and its
+//     (m, l) straight into the owners' freed K tiles over distributed shared
+//     memory; after a second barrier every owner weights the rows by
+//     2^(m - max m), sums them in split order and writes the normalised
+//     output.  More CTAs per sequence: attn_merge.
 // Every wait on an mbarrier is bounded; on expiry the CTA sets
 // KVC_DEV_TIMEOUT, waits (bounded) for the copies and products it issued,
 // frees its tensor memory and returns.
