@@ -435,6 +435,36 @@ __device__ __forceinline__ float gate_chunk(float acc, const Chunk<T>& x0, const
     }
     return acc;
 }
+// bf16 tokens: k0's halves enter the subtraction as bf16 operands (the
+// mixed-precision sub widens them exactly, then rounds k0 - k1 once in fp32,
+// as the pair subtraction does), so only k1 is unpacked.
+__device__ __forceinline__ float bf16_minus_f32(uint32_t w, bool hi, float c) {
+    float r;
+    if (hi)
+        asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tsub.rn.f32.bf16 %0, h, %2;\n\t}"
+            : "=f"(r)
+            : "r"(w), "f"(c));
+    else
+        asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tsub.rn.f32.bf16 %0, l, %2;\n\t}"
+            : "=f"(r)
+            : "r"(w), "f"(c));
+    return r;
+}
+template <>
+__device__ __forceinline__ float gate_chunk(float acc, const Chunk<__nv_bfloat16>& x0,
+                                            const Chunk<__nv_bfloat16>& x1,
+                                            const float (&g)[8]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t w0 = k == 0 ? x0.v.x : k == 1 ? x0.v.y : k == 2 ? x0.v.z : x0.v.w;
+        const uint32_t w1 = k == 0 ? x1.v.x : k == 1 ? x1.v.y : k == 2 ? x1.v.z : x1.v.w;
+        const float dlo = bf16_minus_f32(w0, false, __uint_as_float(w1 << 16));
+        const float dhi = bf16_minus_f32(w0, true, __uint_as_float(w1 & 0xFFFF0000u));
+        acc = __fmaf_rn(g[2 * k], dlo, acc);
+        acc = __fmaf_rn(g[2 * k + 1], dhi, acc);
+    }
+    return acc;
+}
 
 // The pair weights from the team's eight running sums (xor tree over 4, 2, 1).
 __device__ __forceinline__ void gate_weights(float acc, uint64_t& W0, uint64_t& W1) {
@@ -456,8 +486,7 @@ __device__ __forceinline__ void gate_weights(float acc, uint64_t& W0, uint64_t& 
 template <typename T, int LPG>
 __device__ __forceinline__ void quantise_chunk(const Chunk<T>& x0, const Chunk<T>& x1,
                                                uint64_t W0, uint64_t W1, bool active, int c,
-                                               int ue4m3, const float* tab_s, const float* tab_rl,
-                                               const float* tab_rh, uint8_t* rec, uint8_t* tail,
+                                               int ue4m3, const float4* tab, uint8_t* rec, uint8_t* tail,
                                                bool& bad) {
     uint64_t v[4];  // v = w0 k0 + w1 k1, rounded as fmaf(w0, k0, w1 * k1)
 #pragma unroll
@@ -496,8 +525,8 @@ __device__ __forceinline__ void quantise_chunk(const Chunk<T>& x0, const Chunk<T
     uint32_t code, sbyte = 0;
     if (ue4m3) {
         sbyte = e4m3_from_f32(sc);
-        const float sv = tab_s[sbyte];
-        code = sv > 0.f ? e2m1x8_quotient_f2(v, sv, tab_rl[sbyte], tab_rh[sbyte]) : 0u;
+        const float4 t = tab[sbyte];  // the scale, its reciprocal brackets
+        code = t.x > 0.f ? e2m1x8_quotient_f2(v, t.x, t.y, t.z) : 0u;
     } else {
         float x[8];
 #pragma unroll
@@ -518,13 +547,10 @@ __device__ __forceinline__ void quantise_chunk(const Chunk<T>& x0, const Chunk<T
 }
 
 // Reciprocal brackets of the 128 UE4M3 scale values (entry i: scale byte i).
-__device__ __forceinline__ void fill_scale_tables(float* tab_s, float* tab_rl, float* tab_rh,
-                                                  int i) {
+__device__ __forceinline__ void fill_scale_tables(float4* tab, int i) {
     const float sv = e4m3_to_f32(i);
     const float r = __frcp_rn(sv);
-    tab_s[i] = sv;
-    tab_rl[i] = __fmul_rn(r, 1.0f - 0x1p-20f);
-    tab_rh[i] = __fmul_rn(r, 1.0f + 0x1p-20f);
+    tab[i] = make_float4(sv, __fmul_rn(r, 1.0f - 0x1p-20f), __fmul_rn(r, 1.0f + 0x1p-20f), 0.f);
 }
 
 // Streaming form of pack_kernel for groups of at most 64 channels (LPG <= 8
@@ -548,7 +574,7 @@ template <typename T, int MAXJ, int LPG>
 __global__ void __launch_bounds__(kThreads, 5)
 pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
     extern __shared__ __align__(16) uint8_t dsm[];  // per-entry tails
-    __shared__ float tab_s[128], tab_rl[128], tab_rh[128];  // per E4M3 scale byte
+    __shared__ float4 tab[128];  // per E4M3 scale byte: scale, reciprocal brackets
     const int tid = threadIdx.x, lane = tid & 31, team = tid >> 3, l = tid & 7;
     const int b = blockIdx.y, half = a.n_new >> 1;
     const int e0 = blockIdx.x * kTeams, ne = min(kTeams, half - e0);
@@ -556,7 +582,7 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
     const int D = sh.D, nchunk = D >> 3;
     uint8_t* tail = dsm + team * tail_stride;
     const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
-    if (ue4m3 && tid < 128) fill_scale_tables(tab_s, tab_rl, tab_rh, tid);
+    if (ue4m3 && tid < 128) fill_scale_tables(tab, tid);
     for (int t = l * 4; t < tail_len; t += 32) *reinterpret_cast<uint32_t*>(tail + t) = 0u;
     __syncthreads();
     pdl_wait();
@@ -603,7 +629,7 @@ pack_stream_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride) {
             x0.zero();
             x1.zero();
         }
-        quantise_chunk<T, LPG>(x0, x1, W0, W1, active, c, ue4m3, tab_s, tab_rl, tab_rh, rec,
+        quantise_chunk<T, LPG>(x0, x1, W0, W1, active, c, ue4m3, tab, rec,
                                tail, bad);
     }
     __syncwarp();
@@ -668,7 +694,7 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
                  uint32_t stage_bytes, long long n_units, unsigned long long wait_ns) {
     using T = __nv_bfloat16;
     extern __shared__ __align__(128) uint8_t rsm[];  // stages | gate | team tails
-    __shared__ float tab_s[128], tab_rl[128], tab_rh[128];
+    __shared__ float4 tab[128];
     // full[f]: unit k's copy has landed, f = k % nfull (nfull = stages +
     // kRingGroups); empty[k % stages]: unit k's stage has been read.  A stage
     // carries the units of every group in turn, so a full barrier per stage
@@ -687,7 +713,7 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
     uint8_t* tails = rsm + (size_t)stages * stage_bytes + (size_t)D * 4;
     const int tail_len = sh.rb - sh.code_bytes;  // multiple of 4
 
-    if (ue4m3 && tid < 128) fill_scale_tables(tab_s, tab_rl, tab_rh, tid);
+    if (ue4m3 && tid < 128) fill_scale_tables(tab, tid);
     const int nfull = stages + kRingGroups;
     if (tid == 0) {
         for (int f = 0; f < nfull; ++f) tc::mbar_init(tc::smem_u32(&full[f]), 1);
@@ -716,7 +742,8 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
                 set_status(a.status, KVC_DEV_TIMEOUT);
                 break;
             }
-            const int b = (int)(u / units_per_seq), e0 = (int)(u % units_per_seq) * kRingE;
+            const unsigned ub = (unsigned)u / (unsigned)units_per_seq;
+            const int b = (int)ub, e0 = (int)((unsigned)u - ub * (unsigned)units_per_seq) * kRingE;
             const int ne = min(kRingE, half - e0);
             ring_bulk_load(ring + (uint32_t)st * stage_bytes,
                            tokens + ((long long)b * a.n_new + 2 * e0) * D,
@@ -749,7 +776,8 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
             if (lane == 0) set_status(a.status, KVC_DEV_TIMEOUT);
             break;
         }
-        const int b = (int)(u / units_per_seq), e0 = (int)(u % units_per_seq) * kRingE;
+        const unsigned ub = (unsigned)u / (unsigned)units_per_seq;
+        const int b = (int)ub, e0 = (int)((unsigned)u - ub * (unsigned)units_per_seq) * kRingE;
         const int ne = min(kRingE, half - e0);
         const bool here = ei < ne;  // this team has an entry in the unit
         const int i = e0 + ei;
@@ -807,7 +835,7 @@ pack_ring_kernel(PackArgs a, Shape sh, int ue4m3, int di, int tail_stride, int s
                 x0.zero();
                 x1.zero();
             }
-            quantise_chunk<T, LPG>(x0, x1, W0, W1, active, c, ue4m3, tab_s, tab_rl, tab_rh, rec,
+            quantise_chunk<T, LPG>(x0, x1, W0, W1, active, c, ue4m3, tab, rec,
                                    tail, bad);
         }
         __syncwarp();
@@ -1302,9 +1330,9 @@ cudaError_t launch_pack_t(const Shape& sh, const PackArgs& a, int ue4m3, int di,
     trace_before("pack", s);
     if (sh.lpg <= 8 && sizeof(T) == 2) {  // bf16 tokens: the ring kernel where it fits
         const RingPlan p = ring_plan(sh, a, di);
-        if (p.stages > 0) {
-            const int half = a.n_new / 2;
-            const long long n_units = (long long)a.batch * ((half + kRingE - 1) / kRingE);
+        const int half = a.n_new / 2;
+        const long long n_units = (long long)a.batch * ((half + kRingE - 1) / kRingE);
+        if (p.stages > 0 && n_units < (1ll << 31) - p.sms) {  // unit indices fit 32 bits
             err = maxj <= 4 ? launch_ring_j<4>(s, a, sh, ue4m3, di, p, n_units)
                             : launch_ring_j<9>(s, a, sh, ue4m3, di, p, n_units);
             trace_after(s);
