@@ -486,8 +486,8 @@ __device__ __forceinline__ void gate_weights(float acc, uint64_t& W0, uint64_t& 
 template <typename T, int LPG>
 __device__ __forceinline__ void quantise_chunk(const Chunk<T>& x0, const Chunk<T>& x1,
                                                uint64_t W0, uint64_t W1, bool active, int c,
-                                               int ue4m3, const float4* tab, uint8_t* rec, uint8_t* tail,
-                                               bool& bad) {
+                                               int ue4m3, const float4* tab, uint8_t* rec,
+                                               uint8_t* tail, bool& bad) {
     uint64_t v[4];  // v = w0 k0 + w1 k1, rounded as fmaf(w0, k0, w1 * k1)
 #pragma unroll
     for (int k = 0; k < 4; ++k) v[k] = f2_fma(W0, x0.pair(k), f2_mul(W1, x1.pair(k)));
